@@ -148,10 +148,11 @@ ft_status ft_moe_set_tensor_scales(ft_ctx* ctx, int32_t layer, int32_t expert, c
 ft_status ft_moe_set_router(ft_ctx* ctx, int32_t layer, const void* w_router_dev);
 
 /* One MoE layer on T tokens, enqueued on the compute stream.
- *   x_dev   [T][d] activations (fp32 or bf16, see ft_wtype), device pointer
+ *   x_dev   [T][d] activations (fp32 or bf16, see ft_wtype), device pointer,
+ *             16-byte aligned
  *   bias_dev  NULL, or fp32 device pointer: [E] (bias_per_token = 0) or
  *             [T][E] (bias_per_token = 1), added to the router logits
- *   y_dev   [T][d] output, same type as x; may not alias x
+ *   y_dev   [T][d] output, same type as x, 16-byte aligned; may not alias x
  *   ids_dev_opt [T][k] int32, w_dev_opt [T][k] fp32: optional outputs of the
  *             routing (rank order), NULL to skip
  * T may be 0 (no work, no lookups). In decode mode (or prefill with C < 2E)

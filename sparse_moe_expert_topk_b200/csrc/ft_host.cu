@@ -1,0 +1,536 @@
+// Host runtime behind include/ft_moe.h: the context, the pinned expert pool,
+// the HBM slot pool, streams and events, and the per-call orchestration of
+// the routing, lookup, copy-engine staging, expert and combine kernels.
+//
+// Two-tier expert memory ([paperlens] "設計: 2階建てのエキスパート記憶", paper §3):
+// the pinned host pool is the source of truth, the slot pool is a cache.
+// Decode call: router -> top-k/permutation -> lookup (q* split, [techfeed]
+// "帯域適応型実行（q*ポリシー）") on the compute stream; the streamed misses run
+// on a side stream straight from the mapped pool while the hits run on the
+// compute stream; the host waits for the lookup kernel (bounded), issues the
+// copy-engine H2D copies of the staged misses on the copy stream, and the
+// staged experts run once their copies land. Prefill call: the whole layer is
+// resident before it computes and the next layer is copied in behind it
+// ([paperlens] "プレフィル: 全層ダブルバッファと「意味の錨」", paper §3.1).
+#include <chrono>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <thread>
+#include <vector>
+
+#include "ft_internal.cuh"
+
+namespace ft {
+cudaError_t route_kernels_init(int E);
+cudaError_t expert_kernels_init(int device);
+void launch_prefill_work(const Shape& sh, int layer, DevState& ds, cudaStream_t st);
+bool prefill_tc_supported(const Shape& sh);
+cudaError_t prefill_tc_init(const Shape& sh, int max_rows);
+void launch_prefill_tc(const Shape& sh, int layer, const void* x, int T, DevState& ds, cudaStream_t st);
+}  // namespace ft
+
+using namespace ft;
+
+struct ft_ctx {
+  ft_config cfg;
+  Shape sh;
+  cudaStream_t s_comp = nullptr, s_copy = nullptr, s_side = nullptr;
+  std::vector<uint8_t*> pool_host;  // per layer, E blobs each (pinned, mapped)
+  std::vector<uint8_t*> pool_dev;   // device addresses of the same
+  std::vector<const void*> router;  // per layer W_r device pointer
+  std::vector<float> tscale_host;   // [L*E*3]
+  DevState ds{};
+  Mailbox* mbox_host = nullptr;
+  cudaEvent_t ev_look = nullptr, ev_side = nullptr, ev_copy = nullptr, ev_pf[2] = {nullptr, nullptr};
+  cudaEvent_t ev_t0 = nullptr, ev_t1 = nullptr;
+  unsigned bp = 1, bh = 1;
+  int prefetched = -1;   // layer whose experts the previous prefill call loaded ahead
+  int last_T = 0;
+  unsigned long long layer_calls = 0;
+  int last_m = 0, last_qstar = 0, last_qstage = 0;
+  ft_status latched = FT_OK;
+  bool use_tc = false;
+  unsigned long long* probe_sink = nullptr;
+};
+
+namespace {
+
+bool fault(const char* what) {
+  const char* f = getenv("FT_FAULT");
+  return f && strstr(f, what) != nullptr;
+}
+
+#define CK(call)                                                                      \
+  do {                                                                                \
+    cudaError_t e_ = (call);                                                          \
+    if (e_ != cudaSuccess) {                                                          \
+      fprintf(stderr, "ft_moe: %s failed: %s (%s:%d)\n", #call, cudaGetErrorString(e_), \
+              __FILE__, __LINE__);                                                    \
+      return e_ == cudaErrorMemoryAllocation ? FT_ENOMEM : FT_ECUDA;                  \
+    }                                                                                 \
+  } while (0)
+
+ft_status validate(const ft_config* c) {
+  if (!c) return FT_EINVAL;
+  if (c->n_layers < 1 || c->n_experts < 1 || c->n_experts > MAX_E) return FT_EINVAL;
+  if (c->top_k < 1 || c->top_k > MAX_K || c->top_k > c->n_experts) return FT_EINVAL;
+  if (c->d_model < 64 || c->d_model % 64 || c->d_model > 16384) return FT_EINVAL;
+  if (c->d_ff < 64 || c->d_ff % 64 || c->d_ff > 16384) return FT_EINVAL;
+  if (c->wtype < FT_W_F32 || c->wtype > FT_W_NVFP4) return FT_EINVAL;
+  const long long le = (long long)c->n_layers * c->n_experts;
+  if (c->cache_slots < 0 || c->cache_slots > le || c->cache_slots >= (1ll << 20)) return FT_EINVAL;
+  if (c->max_tokens < 1 || c->max_tokens > 65536) return FT_EINVAL;
+  if (c->device < 0) return FT_EINVAL;
+  return FT_OK;
+}
+
+size_t slot_bytes_of(const ft_config* c) {
+  const size_t n = 3ull * c->d_model * c->d_ff;
+  return c->wtype == FT_W_F32 ? 4 * n : (c->wtype == FT_W_BF16 ? 2 * n : n / 2 + n / 16);
+}
+
+// Host wait for an event with a deadline; the compute stream keeps running.
+ft_status wait_event(cudaEvent_t ev, double seconds) {
+  const auto t0 = std::chrono::steady_clock::now();
+  long spins = 0;
+  for (;;) {
+    const cudaError_t e = cudaEventQuery(ev);
+    if (e == cudaSuccess) return FT_OK;
+    if (e != cudaErrorNotReady) return FT_ECUDA;
+    if (fault("poll_timeout")) return FT_ETIMEOUT;
+    if ((++spins & 1023) == 0) {
+      const double dt = std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count();
+      if (dt > seconds) return FT_ETIMEOUT;
+      std::this_thread::yield();
+    }
+  }
+}
+
+constexpr double WAIT_S = 30.0;
+
+void free_all(ft_ctx* c) {
+  if (!c) return;
+  if (c->s_comp || c->s_side) cudaDeviceSynchronize();
+  DevState& d = c->ds;
+  void* dev_ptrs[] = {d.slot_of, d.key_of, d.stamp, d.clk, d.ctr, d.error, d.work, d.scores, d.ids, d.wts,
+                      d.counts, d.offsets, d.perm, d.inv, d.hbuf, d.ybuf, d.xs, d.hs, d.tscale, d.slots,
+                      c->probe_sink};
+  for (void* p : dev_ptrs)
+    if (p) cudaFree(p);
+  for (uint8_t* p : c->pool_host)
+    if (p) cudaFreeHost(p);
+  if (c->mbox_host) cudaFreeHost(c->mbox_host);
+  cudaEvent_t evs[] = {c->ev_look, c->ev_side, c->ev_copy, c->ev_pf[0], c->ev_pf[1], c->ev_t0, c->ev_t1};
+  for (cudaEvent_t e : evs)
+    if (e) cudaEventDestroy(e);
+  if (c->s_side) cudaStreamDestroy(c->s_side);
+  delete c;
+}
+
+ft_status reset_state(ft_ctx* c) {
+  const Shape& sh = c->sh;
+  DevState& d = c->ds;
+  CK(cudaMemsetAsync(d.slot_of, 0xFF, sizeof(int32_t) * sh.L * sh.E, c->s_comp));
+  if (sh.C > 0) {
+    CK(cudaMemsetAsync(d.key_of, 0xFF, sizeof(int32_t) * sh.C, c->s_comp));
+    CK(cudaMemsetAsync(d.stamp, 0, sizeof(unsigned long long) * sh.C, c->s_comp));
+  }
+  CK(cudaMemsetAsync(d.clk, 0, sizeof(LruClock), c->s_comp));
+  CK(cudaMemsetAsync(d.ctr, 0, sizeof(DevCounters), c->s_comp));
+  CK(cudaMemsetAsync(d.error, 0, sizeof(uint32_t), c->s_comp));
+  CK(cudaStreamSynchronize(c->s_comp));
+  memset(c->mbox_host, 0, sizeof(Mailbox));
+  c->prefetched = -1;
+  c->latched = FT_OK;
+  c->last_m = c->last_qstar = c->last_qstage = 0;
+  c->layer_calls = 0;
+  return FT_OK;
+}
+
+ft_status check_device_error(ft_ctx* c) {
+  // the lookup kernel mirrors the device error word into the mailbox
+  const uint32_t e = ((volatile Mailbox*)c->mbox_host)->pad_error;
+  if (e) c->latched = e == DERR_TIMEOUT ? FT_ETIMEOUT : FT_ESTATE;
+  return c->latched;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ft_status_str(ft_status s) {
+  switch (s) {
+    case FT_OK: return "ok";
+    case FT_EINVAL: return "invalid argument";
+    case FT_ENOMEM: return "out of memory";
+    case FT_ECUDA: return "CUDA error";
+    case FT_ETIMEOUT: return "timed out";
+    case FT_ESTATE: return "bad state";
+    case FT_EUNSUPPORTED: return "unsupported";
+  }
+  return "unknown status";
+}
+
+ft_status ft_moe_slot_bytes(const ft_config* cfg, uint64_t* out) {
+  if (!out) return FT_EINVAL;
+  const ft_status v = validate(cfg);
+  if (v != FT_OK) return v;
+  *out = slot_bytes_of(cfg);
+  return FT_OK;
+}
+
+ft_status ft_moe_init(const ft_config* cfg, void* compute_stream, void* copy_stream, ft_ctx** out) {
+  if (!out) return FT_EINVAL;
+  *out = nullptr;
+  const ft_status v = validate(cfg);
+  if (v != FT_OK) return v;
+  if (!copy_stream || copy_stream == compute_stream) return FT_EINVAL;
+  CK(cudaSetDevice(cfg->device));
+  ft_ctx* c = new (std::nothrow) ft_ctx();
+  if (!c) return FT_ENOMEM;
+  c->cfg = *cfg;
+  Shape& sh = c->sh;
+  sh.L = cfg->n_layers;
+  sh.E = cfg->n_experts;
+  sh.k = cfg->top_k;
+  sh.d = cfg->d_model;
+  sh.d_ff = cfg->d_ff;
+  sh.wtype = cfg->wtype;
+  sh.C = cfg->cache_slots;
+  sh.slot_bytes = slot_bytes_of(cfg);
+  c->s_comp = (cudaStream_t)compute_stream;
+  c->s_copy = (cudaStream_t)copy_stream;
+  c->router.assign(sh.L, nullptr);
+  c->tscale_host.assign((size_t)sh.L * sh.E * 3, 1.0f);
+  ft_status st = FT_OK;
+#define TRY(call)                    \
+  do {                               \
+    st = (call);                     \
+    if (st != FT_OK) {               \
+      free_all(c);                   \
+      return st;                     \
+    }                                \
+  } while (0)
+  auto cuda_try = [&](cudaError_t e) -> ft_status {
+    if (e == cudaSuccess) return FT_OK;
+    fprintf(stderr, "ft_moe_init: %s\n", cudaGetErrorString(e));
+    return e == cudaErrorMemoryAllocation ? FT_ENOMEM : FT_ECUDA;
+  };
+  TRY(cuda_try(cudaStreamCreateWithFlags(&c->s_side, cudaStreamNonBlocking)));
+  // pinned, mapped host pool, one chunk per layer
+  c->pool_host.assign(sh.L, nullptr);
+  c->pool_dev.assign(sh.L, nullptr);
+  for (int l = 0; l < sh.L; ++l) {
+    if (fault("pool_alloc")) TRY(FT_ENOMEM);
+    TRY(cuda_try(cudaHostAlloc((void**)&c->pool_host[l], sh.slot_bytes * sh.E,
+                               cudaHostAllocMapped | cudaHostAllocPortable)));
+    TRY(cuda_try(cudaHostGetDevicePointer((void**)&c->pool_dev[l], c->pool_host[l], 0)));
+  }
+  TRY(cuda_try(cudaHostAlloc((void**)&c->mbox_host, sizeof(Mailbox), cudaHostAllocMapped)));
+  memset(c->mbox_host, 0, sizeof(Mailbox));
+  DevState& d = c->ds;
+  TRY(cuda_try(cudaHostGetDevicePointer((void**)&d.mbox, c->mbox_host, 0)));
+  const size_t Tk = (size_t)cfg->max_tokens * sh.k;
+  if (fault("slot_alloc")) TRY(FT_ENOMEM);
+  if (sh.C > 0) TRY(cuda_try(cudaMalloc((void**)&d.slots, sh.slot_bytes * (size_t)sh.C)));
+  TRY(cuda_try(cudaMalloc((void**)&d.slot_of, sizeof(int32_t) * sh.L * sh.E)));
+  TRY(cuda_try(cudaMalloc((void**)&d.key_of, sizeof(int32_t) * (sh.C > 0 ? sh.C : 1))));
+  TRY(cuda_try(cudaMalloc((void**)&d.stamp, sizeof(unsigned long long) * (sh.C > 0 ? sh.C : 1))));
+  TRY(cuda_try(cudaMalloc((void**)&d.clk, sizeof(LruClock))));
+  TRY(cuda_try(cudaMalloc((void**)&d.ctr, sizeof(DevCounters))));
+  TRY(cuda_try(cudaMalloc((void**)&d.error, sizeof(uint32_t))));
+  TRY(cuda_try(cudaMalloc((void**)&d.work, sizeof(WorkLists))));
+  TRY(cuda_try(cudaMalloc((void**)&d.scores, sizeof(float) * cfg->max_tokens * sh.E)));
+  TRY(cuda_try(cudaMalloc((void**)&d.ids, sizeof(int32_t) * Tk)));
+  TRY(cuda_try(cudaMalloc((void**)&d.wts, sizeof(float) * Tk)));
+  TRY(cuda_try(cudaMalloc((void**)&d.counts, sizeof(int32_t) * sh.E)));
+  TRY(cuda_try(cudaMalloc((void**)&d.offsets, sizeof(int32_t) * (sh.E + 1))));
+  TRY(cuda_try(cudaMalloc((void**)&d.perm, sizeof(int32_t) * Tk)));
+  TRY(cuda_try(cudaMalloc((void**)&d.inv, sizeof(int32_t) * Tk)));
+  TRY(cuda_try(cudaMalloc((void**)&d.hbuf, sizeof(float) * Tk * sh.d_ff)));
+  TRY(cuda_try(cudaMalloc((void**)&d.ybuf, sizeof(float) * Tk * sh.d)));
+  TRY(cuda_try(cudaMalloc((void**)&d.tscale, sizeof(float) * sh.L * sh.E * 3)));
+  TRY(cuda_try(cudaMalloc((void**)&c->probe_sink, sizeof(unsigned long long))));
+  c->use_tc = prefill_tc_supported(sh) && sh.C >= 2ll * sh.E;
+  if (c->use_tc) {
+    TRY(cuda_try(cudaMalloc((void**)&d.xs, sizeof(__nv_bfloat16) * (Tk + 256) * sh.d)));
+    TRY(cuda_try(cudaMalloc((void**)&d.hs, sizeof(__nv_bfloat16) * (Tk + 256) * sh.d_ff)));
+    TRY(cuda_try(prefill_tc_init(sh, (int)Tk)));
+  }
+  d.pool_dev = nullptr;
+  TRY(cuda_try(cudaMemcpy(d.tscale, c->tscale_host.data(), sizeof(float) * c->tscale_host.size(),
+                          cudaMemcpyHostToDevice)));
+  TRY(cuda_try(cudaEventCreateWithFlags(&c->ev_look, cudaEventDisableTiming)));
+  TRY(cuda_try(cudaEventCreateWithFlags(&c->ev_side, cudaEventDisableTiming)));
+  TRY(cuda_try(cudaEventCreateWithFlags(&c->ev_copy, cudaEventDisableTiming)));
+  TRY(cuda_try(cudaEventCreateWithFlags(&c->ev_pf[0], cudaEventDisableTiming)));
+  TRY(cuda_try(cudaEventCreateWithFlags(&c->ev_pf[1], cudaEventDisableTiming)));
+  TRY(cuda_try(cudaEventCreate(&c->ev_t0)));
+  TRY(cuda_try(cudaEventCreate(&c->ev_t1)));
+  TRY(cuda_try(route_kernels_init(sh.E)));
+  TRY(cuda_try(expert_kernels_init(cfg->device)));
+  TRY(reset_state(c));
+#undef TRY
+  *out = c;
+  return FT_OK;
+}
+
+void ft_moe_destroy(ft_ctx* c) { free_all(c); }
+
+ft_status ft_moe_expert_ptr(ft_ctx* c, int32_t layer, int32_t expert, void** host_blob) {
+  if (!c || !host_blob || layer < 0 || layer >= c->sh.L || expert < 0 || expert >= c->sh.E) return FT_EINVAL;
+  *host_blob = c->pool_host[layer] + (size_t)expert * c->sh.slot_bytes;
+  return FT_OK;
+}
+
+ft_status ft_moe_set_tensor_scales(ft_ctx* c, int32_t layer, int32_t expert, const float* scales) {
+  if (!c || !scales || layer < 0 || layer >= c->sh.L || expert < 0 || expert >= c->sh.E) return FT_EINVAL;
+  if (c->sh.wtype != FT_W_NVFP4) return FT_EINVAL;
+  const size_t o = ((size_t)layer * c->sh.E + expert) * 3;
+  memcpy(&c->tscale_host[o], scales, 3 * sizeof(float));
+  CK(cudaMemcpyAsync(c->ds.tscale + o, &c->tscale_host[o], 3 * sizeof(float), cudaMemcpyHostToDevice, c->s_comp));
+  CK(cudaStreamSynchronize(c->s_comp));
+  return FT_OK;
+}
+
+ft_status ft_moe_set_router(ft_ctx* c, int32_t layer, const void* w) {
+  if (!c || !w || layer < 0 || layer >= c->sh.L) return FT_EINVAL;
+  if ((uintptr_t)w & 15) return FT_EINVAL;
+  c->router[layer] = w;
+  return FT_OK;
+}
+
+ft_status ft_set_bandwidths(ft_ctx* c, uint32_t bp, uint32_t bh) {
+  if (!c || bh == 0) return FT_EINVAL;
+  c->bp = bp;
+  c->bh = bh;
+  return FT_OK;
+}
+
+ft_status ft_moe_reset_cache(ft_ctx* c) {
+  if (!c) return FT_EINVAL;
+  CK(cudaStreamSynchronize(c->s_copy));
+  CK(cudaStreamSynchronize(c->s_side));
+  return reset_state(c);
+}
+
+static ft_status issue_copies(ft_ctx* c, int from, int to) {
+  const Mailbox* mb = c->mbox_host;
+  const Shape& sh = c->sh;
+  for (int i = from; i < to; ++i) {
+    const int key = mb->copy_key[i], slot = mb->copy_slot[i];
+    const int l = key / sh.E, e = key % sh.E;
+    if (l < 0 || l >= sh.L || slot < 0 || slot >= sh.C) return FT_ESTATE;
+    if (fault("memcpy")) return FT_ECUDA;
+    CK(cudaMemcpyAsync(c->ds.slots + (size_t)slot * sh.slot_bytes, c->pool_host[l] + (size_t)e * sh.slot_bytes,
+                       sh.slot_bytes, cudaMemcpyHostToDevice, c->s_copy));
+  }
+  return FT_OK;
+}
+
+ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const void* x, int32_t T, const float* bias,
+                               int32_t bias_per_token, void* y, int32_t* ids_opt, float* w_opt) {
+  if (!c) return FT_EINVAL;
+  const Shape& sh = c->sh;
+  if (layer < 0 || layer >= sh.L || (mode != FT_DECODE && mode != FT_PREFILL)) return FT_EINVAL;
+  if (T < 0 || T > c->cfg.max_tokens) return FT_EINVAL;
+  if (c->latched != FT_OK) return c->latched;
+  if (T == 0) return FT_OK;
+  if (!x || !y || x == y) return FT_EINVAL;
+  if (((uintptr_t)x | (uintptr_t)y) & 15) return FT_EINVAL;  // 16-byte vector loads and stores
+  if (bias && ((uintptr_t)bias & 3)) return FT_EINVAL;
+  if (!c->router[layer]) return FT_ESTATE;
+  DevState& d = c->ds;
+  cudaStream_t cs = c->s_comp;
+  c->last_T = T;
+  c->layer_calls += 1;
+  launch_router_scores(sh, x, c->router[layer], bias, bias_per_token, T, d.scores, cs);
+  launch_topk_permute(sh, d.scores, T, d, ids_opt, w_opt, cs);
+  const int Tk = T * sh.k;
+  const int max_items = Tk < sh.E ? Tk : sh.E;
+  const bool full_prefill = mode == FT_PREFILL && sh.C >= 2ll * sh.E;
+  ft_status st = FT_OK;
+  if (!full_prefill) {
+    LookupArgs a{};
+    a.layer = layer;
+    a.use_counts = 1;
+    a.limit_q = 1;
+    a.is_current = 1;
+    a.build_work = 1;
+    a.bp_mbps = c->bp;
+    a.bh_mbps = c->bh;
+    d.pool_dev = c->pool_dev[layer];
+    launch_lookup(sh, a, d, cs);
+    CK(cudaEventRecord(c->ev_look, cs));
+    CK(cudaStreamWaitEvent(c->s_side, c->ev_look, 0));
+    launch_expert_gemv(sh, KIND_STREAMED, layer, x, T, d, max_items, Tk, c->s_side);
+    CK(cudaEventRecord(c->ev_side, c->s_side));
+    launch_expert_gemv(sh, KIND_HIT, layer, x, T, d, max_items, Tk, cs);
+    st = wait_event(c->ev_look, WAIT_S);
+    if (st != FT_OK) return c->latched = st;
+    if (check_device_error(c) != FT_OK) return c->latched;
+    const int n_copy = c->mbox_host->n_copy;
+    c->last_m = c->mbox_host->m;
+    c->last_qstar = c->mbox_host->qstar;
+    c->last_qstage = c->mbox_host->qstage;
+    if (n_copy > 0) {
+      st = issue_copies(c, 0, n_copy);
+      if (st != FT_OK) return c->latched = st;
+      CK(cudaEventRecord(c->ev_copy, c->s_copy));
+      CK(cudaStreamWaitEvent(cs, c->ev_copy, 0));
+      launch_expert_gemv(sh, KIND_STAGED, layer, x, T, d, max_items, Tk, cs);
+    }
+    CK(cudaStreamWaitEvent(cs, c->ev_side, 0));
+    c->prefetched = -1;
+  } else {
+    const bool load_cur = c->prefetched != layer;
+    const bool load_next = layer + 1 < sh.L;
+    if (load_cur) {
+      LookupArgs a{};
+      a.layer = layer;
+      a.is_current = 1;
+      launch_lookup(sh, a, d, cs);
+    }
+    if (load_next) {
+      LookupArgs a{};
+      a.layer = layer + 1;
+      a.pin_prev = 1;
+      a.append = load_cur ? 1 : 0;
+      launch_lookup(sh, a, d, cs);
+    }
+    if (load_cur || load_next) {
+      CK(cudaEventRecord(c->ev_look, cs));
+      st = wait_event(c->ev_look, WAIT_S);
+      if (st != FT_OK) return c->latched = st;
+      if (check_device_error(c) != FT_OK) return c->latched;
+      const Mailbox* mb = c->mbox_host;
+      int split = 0;
+      while (split < mb->n_copy && mb->copy_key[split] / sh.E == layer) ++split;
+      if (load_cur) {
+        c->last_m = mb->m;
+        c->last_qstar = -1;
+        c->last_qstage = mb->qstage;
+        st = issue_copies(c, 0, split);
+        if (st != FT_OK) return c->latched = st;
+        CK(cudaEventRecord(c->ev_pf[layer & 1], c->s_copy));
+      } else {
+        c->last_m = c->last_qstage = 0;
+        c->last_qstar = -1;
+      }
+      if (load_next) {
+        st = issue_copies(c, split, mb->n_copy);
+        if (st != FT_OK) return c->latched = st;
+        CK(cudaEventRecord(c->ev_pf[(layer + 1) & 1], c->s_copy));
+      }
+    }
+    c->prefetched = load_next ? layer + 1 : -1;
+    launch_prefill_work(sh, layer, d, cs);
+    CK(cudaStreamWaitEvent(cs, c->ev_pf[layer & 1], 0));
+    if (c->use_tc) {
+      launch_prefill_tc(sh, layer, x, T, d, cs);
+    } else {
+      d.pool_dev = c->pool_dev[layer];
+      launch_expert_gemv(sh, KIND_HIT, layer, x, T, d, max_items, Tk, cs);
+    }
+  }
+  launch_combine(sh, T, d, y, cs);
+  CK(cudaGetLastError());
+  return FT_OK;
+}
+
+ft_status ft_cache_stats(ft_ctx* c, ft_stats* out) {
+  if (!c || !out) return FT_EINVAL;
+  CK(cudaStreamSynchronize(c->s_copy));
+  CK(cudaStreamSynchronize(c->s_side));
+  CK(cudaStreamSynchronize(c->s_comp));
+  DevCounters h{};
+  uint32_t err = 0;
+  CK(cudaMemcpy(&h, c->ds.ctr, sizeof(h), cudaMemcpyDeviceToHost));
+  CK(cudaMemcpy(&err, c->ds.error, sizeof(err), cudaMemcpyDeviceToHost));
+  out->layer_calls = c->layer_calls;
+  out->lookups = h.lookups;
+  out->hits = h.hits;
+  out->misses = h.misses;
+  out->staged = h.staged;
+  out->streamed = h.streamed;
+  out->bytes_h2d = h.bytes_h2d;
+  out->bytes_zero_copy = h.bytes_zero_copy;
+  out->last_m = c->last_m;
+  out->last_qstar = c->last_qstar;
+  out->last_qstage = c->last_qstage;
+  out->device_error = err ? (err == DERR_TIMEOUT ? FT_ETIMEOUT : FT_ESTATE) : (int32_t)c->latched;
+  return FT_OK;
+}
+
+ft_status ft_moe_last_route(ft_ctx* c, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                            int32_t* lookup_e, int32_t* lookup_kind, int32_t* n_lookup, int32_t* n_lookup_cur,
+                            int32_t* m, int32_t* qstar, int32_t* qstage) {
+  if (!c) return FT_EINVAL;
+  CK(cudaStreamSynchronize(c->s_copy));
+  CK(cudaStreamSynchronize(c->s_side));
+  CK(cudaStreamSynchronize(c->s_comp));
+  const Shape& sh = c->sh;
+  const size_t Tk = (size_t)c->last_T * sh.k;
+  if (counts) CK(cudaMemcpy(counts, c->ds.counts, sizeof(int32_t) * sh.E, cudaMemcpyDeviceToHost));
+  if (offsets) CK(cudaMemcpy(offsets, c->ds.offsets, sizeof(int32_t) * (sh.E + 1), cudaMemcpyDeviceToHost));
+  if (perm && Tk) CK(cudaMemcpy(perm, c->ds.perm, sizeof(int32_t) * Tk, cudaMemcpyDeviceToHost));
+  if (inv && Tk) CK(cudaMemcpy(inv, c->ds.inv, sizeof(int32_t) * Tk, cudaMemcpyDeviceToHost));
+  const Mailbox* mb = c->mbox_host;
+  if (lookup_e) memcpy(lookup_e, mb->lookup_e, sizeof(int32_t) * mb->n_lookup);
+  if (lookup_kind) memcpy(lookup_kind, mb->lookup_kind, sizeof(int32_t) * mb->n_lookup);
+  if (n_lookup) *n_lookup = mb->n_lookup;
+  if (n_lookup_cur) *n_lookup_cur = mb->n_lookup_cur;
+  if (m) *m = c->last_m;
+  if (qstar) *qstar = c->last_qstar;
+  if (qstage) *qstage = c->last_qstage;
+  return FT_OK;
+}
+
+ft_status ft_moe_cache_contents(ft_ctx* c, int32_t* key_of, uint64_t* stamp) {
+  if (!c) return FT_EINVAL;
+  CK(cudaStreamSynchronize(c->s_copy));
+  CK(cudaStreamSynchronize(c->s_side));
+  CK(cudaStreamSynchronize(c->s_comp));
+  if (c->sh.C == 0) return FT_OK;
+  if (key_of) CK(cudaMemcpy(key_of, c->ds.key_of, sizeof(int32_t) * c->sh.C, cudaMemcpyDeviceToHost));
+  if (stamp) CK(cudaMemcpy(stamp, c->ds.stamp, sizeof(uint64_t) * c->sh.C, cudaMemcpyDeviceToHost));
+  return FT_OK;
+}
+
+ft_status ft_moe_probe_link(ft_ctx* c, uint64_t bytes, double* h2d_gbs, double* zc_gbs) {
+  if (!c || bytes == 0 || bytes % 4096) return FT_EINVAL;
+  const Shape& sh = c->sh;
+  if (bytes > sh.slot_bytes * (size_t)sh.E) return FT_EINVAL;
+  CK(cudaStreamSynchronize(c->s_comp));
+  CK(cudaStreamSynchronize(c->s_copy));
+  uint8_t* tmp = nullptr;
+  CK(cudaMalloc((void**)&tmp, bytes));
+  float ms = 0.f;
+  cudaError_t e = cudaSuccess;
+  for (int rep = 0; rep < 2 && e == cudaSuccess; ++rep) {  // first pass warms up
+    e = cudaEventRecord(c->ev_t0, c->s_copy);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(tmp, c->pool_host[0], bytes, cudaMemcpyHostToDevice, c->s_copy);
+    if (e == cudaSuccess) e = cudaEventRecord(c->ev_t1, c->s_copy);
+    if (e == cudaSuccess) e = cudaEventSynchronize(c->ev_t1);
+  }
+  if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, c->ev_t0, c->ev_t1);
+  if (e == cudaSuccess && h2d_gbs) *h2d_gbs = bytes / (ms * 1e6);
+  for (int rep = 0; rep < 2 && e == cudaSuccess; ++rep) {
+    e = cudaEventRecord(c->ev_t0, c->s_comp);
+    if (e == cudaSuccess) {
+      launch_read_probe(c->pool_dev[0], bytes, c->probe_sink, c->s_comp);
+      e = cudaGetLastError();
+    }
+    if (e == cudaSuccess) e = cudaEventRecord(c->ev_t1, c->s_comp);
+    if (e == cudaSuccess) e = cudaEventSynchronize(c->ev_t1);
+  }
+  if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, c->ev_t0, c->ev_t1);
+  if (e == cudaSuccess && zc_gbs) *zc_gbs = bytes / (ms * 1e6);
+  cudaFree(tmp);
+  CK(e);
+  return FT_OK;
+}
+
+}  // extern "C"

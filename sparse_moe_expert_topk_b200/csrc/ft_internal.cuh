@@ -1,0 +1,137 @@
+// Internal declarations shared by the library's translation units: the
+// device-side state of a context, the expert work list written by the lookup
+// kernel, the host mailbox, and the kernel launchers. Not part of the ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include "../../include/ft_moe.h"
+
+namespace ft {
+
+// Outcome of one expert lookup. Hit and staged experts are read from their
+// HBM slot; streamed experts are read by the expert kernels directly from the
+// mapped host pool (the "compute where the weights are" leg of the q* split,
+// done by the GPU here).
+enum Kind : int32_t { KIND_HIT = 0, KIND_STAGED = 1, KIND_STREAMED = 2 };
+constexpr int N_CLASSES = 3;  // work-list classes, indexed by Kind
+
+// Device error codes latched in DevState::error (0 = none).
+enum DevError : uint32_t { DERR_NONE = 0, DERR_NO_VICTIM = 1, DERR_BAD_INDEX = 2, DERR_TIMEOUT = 3 };
+
+constexpr int MAX_E = 512;
+constexpr int MAX_K = 16;
+constexpr int TOK_CHUNK = 8;  // tokens one decode GEMV pass carries
+
+// One routed expert of the current call, in ascending expert order inside
+// its class. tok_off / n_tok index the sorted (perm) order.
+struct WorkItem {
+  int32_t e;
+  int32_t slot;     // HBM slot (hit / staged), -1 when streamed
+  int32_t tok_off;  // first sorted position of this expert's tokens
+  int32_t n_tok;    // number of tokens routed to it (>= 1)
+};
+
+// Per-class compact work lists: items [cls][0..n_items) and, for the GEMV
+// kernels, the number of (row block x token chunk) units.
+struct WorkLists {
+  int32_t n_items[N_CLASSES];
+  int32_t pad;
+  WorkItem items[N_CLASSES][MAX_E];
+};
+
+// Host-visible record of the last lookup batch, written by the lookup kernel
+// into mapped pinned memory. The host copy thread reads it after the lookup
+// kernel's event completed.
+struct Mailbox {
+  int32_t seq;        // incremented by each lookup kernel
+  int32_t n_copy;     // slots to fill by H2D copy (staged + prefill loads)
+  int32_t m, qstar, qstage;
+  int32_t n_lookup, n_lookup_cur;
+  int32_t n_hit_cls, n_staged_cls, n_streamed_cls;
+  uint32_t pad_error;  // copy of the device error word at the end of the lookup
+  int32_t copy_key[2 * MAX_E];   // layer*E + e
+  int32_t copy_slot[2 * MAX_E];
+  int32_t lookup_e[2 * MAX_E];
+  int32_t lookup_kind[2 * MAX_E];
+};
+
+// Counters (device), mirrored into ft_stats.
+struct DevCounters {
+  unsigned long long layer_calls, lookups, hits, misses, staged, streamed, bytes_h2d, bytes_zero_copy;
+  int32_t last_m, last_qstar, last_qstage, pad;
+};
+
+// LRU clock state (device).
+struct LruClock {
+  unsigned long long clock;        // last stamp handed out
+  unsigned long long batch_start;  // first stamp of the latest lookup batch
+};
+
+struct Shape {
+  int L, E, k, d, d_ff, wtype;
+  long long C;
+  size_t slot_bytes;
+};
+
+// Arguments of the lookup kernel (one batch of keys of one layer).
+struct LookupArgs {
+  int layer;
+  int use_counts;     // 1: routed experts (counts > 0); 0: all E experts (prefill load)
+  int limit_q;        // 1: apply q* (decode rules); 0: stage every miss
+  int pin_prev;       // 1: also pin the previous batch (prefill prefetch of layer+1)
+  int append;         // 1: append to the mailbox lookup record (prefill second batch)
+  int is_current;     // 1: this batch is the called layer's (m, q*, q_stage are reported)
+  int build_work;     // 1: (re)build the work lists from this batch
+  unsigned bp_mbps, bh_mbps;
+};
+
+// Device pointers of a context.
+struct DevState {
+  int32_t* slot_of;          // [L*E] slot or -1
+  int32_t* key_of;           // [C] key or -1
+  unsigned long long* stamp; // [C]
+  LruClock* clk;
+  DevCounters* ctr;
+  uint32_t* error;
+  WorkLists* work;
+  Mailbox* mbox;             // mapped host memory (device address)
+  // routing scratch
+  float* scores;             // [Tmax*E]
+  int32_t* ids;              // [Tmax*k]
+  float* wts;                // [Tmax*k]
+  int32_t* counts;           // [E]
+  int32_t* offsets;          // [E+1]
+  int32_t* perm;             // [Tmax*k]
+  int32_t* inv;              // [Tmax*k]
+  // expert scratch
+  float* hbuf;               // [Tmax*k, d_ff] SwiGLU activations (fp32)
+  float* ybuf;               // [Tmax*k, d] expert outputs (fp32)
+  __nv_bfloat16* xs;         // [Tmax*k, d] gathered bf16 activations (prefill)
+  __nv_bfloat16* hs;         // [Tmax*k, d_ff] bf16 SwiGLU activations (prefill)
+  float* tscale;             // [L*E*3] NVFP4 tensor scales
+  uint8_t* slots;            // HBM slot pool [C * slot_bytes]
+  const uint8_t* pool_dev;   // device address of the called layer's blobs in the mapped host pool
+};
+
+// ---- launchers (all enqueue on `st`) ----
+// router logits s = x W_r^T + b, fp32 [T, E]
+void launch_router_scores(const Shape& sh, const void* x, const void* w_router, const float* bias, int bias_per_token,
+                          int T, float* scores, cudaStream_t st);
+// top-k + softmax + permutation (counts, offsets, perm, inv)
+void launch_topk_permute(const Shape& sh, const float* scores, int T, DevState& ds, int32_t* ids_out,
+                         float* w_out, cudaStream_t st);
+// one lookup batch; writes work lists, mailbox, counters
+void launch_lookup(const Shape& sh, const LookupArgs& a, DevState& ds, cudaStream_t st);
+// decode / fallback experts (SIMT grouped GEMV) for one work class
+void launch_expert_gemv(const Shape& sh, int cls, int layer, const void* x, int T, DevState& ds, int max_items,
+                        int max_tok, cudaStream_t st);
+// y[t] = sum_j w[t,j] Y[inv[t*k+j]]
+void launch_combine(const Shape& sh, int T, DevState& ds, void* y, cudaStream_t st);
+// zero-copy read probe: reads `bytes` from src, returns nothing useful
+void launch_read_probe(const uint8_t* src, size_t bytes, unsigned long long* sink, cudaStream_t st);
+
+}  // namespace ft

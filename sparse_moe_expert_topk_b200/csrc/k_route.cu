@@ -1,0 +1,249 @@
+// Router of one MoE layer: logits, top-k with softmax weights, and the stable
+// token -> expert permutation.
+//
+// Each token passes through k of the layer's E experts ([paperlens]
+// "MoEは扉を開けると同時に、別の扉を閉める", paper §1). The pages do not give the
+// router function; this follows the reading documented with the C ABI:
+// logits s = x W_r^T + b in fp32, the k largest logits (equal logits -> lower
+// expert index), softmax over those k.
+#include "ft_internal.cuh"
+
+namespace ft {
+
+namespace {
+
+__device__ __forceinline__ void to_f32x8(const uint4 v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+// Logits for 8 experts (one warp each) x up to TT tokens per CTA.
+// grid: (ceil(E/8), ceil(T/TT)); block 256.
+template <typename AT, int TT>
+__global__ void __launch_bounds__(256) router_scores_kernel(const AT* __restrict__ x, const AT* __restrict__ wr,
+                                                            const float* __restrict__ bias, int bias_per_token,
+                                                            int T, int E, int d, float* __restrict__ scores) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.x * 8 + warp;
+  const int t0 = blockIdx.y * TT;
+  if (e >= E) return;
+  const int nt = min(TT, T - t0);
+  float acc[TT];
+#pragma unroll
+  for (int t = 0; t < TT; ++t) acc[t] = 0.f;
+  constexpr int VN = 16 / sizeof(AT);  // elements per 16-byte vector
+  const int nv = d / VN;
+  const uint4* wrow = reinterpret_cast<const uint4*>(wr + (size_t)e * d);
+  for (int v = lane; v < nv; v += 32) {
+    const uint4 wv = __ldg(wrow + v);
+#pragma unroll
+    for (int t = 0; t < TT; ++t) {
+      if (t < nt) {
+        const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + (size_t)(t0 + t) * d) + v);
+        if constexpr (sizeof(AT) == 2) {
+          float wf[8], xf[8];
+          to_f32x8(wv, wf);
+          to_f32x8(xv, xf);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[t] = fmaf(wf[i], xf[i], acc[t]);
+        } else {
+          acc[t] = fmaf(__uint_as_float(wv.x), __uint_as_float(xv.x), acc[t]);
+          acc[t] = fmaf(__uint_as_float(wv.y), __uint_as_float(xv.y), acc[t]);
+          acc[t] = fmaf(__uint_as_float(wv.z), __uint_as_float(xv.z), acc[t]);
+          acc[t] = fmaf(__uint_as_float(wv.w), __uint_as_float(xv.w), acc[t]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < TT; ++t) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
+  }
+  if (lane < nt) {
+    float a = 0.f;
+#pragma unroll
+    for (int t = 0; t < TT; ++t)
+      if (t == lane) a = acc[t];
+    const int tt = t0 + lane;
+    float b = 0.f;
+    if (bias) b = bias_per_token ? bias[(size_t)tt * E + e] : bias[e];
+    scores[(size_t)tt * E + e] = a + b;
+  }
+}
+
+// One warp per token: k rounds of a warp arg-max (larger logit first, equal
+// logits -> lower index), then softmax over the chosen k.
+__global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restrict__ scores, int T, int E, int k,
+                                                           int32_t* __restrict__ ids, float* __restrict__ wts) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= T) return;
+  constexpr int PER = MAX_E / 32;
+  float v[PER];
+  uint32_t taken = 0;
+  const float* s = scores + (size_t)warp * E;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int e = i * 32 + lane;
+    v[i] = e < E ? s[e] : 0.f;
+  }
+  float top0 = 0.f, sel[MAX_K];
+  int sid[MAX_K];
+  for (int j = 0; j < k; ++j) {
+    float bv = 0.f;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int e = i * 32 + lane;
+      if (e < E && !((taken >> i) & 1u)) {
+        if (be == 0x7fffffff || v[i] > bv) {  // ascending e per lane: strict > keeps the lower index
+          bv = v[i];
+          be = e;
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      const bool better = (oe != 0x7fffffff) && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be));
+      if (better) {
+        bv = ov;
+        be = oe;
+      }
+    }
+    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    sel[j] = bv;
+    sid[j] = be;
+    if (j == 0) top0 = bv;
+  }
+  float den = 0.f, ex[MAX_K];
+  for (int j = 0; j < k; ++j) {
+    ex[j] = expf(sel[j] - top0);
+    den += ex[j];
+  }
+  if (lane == 0) {
+    for (int j = 0; j < k; ++j) {
+      ids[(size_t)warp * k + j] = sid[j];
+      wts[(size_t)warp * k + j] = ex[j] / den;
+    }
+  }
+}
+
+// Stable counting sort of the n = T*k routing ids by expert, one CTA of 1024
+// threads. Sorted order = (expert, flat index t*k+j). Within a 1024-entry
+// chunk a thread's rank among equal experts comes from __match_any_sync
+// inside its warp plus the counts of the lower warps.
+__global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict__ ids, int n, int E,
+                                                       int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                                       int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
+  extern __shared__ int32_t smem[];
+  int32_t* wcnt = smem;                // [32][E]
+  int32_t* run = smem + 32 * E;        // [E] next free position per expert
+  int32_t* tot = run + E;              // [E] per-chunk totals
+  int32_t* cnt = tot + E;              // [E]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int e = tid; e < E; e += 1024) cnt[e] = 0;
+  __syncthreads();
+  for (int i = tid; i < n; i += 1024) atomicAdd(&cnt[ids[i]], 1);
+  __syncthreads();
+  if (warp == 0) {  // exclusive scan of cnt over E <= 512 entries, 16 per lane
+    constexpr int PER = MAX_E / 32;
+    int local[PER], s = 0;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int e = lane * PER + i;
+      local[i] = e < E ? cnt[e] : 0;
+      s += local[i];
+    }
+    int incl = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int base = incl - s;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int e = lane * PER + i;
+      if (e < E) {
+        run[e] = base;
+        offsets[e] = base;
+        counts[e] = local[i];
+      }
+      base += local[i];
+    }
+    if (lane == 31) offsets[E] = incl;
+  }
+  __syncthreads();
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int base = 0; base < n; base += 1024) {
+    for (int i = tid; i < 32 * E; i += 1024) wcnt[i] = 0;
+    __syncthreads();
+    const int i = base + tid;
+    const bool valid = i < n;
+    const int e = valid ? ids[i] : E;  // E = sentinel for padding lanes
+    const unsigned same = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(same & lt_mask);
+    if (valid && rank == 0) wcnt[warp * E + e] = __popc(same);
+    __syncthreads();
+    for (int x = tid; x < E; x += 1024) {
+      int r = 0;
+      for (int w = 0; w < 32; ++w) {
+        const int c = wcnt[w * E + x];
+        wcnt[w * E + x] = r;
+        r += c;
+      }
+      tot[x] = r;
+    }
+    __syncthreads();
+    if (valid) {
+      const int pos = run[e] + wcnt[warp * E + e] + rank;
+      perm[pos] = i;
+      inv[i] = pos;
+    }
+    __syncthreads();
+    for (int x = tid; x < E; x += 1024) run[x] += tot[x];
+    __syncthreads();
+  }
+}
+
+}  // namespace
+
+void launch_router_scores(const Shape& sh, const void* x, const void* w_router, const float* bias, int bias_per_token,
+                          int T, float* scores, cudaStream_t st) {
+  constexpr int TT = 8;
+  dim3 grid((sh.E + 7) / 8, (T + TT - 1) / TT);
+  if (sh.wtype == FT_W_F32)
+    router_scores_kernel<float, TT><<<grid, 256, 0, st>>>((const float*)x, (const float*)w_router, bias,
+                                                          bias_per_token, T, sh.E, sh.d, scores);
+  else
+    router_scores_kernel<__nv_bfloat16, TT><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x,
+                                                                  (const __nv_bfloat16*)w_router, bias,
+                                                                  bias_per_token, T, sh.E, sh.d, scores);
+}
+
+size_t permute_smem_bytes(int E) { return sizeof(int32_t) * (size_t)(32 * E + 3 * E); }
+
+void launch_topk_permute(const Shape& sh, const float* scores, int T, DevState& ds, int32_t* ids_out, float* w_out,
+                         cudaStream_t st) {
+  const int warps_per_cta = 8;
+  topk_softmax_kernel<<<(T + warps_per_cta - 1) / warps_per_cta, 32 * warps_per_cta, 0, st>>>(
+      scores, T, sh.E, sh.k, ds.ids, ds.wts);
+  permute_kernel<<<1, 1024, permute_smem_bytes(sh.E), st>>>(ds.ids, T * sh.k, sh.E, ds.counts, ds.offsets, ds.perm,
+                                                           ds.inv);
+  if (ids_out) cudaMemcpyAsync(ids_out, ds.ids, sizeof(int32_t) * T * sh.k, cudaMemcpyDeviceToDevice, st);
+  if (w_out) cudaMemcpyAsync(w_out, ds.wts, sizeof(float) * T * sh.k, cudaMemcpyDeviceToDevice, st);
+}
+
+cudaError_t route_kernels_init(int E) {
+  return cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)permute_smem_bytes(E));
+}
+
+}  // namespace ft

@@ -1,0 +1,92 @@
+"""Helpers for the GPU parity tests: seeded inputs with a guaranteed top-k
+gap, and an oracle replay of a sequence of layer calls over the same pinned
+expert blobs the library reads."""
+from __future__ import annotations
+
+from collections import OrderedDict
+
+import numpy as np
+import torch
+
+import ftgen
+from oracle import cache as ocache
+from oracle import formats as ofmt
+from oracle import moe as omoe
+
+GAP = 1e-3  # minimum k-th vs (k+1)-th logit gap of every token
+
+
+def gap_hidden(wl, T, seed, w_router, bias, max_rounds=60):
+    """x [T, d] from ftgen with every token's top-k gap >= GAP (tokens whose
+    oracle logits fall short are redrawn with the next attempt number)."""
+    attempts = np.zeros(T, dtype=np.int64)
+    x = ftgen.hidden(T, wl.d, wl.wtype, seed)
+    wr = w_router.float().cpu().numpy()
+    for _ in range(max_rounds):
+        s32 = omoe.router_logits(x.float().numpy(), wr, bias)
+        bad = np.nonzero(omoe.topk_gap(s32, wl.k) < GAP)[0]
+        if bad.size == 0:
+            return x
+        for t in bad:
+            attempts[t] += 1
+            x[t] = ftgen.hidden_row(wl.d, wl.wtype, seed, int(t), int(attempts[t]))
+        if bias is not None and np.ndim(bias) == 2:
+            pass
+    raise RuntimeError("could not enforce the top-k gap")
+
+
+class ExpertWeights:
+    """fp64 expert matrices decoded by the oracle from the pinned pool blobs,
+    with a small LRU of decoded experts."""
+
+    def __init__(self, harness, keep=24):
+        self.h = harness
+        self.keep = keep
+        self.cache = OrderedDict()
+
+    def __call__(self, layer, e):
+        key = (layer, e)
+        if key in self.cache:
+            self.cache.move_to_end(key)
+            return self.cache[key]
+        wl = self.h.wl
+        ts = self.h.tscales.get(key)
+        w = ofmt.unpack_expert(self.h.blob(layer, e).copy(), wl.d, wl.d_ff, wl.wtype, ts)
+        self.cache[key] = w
+        if len(self.cache) > self.keep:
+            self.cache.popitem(last=False)
+        return w
+
+
+def tol_for(wtype):
+    """max |gpu - oracle| allowed, as a fraction of rms(oracle)."""
+    return {ftgen.W_F32: 1e-4, ftgen.W_BF16: 2e-2, ftgen.W_NVFP4: 4e-2}[wtype]
+
+
+def check_close(y_gpu, y_ref, wtype, what=""):
+    y_gpu = np.asarray(y_gpu, np.float64)
+    rms = float(np.sqrt(np.mean(y_ref ** 2)))
+    err = float(np.max(np.abs(y_gpu - y_ref))) if y_ref.size else 0.0
+    assert err <= tol_for(wtype) * rms, f"{what}: max|d| {err:.3e} > {tol_for(wtype)} * rms {rms:.3e}"
+    return err / rms if rms > 0 else 0.0
+
+
+def gpu_route(harness, T):
+    import sparse_moe_expert_topk_b200 as ft
+    return ft.ft_moe_last_route(harness.ctx, harness.wl.E, T * harness.wl.k)
+
+
+def expected_record(rec, E):
+    """Oracle cache record -> (lookup experts, kinds) in lookup order."""
+    es = [e for (_, e, _) in rec["lookups"]]
+    ks = [k for (_, _, k) in rec["lookups"]]
+    return es, ks
+
+
+def oracle_cache(harness):
+    wl = harness.wl
+    return ocache.ExpertCache(harness.L, wl.E, harness.C, wl.bp_mbps, wl.bh_mbps)
+
+
+def to_np(t):
+    return t.detach().float().cpu().numpy()

@@ -1,0 +1,78 @@
+"""The C-ABI library loads and exports every entry point include/ft_moe.h
+declares; argument validation works without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import sparse_moe_expert_topk_b200 as ft
+from conftest import ROOT
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_moe_expert_topk_b200 import build
+    build.build()
+    return ft.lib()
+
+
+def _declared():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z_0-9]*\s*\*?\s*(ft_[a-z_0-9]+)\s*\(", src, re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = _declared()
+    assert len(declared) >= 14
+    assert sorted(ft.EXPORTS) == declared
+    for name in declared:
+        assert isinstance(getattr(lib, name), ctypes._CFuncPtr), name
+
+
+def test_slot_bytes(lib):
+    for wtype, n in ((ft.FT_W_F32, 98304), (ft.FT_W_BF16, 37748736), (ft.FT_W_NVFP4, 10616832)):
+        d, dff = (64, 128) if wtype == ft.FT_W_F32 else (4096, 1536)
+        cfg = ft.make_config(1, 8, 2, d, dff, wtype, 4, 16)
+        assert ft.ft_moe_slot_bytes(cfg) == n
+
+
+@pytest.mark.parametrize("field,value", [("n_layers", 0), ("n_experts", 0), ("n_experts", 513), ("top_k", 0),
+                                         ("top_k", 9), ("d_model", 100), ("d_ff", 32), ("wtype", 3),
+                                         ("cache_slots", -1), ("cache_slots", 9), ("max_tokens", 0),
+                                         ("device", -1)])
+def test_config_validation(lib, field, value):
+    cfg = ft.make_config(1, 8, 2, 64, 128, ft.FT_W_F32, 4, 16)
+    setattr(cfg, field, value)
+    with pytest.raises(ft.FtError) as ei:
+        ft.ft_moe_slot_bytes(cfg)
+    assert ei.value.status == ft.FT_EINVAL
+
+
+def test_status_strings(lib):
+    assert ft.status_str(ft.FT_OK) == "ok"
+    assert ft.status_str(ft.FT_ETIMEOUT) == "timed out"
+    assert ft.status_str(99) == "unknown status"
+
+
+def test_null_arguments_are_rejected(lib):
+    P = ctypes.c_void_p
+    assert lib.ft_moe_set_router(None, 0, P(1)) == ft.FT_EINVAL
+    assert lib.ft_set_bandwidths(None, 1, 1) == ft.FT_EINVAL
+    assert lib.ft_cache_stats(None, None) == ft.FT_EINVAL
+    assert lib.ft_moe_layer_forward(None, 0, 0, None, 0, None, 0, None, None, None) == ft.FT_EINVAL
+    lib.ft_moe_destroy(None)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
+def test_init_without_gpu_fails_cleanly(lib):
+    cfg = ft.make_config(1, 8, 2, 64, 128, ft.FT_W_F32, 4, 16)
+    with pytest.raises(ft.FtError) as ei:
+        ft.ft_moe_init(cfg, None, 1)
+    assert ei.value.status == ft.FT_ECUDA
