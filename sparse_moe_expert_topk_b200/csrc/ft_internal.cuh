@@ -53,6 +53,7 @@ struct Mailbox {
   int32_t n_lookup, n_lookup_cur;
   int32_t n_hit_cls, n_staged_cls, n_streamed_cls;
   uint32_t pad_error;  // copy of the device error word at the end of the lookup
+  int32_t n_tok_cls[3];  // tokens routed to the experts of each work class
   int32_t copy_key[2 * MAX_E];   // layer*E + e
   int32_t copy_slot[2 * MAX_E];
   int32_t lookup_e[2 * MAX_E];
@@ -121,14 +122,16 @@ struct DevState {
 // router logits s = x W_r^T + b, fp32 [T, E]
 void launch_router_scores(const Shape& sh, const void* x, const void* w_router, const float* bias, int bias_per_token,
                           int T, float* scores, cudaStream_t st);
-// top-k + softmax + permutation (counts, offsets, perm, inv)
-void launch_topk_permute(const Shape& sh, const float* scores, int T, DevState& ds, int32_t* ids_out,
-                         float* w_out, cudaStream_t st);
+// top-k + softmax weights (ids, wts)
+void launch_topk(const Shape& sh, const float* scores, int T, DevState& ds, cudaStream_t st);
+// stable permutation (counts, offsets, perm, inv)
+void launch_permute(const Shape& sh, int T, DevState& ds, cudaStream_t st);
 // one lookup batch; writes work lists, mailbox, counters
 void launch_lookup(const Shape& sh, const LookupArgs& a, DevState& ds, cudaStream_t st);
-// decode / fallback experts (SIMT grouped GEMV) for one work class
-void launch_expert_gemv(const Shape& sh, int cls, int layer, const void* x, int T, DevState& ds, int max_items,
-                        int max_tok, cudaStream_t st);
+// decode / fallback experts (SIMT grouped GEMV) for one work class;
+// phase 0: gate/up + SwiGLU into hbuf, phase 1: down into ybuf
+void launch_expert_gemv(const Shape& sh, int cls, int phase, int layer, const void* x, int T, DevState& ds,
+                        int max_items, int max_tok, cudaStream_t st);
 // y[t] = sum_j w[t,j] Y[inv[t*k+j]]
 void launch_combine(const Shape& sh, int T, DevState& ds, void* y, cudaStream_t st);
 // zero-copy read probe: reads `bytes` from src, returns nothing useful

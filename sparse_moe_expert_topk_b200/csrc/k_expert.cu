@@ -252,7 +252,7 @@ __device__ __forceinline__ size_t row_bytes(int wt, int K) {
 }
 
 __device__ __forceinline__ const uint8_t* blob_of(const GemvArgs& a, const WorkItem& it) {
-  if (a.cls == KIND_STREAMED) return a.pool + ((size_t)a.layer * a.E + it.e) * a.slot_bytes;
+  if (a.cls == KIND_STREAMED) return a.pool + (size_t)it.e * a.slot_bytes;  // a.pool: this layer's chunk
   return a.slots + (size_t)it.slot * a.slot_bytes;
 }
 
@@ -472,8 +472,8 @@ void launch_gemv_variant(int wtype, int ntmax, int grid, const GemvArgs& a, int 
   }
 }
 
-void launch_expert_gemv(const Shape& sh, int cls, int layer, const void* x, int T, DevState& ds, int max_items,
-                        int max_tok, cudaStream_t st) {
+void launch_expert_gemv(const Shape& sh, int cls, int phase, int layer, const void* x, int T, DevState& ds,
+                        int max_items, int max_tok, cudaStream_t st) {
   GemvArgs a;
   a.work = ds.work;
   a.cls = cls;
@@ -491,16 +491,15 @@ void launch_expert_gemv(const Shape& sh, int cls, int layer, const void* x, int 
   a.tscale = ds.tscale;
   a.hbuf = ds.hbuf;
   a.ybuf = ds.ybuf;
-  // upper bound of units, to size the grid without reading the device list
+  // upper bound of (item x token chunk) pairs, to size the grid without
+  // reading the device work list; the kernel strides over the true count
   const long long chunks = (long long)max_items + (long long)max_tok / TOK_CHUNK;
-  for (int phase = 0; phase < 2; ++phase) {
-    const int rows = WARPS * (phase == 0 ? RW_GU : RW_DN);
-    const long long units = chunks * ((phase == 0 ? sh.d_ff : sh.d) / rows);
-    const int grid = (int)(units < g_gemv_grid ? units : g_gemv_grid);
-    if (grid <= 0) return;
-    const int ntmax = T >= 5 ? 8 : (T >= 3 ? 4 : T);
-    launch_gemv_variant(sh.wtype, ntmax, grid, a, phase, st);
-  }
+  const int rows = WARPS * (phase == 0 ? RW_GU : RW_DN);
+  const long long units = chunks * ((phase == 0 ? sh.d_ff : sh.d) / rows);
+  const int grid = (int)(units < g_gemv_grid ? units : g_gemv_grid);
+  if (grid <= 0) return;
+  const int ntmax = T >= 5 ? 8 : (T >= 3 ? 4 : T);
+  launch_gemv_variant(sh.wtype, ntmax, grid, a, phase, st);
 }
 
 void launch_combine(const Shape& sh, int T, DevState& ds, void* y, cudaStream_t st) {

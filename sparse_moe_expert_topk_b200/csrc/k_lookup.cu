@@ -73,7 +73,7 @@ __global__ void __launch_bounds__(NT) lookup_kernel(LookupArgs a, int E, long lo
   __shared__ unsigned long long s_prefix, s_mask;
   __shared__ int s_remaining, s_ncand, s_avail;
   __shared__ unsigned long long s_c0, s_epoch, s_bstart;
-  __shared__ int s_cbase, s_lbase;
+  __shared__ int s_cbase, s_lbase, s_tok;
 
   const int tid = threadIdx.x;
   Mailbox* mb = ds.mbox;
@@ -224,6 +224,13 @@ __global__ void __launch_bounds__(NT) lookup_kernel(LookupArgs a, int E, long lo
     for (int c = 0; c < N_CLASSES; ++c) {
       int n_c;
       const int r = block_scan_flag(act && kind == c, scan, n_c);
+      int tok = (act && kind == c) ? ds.counts[e] : 0;
+      for (int o = 16; o > 0; o >>= 1) tok += __shfl_xor_sync(0xffffffffu, tok, o);
+      if (tid == 0) s_tok = 0;
+      __syncthreads();
+      if ((tid & 31) == 0) atomicAdd(&s_tok, tok);
+      __syncthreads();
+      if (tid == 0) mb->n_tok_cls[c] = s_tok;
       if (act && kind == c) {
         WorkItem it;
         it.e = e;

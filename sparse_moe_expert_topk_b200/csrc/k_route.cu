@@ -230,15 +230,15 @@ void launch_router_scores(const Shape& sh, const void* x, const void* w_router, 
 
 size_t permute_smem_bytes(int E) { return sizeof(int32_t) * (size_t)(32 * E + 3 * E); }
 
-void launch_topk_permute(const Shape& sh, const float* scores, int T, DevState& ds, int32_t* ids_out, float* w_out,
-                         cudaStream_t st) {
+void launch_topk(const Shape& sh, const float* scores, int T, DevState& ds, cudaStream_t st) {
   const int warps_per_cta = 8;
   topk_softmax_kernel<<<(T + warps_per_cta - 1) / warps_per_cta, 32 * warps_per_cta, 0, st>>>(
       scores, T, sh.E, sh.k, ds.ids, ds.wts);
+}
+
+void launch_permute(const Shape& sh, int T, DevState& ds, cudaStream_t st) {
   permute_kernel<<<1, 1024, permute_smem_bytes(sh.E), st>>>(ds.ids, T * sh.k, sh.E, ds.counts, ds.offsets, ds.perm,
                                                            ds.inv);
-  if (ids_out) cudaMemcpyAsync(ids_out, ds.ids, sizeof(int32_t) * T * sh.k, cudaMemcpyDeviceToDevice, st);
-  if (w_out) cudaMemcpyAsync(w_out, ds.wts, sizeof(float) * T * sh.k, cudaMemcpyDeviceToDevice, st);
 }
 
 cudaError_t route_kernels_init(int E) {
