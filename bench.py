@@ -1,0 +1,453 @@
+"""Benchmark of the routed-MoE layer over the HBM expert cache.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload decode_bf16]
+
+One step is one pass of the whole hot path over one batch of synthetic input:
+for the default workload (single-layer BF16 decode: E=256, top-6, d=4096,
+d_ff=1536, 37% cache = 94 slots, LRU, B_P:B_H = 52.7:77.3) a step starts from
+a cold cache (every expert on the host, as on a first request) and runs the
+64-step decode trace at batch 1, 4 and 16 -- 192 layer calls, 1344 tokens.
+Inputs (hidden states, router weights, Zipf router bias) are resident in HBM
+before the timed region; the expert pool lives in pinned host memory and
+reaches the GPU through the cache (copy engine) or zero-copy reads, which is
+the workload. The pool (9.7 GB) and the slot pool (3.5 GB) are larger than
+L2, so no L2 flush is needed between steps.
+
+Rank 0 prints one JSON line. With N > 1 (torchrun) every rank runs an
+independent replica on its own data (weak scaling, no collective on the data
+path); value = all ranks' tokens / the max over ranks of the device time.
+
+--impl reference times the CPU oracle (oracle/) on the host cores, on the
+same workload, metric and units: each step is a bounded sample of it.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "MoE-layer tokens/s (decode, prefill) and % of HBM/tensor/host-link roofline"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.dev)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.strip().splitlines():
+            f = [v.strip() for v in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, world, device):
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(v, world, device):
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------
+# workload inputs
+# --------------------------------------------------------------------------
+def decode_inputs(wl, rank, device):
+    """Per batch size T: 64 steps of hidden states [T, d] (bf16, device) and
+    the Zipf(1.1) router log-bias [E] (fp32, device)."""
+    import ftgen
+    bias = torch.as_tensor(ftgen.zipf_log_bias(wl.E, wl.extra["zipf_s"], wl.seed("zipf"))).to(device)
+    xs = {}
+    for T in wl.batches:
+        xs[T] = [ftgen.hidden(T, wl.d, wl.wtype, wl.seed("bench", rank, T, s)).to(device) for s in range(wl.steps)]
+    return xs, bias
+
+
+def run_step(h, xs, bias, ys):
+    import sparse_moe_expert_topk_b200 as ft
+    ft.ft_moe_reset_cache(h.ctx)
+    for T, seq in xs.items():
+        y = ys[T]
+        for x in seq:
+            ft.ft_moe_layer_forward(h.ctx, 0, ft.FT_DECODE, x, T, bias, 0, y)
+
+
+def run_step_e2e(h, xs_host, bias, x_dev, y_dev, y_host):
+    """Same step through the public call with host buffers: every call copies
+    its hidden states host->device and its output device->host."""
+    import sparse_moe_expert_topk_b200 as ft
+    ft.ft_moe_reset_cache(h.ctx)
+    for T, seq in xs_host.items():
+        for i, xh in enumerate(seq):
+            x_dev[T].copy_(xh, non_blocking=True)
+            ft.ft_moe_layer_forward(h.ctx, 0, ft.FT_DECODE, x_dev[T], T, bias, 0, y_dev[T])
+            y_host[T][i].copy_(y_dev[T], non_blocking=True)
+
+
+# --------------------------------------------------------------------------
+# roofline from the per-kernel profile
+# --------------------------------------------------------------------------
+KERNEL_SOURCES = {"gemv": "sparse_moe_expert_topk_b200/csrc/k_expert.cu",
+                  "gemm_tc": "sparse_moe_expert_topk_b200/csrc/k_gemm_tc.cu",
+                  "router": "sparse_moe_expert_topk_b200/csrc/k_route.cu",
+                  "lookup": "sparse_moe_expert_topk_b200/csrc/k_lookup.cu"}
+
+
+def _source_sha(kernel_name):
+    import hashlib
+    key = next((k for k in KERNEL_SOURCES if kernel_name.startswith(k)), None)
+    if key is None:
+        return None
+    with open(os.path.join(ROOT, KERNEL_SOURCES[key]), "rb") as f:
+        return hashlib.sha1(f.read()).hexdigest()[:12]
+
+
+def ncu_traffic(kernel_name, launches_per_step):
+    """DRAM bytes per launch of `kernel_name` from the committed ncu summary,
+    or None if there is none or the kernel source changed since."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel_name)
+    if not e or e.get("source_sha") != _source_sha(kernel_name):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def roofline(prof, peaks, peak_kind, link_gbs):
+    rows = {}
+    for name, r in prof.items():
+        if r["ms"] <= 0 or name == "h2d_stage_copies":
+            continue
+        gbs = r["bytes"] / (r["ms"] * 1e6)
+        if name.startswith("gemm_tc"):
+            bound, peak, unit, ach = "tensor", peaks["bf16_tflops"], "TFLOP/s", r["flops"] / (r["ms"] * 1e9)
+        elif name.endswith("streamed"):
+            bound, peak, unit, ach = "host_link", link_gbs, "GB/s", gbs
+        else:
+            bound, peak, unit, ach = "hbm", peaks["hbm_gbs"], "GB/s", gbs
+        rows[name] = {"bound": bound, "achieved": round(ach, 2), "peak": round(peak, 2), "unit": unit,
+                      "frac": round(ach / peak, 4) if peak else None, "ms_total": round(r["ms"], 3),
+                      "launches": int(r["launches"]), "bytes_per_launch": r["bytes"] / max(r["launches"], 1)}
+    tot = sum(v["ms_total"] for v in rows.values()) or 1.0
+    for v in rows.values():
+        v["share"] = round(v["ms_total"] / tot, 4)
+    dom = max(rows, key=lambda k: rows[k]["ms_total"]) if rows else None
+    out = None
+    if dom:
+        v = rows[dom]
+        out = {"kernel": dom, "bound": v["bound"], "achieved": v["achieved"], "peak": v["peak"], "unit": v["unit"],
+               "frac": v["frac"], "traffic": ncu_traffic(dom, v["launches"]),
+               "peak_source": (peak_kind if v["bound"] != "host_link" else "measured H2D copy-engine GB/s, this run"),
+               "algorithmic_bytes_per_launch": round(v["bytes_per_launch"])}
+    return out, rows
+
+
+# --------------------------------------------------------------------------
+# CPU oracle timing (baseline and reference arm)
+# --------------------------------------------------------------------------
+def oracle_sample(wl, blob_of, seconds, rank=0):
+    """Run the oracle (routing + shared LRU with q* + per-token SwiGLU experts)
+    over the workload's decode calls, in trace order, until `seconds` elapse.
+    Returns (tokens, elapsed_s, calls)."""
+    import ftgen
+    from oracle import cache as ocache
+    from oracle import formats as ofmt
+    from oracle import moe as omoe
+    bias = ftgen.zipf_log_bias(wl.E, wl.extra["zipf_s"], wl.seed("zipf"))
+    wr = ftgen.router_weight(wl.E, wl.d, wl.wtype, wl.seed("router", 0)).float().numpy()
+    oc = ocache.ExpertCache(1, wl.E, wl.cache_slots, wl.bp_mbps, wl.bh_mbps)
+    tokens = calls = 0
+    t0 = time.perf_counter()
+    for T in wl.batches:
+        for s in range(wl.steps):
+            x = ftgen.hidden(T, wl.d, wl.wtype, wl.seed("bench", rank, T, s)).float().numpy()
+            ids, _, _ = omoe.route(x, wr, bias, wl.k)
+            counts, _, _, _ = omoe.permutation(ids, wl.E)
+            oc.forward(0, ocache.DECODE, counts)
+            omoe.layer_forward(x, wr, bias, wl.k, lambda e: ofmt.unpack_expert(blob_of(e), wl.d, wl.d_ff, wl.wtype))
+            tokens += T
+            calls += 1
+            if time.perf_counter() - t0 >= seconds:
+                return tokens, time.perf_counter() - t0, calls
+    return tokens, time.perf_counter() - t0, calls
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def cpu_blob_source(wl):
+    """Expert blobs generated on the CPU from the workload's seeds (same
+    recipe as the pool the GPU arm reads)."""
+    import ftgen
+    cache = {}
+
+    def blob(e):
+        if e not in cache:
+            cache[e] = ftgen.expert_blob(wl.d, wl.d_ff, wl.wtype, wl.seed("expert", 0, e)).numpy()
+        return cache[e]
+    return blob
+
+
+def run_reference(args, wl, world, rank):
+    if rank != 0:
+        return 0
+    blob = cpu_blob_source(wl)
+    per_step_s = 10.0
+    for _ in range(args.warmup):
+        oracle_sample(wl, blob, 0.5)
+    tok = el = 0.0
+    calls = 0
+    for _ in range(args.steps):
+        t, e, c = oracle_sample(wl, blob, per_step_s)
+        tok += t
+        el += e
+        calls += c
+    value = tok / el
+    cores = blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * el / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "E": wl.E, "top_k": wl.k, "d": wl.d, "d_ff": wl.d_ff,
+                       "cache_slots": wl.cache_slots, "batches": list(wl.batches), "decode_steps": wl.steps},
+            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"first {calls} decode calls of the trace in {args.steps} steps of "
+                                       f"~{per_step_s:.0f} s each (routing, shared LRU with q*, fp64 experts)"},
+            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode_bf16")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-only", action="store_true", help="one warm-up and one profiled step (for ncu)")
+    args = ap.parse_args()
+    if args.warmup < 3 and not args.profile_only:
+        raise SystemExit("--warmup must be >= 3")
+
+    import ftgen
+    wl = ftgen.workload(args.workload)
+    if args.workload != "decode_bf16":
+        raise SystemExit("bench.py times the single-layer BF16 decode workload (decode_bf16)")
+    world, rank, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        r = run_reference(args, wl, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return r
+
+    import sparse_moe_expert_topk_b200 as ft
+    from ftgen.ctx import Harness
+    if not os.path.exists(ft.LIB_PATH):
+        from sparse_moe_expert_topk_b200 import build
+        build.build()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    h = Harness(wl, max_tokens=max(wl.batches), device=local)
+    xs, bias = decode_inputs(wl, rank, device)
+    ys = {T: torch.empty(T, wl.d, dtype=torch.bfloat16, device=device) for T in wl.batches}
+    tokens_per_step = wl.steps * sum(wl.batches)
+    stream = h.stream
+
+    if args.profile_only:
+        run_step(h, xs, bias, ys)
+        ft.ft_moe_profile(h.ctx, True)
+        run_step(h, xs, bias, ys)
+        prof = ft.ft_moe_profile_read(h.ctx)
+        if rank == 0:
+            print(json.dumps({k: {kk: round(vv, 4) if isinstance(vv, float) else vv for kk, vv in v.items()}
+                              for k, v in prof.items()}), flush=True)
+        h.close()
+        return 0
+
+    for _ in range(args.warmup):
+        run_step(h, xs, bias, ys)
+    launches0 = ft.ft_cache_stats(h.ctx)["kernel_launches"]
+    barrier(world)
+    torch.cuda.synchronize(device)
+    sampler = ClockSampler(local)
+    sampler.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        run_step(h, xs, bias, ys)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    clocks = sampler.stop()
+    barrier(world)
+    ms = e0.elapsed_time(e1)
+    st = ft.ft_cache_stats(h.ctx)
+    launches = (st["kernel_launches"] - launches0) / args.steps
+    ms_max = max_over_ranks(ms, world, device)
+    total_tokens = sum_over_ranks(tokens_per_step * args.steps, world, device)
+    value = total_tokens / (ms_max / 1e3)
+
+    # per-kernel profile of one more step (events around every launch)
+    ft.ft_moe_profile(h.ctx, True)
+    run_step(h, xs, bias, ys)
+    prof = ft.ft_moe_profile_read(h.ctx)
+    ft.ft_moe_profile(h.ctx, False)
+    st1 = ft.ft_cache_stats(h.ctx)
+    miss_rate = st1["misses"] / max(st1["lookups"], 1)
+
+    # host link: copy engine and zero-copy kernel reads, 1 GiB
+    h2d_gbs, zc_gbs = ft.ft_moe_probe_link(h.ctx, 1 << 30)
+    peaks, peak_kind = load_peaks()
+    roof, rows = roofline(prof, peaks, peak_kind, h2d_gbs)
+
+    # end to end through the public call with host buffers
+    e2e = None
+    if not args.no_e2e:
+        xs_host = {T: [x.cpu().pin_memory() for x in seq] for T, seq in xs.items()}
+        x_dev = {T: torch.empty(T, wl.d, dtype=torch.bfloat16, device=device) for T in wl.batches}
+        y_host = {T: [torch.empty(T, wl.d, dtype=torch.bfloat16).pin_memory() for _ in seq] for T, seq in xs.items()}
+        run_step_e2e(h, xs_host, bias, x_dev, ys, y_host)
+        barrier(world)
+        torch.cuda.synchronize(device)
+        e0.record(stream)
+        for _ in range(args.steps):
+            run_step_e2e(h, xs_host, bias, x_dev, ys, y_host)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1), world, device)
+        io_bytes = tokens_per_step * wl.d * 2
+        e2e = {"value": round(total_tokens / (ms_e2e / 1e3), 3), "unit": UNIT, "h2d_bytes_per_step": io_bytes,
+               "d2h_bytes_per_step": io_bytes}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tok, el, calls = oracle_sample(wl, lambda e: h.blob(0, e), args.cpu_seconds, rank)
+        cpu = {"value": round(tok / el, 4), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"first {calls} decode calls ({tok} tokens, batch 1 first) of the same trace and pool, "
+                         f"{el:.1f} s of CPU work"}
+
+    h.close()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "single-layer BF16 decode, E=256 top-6 d=4096 d_ff=1536, 37% cache (94 slots), "
+                                   "LRU, B_P:B_H=52.7:77.3, 64-step trace at batch 1/4/16 from a cold cache",
+                       "tokens_per_step": tokens_per_step, "layer_calls_per_step": wl.steps * len(wl.batches),
+                       "l2": "inputs larger than L2 (9.7 GB pinned pool, 3.5 GB slot pool)",
+                       "parallelism": f"replicas x{world}"},
+            "miss_rate": round(miss_rate, 4),
+            "cache": {k: st1[k] for k in ("lookups", "hits", "misses", "staged", "streamed")},
+            "host_link": {"h2d_copy_gbs": round(h2d_gbs, 2), "zero_copy_read_gbs": round(zc_gbs, 2)},
+            "roofline": roof, "kernels": rows, "gpu_launches": int(round(launches * args.steps)),
+            "gpu_launches_per_step": round(launches, 1), "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,
+            "peaks": {"kind": peak_kind, "hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"]},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

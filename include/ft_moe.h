@@ -176,6 +176,7 @@ typedef struct {
   int32_t last_qstar;       /* q* of the last decode batch (before the capacity clamp) */
   int32_t last_qstage;      /* misses actually staged in that batch */
   int32_t device_error;     /* 0, or the latched ft_status of a device failure */
+  uint64_t kernel_launches; /* CUDA kernels this context launched */
 } ft_stats;
 ft_status ft_cache_stats(ft_ctx* ctx, ft_stats* out);
 
@@ -213,6 +214,25 @@ ft_status ft_moe_cache_contents(ft_ctx* ctx, int32_t* key_of, uint64_t* stamp);
  * pool into HBM, and GB/s of a kernel reading the same bytes zero-copy from
  * the mapped pool. Synchronises. bytes <= pool size, multiple of 4096. */
 ft_status ft_moe_probe_link(ft_ctx* ctx, uint64_t bytes, double* h2d_gbs, double* zero_copy_gbs);
+
+/* Per-kernel timing. While enabled, every kernel launch (and each group of
+ * staging copies) is bracketed by CUDA events on the stream it runs on, and
+ * tagged with its algorithmic bytes and flops (each weight read once plus
+ * activations in and out). This adds two event records per launch. */
+ft_status ft_moe_profile(ft_ctx* ctx, int32_t enable);
+
+typedef struct {
+  char name[32];        /* kernel, e.g. "gemv_gateup_hit" */
+  uint64_t launches;
+  double ms;            /* summed event time of those launches */
+  double bytes;         /* summed algorithmic bytes */
+  double flops;         /* summed algorithmic flops */
+} ft_kernel_time;
+
+/* Fold finished records into per-kernel totals (synchronises) and copy up to
+ * cap of them to out; *n_out = number of kernels with records. reset != 0
+ * clears the totals after copying. */
+ft_status ft_moe_profile_read(ft_ctx* ctx, ft_kernel_time* out, int32_t cap, int32_t* n_out, int32_t reset);
 
 /* Static string for a status code. */
 const char* ft_status_str(ft_status s);

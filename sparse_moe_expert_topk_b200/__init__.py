@@ -27,7 +27,8 @@ KIND_HIT, KIND_STAGED, KIND_STREAMED = 0, 1, 2
 EXPORTS = (
     "ft_moe_slot_bytes", "ft_moe_init", "ft_moe_destroy", "ft_moe_expert_ptr", "ft_moe_set_tensor_scales",
     "ft_moe_set_router", "ft_moe_layer_forward", "ft_cache_stats", "ft_set_bandwidths", "ft_moe_reset_cache",
-    "ft_moe_last_route", "ft_moe_cache_contents", "ft_moe_probe_link", "ft_status_str",
+    "ft_moe_last_route", "ft_moe_cache_contents", "ft_moe_probe_link", "ft_moe_profile", "ft_moe_profile_read",
+    "ft_status_str",
 )
 
 
@@ -42,10 +43,15 @@ class FtStats(ctypes.Structure):
                 ("misses", ctypes.c_uint64), ("staged", ctypes.c_uint64), ("streamed", ctypes.c_uint64),
                 ("bytes_h2d", ctypes.c_uint64), ("bytes_zero_copy", ctypes.c_uint64),
                 ("last_m", ctypes.c_int32), ("last_qstar", ctypes.c_int32), ("last_qstage", ctypes.c_int32),
-                ("device_error", ctypes.c_int32)]
+                ("device_error", ctypes.c_int32), ("kernel_launches", ctypes.c_uint64)]
 
     def as_dict(self):
         return {k: getattr(self, k) for k, _ in self._fields_}
+
+
+class FtKernelTime(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_uint64), ("ms", ctypes.c_double),
+                ("bytes", ctypes.c_double), ("flops", ctypes.c_double)]
 
 
 class FtError(RuntimeError):
@@ -79,6 +85,8 @@ def lib() -> ctypes.CDLL:
             "ft_moe_last_route": [P] + [P] * 11,
             "ft_moe_cache_contents": [P, P, P],
             "ft_moe_probe_link": [P, U64, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)],
+            "ft_moe_profile": [P, I32],
+            "ft_moe_profile_read": [P, ctypes.POINTER(FtKernelTime), I32, ctypes.POINTER(I32), I32],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -202,3 +210,17 @@ def ft_moe_probe_link(ctx, nbytes):
     h2d, zc = ctypes.c_double(), ctypes.c_double()
     _check("ft_moe_probe_link", lib().ft_moe_probe_link(ctx, nbytes, ctypes.byref(h2d), ctypes.byref(zc)))
     return h2d.value, zc.value
+
+
+def ft_moe_profile(ctx, enable: bool):
+    _check("ft_moe_profile", lib().ft_moe_profile(ctx, 1 if enable else 0))
+
+
+def ft_moe_profile_read(ctx, reset=True) -> dict:
+    """{kernel name: {launches, ms, bytes, flops}} (synchronises)."""
+    cap = 32
+    arr = (FtKernelTime * cap)()
+    n = ctypes.c_int32()
+    _check("ft_moe_profile_read", lib().ft_moe_profile_read(ctx, arr, cap, ctypes.byref(n), 1 if reset else 0))
+    return {arr[i].name.decode(): dict(launches=arr[i].launches, ms=arr[i].ms, bytes=arr[i].bytes,
+                                       flops=arr[i].flops) for i in range(min(n.value, cap))}

@@ -27,8 +27,10 @@ cudaError_t route_kernels_init(int E);
 cudaError_t expert_kernels_init(int device);
 void launch_prefill_work(const Shape& sh, int layer, DevState& ds, cudaStream_t st);
 bool prefill_tc_supported(const Shape& sh);
-cudaError_t prefill_tc_init(const Shape& sh, int max_rows);
-void launch_prefill_tc(const Shape& sh, int layer, const void* x, int T, DevState& ds, cudaStream_t st);
+cudaError_t prefill_tc_init(const Shape& sh, DevState& ds, int max_rows);
+void prefill_tc_free(DevState& ds);
+void launch_prefill_gather(const Shape& sh, const void* x, int T, DevState& ds, cudaStream_t st);
+void launch_gemm_tc(const Shape& sh, int phase, int T, DevState& ds, cudaStream_t st);
 }  // namespace ft
 
 using namespace ft;
@@ -53,6 +55,21 @@ struct ft_ctx {
   ft_status latched = FT_OK;
   bool use_tc = false;
   unsigned long long* probe_sink = nullptr;
+  // launch accounting and optional per-launch CUDA-event profiling
+  unsigned long long kernel_launches = 0;
+  bool profiling = false;
+  struct ProfRec {
+    int name;
+    cudaEvent_t a, b;
+    double bytes, flops;
+  };
+  std::vector<ProfRec> pend;
+  std::vector<cudaEvent_t> evpool;
+  struct Agg {
+    unsigned long long n = 0;
+    double ms = 0, bytes = 0, flops = 0;
+  };
+  std::vector<Agg> agg;
 };
 
 namespace {
@@ -121,10 +138,16 @@ void free_all(ft_ctx* c) {
     if (p) cudaFree(p);
   for (uint8_t* p : c->pool_host)
     if (p) cudaFreeHost(p);
+  prefill_tc_free(d);
   if (c->mbox_host) cudaFreeHost(c->mbox_host);
   cudaEvent_t evs[] = {c->ev_look, c->ev_side, c->ev_copy, c->ev_pf[0], c->ev_pf[1], c->ev_t0, c->ev_t1};
   for (cudaEvent_t e : evs)
     if (e) cudaEventDestroy(e);
+  for (auto& r : c->pend) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  for (cudaEvent_t e : c->evpool) cudaEventDestroy(e);
   if (c->s_side) cudaStreamDestroy(c->s_side);
   delete c;
 }
@@ -154,6 +177,67 @@ ft_status check_device_error(ft_ctx* c) {
   const uint32_t e = ((volatile Mailbox*)c->mbox_host)->pad_error;
   if (e) c->latched = e == DERR_TIMEOUT ? FT_ETIMEOUT : FT_ESTATE;
   return c->latched;
+}
+
+
+enum ProfName {
+  P_ROUTER, P_TOPK, P_PERMUTE, P_LOOKUP, P_GU_HIT, P_DN_HIT, P_GU_STAGED, P_DN_STAGED, P_GU_STREAM, P_DN_STREAM,
+  P_COMBINE, P_STAGE_COPY, P_PREFILL_WORK, P_GATHER, P_GEMM_GU, P_GEMM_DN, P_COUNT
+};
+const char* const kProfNames[P_COUNT] = {
+    "router_scores", "topk_softmax", "permute", "lookup", "gemv_gateup_hit", "gemv_down_hit",
+    "gemv_gateup_staged", "gemv_down_staged", "gemv_gateup_streamed", "gemv_down_streamed", "combine",
+    "h2d_stage_copies", "prefill_work", "prefill_gather", "gemm_tc_gateup", "gemm_tc_down"};
+
+cudaEvent_t pooled_event(ft_ctx* c) {
+  if (!c->evpool.empty()) {
+    cudaEvent_t e = c->evpool.back();
+    c->evpool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Bracket one launch (or a group of copies) on its stream when profiling.
+// Returns the record index, or -1.
+int prof_begin(ft_ctx* c, int name, cudaStream_t s, double bytes = 0, double flops = 0) {
+  if (!c->profiling) return -1;
+  ft_ctx::ProfRec r{name, pooled_event(c), pooled_event(c), bytes, flops};
+  cudaEventRecord(r.a, s);
+  c->pend.push_back(r);
+  return (int)c->pend.size() - 1;
+}
+
+void prof_end(ft_ctx* c, int idx, cudaStream_t s) {
+  if (idx >= 0) cudaEventRecord(c->pend[idx].b, s);
+}
+
+void prof_bytes(ft_ctx* c, int idx, double bytes, double flops) {
+  if (idx >= 0) {
+    c->pend[idx].bytes = bytes;
+    c->pend[idx].flops = flops;
+  }
+}
+
+// Weight bytes per element of the expert format (codes plus block scales for NVFP4).
+double weight_bytes_per_elem(int wtype) {
+  return wtype == FT_W_F32 ? 4.0 : (wtype == FT_W_BF16 ? 2.0 : 0.5 + 1.0 / 16.0);
+}
+
+// Algorithmic bytes / flops of one grouped-GEMV phase over n_items experts
+// carrying n_tok tokens: each weight once, activations in, outputs out.
+void gemv_cost(const Shape& sh, int phase, int n_items, int n_tok, double& bytes, double& flops) {
+  const double wb = weight_bytes_per_elem(sh.wtype), ab = sh.wtype == FT_W_F32 ? 4.0 : 2.0;
+  const double dd = (double)sh.d * sh.d_ff;
+  if (phase == 0) {
+    bytes = n_items * 2.0 * dd * wb + n_tok * (double)sh.d * ab + n_tok * (double)sh.d_ff * 4.0;
+    flops = 2.0 * n_tok * 2.0 * dd;
+  } else {
+    bytes = n_items * dd * wb + n_tok * (double)sh.d_ff * 4.0 + n_tok * (double)sh.d * 4.0;
+    flops = 2.0 * n_tok * dd;
+  }
 }
 
 }  // namespace
@@ -204,6 +288,7 @@ ft_status ft_moe_init(const ft_config* cfg, void* compute_stream, void* copy_str
   c->s_copy = (cudaStream_t)copy_stream;
   c->router.assign(sh.L, nullptr);
   c->tscale_host.assign((size_t)sh.L * sh.E * 3, 1.0f);
+  c->agg.assign(P_COUNT, ft_ctx::Agg{});
   ft_status st = FT_OK;
 #define TRY(call)                    \
   do {                               \
@@ -257,7 +342,7 @@ ft_status ft_moe_init(const ft_config* cfg, void* compute_stream, void* copy_str
   if (c->use_tc) {
     TRY(cuda_try(cudaMalloc((void**)&d.xs, sizeof(__nv_bfloat16) * (Tk + 256) * sh.d)));
     TRY(cuda_try(cudaMalloc((void**)&d.hs, sizeof(__nv_bfloat16) * (Tk + 256) * sh.d_ff)));
-    TRY(cuda_try(prefill_tc_init(sh, (int)Tk)));
+    TRY(cuda_try(prefill_tc_init(sh, d, (int)Tk)));
   }
   d.pool_dev = nullptr;
   TRY(cuda_try(cudaMemcpy(d.tscale, c->tscale_host.data(), sizeof(float) * c->tscale_host.size(),
@@ -346,9 +431,21 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
   cudaStream_t cs = c->s_comp;
   c->last_T = T;
   c->layer_calls += 1;
-  launch_router_scores(sh, x, c->router[layer], bias, bias_per_token, T, d.scores, cs);
-  launch_topk_permute(sh, d.scores, T, d, ids_opt, w_opt, cs);
+  const double ab = sh.wtype == FT_W_F32 ? 4.0 : 2.0;
   const int Tk = T * sh.k;
+  int p = prof_begin(c, P_ROUTER, cs, T * (double)sh.d * ab + sh.E * (double)sh.d * ab + T * (double)sh.E * 4.0,
+                     2.0 * T * sh.E * (double)sh.d);
+  launch_router_scores(sh, x, c->router[layer], bias, bias_per_token, T, d.scores, cs);
+  prof_end(c, p, cs);
+  p = prof_begin(c, P_TOPK, cs, T * (double)sh.E * 4.0 + Tk * 8.0);
+  launch_topk(sh, d.scores, T, d, cs);
+  prof_end(c, p, cs);
+  p = prof_begin(c, P_PERMUTE, cs, Tk * 12.0 + sh.E * 8.0);
+  launch_permute(sh, T, d, cs);
+  prof_end(c, p, cs);
+  c->kernel_launches += 3;
+  if (ids_opt) CK(cudaMemcpyAsync(ids_opt, d.ids, sizeof(int32_t) * Tk, cudaMemcpyDeviceToDevice, cs));
+  if (w_opt) CK(cudaMemcpyAsync(w_opt, d.wts, sizeof(float) * Tk, cudaMemcpyDeviceToDevice, cs));
   const int max_items = Tk < sh.E ? Tk : sh.E;
   const bool full_prefill = mode == FT_PREFILL && sh.C >= 2ll * sh.E;
   ft_status st = FT_OK;
@@ -362,25 +459,60 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
     a.bp_mbps = c->bp;
     a.bh_mbps = c->bh;
     d.pool_dev = c->pool_dev[layer];
+    p = prof_begin(c, P_LOOKUP, cs, sh.C * 8.0 + sh.E * 16.0);
     launch_lookup(sh, a, d, cs);
+    prof_end(c, p, cs);
     CK(cudaEventRecord(c->ev_look, cs));
     CK(cudaStreamWaitEvent(c->s_side, c->ev_look, 0));
-    launch_expert_gemv(sh, KIND_STREAMED, layer, x, T, d, max_items, Tk, c->s_side);
+    int pr[6];  // gate/up and down of the streamed, hit, staged classes
+    pr[0] = prof_begin(c, P_GU_STREAM, c->s_side);
+    launch_expert_gemv(sh, KIND_STREAMED, 0, layer, x, T, d, max_items, Tk, c->s_side);
+    prof_end(c, pr[0], c->s_side);
+    pr[1] = prof_begin(c, P_DN_STREAM, c->s_side);
+    launch_expert_gemv(sh, KIND_STREAMED, 1, layer, x, T, d, max_items, Tk, c->s_side);
+    prof_end(c, pr[1], c->s_side);
     CK(cudaEventRecord(c->ev_side, c->s_side));
-    launch_expert_gemv(sh, KIND_HIT, layer, x, T, d, max_items, Tk, cs);
+    pr[2] = prof_begin(c, P_GU_HIT, cs);
+    launch_expert_gemv(sh, KIND_HIT, 0, layer, x, T, d, max_items, Tk, cs);
+    prof_end(c, pr[2], cs);
+    pr[3] = prof_begin(c, P_DN_HIT, cs);
+    launch_expert_gemv(sh, KIND_HIT, 1, layer, x, T, d, max_items, Tk, cs);
+    prof_end(c, pr[3], cs);
+    c->kernel_launches += 5;
     st = wait_event(c->ev_look, WAIT_S);
     if (st != FT_OK) return c->latched = st;
     if (check_device_error(c) != FT_OK) return c->latched;
-    const int n_copy = c->mbox_host->n_copy;
-    c->last_m = c->mbox_host->m;
-    c->last_qstar = c->mbox_host->qstar;
-    c->last_qstage = c->mbox_host->qstage;
+    const Mailbox* mb = c->mbox_host;
+    const int n_copy = mb->n_copy;
+    c->last_m = mb->m;
+    c->last_qstar = mb->qstar;
+    c->last_qstage = mb->qstage;
+    if (c->profiling) {
+      double b, f;
+      gemv_cost(sh, 0, mb->n_streamed_cls, mb->n_tok_cls[KIND_STREAMED], b, f);
+      prof_bytes(c, pr[0], b, f);
+      gemv_cost(sh, 1, mb->n_streamed_cls, mb->n_tok_cls[KIND_STREAMED], b, f);
+      prof_bytes(c, pr[1], b, f);
+      gemv_cost(sh, 0, mb->n_hit_cls, mb->n_tok_cls[KIND_HIT], b, f);
+      prof_bytes(c, pr[2], b, f);
+      gemv_cost(sh, 1, mb->n_hit_cls, mb->n_tok_cls[KIND_HIT], b, f);
+      prof_bytes(c, pr[3], b, f);
+    }
     if (n_copy > 0) {
+      p = prof_begin(c, P_STAGE_COPY, c->s_copy, n_copy * (double)sh.slot_bytes);
       st = issue_copies(c, 0, n_copy);
+      prof_end(c, p, c->s_copy);
       if (st != FT_OK) return c->latched = st;
       CK(cudaEventRecord(c->ev_copy, c->s_copy));
       CK(cudaStreamWaitEvent(cs, c->ev_copy, 0));
-      launch_expert_gemv(sh, KIND_STAGED, layer, x, T, d, max_items, Tk, cs);
+      double b = 0, f = 0;
+      for (int ph = 0; ph < 2; ++ph) {
+        gemv_cost(sh, ph, mb->n_staged_cls, mb->n_tok_cls[KIND_STAGED], b, f);
+        pr[4 + ph] = prof_begin(c, ph == 0 ? P_GU_STAGED : P_DN_STAGED, cs, b, f);
+        launch_expert_gemv(sh, KIND_STAGED, ph, layer, x, T, d, max_items, Tk, cs);
+        prof_end(c, pr[4 + ph], cs);
+      }
+      c->kernel_launches += 2;
     }
     CK(cudaStreamWaitEvent(cs, c->ev_side, 0));
     c->prefetched = -1;
@@ -392,6 +524,7 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
       a.layer = layer;
       a.is_current = 1;
       launch_lookup(sh, a, d, cs);
+      c->kernel_launches += 1;
     }
     if (load_next) {
       LookupArgs a{};
@@ -399,6 +532,7 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
       a.pin_prev = 1;
       a.append = load_cur ? 1 : 0;
       launch_lookup(sh, a, d, cs);
+      c->kernel_launches += 1;
     }
     if (load_cur || load_next) {
       CK(cudaEventRecord(c->ev_look, cs));
@@ -412,7 +546,9 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
         c->last_m = mb->m;
         c->last_qstar = -1;
         c->last_qstage = mb->qstage;
+        p = prof_begin(c, P_STAGE_COPY, c->s_copy, split * (double)sh.slot_bytes);
         st = issue_copies(c, 0, split);
+        prof_end(c, p, c->s_copy);
         if (st != FT_OK) return c->latched = st;
         CK(cudaEventRecord(c->ev_pf[layer & 1], c->s_copy));
       } else {
@@ -420,22 +556,53 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
         c->last_qstar = -1;
       }
       if (load_next) {
+        p = prof_begin(c, P_STAGE_COPY, c->s_copy, (mb->n_copy - split) * (double)sh.slot_bytes);
         st = issue_copies(c, split, mb->n_copy);
+        prof_end(c, p, c->s_copy);
         if (st != FT_OK) return c->latched = st;
         CK(cudaEventRecord(c->ev_pf[(layer + 1) & 1], c->s_copy));
       }
     }
     c->prefetched = load_next ? layer + 1 : -1;
+    p = prof_begin(c, P_PREFILL_WORK, cs);
     launch_prefill_work(sh, layer, d, cs);
+    prof_end(c, p, cs);
+    c->kernel_launches += 1;
     CK(cudaStreamWaitEvent(cs, c->ev_pf[layer & 1], 0));
     if (c->use_tc) {
-      launch_prefill_tc(sh, layer, x, T, d, cs);
+      // algorithmic bytes with every routed expert read once; at prefill
+      // sizes nearly all E experts are routed, so min(E, T*k) is used
+      const double n_it = max_items, dd = (double)sh.d * sh.d_ff;
+      p = prof_begin(c, P_GATHER, cs, Tk * (double)sh.d * 2.0 + T * (double)sh.d * ab);
+      launch_prefill_gather(sh, x, T, d, cs);
+      prof_end(c, p, cs);
+      p = prof_begin(c, P_GEMM_GU, cs, n_it * 2.0 * dd * 2.0 + Tk * (double)sh.d * 2.0 + Tk * (double)sh.d_ff * 2.0,
+                     2.0 * Tk * 2.0 * dd);
+      launch_gemm_tc(sh, 0, T, d, cs);
+      prof_end(c, p, cs);
+      p = prof_begin(c, P_GEMM_DN, cs, n_it * dd * 2.0 + Tk * (double)sh.d_ff * 2.0 + Tk * (double)sh.d * 4.0,
+                     2.0 * Tk * dd);
+      launch_gemm_tc(sh, 1, T, d, cs);
+      prof_end(c, p, cs);
+      c->kernel_launches += 3;
     } else {
       d.pool_dev = c->pool_dev[layer];
-      launch_expert_gemv(sh, KIND_HIT, layer, x, T, d, max_items, Tk, cs);
+      int n_items = 0;
+      for (int ph = 0; ph < 2; ++ph) {
+        double b = 0, f = 0;
+        gemv_cost(sh, ph, sh.E, Tk, b, f);  // upper bound: every expert routed
+        (void)n_items;
+        p = prof_begin(c, ph == 0 ? P_GU_HIT : P_DN_HIT, cs, b, f);
+        launch_expert_gemv(sh, KIND_HIT, ph, layer, x, T, d, max_items, Tk, cs);
+        prof_end(c, p, cs);
+      }
+      c->kernel_launches += 2;
     }
   }
+  p = prof_begin(c, P_COMBINE, cs, Tk * (double)sh.d * 4.0 + T * (double)sh.d * ab + Tk * 8.0);
   launch_combine(sh, T, d, y, cs);
+  prof_end(c, p, cs);
+  c->kernel_launches += 1;
   CK(cudaGetLastError());
   return FT_OK;
 }
@@ -461,6 +628,7 @@ ft_status ft_cache_stats(ft_ctx* c, ft_stats* out) {
   out->last_qstar = c->last_qstar;
   out->last_qstage = c->last_qstage;
   out->device_error = err ? (err == DERR_TIMEOUT ? FT_ETIMEOUT : FT_ESTATE) : (int32_t)c->latched;
+  out->kernel_launches = c->kernel_launches;
   return FT_OK;
 }
 
@@ -530,6 +698,48 @@ ft_status ft_moe_probe_link(ft_ctx* c, uint64_t bytes, double* h2d_gbs, double* 
   if (e == cudaSuccess && zc_gbs) *zc_gbs = bytes / (ms * 1e6);
   cudaFree(tmp);
   CK(e);
+  return FT_OK;
+}
+
+ft_status ft_moe_profile(ft_ctx* c, int32_t enable) {
+  if (!c) return FT_EINVAL;
+  c->profiling = enable != 0;
+  return FT_OK;
+}
+
+ft_status ft_moe_profile_read(ft_ctx* c, ft_kernel_time* out, int32_t cap, int32_t* n_out, int32_t reset) {
+  if (!c || !n_out || cap < 0 || (cap > 0 && !out)) return FT_EINVAL;
+  CK(cudaStreamSynchronize(c->s_copy));
+  CK(cudaStreamSynchronize(c->s_side));
+  CK(cudaStreamSynchronize(c->s_comp));
+  for (auto& r : c->pend) {
+    float ms = 0.f;
+    CK(cudaEventElapsedTime(&ms, r.a, r.b));
+    ft_ctx::Agg& g = c->agg[r.name];
+    g.n += 1;
+    g.ms += ms;
+    g.bytes += r.bytes;
+    g.flops += r.flops;
+    c->evpool.push_back(r.a);
+    c->evpool.push_back(r.b);
+  }
+  c->pend.clear();
+  int n = 0;
+  for (int i = 0; i < P_COUNT; ++i) {
+    const ft_ctx::Agg& g = c->agg[i];
+    if (g.n == 0) continue;
+    if (n < cap) {
+      memset(out[n].name, 0, sizeof(out[n].name));
+      strncpy(out[n].name, kProfNames[i], sizeof(out[n].name) - 1);
+      out[n].launches = g.n;
+      out[n].ms = g.ms;
+      out[n].bytes = g.bytes;
+      out[n].flops = g.flops;
+    }
+    ++n;
+  }
+  *n_out = n;
+  if (reset) c->agg.assign(P_COUNT, ft_ctx::Agg{});
   return FT_OK;
 }
 

@@ -116,6 +116,7 @@ struct DevState {
   float* tscale;             // [L*E*3] NVFP4 tensor scales
   uint8_t* slots;            // HBM slot pool [C * slot_bytes]
   const uint8_t* pool_dev;   // device address of the called layer's blobs in the mapped host pool
+  void* tc_plan;             // host: tensor maps of the prefill GEMM (owned, see prefill_tc_free)
 };
 
 // ---- launchers (all enqueue on `st`) ----

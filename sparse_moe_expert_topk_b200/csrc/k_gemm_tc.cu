@@ -1,9 +1,446 @@
-// Prefill grouped GEMM on the tensor cores (placeholder until the tcgen05
-// kernel lands: reports unsupported, so prefill uses the grouped GEMV).
+// Prefill grouped GEMM on the 5th-generation tensor cores (tcgen05 + TMEM,
+// operands staged by TMA), with SwiGLU fused into the gate/up epilogue.
+//
+// Prefill pushes thousands of tokens through a layer, so nearly every expert
+// is active ([paperlens] "壁1: プレフィルではスパース性が消える", paper §2.1) and
+// the whole layer is resident in HBM slots before it computes ([paperlens]
+// "プレフィル: 全層ダブルバッファと「意味の錨」", paper §3.1). Per expert the work
+// is a GEMM with a ragged number of tokens (about 96 at T=4096, top-6 of 256).
+//
+// Formulation (swap-AB): the weight rows are the MMA's M = 128 side and the
+// expert's tokens the N side (N = tokens rounded up to 16, <= 256), so no
+// weight tile is padded:
+//   phase 0: D_g[f, p] = W_gate[f, :] . X_s[p, :],  D_u[f, p] = W_up[f, :] . X_s[p, :]
+//            H_s[p, f] = bf16(silu(D_g) * D_u)          (two accumulators in TMEM)
+//   phase 1: Y[p, r]   = W_down[r, :] . H_s[p, :]        (fp32 into the expert output buffer)
+// X_s / H_s hold the activations in expert-sorted order (row p = sorted
+// position), so an expert's tokens are consecutive rows.
+//
+// One persistent CTA per SM: warp 0 issues TMA loads (one elected lane) into a
+// 3-stage ring of 128B-swizzled K-major tiles, warp 1 allocates TMEM and
+// issues tcgen05.mma (one elected lane), warps 2..5 drain the accumulators
+// with tcgen05.ld and run the epilogue. All waits are bounded: a wait that
+// runs out latches a device error and the CTA drains and returns.
+// No TMA load uses cluster multicast.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <new>
+
 #include "ft_internal.cuh"
 
 namespace ft {
-bool prefill_tc_supported(const Shape&) { return false; }
-cudaError_t prefill_tc_init(const Shape&, int) { return cudaSuccess; }
-void launch_prefill_tc(const Shape&, int, const void*, int, DevState&, cudaStream_t) {}
+
+struct TcPlan {
+  CUtensorMap a_gu;  // slot pool as rows of d bf16 (gate/up rows)
+  CUtensorMap a_dn;  // slot pool as rows of d_ff bf16 (down rows)
+  CUtensorMap b_x;   // X_s [rows, d]
+  CUtensorMap b_h;   // H_s [rows, d_ff]
+  int sms;
+};
+
+namespace {
+
+constexpr int BM = 128;       // weight rows per tile (MMA M)
+constexpr int BK = 64;        // K per stage: 64 bf16 = one 128-byte swizzle row
+constexpr int MAX_N = 256;    // tokens per MMA (N)
+constexpr int BOX_ROWS = 32;  // rows per TMA box of the token operand
+constexpr int STAGES = 3;
+constexpr int A_BYTES = BM * BK * 2;       // 16 KB
+constexpr int B_BYTES = MAX_N * BK * 2;    // 32 KB
+constexpr int STAGE_BYTES = 2 * A_BYTES + B_BYTES;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr int THREADS = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr long long WAIT_CYCLES = 4000000000ll;  // ~2 s at 2 GHz
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait on an mbarrier phase. Returns false (and raises the CTA's
+// abort flag and the device error) if it does not complete in time or the
+// CTA already aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, uint32_t* err) {
+  const long long t0 = clock64();
+  for (uint32_t i = 0;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255) == 255) {
+      if (*abort) return false;
+      if (clock64() - t0 > WAIT_CYCLES) {
+        *abort = 1;
+        atomicExch(err, (uint32_t)DERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on `bar` once every previously issued tcgen05.mma of this thread completed.
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
+      "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, rows of 128 bytes,
+// 8-row atoms 1024 bytes apart (SBO), LBO unused (1), descriptor version 1.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Instruction descriptor of kind::f16: bf16 A and B (K-major), fp32 D, M x N.
+__device__ __forceinline__ uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+struct TcArgs {
+  const WorkLists* work;
+  int phase;
+  int d, d_ff;
+  int m_tiles;   // weight-row tiles of 128
+  int k_blocks;  // K / 64
+  __nv_bfloat16* hs;  // phase 0 output [rows, d_ff]
+  float* ybuf;        // phase 1 output [rows, d]
+  uint32_t* error;
+};
+
+struct Unit {
+  int slot, p0, nrows, mt;
+};
+
+// Units: (item, token tile of <= 256, weight-row tile); item-major so that the
+// CTAs working at one time share an expert's activations in L2.
+__device__ __forceinline__ bool unit_at(const TcArgs& a, const WorkItem* items, const int* pref, int n_items, int u,
+                                        Unit& out) {
+  const int q = u / a.m_tiles;
+  if (q >= pref[n_items]) return false;
+  int lo = 0, hi = n_items - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (pref[mid] <= q) lo = mid; else hi = mid - 1;
+  }
+  const WorkItem it = items[lo];
+  const int j = q - pref[lo];
+  out.slot = it.slot;
+  out.p0 = it.tok_off + j * MAX_N;
+  out.nrows = min(MAX_N, it.n_tok - j * MAX_N);
+  out.mt = u - q * a.m_tiles;
+  return true;
+}
+
+__global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a,
+                                                             const __grid_constant__ CUtensorMap tm_b, TcArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ WorkItem s_items[MAX_E];
+  __shared__ int s_pref[MAX_E + 1];
+  __shared__ int s_abort;
+  __shared__ uint32_t s_tmem;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  // bars: full[STAGES], empty[STAGES], acc_full, acc_empty, drain
+  const uint32_t bar_full = smem_u32(bars), bar_empty = bar_full + 8 * STAGES;
+  const uint32_t bar_acc_full = bar_full + 16 * STAGES, bar_acc_empty = bar_acc_full + 8;
+  const uint32_t bar_drain = bar_acc_empty + 8;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort = &s_abort;
+
+  const int n_items = a.work->n_items[KIND_HIT];
+  for (int i = threadIdx.x; i < n_items; i += THREADS) s_items[i] = a.work->items[KIND_HIT][i];
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    mbar_init(bar_acc_full, 1);
+    mbar_init(bar_acc_empty, 4);
+    mbar_init(bar_drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&s_tmem), 512);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int p = 0;
+    for (int i = 0; i < n_items; ++i) {
+      s_pref[i] = p;
+      p += (s_items[i].n_tok + MAX_N - 1) / MAX_N;
+    }
+    s_pref[n_items] = p;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  const int n_units = n_items > 0 ? s_pref[n_items] * a.m_tiles : 0;
+  const int two_a = a.phase == 0;
+
+  int last_round[STAGES];  // producer: last ring round issued per stage (-1 none)
+#pragma unroll
+  for (int s = 0; s < STAGES; ++s) last_round[s] = -1;
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    int it = 0;
+    for (int u = blockIdx.x; u < n_units && !*abort; u += gridDim.x) {
+      Unit un;
+      if (!unit_at(a, s_items, s_pref, n_items, u, un)) break;
+      const int nb = (un.nrows + BOX_ROWS - 1) / BOX_ROWS;
+      const uint32_t bytes = (two_a ? 2 : 1) * A_BYTES + nb * BOX_ROWS * BK * 2;
+      int row_a0, row_a1;
+      if (two_a) {
+        row_a0 = un.slot * 3 * a.d_ff + un.mt * BM;          // gate rows
+        row_a1 = un.slot * 3 * a.d_ff + a.d_ff + un.mt * BM;  // up rows
+      } else {
+        row_a0 = un.slot * 3 * a.d + 2 * a.d + un.mt * BM;    // down rows
+        row_a1 = 0;
+      }
+      for (int kb = 0; kb < a.k_blocks; ++kb, ++it) {
+        const int s = it % STAGES, r = it / STAGES;
+        if (!mbar_wait(bar_empty + 8 * s, (r & 1) ^ 1, abort, a.error)) break;
+        last_round[s] = r;
+        if (lane == 0) {
+          const uint32_t base = smem_u32(smem + s * STAGE_BYTES);
+          mbar_expect_tx(bar_full + 8 * s, bytes);
+          tma_load_2d(base, &tm_a, bar_full + 8 * s, kb * BK, row_a0);
+          if (two_a) tma_load_2d(base + A_BYTES, &tm_a, bar_full + 8 * s, kb * BK, row_a1);
+          for (int b = 0; b < nb; ++b)
+            tma_load_2d(base + 2 * A_BYTES + b * BOX_ROWS * 128, &tm_b, bar_full + 8 * s, kb * BK,
+                        un.p0 + b * BOX_ROWS);
+        }
+        __syncwarp();
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    int it = 0, ui = 0;
+    for (int u = blockIdx.x; u < n_units && !*abort; u += gridDim.x, ++ui) {
+      Unit un;
+      if (!unit_at(a, s_items, s_pref, n_items, u, un)) break;
+      const int n_mma = (un.nrows + 15) & ~15;
+      const uint32_t idesc = idesc_bf16(BM, n_mma);
+      if (!mbar_wait(bar_acc_empty, (ui & 1) ^ 1, abort, a.error)) break;
+      tc_fence_after();
+      bool ok = true;
+      for (int kb = 0; kb < a.k_blocks; ++kb, ++it) {
+        const int s = it % STAGES, r = it / STAGES;
+        if (!mbar_wait(bar_full + 8 * s, r & 1, abort, a.error)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t base = smem_u32(smem + s * STAGE_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t bd = sw128_desc(base + 2 * A_BYTES + kk * 32);
+            umma_bf16(tmem, sw128_desc(base + kk * 32), bd, idesc, (kb | kk) != 0);
+            if (two_a) umma_bf16(tmem + 256, sw128_desc(base + A_BYTES + kk * 32), bd, idesc, (kb | kk) != 0);
+          }
+          umma_commit(bar_empty + 8 * s);  // stage free once these MMAs have read it
+          if (kb == a.k_blocks - 1) umma_commit(bar_acc_full);
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    int ui = 0;
+    for (int u = blockIdx.x; u < n_units && !*abort; u += gridDim.x, ++ui) {
+      Unit un;
+      if (!unit_at(a, s_items, s_pref, n_items, u, un)) break;
+      if (!mbar_wait(bar_acc_full, ui & 1, abort, a.error)) break;
+      tc_fence_after();
+      const int row = un.mt * BM + 32 * q + lane;  // weight row = output feature
+      for (int c0 = 0; c0 < un.nrows; c0 += 32) {
+        uint32_t g[32];
+        tmem_ld32(tmem + lane_base + c0, g);
+        if (two_a) {
+          uint32_t uu[32];
+          tmem_ld32(tmem + lane_base + 256 + c0, uu);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (c0 + i < un.nrows) {
+              const float gv = __uint_as_float(g[i]), uv = __uint_as_float(uu[i]);
+              const float hv = gv / (1.f + expf(-gv)) * uv;
+              a.hs[(size_t)(un.p0 + c0 + i) * a.d_ff + row] = __float2bfloat16_rn(hv);
+            }
+          }
+        } else {
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (c0 + i < un.nrows) a.ybuf[(size_t)(un.p0 + c0 + i) * a.d + row] = __uint_as_float(g[i]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_acc_empty);
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // producer tail: every stage's last round must be released by the MMAs
+    // (normal exit) or at least have landed (abort) before smem goes away
+    for (int s = 0; s < STAGES; ++s) {
+      if (last_round[s] < 0) continue;
+      const uint32_t bar = *abort ? bar_full + 8 * s : bar_empty + 8 * s;
+      const long long t0 = clock64();
+      while (!mbar_try_wait(bar, last_round[s] & 1) && clock64() - t0 < WAIT_CYCLES / 4) {
+      }
+    }
+  } else if (warp == 1 && *abort) {
+    // let every issued MMA finish before the accumulators are freed
+    if (lane == 0) umma_commit(bar_drain);
+    __syncwarp();
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar_drain, 0) && clock64() - t0 < WAIT_CYCLES / 4) {
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// X_s[p, :] = x[perm[p] / k, :] (bf16 rows, 16-byte vectors); grid (rows), 256 threads.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* __restrict__ x,
+                                                          const int32_t* __restrict__ perm, int k, int d,
+                                                          __nv_bfloat16* __restrict__ xs) {
+  const int p = blockIdx.x;
+  const int t = perm[p] / k;
+  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+  uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)p * d);
+  for (int i = threadIdx.x; i < d / 8; i += 256) dst[i] = __ldg(src + i);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+bool encode_2d(CUtensorMap* m, void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool prefill_tc_supported(const Shape& sh) {
+  return sh.wtype == FT_W_BF16 && sh.d % BM == 0 && sh.d_ff % BM == 0 && sh.C > 0;
+}
+
+cudaError_t prefill_tc_init(const Shape& sh, DevState& ds, int max_rows) {
+  if (!g_encode) {
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", (void**)&g_encode, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !g_encode) return cudaErrorNotSupported;
+  }
+  TcPlan* p = new (std::nothrow) TcPlan();
+  if (!p) return cudaErrorMemoryAllocation;
+  ds.tc_plan = p;  // owned by the context (prefill_tc_free)
+  const uint64_t C = (uint64_t)sh.C;
+  if (!encode_2d(&p->a_gu, ds.slots, C * 3 * sh.d_ff, sh.d, BM)) return cudaErrorInvalidValue;
+  if (!encode_2d(&p->a_dn, ds.slots, C * 3 * sh.d, sh.d_ff, BM)) return cudaErrorInvalidValue;
+  if (!encode_2d(&p->b_x, ds.xs, (uint64_t)max_rows + 256, sh.d, BOX_ROWS)) return cudaErrorInvalidValue;
+  if (!encode_2d(&p->b_h, ds.hs, (uint64_t)max_rows + 256, sh.d_ff, BOX_ROWS)) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return cudaDeviceGetAttribute(&p->sms, cudaDevAttrMultiProcessorCount, dev);
+}
+
+void prefill_tc_free(DevState& ds) {
+  delete static_cast<TcPlan*>(ds.tc_plan);
+  ds.tc_plan = nullptr;
+}
+
+void launch_prefill_gather(const Shape& sh, const void* x, int T, DevState& ds, cudaStream_t st) {
+  gather_rows_kernel<<<T * sh.k, 256, 0, st>>>((const __nv_bfloat16*)x, ds.perm, sh.k, sh.d, ds.xs);
+}
+
+void launch_gemm_tc(const Shape& sh, int phase, int T, DevState& ds, cudaStream_t st) {
+  (void)T;
+  const TcPlan& p = *static_cast<const TcPlan*>(ds.tc_plan);
+  TcArgs a;
+  a.work = ds.work;
+  a.phase = phase;
+  a.d = sh.d;
+  a.d_ff = sh.d_ff;
+  a.m_tiles = (phase == 0 ? sh.d_ff : sh.d) / BM;
+  a.k_blocks = (phase == 0 ? sh.d : sh.d_ff) / BK;
+  a.hs = ds.hs;
+  a.ybuf = ds.ybuf;
+  a.error = ds.error;
+  gemm_tc_kernel<<<p.sms, THREADS, SMEM_BYTES, st>>>(phase == 0 ? p.a_gu : p.a_dn, phase == 0 ? p.b_x : p.b_h, a);
+}
+
 }  // namespace ft
