@@ -385,10 +385,21 @@ def main():
     total_tokens = sum_over_ranks(tokens_per_step * args.steps, world, device)
     value = total_tokens / (ms_max / 1e3)
 
-    # per-kernel profile of one more step (events around every launch)
+    # per-kernel profile of one more step (events around every launch),
+    # split by batch size
+    ft.ft_moe_reset_cache(h.ctx)
     ft.ft_moe_profile(h.ctx, True)
-    run_step(h, xs, bias, ys)
-    prof = ft.ft_moe_profile_read(h.ctx)
+    prof, by_batch = {}, {}
+    for T, seq in xs.items():
+        for x in seq:
+            ft.ft_moe_layer_forward(h.ctx, 0, ft.FT_DECODE, x, T, bias, 0, ys[T])
+        pT = ft.ft_moe_profile_read(h.ctx)
+        by_batch[T] = {k: {"ms": round(v["ms"], 3), "GBps": round(v["bytes"] / max(v["ms"], 1e-9) / 1e6, 1),
+                           "launches": v["launches"]} for k, v in pT.items()}
+        for k, v in pT.items():
+            a = prof.setdefault(k, {"launches": 0, "ms": 0.0, "bytes": 0.0, "flops": 0.0})
+            for f in a:
+                a[f] += v[f]
     ft.ft_moe_profile(h.ctx, False)
     st1 = ft.ft_cache_stats(h.ctx)
     miss_rate = st1["misses"] / max(st1["lookups"], 1)
@@ -438,7 +449,7 @@ def main():
             "miss_rate": round(miss_rate, 4),
             "cache": {k: st1[k] for k in ("lookups", "hits", "misses", "staged", "streamed")},
             "host_link": {"h2d_copy_gbs": round(h2d_gbs, 2), "zero_copy_read_gbs": round(zc_gbs, 2)},
-            "roofline": roof, "kernels": rows, "gpu_launches": int(round(launches * args.steps)),
+            "roofline": roof, "kernels": rows, "kernels_by_batch": by_batch, "gpu_launches": int(round(launches * args.steps)),
             "gpu_launches_per_step": round(launches, 1), "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,
             "peaks": {"kind": peak_kind, "hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"]},
         }

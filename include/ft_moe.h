@@ -92,7 +92,7 @@ typedef struct {
   int32_t d_model;     /* d, multiple of 64, <= 16384 */
   int32_t d_ff;        /* d_ff, multiple of 64, <= 16384 */
   int32_t wtype;       /* ft_wtype */
-  int64_t cache_slots; /* C, 0..L*E HBM slots of ft_moe_slot_bytes() each */
+  int64_t cache_slots; /* C, 0..max(L*E, 2E) HBM slots of ft_moe_slot_bytes() each */
   int32_t max_tokens;  /* T upper bound of one forward, 1..65536 */
   int32_t device;      /* CUDA device ordinal */
 } ft_config;

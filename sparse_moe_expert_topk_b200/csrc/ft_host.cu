@@ -96,8 +96,11 @@ ft_status validate(const ft_config* c) {
   if (c->d_model < 64 || c->d_model % 64 || c->d_model > 16384) return FT_EINVAL;
   if (c->d_ff < 64 || c->d_ff % 64 || c->d_ff > 16384) return FT_EINVAL;
   if (c->wtype < FT_W_F32 || c->wtype > FT_W_NVFP4) return FT_EINVAL;
-  const long long le = (long long)c->n_layers * c->n_experts;
-  if (c->cache_slots < 0 || c->cache_slots > le || c->cache_slots >= (1ll << 20)) return FT_EINVAL;
+  // up to every expert of every layer, or two layers' worth (the prefill
+  // double buffer) when that is more
+  const long long le = (long long)c->n_layers * c->n_experts, two = 2ll * c->n_experts;
+  if (c->cache_slots < 0 || c->cache_slots > (le > two ? le : two) || c->cache_slots >= (1ll << 20))
+    return FT_EINVAL;
   if (c->max_tokens < 1 || c->max_tokens > 65536) return FT_EINVAL;
   if (c->device < 0) return FT_EINVAL;
   return FT_OK;

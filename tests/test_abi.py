@@ -45,7 +45,7 @@ def test_slot_bytes(lib):
 
 @pytest.mark.parametrize("field,value", [("n_layers", 0), ("n_experts", 0), ("n_experts", 513), ("top_k", 0),
                                          ("top_k", 9), ("d_model", 100), ("d_ff", 32), ("wtype", 3),
-                                         ("cache_slots", -1), ("cache_slots", 9), ("max_tokens", 0),
+                                         ("cache_slots", -1), ("cache_slots", 17), ("max_tokens", 0),
                                          ("device", -1)])
 def test_config_validation(lib, field, value):
     cfg = ft.make_config(1, 8, 2, 64, 128, ft.FT_W_F32, 4, 16)
