@@ -30,6 +30,11 @@ bool prefill_tc_supported(const Shape& sh);
 cudaError_t prefill_tc_init(const Shape& sh, DevState& ds, int max_rows);
 void prefill_tc_free(DevState& ds);
 void launch_prefill_gather(const Shape& sh, const void* x, int T, DevState& ds, cudaStream_t st);
+bool gemv_mma_supported(const Shape& sh);
+cudaError_t gemv_mma_init(int device);
+void launch_to_f16(const void* x, int n, void* y, cudaStream_t st);
+void launch_gemv_mma(const Shape& sh, int cls, int phase, int layer, const void* x16, int T, DevState& ds,
+                     int max_items, int max_tok, cudaStream_t st);
 void launch_gemm_tc(const Shape& sh, int phase, int T, DevState& ds, cudaStream_t st);
 }  // namespace ft
 
@@ -54,6 +59,7 @@ struct ft_ctx {
   int last_m = 0, last_qstar = 0, last_qstage = 0;
   ft_status latched = FT_OK;
   bool use_tc = false;
+  bool use_mma = false;  // tensor-core decode GEMV (BF16 / NVFP4), else SIMT
   unsigned long long* probe_sink = nullptr;
   // launch accounting and optional per-launch CUDA-event profiling
   unsigned long long kernel_launches = 0;
@@ -136,7 +142,7 @@ void free_all(ft_ctx* c) {
   DevState& d = c->ds;
   void* dev_ptrs[] = {d.slot_of, d.key_of, d.stamp, d.clk, d.ctr, d.error, d.work, d.scores, d.ids, d.wts,
                       d.counts, d.offsets, d.perm, d.inv, d.hbuf, d.ybuf, d.xs, d.hs, d.tscale, d.slots,
-                      c->probe_sink};
+                      d.h16, d.x16, c->probe_sink};
   for (void* p : dev_ptrs)
     if (p) cudaFree(p);
   for (uint8_t* p : c->pool_host)
@@ -341,6 +347,13 @@ ft_status ft_moe_init(const ft_config* cfg, void* compute_stream, void* copy_str
   TRY(cuda_try(cudaMalloc((void**)&d.ybuf, sizeof(float) * Tk * sh.d)));
   TRY(cuda_try(cudaMalloc((void**)&d.tscale, sizeof(float) * sh.L * sh.E * 3)));
   TRY(cuda_try(cudaMalloc((void**)&c->probe_sink, sizeof(unsigned long long))));
+  c->use_mma = gemv_mma_supported(sh);
+  if (c->use_mma) {
+    TRY(cuda_try(cudaMalloc((void**)&d.h16, sizeof(uint16_t) * Tk * sh.d_ff)));
+    if (sh.wtype == FT_W_NVFP4)
+      TRY(cuda_try(cudaMalloc((void**)&d.x16, sizeof(uint16_t) * (size_t)cfg->max_tokens * sh.d)));
+    TRY(cuda_try(gemv_mma_init(cfg->device)));
+  }
   c->use_tc = prefill_tc_supported(sh) && sh.C >= 2ll * sh.E;
   if (c->use_tc) {
     TRY(cuda_try(cudaMalloc((void**)&d.xs, sizeof(__nv_bfloat16) * (Tk + 256) * sh.d)));
@@ -404,6 +417,16 @@ ft_status ft_moe_reset_cache(ft_ctx* c) {
   return reset_state(c);
 }
 
+// One phase of the decode grouped GEMV for one work class.
+static void gemv(ft_ctx* c, int cls, int phase, int layer, const void* x, int T, int max_items, int Tk,
+                 cudaStream_t st) {
+  if (c->use_mma)
+    launch_gemv_mma(c->sh, cls, phase, layer, c->sh.wtype == FT_W_NVFP4 ? (const void*)c->ds.x16 : x, T, c->ds,
+                    max_items, Tk, st);
+  else
+    launch_expert_gemv(c->sh, cls, phase, layer, x, T, c->ds, max_items, Tk, st);
+}
+
 static ft_status issue_copies(ft_ctx* c, int from, int to) {
   const Mailbox* mb = c->mbox_host;
   const Shape& sh = c->sh;
@@ -462,6 +485,10 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
     a.bp_mbps = c->bp;
     a.bh_mbps = c->bh;
     d.pool_dev = c->pool_dev[layer];
+    if (c->use_mma && sh.wtype == FT_W_NVFP4) {
+      launch_to_f16(x, T * sh.d, d.x16, cs);
+      c->kernel_launches += 1;
+    }
     p = prof_begin(c, P_LOOKUP, cs, sh.C * 8.0 + sh.E * 16.0);
     launch_lookup(sh, a, d, cs);
     prof_end(c, p, cs);
@@ -469,17 +496,17 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
     CK(cudaStreamWaitEvent(c->s_side, c->ev_look, 0));
     int pr[6];  // gate/up and down of the streamed, hit, staged classes
     pr[0] = prof_begin(c, P_GU_STREAM, c->s_side);
-    launch_expert_gemv(sh, KIND_STREAMED, 0, layer, x, T, d, max_items, Tk, c->s_side);
+    gemv(c, KIND_STREAMED, 0, layer, x, T, max_items, Tk, c->s_side);
     prof_end(c, pr[0], c->s_side);
     pr[1] = prof_begin(c, P_DN_STREAM, c->s_side);
-    launch_expert_gemv(sh, KIND_STREAMED, 1, layer, x, T, d, max_items, Tk, c->s_side);
+    gemv(c, KIND_STREAMED, 1, layer, x, T, max_items, Tk, c->s_side);
     prof_end(c, pr[1], c->s_side);
     CK(cudaEventRecord(c->ev_side, c->s_side));
     pr[2] = prof_begin(c, P_GU_HIT, cs);
-    launch_expert_gemv(sh, KIND_HIT, 0, layer, x, T, d, max_items, Tk, cs);
+    gemv(c, KIND_HIT, 0, layer, x, T, max_items, Tk, cs);
     prof_end(c, pr[2], cs);
     pr[3] = prof_begin(c, P_DN_HIT, cs);
-    launch_expert_gemv(sh, KIND_HIT, 1, layer, x, T, d, max_items, Tk, cs);
+    gemv(c, KIND_HIT, 1, layer, x, T, max_items, Tk, cs);
     prof_end(c, pr[3], cs);
     c->kernel_launches += 5;
     st = wait_event(c->ev_look, WAIT_S);
@@ -512,7 +539,7 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
       for (int ph = 0; ph < 2; ++ph) {
         gemv_cost(sh, ph, mb->n_staged_cls, mb->n_tok_cls[KIND_STAGED], b, f);
         pr[4 + ph] = prof_begin(c, ph == 0 ? P_GU_STAGED : P_DN_STAGED, cs, b, f);
-        launch_expert_gemv(sh, KIND_STAGED, ph, layer, x, T, d, max_items, Tk, cs);
+        gemv(c, KIND_STAGED, ph, layer, x, T, max_items, Tk, cs);
         prof_end(c, pr[4 + ph], cs);
       }
       c->kernel_launches += 2;
@@ -566,6 +593,16 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
         CK(cudaEventRecord(c->ev_pf[(layer + 1) & 1], c->s_copy));
       }
     }
+    if (!load_cur && !load_next) {
+      // no lookup this call: clear the record (the last lookup kernel has
+      // finished, the host waited for it)
+      Mailbox* mb = c->mbox_host;
+      mb->n_copy = mb->n_lookup = mb->n_lookup_cur = 0;
+      mb->m = mb->qstage = 0;
+      mb->qstar = -1;
+      c->last_m = c->last_qstage = 0;
+      c->last_qstar = -1;
+    }
     c->prefetched = load_next ? layer + 1 : -1;
     p = prof_begin(c, P_PREFILL_WORK, cs);
     launch_prefill_work(sh, layer, d, cs);
@@ -590,13 +627,17 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
       c->kernel_launches += 3;
     } else {
       d.pool_dev = c->pool_dev[layer];
+      if (c->use_mma && sh.wtype == FT_W_NVFP4) {
+        launch_to_f16(x, T * sh.d, d.x16, cs);
+        c->kernel_launches += 1;
+      }
       int n_items = 0;
       for (int ph = 0; ph < 2; ++ph) {
         double b = 0, f = 0;
         gemv_cost(sh, ph, sh.E, Tk, b, f);  // upper bound: every expert routed
         (void)n_items;
         p = prof_begin(c, ph == 0 ? P_GU_HIT : P_DN_HIT, cs, b, f);
-        launch_expert_gemv(sh, KIND_HIT, ph, layer, x, T, d, max_items, Tk, cs);
+        gemv(c, KIND_HIT, ph, layer, x, T, max_items, Tk, cs);
         prof_end(c, p, cs);
       }
       c->kernel_launches += 2;

@@ -1,0 +1,397 @@
+// Decode grouped GEMV for BF16 and NVFP4 experts on warp-level tensor-core
+// MMAs (mma.sync m16n8k16, fp32 accumulate), weights streamed straight from
+// HBM slots or from the mapped host pool with 128-bit loads.
+//
+// Small-batch decode is memory bound ([paperlens] "壁2: デコードのミスを「どう捌く
+// か」が決まっていない", paper §2.2): every weight byte is read once, so the
+// kernel's job is to keep enough loads in flight and spend few instructions
+// per byte. A warp owns 16 weight rows and one chunk of up to 16 tokens; each
+// lane loads 16 consecutive bytes of two rows (g and g+8, g = lane / 4) and
+// hands them to the MMA unchanged as its A fragment. That assigns the K
+// positions of the MMA in a lane-dependent order, which is harmless for a dot
+// product as long as the activations use the same order: each lane loads the
+// 16 matching bytes of its token's row as the B fragment. No shuffles, no
+// shared memory; the accumulation order is fixed by the code, so an expert's
+// result does not depend on where its weights were read from ([paperlens]
+// "設計: 2階建てのエキスパート記憶", paper §3.3).
+//
+// Gate/up phase: rows 0..7 of the MMA tile are gate rows f0..f0+7 and rows
+// 8..15 the matching up rows, so each lane holds gate and up of the same
+// (feature, token) pairs and applies SwiGLU in registers; h is written as a
+// 16-bit activation (bf16 for BF16 experts, f16 for NVFP4) for the down phase.
+// NVFP4: 32 e2m1 codes per lane are converted to f16 pairs (cvt e2m1x2) and
+// multiplied by their e4m3 block scale (exact in f16), the per-matrix fp32
+// tensor scale is applied to the fp32 result.
+#include <cuda_fp16.h>
+
+#include "ft_internal.cuh"
+
+namespace ft {
+
+namespace {
+
+constexpr int WARPS = 8;
+
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                        uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Four bytes of e2m1 pairs -> four f16x2 (byte i -> out[i]; the even element
+// of a pair sits in the low nibble and lands in the low half).
+__device__ __forceinline__ void e2m1x8_to_f16x8(uint32_t w, uint32_t (&o)[4]) {
+  asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %4;\n"
+      " cvt.rn.f16x2.e2m1x2 %0, b0;\n cvt.rn.f16x2.e2m1x2 %1, b1;\n"
+      " cvt.rn.f16x2.e2m1x2 %2, b2;\n cvt.rn.f16x2.e2m1x2 %3, b3;\n}"
+      : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3])
+      : "r"(w));
+}
+
+// Two e4m3 scale bytes (low byte = first block) -> f16x2 {s0, s1}.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t s) {
+  uint32_t r;
+  asm("{\n .reg .b16 t;\n cvt.u16.u32 t, %1;\n cvt.rn.f16x2.e4m3x2 %0, t;\n}" : "=r"(r) : "r"(s));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+struct MmaArgs {
+  const WorkLists* work;
+  int cls, layer, E, k, d, d_ff, nvfp4;
+  long long C;
+  size_t slot_bytes;
+  const uint8_t* slots;
+  const uint8_t* pool;
+  const void* x;        // [T, d] bf16 activations (BF16) or f16 copy (NVFP4)
+  const int32_t* perm;
+  const float* tscale;  // [L*E*3]
+  uint16_t* h16;        // [T*k, d_ff] bf16 (BF16) or f16 (NVFP4) SwiGLU output
+  float* ybuf;          // [T*k, d]
+};
+
+__device__ __forceinline__ const uint8_t* blob_of(const MmaArgs& a, const WorkItem& it) {
+  if (a.cls == KIND_STREAMED) return a.pool + (size_t)it.e * a.slot_bytes;
+  return a.slots + (size_t)it.slot * a.slot_bytes;
+}
+
+// acc[t][.] += W[rows g, g+8] . X[tokens] over K for one warp; t = n8 token tile.
+// BF16: per step each lane covers 8 K values of each row (4 lanes: 32 K).
+template <int NB, int U>
+__device__ __forceinline__ void dot_bf16(const uint8_t* ra, const uint8_t* rb, const uint16_t* const (&xr)[NB], int K,
+                                         int q, float (&acc)[NB][4]) {
+  const int steps = K / 32;
+  const uint8_t* pa = ra + q * 16;
+  const uint8_t* pb = rb + q * 16;
+  int s = 0;
+  for (; s + U <= steps; s += U) {
+    uint4 wa[U], wb[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      wa[u] = ld_stream(pa + (size_t)(s + u) * 64);
+      wb[u] = ld_stream(pb + (size_t)(s + u) * 64);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+#pragma unroll
+      for (int t = 0; t < NB; ++t) {
+        const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xr[t] + (s + u) * 32 + q * 8));
+        mma_bf16(acc[t], wa[u].x, wb[u].x, wa[u].y, wb[u].y, xv.x, xv.y);
+        mma_bf16(acc[t], wa[u].z, wb[u].z, wa[u].w, wb[u].w, xv.z, xv.w);
+      }
+    }
+  }
+  for (; s < steps; ++s) {
+    const uint4 wa = ld_stream(pa + (size_t)s * 64), wb = ld_stream(pb + (size_t)s * 64);
+#pragma unroll
+    for (int t = 0; t < NB; ++t) {
+      const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xr[t] + s * 32 + q * 8));
+      mma_bf16(acc[t], wa.x, wb.x, wa.y, wb.y, xv.x, xv.y);
+      mma_bf16(acc[t], wa.z, wb.z, wa.w, wb.w, xv.z, xv.w);
+    }
+  }
+}
+
+// NVFP4: per step each lane covers 32 K values (16 code bytes, two scale
+// blocks) of each row (4 lanes: 128 K); eight MMAs per step.
+__device__ __forceinline__ void decode_nvfp4(const uint4 w, uint32_t sc, uint32_t (&h)[16]) {
+  e2m1x8_to_f16x8(w.x, *reinterpret_cast<uint32_t(*)[4]>(&h[0]));
+  e2m1x8_to_f16x8(w.y, *reinterpret_cast<uint32_t(*)[4]>(&h[4]));
+  e2m1x8_to_f16x8(w.z, *reinterpret_cast<uint32_t(*)[4]>(&h[8]));
+  e2m1x8_to_f16x8(w.w, *reinterpret_cast<uint32_t(*)[4]>(&h[12]));
+  const uint32_t s2 = e4m3x2_to_f16x2(sc);
+  const __half2 hs = *reinterpret_cast<const __half2*>(&s2);
+  const __half2 lo = __low2half2(hs), hi = __high2half2(hs);
+  const uint32_t slo = *reinterpret_cast<const uint32_t*>(&lo), shi = *reinterpret_cast<const uint32_t*>(&hi);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) h[j] = hmul2(h[j], slo);
+#pragma unroll
+  for (int j = 8; j < 16; ++j) h[j] = hmul2(h[j], shi);
+}
+
+template <int NB, int U>
+__device__ __forceinline__ void dot_nvfp4(const uint8_t* ra, const uint8_t* rb, const uint8_t* sa, const uint8_t* sb,
+                                          const uint16_t* const (&xr)[NB], int K, int q, float (&acc)[NB][4]) {
+  const int steps = K / 128;
+  const uint8_t* pa = ra + q * 16;
+  const uint8_t* pb = rb + q * 16;
+  const unsigned short* qa = reinterpret_cast<const unsigned short*>(sa) + q;
+  const unsigned short* qb = reinterpret_cast<const unsigned short*>(sb) + q;
+  int s = 0;
+  for (; s < steps; s += U) {
+    const int n = steps - s < U ? steps - s : U;
+    uint4 wa[U], wb[U];
+    uint32_t ca[U], cb[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (u < n) {
+        wa[u] = ld_stream(pa + (size_t)(s + u) * 64);
+        wb[u] = ld_stream(pb + (size_t)(s + u) * 64);
+        ca[u] = __ldg(qa + (s + u) * 4);
+        cb[u] = __ldg(qb + (s + u) * 4);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (u < n) {
+        uint32_t ha[16], hb[16];
+        decode_nvfp4(wa[u], ca[u], ha);
+        decode_nvfp4(wb[u], cb[u], hb);
+#pragma unroll
+        for (int t = 0; t < NB; ++t) {
+          const uint4* xp = reinterpret_cast<const uint4*>(xr[t] + (s + u) * 128 + q * 32);
+          uint32_t xh[16];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const uint4 xv = __ldg(xp + v);
+            xh[4 * v] = xv.x;
+            xh[4 * v + 1] = xv.y;
+            xh[4 * v + 2] = xv.z;
+            xh[4 * v + 3] = xv.w;
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            mma_f16(acc[t], ha[2 * j], hb[2 * j], ha[2 * j + 1], hb[2 * j + 1], xh[2 * j], xh[2 * j + 1]);
+        }
+      }
+    }
+  }
+}
+
+// Map warp-unit u of this class to (item, 16-token chunk, row block).
+__device__ __forceinline__ bool unit_of(const int* pref, int n_items, int rblocks, int u, int& item, int& chunk,
+                                        int& rb) {
+  const int qi = u / rblocks;
+  rb = u - qi * rblocks;
+  if (qi >= pref[n_items]) return false;
+  int lo = 0, hi = n_items - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (pref[mid] <= qi) lo = mid; else hi = mid - 1;
+  }
+  item = lo;
+  chunk = qi - pref[lo];
+  return true;
+}
+
+constexpr int CHUNK = 16;  // tokens per warp-unit (two n8 tiles)
+
+template <int NB, int PHASE, bool FP4>
+__device__ void unit_work(const MmaArgs& a, const WorkItem& it, int chunk, int rb, int lane) {
+  const int g = lane >> 2, q = lane & 3;
+  const uint8_t* blob = blob_of(a, it);
+  const size_t n = (size_t)a.d * a.d_ff;
+  const int K = PHASE == 0 ? a.d : a.d_ff;
+  const size_t rbytes = a.nvfp4 ? (size_t)K / 2 : (size_t)K * 2;
+  const size_t sbytes = (size_t)K / 16;
+  int rowa, rowb;          // rows inside their matrices
+  size_t ma, mb, sa0, sb0;  // matrix byte offsets (codes, scales)
+  if (PHASE == 0) {
+    rowa = rowb = rb * 8 + g;
+    ma = 0;
+    mb = a.nvfp4 ? n / 2 : n * 2;
+    sa0 = 3 * (n / 2);
+    sb0 = 3 * (n / 2) + n / 16;
+  } else {
+    rowa = rb * 16 + g;
+    rowb = rowa + 8;
+    ma = mb = a.nvfp4 ? n : n * 4;
+    sa0 = sb0 = 3 * (n / 2) + 2 * (n / 16);
+  }
+  const uint8_t* ra = blob + ma + (size_t)rowa * rbytes;
+  const uint8_t* rbp = blob + mb + (size_t)rowb * rbytes;
+  const int base = it.tok_off + chunk * CHUNK;
+  const int nt = min(CHUNK, it.n_tok - chunk * CHUNK);
+  const uint16_t* xr[NB];
+#pragma unroll
+  for (int t = 0; t < NB; ++t) {
+    const int j = t * 8 + g;
+    const int pos = base + (j < nt ? j : 0);
+    if (PHASE == 0)
+      xr[t] = reinterpret_cast<const uint16_t*>(a.x) + (size_t)(a.perm[pos] / a.k) * a.d;
+    else
+      xr[t] = a.h16 + (size_t)pos * a.d_ff;
+  }
+  float acc[NB][4];
+#pragma unroll
+  for (int t = 0; t < NB; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+  if constexpr (FP4)
+    dot_nvfp4<NB, 4>(ra, rbp, blob + sa0 + (size_t)rowa * sbytes, blob + sb0 + (size_t)rowb * sbytes, xr, K, q, acc);
+  else
+    dot_bf16<NB, (NB == 1 ? 8 : 4)>(ra, rbp, xr, K, q, acc);
+  // d0,d1: row g, tokens 2q, 2q+1; d2,d3: row g+8, same tokens (per n8 tile)
+  float t0 = 1.f, t1 = 1.f;
+  if (a.nvfp4) {
+    const float* ts = a.tscale + ((size_t)a.layer * a.E + it.e) * 3;
+    t0 = PHASE == 0 ? ts[0] : ts[2];
+    t1 = PHASE == 0 ? ts[1] : ts[2];
+  }
+#pragma unroll
+  for (int t = 0; t < NB; ++t) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int j = t * 8 + 2 * q + c;
+      if (j >= nt) continue;
+      const float v0 = acc[t][c] * t0, v1 = acc[t][2 + c] * t1;
+      if (PHASE == 0) {
+        const float hv = v0 / (1.f + expf(-v0)) * v1;
+        const uint16_t hb = a.nvfp4 ? __half_as_ushort(__float2half_rn(hv)) : __bfloat16_as_ushort(__float2bfloat16_rn(hv));
+        a.h16[(size_t)(base + j) * a.d_ff + rb * 8 + g] = hb;
+      } else {
+        float* yr = a.ybuf + (size_t)(base + j) * a.d;
+        yr[rb * 16 + g] = v0;
+        yr[rb * 16 + g + 8] = v1;
+      }
+    }
+  }
+}
+
+template <int NB, bool FP4>
+__global__ void __launch_bounds__(WARPS * 32) gemv_mma_kernel(MmaArgs a, int phase) {
+  __shared__ int s_pref[MAX_E + 1];
+  __shared__ WorkItem s_items[MAX_E];
+  const int n_items = a.work->n_items[a.cls];
+  if (n_items == 0) return;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < n_items; i += blockDim.x) s_items[i] = a.work->items[a.cls][i];
+  __syncthreads();
+  if (tid == 0) {
+    int p = 0;
+    for (int i = 0; i < n_items; ++i) {
+      s_pref[i] = p;
+      p += (s_items[i].n_tok + CHUNK - 1) / CHUNK;
+    }
+    s_pref[n_items] = p;
+  }
+  __syncthreads();
+  const int rblocks = phase == 0 ? a.d_ff / 8 : a.d / 16;
+  const int n_units = s_pref[n_items] * rblocks;
+  for (int u = blockIdx.x * WARPS + warp; u < n_units; u += gridDim.x * WARPS) {
+    int item, chunk, rb;
+    if (!unit_of(s_pref, n_items, rblocks, u, item, chunk, rb)) break;
+    const WorkItem it = s_items[item];
+    if (a.cls != KIND_STREAMED && (it.slot < 0 || it.slot >= a.C)) continue;  // error already latched
+    if (phase == 0) unit_work<NB, 0, FP4>(a, it, chunk, rb, lane);
+    else unit_work<NB, 1, FP4>(a, it, chunk, rb, lane);
+  }
+}
+
+// bf16 -> f16 copy of the activations (NVFP4 experts take f16 MMA operands).
+__global__ void __launch_bounds__(256) to_f16_kernel(const __nv_bfloat16* __restrict__ x, int n, __half* __restrict__ y) {
+  for (int i = blockIdx.x * 256 + threadIdx.x; i < n; i += gridDim.x * 256) y[i] = __float2half_rn(__bfloat162float(x[i]));
+}
+
+int g_grid[2][3] = {{0, 0, 0}, {0, 0, 0}};  // [fp4][NB]
+
+}  // namespace
+
+bool gemv_mma_supported(const Shape& sh) {
+  if (sh.wtype == FT_W_BF16) return sh.d % 32 == 0 && sh.d_ff % 32 == 0;
+  if (sh.wtype == FT_W_NVFP4) return sh.d % 128 == 0 && sh.d_ff % 128 == 0;
+  return false;
+}
+
+template <int NB, bool FP4>
+cudaError_t grid_for(int sms) {
+  int per = 0;
+  const cudaError_t e =
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, gemv_mma_kernel<NB, FP4>, WARPS * 32, 0);
+  g_grid[FP4][NB] = sms * (per > 0 ? per : 1);
+  return e;
+}
+
+cudaError_t gemv_mma_init(int device) {
+  int sms = 0;
+  cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
+  if (e == cudaSuccess) e = grid_for<1, false>(sms);
+  if (e == cudaSuccess) e = grid_for<2, false>(sms);
+  if (e == cudaSuccess) e = grid_for<1, true>(sms);
+  if (e == cudaSuccess) e = grid_for<2, true>(sms);
+  return e;
+}
+
+void launch_to_f16(const void* x, int n, void* y, cudaStream_t st) {
+  const int grid = (n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184;
+  to_f16_kernel<<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, n, (__half*)y);
+}
+
+void launch_gemv_mma(const Shape& sh, int cls, int phase, int layer, const void* x16, int T, DevState& ds,
+                     int max_items, int max_tok, cudaStream_t st) {
+  MmaArgs a;
+  a.work = ds.work;
+  a.cls = cls;
+  a.layer = layer;
+  a.E = sh.E;
+  a.k = sh.k;
+  a.d = sh.d;
+  a.d_ff = sh.d_ff;
+  a.nvfp4 = sh.wtype == FT_W_NVFP4;
+  a.C = sh.C;
+  a.slot_bytes = sh.slot_bytes;
+  a.slots = ds.slots;
+  a.pool = ds.pool_dev;
+  a.x = x16;
+  a.perm = ds.perm;
+  a.tscale = ds.tscale;
+  a.h16 = ds.h16;
+  a.ybuf = ds.ybuf;
+  const int NB = T > 8 ? 2 : 1;
+  const long long chunks = (long long)max_items + (long long)max_tok / CHUNK;
+  const long long units = chunks * (phase == 0 ? sh.d_ff / 8 : sh.d / 16);
+  const long long ctas = (units + WARPS - 1) / WARPS;
+  const int cap = g_grid[a.nvfp4][NB];
+  const int grid = (int)(ctas < cap ? ctas : cap);
+  if (grid <= 0) return;
+  if (a.nvfp4) {
+    if (NB == 1) gemv_mma_kernel<1, true><<<grid, WARPS * 32, 0, st>>>(a, phase);
+    else gemv_mma_kernel<2, true><<<grid, WARPS * 32, 0, st>>>(a, phase);
+  } else {
+    if (NB == 1) gemv_mma_kernel<1, false><<<grid, WARPS * 32, 0, st>>>(a, phase);
+    else gemv_mma_kernel<2, false><<<grid, WARPS * 32, 0, st>>>(a, phase);
+  }
+}
+
+}  // namespace ft
