@@ -142,7 +142,7 @@ void free_all(ft_ctx* c) {
   DevState& d = c->ds;
   void* dev_ptrs[] = {d.slot_of, d.key_of, d.stamp, d.clk, d.ctr, d.error, d.work, d.scores, d.ids, d.wts,
                       d.counts, d.offsets, d.perm, d.inv, d.hbuf, d.ybuf, d.xs, d.hs, d.tscale, d.slots,
-                      d.h16, d.x16, c->probe_sink};
+                      d.h16, d.h16lo, d.x16, c->probe_sink};
   for (void* p : dev_ptrs)
     if (p) cudaFree(p);
   for (uint8_t* p : c->pool_host)
@@ -350,6 +350,7 @@ ft_status ft_moe_init(const ft_config* cfg, void* compute_stream, void* copy_str
   c->use_mma = gemv_mma_supported(sh);
   if (c->use_mma) {
     TRY(cuda_try(cudaMalloc((void**)&d.h16, sizeof(uint16_t) * Tk * sh.d_ff)));
+    if (sh.wtype == FT_W_BF16) TRY(cuda_try(cudaMalloc((void**)&d.h16lo, sizeof(uint16_t) * Tk * sh.d_ff)));
     if (sh.wtype == FT_W_NVFP4)
       TRY(cuda_try(cudaMalloc((void**)&d.x16, sizeof(uint16_t) * (size_t)cfg->max_tokens * sh.d)));
     TRY(cuda_try(gemv_mma_init(cfg->device)));

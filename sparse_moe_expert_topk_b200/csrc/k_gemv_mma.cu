@@ -18,7 +18,10 @@
 // Gate/up phase: rows 0..7 of the MMA tile are gate rows f0..f0+7 and rows
 // 8..15 the matching up rows, so each lane holds gate and up of the same
 // (feature, token) pairs and applies SwiGLU in registers; h is written as a
-// 16-bit activation (bf16 for BF16 experts, f16 for NVFP4) for the down phase.
+// 16-bit activation for the down phase: f16 for NVFP4 experts, and for BF16
+// experts as two bf16 parts hi + lo (both multiplied by W_down), which keeps h
+// to about 2^-16 relative -- a single bf16 rounding of h would spend most of
+// the 2e-2 rms error budget that the bf16 output rounding leaves.
 // NVFP4: 32 e2m1 codes per lane are converted to f16 pairs (cvt e2m1x2) and
 // multiplied by their e4m3 block scale (exact in f16), the per-matrix fp32
 // tensor scale is applied to the fp32 result.
@@ -90,6 +93,7 @@ struct MmaArgs {
   const int32_t* perm;
   const float* tscale;  // [L*E*3]
   uint16_t* h16;        // [T*k, d_ff] bf16 (BF16) or f16 (NVFP4) SwiGLU output
+  uint16_t* h16lo;      // [T*k, d_ff] BF16 experts: bf16 residual h - h16 (h = hi + lo to ~2^-16)
   float* ybuf;          // [T*k, d]
 };
 
@@ -100,9 +104,25 @@ __device__ __forceinline__ const uint8_t* blob_of(const MmaArgs& a, const WorkIt
 
 // acc[t][.] += W[rows g, g+8] . X[tokens] over K for one warp; t = n8 token tile.
 // BF16: per step each lane covers 8 K values of each row (4 lanes: 32 K).
-template <int NB, int U>
-__device__ __forceinline__ void dot_bf16(const uint8_t* ra, const uint8_t* rb, const uint16_t* const (&xr)[NB], int K,
-                                         int q, float (&acc)[NB][4]) {
+template <int NB, bool LO>
+__device__ __forceinline__ void bf16_step(const uint4 wa, const uint4 wb, const uint16_t* const (&xr)[NB],
+                                          const uint16_t* const (&xl)[NB], int e0, float (&acc)[NB][4]) {
+#pragma unroll
+  for (int t = 0; t < NB; ++t) {
+    const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xr[t] + e0));
+    mma_bf16(acc[t], wa.x, wb.x, wa.y, wb.y, xv.x, xv.y);
+    mma_bf16(acc[t], wa.z, wb.z, wa.w, wb.w, xv.z, xv.w);
+    if constexpr (LO) {
+      const uint4 xo = __ldg(reinterpret_cast<const uint4*>(xl[t] + e0));
+      mma_bf16(acc[t], wa.x, wb.x, wa.y, wb.y, xo.x, xo.y);
+      mma_bf16(acc[t], wa.z, wb.z, wa.w, wb.w, xo.z, xo.w);
+    }
+  }
+}
+
+template <int NB, int U, bool LO>
+__device__ __forceinline__ void dot_bf16(const uint8_t* ra, const uint8_t* rb, const uint16_t* const (&xr)[NB],
+                                         const uint16_t* const (&xl)[NB], int K, int q, float (&acc)[NB][4]) {
   const int steps = K / 32;
   const uint8_t* pa = ra + q * 16;
   const uint8_t* pb = rb + q * 16;
@@ -115,24 +135,10 @@ __device__ __forceinline__ void dot_bf16(const uint8_t* ra, const uint8_t* rb, c
       wb[u] = ld_stream(pb + (size_t)(s + u) * 64);
     }
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-#pragma unroll
-      for (int t = 0; t < NB; ++t) {
-        const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xr[t] + (s + u) * 32 + q * 8));
-        mma_bf16(acc[t], wa[u].x, wb[u].x, wa[u].y, wb[u].y, xv.x, xv.y);
-        mma_bf16(acc[t], wa[u].z, wb[u].z, wa[u].w, wb[u].w, xv.z, xv.w);
-      }
-    }
+    for (int u = 0; u < U; ++u) bf16_step<NB, LO>(wa[u], wb[u], xr, xl, (s + u) * 32 + q * 8, acc);
   }
-  for (; s < steps; ++s) {
-    const uint4 wa = ld_stream(pa + (size_t)s * 64), wb = ld_stream(pb + (size_t)s * 64);
-#pragma unroll
-    for (int t = 0; t < NB; ++t) {
-      const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xr[t] + s * 32 + q * 8));
-      mma_bf16(acc[t], wa.x, wb.x, wa.y, wb.y, xv.x, xv.y);
-      mma_bf16(acc[t], wa.z, wb.z, wa.w, wb.w, xv.z, xv.w);
-    }
-  }
+  for (; s < steps; ++s)
+    bf16_step<NB, LO>(ld_stream(pa + (size_t)s * 64), ld_stream(pb + (size_t)s * 64), xr, xl, s * 32 + q * 8, acc);
 }
 
 // NVFP4: per step each lane covers 32 K values (16 code bytes, two scale
@@ -246,14 +252,18 @@ __device__ void unit_work(const MmaArgs& a, const WorkItem& it, int chunk, int r
   const int base = it.tok_off + chunk * CHUNK;
   const int nt = min(CHUNK, it.n_tok - chunk * CHUNK);
   const uint16_t* xr[NB];
+  const uint16_t* xl[NB];
 #pragma unroll
   for (int t = 0; t < NB; ++t) {
     const int j = t * 8 + g;
     const int pos = base + (j < nt ? j : 0);
-    if (PHASE == 0)
+    if (PHASE == 0) {
       xr[t] = reinterpret_cast<const uint16_t*>(a.x) + (size_t)(a.perm[pos] / a.k) * a.d;
-    else
+      xl[t] = xr[t];
+    } else {
       xr[t] = a.h16 + (size_t)pos * a.d_ff;
+      xl[t] = a.h16lo + (size_t)pos * a.d_ff;
+    }
   }
   float acc[NB][4];
 #pragma unroll
@@ -261,7 +271,7 @@ __device__ void unit_work(const MmaArgs& a, const WorkItem& it, int chunk, int r
   if constexpr (FP4)
     dot_nvfp4<NB, 4>(ra, rbp, blob + sa0 + (size_t)rowa * sbytes, blob + sb0 + (size_t)rowb * sbytes, xr, K, q, acc);
   else
-    dot_bf16<NB, (NB == 1 ? 8 : 4)>(ra, rbp, xr, K, q, acc);
+    dot_bf16<NB, (NB == 1 ? 8 : 4), PHASE == 1>(ra, rbp, xr, xl, K, q, acc);
   // d0,d1: row g, tokens 2q, 2q+1; d2,d3: row g+8, same tokens (per n8 tile)
   float t0 = 1.f, t1 = 1.f;
   if (a.nvfp4) {
@@ -278,8 +288,14 @@ __device__ void unit_work(const MmaArgs& a, const WorkItem& it, int chunk, int r
       const float v0 = acc[t][c] * t0, v1 = acc[t][2 + c] * t1;
       if (PHASE == 0) {
         const float hv = v0 / (1.f + expf(-v0)) * v1;
-        const uint16_t hb = a.nvfp4 ? __half_as_ushort(__float2half_rn(hv)) : __bfloat16_as_ushort(__float2bfloat16_rn(hv));
-        a.h16[(size_t)(base + j) * a.d_ff + rb * 8 + g] = hb;
+        const size_t o = (size_t)(base + j) * a.d_ff + rb * 8 + g;
+        if constexpr (FP4) {
+          a.h16[o] = __half_as_ushort(__float2half_rn(hv));
+        } else {
+          const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
+          a.h16[o] = __bfloat16_as_ushort(hi);
+          a.h16lo[o] = __bfloat16_as_ushort(__float2bfloat16_rn(hv - __bfloat162float(hi)));
+        }
       } else {
         float* yr = a.ybuf + (size_t)(base + j) * a.d;
         yr[rb * 16 + g] = v0;
@@ -377,12 +393,17 @@ void launch_gemv_mma(const Shape& sh, int cls, int phase, int layer, const void*
   a.perm = ds.perm;
   a.tscale = ds.tscale;
   a.h16 = ds.h16;
+  a.h16lo = ds.h16lo;
   a.ybuf = ds.ybuf;
   const int NB = T > 8 ? 2 : 1;
   const long long chunks = (long long)max_items + (long long)max_tok / CHUNK;
   const long long units = chunks * (phase == 0 ? sh.d_ff / 8 : sh.d / 16);
   const long long ctas = (units + WARPS - 1) / WARPS;
-  const int cap = g_grid[a.nvfp4][NB];
+  // Streamed experts are read over the host link (~55 GB/s): a few dozen CTAs
+  // keep enough requests in flight for it, and leave the SMs to the HBM work
+  // of the hit and staged experts running at the same time.
+  const int cap = cls == KIND_STREAMED ? (g_grid[a.nvfp4][NB] < 64 ? g_grid[a.nvfp4][NB] : 64)
+                                       : g_grid[a.nvfp4][NB];
   const int grid = (int)(ctas < cap ? ctas : cap);
   if (grid <= 0) return;
   if (a.nvfp4) {
