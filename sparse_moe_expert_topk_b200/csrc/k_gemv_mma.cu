@@ -102,8 +102,8 @@ __device__ __forceinline__ const uint8_t* blob_of(const MmaArgs& a, const WorkIt
   return a.slots + (size_t)it.slot * a.slot_bytes;
 }
 
-// acc[t][.] += W[rows g, g+8] . X[tokens] over K for one warp; t = n8 token tile.
-// BF16: per step each lane covers 8 K values of each row (4 lanes: 32 K).
+// One BF16 step: 8 K values of rows g and g+8 per lane, two MMAs per token
+// tile (and two more for the low part of h in the down phase).
 template <int NB, bool LO>
 __device__ __forceinline__ void bf16_step(const uint4 wa, const uint4 wb, const uint16_t* const (&xr)[NB],
                                           const uint16_t* const (&xl)[NB], int e0, float (&acc)[NB][4]) {
@@ -120,29 +120,7 @@ __device__ __forceinline__ void bf16_step(const uint4 wa, const uint4 wb, const 
   }
 }
 
-template <int NB, int U, bool LO>
-__device__ __forceinline__ void dot_bf16(const uint8_t* ra, const uint8_t* rb, const uint16_t* const (&xr)[NB],
-                                         const uint16_t* const (&xl)[NB], int K, int q, float (&acc)[NB][4]) {
-  const int steps = K / 32;
-  const uint8_t* pa = ra + q * 16;
-  const uint8_t* pb = rb + q * 16;
-  int s = 0;
-  for (; s + U <= steps; s += U) {
-    uint4 wa[U], wb[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      wa[u] = ld_stream(pa + (size_t)(s + u) * 64);
-      wb[u] = ld_stream(pb + (size_t)(s + u) * 64);
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) bf16_step<NB, LO>(wa[u], wb[u], xr, xl, (s + u) * 32 + q * 8, acc);
-  }
-  for (; s < steps; ++s)
-    bf16_step<NB, LO>(ld_stream(pa + (size_t)s * 64), ld_stream(pb + (size_t)s * 64), xr, xl, s * 32 + q * 8, acc);
-}
-
-// NVFP4: per step each lane covers 32 K values (16 code bytes, two scale
-// blocks) of each row (4 lanes: 128 K); eight MMAs per step.
+// 16 code bytes (32 e2m1 values) and their two e4m3 scales -> 16 f16 pairs.
 __device__ __forceinline__ void decode_nvfp4(const uint4 w, uint32_t sc, uint32_t (&h)[16]) {
   e2m1x8_to_f16x8(w.x, *reinterpret_cast<uint32_t(*)[4]>(&h[0]));
   e2m1x8_to_f16x8(w.y, *reinterpret_cast<uint32_t(*)[4]>(&h[4]));
@@ -158,31 +136,86 @@ __device__ __forceinline__ void decode_nvfp4(const uint4 w, uint32_t sc, uint32_
   for (int j = 8; j < 16; ++j) h[j] = hmul2(h[j], shi);
 }
 
-template <int NB, int U>
-__device__ __forceinline__ void dot_nvfp4(const uint8_t* ra, const uint8_t* rb, const uint8_t* sa, const uint8_t* sb,
-                                          const uint16_t* const (&xr)[NB], int K, int q, float (&acc)[NB][4]) {
-  const int steps = K / 128;
-  const uint8_t* pa = ra + q * 16;
-  const uint8_t* pb = rb + q * 16;
-  const unsigned short* qa = reinterpret_cast<const unsigned short*>(sa) + q;
-  const unsigned short* qb = reinterpret_cast<const unsigned short*>(sb) + q;
-  int s = 0;
-  for (; s < steps; s += U) {
-    const int n = steps - s < U ? steps - s : U;
+// Where a warp's two weight rows come from: straight from global memory
+// (HBM slots: 128-bit non-caching loads) or from the warp's shared-memory
+// tile, filled beforehand with cp.async (streamed experts: each warp
+// instruction reads a contiguous run of a row, which the host link moves in
+// large requests). Both hand the MMAs the same 16-byte vectors in the same
+// order, so the arithmetic does not depend on the source.
+template <bool STAGED>
+struct RowSrc {
+  const uint8_t* ga;  // global row g (+ q*16), direct mode
+  const uint8_t* gb;  // global row g+8 (+ q*16)
+  const uint8_t* ta;  // smem row g of this warp's tile (+ q*16), staged mode
+  const uint8_t* tb;
+  int s0;             // first step of this warp
+  __device__ __forceinline__ uint4 a(int s) const {
+    if constexpr (STAGED) return *reinterpret_cast<const uint4*>(ta + (s - s0) * 64);
+    else return ld_stream(ga + (size_t)s * 64);
+  }
+  __device__ __forceinline__ uint4 b(int s) const {
+    if constexpr (STAGED) return *reinterpret_cast<const uint4*>(tb + (s - s0) * 64);
+    else return ld_stream(gb + (size_t)s * 64);
+  }
+};
+
+// Scale pair (two e4m3 bytes) of step s for rows g and g+8 (NVFP4).
+template <bool STAGED>
+struct ScaleSrc {
+  const unsigned short* ga;  // global scale row g (+ q)
+  const unsigned short* gb;
+  const unsigned short* ta;  // smem scale row g (+ q)
+  const unsigned short* tb;
+  int s0;
+  __device__ __forceinline__ uint32_t a(int s) const {
+    if constexpr (STAGED) return ta[(s - s0) * 4];
+    else return __ldg(ga + s * 4);
+  }
+  __device__ __forceinline__ uint32_t b(int s) const {
+    if constexpr (STAGED) return tb[(s - s0) * 4];
+    else return __ldg(gb + s * 4);
+  }
+};
+
+// acc[t][.] += W[rows g, g+8] . X[tokens] over steps [s0, s1) of 32 K values
+// (BF16: lane q covers K = 32 s + 8 q .. +8). U steps of loads in flight;
+// steps past s1 reload the last step (its result is not used).
+template <int NB, int U, bool LO, class Src>
+__device__ __forceinline__ void dot_bf16(const Src& src, int s0, int s1, const uint16_t* const (&xr)[NB],
+                                         const uint16_t* const (&xl)[NB], int q, float (&acc)[NB][4]) {
+  for (int s = s0; s < s1; s += U) {
+    uint4 wa[U], wb[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int ss = s + u < s1 ? s + u : s1 - 1;
+      wa[u] = src.a(ss);
+      wb[u] = src.b(ss);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (s + u < s1) bf16_step<NB, LO>(wa[u], wb[u], xr, xl, (s + u) * 32 + q * 8, acc);
+  }
+}
+
+// NVFP4: steps of 128 K values (lane q covers K = 128 s + 32 q .. +32: 16
+// code bytes and one scale pair per row); eight MMAs per step.
+template <int NB, int U, class Src, class Sc>
+__device__ __forceinline__ void dot_nvfp4(const Src& src, const Sc& sc, int s0, int s1,
+                                          const uint16_t* const (&xr)[NB], int q, float (&acc)[NB][4]) {
+  for (int s = s0; s < s1; s += U) {
     uint4 wa[U], wb[U];
     uint32_t ca[U], cb[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      if (u < n) {
-        wa[u] = ld_stream(pa + (size_t)(s + u) * 64);
-        wb[u] = ld_stream(pb + (size_t)(s + u) * 64);
-        ca[u] = __ldg(qa + (s + u) * 4);
-        cb[u] = __ldg(qb + (s + u) * 4);
-      }
+      const int ss = s + u < s1 ? s + u : s1 - 1;
+      wa[u] = src.a(ss);
+      wb[u] = src.b(ss);
+      ca[u] = sc.a(ss);
+      cb[u] = sc.b(ss);
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      if (u < n) {
+      if (s + u < s1) {
         uint32_t ha[16], hb[16];
         decode_nvfp4(wa[u], ca[u], ha);
         decode_nvfp4(wb[u], cb[u], hb);
@@ -207,7 +240,18 @@ __device__ __forceinline__ void dot_nvfp4(const uint8_t* ra, const uint8_t* rb, 
   }
 }
 
-// Map warp-unit u of this class to (item, 16-token chunk, row block).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async8(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Map CTA-unit u of this class to (item, 16-token chunk, 16-row block).
 __device__ __forceinline__ bool unit_of(const int* pref, int n_items, int rblocks, int u, int& item, int& chunk,
                                         int& rb) {
   const int qi = u / rblocks;
@@ -223,32 +267,68 @@ __device__ __forceinline__ bool unit_of(const int* pref, int n_items, int rblock
   return true;
 }
 
-constexpr int CHUNK = 16;  // tokens per warp-unit (two n8 tiles)
+constexpr int CHUNK = 16;  // tokens per unit (two n8 tiles)
 
-template <int NB, int PHASE, bool FP4>
-__device__ void unit_work(const MmaArgs& a, const WorkItem& it, int chunk, int rb, int lane) {
+// Per-warp tile geometry of the staged mode (bytes per row, padded so the
+// 8 rows a warp's lanes read at once fall in distinct bank groups).
+__host__ __device__ __forceinline__ int tile_row_bytes(int steps_w) { return steps_w * 64 + 16; }
+__host__ __device__ __forceinline__ int tile_scale_bytes(int steps_w) { return steps_w * 8 + 16; }
+__host__ __device__ __forceinline__ int max_steps_per_warp(int steps) { return (steps + WARPS - 1) / WARPS; }
+__host__ __device__ __forceinline__ int warp_tile_bytes(int steps, bool fp4) {
+  const int sw = max_steps_per_warp(steps);
+  return 16 * tile_row_bytes(sw) + (fp4 ? 16 * tile_scale_bytes(sw) : 0);
+}
+
+// One CTA-unit: 16 weight rows x one chunk of <= 16 tokens, the K range split
+// over the 8 warps, partial sums reduced in warp order, epilogue by warp 0.
+template <int NB, int PHASE, bool FP4, bool STAGED>
+__device__ void unit_work(const MmaArgs& a, const WorkItem& it, int chunk, int rb, int warp, int lane,
+                          uint8_t* tiles, float* red) {
   const int g = lane >> 2, q = lane & 3;
   const uint8_t* blob = blob_of(a, it);
   const size_t n = (size_t)a.d * a.d_ff;
   const int K = PHASE == 0 ? a.d : a.d_ff;
-  const size_t rbytes = a.nvfp4 ? (size_t)K / 2 : (size_t)K * 2;
+  const size_t rbytes = FP4 ? (size_t)K / 2 : (size_t)K * 2;
   const size_t sbytes = (size_t)K / 16;
-  int rowa, rowb;          // rows inside their matrices
-  size_t ma, mb, sa0, sb0;  // matrix byte offsets (codes, scales)
-  if (PHASE == 0) {
-    rowa = rowb = rb * 8 + g;
-    ma = 0;
-    mb = a.nvfp4 ? n / 2 : n * 2;
-    sa0 = 3 * (n / 2);
-    sb0 = 3 * (n / 2) + n / 16;
-  } else {
-    rowa = rb * 16 + g;
-    rowb = rowa + 8;
-    ma = mb = a.nvfp4 ? n : n * 4;
-    sa0 = sb0 = 3 * (n / 2) + 2 * (n / 16);
+  const int steps = FP4 ? K / 128 : K / 32;
+  const int s0 = (warp * steps) / WARPS, s1 = ((warp + 1) * steps) / WARPS;
+  // rows 0..7 / 8..15 of the tile: gate / up rows rb*8.. (phase 0), down rows rb*16.. (phase 1)
+  auto row_ptr = [&](int r) -> const uint8_t* {
+    if (PHASE == 0) return blob + (r < 8 ? 0 : (FP4 ? n / 2 : n * 2)) + (size_t)(rb * 8 + (r & 7)) * rbytes;
+    return blob + (FP4 ? n : n * 4) + (size_t)(rb * 16 + r) * rbytes;
+  };
+  auto scale_ptr = [&](int r) -> const uint8_t* {
+    const size_t base = 3 * (n / 2);
+    if (PHASE == 0) return blob + base + (r < 8 ? 0 : n / 16) + (size_t)(rb * 8 + (r & 7)) * sbytes;
+    return blob + base + 2 * (n / 16) + (size_t)(rb * 16 + r) * sbytes;
+  };
+  const int sw = max_steps_per_warp(steps);
+  uint8_t* tile = tiles + (size_t)warp * warp_tile_bytes(steps, FP4);
+  const int trow = tile_row_bytes(sw), tsrow = tile_scale_bytes(sw);
+  if (STAGED && s1 > s0) {
+    // contiguous per-row runs: flattened (row, byte) index, 16 bytes per lane
+    const int nb = (s1 - s0) * 64;
+    for (int e = lane * 16; e < 16 * nb; e += 512) {
+      const int r = e / nb, off = e - r * nb;
+      cp_async16(tile + r * trow + off, row_ptr(r) + (size_t)s0 * 64 + off);
+    }
+    if (FP4) {
+      const int ns = (s1 - s0) * 8;
+      uint8_t* st = tile + 16 * trow;
+      for (int e = lane * 8; e < 16 * ns; e += 256) {
+        const int r = e / ns, off = e - r * ns;
+        cp_async8(st + r * tsrow + off, scale_ptr(r) + (size_t)s0 * 8 + off);
+      }
+    }
+    cp_async_wait_all();
+    __syncwarp();
   }
-  const uint8_t* ra = blob + ma + (size_t)rowa * rbytes;
-  const uint8_t* rbp = blob + mb + (size_t)rowb * rbytes;
+  RowSrc<STAGED> src;
+  src.ga = row_ptr(g) + q * 16;
+  src.gb = row_ptr(g + 8) + q * 16;
+  src.ta = tile + g * trow + q * 16;
+  src.tb = tile + (g + 8) * trow + q * 16;
+  src.s0 = s0;
   const int base = it.tok_off + chunk * CHUNK;
   const int nt = min(CHUNK, it.n_tok - chunk * CHUNK);
   const uint16_t* xr[NB];
@@ -268,47 +348,73 @@ __device__ void unit_work(const MmaArgs& a, const WorkItem& it, int chunk, int r
   float acc[NB][4];
 #pragma unroll
   for (int t = 0; t < NB; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-  if constexpr (FP4)
-    dot_nvfp4<NB, 4>(ra, rbp, blob + sa0 + (size_t)rowa * sbytes, blob + sb0 + (size_t)rowb * sbytes, xr, K, q, acc);
-  else
-    dot_bf16<NB, (NB == 1 ? 8 : 4), PHASE == 1>(ra, rbp, xr, xl, K, q, acc);
-  // d0,d1: row g, tokens 2q, 2q+1; d2,d3: row g+8, same tokens (per n8 tile)
-  float t0 = 1.f, t1 = 1.f;
-  if (a.nvfp4) {
-    const float* ts = a.tscale + ((size_t)a.layer * a.E + it.e) * 3;
-    t0 = PHASE == 0 ? ts[0] : ts[2];
-    t1 = PHASE == 0 ? ts[1] : ts[2];
+  if constexpr (FP4) {
+    ScaleSrc<STAGED> sc;
+    sc.ga = reinterpret_cast<const unsigned short*>(scale_ptr(g)) + q;
+    sc.gb = reinterpret_cast<const unsigned short*>(scale_ptr(g + 8)) + q;
+    sc.ta = reinterpret_cast<const unsigned short*>(tile + 16 * trow + g * tsrow) + q;
+    sc.tb = reinterpret_cast<const unsigned short*>(tile + 16 * trow + (g + 8) * tsrow) + q;
+    sc.s0 = s0;
+    dot_nvfp4<NB, 4>(src, sc, s0, s1, xr, q, acc);
+  } else {
+    dot_bf16<NB, (NB == 1 ? 8 : 4), PHASE == 1>(src, s0, s1, xr, xl, q, acc);
   }
+  // split-K reduction over the warps, in warp order
 #pragma unroll
-  for (int t = 0; t < NB; ++t) {
+  for (int t = 0; t < NB; ++t)
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const int j = t * 8 + 2 * q + c;
-      if (j >= nt) continue;
-      const float v0 = acc[t][c] * t0, v1 = acc[t][2 + c] * t1;
-      if (PHASE == 0) {
-        const float hv = v0 / (1.f + expf(-v0)) * v1;
-        const size_t o = (size_t)(base + j) * a.d_ff + rb * 8 + g;
-        if constexpr (FP4) {
-          a.h16[o] = __half_as_ushort(__float2half_rn(hv));
+    for (int c = 0; c < 4; ++c) red[(warp * NB * 4 + t * 4 + c) * 32 + lane] = acc[t][c];
+  __syncthreads();
+  if (warp == 0) {
+#pragma unroll
+    for (int t = 0; t < NB; ++t)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float v = red[(t * 4 + c) * 32 + lane];
+        for (int w = 1; w < WARPS; ++w) v += red[(w * NB * 4 + t * 4 + c) * 32 + lane];
+        acc[t][c] = v;
+      }
+    // d0,d1: row g, tokens 2q, 2q+1; d2,d3: row g+8, same tokens (per n8 tile)
+    float t0 = 1.f, t1 = 1.f;
+    if constexpr (FP4) {
+      const float* ts = a.tscale + ((size_t)a.layer * a.E + it.e) * 3;
+      t0 = PHASE == 0 ? ts[0] : ts[2];
+      t1 = PHASE == 0 ? ts[1] : ts[2];
+    }
+#pragma unroll
+    for (int t = 0; t < NB; ++t) {
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int j = t * 8 + 2 * q + c;
+        if (j >= nt) continue;
+        const float v0 = acc[t][c] * t0, v1 = acc[t][2 + c] * t1;
+        if (PHASE == 0) {
+          const float hv = v0 / (1.f + expf(-v0)) * v1;
+          const size_t o = (size_t)(base + j) * a.d_ff + rb * 8 + g;
+          if constexpr (FP4) {
+            a.h16[o] = __half_as_ushort(__float2half_rn(hv));
+          } else {
+            const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
+            a.h16[o] = __bfloat16_as_ushort(hi);
+            a.h16lo[o] = __bfloat16_as_ushort(__float2bfloat16_rn(hv - __bfloat162float(hi)));
+          }
         } else {
-          const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
-          a.h16[o] = __bfloat16_as_ushort(hi);
-          a.h16lo[o] = __bfloat16_as_ushort(__float2bfloat16_rn(hv - __bfloat162float(hi)));
+          float* yr = a.ybuf + (size_t)(base + j) * a.d;
+          yr[rb * 16 + g] = v0;
+          yr[rb * 16 + g + 8] = v1;
         }
-      } else {
-        float* yr = a.ybuf + (size_t)(base + j) * a.d;
-        yr[rb * 16 + g] = v0;
-        yr[rb * 16 + g + 8] = v1;
       }
     }
   }
+  __syncthreads();  // red and the tiles are reused by the next unit
 }
 
-template <int NB, bool FP4>
+template <int NB, bool FP4, bool STAGED>
 __global__ void __launch_bounds__(WARPS * 32) gemv_mma_kernel(MmaArgs a, int phase) {
+  extern __shared__ __align__(16) uint8_t tiles[];
   __shared__ int s_pref[MAX_E + 1];
   __shared__ WorkItem s_items[MAX_E];
+  __shared__ float red[WARPS * NB * 4 * 32];
   const int n_items = a.work->n_items[a.cls];
   if (n_items == 0) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -325,13 +431,13 @@ __global__ void __launch_bounds__(WARPS * 32) gemv_mma_kernel(MmaArgs a, int pha
   __syncthreads();
   const int rblocks = phase == 0 ? a.d_ff / 8 : a.d / 16;
   const int n_units = s_pref[n_items] * rblocks;
-  for (int u = blockIdx.x * WARPS + warp; u < n_units; u += gridDim.x * WARPS) {
+  for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
     int item, chunk, rb;
     if (!unit_of(s_pref, n_items, rblocks, u, item, chunk, rb)) break;
     const WorkItem it = s_items[item];
     if (a.cls != KIND_STREAMED && (it.slot < 0 || it.slot >= a.C)) continue;  // error already latched
-    if (phase == 0) unit_work<NB, 0, FP4>(a, it, chunk, rb, lane);
-    else unit_work<NB, 1, FP4>(a, it, chunk, rb, lane);
+    if (phase == 0) unit_work<NB, 0, FP4, STAGED>(a, it, chunk, rb, warp, lane, tiles, red);
+    else unit_work<NB, 1, FP4, STAGED>(a, it, chunk, rb, warp, lane, tiles, red);
   }
 }
 
@@ -340,7 +446,8 @@ __global__ void __launch_bounds__(256) to_f16_kernel(const __nv_bfloat16* __rest
   for (int i = blockIdx.x * 256 + threadIdx.x; i < n; i += gridDim.x * 256) y[i] = __float2half_rn(__bfloat162float(x[i]));
 }
 
-int g_grid[2][3] = {{0, 0, 0}, {0, 0, 0}};  // [fp4][NB]
+int g_grid[2][3] = {{0, 0, 0}, {0, 0, 0}};  // [fp4][NB], direct mode
+constexpr int STAGED_SMEM_MAX = 200 * 1024;
 
 }  // namespace
 
@@ -351,10 +458,12 @@ bool gemv_mma_supported(const Shape& sh) {
 }
 
 template <int NB, bool FP4>
-cudaError_t grid_for(int sms) {
+cudaError_t kernel_setup(int sms) {
+  cudaError_t e = cudaFuncSetAttribute(gemv_mma_kernel<NB, FP4, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       STAGED_SMEM_MAX);
+  if (e != cudaSuccess) return e;
   int per = 0;
-  const cudaError_t e =
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, gemv_mma_kernel<NB, FP4>, WARPS * 32, 0);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, gemv_mma_kernel<NB, FP4, false>, WARPS * 32, 0);
   g_grid[FP4][NB] = sms * (per > 0 ? per : 1);
   return e;
 }
@@ -362,11 +471,17 @@ cudaError_t grid_for(int sms) {
 cudaError_t gemv_mma_init(int device) {
   int sms = 0;
   cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
-  if (e == cudaSuccess) e = grid_for<1, false>(sms);
-  if (e == cudaSuccess) e = grid_for<2, false>(sms);
-  if (e == cudaSuccess) e = grid_for<1, true>(sms);
-  if (e == cudaSuccess) e = grid_for<2, true>(sms);
+  if (e == cudaSuccess) e = kernel_setup<1, false>(sms);
+  if (e == cudaSuccess) e = kernel_setup<2, false>(sms);
+  if (e == cudaSuccess) e = kernel_setup<1, true>(sms);
+  if (e == cudaSuccess) e = kernel_setup<2, true>(sms);
   return e;
+}
+
+template <int NB, bool FP4>
+void launch_variant(bool staged, int grid, int dyn, const MmaArgs& a, int phase, cudaStream_t st) {
+  if (staged) gemv_mma_kernel<NB, FP4, true><<<grid, WARPS * 32, dyn, st>>>(a, phase);
+  else gemv_mma_kernel<NB, FP4, false><<<grid, WARPS * 32, 0, st>>>(a, phase);
 }
 
 void launch_to_f16(const void* x, int n, void* y, cudaStream_t st) {
@@ -398,20 +513,23 @@ void launch_gemv_mma(const Shape& sh, int cls, int phase, int layer, const void*
   const int NB = T > 8 ? 2 : 1;
   const long long chunks = (long long)max_items + (long long)max_tok / CHUNK;
   const long long units = chunks * (phase == 0 ? sh.d_ff / 8 : sh.d / 16);
-  const long long ctas = (units + WARPS - 1) / WARPS;
-  // Streamed experts are read over the host link (~55 GB/s): a few dozen CTAs
-  // keep enough requests in flight for it, and leave the SMs to the HBM work
-  // of the hit and staged experts running at the same time.
-  const int cap = cls == KIND_STREAMED ? (g_grid[a.nvfp4][NB] < 64 ? g_grid[a.nvfp4][NB] : 64)
-                                       : g_grid[a.nvfp4][NB];
-  const int grid = (int)(ctas < cap ? ctas : cap);
+  // Streamed experts come over the host link (~55 GB/s): they are staged
+  // through shared memory in contiguous runs, on a few dozen CTAs, leaving
+  // the SMs to the HBM work of the hit and staged experts meanwhile.
+  const int K = phase == 0 ? sh.d : sh.d_ff;
+  const int steps = a.nvfp4 ? K / 128 : K / 32;
+  const int smem = WARPS * warp_tile_bytes(steps, a.nvfp4);
+  const bool staged = cls == KIND_STREAMED && smem <= STAGED_SMEM_MAX;
+  int cap = g_grid[a.nvfp4][NB];
+  if (cls == KIND_STREAMED && cap > 64) cap = 64;
+  const int grid = (int)(units < cap ? units : cap);
   if (grid <= 0) return;
   if (a.nvfp4) {
-    if (NB == 1) gemv_mma_kernel<1, true><<<grid, WARPS * 32, 0, st>>>(a, phase);
-    else gemv_mma_kernel<2, true><<<grid, WARPS * 32, 0, st>>>(a, phase);
+    if (NB == 1) launch_variant<1, true>(staged, grid, smem, a, phase, st);
+    else launch_variant<2, true>(staged, grid, smem, a, phase, st);
   } else {
-    if (NB == 1) gemv_mma_kernel<1, false><<<grid, WARPS * 32, 0, st>>>(a, phase);
-    else gemv_mma_kernel<2, false><<<grid, WARPS * 32, 0, st>>>(a, phase);
+    if (NB == 1) launch_variant<1, false>(staged, grid, smem, a, phase, st);
+    else launch_variant<2, false>(staged, grid, smem, a, phase, st);
   }
 }
 
