@@ -234,6 +234,39 @@ typedef struct {
  * clears the totals after copying. */
 ft_status ft_moe_profile_read(ft_ctx* ctx, ft_kernel_time* out, int32_t cap, int32_t* n_out, int32_t reset);
 
+/* Router logits, top-k and softmax weights of one layer WITHOUT allocating
+ * anything: the same kernels as ft_moe_layer_forward's routing, with their
+ * logits scratch in a fixed device array compiled into this library.
+ *
+ * The paper has no counterpart for this entry point. It exists for callers
+ * that cannot call cudaMalloc at the point where they route: a serving loop
+ * whose memory manager has already handed every free byte of HBM to the KV
+ * cache and the expert slots (an allocation would fail or force an eviction),
+ * code that must not take the implicit device synchronisation of cudaMalloc /
+ * cudaFree in the middle of a decode step, or a host program that forbids
+ * allocations outside its own allocator. No context is needed.
+ *
+ *   x_dev [T][d_model] activations (fp32 when wtype is FT_W_F32, else bf16),
+ *   w_router_dev [n_experts][d_model] (same type), both 16-byte aligned;
+ *   bias_dev NULL, [n_experts] or [T][n_experts] fp32 (bias_per_token);
+ *   ids_dev [T][top_k] int32 and w_dev [T][top_k] fp32 receive the result in
+ *   rank order, exactly as ft_moe_layer_forward's ids/weights outputs.
+ *   stream: cudaStream_t to enqueue on (0 = legacy default stream).
+ * Limits: T <= FT_ROUTE_STATIC_MAX_TOKENS (the scratch holds that many tokens
+ * times 512 experts of fp32 logits, 2 MiB, resident on every GPU that loads
+ * the library until the process exits); n_experts <= 512, top_k <= 16,
+ * d_model a multiple of 64. Larger sizes return FT_EINVAL, nothing is launched.
+ * The first call on a device looks up the scratch's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call before
+ * any stream capture. It calls no cudaMalloc, cudaFree or allocating routine.
+ * All calls share the one scratch array: calls that may overlap on the GPU
+ * (different streams without ordering between them) race on it; order them.
+ * The scratch needs no clearing: every logit a call reads it wrote first. */
+#define FT_ROUTE_STATIC_MAX_TOKENS 1024
+ft_status ft_route_topk_static(const void* x_dev, const void* w_router_dev, const float* bias_dev,
+                               int32_t bias_per_token, int32_t T, int32_t n_experts, int32_t d_model, int32_t top_k,
+                               int32_t wtype, int32_t* ids_dev, float* w_dev, void* stream);
+
 /* Static string for a status code. */
 const char* ft_status_str(ft_status s);
 

@@ -28,8 +28,9 @@ EXPORTS = (
     "ft_moe_slot_bytes", "ft_moe_init", "ft_moe_destroy", "ft_moe_expert_ptr", "ft_moe_set_tensor_scales",
     "ft_moe_set_router", "ft_moe_layer_forward", "ft_cache_stats", "ft_set_bandwidths", "ft_moe_reset_cache",
     "ft_moe_last_route", "ft_moe_cache_contents", "ft_moe_probe_link", "ft_moe_profile", "ft_moe_profile_read",
-    "ft_status_str",
+    "ft_route_topk_static", "ft_status_str",
 )
+FT_ROUTE_STATIC_MAX_TOKENS = 1024
 
 
 class FtConfig(ctypes.Structure):
@@ -87,6 +88,7 @@ def lib() -> ctypes.CDLL:
             "ft_moe_probe_link": [P, U64, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)],
             "ft_moe_profile": [P, I32],
             "ft_moe_profile_read": [P, ctypes.POINTER(FtKernelTime), I32, ctypes.POINTER(I32), I32],
+            "ft_route_topk_static": [P, P, P, I32, I32, I32, I32, I32, I32, P, P, P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -224,3 +226,10 @@ def ft_moe_profile_read(ctx, reset=True) -> dict:
     _check("ft_moe_profile_read", lib().ft_moe_profile_read(ctx, arr, cap, ctypes.byref(n), 1 if reset else 0))
     return {arr[i].name.decode(): dict(launches=arr[i].launches, ms=arr[i].ms, bytes=arr[i].bytes,
                                        flops=arr[i].flops) for i in range(min(n.value, cap))}
+
+
+def ft_route_topk_static(x, w_router, bias, bias_per_token, T, n_experts, d_model, top_k, wtype, ids, w, stream):
+    """Router + top-k with no allocation (scratch in a static device array)."""
+    _check("ft_route_topk_static",
+           lib().ft_route_topk_static(_ptr(x), _ptr(w_router), _ptr(bias), bias_per_token, T, n_experts, d_model,
+                                      top_k, wtype, _ptr(ids), _ptr(w), _stream(stream)))

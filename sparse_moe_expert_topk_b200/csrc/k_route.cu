@@ -6,6 +6,8 @@
 // router function; this follows the reading documented with the C ABI:
 // logits s = x W_r^T + b in fp32, the k largest logits (equal logits -> lower
 // expert index), softmax over those k.
+#include <atomic>
+
 #include "ft_internal.cuh"
 
 namespace ft {
@@ -240,6 +242,56 @@ void launch_permute(const Shape& sh, int T, DevState& ds, cudaStream_t st) {
   permute_kernel<<<1, 1024, permute_smem_bytes(sh.E), st>>>(ds.ids, T * sh.k, sh.E, ds.counts, ds.offsets, ds.perm,
                                                            ds.inv);
 }
+
+// ---------------------------------------------------------------------------
+// Router + top-k without any allocation (ft_route_topk_static in ft_moe.h).
+// The logits scratch is this file-scope device array instead of a buffer the
+// library or the caller allocates. Its host-side name is only a stand-in, so
+// the device address is looked up once per device with cudaGetSymbolAddress
+// and cached.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr int STATIC_MAX_TOKENS = FT_ROUTE_STATIC_MAX_TOKENS;
+constexpr int MAX_DEVICES = 64;
+static __device__ __align__(256) float g_static_scores[STATIC_MAX_TOKENS * MAX_E];
+std::atomic<float*> g_static_ptr[MAX_DEVICES];
+}  // namespace
+
+}  // namespace ft
+
+extern "C" ft_status ft_route_topk_static(const void* x_dev, const void* w_router_dev, const float* bias_dev,
+                                          int32_t bias_per_token, int32_t T, int32_t n_experts, int32_t d_model,
+                                          int32_t top_k, int32_t wtype, int32_t* ids_dev, float* w_dev,
+                                          void* stream) {
+  using namespace ft;
+  if (T < 0 || T > STATIC_MAX_TOKENS || n_experts < 1 || n_experts > MAX_E || top_k < 1 || top_k > MAX_K ||
+      top_k > n_experts || d_model < 64 || d_model % 64 || (wtype != FT_W_F32 && wtype != FT_W_BF16 &&
+      wtype != FT_W_NVFP4))
+    return FT_EINVAL;
+  if (T == 0) return FT_OK;
+  if (!x_dev || !w_router_dev || !ids_dev || !w_dev) return FT_EINVAL;
+  if (((uintptr_t)x_dev | (uintptr_t)w_router_dev) & 15) return FT_EINVAL;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return FT_ECUDA;
+  float* scores = g_static_ptr[dev].load(std::memory_order_acquire);
+  if (!scores) {  // first call on this device: resolve the array's device address
+    if (cudaGetSymbolAddress((void**)&scores, g_static_scores) != cudaSuccess || !scores) return FT_ECUDA;
+    g_static_ptr[dev].store(scores, std::memory_order_release);
+  }
+  Shape sh{};
+  sh.E = n_experts;
+  sh.k = top_k;
+  sh.d = d_model;
+  sh.wtype = wtype;
+  const cudaStream_t st = (cudaStream_t)stream;
+  launch_router_scores(sh, x_dev, w_router_dev, bias_dev, bias_per_token, T, scores, st);
+  const int warps_per_cta = 8;
+  topk_softmax_kernel<<<(T + warps_per_cta - 1) / warps_per_cta, 32 * warps_per_cta, 0, st>>>(
+      scores, T, n_experts, top_k, ids_dev, w_dev);
+  return cudaGetLastError() == cudaSuccess ? FT_OK : FT_ECUDA;
+}
+
+namespace ft {
 
 cudaError_t route_kernels_init(int E) {
   return cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
