@@ -311,6 +311,104 @@ def run_reference(args, wl, world, rank):
     return 0
 
 
+
+# --------------------------------------------------------------------------
+# secondary workloads (not the default line): single-layer prefill, 43-layer
+# NVFP4 decode trace
+# --------------------------------------------------------------------------
+def _timed(stream, device, fn, steps):
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    return e0.elapsed_time(e1) / steps
+
+
+def run_secondary(args, wl, world, rank, local):
+    import ftgen
+    import sparse_moe_expert_topk_b200 as ft
+    from ftgen.ctx import Harness
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    peaks, peak_kind = load_peaks()
+    out = {"metric": METRIC, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "data": "synthetic"}
+    if wl.name == "prefill_bf16":
+        T = wl.batches[0]
+        h = Harness(wl, max_tokens=T, device=local)
+        x = ftgen.hidden(T, wl.d, wl.wtype, wl.seed("bench", rank)).to(device)
+        y = torch.empty_like(x)
+
+        def call():
+            ft.ft_moe_layer_forward(h.ctx, 0, ft.FT_PREFILL, x, T, None, 0, y)
+
+        def cold():
+            ft.ft_moe_reset_cache(h.ctx)
+            call()
+        for _ in range(args.warmup):
+            cold()
+        ms_cold = _timed(h.stream, device, cold, args.steps)
+        ms_hot = _timed(h.stream, device, call, args.steps)
+        ft.ft_moe_profile(h.ctx, True)
+        call()
+        prof = ft.ft_moe_profile_read(h.ctx)
+        ft.ft_moe_profile(h.ctx, False)
+        h2d, zc = ft.ft_moe_probe_link(h.ctx, 1 << 30)
+        roof, rows = roofline(prof, peaks, peak_kind, h2d)
+        h.close()
+        link_bytes = wl.E * wl.slot_bytes
+        out.update(value=round(T / (ms_hot / 1e3), 1), ms_per_step=round(ms_hot, 3), dtype="bf16",
+                   config={"workload": f"single-layer BF16 prefill, T={T}, E=256 top-6 d=4096 d_ff=1536, b=0"},
+                   hot={"tokens_per_s": round(T / (ms_hot / 1e3), 1), "ms": round(ms_hot, 3)},
+                   cold={"tokens_per_s": round(T / (ms_cold / 1e3), 1), "ms": round(ms_cold, 3),
+                         "link_gbs": round(link_bytes / (ms_cold * 1e6), 2),
+                         "link_frac": round(link_bytes / (ms_cold * 1e6) / h2d, 4)},
+                   host_link={"h2d_copy_gbs": round(h2d, 2), "zero_copy_read_gbs": round(zc, 2)},
+                   roofline=roof, kernels=rows)
+    else:  # trace_nvfp4: 43 layers, Markov routing realised as a per-token bias
+        L = wl.L
+        steps = min(wl.steps, int(os.environ.get("FT_TRACE_STEPS", wl.steps)))
+        h = Harness(wl, max_tokens=1, device=local)
+        traces = [ftgen.markov_trace(steps, 1, wl.E, wl.k, wl.extra["p_reuse"], wl.extra["zipf_s"],
+                                     wl.seed("trace", rank, l)) for l in range(L)]
+        zb = [ftgen.zipf_log_bias(wl.E, wl.extra["zipf_s"], wl.seed("pi", l)) for l in range(L)]
+        xs = [[ftgen.hidden(1, wl.d, wl.wtype, wl.seed("x", rank, st, l)).to(device) for l in range(L)]
+              for st in range(steps)]
+        bs = [[torch.as_tensor(ftgen.trace_bias(traces[l][st], zb[l], wl.extra["beta"])).to(device)
+               for l in range(L)] for st in range(steps)]
+        y = torch.empty(1, wl.d, dtype=torch.bfloat16, device=device)
+
+        def trace():
+            ft.ft_moe_reset_cache(h.ctx)
+            for st in range(steps):
+                for l in range(L):
+                    ft.ft_moe_layer_forward(h.ctx, l, ft.FT_DECODE, xs[st][l], 1, bs[st][l], 1, y)
+        trace()
+        ms = _timed(h.stream, device, trace, 1)
+        stt = h.stats()
+        ft.ft_moe_profile(h.ctx, True)
+        trace()
+        prof = ft.ft_moe_profile_read(h.ctx)
+        ft.ft_moe_profile(h.ctx, False)
+        h2d, zc = ft.ft_moe_probe_link(h.ctx, 1 << 30)
+        roof, rows = roofline(prof, peaks, peak_kind, h2d)
+        h.close()
+        out.update(value=round(steps / (ms / 1e3), 2), ms_per_step=round(ms / steps, 4), dtype="nvfp4",
+                   config={"workload": f"43-layer NVFP4 decode trace, batch 1, {steps} steps, Markov p=0.8 + "
+                                       "Zipf(1.1), shared LRU at 37% (4072 slots), 52.7:77.3"},
+                   tokens_per_s_43_layers=round(steps / (ms / 1e3), 2),
+                   layer_calls_per_s=round(steps * L / (ms / 1e3), 1),
+                   miss_rate=round(stt["misses"] / max(stt["lookups"], 1), 4),
+                   cache={k: stt[k] for k in ("lookups", "hits", "misses", "staged", "streamed")},
+                   host_link={"h2d_copy_gbs": round(h2d, 2), "zero_copy_read_gbs": round(zc, 2)},
+                   roofline=roof, kernels=rows)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    return 0
+
 # --------------------------------------------------------------------------
 def main():
     ap = argparse.ArgumentParser()
@@ -329,9 +427,11 @@ def main():
 
     import ftgen
     wl = ftgen.workload(args.workload)
-    if args.workload != "decode_bf16":
-        raise SystemExit("bench.py times the single-layer BF16 decode workload (decode_bf16)")
     world, rank, local = dist_setup(args.gpus)
+    if args.workload in ("prefill_bf16", "trace_nvfp4") and args.impl == "ours":
+        return run_secondary(args, wl, world, rank, local)
+    if args.workload != "decode_bf16":
+        raise SystemExit("workloads: decode_bf16 (default), prefill_bf16, trace_nvfp4")
     if args.impl == "reference":
         r = run_reference(args, wl, world, rank)
         if world > 1:
