@@ -33,8 +33,8 @@ void launch_prefill_gather(const Shape& sh, const void* x, int T, DevState& ds, 
 bool gemv_mma_supported(const Shape& sh);
 cudaError_t gemv_mma_init(int device);
 void launch_to_f16(const void* x, int n, void* y, cudaStream_t st);
-void launch_gemv_mma(const Shape& sh, int cls, int phase, int layer, const void* x16, int T, DevState& ds,
-                     int max_items, int max_tok, cudaStream_t st);
+void launch_gemv_mma(const Shape& sh, int cls, int layer, const void* x16, int T, DevState& ds, int max_items,
+                     int max_tok, cudaStream_t st);
 void launch_gemm_tc(const Shape& sh, int phase, int T, DevState& ds, cudaStream_t st);
 }  // namespace ft
 
@@ -142,7 +142,7 @@ void free_all(ft_ctx* c) {
   DevState& d = c->ds;
   void* dev_ptrs[] = {d.slot_of, d.key_of, d.stamp, d.clk, d.ctr, d.error, d.work, d.scores, d.ids, d.wts,
                       d.counts, d.offsets, d.perm, d.inv, d.hbuf, d.ybuf, d.xs, d.hs, d.tscale, d.slots,
-                      d.h16, d.h16lo, d.x16, c->probe_sink};
+                      d.h16, d.h16lo, d.x16, d.sched, c->probe_sink};
   for (void* p : dev_ptrs)
     if (p) cudaFree(p);
   for (uint8_t* p : c->pool_host)
@@ -191,12 +191,14 @@ ft_status check_device_error(ft_ctx* c) {
 
 enum ProfName {
   P_ROUTER, P_TOPK, P_PERMUTE, P_LOOKUP, P_GU_HIT, P_DN_HIT, P_GU_STAGED, P_DN_STAGED, P_GU_STREAM, P_DN_STREAM,
-  P_COMBINE, P_STAGE_COPY, P_PREFILL_WORK, P_GATHER, P_GEMM_GU, P_GEMM_DN, P_COUNT
+  P_COMBINE, P_STAGE_COPY, P_PREFILL_WORK, P_GATHER, P_GEMM_GU, P_GEMM_DN, P_GEMV_HIT, P_GEMV_STAGED,
+  P_GEMV_STREAM, P_TO_F16, P_COUNT
 };
 const char* const kProfNames[P_COUNT] = {
     "router_scores", "topk_softmax", "permute", "lookup", "gemv_gateup_hit", "gemv_down_hit",
     "gemv_gateup_staged", "gemv_down_staged", "gemv_gateup_streamed", "gemv_down_streamed", "combine",
-    "h2d_stage_copies", "prefill_work", "prefill_gather", "gemm_tc_gateup", "gemm_tc_down"};
+    "h2d_stage_copies", "prefill_work", "prefill_gather", "gemm_tc_gateup", "gemm_tc_down", "gemv_hit",
+    "gemv_staged", "gemv_streamed", "to_f16"};
 
 cudaEvent_t pooled_event(ft_ctx* c) {
   if (!c->evpool.empty()) {
@@ -355,6 +357,9 @@ ft_status ft_moe_init(const ft_config* cfg, void* compute_stream, void* copy_str
       TRY(cuda_try(cudaMalloc((void**)&d.x16, sizeof(uint16_t) * (size_t)cfg->max_tokens * sh.d)));
     TRY(cuda_try(gemv_mma_init(cfg->device)));
   }
+  d.sched_chunks = sh.E + (int)((Tk + MMA_CHUNK - 1) / MMA_CHUNK) + 1;
+  TRY(cuda_try(cudaMalloc((void**)&d.sched, sizeof(int32_t) * (N_CLASSES + (size_t)N_CLASSES * d.sched_chunks))));
+  TRY(cuda_try(cudaMemset(d.sched, 0, sizeof(int32_t) * (N_CLASSES + (size_t)N_CLASSES * d.sched_chunks))));
   c->use_tc = prefill_tc_supported(sh) && sh.C >= 2ll * sh.E;
   if (c->use_tc) {
     TRY(cuda_try(cudaMalloc((void**)&d.xs, sizeof(__nv_bfloat16) * (Tk + 256) * sh.d)));
@@ -418,14 +423,42 @@ ft_status ft_moe_reset_cache(ft_ctx* c) {
   return reset_state(c);
 }
 
-// One phase of the decode grouped GEMV for one work class.
-static void gemv(ft_ctx* c, int cls, int phase, int layer, const void* x, int T, int max_items, int Tk,
-                 cudaStream_t st) {
-  if (c->use_mma)
-    launch_gemv_mma(c->sh, cls, phase, layer, c->sh.wtype == FT_W_NVFP4 ? (const void*)c->ds.x16 : x, T, c->ds,
-                    max_items, Tk, st);
-  else
-    launch_expert_gemv(c->sh, cls, phase, layer, x, T, c->ds, max_items, Tk, st);
+// The experts of one work class: one fused tensor-core launch (BF16 /
+// NVFP4), or the two SIMT phases (fp32). pr receives the profile records.
+static void gemv_class(ft_ctx* c, int cls, int layer, const void* x, int T, int max_items, int Tk, cudaStream_t st,
+                       int (&pr)[2]) {
+  static const int fused[3] = {P_GEMV_HIT, P_GEMV_STAGED, P_GEMV_STREAM};
+  static const int gu[3] = {P_GU_HIT, P_GU_STAGED, P_GU_STREAM};
+  static const int dn[3] = {P_DN_HIT, P_DN_STAGED, P_DN_STREAM};
+  if (c->use_mma) {
+    pr[0] = prof_begin(c, fused[cls], st);
+    launch_gemv_mma(c->sh, cls, layer, c->sh.wtype == FT_W_NVFP4 ? (const void*)c->ds.x16 : x, T, c->ds, max_items, Tk,
+                    st);
+    prof_end(c, pr[0], st);
+    pr[1] = -1;
+    c->kernel_launches += 1;
+  } else {
+    for (int ph = 0; ph < 2; ++ph) {
+      pr[ph] = prof_begin(c, ph == 0 ? gu[cls] : dn[cls], st);
+      launch_expert_gemv(c->sh, cls, ph, layer, x, T, c->ds, max_items, Tk, st);
+      prof_end(c, pr[ph], st);
+    }
+    c->kernel_launches += 2;
+  }
+}
+
+// Algorithmic bytes / flops of a class's launches, once its size is known.
+static void gemv_class_cost(ft_ctx* c, const int (&pr)[2], int n_items, int n_tok) {
+  if (!c->profiling) return;
+  double b0, f0, b1, f1;
+  gemv_cost(c->sh, 0, n_items, n_tok, b0, f0);
+  gemv_cost(c->sh, 1, n_items, n_tok, b1, f1);
+  if (pr[1] < 0) {
+    prof_bytes(c, pr[0], b0 + b1, f0 + f1);
+  } else {
+    prof_bytes(c, pr[0], b0, f0);
+    prof_bytes(c, pr[1], b1, f1);
+  }
 }
 
 static ft_status issue_copies(ft_ctx* c, int from, int to) {
@@ -495,21 +528,10 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
     prof_end(c, p, cs);
     CK(cudaEventRecord(c->ev_look, cs));
     CK(cudaStreamWaitEvent(c->s_side, c->ev_look, 0));
-    int pr[6];  // gate/up and down of the streamed, hit, staged classes
-    pr[0] = prof_begin(c, P_GU_STREAM, c->s_side);
-    gemv(c, KIND_STREAMED, 0, layer, x, T, max_items, Tk, c->s_side);
-    prof_end(c, pr[0], c->s_side);
-    pr[1] = prof_begin(c, P_DN_STREAM, c->s_side);
-    gemv(c, KIND_STREAMED, 1, layer, x, T, max_items, Tk, c->s_side);
-    prof_end(c, pr[1], c->s_side);
+    int pr_stream[2], pr_hit[2], pr_staged[2];
+    gemv_class(c, KIND_STREAMED, layer, x, T, max_items, Tk, c->s_side, pr_stream);
     CK(cudaEventRecord(c->ev_side, c->s_side));
-    pr[2] = prof_begin(c, P_GU_HIT, cs);
-    gemv(c, KIND_HIT, 0, layer, x, T, max_items, Tk, cs);
-    prof_end(c, pr[2], cs);
-    pr[3] = prof_begin(c, P_DN_HIT, cs);
-    gemv(c, KIND_HIT, 1, layer, x, T, max_items, Tk, cs);
-    prof_end(c, pr[3], cs);
-    c->kernel_launches += 5;
+    gemv_class(c, KIND_HIT, layer, x, T, max_items, Tk, cs, pr_hit);
     st = wait_event(c->ev_look, WAIT_S);
     if (st != FT_OK) return c->latched = st;
     if (check_device_error(c) != FT_OK) return c->latched;
@@ -518,17 +540,8 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
     c->last_m = mb->m;
     c->last_qstar = mb->qstar;
     c->last_qstage = mb->qstage;
-    if (c->profiling) {
-      double b, f;
-      gemv_cost(sh, 0, mb->n_streamed_cls, mb->n_tok_cls[KIND_STREAMED], b, f);
-      prof_bytes(c, pr[0], b, f);
-      gemv_cost(sh, 1, mb->n_streamed_cls, mb->n_tok_cls[KIND_STREAMED], b, f);
-      prof_bytes(c, pr[1], b, f);
-      gemv_cost(sh, 0, mb->n_hit_cls, mb->n_tok_cls[KIND_HIT], b, f);
-      prof_bytes(c, pr[2], b, f);
-      gemv_cost(sh, 1, mb->n_hit_cls, mb->n_tok_cls[KIND_HIT], b, f);
-      prof_bytes(c, pr[3], b, f);
-    }
+    gemv_class_cost(c, pr_stream, mb->n_streamed_cls, mb->n_tok_cls[KIND_STREAMED]);
+    gemv_class_cost(c, pr_hit, mb->n_hit_cls, mb->n_tok_cls[KIND_HIT]);
     if (n_copy > 0) {
       p = prof_begin(c, P_STAGE_COPY, c->s_copy, n_copy * (double)sh.slot_bytes);
       st = issue_copies(c, 0, n_copy);
@@ -536,14 +549,8 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
       if (st != FT_OK) return c->latched = st;
       CK(cudaEventRecord(c->ev_copy, c->s_copy));
       CK(cudaStreamWaitEvent(cs, c->ev_copy, 0));
-      double b = 0, f = 0;
-      for (int ph = 0; ph < 2; ++ph) {
-        gemv_cost(sh, ph, mb->n_staged_cls, mb->n_tok_cls[KIND_STAGED], b, f);
-        pr[4 + ph] = prof_begin(c, ph == 0 ? P_GU_STAGED : P_DN_STAGED, cs, b, f);
-        gemv(c, KIND_STAGED, ph, layer, x, T, max_items, Tk, cs);
-        prof_end(c, pr[4 + ph], cs);
-      }
-      c->kernel_launches += 2;
+      gemv_class(c, KIND_STAGED, layer, x, T, max_items, Tk, cs, pr_staged);
+      gemv_class_cost(c, pr_staged, mb->n_staged_cls, mb->n_tok_cls[KIND_STAGED]);
     }
     CK(cudaStreamWaitEvent(cs, c->ev_side, 0));
     c->prefetched = -1;
@@ -632,16 +639,9 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
         launch_to_f16(x, T * sh.d, d.x16, cs);
         c->kernel_launches += 1;
       }
-      int n_items = 0;
-      for (int ph = 0; ph < 2; ++ph) {
-        double b = 0, f = 0;
-        gemv_cost(sh, ph, sh.E, Tk, b, f);  // upper bound: every expert routed
-        (void)n_items;
-        p = prof_begin(c, ph == 0 ? P_GU_HIT : P_DN_HIT, cs, b, f);
-        gemv(c, KIND_HIT, ph, layer, x, T, max_items, Tk, cs);
-        prof_end(c, p, cs);
-      }
-      c->kernel_launches += 2;
+      int pr[2];
+      gemv_class(c, KIND_HIT, layer, x, T, max_items, Tk, cs, pr);
+      gemv_class_cost(c, pr, max_items, Tk);  // upper bound: every routed expert
     }
   }
   p = prof_begin(c, P_COMBINE, cs, Tk * (double)sh.d * 4.0 + T * (double)sh.d * ab + Tk * 8.0);

@@ -24,7 +24,8 @@ enum DevError : uint32_t { DERR_NONE = 0, DERR_NO_VICTIM = 1, DERR_BAD_INDEX = 2
 
 constexpr int MAX_E = 512;
 constexpr int MAX_K = 16;
-constexpr int TOK_CHUNK = 8;  // tokens one decode GEMV pass carries
+constexpr int TOK_CHUNK = 8;   // tokens one SIMT GEMV pass carries
+constexpr int MMA_CHUNK = 16;  // tokens one tensor-core GEMV unit carries
 
 // One routed expert of the current call, in ascending expert order inside
 // its class. tok_off / n_tok index the sorted (perm) order.
@@ -120,6 +121,8 @@ struct DevState {
   uint8_t* slots;            // HBM slot pool [C * slot_bytes]
   const uint8_t* pool_dev;   // device address of the called layer's blobs in the mapped host pool
   void* tc_plan;             // host: tensor maps of the prefill GEMM (owned, see prefill_tc_free)
+  int32_t* sched;            // [N_CLASSES] unit tickets + [N_CLASSES][sched_chunks] chunk completion counters
+  int sched_chunks;
 };
 
 // ---- launchers (all enqueue on `st`) ----

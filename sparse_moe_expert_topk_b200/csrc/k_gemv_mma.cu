@@ -1,29 +1,38 @@
 // Decode grouped GEMV for BF16 and NVFP4 experts on warp-level tensor-core
-// MMAs (mma.sync m16n8k16, fp32 accumulate), weights streamed straight from
-// HBM slots or from the mapped host pool with 128-bit loads.
+// MMAs (mma.sync m16n8k16, fp32 accumulate): gate/up + SwiGLU and down in one
+// persistent launch per work class, weights streamed with 128-bit loads from
+// HBM slots or straight from the mapped host pool.
 //
 // Small-batch decode is memory bound ([paperlens] "壁2: デコードのミスを「どう捌く
 // か」が決まっていない", paper §2.2): every weight byte is read once, so the
-// kernel's job is to keep enough loads in flight and spend few instructions
-// per byte. A warp owns 16 weight rows and one chunk of up to 16 tokens; each
-// lane loads 16 consecutive bytes of two rows (g and g+8, g = lane / 4) and
-// hands them to the MMA unchanged as its A fragment. That assigns the K
-// positions of the MMA in a lane-dependent order, which is harmless for a dot
-// product as long as the activations use the same order: each lane loads the
-// 16 matching bytes of its token's row as the B fragment. No shuffles, no
-// shared memory; the accumulation order is fixed by the code, so an expert's
-// result does not depend on where its weights were read from ([paperlens]
-// "設計: 2階建てのエキスパート記憶", paper §3.3).
+// kernel keeps many loads in flight and spends few instructions per byte.
 //
-// Gate/up phase: rows 0..7 of the MMA tile are gate rows f0..f0+7 and rows
-// 8..15 the matching up rows, so each lane holds gate and up of the same
-// (feature, token) pairs and applies SwiGLU in registers; h is written as a
-// 16-bit activation for the down phase: f16 for NVFP4 experts, and for BF16
-// experts as two bf16 parts hi + lo (both multiplied by W_down), which keeps h
-// to about 2^-16 relative -- a single bf16 rounding of h would spend most of
-// the 2e-2 rms error budget that the bf16 output rounding leaves.
+// Work unit: 16 weight rows x one chunk of <= 16 tokens of one expert, done
+// by one CTA of 8 warps that split the unit's K range (split-K) and reduce
+// their partial sums in warp order through shared memory. Inside a warp,
+// lane (g, q) = (lane/4, lane%4) loads 16 consecutive bytes of rows g and
+// g+8 per step and hands them to the MMA unchanged as its A fragment; that
+// fixes a lane-dependent order of the K positions, which a dot product does
+// not care about as long as the activations (B fragment) are loaded in the
+// same order. No shuffles, and the summation order is fixed by the code, so an
+// expert's result does not depend on where its weights were read from
+// ([paperlens] "設計: 2階建てのエキスパート記憶", paper §3.3).
+//
+// Phase 0 units (gate/up): tile rows 0..7 are gate rows f0..f0+7 and rows
+// 8..15 the matching up rows, so one lane holds gate and up of the same
+// (feature, token) pairs and applies SwiGLU in registers. h goes to memory as
+// f16 (NVFP4 experts) or as bf16 hi + lo parts (BF16 experts: both parts are
+// multiplied by W_down, keeping h to ~2^-16; one bf16 rounding of h would eat
+// most of the 2e-2 rms budget that the bf16 output rounding leaves).
+// Phase 1 units (down) of an (expert, chunk) start once all its phase-0 units
+// have published h: units are handed out in ticket order (gate/up tickets
+// first) and a down unit waits, bounded, on a per-chunk completion counter.
+// Tickets are only taken by running CTAs, so every unit a CTA waits for is
+// held by a running CTA that never waits itself: no deadlock whatever the
+// residency.
+//
 // NVFP4: 32 e2m1 codes per lane are converted to f16 pairs (cvt e2m1x2) and
-// multiplied by their e4m3 block scale (exact in f16), the per-matrix fp32
+// multiplied by their e4m3 block scale (exact in f16); the per-matrix fp32
 // tensor scale is applied to the fp32 result.
 #include <cuda_fp16.h>
 
@@ -34,12 +43,21 @@ namespace ft {
 namespace {
 
 constexpr int WARPS = 8;
+constexpr int CHUNK = 16;  // tokens per unit (two n8 tiles)
+constexpr long long WAIT_CYCLES = 4000000000ll;  // ~2 s
 
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
   uint4 r;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
                : "l"(p));
+  return r;
+}
+
+// L2-coherent load (for h, written by other CTAs of the same launch).
+__device__ __forceinline__ uint4 ld_cg(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
   return r;
 }
 
@@ -82,44 +100,6 @@ __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
   return *reinterpret_cast<uint32_t*>(&r);
 }
 
-struct MmaArgs {
-  const WorkLists* work;
-  int cls, layer, E, k, d, d_ff, nvfp4;
-  long long C;
-  size_t slot_bytes;
-  const uint8_t* slots;
-  const uint8_t* pool;
-  const void* x;        // [T, d] bf16 activations (BF16) or f16 copy (NVFP4)
-  const int32_t* perm;
-  const float* tscale;  // [L*E*3]
-  uint16_t* h16;        // [T*k, d_ff] bf16 (BF16) or f16 (NVFP4) SwiGLU output
-  uint16_t* h16lo;      // [T*k, d_ff] BF16 experts: bf16 residual h - h16 (h = hi + lo to ~2^-16)
-  float* ybuf;          // [T*k, d]
-};
-
-__device__ __forceinline__ const uint8_t* blob_of(const MmaArgs& a, const WorkItem& it) {
-  if (a.cls == KIND_STREAMED) return a.pool + (size_t)it.e * a.slot_bytes;
-  return a.slots + (size_t)it.slot * a.slot_bytes;
-}
-
-// One BF16 step: 8 K values of rows g and g+8 per lane, two MMAs per token
-// tile (and two more for the low part of h in the down phase).
-template <int NB, bool LO>
-__device__ __forceinline__ void bf16_step(const uint4 wa, const uint4 wb, const uint16_t* const (&xr)[NB],
-                                          const uint16_t* const (&xl)[NB], int e0, float (&acc)[NB][4]) {
-#pragma unroll
-  for (int t = 0; t < NB; ++t) {
-    const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xr[t] + e0));
-    mma_bf16(acc[t], wa.x, wb.x, wa.y, wb.y, xv.x, xv.y);
-    mma_bf16(acc[t], wa.z, wb.z, wa.w, wb.w, xv.z, xv.w);
-    if constexpr (LO) {
-      const uint4 xo = __ldg(reinterpret_cast<const uint4*>(xl[t] + e0));
-      mma_bf16(acc[t], wa.x, wb.x, wa.y, wb.y, xo.x, xo.y);
-      mma_bf16(acc[t], wa.z, wb.z, wa.w, wb.w, xo.z, xo.w);
-    }
-  }
-}
-
 // 16 code bytes (32 e2m1 values) and their two e4m3 scales -> 16 f16 pairs.
 __device__ __forceinline__ void decode_nvfp4(const uint4 w, uint32_t sc, uint32_t (&h)[16]) {
   e2m1x8_to_f16x8(w.x, *reinterpret_cast<uint32_t(*)[4]>(&h[0]));
@@ -136,82 +116,84 @@ __device__ __forceinline__ void decode_nvfp4(const uint4 w, uint32_t sc, uint32_
   for (int j = 8; j < 16; ++j) h[j] = hmul2(h[j], shi);
 }
 
-// Where a warp's two weight rows come from: straight from global memory
-// (HBM slots: 128-bit non-caching loads) or from the warp's shared-memory
-// tile, filled beforehand with cp.async (streamed experts: each warp
-// instruction reads a contiguous run of a row, which the host link moves in
-// large requests). Both hand the MMAs the same 16-byte vectors in the same
-// order, so the arithmetic does not depend on the source.
-template <bool STAGED>
-struct RowSrc {
-  const uint8_t* ga;  // global row g (+ q*16), direct mode
-  const uint8_t* gb;  // global row g+8 (+ q*16)
-  const uint8_t* ta;  // smem row g of this warp's tile (+ q*16), staged mode
-  const uint8_t* tb;
-  int s0;             // first step of this warp
-  __device__ __forceinline__ uint4 a(int s) const {
-    if constexpr (STAGED) return *reinterpret_cast<const uint4*>(ta + (s - s0) * 64);
-    else return ld_stream(ga + (size_t)s * 64);
-  }
-  __device__ __forceinline__ uint4 b(int s) const {
-    if constexpr (STAGED) return *reinterpret_cast<const uint4*>(tb + (s - s0) * 64);
-    else return ld_stream(gb + (size_t)s * 64);
-  }
+struct MmaArgs {
+  const WorkLists* work;
+  int cls, layer, E, k, d, d_ff;
+  long long C;
+  size_t slot_bytes;
+  const uint8_t* slots;
+  const uint8_t* pool;
+  const void* x;        // [T, d] bf16 activations (BF16) or f16 copy (NVFP4)
+  const int32_t* perm;
+  const float* tscale;  // [L*E*3]
+  uint16_t* h16;        // [T*k, d_ff] bf16 (BF16) or f16 (NVFP4) SwiGLU output
+  uint16_t* h16lo;      // [T*k, d_ff] BF16 experts: bf16 residual h - h16
+  float* ybuf;          // [T*k, d]
+  int32_t* ticket;      // this class's unit ticket counter (zeroed by the lookup)
+  int32_t* done;        // this class's per-(item, chunk) phase-0 completion counters (zeroed)
+  uint32_t* error;
 };
 
-// Scale pair (two e4m3 bytes) of step s for rows g and g+8 (NVFP4).
-template <bool STAGED>
-struct ScaleSrc {
-  const unsigned short* ga;  // global scale row g (+ q)
-  const unsigned short* gb;
-  const unsigned short* ta;  // smem scale row g (+ q)
-  const unsigned short* tb;
-  int s0;
-  __device__ __forceinline__ uint32_t a(int s) const {
-    if constexpr (STAGED) return ta[(s - s0) * 4];
-    else return __ldg(ga + s * 4);
+__device__ __forceinline__ const uint8_t* blob_of(const MmaArgs& a, const WorkItem& it) {
+  if (a.cls == KIND_STREAMED) return a.pool + (size_t)it.e * a.slot_bytes;
+  return a.slots + (size_t)it.slot * a.slot_bytes;
+}
+
+// One BF16 step: 8 K values of rows g and g+8 per lane, two MMAs per token
+// tile (and two more for the low part of h in phase 1).
+template <int NB, bool P1>
+__device__ __forceinline__ void bf16_step(const uint4 wa, const uint4 wb, const uint16_t* const (&xr)[NB],
+                                          const uint16_t* const (&xl)[NB], int e0, float (&acc)[NB][4]) {
+#pragma unroll
+  for (int t = 0; t < NB; ++t) {
+    const uint4 xv = P1 ? ld_cg(xr[t] + e0) : __ldg(reinterpret_cast<const uint4*>(xr[t] + e0));
+    mma_bf16(acc[t], wa.x, wb.x, wa.y, wb.y, xv.x, xv.y);
+    mma_bf16(acc[t], wa.z, wb.z, wa.w, wb.w, xv.z, xv.w);
+    if constexpr (P1) {
+      const uint4 xo = ld_cg(xl[t] + e0);
+      mma_bf16(acc[t], wa.x, wb.x, wa.y, wb.y, xo.x, xo.y);
+      mma_bf16(acc[t], wa.z, wb.z, wa.w, wb.w, xo.z, xo.w);
+    }
   }
-  __device__ __forceinline__ uint32_t b(int s) const {
-    if constexpr (STAGED) return tb[(s - s0) * 4];
-    else return __ldg(gb + s * 4);
-  }
-};
+}
 
 // acc[t][.] += W[rows g, g+8] . X[tokens] over steps [s0, s1) of 32 K values
-// (BF16: lane q covers K = 32 s + 8 q .. +8). U steps of loads in flight;
-// steps past s1 reload the last step (its result is not used).
-template <int NB, int U, bool LO, class Src>
-__device__ __forceinline__ void dot_bf16(const Src& src, int s0, int s1, const uint16_t* const (&xr)[NB],
-                                         const uint16_t* const (&xl)[NB], int q, float (&acc)[NB][4]) {
+// (lane q covers K = 32 s + 8 q .. +8). U steps of loads in flight; steps past
+// s1 reload the last step and are not used.
+template <int NB, int U, bool P1>
+__device__ __forceinline__ void dot_bf16(const uint8_t* ra, const uint8_t* rb, int s0, int s1,
+                                         const uint16_t* const (&xr)[NB], const uint16_t* const (&xl)[NB], int q,
+                                         float (&acc)[NB][4]) {
   for (int s = s0; s < s1; s += U) {
     uint4 wa[U], wb[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int ss = s + u < s1 ? s + u : s1 - 1;
-      wa[u] = src.a(ss);
-      wb[u] = src.b(ss);
+      wa[u] = ld_stream(ra + (size_t)ss * 64);
+      wb[u] = ld_stream(rb + (size_t)ss * 64);
     }
 #pragma unroll
     for (int u = 0; u < U; ++u)
-      if (s + u < s1) bf16_step<NB, LO>(wa[u], wb[u], xr, xl, (s + u) * 32 + q * 8, acc);
+      if (s + u < s1) bf16_step<NB, P1>(wa[u], wb[u], xr, xl, (s + u) * 32 + q * 8, acc);
   }
 }
 
 // NVFP4: steps of 128 K values (lane q covers K = 128 s + 32 q .. +32: 16
-// code bytes and one scale pair per row); eight MMAs per step.
-template <int NB, int U, class Src, class Sc>
-__device__ __forceinline__ void dot_nvfp4(const Src& src, const Sc& sc, int s0, int s1,
-                                          const uint16_t* const (&xr)[NB], int q, float (&acc)[NB][4]) {
+// code bytes and one scale pair per row); eight MMAs per step and token tile.
+template <int NB, int U, bool P1>
+__device__ __forceinline__ void dot_nvfp4(const uint8_t* ra, const uint8_t* rb, const unsigned short* sa,
+                                          const unsigned short* sb, int s0, int s1, const uint16_t* const (&xr)[NB],
+                                          int q, float (&acc)[NB][4]) {
   for (int s = s0; s < s1; s += U) {
     uint4 wa[U], wb[U];
     uint32_t ca[U], cb[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int ss = s + u < s1 ? s + u : s1 - 1;
-      wa[u] = src.a(ss);
-      wb[u] = src.b(ss);
-      ca[u] = sc.a(ss);
-      cb[u] = sc.b(ss);
+      wa[u] = ld_stream(ra + (size_t)ss * 64);
+      wb[u] = ld_stream(rb + (size_t)ss * 64);
+      ca[u] = __ldg(sa + ss * 4);
+      cb[u] = __ldg(sb + ss * 4);
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -221,11 +203,11 @@ __device__ __forceinline__ void dot_nvfp4(const Src& src, const Sc& sc, int s0, 
         decode_nvfp4(wb[u], cb[u], hb);
 #pragma unroll
         for (int t = 0; t < NB; ++t) {
-          const uint4* xp = reinterpret_cast<const uint4*>(xr[t] + (s + u) * 128 + q * 32);
+          const uint16_t* xp = xr[t] + (s + u) * 128 + q * 32;
           uint32_t xh[16];
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
-            const uint4 xv = __ldg(xp + v);
+            const uint4 xv = P1 ? ld_cg(xp + 8 * v) : __ldg(reinterpret_cast<const uint4*>(xp) + v);
             xh[4 * v] = xv.x;
             xh[4 * v + 1] = xv.y;
             xh[4 * v + 2] = xv.z;
@@ -240,21 +222,11 @@ __device__ __forceinline__ void dot_nvfp4(const Src& src, const Sc& sc, int s0, 
   }
 }
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
-               "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async8(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-
-// Map CTA-unit u of this class to (item, 16-token chunk, 16-row block).
+// Map a unit index within a phase to (item, 16-token chunk, row block) and
+// the item-chunk index qi.
 __device__ __forceinline__ bool unit_of(const int* pref, int n_items, int rblocks, int u, int& item, int& chunk,
-                                        int& rb) {
-  const int qi = u / rblocks;
+                                        int& rb, int& qi) {
+  qi = u / rblocks;
   rb = u - qi * rblocks;
   if (qi >= pref[n_items]) return false;
   int lo = 0, hi = n_items - 1;
@@ -267,23 +239,10 @@ __device__ __forceinline__ bool unit_of(const int* pref, int n_items, int rblock
   return true;
 }
 
-constexpr int CHUNK = 16;  // tokens per unit (two n8 tiles)
-
-// Per-warp tile geometry of the staged mode (bytes per row, padded so the
-// 8 rows a warp's lanes read at once fall in distinct bank groups).
-__host__ __device__ __forceinline__ int tile_row_bytes(int steps_w) { return steps_w * 64 + 16; }
-__host__ __device__ __forceinline__ int tile_scale_bytes(int steps_w) { return steps_w * 8 + 16; }
-__host__ __device__ __forceinline__ int max_steps_per_warp(int steps) { return (steps + WARPS - 1) / WARPS; }
-__host__ __device__ __forceinline__ int warp_tile_bytes(int steps, bool fp4) {
-  const int sw = max_steps_per_warp(steps);
-  return 16 * tile_row_bytes(sw) + (fp4 ? 16 * tile_scale_bytes(sw) : 0);
-}
-
-// One CTA-unit: 16 weight rows x one chunk of <= 16 tokens, the K range split
-// over the 8 warps, partial sums reduced in warp order, epilogue by warp 0.
-template <int NB, int PHASE, bool FP4, bool STAGED>
-__device__ void unit_work(const MmaArgs& a, const WorkItem& it, int chunk, int rb, int warp, int lane,
-                          uint8_t* tiles, float* red) {
+// One unit: 16 weight rows x one chunk of <= 16 tokens, the K range split over
+// the 8 warps, partial sums reduced in warp order, epilogue by warp 0.
+template <int NB, int PHASE, bool FP4>
+__device__ void unit_work(const MmaArgs& a, const WorkItem& it, int chunk, int rb, int warp, int lane, float* red) {
   const int g = lane >> 2, q = lane & 3;
   const uint8_t* blob = blob_of(a, it);
   const size_t n = (size_t)a.d * a.d_ff;
@@ -292,43 +251,19 @@ __device__ void unit_work(const MmaArgs& a, const WorkItem& it, int chunk, int r
   const size_t sbytes = (size_t)K / 16;
   const int steps = FP4 ? K / 128 : K / 32;
   const int s0 = (warp * steps) / WARPS, s1 = ((warp + 1) * steps) / WARPS;
-  // rows 0..7 / 8..15 of the tile: gate / up rows rb*8.. (phase 0), down rows rb*16.. (phase 1)
-  auto row_ptr = [&](int r) -> const uint8_t* {
-    if (PHASE == 0) return blob + (r < 8 ? 0 : (FP4 ? n / 2 : n * 2)) + (size_t)(rb * 8 + (r & 7)) * rbytes;
-    return blob + (FP4 ? n : n * 4) + (size_t)(rb * 16 + r) * rbytes;
-  };
-  auto scale_ptr = [&](int r) -> const uint8_t* {
-    const size_t base = 3 * (n / 2);
-    if (PHASE == 0) return blob + base + (r < 8 ? 0 : n / 16) + (size_t)(rb * 8 + (r & 7)) * sbytes;
-    return blob + base + 2 * (n / 16) + (size_t)(rb * 16 + r) * sbytes;
-  };
-  const int sw = max_steps_per_warp(steps);
-  uint8_t* tile = tiles + (size_t)warp * warp_tile_bytes(steps, FP4);
-  const int trow = tile_row_bytes(sw), tsrow = tile_scale_bytes(sw);
-  if (STAGED && s1 > s0) {
-    // contiguous per-row runs: flattened (row, byte) index, 16 bytes per lane
-    const int nb = (s1 - s0) * 64;
-    for (int e = lane * 16; e < 16 * nb; e += 512) {
-      const int r = e / nb, off = e - r * nb;
-      cp_async16(tile + r * trow + off, row_ptr(r) + (size_t)s0 * 64 + off);
-    }
-    if (FP4) {
-      const int ns = (s1 - s0) * 8;
-      uint8_t* st = tile + 16 * trow;
-      for (int e = lane * 8; e < 16 * ns; e += 256) {
-        const int r = e / ns, off = e - r * ns;
-        cp_async8(st + r * tsrow + off, scale_ptr(r) + (size_t)s0 * 8 + off);
-      }
-    }
-    cp_async_wait_all();
-    __syncwarp();
+  // rows g / g+8 of the tile: gate / up row rb*8+g (phase 0); down rows rb*16+g, +8 (phase 1)
+  size_t oa, ob, sa0, sb0;
+  if (PHASE == 0) {
+    oa = (size_t)(rb * 8 + g) * rbytes;
+    ob = (FP4 ? n / 2 : n * 2) + (size_t)(rb * 8 + g) * rbytes;
+    sa0 = 3 * (n / 2) + (size_t)(rb * 8 + g) * sbytes;
+    sb0 = 3 * (n / 2) + n / 16 + (size_t)(rb * 8 + g) * sbytes;
+  } else {
+    oa = (FP4 ? n : n * 4) + (size_t)(rb * 16 + g) * rbytes;
+    ob = oa + 8 * rbytes;
+    sa0 = 3 * (n / 2) + 2 * (n / 16) + (size_t)(rb * 16 + g) * sbytes;
+    sb0 = sa0 + 8 * sbytes;
   }
-  RowSrc<STAGED> src;
-  src.ga = row_ptr(g) + q * 16;
-  src.gb = row_ptr(g + 8) + q * 16;
-  src.ta = tile + g * trow + q * 16;
-  src.tb = tile + (g + 8) * trow + q * 16;
-  src.s0 = s0;
   const int base = it.tok_off + chunk * CHUNK;
   const int nt = min(CHUNK, it.n_tok - chunk * CHUNK);
   const uint16_t* xr[NB];
@@ -342,23 +277,18 @@ __device__ void unit_work(const MmaArgs& a, const WorkItem& it, int chunk, int r
       xl[t] = xr[t];
     } else {
       xr[t] = a.h16 + (size_t)pos * a.d_ff;
-      xl[t] = a.h16lo + (size_t)pos * a.d_ff;
+      xl[t] = FP4 ? xr[t] : a.h16lo + (size_t)pos * a.d_ff;
     }
   }
   float acc[NB][4];
 #pragma unroll
   for (int t = 0; t < NB; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-  if constexpr (FP4) {
-    ScaleSrc<STAGED> sc;
-    sc.ga = reinterpret_cast<const unsigned short*>(scale_ptr(g)) + q;
-    sc.gb = reinterpret_cast<const unsigned short*>(scale_ptr(g + 8)) + q;
-    sc.ta = reinterpret_cast<const unsigned short*>(tile + 16 * trow + g * tsrow) + q;
-    sc.tb = reinterpret_cast<const unsigned short*>(tile + 16 * trow + (g + 8) * tsrow) + q;
-    sc.s0 = s0;
-    dot_nvfp4<NB, 4>(src, sc, s0, s1, xr, q, acc);
-  } else {
-    dot_bf16<NB, (NB == 1 ? 8 : 4), PHASE == 1>(src, s0, s1, xr, xl, q, acc);
-  }
+  if constexpr (FP4)
+    dot_nvfp4<NB, 4, PHASE == 1>(blob + oa + q * 16, blob + ob + q * 16,
+                                 reinterpret_cast<const unsigned short*>(blob + sa0) + q,
+                                 reinterpret_cast<const unsigned short*>(blob + sb0) + q, s0, s1, xr, q, acc);
+  else
+    dot_bf16<NB, (NB == 1 ? 8 : 4), PHASE == 1>(blob + oa + q * 16, blob + ob + q * 16, s0, s1, xr, xl, q, acc);
   // split-K reduction over the warps, in warp order
 #pragma unroll
   for (int t = 0; t < NB; ++t)
@@ -405,39 +335,72 @@ __device__ void unit_work(const MmaArgs& a, const WorkItem& it, int chunk, int r
         }
       }
     }
+    if (PHASE == 0) __threadfence();  // publish h before the unit is counted done
   }
-  __syncthreads();  // red and the tiles are reused by the next unit
+  __syncthreads();  // red is reused by the next unit
 }
 
-template <int NB, bool FP4, bool STAGED>
-__global__ void __launch_bounds__(WARPS * 32) gemv_mma_kernel(MmaArgs a, int phase) {
-  extern __shared__ __align__(16) uint8_t tiles[];
+template <int NB, bool FP4>
+__global__ void __launch_bounds__(WARPS * 32) gemv_fused_kernel(MmaArgs a) {
   __shared__ int s_pref[MAX_E + 1];
   __shared__ WorkItem s_items[MAX_E];
   __shared__ float red[WARPS * NB * 4 * 32];
+  __shared__ int s_unit;
   const int n_items = a.work->n_items[a.cls];
   if (n_items == 0) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int i = tid; i < n_items; i += blockDim.x) s_items[i] = a.work->items[a.cls][i];
   __syncthreads();
-  if (tid == 0) {
-    int p = 0;
-    for (int i = 0; i < n_items; ++i) {
-      s_pref[i] = p;
-      p += (s_items[i].n_tok + CHUNK - 1) / CHUNK;
+  if (warp == 0) {  // exclusive scan of the chunks per item
+    int carry = 0;
+    for (int b = 0; b < n_items; b += 32) {
+      const int i = b + lane;
+      const int c = i < n_items ? (s_items[i].n_tok + CHUNK - 1) / CHUNK : 0;
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (i < n_items) s_pref[i] = carry + incl - c;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    s_pref[n_items] = p;
+    if (lane == 0) s_pref[n_items] = carry;
   }
   __syncthreads();
-  const int rblocks = phase == 0 ? a.d_ff / 8 : a.d / 16;
-  const int n_units = s_pref[n_items] * rblocks;
-  for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-    int item, chunk, rb;
-    if (!unit_of(s_pref, n_items, rblocks, u, item, chunk, rb)) break;
+  const int n_qi = s_pref[n_items];
+  const int rb0 = a.d_ff / 8, rb1 = a.d / 16;
+  const int U0 = n_qi * rb0, U1 = n_qi * rb1;
+  for (;;) {
+    __syncthreads();  // every thread has read the previous ticket
+    if (tid == 0) s_unit = atomicAdd(a.ticket, 1);
+    __syncthreads();
+    const int u = s_unit;
+    if (u >= U0 + U1) break;
+    const int phase = u < U0 ? 0 : 1;
+    int item, chunk, rb, qi;
+    unit_of(s_pref, n_items, phase == 0 ? rb0 : rb1, phase == 0 ? u : u - U0, item, chunk, rb, qi);
     const WorkItem it = s_items[item];
-    if (a.cls != KIND_STREAMED && (it.slot < 0 || it.slot >= a.C)) continue;  // error already latched
-    if (phase == 0) unit_work<NB, 0, FP4, STAGED>(a, it, chunk, rb, warp, lane, tiles, red);
-    else unit_work<NB, 1, FP4, STAGED>(a, it, chunk, rb, warp, lane, tiles, red);
+    const bool bad = a.cls != KIND_STREAMED && (it.slot < 0 || it.slot >= a.C);  // error already latched
+    if (phase == 1) {
+      // wait until every gate/up unit of this (item, chunk) has published h
+      if (tid == 0) {
+        const long long t0 = clock64();
+        volatile int32_t* dn = a.done + qi;
+        while (*dn < rb0) {
+          if (clock64() - t0 > WAIT_CYCLES) {
+            atomicExch(a.error, (uint32_t)DERR_TIMEOUT);
+            break;
+          }
+        }
+        __threadfence();
+      }
+      __syncthreads();
+      if (!bad) unit_work<NB, 1, FP4>(a, it, chunk, rb, warp, lane, red);
+    } else {
+      if (!bad) unit_work<NB, 0, FP4>(a, it, chunk, rb, warp, lane, red);
+      if (tid == 0) atomicAdd(a.done + qi, 1);
+    }
   }
 }
 
@@ -446,8 +409,15 @@ __global__ void __launch_bounds__(256) to_f16_kernel(const __nv_bfloat16* __rest
   for (int i = blockIdx.x * 256 + threadIdx.x; i < n; i += gridDim.x * 256) y[i] = __float2half_rn(__bfloat162float(x[i]));
 }
 
-int g_grid[2][3] = {{0, 0, 0}, {0, 0, 0}};  // [fp4][NB], direct mode
-constexpr int STAGED_SMEM_MAX = 200 * 1024;
+int g_grid[2][3] = {{0, 0, 0}, {0, 0, 0}};  // [fp4][NB]
+
+template <int NB, bool FP4>
+cudaError_t kernel_setup(int sms) {
+  int per = 0;
+  const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, gemv_fused_kernel<NB, FP4>, WARPS * 32, 0);
+  g_grid[FP4][NB] = sms * (per > 0 ? per : 1);
+  return e;
+}
 
 }  // namespace
 
@@ -455,17 +425,6 @@ bool gemv_mma_supported(const Shape& sh) {
   if (sh.wtype == FT_W_BF16) return sh.d % 32 == 0 && sh.d_ff % 32 == 0;
   if (sh.wtype == FT_W_NVFP4) return sh.d % 128 == 0 && sh.d_ff % 128 == 0;
   return false;
-}
-
-template <int NB, bool FP4>
-cudaError_t kernel_setup(int sms) {
-  cudaError_t e = cudaFuncSetAttribute(gemv_mma_kernel<NB, FP4, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       STAGED_SMEM_MAX);
-  if (e != cudaSuccess) return e;
-  int per = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, gemv_mma_kernel<NB, FP4, false>, WARPS * 32, 0);
-  g_grid[FP4][NB] = sms * (per > 0 ? per : 1);
-  return e;
 }
 
 cudaError_t gemv_mma_init(int device) {
@@ -478,19 +437,14 @@ cudaError_t gemv_mma_init(int device) {
   return e;
 }
 
-template <int NB, bool FP4>
-void launch_variant(bool staged, int grid, int dyn, const MmaArgs& a, int phase, cudaStream_t st) {
-  if (staged) gemv_mma_kernel<NB, FP4, true><<<grid, WARPS * 32, dyn, st>>>(a, phase);
-  else gemv_mma_kernel<NB, FP4, false><<<grid, WARPS * 32, 0, st>>>(a, phase);
-}
-
 void launch_to_f16(const void* x, int n, void* y, cudaStream_t st) {
   const int grid = (n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184;
   to_f16_kernel<<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, n, (__half*)y);
 }
 
-void launch_gemv_mma(const Shape& sh, int cls, int phase, int layer, const void* x16, int T, DevState& ds,
-                     int max_items, int max_tok, cudaStream_t st) {
+// Both phases of one work class in one launch.
+void launch_gemv_mma(const Shape& sh, int cls, int layer, const void* x16, int T, DevState& ds, int max_items,
+                     int max_tok, cudaStream_t st) {
   MmaArgs a;
   a.work = ds.work;
   a.cls = cls;
@@ -499,7 +453,6 @@ void launch_gemv_mma(const Shape& sh, int cls, int phase, int layer, const void*
   a.k = sh.k;
   a.d = sh.d;
   a.d_ff = sh.d_ff;
-  a.nvfp4 = sh.wtype == FT_W_NVFP4;
   a.C = sh.C;
   a.slot_bytes = sh.slot_bytes;
   a.slots = ds.slots;
@@ -510,26 +463,26 @@ void launch_gemv_mma(const Shape& sh, int cls, int phase, int layer, const void*
   a.h16 = ds.h16;
   a.h16lo = ds.h16lo;
   a.ybuf = ds.ybuf;
+  a.ticket = ds.sched + cls;
+  a.done = ds.sched + N_CLASSES + (size_t)cls * ds.sched_chunks;
+  a.error = ds.error;
+  const bool fp4 = sh.wtype == FT_W_NVFP4;
   const int NB = T > 8 ? 2 : 1;
   const long long chunks = (long long)max_items + (long long)max_tok / CHUNK;
-  const long long units = chunks * (phase == 0 ? sh.d_ff / 8 : sh.d / 16);
-  // Streamed experts come over the host link (~55 GB/s): they are staged
-  // through shared memory in contiguous runs, on a few dozen CTAs, leaving
-  // the SMs to the HBM work of the hit and staged experts meanwhile.
-  const int K = phase == 0 ? sh.d : sh.d_ff;
-  const int steps = a.nvfp4 ? K / 128 : K / 32;
-  const int smem = WARPS * warp_tile_bytes(steps, a.nvfp4);
-  const bool staged = cls == KIND_STREAMED && smem <= STAGED_SMEM_MAX;
-  int cap = g_grid[a.nvfp4][NB];
-  if (cls == KIND_STREAMED && cap > 64) cap = 64;
+  const long long units = chunks * (sh.d_ff / 8 + sh.d / 16);
+  // Streamed experts come over the host link: a few dozen CTAs reach its
+  // bandwidth best (fewer concurrent scattered streams into host memory) and
+  // leave the SMs to the HBM work of the hit and staged experts meanwhile.
+  int cap = g_grid[fp4][NB];
+  if (cls == KIND_STREAMED && cap > 32) cap = 32;
   const int grid = (int)(units < cap ? units : cap);
   if (grid <= 0) return;
-  if (a.nvfp4) {
-    if (NB == 1) launch_variant<1, true>(staged, grid, smem, a, phase, st);
-    else launch_variant<2, true>(staged, grid, smem, a, phase, st);
+  if (fp4) {
+    if (NB == 1) gemv_fused_kernel<1, true><<<grid, WARPS * 32, 0, st>>>(a);
+    else gemv_fused_kernel<2, true><<<grid, WARPS * 32, 0, st>>>(a);
   } else {
-    if (NB == 1) launch_variant<1, false>(staged, grid, smem, a, phase, st);
-    else launch_variant<2, false>(staged, grid, smem, a, phase, st);
+    if (NB == 1) gemv_fused_kernel<1, false><<<grid, WARPS * 32, 0, st>>>(a);
+    else gemv_fused_kernel<2, false><<<grid, WARPS * 32, 0, st>>>(a);
   }
 }
 

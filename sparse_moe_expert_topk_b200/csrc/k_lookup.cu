@@ -73,7 +73,7 @@ __global__ void __launch_bounds__(NT) lookup_kernel(LookupArgs a, int E, long lo
   __shared__ unsigned long long s_prefix, s_mask;
   __shared__ int s_remaining, s_ncand, s_avail;
   __shared__ unsigned long long s_c0, s_epoch, s_bstart;
-  __shared__ int s_cbase, s_lbase, s_tok;
+  __shared__ int s_cbase, s_lbase, s_tok, s_chunks;
 
   const int tid = threadIdx.x;
   Mailbox* mb = ds.mbox;
@@ -231,6 +231,18 @@ __global__ void __launch_bounds__(NT) lookup_kernel(LookupArgs a, int E, long lo
       if ((tid & 31) == 0) atomicAdd(&s_tok, tok);
       __syncthreads();
       if (tid == 0) mb->n_tok_cls[c] = s_tok;
+      // tensor-core GEMV scheduling state of this class: ticket and one
+      // completion counter per (item, 16-token chunk)
+      int ch = (act && kind == c) ? (ds.counts[e] + MMA_CHUNK - 1) / MMA_CHUNK : 0;
+      for (int o = 16; o > 0; o >>= 1) ch += __shfl_xor_sync(0xffffffffu, ch, o);
+      if (tid == 0) s_chunks = 0;
+      __syncthreads();
+      if ((tid & 31) == 0) atomicAdd(&s_chunks, ch);
+      __syncthreads();
+      const int nch = s_chunks < ds.sched_chunks ? s_chunks : ds.sched_chunks;
+      int32_t* done = ds.sched + N_CLASSES + (size_t)c * ds.sched_chunks;
+      for (int i = tid; i < nch; i += NT) done[i] = 0;
+      if (tid == 0) ds.sched[c] = 0;
       if (act && kind == c) {
         WorkItem it;
         it.e = e;
@@ -298,6 +310,19 @@ __global__ void __launch_bounds__(NT) prefill_work_kernel(int layer, int E, DevS
   const bool in = tid < E && ds.counts[tid] > 0;
   int n;
   const int r = block_scan_flag(in, scan, n);
+  {
+    __shared__ int s_ch;
+    int ch = in ? (ds.counts[tid] + MMA_CHUNK - 1) / MMA_CHUNK : 0;
+    for (int o = 16; o > 0; o >>= 1) ch += __shfl_xor_sync(0xffffffffu, ch, o);
+    if (tid == 0) s_ch = 0;
+    __syncthreads();
+    if ((tid & 31) == 0) atomicAdd(&s_ch, ch);
+    __syncthreads();
+    const int nch = s_ch < ds.sched_chunks ? s_ch : ds.sched_chunks;
+    int32_t* done = ds.sched + N_CLASSES + (size_t)KIND_HIT * ds.sched_chunks;
+    for (int i = tid; i < nch; i += NT) done[i] = 0;
+    if (tid == 0) ds.sched[KIND_HIT] = 0;
+  }
   if (in) {
     WorkItem it;
     it.e = tid;
