@@ -142,7 +142,7 @@ void free_all(ft_ctx* c) {
   DevState& d = c->ds;
   void* dev_ptrs[] = {d.slot_of, d.key_of, d.stamp, d.clk, d.ctr, d.error, d.work, d.scores, d.ids, d.wts,
                       d.counts, d.offsets, d.perm, d.inv, d.hbuf, d.ybuf, d.xs, d.hs, d.tscale, d.slots,
-                      d.h16, d.h16lo, d.x16, d.sched, c->probe_sink};
+                      d.h16, d.h16lo, d.x16, d.sched, d.route_ctr, c->probe_sink};
   for (void* p : dev_ptrs)
     if (p) cudaFree(p);
   for (uint8_t* p : c->pool_host)
@@ -192,13 +192,13 @@ ft_status check_device_error(ft_ctx* c) {
 enum ProfName {
   P_ROUTER, P_TOPK, P_PERMUTE, P_LOOKUP, P_GU_HIT, P_DN_HIT, P_GU_STAGED, P_DN_STAGED, P_GU_STREAM, P_DN_STREAM,
   P_COMBINE, P_STAGE_COPY, P_PREFILL_WORK, P_GATHER, P_GEMM_GU, P_GEMM_DN, P_GEMV_HIT, P_GEMV_STAGED,
-  P_GEMV_STREAM, P_TO_F16, P_COUNT
+  P_GEMV_STREAM, P_TO_F16, P_ROUTE_FUSED, P_COUNT
 };
 const char* const kProfNames[P_COUNT] = {
     "router_scores", "topk_softmax", "permute", "lookup", "gemv_gateup_hit", "gemv_down_hit",
     "gemv_gateup_staged", "gemv_down_staged", "gemv_gateup_streamed", "gemv_down_streamed", "combine",
     "h2d_stage_copies", "prefill_work", "prefill_gather", "gemm_tc_gateup", "gemm_tc_down", "gemv_hit",
-    "gemv_staged", "gemv_streamed", "to_f16"};
+    "gemv_staged", "gemv_streamed", "to_f16", "route_decode_fused"};
 
 cudaEvent_t pooled_event(ft_ctx* c) {
   if (!c->evpool.empty()) {
@@ -360,6 +360,8 @@ ft_status ft_moe_init(const ft_config* cfg, void* compute_stream, void* copy_str
   d.sched_chunks = sh.E + (int)((Tk + MMA_CHUNK - 1) / MMA_CHUNK) + 1;
   TRY(cuda_try(cudaMalloc((void**)&d.sched, sizeof(int32_t) * (N_CLASSES + (size_t)N_CLASSES * d.sched_chunks))));
   TRY(cuda_try(cudaMemset(d.sched, 0, sizeof(int32_t) * (N_CLASSES + (size_t)N_CLASSES * d.sched_chunks))));
+  TRY(cuda_try(cudaMalloc((void**)&d.route_ctr, sizeof(int32_t))));
+  TRY(cuda_try(cudaMemset(d.route_ctr, 0, sizeof(int32_t))));
   c->use_tc = prefill_tc_supported(sh) && sh.C >= 2ll * sh.E;
   if (c->use_tc) {
     TRY(cuda_try(cudaMalloc((void**)&d.xs, sizeof(__nv_bfloat16) * (Tk + 256) * sh.d)));
@@ -493,39 +495,53 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
   c->layer_calls += 1;
   const double ab = sh.wtype == FT_W_F32 ? 4.0 : 2.0;
   const int Tk = T * sh.k;
-  int p = prof_begin(c, P_ROUTER, cs, T * (double)sh.d * ab + sh.E * (double)sh.d * ab + T * (double)sh.E * 4.0,
-                     2.0 * T * sh.E * (double)sh.d);
-  launch_router_scores(sh, x, c->router[layer], bias, bias_per_token, T, d.scores, cs);
-  prof_end(c, p, cs);
-  p = prof_begin(c, P_TOPK, cs, T * (double)sh.E * 4.0 + Tk * 8.0);
-  launch_topk(sh, d.scores, T, d, cs);
-  prof_end(c, p, cs);
-  p = prof_begin(c, P_PERMUTE, cs, Tk * 12.0 + sh.E * 8.0);
-  launch_permute(sh, T, d, cs);
-  prof_end(c, p, cs);
-  c->kernel_launches += 3;
+  const bool full_prefill = mode == FT_PREFILL && sh.C >= 2ll * sh.E;
+  // decode (and the on-demand prefill fallback) at small T: router, top-k,
+  // permutation and lookup in one launch
+  const bool fused_route = !full_prefill && T <= 32;
+  LookupArgs la{};
+  la.layer = layer;
+  la.use_counts = 1;
+  la.limit_q = 1;
+  la.is_current = 1;
+  la.build_work = 1;
+  la.bp_mbps = c->bp;
+  la.bh_mbps = c->bh;
+  d.pool_dev = c->pool_dev[layer];
+  if (c->use_mma && sh.wtype == FT_W_NVFP4 && !(full_prefill && c->use_tc)) {
+    launch_to_f16(x, T * sh.d, d.x16, cs);
+    c->kernel_launches += 1;
+  }
+  int p = -1;
+  if (fused_route) {
+    p = prof_begin(c, P_ROUTE_FUSED, cs, T * (double)sh.d * ab + sh.E * (double)sh.d * ab + sh.C * 8.0);
+    launch_route_decode(sh, x, c->router[layer], bias, bias_per_token, T, la, d, cs);
+    prof_end(c, p, cs);
+    c->kernel_launches += 1;
+  } else {
+    p = prof_begin(c, P_ROUTER, cs, T * (double)sh.d * ab + sh.E * (double)sh.d * ab + T * (double)sh.E * 4.0,
+                   2.0 * T * sh.E * (double)sh.d);
+    launch_router_scores(sh, x, c->router[layer], bias, bias_per_token, T, d.scores, cs);
+    prof_end(c, p, cs);
+    p = prof_begin(c, P_TOPK, cs, T * (double)sh.E * 4.0 + Tk * 8.0);
+    launch_topk(sh, d.scores, T, d, cs);
+    prof_end(c, p, cs);
+    p = prof_begin(c, P_PERMUTE, cs, Tk * 12.0 + sh.E * 8.0);
+    launch_permute(sh, T, d, cs);
+    prof_end(c, p, cs);
+    c->kernel_launches += 3;
+  }
   if (ids_opt) CK(cudaMemcpyAsync(ids_opt, d.ids, sizeof(int32_t) * Tk, cudaMemcpyDeviceToDevice, cs));
   if (w_opt) CK(cudaMemcpyAsync(w_opt, d.wts, sizeof(float) * Tk, cudaMemcpyDeviceToDevice, cs));
   const int max_items = Tk < sh.E ? Tk : sh.E;
-  const bool full_prefill = mode == FT_PREFILL && sh.C >= 2ll * sh.E;
   ft_status st = FT_OK;
   if (!full_prefill) {
-    LookupArgs a{};
-    a.layer = layer;
-    a.use_counts = 1;
-    a.limit_q = 1;
-    a.is_current = 1;
-    a.build_work = 1;
-    a.bp_mbps = c->bp;
-    a.bh_mbps = c->bh;
-    d.pool_dev = c->pool_dev[layer];
-    if (c->use_mma && sh.wtype == FT_W_NVFP4) {
-      launch_to_f16(x, T * sh.d, d.x16, cs);
+    if (!fused_route) {
+      p = prof_begin(c, P_LOOKUP, cs, sh.C * 8.0 + sh.E * 16.0);
+      launch_lookup(sh, la, d, cs);
+      prof_end(c, p, cs);
       c->kernel_launches += 1;
     }
-    p = prof_begin(c, P_LOOKUP, cs, sh.C * 8.0 + sh.E * 16.0);
-    launch_lookup(sh, a, d, cs);
-    prof_end(c, p, cs);
     CK(cudaEventRecord(c->ev_look, cs));
     CK(cudaStreamWaitEvent(c->s_side, c->ev_look, 0));
     int pr_stream[2], pr_hit[2], pr_staged[2];
@@ -635,10 +651,6 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
       c->kernel_launches += 3;
     } else {
       d.pool_dev = c->pool_dev[layer];
-      if (c->use_mma && sh.wtype == FT_W_NVFP4) {
-        launch_to_f16(x, T * sh.d, d.x16, cs);
-        c->kernel_launches += 1;
-      }
       int pr[2];
       gemv_class(c, KIND_HIT, layer, x, T, max_items, Tk, cs, pr);
       gemv_class_cost(c, pr, max_items, Tk);  // upper bound: every routed expert

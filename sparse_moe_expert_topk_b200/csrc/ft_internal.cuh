@@ -123,6 +123,7 @@ struct DevState {
   void* tc_plan;             // host: tensor maps of the prefill GEMM (owned, see prefill_tc_free)
   int32_t* sched;            // [N_CLASSES] unit tickets + [N_CLASSES][sched_chunks] chunk completion counters
   int sched_chunks;
+  int32_t* route_ctr;        // last-CTA ticket of the fused decode routing kernel (0 between calls)
 };
 
 // ---- launchers (all enqueue on `st`) ----
@@ -133,6 +134,9 @@ void launch_router_scores(const Shape& sh, const void* x, const void* w_router, 
 void launch_topk(const Shape& sh, const float* scores, int T, DevState& ds, cudaStream_t st);
 // stable permutation (counts, offsets, perm, inv)
 void launch_permute(const Shape& sh, int T, DevState& ds, cudaStream_t st);
+// decode routing in one launch (T <= 32): logits, top-k, permutation, lookup
+void launch_route_decode(const Shape& sh, const void* x, const void* w_router, const float* bias, int bias_per_token,
+                         int T, const LookupArgs& la, DevState& ds, cudaStream_t st);
 // one lookup batch; writes work lists, mailbox, counters
 void launch_lookup(const Shape& sh, const LookupArgs& a, DevState& ds, cudaStream_t st);
 // decode / fallback experts (SIMT grouped GEMV) for one work class;

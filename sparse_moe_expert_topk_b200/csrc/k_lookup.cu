@@ -17,290 +17,17 @@
 // inserted entry is pinned, the victims of a batch are exactly its q_stage
 // smallest (stamp, slot) pairs among unpinned slots (free slots carry stamp 0),
 // handed out in increasing order; this kernel finds them with a radix select.
-#include "ft_internal.cuh"
+#include "lookup_body.cuh"
 
 namespace ft {
 
 namespace {
 
-constexpr int NT = 1024;
-constexpr unsigned long long NOKEY = ~0ull;
-constexpr int SLOT_BITS = 20;
-
-struct ScanTmp {
-  int warp_tot[32];
-  int total;
-};
-
-// Exclusive prefix of a 0/1 flag over the 1024 threads; *total = sum.
-__device__ __forceinline__ int block_scan_flag(bool f, ScanTmp& s, int& total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const unsigned b = __ballot_sync(0xffffffffu, f);
-  const int in_warp = __popc(b & ((1u << lane) - 1u));
-  __syncthreads();
-  if (lane == 0) s.warp_tot[warp] = __popc(b);
-  __syncthreads();
-  if (warp == 0) {
-    const int v = s.warp_tot[lane];
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    s.warp_tot[lane] = incl - v;
-    if (lane == 31) s.total = incl;
-  }
-  __syncthreads();
-  total = s.total;
-  return s.warp_tot[warp] + in_warp;
-}
-
-__device__ __forceinline__ unsigned long long slot_key(const unsigned long long* stamp, long long s,
-                                                       unsigned long long epoch) {
-  const unsigned long long st = stamp[s];
-  return st < epoch ? ((st << SLOT_BITS) | (unsigned long long)s) : NOKEY;
-}
+using namespace lookup_detail;
 
 __global__ void __launch_bounds__(NT) lookup_kernel(LookupArgs a, int E, long long C, size_t slot_bytes,
                                                     DevState ds) {
-  __shared__ int s_e[MAX_E];
-  __shared__ int s_slot[MAX_E];
-  __shared__ int s_vic[MAX_E];
-  __shared__ unsigned long long s_cand[MAX_E];
-  __shared__ int s_hist[256];
-  __shared__ ScanTmp scan;
-  __shared__ unsigned long long s_prefix, s_mask;
-  __shared__ int s_remaining, s_ncand, s_avail;
-  __shared__ unsigned long long s_c0, s_epoch, s_bstart;
-  __shared__ int s_cbase, s_lbase, s_tok, s_chunks;
-
-  const int tid = threadIdx.x;
-  Mailbox* mb = ds.mbox;
-  const int layer = a.layer;
-
-  // 1. the batch: routed experts (counts > 0) or all E, ascending
-  const bool in = tid < E && (a.use_counts ? ds.counts[tid] > 0 : true);
-  int n_u;
-  const int upos = block_scan_flag(in, scan, n_u);
-  if (in) s_e[upos] = tid;
-  __syncthreads();
-
-  // 2. hits
-  const bool act = tid < n_u;
-  int e = -1, key = -1, sl = -1;
-  if (act) {
-    e = s_e[tid];
-    key = layer * E + e;
-    sl = ds.slot_of[key];
-    if (sl >= C) {  // corrupt table: report and treat as a miss
-      atomicExch(ds.error, (uint32_t)DERR_BAD_INDEX);
-      sl = -1;
-    }
-  }
-  const bool hit = act && sl >= 0;
-  int h;
-  const int hrank = block_scan_flag(hit, scan, h);
-  int m;
-  const int mrank = block_scan_flag(act && !hit, scan, m);
-
-  // 3. clock and pins
-  if (tid == 0) {
-    const unsigned long long c0 = ds.clk->clock;
-    s_c0 = c0;
-    s_bstart = c0 + 1;
-    s_epoch = a.pin_prev ? ds.clk->batch_start : c0 + 1;
-    s_cbase = a.append ? mb->n_copy : 0;
-    s_lbase = a.append ? mb->n_lookup : 0;
-  }
-  __syncthreads();
-  const unsigned long long c0 = s_c0, epoch = s_epoch;
-  if (hit) ds.stamp[sl] = c0 + 1 + (unsigned long long)hrank;
-
-  // 4. q*
-  int q, q_stage;
-  if (a.limit_q) {
-    q = 0;
-    if (m > 0) {
-      const unsigned long long num = 2ull * (unsigned long long)m * a.bp_mbps + a.bh_mbps;
-      const unsigned long long qq = num / (2ull * a.bh_mbps);
-      q = (int)(qq > (unsigned long long)m ? m : qq);
-    }
-    const long long room = C - h;
-    q_stage = (long long)q < room ? q : (int)room;
-  } else {
-    q = -1;
-    q_stage = m;
-  }
-  __syncthreads();  // hit stamps visible before victim selection
-
-  // 5. victims: the q_stage smallest keys among unpinned slots
-  if (q_stage > 0) {
-    int avail_local = 0;
-    for (long long s = tid; s < C; s += NT) avail_local += slot_key(ds.stamp, s, epoch) != NOKEY;
-    if (tid == 0) s_avail = 0;
-    __syncthreads();
-    for (int o = 16; o > 0; o >>= 1) avail_local += __shfl_xor_sync(0xffffffffu, avail_local, o);
-    if ((tid & 31) == 0) atomicAdd(&s_avail, avail_local);
-    __syncthreads();
-    if (s_avail < q_stage) {
-      if (tid == 0) atomicExch(ds.error, (uint32_t)DERR_NO_VICTIM);
-      q_stage = s_avail;
-    }
-  }
-  if (q_stage > 0) {
-    if (tid == 0) {
-      s_prefix = 0;
-      s_mask = 0;
-      s_remaining = q_stage;
-    }
-    for (int shift = 56; shift >= 0; shift -= 8) {
-      for (int i = tid; i < 256; i += NT) s_hist[i] = 0;
-      __syncthreads();
-      const unsigned long long pre = s_prefix, msk = s_mask;
-      for (long long s = tid; s < C; s += NT) {
-        const unsigned long long k = slot_key(ds.stamp, s, epoch);
-        if (k != NOKEY && (k & msk) == pre) atomicAdd(&s_hist[(k >> shift) & 255], 1);
-      }
-      __syncthreads();
-      if (tid == 0) {
-        int rem = s_remaining, b = 0;
-        for (; b < 256; ++b) {
-          if (s_hist[b] >= rem) break;
-          rem -= s_hist[b];
-        }
-        s_remaining = rem;
-        s_prefix = pre | ((unsigned long long)b << shift);
-        s_mask = msk | (255ull << shift);
-      }
-      __syncthreads();
-    }
-    const unsigned long long thr = s_prefix;  // the q_stage-th smallest key
-    if (tid == 0) s_ncand = 0;
-    __syncthreads();
-    for (long long s = tid; s < C; s += NT) {
-      const unsigned long long k = slot_key(ds.stamp, s, epoch);
-      if (k != NOKEY && k <= thr) {
-        const int i = atomicAdd(&s_ncand, 1);
-        if (i < MAX_E) s_cand[i] = k;
-      }
-    }
-    __syncthreads();
-    if (s_ncand != q_stage) {  // cannot happen with unique keys; stay memory safe if it does
-      if (tid == 0) atomicExch(ds.error, (uint32_t)DERR_NO_VICTIM);
-      q_stage = 0;
-    }
-    if (tid < q_stage) {
-      const unsigned long long mine = s_cand[tid];
-      int r = 0;
-      for (int j = 0; j < q_stage; ++j) r += s_cand[j] < mine;
-      s_vic[r] = (int)(mine & ((1ull << SLOT_BITS) - 1));
-    }
-    __syncthreads();
-  }
-
-  // 6. insert the staged misses
-  const bool staged = act && !hit && mrank < q_stage;
-  if (staged) {
-    const int v = s_vic[mrank];
-    const int old = ds.key_of[v];
-    if (old >= 0) ds.slot_of[old] = -1;
-    ds.key_of[v] = key;
-    ds.slot_of[key] = v;
-    ds.stamp[v] = c0 + (unsigned long long)h + 1ull + (unsigned long long)mrank;
-    s_slot[tid] = v;
-  } else if (act) {
-    s_slot[tid] = hit ? sl : -1;
-  }
-  if (tid == 0) {
-    ds.clk->clock = c0 + (unsigned long long)h + (unsigned long long)q_stage;
-    ds.clk->batch_start = s_bstart;
-  }
-  __syncthreads();
-  const int kind = hit ? KIND_HIT : (staged ? KIND_STAGED : KIND_STREAMED);
-
-  // 7. work lists of the routed experts, per class, ascending e
-  if (a.build_work) {
-    for (int c = 0; c < N_CLASSES; ++c) {
-      int n_c;
-      const int r = block_scan_flag(act && kind == c, scan, n_c);
-      int tok = (act && kind == c) ? ds.counts[e] : 0;
-      for (int o = 16; o > 0; o >>= 1) tok += __shfl_xor_sync(0xffffffffu, tok, o);
-      if (tid == 0) s_tok = 0;
-      __syncthreads();
-      if ((tid & 31) == 0) atomicAdd(&s_tok, tok);
-      __syncthreads();
-      if (tid == 0) mb->n_tok_cls[c] = s_tok;
-      // tensor-core GEMV scheduling state of this class: ticket and one
-      // completion counter per (item, 16-token chunk)
-      int ch = (act && kind == c) ? (ds.counts[e] + MMA_CHUNK - 1) / MMA_CHUNK : 0;
-      for (int o = 16; o > 0; o >>= 1) ch += __shfl_xor_sync(0xffffffffu, ch, o);
-      if (tid == 0) s_chunks = 0;
-      __syncthreads();
-      if ((tid & 31) == 0) atomicAdd(&s_chunks, ch);
-      __syncthreads();
-      const int nch = s_chunks < ds.sched_chunks ? s_chunks : ds.sched_chunks;
-      int32_t* done = ds.sched + N_CLASSES + (size_t)c * ds.sched_chunks;
-      for (int i = tid; i < nch; i += NT) done[i] = 0;
-      if (tid == 0) ds.sched[c] = 0;
-      if (act && kind == c) {
-        WorkItem it;
-        it.e = e;
-        it.slot = s_slot[tid];
-        it.tok_off = ds.offsets[e];
-        it.n_tok = ds.counts[e];
-        ds.work->items[c][r] = it;
-      }
-      if (tid == 0) ds.work->n_items[c] = n_c;
-    }
-  }
-
-  // 8. mailbox for the host (mapped memory) and counters
-  const int cbase = s_cbase, lbase = s_lbase;
-  if (staged) {
-    mb->copy_key[cbase + mrank] = key;
-    mb->copy_slot[cbase + mrank] = s_slot[tid];
-  }
-  if (act) {
-    mb->lookup_e[lbase + tid] = e;
-    mb->lookup_kind[lbase + tid] = kind;
-  }
-  __syncthreads();
-  if (tid == 0) {
-    mb->n_copy = cbase + q_stage;
-    mb->n_lookup = lbase + n_u;
-    if (a.is_current) {
-      mb->m = m;
-      mb->qstar = q;
-      mb->qstage = q_stage;
-      mb->n_lookup_cur = n_u;
-      ds.ctr->last_m = m;
-      ds.ctr->last_qstar = q;
-      ds.ctr->last_qstage = q_stage;
-    } else if (!a.append) {
-      mb->m = 0;
-      mb->qstar = -1;
-      mb->qstage = 0;
-      mb->n_lookup_cur = 0;
-    }
-    if (a.build_work) {
-      mb->n_hit_cls = ds.work->n_items[KIND_HIT];
-      mb->n_staged_cls = ds.work->n_items[KIND_STAGED];
-      mb->n_streamed_cls = ds.work->n_items[KIND_STREAMED];
-    }
-    mb->pad_error = *ds.error;
-    DevCounters* c = ds.ctr;
-    c->lookups += n_u;
-    c->hits += h;
-    c->misses += m;
-    c->staged += q_stage;
-    c->streamed += m - q_stage;
-    c->bytes_h2d += (unsigned long long)q_stage * slot_bytes;
-    c->bytes_zero_copy += (unsigned long long)(m - q_stage) * slot_bytes;
-    __threadfence_system();
-    mb->seq = mb->seq + 1;
-    __threadfence_system();
-  }
+  lookup_body(a, E, C, slot_bytes, ds);
 }
 
 // Work list of a prefill call: every routed expert, read from its slot.

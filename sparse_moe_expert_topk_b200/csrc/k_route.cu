@@ -8,7 +8,7 @@
 // expert index), softmax over those k.
 #include <atomic>
 
-#include "ft_internal.cuh"
+#include "lookup_body.cuh"
 
 namespace ft {
 
@@ -80,19 +80,16 @@ __global__ void __launch_bounds__(256) router_scores_kernel(const AT* __restrict
 
 // One warp per token: k rounds of a warp arg-max (larger logit first, equal
 // logits -> lower index), then softmax over the chosen k.
-__global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restrict__ scores, int T, int E, int k,
-                                                           int32_t* __restrict__ ids, float* __restrict__ wts) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (warp >= T) return;
+__device__ __forceinline__ void topk_token(const float* __restrict__ scores, int warp, int E, int k,
+                                           int32_t* __restrict__ ids, float* __restrict__ wts, int lane) {
   constexpr int PER = MAX_E / 32;
   float v[PER];
   uint32_t taken = 0;
-  const float* s = scores + (size_t)warp * E;
+  const float* s = scores + (size_t)warp * E;  // warp = token index
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int e = i * 32 + lane;
-    v[i] = e < E ? s[e] : 0.f;
+    v[i] = e < E ? __ldcg(s + e) : 0.f;  // L2: in the fused kernel other CTAs wrote these
   }
   float top0 = 0.f, sel[MAX_K];
   int sid[MAX_K];
@@ -137,14 +134,21 @@ __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restri
   }
 }
 
+__global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restrict__ scores, int T, int E, int k,
+                                                           int32_t* __restrict__ ids, float* __restrict__ wts) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (warp >= T) return;
+  topk_token(scores, warp, E, k, ids, wts, threadIdx.x & 31);
+}
+
 // Stable counting sort of the n = T*k routing ids by expert, one CTA of 1024
 // threads. Sorted order = (expert, flat index t*k+j). Within a 1024-entry
 // chunk a thread's rank among equal experts comes from __match_any_sync
 // inside its warp plus the counts of the lower warps.
-__global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict__ ids, int n, int E,
-                                                       int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                                                       int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
-  extern __shared__ int32_t smem[];
+__device__ __forceinline__ void permute_body(const int32_t* __restrict__ ids, int n, int E,
+                                             int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                             int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                             int32_t* smem) {
   int32_t* wcnt = smem;                // [32][E]
   int32_t* run = smem + 32 * E;        // [E] next free position per expert
   int32_t* tot = run + E;              // [E] per-chunk totals
@@ -213,6 +217,88 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict
     for (int x = tid; x < E; x += 1024) run[x] += tot[x];
     __syncthreads();
   }
+}
+
+__global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict__ ids, int n, int E,
+                                                       int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                                       int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
+  extern __shared__ int32_t smem[];
+  permute_body(ids, n, E, counts, offsets, perm, inv, smem);
+}
+
+// Decode routing in one launch (T <= 32 tokens): CTAs of 32 warps compute the
+// logits of 32 experts each (one warp per expert, all tokens); the last CTA to
+// finish (ticket on ds.route_ctr) runs top-k + softmax, the stable
+// permutation and the LRU lookup of the layer. Same device code as the
+// separate kernels, so the results are the same.
+template <typename AT>
+__global__ void __launch_bounds__(1024) route_decode_kernel(const AT* __restrict__ x, const AT* __restrict__ wr,
+                                                            const float* __restrict__ bias, int bias_per_token, int T,
+                                                            int E, int d, int k, LookupArgs la, long long C,
+                                                            size_t slot_bytes, DevState ds) {
+  extern __shared__ int32_t smem[];
+  __shared__ int s_last;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.x * 32 + warp;
+  if (e < E) {
+    constexpr int VN = 16 / sizeof(AT);
+    const int nv = d / VN;
+    const uint4* wrow = reinterpret_cast<const uint4*>(wr + (size_t)e * d);
+    for (int t0 = 0; t0 < T; t0 += 8) {
+      const int nt = min(8, T - t0);
+      float acc[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) acc[t] = 0.f;
+      for (int v = lane; v < nv; v += 32) {
+        const uint4 wv = __ldg(wrow + v);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          if (t < nt) {
+            const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + (size_t)(t0 + t) * d) + v);
+            if constexpr (sizeof(AT) == 2) {
+              float wf[8], xf[8];
+              to_f32x8(wv, wf);
+              to_f32x8(xv, xf);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) acc[t] = fmaf(wf[i], xf[i], acc[t]);
+            } else {
+              acc[t] = fmaf(__uint_as_float(wv.x), __uint_as_float(xv.x), acc[t]);
+              acc[t] = fmaf(__uint_as_float(wv.y), __uint_as_float(xv.y), acc[t]);
+              acc[t] = fmaf(__uint_as_float(wv.z), __uint_as_float(xv.z), acc[t]);
+              acc[t] = fmaf(__uint_as_float(wv.w), __uint_as_float(xv.w), acc[t]);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
+      }
+      if (lane < nt) {
+        float a = 0.f;
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+          if (t == lane) a = acc[t];
+        const int tt = t0 + lane;
+        float b = 0.f;
+        if (bias) b = bias_per_token ? bias[(size_t)tt * E + e] : bias[e];
+        ds.scores[(size_t)tt * E + e] = a + b;
+      }
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(ds.route_ctr, 1) == (int)gridDim.x - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  if (warp < T) topk_token(ds.scores, warp, E, k, ds.ids, ds.wts, lane);
+  __syncthreads();
+  permute_body(ds.ids, T * k, E, ds.counts, ds.offsets, ds.perm, ds.inv, smem);
+  __syncthreads();
+  lookup_detail::lookup_body(la, E, C, slot_bytes, ds);
+  if (threadIdx.x == 0) *ds.route_ctr = 0;  // ready for the next call
 }
 
 }  // namespace
@@ -293,9 +379,28 @@ extern "C" ft_status ft_route_topk_static(const void* x_dev, const void* w_route
 
 namespace ft {
 
+void launch_route_decode(const Shape& sh, const void* x, const void* w_router, const float* bias, int bias_per_token,
+                         int T, const LookupArgs& la, DevState& ds, cudaStream_t st) {
+  const int grid = (sh.E + 31) / 32;
+  const size_t smem = permute_smem_bytes(sh.E);
+  if (sh.wtype == FT_W_F32)
+    route_decode_kernel<float><<<grid, 1024, smem, st>>>((const float*)x, (const float*)w_router, bias,
+                                                         bias_per_token, T, sh.E, sh.d, sh.k, la, sh.C, sh.slot_bytes,
+                                                         ds);
+  else
+    route_decode_kernel<__nv_bfloat16><<<grid, 1024, smem, st>>>((const __nv_bfloat16*)x,
+                                                                 (const __nv_bfloat16*)w_router, bias, bias_per_token,
+                                                                 T, sh.E, sh.d, sh.k, la, sh.C, sh.slot_bytes, ds);
+}
+
 cudaError_t route_kernels_init(int E) {
-  return cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)permute_smem_bytes(E));
+  const int smem = (int)permute_smem_bytes(E);
+  cudaError_t e = cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(route_decode_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(route_decode_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  return e;
 }
 
 }  // namespace ft
