@@ -48,7 +48,7 @@ struct WorkLists {
 // into mapped pinned memory. The host copy thread reads it after the lookup
 // kernel's event completed.
 struct Mailbox {
-  int32_t seq;        // incremented by each lookup kernel
+  int32_t reserved;
   int32_t n_copy;     // slots to fill by H2D copy (staged + prefill loads)
   int32_t m, qstar, qstage;
   int32_t n_lookup, n_lookup_cur;

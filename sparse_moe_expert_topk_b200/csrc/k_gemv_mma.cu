@@ -8,7 +8,7 @@
 // kernel keeps many loads in flight and spends few instructions per byte.
 //
 // Work unit: 16 weight rows x one chunk of <= 16 tokens of one expert, done
-// by one CTA of 8 warps that split the unit's K range (split-K) and reduce
+// by one CTA of 4 warps that split the unit's K range (split-K) and reduce
 // their partial sums in warp order through shared memory. Inside a warp,
 // lane (g, q) = (lane/4, lane%4) loads 16 consecutive bytes of rows g and
 // g+8 per step and hands them to the MMA unchanged as its A fragment; that
@@ -42,7 +42,7 @@ namespace ft {
 
 namespace {
 
-constexpr int WARPS = 8;
+constexpr int WARPS = 4;  // warps per CTA; they split a unit's K range
 constexpr int CHUNK = 16;  // tokens per unit (two n8 tiles)
 constexpr long long WAIT_CYCLES = 4000000000ll;  // ~2 s
 
@@ -371,12 +371,15 @@ __global__ void __launch_bounds__(WARPS * 32) gemv_fused_kernel(MmaArgs a) {
   const int n_qi = s_pref[n_items];
   const int rb0 = a.d_ff / 8, rb1 = a.d / 16;
   const int U0 = n_qi * rb0, U1 = n_qi * rb1;
+  if (tid == 0) s_unit = atomicAdd(a.ticket, 1);
+  __syncthreads();
   for (;;) {
-    __syncthreads();  // every thread has read the previous ticket
-    if (tid == 0) s_unit = atomicAdd(a.ticket, 1);
-    __syncthreads();
     const int u = s_unit;
     if (u >= U0 + U1) break;
+    // the next ticket is fetched while this unit runs (phase-0 tickets all
+    // precede phase-1 ones, so holding one never blocks a waited-on unit)
+    int nxt = 0;
+    if (tid == 0) nxt = atomicAdd(a.ticket, 1);
     const int phase = u < U0 ? 0 : 1;
     int item, chunk, rb, qi;
     unit_of(s_pref, n_items, phase == 0 ? rb0 : rb1, phase == 0 ? u : u - U0, item, chunk, rb, qi);
@@ -401,6 +404,9 @@ __global__ void __launch_bounds__(WARPS * 32) gemv_fused_kernel(MmaArgs a) {
       if (!bad) unit_work<NB, 0, FP4>(a, it, chunk, rb, warp, lane, red);
       if (tid == 0) atomicAdd(a.done + qi, 1);
     }
+    __syncthreads();  // every thread has read s_unit
+    if (tid == 0) s_unit = nxt;
+    __syncthreads();
   }
 }
 

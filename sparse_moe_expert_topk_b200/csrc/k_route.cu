@@ -226,6 +226,73 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict
   permute_body(ids, n, E, counts, offsets, perm, inv, smem);
 }
 
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// BF16 logits of 16 experts (rows e0..e0+15 of W_r) for all T tokens, by one
+// CTA of 32 warps: warp w takes K steps [w*S/32, (w+1)*S/32) of 32 values;
+// lane (g, q) feeds 16 bytes of rows g and g+8 to the MMA as its A fragment and
+// the matching 16 bytes of token rows as the B fragment (the lane-dependent K
+// order is the same on both sides). Partial sums are reduced in warp order in
+// shared memory (red: 32 warps x 8 values x 32 lanes floats).
+__device__ void logits_bf16_block(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wr,
+                                  const float* __restrict__ bias, int bias_per_token, int T, int E, int d, int e0,
+                                  float* __restrict__ scores, float* red) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+  const int steps = d / 32;
+  const int s0 = (warp * steps) / 32, s1 = ((warp + 1) * steps) / 32;
+  const int ra = min(e0 + g, E - 1), rb = min(e0 + g + 8, E - 1);  // clamp: rows past E are not stored
+  const uint8_t* pa = reinterpret_cast<const uint8_t*>(wr + (size_t)ra * d) + q * 16;
+  const uint8_t* pb = reinterpret_cast<const uint8_t*>(wr + (size_t)rb * d) + q * 16;
+  for (int t0 = 0; t0 < T; t0 += 16) {
+    const int nt = min(16, T - t0);
+    const __nv_bfloat16* xr0 = x + (size_t)(t0 + (g < nt ? g : 0)) * d;
+    const __nv_bfloat16* xr1 = x + (size_t)(t0 + (g + 8 < nt ? g + 8 : 0)) * d;
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    for (int s = s0; s < s1; ++s) {
+      const uint4 wa = __ldg(reinterpret_cast<const uint4*>(pa + (size_t)s * 64));
+      const uint4 wb = __ldg(reinterpret_cast<const uint4*>(pb + (size_t)s * 64));
+      const uint4 x0 = __ldg(reinterpret_cast<const uint4*>(xr0 + s * 32 + q * 8));
+      mma_bf16_16816(acc[0], wa.x, wb.x, wa.y, wb.y, x0.x, x0.y);
+      mma_bf16_16816(acc[0], wa.z, wb.z, wa.w, wb.w, x0.z, x0.w);
+      if (nt > 8) {
+        const uint4 x1 = __ldg(reinterpret_cast<const uint4*>(xr1 + s * 32 + q * 8));
+        mma_bf16_16816(acc[1], wa.x, wb.x, wa.y, wb.y, x1.x, x1.y);
+        mma_bf16_16816(acc[1], wa.z, wb.z, wa.w, wb.w, x1.z, x1.w);
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) red[(warp * 8 + t * 4 + c) * 32 + lane] = acc[t][c];
+    __syncthreads();
+    if (warp == 0) {
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float v = red[(t * 4 + c) * 32 + lane];
+          for (int w = 1; w < 32; ++w) v += red[(w * 8 + t * 4 + c) * 32 + lane];
+          // d0,d1: expert e0+g, tokens 2q, 2q+1; d2,d3: expert e0+g+8
+          const int tok = t0 + t * 8 + 2 * q + (c & 1);
+          const int e = e0 + g + (c >> 1) * 8;
+          if (tok < T && t * 8 + 2 * q + (c & 1) < nt && e < E) {
+            float b = 0.f;
+            if (bias) b = bias_per_token ? bias[(size_t)tok * E + e] : bias[e];
+            scores[(size_t)tok * E + e] = v + b;
+          }
+        }
+    }
+    __syncthreads();
+  }
+}
+
 // Decode routing in one launch (T <= 32 tokens): CTAs of 32 warps compute the
 // logits of 32 experts each (one warp per expert, all tokens); the last CTA to
 // finish (ticket on ds.route_ctr) runs top-k + softmax, the stable
@@ -239,8 +306,12 @@ __global__ void __launch_bounds__(1024) route_decode_kernel(const AT* __restrict
   extern __shared__ int32_t smem[];
   __shared__ int s_last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int e = blockIdx.x * 32 + warp;
-  if (e < E) {
+  if constexpr (sizeof(AT) == 2) {
+    // BF16: 16 experts per CTA on the tensor cores (red reuses the dynamic smem)
+    logits_bf16_block(x, wr, bias, bias_per_token, T, E, d, blockIdx.x * 16, ds.scores,
+                      reinterpret_cast<float*>(smem));
+  } else if (blockIdx.x * 32 + warp < E) {
+    const int e = blockIdx.x * 32 + warp;
     constexpr int VN = 16 / sizeof(AT);
     const int nv = d / VN;
     const uint4* wrow = reinterpret_cast<const uint4*>(wr + (size_t)e * d);
@@ -379,10 +450,16 @@ extern "C" ft_status ft_route_topk_static(const void* x_dev, const void* w_route
 
 namespace ft {
 
+size_t route_decode_smem(int E) {
+  const size_t red = sizeof(float) * 32 * 8 * 32;  // logits partial sums (BF16)
+  const size_t perm = permute_smem_bytes(E);
+  return red > perm ? red : perm;
+}
+
 void launch_route_decode(const Shape& sh, const void* x, const void* w_router, const float* bias, int bias_per_token,
                          int T, const LookupArgs& la, DevState& ds, cudaStream_t st) {
-  const int grid = (sh.E + 31) / 32;
-  const size_t smem = permute_smem_bytes(sh.E);
+  const int grid = sh.wtype == FT_W_F32 ? (sh.E + 31) / 32 : (sh.E + 15) / 16;
+  const size_t smem = route_decode_smem(sh.E);
   if (sh.wtype == FT_W_F32)
     route_decode_kernel<float><<<grid, 1024, smem, st>>>((const float*)x, (const float*)w_router, bias,
                                                          bias_per_token, T, sh.E, sh.d, sh.k, la, sh.C, sh.slot_bytes,
@@ -394,12 +471,13 @@ void launch_route_decode(const Shape& sh, const void* x, const void* w_router, c
 }
 
 cudaError_t route_kernels_init(int E) {
-  const int smem = (int)permute_smem_bytes(E);
+  const int smem = (int)permute_smem_bytes(E), smem_f = (int)route_decode_smem(E);
   cudaError_t e = cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(route_decode_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(route_decode_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_f);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(route_decode_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(route_decode_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem_f);
   return e;
 }
 

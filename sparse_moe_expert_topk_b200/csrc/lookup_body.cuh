@@ -282,9 +282,8 @@ __device__ __forceinline__ void lookup_body(const LookupArgs& a, int E, long lon
     c->streamed += m - q_stage;
     c->bytes_h2d += (unsigned long long)q_stage * slot_bytes;
     c->bytes_zero_copy += (unsigned long long)(m - q_stage) * slot_bytes;
-    __threadfence_system();
-    mb->seq = mb->seq + 1;
-    __threadfence_system();
+    // no fence needed: the host reads the mailbox only after an event recorded
+    // behind this kernel has completed
   }
 }
 

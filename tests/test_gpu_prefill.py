@@ -118,3 +118,31 @@ def test_prefill_fallback_when_two_layers_do_not_fit(cuda_ok):
             _call(h, oc, W, l, ft.FT_PREFILL, x, None, sample=[0, T - 1])
         _check_state(h, oc)
         assert h.stats()["streamed"] > 0
+
+
+NVFP4_SMALL = ftgen.Workload("mixed_small", L=3, E=32, k=4, d=1024, d_ff=512, wtype=ftgen.W_NVFP4, cache_slots=64,
+                             bp_mbps=11800, bh_mbps=47500)
+
+
+def test_nvfp4_prefill_then_batched_decode(cuda_ok):
+    """Mixed-workload sequence at reduced size: NVFP4 prefill of every layer
+    (double buffer, C = 2E), then decode at batch 1..8 with Markov routing
+    biases on the shared cache, at the 11.8:47.5 profile."""
+    wl = NVFP4_SMALL
+    T = 300
+    with _harness(wl, max_tokens=T) as h:
+        oc = oracle_cache(h)
+        W = ExpertWeights(h, keep=40)
+        for l in range(wl.L):
+            x = gap_hidden(wl, T, wl.seed("pf", l), h.routers[l], None)
+            _call(h, oc, W, l, ft.FT_PREFILL, x, None, sample=[0, 7, T - 1])
+        steps = 5
+        traces = [ftgen.markov_trace(steps, 8, wl.E, wl.k, 0.8, 1.1, wl.seed("tr", l)) for l in range(wl.L)]
+        zb = [ftgen.zipf_log_bias(wl.E, 1.1, wl.seed("pi", l)) for l in range(wl.L)]
+        for st in range(steps):
+            B = (1, 2, 4, 8, 8)[st]
+            for l in range(wl.L):
+                bias = ftgen.trace_bias(traces[l][st][:B], zb[l], 8.0)
+                x = gap_hidden(wl, B, wl.seed("dec", st, l), h.routers[l], bias)
+                _call(h, oc, W, l, ft.FT_DECODE, x, bias, sample=list(range(B)) if st in (1, 4) else None)
+        _check_state(h, oc)
