@@ -8,7 +8,7 @@
 // kernel keeps many loads in flight and spends few instructions per byte.
 //
 // Work unit: 16 weight rows x one chunk of <= 16 tokens of one expert, done
-// by one CTA of 4 warps that split the unit's K range (split-K) and reduce
+// by one CTA of NW warps that split the unit's K range (split-K) and reduce
 // their partial sums in warp order through shared memory. Inside a warp,
 // lane (g, q) = (lane/4, lane%4) loads 16 consecutive bytes of rows g and
 // g+8 per step and hands them to the MMA unchanged as its A fragment; that
@@ -42,7 +42,6 @@ namespace ft {
 
 namespace {
 
-constexpr int WARPS = 4;  // warps per CTA; they split a unit's K range
 constexpr int CHUNK = 16;  // tokens per unit (two n8 tiles)
 constexpr long long WAIT_CYCLES = 4000000000ll;  // ~2 s
 
@@ -241,7 +240,7 @@ __device__ __forceinline__ bool unit_of(const int* pref, int n_items, int rblock
 
 // One unit: 16 weight rows x one chunk of <= 16 tokens, the K range split over
 // the 8 warps, partial sums reduced in warp order, epilogue by warp 0.
-template <int NB, int PHASE, bool FP4>
+template <int NB, int PHASE, bool FP4, int NW>
 __device__ void unit_work(const MmaArgs& a, const WorkItem& it, int chunk, int rb, int warp, int lane, float* red) {
   const int g = lane >> 2, q = lane & 3;
   const uint8_t* blob = blob_of(a, it);
@@ -250,7 +249,7 @@ __device__ void unit_work(const MmaArgs& a, const WorkItem& it, int chunk, int r
   const size_t rbytes = FP4 ? (size_t)K / 2 : (size_t)K * 2;
   const size_t sbytes = (size_t)K / 16;
   const int steps = FP4 ? K / 128 : K / 32;
-  const int s0 = (warp * steps) / WARPS, s1 = ((warp + 1) * steps) / WARPS;
+  const int s0 = (warp * steps) / NW, s1 = ((warp + 1) * steps) / NW;
   // rows g / g+8 of the tile: gate / up row rb*8+g (phase 0); down rows rb*16+g, +8 (phase 1)
   size_t oa, ob, sa0, sb0;
   if (PHASE == 0) {
@@ -301,7 +300,7 @@ __device__ void unit_work(const MmaArgs& a, const WorkItem& it, int chunk, int r
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         float v = red[(t * 4 + c) * 32 + lane];
-        for (int w = 1; w < WARPS; ++w) v += red[(w * NB * 4 + t * 4 + c) * 32 + lane];
+        for (int w = 1; w < NW; ++w) v += red[(w * NB * 4 + t * 4 + c) * 32 + lane];
         acc[t][c] = v;
       }
     // d0,d1: row g, tokens 2q, 2q+1; d2,d3: row g+8, same tokens (per n8 tile)
@@ -340,11 +339,11 @@ __device__ void unit_work(const MmaArgs& a, const WorkItem& it, int chunk, int r
   __syncthreads();  // red is reused by the next unit
 }
 
-template <int NB, bool FP4>
-__global__ void __launch_bounds__(WARPS * 32) gemv_fused_kernel(MmaArgs a) {
+template <int NB, bool FP4, int NW>
+__global__ void __launch_bounds__(NW * 32) gemv_fused_kernel(MmaArgs a) {
   __shared__ int s_pref[MAX_E + 1];
   __shared__ WorkItem s_items[MAX_E];
-  __shared__ float red[WARPS * NB * 4 * 32];
+  __shared__ float red[NW * NB * 4 * 32];
   __shared__ int s_unit;
   const int n_items = a.work->n_items[a.cls];
   if (n_items == 0) return;
@@ -399,9 +398,9 @@ __global__ void __launch_bounds__(WARPS * 32) gemv_fused_kernel(MmaArgs a) {
         __threadfence();
       }
       __syncthreads();
-      if (!bad) unit_work<NB, 1, FP4>(a, it, chunk, rb, warp, lane, red);
+      if (!bad) unit_work<NB, 1, FP4, NW>(a, it, chunk, rb, warp, lane, red);
     } else {
-      if (!bad) unit_work<NB, 0, FP4>(a, it, chunk, rb, warp, lane, red);
+      if (!bad) unit_work<NB, 0, FP4, NW>(a, it, chunk, rb, warp, lane, red);
       if (tid == 0) atomicAdd(a.done + qi, 1);
     }
     __syncthreads();  // every thread has read s_unit
@@ -415,14 +414,28 @@ __global__ void __launch_bounds__(256) to_f16_kernel(const __nv_bfloat16* __rest
   for (int i = blockIdx.x * 256 + threadIdx.x; i < n; i += gridDim.x * 256) y[i] = __float2half_rn(__bfloat162float(x[i]));
 }
 
+// Warps per CTA: up to 8 tokens per unit (small decode batches, single
+// staged experts) the work is short and 8 warps split K finer; at 9..16
+// tokens 4 warps per CTA give more CTAs per SM to overlap their stalls.
+template <int NB>
+constexpr int warps_for() { return NB == 1 ? 8 : 4; }
+
 int g_grid[2][3] = {{0, 0, 0}, {0, 0, 0}};  // [fp4][NB]
 
 template <int NB, bool FP4>
 cudaError_t kernel_setup(int sms) {
+  constexpr int NW = warps_for<NB>();
   int per = 0;
-  const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, gemv_fused_kernel<NB, FP4>, WARPS * 32, 0);
+  const cudaError_t e =
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, gemv_fused_kernel<NB, FP4, NW>, NW * 32, 0);
   g_grid[FP4][NB] = sms * (per > 0 ? per : 1);
   return e;
+}
+
+template <int NB, bool FP4>
+void launch_nb(int grid, const MmaArgs& a, cudaStream_t st) {
+  constexpr int NW = warps_for<NB>();
+  gemv_fused_kernel<NB, FP4, NW><<<grid, NW * 32, 0, st>>>(a);
 }
 
 }  // namespace
@@ -476,19 +489,21 @@ void launch_gemv_mma(const Shape& sh, int cls, int layer, const void* x16, int T
   const int NB = T > 8 ? 2 : 1;
   const long long chunks = (long long)max_items + (long long)max_tok / CHUNK;
   const long long units = chunks * (sh.d_ff / 8 + sh.d / 16);
-  // Streamed experts come over the host link: a few dozen CTAs reach its
-  // bandwidth best (fewer concurrent scattered streams into host memory) and
-  // leave the SMs to the HBM work of the hit and staged experts meanwhile.
+  // Streamed experts come over the host link: reads from host memory peak at
+  // about 128 warps in flight (more warps, more scattered streams, less
+  // bandwidth), which also leaves the SMs to the HBM work of the hit and
+  // staged experts running meanwhile.
   int cap = g_grid[fp4][NB];
-  if (cls == KIND_STREAMED && cap > 32) cap = 32;
+  const int stream_ctas = 128 / (NB == 1 ? warps_for<1>() : warps_for<2>());
+  if (cls == KIND_STREAMED && cap > stream_ctas) cap = stream_ctas;
   const int grid = (int)(units < cap ? units : cap);
   if (grid <= 0) return;
   if (fp4) {
-    if (NB == 1) gemv_fused_kernel<1, true><<<grid, WARPS * 32, 0, st>>>(a);
-    else gemv_fused_kernel<2, true><<<grid, WARPS * 32, 0, st>>>(a);
+    if (NB == 1) launch_nb<1, true>(grid, a, st);
+    else launch_nb<2, true>(grid, a, st);
   } else {
-    if (NB == 1) gemv_fused_kernel<1, false><<<grid, WARPS * 32, 0, st>>>(a);
-    else gemv_fused_kernel<2, false><<<grid, WARPS * 32, 0, st>>>(a);
+    if (NB == 1) launch_nb<1, false>(grid, a, st);
+    else launch_nb<2, false>(grid, a, st);
   }
 }
 
