@@ -207,7 +207,10 @@ def roofline(prof, peaks, peak_kind, link_gbs):
         if r["ms"] <= 0 or name == "h2d_stage_copies":
             continue
         gbs = r["bytes"] / (r["ms"] * 1e6)
-        if name.startswith("gemm_tc"):
+        # the binding roof is the larger of the HBM time and the tensor time
+        t_hbm = r["bytes"] / (peaks["hbm_gbs"] * 1e9)
+        t_tc = r["flops"] / (peaks["bf16_tflops"] * 1e12)
+        if name.startswith("gemm_tc") and t_tc > t_hbm:
             bound, peak, unit, ach = "tensor", peaks["bf16_tflops"], "TFLOP/s", r["flops"] / (r["ms"] * 1e9)
         elif name.endswith("streamed"):
             bound, peak, unit, ach = "host_link", link_gbs, "GB/s", gbs

@@ -41,6 +41,59 @@ __device__ __forceinline__ int block_scan_flag(bool f, ScanTmp& s, int& total) {
   return s.warp_tot[warp] + in_warp;
 }
 
+// Per-class ranks and totals of a class tag (0..2, or -1) over the 1024
+// threads in two barriers: rank of the thread among its class (in thread
+// order), and per class the count, a token sum and a chunk sum.
+struct Scan3Tmp {
+  int cnt[3][32], tok[3][32], ch[3][32], base[3][32];
+  int tot_cnt[3], tot_tok[3], tot_ch[3];
+};
+__device__ __forceinline__ int block_scan3(int cls, int tok, int ch, Scan3Tmp& s) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int in_warp = 0;
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    const unsigned b = __ballot_sync(0xffffffffu, cls == c);
+    if (cls == c) in_warp = __popc(b & ((1u << lane) - 1u));
+    int t = cls == c ? tok : 0, h = cls == c ? ch : 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      t += __shfl_xor_sync(0xffffffffu, t, o);
+      h += __shfl_xor_sync(0xffffffffu, h, o);
+    }
+    if (lane == 0) {
+      s.cnt[c][warp] = __popc(b);
+      s.tok[c][warp] = t;
+      s.ch[c][warp] = h;
+    }
+  }
+  __syncthreads();
+  if (warp < 3) {
+    const int c = warp;
+    const int v = s.cnt[c][lane];
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    s.base[c][lane] = incl - v;
+    int t = s.tok[c][lane], h = s.ch[c][lane];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      t += __shfl_xor_sync(0xffffffffu, t, o);
+      h += __shfl_xor_sync(0xffffffffu, h, o);
+    }
+    if (lane == 31) s.tot_cnt[c] = incl;
+    if (lane == 0) {
+      s.tot_tok[c] = t;
+      s.tot_ch[c] = h;
+    }
+  }
+  __syncthreads();
+  return cls >= 0 ? s.base[cls][warp] + in_warp : 0;
+}
+
 __device__ __forceinline__ unsigned long long slot_key(const unsigned long long* stamp, long long s,
                                                        unsigned long long epoch) {
   const unsigned long long st = stamp[s];
@@ -55,6 +108,7 @@ __device__ __forceinline__ void lookup_body(const LookupArgs& a, int E, long lon
   __shared__ unsigned long long s_cand[MAX_E];
   __shared__ int s_hist[256];
   __shared__ ScanTmp scan;
+  __shared__ Scan3Tmp scan3;
   __shared__ unsigned long long s_prefix, s_mask;
   __shared__ int s_remaining, s_ncand, s_avail;
   __shared__ unsigned long long s_c0, s_epoch, s_bstart;
@@ -84,10 +138,9 @@ __device__ __forceinline__ void lookup_body(const LookupArgs& a, int E, long lon
     }
   }
   const bool hit = act && sl >= 0;
-  int h;
-  const int hrank = block_scan_flag(hit, scan, h);
-  int m;
-  const int mrank = block_scan_flag(act && !hit, scan, m);
+  const int hm_rank = block_scan3(act ? (hit ? 0 : 1) : -1, 0, 0, scan3);
+  const int h = scan3.tot_cnt[0], m = scan3.tot_cnt[1];
+  const int hrank = hit ? hm_rank : 0, mrank = (act && !hit) ? hm_rank : 0;
 
   // 3. clock and pins
   if (tid == 0) {
@@ -133,7 +186,38 @@ __device__ __forceinline__ void lookup_body(const LookupArgs& a, int E, long lon
       q_stage = s_avail;
     }
   }
-  if (q_stage > 0) {
+  if (q_stage > 0 && q_stage <= 8) {
+    // a few victims: repeated arg-min over the keys above the previous pick
+    unsigned long long prev = 0;
+    for (int v = 0; v < q_stage; ++v) {
+      unsigned long long best = NOKEY;
+      for (long long sidx = tid; sidx < C; sidx += NT) {
+        const unsigned long long k = slot_key(ds.stamp, sidx, epoch);
+        if (k != NOKEY && (v == 0 || k > prev) && k < best) best = k;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long ob = __shfl_xor_sync(0xffffffffu, best, o);
+        best = ob < best ? ob : best;
+      }
+      if ((tid & 31) == 0) s_cand[tid >> 5] = best;
+      __syncthreads();
+      if (tid < 32) {
+        unsigned long long b2 = s_cand[tid];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const unsigned long long ob = __shfl_xor_sync(0xffffffffu, b2, o);
+          b2 = ob < b2 ? ob : b2;
+        }
+        if (tid == 0) {
+          s_prefix = b2;
+          s_vic[v] = (int)(b2 & ((1ull << SLOT_BITS) - 1));
+        }
+      }
+      __syncthreads();
+      prev = s_prefix;
+    }
+  } else if (q_stage > 0) {
     if (tid == 0) {
       s_prefix = 0;
       s_mask = 0;
@@ -204,39 +288,29 @@ __device__ __forceinline__ void lookup_body(const LookupArgs& a, int E, long lon
   __syncthreads();
   const int kind = hit ? KIND_HIT : (staged ? KIND_STAGED : KIND_STREAMED);
 
-  // 7. work lists of the routed experts, per class, ascending e
+  // 7. work lists of the routed experts, per class, ascending e, with the
+  // tensor-core GEMV scheduling state of each class (ticket and one
+  // completion counter per (item, 16-token chunk)) cleared
   if (a.build_work) {
+    const int tok = act ? ds.counts[e] : 0;
+    const int r = block_scan3(act ? kind : -1, tok, (tok + MMA_CHUNK - 1) / MMA_CHUNK, scan3);
+    if (act) {
+      WorkItem it;
+      it.e = e;
+      it.slot = s_slot[tid];
+      it.tok_off = ds.offsets[e];
+      it.n_tok = tok;
+      ds.work->items[kind][r] = it;
+    }
     for (int c = 0; c < N_CLASSES; ++c) {
-      int n_c;
-      const int r = block_scan_flag(act && kind == c, scan, n_c);
-      int tok = (act && kind == c) ? ds.counts[e] : 0;
-      for (int o = 16; o > 0; o >>= 1) tok += __shfl_xor_sync(0xffffffffu, tok, o);
-      if (tid == 0) s_tok = 0;
-      __syncthreads();
-      if ((tid & 31) == 0) atomicAdd(&s_tok, tok);
-      __syncthreads();
-      if (tid == 0) mb->n_tok_cls[c] = s_tok;
-      // tensor-core GEMV scheduling state of this class: ticket and one
-      // completion counter per (item, 16-token chunk)
-      int ch = (act && kind == c) ? (ds.counts[e] + MMA_CHUNK - 1) / MMA_CHUNK : 0;
-      for (int o = 16; o > 0; o >>= 1) ch += __shfl_xor_sync(0xffffffffu, ch, o);
-      if (tid == 0) s_chunks = 0;
-      __syncthreads();
-      if ((tid & 31) == 0) atomicAdd(&s_chunks, ch);
-      __syncthreads();
-      const int nch = s_chunks < ds.sched_chunks ? s_chunks : ds.sched_chunks;
+      const int nch = scan3.tot_ch[c] < ds.sched_chunks ? scan3.tot_ch[c] : ds.sched_chunks;
       int32_t* done = ds.sched + N_CLASSES + (size_t)c * ds.sched_chunks;
       for (int i = tid; i < nch; i += NT) done[i] = 0;
-      if (tid == 0) ds.sched[c] = 0;
-      if (act && kind == c) {
-        WorkItem it;
-        it.e = e;
-        it.slot = s_slot[tid];
-        it.tok_off = ds.offsets[e];
-        it.n_tok = ds.counts[e];
-        ds.work->items[c][r] = it;
-      }
-      if (tid == 0) ds.work->n_items[c] = n_c;
+    }
+    if (tid < N_CLASSES) {
+      ds.sched[tid] = 0;
+      ds.work->n_items[tid] = scan3.tot_cnt[tid];
+      mb->n_tok_cls[tid] = scan3.tot_tok[tid];
     }
   }
 
