@@ -71,6 +71,28 @@ def check_close(y_gpu, y_ref, wtype, what=""):
     return err / rms if rms > 0 else 0.0
 
 
+def check_route_weights(w_gpu, w_ref, x, w_router, what=""):
+    """Top-k softmax weights against the oracle's.
+
+    A logit is an fp32 dot product of length d. Whatever order the kernel
+    sums in (one FMA chain, or tensor-core k-groups), its rounding error stays
+    within the probabilistic bound sqrt(d) * u * sum_i |x_i W_ei|, u = 2^-24.
+    A weight exp(s_j - s_max) / sum is off, relative to itself, by at most
+    twice its token's largest logit error. That bound, per token, is the
+    tolerance; the selected ids are checked bit-exact separately."""
+    w_gpu = np.asarray(w_gpu, np.float64)
+    w_ref = np.asarray(w_ref, np.float64)
+    xa = np.abs(np.asarray(x, np.float64))
+    wa = np.abs(np.asarray(w_router, np.float64))
+    d = xa.shape[1]
+    bound = 2.0 * np.sqrt(d) * 2.0 ** -24 * (xa @ wa.T).max(axis=1)
+    err = np.abs(w_gpu - w_ref)
+    lim = bound[:, None] * w_ref + 1e-7
+    bad = np.argwhere(err > lim)
+    assert bad.size == 0, (f"{what}: {len(bad)} weights off, first (t, j) = {tuple(bad[0])}: "
+                           f"|d| {err[tuple(bad[0])]:.3e} > {lim[tuple(bad[0])]:.3e}")
+
+
 def gpu_route(harness, T):
     import sparse_moe_expert_topk_b200 as ft
     return ft.ft_moe_last_route(harness.ctx, harness.wl.E, T * harness.wl.k)

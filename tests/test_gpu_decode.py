@@ -9,7 +9,7 @@ import ftgen
 import sparse_moe_expert_topk_b200 as ft
 from oracle import moe as omoe
 from oracle.cache import DECODE
-from parity import (ExpertWeights, check_close, gap_hidden, gpu_route, oracle_cache, to_np)
+from parity import (ExpertWeights, check_close, check_route_weights, gap_hidden, gpu_route, oracle_cache, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -28,7 +28,7 @@ def _run_and_check(h, oc, W, layer, x, bias, check_y=True, mode=ft.FT_DECODE):
     xn = x.float().numpy()
     ids_ref, w_ref, _ = omoe.route(xn, h.routers[layer].float().cpu().numpy(), bias, wl.k)
     np.testing.assert_array_equal(ids.cpu().numpy(), ids_ref)
-    np.testing.assert_allclose(w.cpu().numpy(), w_ref, rtol=1e-5, atol=1e-6)
+    check_route_weights(w.cpu().numpy(), w_ref, xn, h.routers[layer].float().cpu().numpy(), f"layer {layer}")
     counts, offsets, perm, inv = omoe.permutation(ids_ref, wl.E)
     r = gpu_route(h, T)
     np.testing.assert_array_equal(r["counts"], counts)

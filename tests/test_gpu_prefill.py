@@ -12,7 +12,7 @@ import ftgen
 import sparse_moe_expert_topk_b200 as ft
 from oracle import moe as omoe
 from oracle.cache import DECODE, PREFILL
-from parity import ExpertWeights, check_close, gap_hidden, gpu_route, oracle_cache, to_np
+from parity import ExpertWeights, check_close, check_route_weights, gap_hidden, gpu_route, oracle_cache, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -32,7 +32,7 @@ def _call(h, oc, W, layer, mode, x, bias, sample=None):
     wr = h.routers[layer].float().cpu().numpy()
     ids_ref, w_ref, _ = omoe.route(xn, wr, bias, wl.k)
     np.testing.assert_array_equal(ids.cpu().numpy(), ids_ref)
-    np.testing.assert_allclose(w.cpu().numpy(), w_ref, rtol=1e-5, atol=1e-6)
+    check_route_weights(w.cpu().numpy(), w_ref, xn, wr, f"layer {layer}")
     counts, offsets, perm, inv = omoe.permutation(ids_ref, wl.E)
     r = gpu_route(h, T)
     np.testing.assert_array_equal(r["perm"], perm)
@@ -103,6 +103,28 @@ def test_multilayer_prefill_double_buffer_then_decode(cuda_ok, T):
         for l in range(wl.L):
             x = gap_hidden(wl, T, wl.seed("pf2", T, l), h.routers[l], None)
             _call(h, oc, W, l, ft.FT_PREFILL, x, None, sample=[1] if l == 1 else None)
+        _check_state(h, oc)
+
+
+def test_prefill_experts_spanning_several_token_tiles(cuda_ok):
+    """Skewed prefill (Zipf log-bias on the logits): the heaviest experts get
+    several hundred tokens each, more than one 256-token MMA tile, with a
+    ragged last tile. Outputs of tokens routed to the heaviest expert, its
+    first and last included, within 2e-2 rms."""
+    wl = SMALL
+    T = 2400
+    with _harness(wl, max_tokens=T) as h:
+        oc = oracle_cache(h)
+        W = ExpertWeights(h, keep=40)
+        bias = ftgen.zipf_log_bias(wl.E, 1.1, wl.seed("skew"))
+        x = gap_hidden(wl, T, wl.seed("skew-x"), h.routers[0], bias)
+        ids_ref, _, _ = omoe.route(x.float().numpy(), h.routers[0].float().cpu().numpy(), bias, wl.k)
+        counts = np.bincount(ids_ref.ravel(), minlength=wl.E)
+        heavy = int(np.argmax(counts))
+        assert counts[heavy] > 256
+        toks = np.nonzero((ids_ref == heavy).any(axis=1))[0]
+        sample = np.unique(np.concatenate([toks[:2], toks[255:258], toks[-2:]]))
+        _call(h, oc, W, 0, ft.FT_PREFILL, x, bias, sample=sample)
         _check_state(h, oc)
 
 
