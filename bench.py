@@ -432,6 +432,121 @@ def run_secondary(args, wl, world, rank, local):
         print(json.dumps(out), flush=True)
     return 0
 
+def run_mixed(args, wl, world, rank, local):
+    """43-layer mixed NVFP4 workload: a cold prefill of T = 8192 tokens through
+    every layer (layer-ahead double buffer), then decode steps at batch 1, 2,
+    4 and 8 (equal blocks) with Markov routing, for every cache capacity and
+    B_P:B_H profile of the sweep. One context serves the whole sweep: the slot
+    pool is resized between capacities (the host pool is filled once)."""
+    import dataclasses
+    import ftgen
+    import sparse_moe_expert_topk_b200 as ft
+    from ftgen.ctx import Harness
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    peaks, peak_kind = load_peaks()
+    L, E, k, d = wl.L, wl.E, wl.k, wl.d
+    ex = wl.extra
+    steps = min(wl.steps, int(os.environ.get("FT_MIXED_STEPS", 256)))
+    steps -= steps % len(wl.batches)
+    per_batch = steps // len(wl.batches)
+    Bmax = max(wl.batches)
+    caps = [int(f * L * E) for f in ex["cache_fracs"]]
+    T_pf = ex["prefill_T"]
+    h = Harness(dataclasses.replace(wl, cache_slots=caps[0]), max_tokens=T_pf, device=local)
+    # inputs: one prefill block reused by every layer (each layer routes it
+    # with its own router), decode activations and per-token trace biases
+    g = torch.Generator(device=device)
+    g.manual_seed(ftgen.subseed("mixed-x", rank))
+    x_pf = torch.randn(T_pf, d, generator=g, device=device).to(torch.bfloat16)
+    y_pf = torch.empty_like(x_pf)
+    x_dec = torch.randn(steps, L, Bmax, d, generator=g, device=device).to(torch.bfloat16)
+    y_dec = torch.empty(Bmax, d, dtype=torch.bfloat16, device=device)
+    zb = [ftgen.zipf_log_bias(E, ex["zipf_s"], wl.seed("pi", l)) for l in range(L)]
+    bias = np.empty((steps, L, Bmax, E), np.float32)
+    for l in range(L):
+        tr = ftgen.markov_trace(steps, Bmax, E, k, ex["p_reuse"], ex["zipf_s"], wl.seed("trace", rank, l))
+        for st in range(steps):
+            bias[st, l] = ftgen.trace_bias(tr[st], zb[l], ex["beta"])
+    bias = torch.from_numpy(bias).to(device)
+    h2d, zc = ft.ft_moe_probe_link(h.ctx, 1 << 30)
+    stream = h.stream
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def prefill():
+        for l in range(L):
+            ft.ft_moe_layer_forward(h.ctx, l, ft.FT_PREFILL, x_pf, T_pf, None, 0, y_pf)
+
+    def decode(st0, n, B):
+        for st in range(st0, st0 + n):
+            for l in range(L):
+                ft.ft_moe_layer_forward(h.ctx, l, ft.FT_DECODE, x_dec[st, l, :B], B, bias[st, l, :B], 1,
+                                        y_dec[:B])
+
+    def timed(fn, *a):
+        torch.cuda.synchronize(device)
+        e0.record(stream)
+        fn(*a)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        return e0.elapsed_time(e1)
+
+    # warm-up on the first point (kernels, events, pages)
+    ft.ft_set_bandwidths(h.ctx, *ex["profiles"][-1])
+    for _ in range(max(1, args.warmup - 2)):
+        ft.ft_moe_reset_cache(h.ctx)
+        prefill()
+        decode(0, min(4, per_batch), 1)
+    sweep = []
+    sampler = ClockSampler(local)
+    sampler.start()
+    for C in caps:
+        ft.ft_moe_resize_cache(h.ctx, C)
+        for bp, bh in ex["profiles"]:
+            ft.ft_moe_reset_cache(h.ctx)
+            ft.ft_set_bandwidths(h.ctx, bp, bh)
+            ms_pf = timed(prefill)
+            st_pf = h.stats()
+            row = {"cache_slots": C, "cache_frac": round(C / (L * E), 3), "bp_bh": f"{bp / 1000:.1f}:{bh / 1000:.1f}",
+                   "prefill": {"tokens_per_s": round(T_pf / (ms_pf / 1e3), 1), "ms_43_layers": round(ms_pf, 1),
+                               "link_gbs": round(st_pf["bytes_h2d"] / (ms_pf * 1e6), 2)},
+                   "decode": {}}
+            tok = 0
+            ms_dec = 0.0
+            for i, B in enumerate(wl.batches):
+                s0 = h.stats()
+                ms = timed(decode, i * per_batch, per_batch, B)
+                s1 = h.stats()
+                look = s1["lookups"] - s0["lookups"]
+                miss = s1["misses"] - s0["misses"]
+                link = (s1["bytes_h2d"] - s0["bytes_h2d"]) + (s1["bytes_zero_copy"] - s0["bytes_zero_copy"])
+                row["decode"][str(B)] = {"tokens_per_s": round(per_batch * B / (ms / 1e3), 2),
+                                         "ms_per_step": round(ms / per_batch, 3),
+                                         "miss_rate": round(miss / max(look, 1), 4),
+                                         "qstar_staged": s1["staged"] - s0["staged"],
+                                         "streamed": s1["streamed"] - s0["streamed"],
+                                         "link_gbs": round(link / (ms * 1e6), 2)}
+                tok += per_batch * B
+                ms_dec += ms
+            row["decode_tokens_per_s"] = round(tok / (ms_dec / 1e3), 2)
+            sweep.append(row)
+    clocks = sampler.stop()
+    h.close()
+    main_pt = next(r for r in sweep if r["cache_slots"] == int(0.37 * L * E) and r["bp_bh"] == "52.7:77.3")
+    out = {"metric": METRIC, "value": main_pt["decode_tokens_per_s"], "unit": UNIT, "n_gpus": world,
+           "steps": steps, "warmup": args.warmup, "ms_per_step": round(1e3 * sum(wl.batches) / len(wl.batches)
+                                                                      / main_pt["decode_tokens_per_s"], 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+           "config": {"workload": f"43-layer mixed NVFP4: cold prefill T={T_pf} then {steps} decode steps at batch "
+                                  f"1/2/4/8 ({per_batch} each), Markov p=0.8 + Zipf(1.1); value at 37% and 52.7:77.3",
+                      "pool_gb": round(L * E * wl.slot_bytes / 1e9, 1)},
+           "host_link": {"h2d_copy_gbs": round(h2d, 2), "zero_copy_read_gbs": round(zc, 2)},
+           "sweep": sweep, "clocks": clocks}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    return 0
+
+
 # --------------------------------------------------------------------------
 def main():
     ap = argparse.ArgumentParser()
@@ -453,8 +568,10 @@ def main():
     world, rank, local = dist_setup(args.gpus)
     if args.workload in ("prefill_bf16", "trace_nvfp4") and args.impl == "ours":
         return run_secondary(args, wl, world, rank, local)
+    if args.workload == "mixed_nvfp4" and args.impl == "ours":
+        return run_mixed(args, wl, world, rank, local)
     if args.workload != "decode_bf16":
-        raise SystemExit("workloads: decode_bf16 (default), prefill_bf16, trace_nvfp4")
+        raise SystemExit("workloads: decode_bf16 (default), prefill_bf16, trace_nvfp4, mixed_nvfp4")
     if args.impl == "reference":
         r = run_reference(args, wl, world, rank)
         if world > 1:

@@ -189,6 +189,24 @@ ft_status ft_set_bandwidths(ft_ctx* ctx, uint32_t bp_mbps, uint32_t bh_mbps);
 /* Empty the cache and zero the counters (cold start). Synchronises. */
 ft_status ft_moe_reset_cache(ft_ctx* ctx);
 
+/* Grow or shrink the HBM slot pool to new_slots at a safe point, without
+ * touching the host pool: the elastic memory manager of [techfeed]
+ * 弾性メモリ管理, which may hand expert-slot memory to the KV cache and take
+ * it back because what the cache holds never changes a result.
+ *   new_slots: 0 .. max(L*E, 2E), like ft_config.cache_slots.
+ * Rule: the min(new_slots, resident) most recently used entries survive with
+ * their stamps; a survivor whose slot index is below new_slots keeps its
+ * slot, the others move, in ascending order of their old slot, to the lowest
+ * free slots below new_slots; the LRU clock and the counters are kept; the
+ * prefill layer-ahead state is cleared (the next prefill call looks its own
+ * layer up again). Synchronises every stream of the context, allocates the
+ * new pool, copies the survivors device-to-device, then frees the old pool,
+ * so both pools exist for a moment.
+ * Errors: FT_EINVAL (range), FT_ENOMEM (the new pool or tables could not be
+ * allocated: the context is unchanged), FT_ESTATE / FT_ETIMEOUT (a device
+ * error is latched: nothing is done). */
+ft_status ft_moe_resize_cache(ft_ctx* ctx, int64_t new_slots);
+
 /* Routing and lookup record of the last forward call, copied to host arrays
  * (synchronises). Any pointer may be NULL.
  *   counts [E], offsets [E+1]: tokens per expert and their exclusive scan

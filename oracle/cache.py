@@ -17,7 +17,10 @@ What the pages fix:
   same slot pool, with two layers' worth of slots; with fewer slots it falls
   back to on-demand ([paperlens] "プレフィル: 全層ダブルバッファと「意味の錨」",
   paper §3.1);
-* the first request meets a cold, empty cache ([techfeed] "弾性メモリ管理").
+* the first request meets a cold, empty cache ([techfeed] "弾性メモリ管理");
+* the memory given to expert slots can grow or shrink at safe points without
+  reloading the model, which is correct because what the cache holds never
+  changes a result ([techfeed] "弾性メモリ管理").
 
 Readings taken where the pages are silent:
 * q* = floor((2 m B_P + B_H) / (2 B_H)) -- m B_P / B_H rounded half up, in
@@ -33,7 +36,12 @@ Readings taken where the pages are silent:
 * prefill with C >= 2E: a call for layer l loads layer l if the previous call
   did not already prefetch it, then prefetches layer l+1 (if l+1 < L), all E
   experts each, no q*; with C < 2E a prefill call follows the decode rules
-  for its routed experts; a call with T = 0 changes nothing.
+  for its routed experts; a call with T = 0 changes nothing;
+* a resize to C' slots between layer calls keeps the min(C', resident)
+  most recently stamped entries with their stamps; a survivor whose slot is
+  below C' stays there, the others move, in ascending order of their old
+  slot, to the lowest free slots below C'; the clock is kept and the
+  layer-ahead prefetch state is cleared.
 
 Pins (tests/test_oracle_cache.py): q* against the table derived from the
 pages' two B_P:B_H profiles (tests/golden/qstar_profiles.txt) and the bound
@@ -164,6 +172,27 @@ class ExpertCache:
         # every expert of this layer is resident now: all are read from slots
         return dict(lookups=look, kinds={e: HIT for e in routed}, m=m, qstar=-1, qstage=qs,
                     n_cur=n_cur)
+
+    # --- elastic capacity -------------------------------------------------
+    def resize(self, C_new: int):
+        """Change the capacity to C_new slots at a safe point (between calls)."""
+        res = [s for s in range(self.C) if self.key_of[s] >= 0]
+        res.sort(key=lambda s: -self.stamp[s])          # most recent first
+        keep = sorted(res[:C_new])                      # ascending old slot
+        key_of, stamp = [-1] * C_new, [0] * C_new
+        movers = []
+        for s in keep:
+            if s < C_new:
+                key_of[s], stamp[s] = self.key_of[s], self.stamp[s]
+            else:
+                movers.append(s)
+        free = [s for s in range(C_new) if key_of[s] < 0]
+        for s, t in zip(movers, free):
+            key_of[t], stamp[t] = self.key_of[s], self.stamp[s]
+        self.C = C_new
+        self.key_of, self.stamp = key_of, stamp
+        self.slot_of = {k: s for s, k in enumerate(key_of) if k >= 0}
+        self.prefetched = -1
 
     def contents(self):
         """(key_of [C], stamp [C]) as lists."""

@@ -27,7 +27,7 @@ KIND_HIT, KIND_STAGED, KIND_STREAMED = 0, 1, 2
 EXPORTS = (
     "ft_moe_slot_bytes", "ft_moe_init", "ft_moe_destroy", "ft_moe_expert_ptr", "ft_moe_set_tensor_scales",
     "ft_moe_set_router", "ft_moe_layer_forward", "ft_cache_stats", "ft_set_bandwidths", "ft_moe_reset_cache",
-    "ft_moe_last_route", "ft_moe_cache_contents", "ft_moe_probe_link", "ft_moe_profile", "ft_moe_profile_read",
+    "ft_moe_resize_cache", "ft_moe_last_route", "ft_moe_cache_contents", "ft_moe_probe_link", "ft_moe_profile", "ft_moe_profile_read",
     "ft_route_topk_static", "ft_status_str",
 )
 FT_ROUTE_STATIC_MAX_TOKENS = 1024
@@ -83,6 +83,7 @@ def lib() -> ctypes.CDLL:
             "ft_cache_stats": [P, ctypes.POINTER(FtStats)],
             "ft_set_bandwidths": [P, U32, U32],
             "ft_moe_reset_cache": [P],
+            "ft_moe_resize_cache": [P, ctypes.c_int64],
             "ft_moe_last_route": [P] + [P] * 11,
             "ft_moe_cache_contents": [P, P, P],
             "ft_moe_probe_link": [P, U64, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)],
@@ -178,6 +179,10 @@ def ft_set_bandwidths(ctx, bp_mbps, bh_mbps):
 
 def ft_moe_reset_cache(ctx):
     _check("ft_moe_reset_cache", lib().ft_moe_reset_cache(ctx))
+
+
+def ft_moe_resize_cache(ctx, new_slots):
+    _check("ft_moe_resize_cache", lib().ft_moe_resize_cache(ctx, int(new_slots)))
 
 
 def ft_moe_last_route(ctx, E, Tk):

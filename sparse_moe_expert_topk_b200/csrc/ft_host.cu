@@ -12,6 +12,7 @@
 // staged experts run once their copies land. Prefill call: the whole layer is
 // resident before it computes and the next layer is copied in behind it
 // ([paperlens] "プレフィル: 全層ダブルバッファと「意味の錨」", paper §3.1).
+#include <algorithm>
 #include <chrono>
 #include <cstdio>
 #include <cstdlib>
@@ -721,6 +722,127 @@ ft_status ft_moe_cache_contents(ft_ctx* c, int32_t* key_of, uint64_t* stamp) {
   if (c->sh.C == 0) return FT_OK;
   if (key_of) CK(cudaMemcpy(key_of, c->ds.key_of, sizeof(int32_t) * c->sh.C, cudaMemcpyDeviceToHost));
   if (stamp) CK(cudaMemcpy(stamp, c->ds.stamp, sizeof(uint64_t) * c->sh.C, cudaMemcpyDeviceToHost));
+  return FT_OK;
+}
+
+ft_status ft_moe_resize_cache(ft_ctx* c, int64_t new_slots) {
+  if (!c) return FT_EINVAL;
+  Shape& sh = c->sh;
+  DevState& d = c->ds;
+  const long long le = (long long)sh.L * sh.E, two = 2ll * sh.E;
+  if (new_slots < 0 || new_slots > (le > two ? le : two) || new_slots >= (1ll << 20)) return FT_EINVAL;
+  CK(cudaStreamSynchronize(c->s_copy));
+  CK(cudaStreamSynchronize(c->s_side));
+  CK(cudaStreamSynchronize(c->s_comp));
+  if (check_device_error(c) != FT_OK) return c->latched;
+  const long long C = sh.C, Cn = new_slots;
+  c->prefetched = -1;
+  if (Cn == C) return FT_OK;
+
+  // 1. what is resident now
+  std::vector<int32_t> key(C > 0 ? C : 1, -1);
+  std::vector<unsigned long long> stamp(C > 0 ? C : 1, 0);
+  if (C > 0) {
+    CK(cudaMemcpy(key.data(), d.key_of, sizeof(int32_t) * C, cudaMemcpyDeviceToHost));
+    CK(cudaMemcpy(stamp.data(), d.stamp, sizeof(unsigned long long) * C, cudaMemcpyDeviceToHost));
+  }
+  // 2. survivors: the Cn most recently used; they keep their slot when it
+  // still exists, else take the lowest free ones (ascending old slot)
+  std::vector<long long> res;
+  for (long long s = 0; s < C; ++s)
+    if (key[s] >= 0) res.push_back(s);
+  std::sort(res.begin(), res.end(), [&](long long a, long long b) { return stamp[a] > stamp[b]; });
+  if ((long long)res.size() > Cn) res.resize(Cn);
+  std::sort(res.begin(), res.end());
+  const size_t nC = Cn > 0 ? (size_t)Cn : 1;
+  std::vector<int32_t> nkey(nC, -1), slot_of((size_t)sh.L * sh.E, -1);
+  std::vector<unsigned long long> nstamp(nC, 0);
+  std::vector<std::pair<long long, long long>> moves;  // (old slot, new slot)
+  for (long long s : res)
+    if (s < Cn) moves.push_back({s, s}), nkey[s] = key[s], nstamp[s] = stamp[s];
+  long long t = 0;
+  for (long long s : res) {
+    if (s < Cn) continue;
+    while (nkey[t] >= 0) ++t;
+    moves.push_back({s, t});
+    nkey[t] = key[s];
+    nstamp[t] = stamp[s];
+  }
+  for (long long s = 0; s < Cn; ++s)
+    if (nkey[s] >= 0) slot_of[nkey[s]] = (int32_t)s;
+
+  // 3. new pool and tables; on any failure the context is left as it was
+  Shape shn = sh;
+  shn.C = Cn;
+  const bool tc_new = prefill_tc_supported(shn) && Cn >= 2ll * sh.E;
+  uint8_t* nslots = nullptr;
+  int32_t* nk = nullptr;
+  unsigned long long* ns = nullptr;
+  __nv_bfloat16 *nxs = nullptr, *nhs = nullptr;
+  const size_t Tk = (size_t)c->cfg.max_tokens * sh.k;
+  auto undo = [&]() {
+    void* ps[] = {nslots, nk, ns, nxs, nhs};
+    for (void* p : ps)
+      if (p) cudaFree(p);
+    cudaGetLastError();
+  };
+  bool ok = !fault("resize_alloc");
+  if (ok && Cn > 0) ok = cudaMalloc((void**)&nslots, sh.slot_bytes * (size_t)Cn) == cudaSuccess;
+  if (ok) ok = cudaMalloc((void**)&nk, sizeof(int32_t) * nC) == cudaSuccess;
+  if (ok) ok = cudaMalloc((void**)&ns, sizeof(unsigned long long) * nC) == cudaSuccess;
+  if (ok && tc_new && !d.xs) {
+    ok = cudaMalloc((void**)&nxs, sizeof(__nv_bfloat16) * (Tk + 256) * sh.d) == cudaSuccess &&
+         cudaMalloc((void**)&nhs, sizeof(__nv_bfloat16) * (Tk + 256) * sh.d_ff) == cudaSuccess;
+  }
+  if (!ok) {
+    undo();
+    return FT_ENOMEM;
+  }
+  // 4. survivors device-to-device, runs of consecutive slots in one copy each
+  std::sort(moves.begin(), moves.end());
+  cudaError_t ce = cudaSuccess;
+  for (size_t i = 0; i < moves.size() && ce == cudaSuccess;) {
+    size_t j = i + 1;
+    while (j < moves.size() && moves[j].first == moves[j - 1].first + 1 && moves[j].second == moves[j - 1].second + 1)
+      ++j;
+    ce = cudaMemcpyAsync(nslots + (size_t)moves[i].second * sh.slot_bytes, d.slots + (size_t)moves[i].first * sh.slot_bytes,
+                         (j - i) * sh.slot_bytes, cudaMemcpyDeviceToDevice, c->s_comp);
+    i = j;
+  }
+  if (ce == cudaSuccess)
+    ce = cudaMemcpyAsync(nk, nkey.data(), sizeof(int32_t) * nC, cudaMemcpyHostToDevice, c->s_comp);
+  if (ce == cudaSuccess)
+    ce = cudaMemcpyAsync(ns, nstamp.data(), sizeof(unsigned long long) * nC, cudaMemcpyHostToDevice, c->s_comp);
+  if (ce == cudaSuccess) ce = cudaStreamSynchronize(c->s_comp);
+  if (ce != cudaSuccess) {
+    cudaStreamSynchronize(c->s_comp);
+    undo();
+    fprintf(stderr, "ft_moe_resize_cache: %s\n", cudaGetErrorString(ce));
+    return FT_ECUDA;
+  }
+  // 5. commit
+  CK(cudaMemcpy(d.slot_of, slot_of.data(), sizeof(int32_t) * slot_of.size(), cudaMemcpyHostToDevice));
+  if (d.slots) cudaFree(d.slots);
+  cudaFree(d.key_of);
+  cudaFree(d.stamp);
+  d.slots = nslots;
+  d.key_of = nk;
+  d.stamp = ns;
+  sh.C = Cn;
+  c->cfg.cache_slots = Cn;
+  prefill_tc_free(d);
+  if (nxs) d.xs = nxs, d.hs = nhs;
+  if (!tc_new && d.xs) {
+    cudaFree(d.xs);
+    cudaFree(d.hs);
+    d.xs = d.hs = nullptr;
+  }
+  c->use_tc = tc_new;
+  if (tc_new && prefill_tc_init(sh, d, (int)Tk) != cudaSuccess) {
+    prefill_tc_free(d);
+    c->use_tc = false;  // prefill keeps working on the GEMV path
+    cudaGetLastError();
+  }
   return FT_OK;
 }
 

@@ -91,8 +91,9 @@ __device__ __forceinline__ void topk_token(const float* __restrict__ scores, int
     const int e = i * 32 + lane;
     v[i] = e < E ? __ldcg(s + e) : 0.f;  // L2: in the fused kernel other CTAs wrote these
   }
-  float top0 = 0.f, sel[MAX_K];
-  int sid[MAX_K];
+  // lane j keeps the j-th pick, so nothing is indexed by the runtime k
+  float top0 = 0.f, my_s = 0.f;
+  int my_e = 0;
   for (int j = 0; j < k; ++j) {
     float bv = 0.f;
     int be = 0x7fffffff;
@@ -117,20 +118,18 @@ __device__ __forceinline__ void topk_token(const float* __restrict__ scores, int
       }
     }
     if ((be & 31) == lane) taken |= 1u << (be >> 5);
-    sel[j] = bv;
-    sid[j] = be;
+    if (lane == j) {
+      my_s = bv;
+      my_e = be;
+    }
     if (j == 0) top0 = bv;
   }
-  float den = 0.f, ex[MAX_K];
-  for (int j = 0; j < k; ++j) {
-    ex[j] = expf(sel[j] - top0);
-    den += ex[j];
-  }
-  if (lane == 0) {
-    for (int j = 0; j < k; ++j) {
-      ids[(size_t)warp * k + j] = sid[j];
-      wts[(size_t)warp * k + j] = ex[j] / den;
-    }
+  const float ex = lane < k ? expf(my_s - top0) : 0.f;
+  float den = 0.f;
+  for (int j = 0; j < k; ++j) den += __shfl_sync(0xffffffffu, ex, j);  // rank order
+  if (lane < k) {
+    ids[(size_t)warp * k + lane] = my_e;
+    wts[(size_t)warp * k + lane] = ex / den;
   }
 }
 
@@ -272,22 +271,22 @@ __device__ void logits_bf16_block(const __nv_bfloat16* __restrict__ x, const __n
 #pragma unroll
       for (int c = 0; c < 4; ++c) red[(warp * 8 + t * 4 + c) * 32 + lane] = acc[t][c];
     __syncthreads();
-    if (warp == 0) {
-#pragma unroll
-      for (int t = 0; t < 2; ++t)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float v = red[(t * 4 + c) * 32 + lane];
-          for (int w = 1; w < 32; ++w) v += red[(w * 8 + t * 4 + c) * 32 + lane];
-          // d0,d1: expert e0+g, tokens 2q, 2q+1; d2,d3: expert e0+g+8
-          const int tok = t0 + t * 8 + 2 * q + (c & 1);
-          const int e = e0 + g + (c >> 1) * 8;
-          if (tok < T && t * 8 + 2 * q + (c & 1) < nt && e < E) {
-            float b = 0.f;
-            if (bias) b = bias_per_token ? bias[(size_t)tok * E + e] : bias[e];
-            scores[(size_t)tok * E + e] = v + b;
-          }
-        }
+    // thread i < 256 sums accumulator element i over the 32 warps, in warp order
+    const int n_out = nt > 8 ? 256 : 128;
+    if ((int)threadIdx.x < n_out) {
+      const int i = threadIdx.x, t = i >> 7, c = (i >> 5) & 3, l = i & 31;
+      float v = 0.f;
+#pragma unroll 8
+      for (int w = 0; w < 32; ++w) v += red[w * 256 + i];
+      // element c of lane l: c = 0,1 expert e0+g, tokens 2q, 2q+1; c = 2,3 expert e0+g+8
+      const int tt = t * 8 + 2 * (l & 3) + (c & 1);
+      const int tok = t0 + tt;
+      const int e = e0 + (l >> 2) + (c >> 1) * 8;
+      if (tt < nt && e < E) {
+        float b = 0.f;
+        if (bias) b = bias_per_token ? bias[(size_t)tok * E + e] : bias[e];
+        scores[(size_t)tok * E + e] = v + b;
+      }
     }
     __syncthreads();
   }

@@ -189,3 +189,76 @@ def test_empty_call_changes_nothing():
     c = cache.ExpertCache(1, 4, 2)
     rec = c.forward(0, DECODE, np.zeros(4, int))
     assert rec["lookups"] == [] and c.n["layer_calls"] == 0 and c.clock == 0
+
+
+@pytest.mark.parametrize("schedule", [(7, 3, 12, 5), (20, 1, 20), (4, 4, 9, 0, 6)])
+def test_resize_equals_truncated_textbook_lru(schedule):
+    """Elastic capacity: with one access per step, running segments of a trace
+    at capacities C_0, C_1, ... with a resize between them gives the same
+    hit/miss sequence as a move-to-front list that, on a shrink, drops its
+    least recently used entries down to the new capacity."""
+    L, E = 3, 8
+    rng = np.random.default_rng(sum(schedule))
+    segs = [[int(k) for k in _single_access_trace(300, L * E, rng)] for _ in schedule]
+    c = cache.ExpertCache(L, E, schedule[0], 1, 1)
+    lru = OrderedDict()
+    for i, (C, seg) in enumerate(zip(schedule, segs)):
+        if i:
+            before = dict(zip(*c.contents()))
+            old_slot = {k: s for s, k in enumerate(c.contents()[0]) if k >= 0}
+            c.resize(C)
+            while len(lru) > C:
+                lru.popitem(last=False)
+            key_of, stamp = c.contents()
+            assert len(key_of) == C
+            assert sorted(k for k in key_of if k >= 0) == sorted(lru)
+            for s, k in enumerate(key_of):
+                if k < 0:
+                    assert stamp[s] == 0
+                    continue
+                assert stamp[s] == before[k]                # stamps survive
+                if old_slot[k] < C:
+                    assert s == old_slot[k]                 # no needless move
+        for key in seg:
+            layer, e = divmod(key, E)
+            counts = np.zeros(E, int); counts[e] = 1
+            kind = c.forward(layer, DECODE, counts)["kinds"][e]
+            if key in lru:
+                lru.move_to_end(key)
+                assert kind == HIT
+            else:
+                assert kind == (STAGED if C > 0 else STREAMED)
+                if C > 0:
+                    if len(lru) >= C:
+                        lru.popitem(last=False)
+                    lru[key] = True
+
+
+def test_resize_moves_survivors_to_lowest_free_slots():
+    """Hand-worked shrink: 6 slots holding keys 10..15 with stamps
+    [5, 1, 6, 2, 4, 3] (slot 0..5) shrunk to 3 keeps the three most recent,
+    keys 12 (stamp 6, slot 2), 10 (stamp 5, slot 0) and 14 (stamp 4, slot 4);
+    12 and 10 stay, 14 moves to the only free slot below 3, slot 1."""
+    c = cache.ExpertCache(1, 16, 6)
+    c.key_of = [10, 11, 12, 13, 14, 15]
+    c.stamp = [5, 1, 6, 2, 4, 3]
+    c.slot_of = {k: s for s, k in enumerate(c.key_of)}
+    c.clock = 6
+    c.resize(3)
+    assert c.contents() == ([10, 14, 12], [5, 4, 6])
+    assert c.slot_of == {10: 0, 14: 1, 12: 2} and c.clock == 6
+    c.resize(5)
+    assert c.contents() == ([10, 14, 12, -1, -1], [5, 4, 6, 0, 0])
+
+
+def test_prefill_after_resize_reloads_its_layer():
+    """The layer-ahead state is cleared by a resize: the next prefill call
+    looks its own layer up again (hits for what survived)."""
+    L, E = 3, 4
+    c = cache.ExpertCache(L, E, 2 * E)
+    full = np.ones(E, int)
+    c.forward(0, PREFILL, full)            # loads 0, prefetches 1
+    c.resize(2 * E + 2)
+    rec = c.forward(1, PREFILL, full)
+    assert [k for (l, _, k) in rec["lookups"] if l == 1] == [HIT] * E
+    assert rec["n_cur"] == E
