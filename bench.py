@@ -392,7 +392,12 @@ def run_secondary(args, wl, world, rank, local):
                    host_link={"h2d_copy_gbs": round(h2d, 2), "zero_copy_read_gbs": round(zc, 2)},
                    roofline=roof, kernels=rows)
     else:  # trace_nvfp4: 43 layers, Markov routing realised as a per-token bias
-        L = wl.L
+        import dataclasses
+        # FT_TRACE_LAYERS < 43 runs the same per-layer shapes on a smaller pool
+        # (a few GB, for profiler captures); capacity stays 37% of the pool
+        L = min(wl.L, int(os.environ.get("FT_TRACE_LAYERS", wl.L)))
+        if L != wl.L:
+            wl = dataclasses.replace(wl, L=L, cache_slots=int(0.37 * L * wl.E))
         steps = min(wl.steps, int(os.environ.get("FT_TRACE_STEPS", wl.steps)))
         h = Harness(wl, max_tokens=1, device=local)
         traces = [ftgen.markov_trace(steps, 1, wl.E, wl.k, wl.extra["p_reuse"], wl.extra["zipf_s"],
@@ -420,9 +425,9 @@ def run_secondary(args, wl, world, rank, local):
         roof, rows = roofline(prof, peaks, peak_kind, h2d)
         h.close()
         out.update(value=round(steps / (ms / 1e3), 2), ms_per_step=round(ms / steps, 4), dtype="nvfp4",
-                   config={"workload": f"43-layer NVFP4 decode trace, batch 1, {steps} steps, Markov p=0.8 + "
-                                       "Zipf(1.1), shared LRU at 37% (4072 slots), 52.7:77.3"},
-                   tokens_per_s_43_layers=round(steps / (ms / 1e3), 2),
+                   config={"workload": f"{L}-layer NVFP4 decode trace, batch 1, {steps} steps, Markov p=0.8 + "
+                                       f"Zipf(1.1), shared LRU at 37% ({wl.cache_slots} slots), 52.7:77.3"},
+                   tokens_per_s_all_layers=round(steps / (ms / 1e3), 2),
                    layer_calls_per_s=round(steps * L / (ms / 1e3), 1),
                    miss_rate=round(stt["misses"] / max(stt["lookups"], 1), 4),
                    cache={k: stt[k] for k in ("lookups", "hits", "misses", "staged", "streamed")},

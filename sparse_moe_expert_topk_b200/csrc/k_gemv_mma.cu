@@ -178,45 +178,46 @@ __device__ __forceinline__ void dot_bf16(const uint8_t* ra, const uint8_t* rb, i
 }
 
 // NVFP4: steps of 128 K values (lane q covers K = 128 s + 32 q .. +32: 16
-// code bytes and one scale pair per row); eight MMAs per step and token tile.
-template <int NB, int U, bool P1>
+// code bytes and one scale pair per row); RT row tiles per step, the tiles
+// tstride code bytes (tsc scale pairs) apart, sharing one activation
+// fragment; eight MMAs per step, tile and token tile.
+template <int NB, int RT, bool P1>
 __device__ __forceinline__ void dot_nvfp4(const uint8_t* ra, const uint8_t* rb, const unsigned short* sa,
-                                          const unsigned short* sb, int s0, int s1, const uint16_t* const (&xr)[NB],
-                                          int q, float (&acc)[NB][4]) {
-  for (int s = s0; s < s1; s += U) {
-    uint4 wa[U], wb[U];
-    uint32_t ca[U], cb[U];
+                                          const unsigned short* sb, size_t tstride, size_t tsc, int s0, int s1,
+                                          const uint16_t* const (&xr)[NB], int q, float (&acc)[RT][NB][4]) {
+  for (int s = s0; s < s1; ++s) {
+    uint4 wa[RT], wb[RT];
+    uint32_t ca[RT], cb[RT];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int ss = s + u < s1 ? s + u : s1 - 1;
-      wa[u] = ld_stream(ra + (size_t)ss * 64);
-      wb[u] = ld_stream(rb + (size_t)ss * 64);
-      ca[u] = __ldg(sa + ss * 4);
-      cb[u] = __ldg(sb + ss * 4);
+    for (int r = 0; r < RT; ++r) {
+      wa[r] = ld_stream(ra + r * tstride + (size_t)s * 64);
+      wb[r] = ld_stream(rb + r * tstride + (size_t)s * 64);
+      ca[r] = __ldg(sa + r * tsc + s * 4);
+      cb[r] = __ldg(sb + r * tsc + s * 4);
+    }
+    uint32_t xh[NB][16];
+#pragma unroll
+    for (int t = 0; t < NB; ++t) {
+      const uint16_t* xp = xr[t] + s * 128 + q * 32;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const uint4 xv = P1 ? ld_cg(xp + 8 * v) : __ldg(reinterpret_cast<const uint4*>(xp) + v);
+        xh[t][4 * v] = xv.x;
+        xh[t][4 * v + 1] = xv.y;
+        xh[t][4 * v + 2] = xv.z;
+        xh[t][4 * v + 3] = xv.w;
+      }
     }
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      if (s + u < s1) {
-        uint32_t ha[16], hb[16];
-        decode_nvfp4(wa[u], ca[u], ha);
-        decode_nvfp4(wb[u], cb[u], hb);
+    for (int r = 0; r < RT; ++r) {
+      uint32_t ha[16], hb[16];
+      decode_nvfp4(wa[r], ca[r], ha);
+      decode_nvfp4(wb[r], cb[r], hb);
 #pragma unroll
-        for (int t = 0; t < NB; ++t) {
-          const uint16_t* xp = xr[t] + (s + u) * 128 + q * 32;
-          uint32_t xh[16];
+      for (int t = 0; t < NB; ++t)
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const uint4 xv = P1 ? ld_cg(xp + 8 * v) : __ldg(reinterpret_cast<const uint4*>(xp) + v);
-            xh[4 * v] = xv.x;
-            xh[4 * v + 1] = xv.y;
-            xh[4 * v + 2] = xv.z;
-            xh[4 * v + 3] = xv.w;
-          }
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            mma_f16(acc[t], ha[2 * j], hb[2 * j], ha[2 * j + 1], hb[2 * j + 1], xh[2 * j], xh[2 * j + 1]);
-        }
-      }
+        for (int j = 0; j < 8; ++j)
+          mma_f16(acc[r][t], ha[2 * j], hb[2 * j], ha[2 * j + 1], hb[2 * j + 1], xh[t][2 * j], xh[t][2 * j + 1]);
     }
   }
 }
@@ -238,9 +239,12 @@ __device__ __forceinline__ bool unit_of(const int* pref, int n_items, int rblock
   return true;
 }
 
-// One unit: 16 weight rows x one chunk of <= 16 tokens, the K range split over
-// the 8 warps, partial sums reduced in warp order, epilogue by warp 0.
-template <int NB, int PHASE, bool FP4, int NW>
+// One unit: RT tiles of 16 weight rows x one chunk of <= 16 tokens, the K
+// range split over the NW warps, partial sums reduced in warp order, epilogue
+// of tile r by warp r. Tile r of unit rb is row block rb*RT + r: gate rows
+// 8 (rb*RT + r) + g with the matching up rows (phase 0), down rows
+// 16 (rb*RT + r) + g and + 8 (phase 1).
+template <int NB, int PHASE, bool FP4, int NW, int RT>
 __device__ void unit_work(const MmaArgs& a, const WorkItem& it, int chunk, int rb, int warp, int lane, float* red) {
   const int g = lane >> 2, q = lane & 3;
   const uint8_t* blob = blob_of(a, it);
@@ -250,17 +254,18 @@ __device__ void unit_work(const MmaArgs& a, const WorkItem& it, int chunk, int r
   const size_t sbytes = (size_t)K / 16;
   const int steps = FP4 ? K / 128 : K / 32;
   const int s0 = (warp * steps) / NW, s1 = ((warp + 1) * steps) / NW;
-  // rows g / g+8 of the tile: gate / up row rb*8+g (phase 0); down rows rb*16+g, +8 (phase 1)
+  const int rows_per_tile = PHASE == 0 ? 8 : 16;  // per weight matrix
+  const int blk0 = rb * RT;                       // first row block of the unit
   size_t oa, ob, sa0, sb0;
   if (PHASE == 0) {
-    oa = (size_t)(rb * 8 + g) * rbytes;
-    ob = (FP4 ? n / 2 : n * 2) + (size_t)(rb * 8 + g) * rbytes;
-    sa0 = 3 * (n / 2) + (size_t)(rb * 8 + g) * sbytes;
-    sb0 = 3 * (n / 2) + n / 16 + (size_t)(rb * 8 + g) * sbytes;
+    oa = (size_t)(blk0 * 8 + g) * rbytes;
+    ob = (FP4 ? n / 2 : n * 2) + (size_t)(blk0 * 8 + g) * rbytes;
+    sa0 = 3 * (n / 2) + (size_t)(blk0 * 8 + g) * sbytes;
+    sb0 = 3 * (n / 2) + n / 16 + (size_t)(blk0 * 8 + g) * sbytes;
   } else {
-    oa = (FP4 ? n : n * 4) + (size_t)(rb * 16 + g) * rbytes;
+    oa = (FP4 ? n : n * 4) + (size_t)(blk0 * 16 + g) * rbytes;
     ob = oa + 8 * rbytes;
-    sa0 = 3 * (n / 2) + 2 * (n / 16) + (size_t)(rb * 16 + g) * sbytes;
+    sa0 = 3 * (n / 2) + 2 * (n / 16) + (size_t)(blk0 * 16 + g) * sbytes;
     sb0 = sa0 + 8 * sbytes;
   }
   const int base = it.tok_off + chunk * CHUNK;
@@ -279,29 +284,39 @@ __device__ void unit_work(const MmaArgs& a, const WorkItem& it, int chunk, int r
       xl[t] = FP4 ? xr[t] : a.h16lo + (size_t)pos * a.d_ff;
     }
   }
-  float acc[NB][4];
+  float acc[RT][NB][4];
 #pragma unroll
-  for (int t = 0; t < NB; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-  if constexpr (FP4)
-    dot_nvfp4<NB, 4, PHASE == 1>(blob + oa + q * 16, blob + ob + q * 16,
-                                 reinterpret_cast<const unsigned short*>(blob + sa0) + q,
-                                 reinterpret_cast<const unsigned short*>(blob + sb0) + q, s0, s1, xr, q, acc);
-  else
-    dot_bf16<NB, (NB == 1 ? 8 : 4), PHASE == 1>(blob + oa + q * 16, blob + ob + q * 16, s0, s1, xr, xl, q, acc);
-  // split-K reduction over the warps, in warp order
+  for (int r = 0; r < RT; ++r)
 #pragma unroll
-  for (int t = 0; t < NB; ++t)
+    for (int t = 0; t < NB; ++t) acc[r][t][0] = acc[r][t][1] = acc[r][t][2] = acc[r][t][3] = 0.f;
+  if constexpr (FP4) {
+    dot_nvfp4<NB, RT, PHASE == 1>(blob + oa + q * 16, blob + ob + q * 16,
+                                  reinterpret_cast<const unsigned short*>(blob + sa0) + q,
+                                  reinterpret_cast<const unsigned short*>(blob + sb0) + q,
+                                  (size_t)rows_per_tile * rbytes, (size_t)rows_per_tile * sbytes / 2, s0, s1, xr, q,
+                                  acc);
+  } else {
+    static_assert(FP4 || RT == 1, "BF16 units are one row tile");
+    dot_bf16<NB, (NB == 1 ? 8 : 4), PHASE == 1>(blob + oa + q * 16, blob + ob + q * 16, s0, s1, xr, xl, q, acc[0]);
+  }
+  // split-K reduction over the warps, in warp order; red is [NW][RT][NB][4][32]
 #pragma unroll
-    for (int c = 0; c < 4; ++c) red[(warp * NB * 4 + t * 4 + c) * 32 + lane] = acc[t][c];
+  for (int r = 0; r < RT; ++r)
+#pragma unroll
+    for (int t = 0; t < NB; ++t)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) red[(((warp * RT + r) * NB + t) * 4 + c) * 32 + lane] = acc[r][t][c];
   __syncthreads();
-  if (warp == 0) {
+  if (warp < RT) {
+    const int r = warp;
+    float v[NB][4];
 #pragma unroll
     for (int t = 0; t < NB; ++t)
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        float v = red[(t * 4 + c) * 32 + lane];
-        for (int w = 1; w < NW; ++w) v += red[(w * NB * 4 + t * 4 + c) * 32 + lane];
-        acc[t][c] = v;
+        float x = red[((r * NB + t) * 4 + c) * 32 + lane];
+        for (int w = 1; w < NW; ++w) x += red[(((w * RT + r) * NB + t) * 4 + c) * 32 + lane];
+        v[t][c] = x;
       }
     // d0,d1: row g, tokens 2q, 2q+1; d2,d3: row g+8, same tokens (per n8 tile)
     float t0 = 1.f, t1 = 1.f;
@@ -310,16 +325,17 @@ __device__ void unit_work(const MmaArgs& a, const WorkItem& it, int chunk, int r
       t0 = PHASE == 0 ? ts[0] : ts[2];
       t1 = PHASE == 0 ? ts[1] : ts[2];
     }
+    const int blk = blk0 + r;
 #pragma unroll
     for (int t = 0; t < NB; ++t) {
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         const int j = t * 8 + 2 * q + c;
         if (j >= nt) continue;
-        const float v0 = acc[t][c] * t0, v1 = acc[t][2 + c] * t1;
+        const float v0 = v[t][c] * t0, v1 = v[t][2 + c] * t1;
         if (PHASE == 0) {
           const float hv = v0 / (1.f + expf(-v0)) * v1;
-          const size_t o = (size_t)(base + j) * a.d_ff + rb * 8 + g;
+          const size_t o = (size_t)(base + j) * a.d_ff + blk * 8 + g;
           if constexpr (FP4) {
             a.h16[o] = __half_as_ushort(__float2half_rn(hv));
           } else {
@@ -329,8 +345,8 @@ __device__ void unit_work(const MmaArgs& a, const WorkItem& it, int chunk, int r
           }
         } else {
           float* yr = a.ybuf + (size_t)(base + j) * a.d;
-          yr[rb * 16 + g] = v0;
-          yr[rb * 16 + g + 8] = v1;
+          yr[blk * 16 + g] = v0;
+          yr[blk * 16 + g + 8] = v1;
         }
       }
     }
@@ -339,11 +355,18 @@ __device__ void unit_work(const MmaArgs& a, const WorkItem& it, int chunk, int r
   __syncthreads();  // red is reused by the next unit
 }
 
+// Row tiles per unit: NVFP4 rows are a quarter of the BF16 bytes, so a unit
+// takes four tiles to keep the loads in flight per warp and the per-unit
+// reduction and barriers amortised.
+template <bool FP4>
+constexpr int tiles_for() { return FP4 ? 4 : 1; }
+
 template <int NB, bool FP4, int NW>
 __global__ void __launch_bounds__(NW * 32) gemv_fused_kernel(MmaArgs a) {
+  constexpr int RT = tiles_for<FP4>();
   __shared__ int s_pref[MAX_E + 1];
   __shared__ WorkItem s_items[MAX_E];
-  __shared__ float red[NW * NB * 4 * 32];
+  __shared__ float red[NW * RT * NB * 4 * 32];
   __shared__ int s_unit;
   const int n_items = a.work->n_items[a.cls];
   if (n_items == 0) return;
@@ -368,7 +391,7 @@ __global__ void __launch_bounds__(NW * 32) gemv_fused_kernel(MmaArgs a) {
   }
   __syncthreads();
   const int n_qi = s_pref[n_items];
-  const int rb0 = a.d_ff / 8, rb1 = a.d / 16;
+  const int rb0 = a.d_ff / 8 / RT, rb1 = a.d / 16 / RT;
   const int U0 = n_qi * rb0, U1 = n_qi * rb1;
   if (tid == 0) s_unit = atomicAdd(a.ticket, 1);
   __syncthreads();
@@ -398,9 +421,9 @@ __global__ void __launch_bounds__(NW * 32) gemv_fused_kernel(MmaArgs a) {
         __threadfence();
       }
       __syncthreads();
-      if (!bad) unit_work<NB, 1, FP4, NW>(a, it, chunk, rb, warp, lane, red);
+      if (!bad) unit_work<NB, 1, FP4, NW, RT>(a, it, chunk, rb, warp, lane, red);
     } else {
-      if (!bad) unit_work<NB, 0, FP4, NW>(a, it, chunk, rb, warp, lane, red);
+      if (!bad) unit_work<NB, 0, FP4, NW, RT>(a, it, chunk, rb, warp, lane, red);
       if (tid == 0) atomicAdd(a.done + qi, 1);
     }
     __syncthreads();  // every thread has read s_unit
@@ -488,7 +511,7 @@ void launch_gemv_mma(const Shape& sh, int cls, int layer, const void* x16, int T
   const bool fp4 = sh.wtype == FT_W_NVFP4;
   const int NB = T > 8 ? 2 : 1;
   const long long chunks = (long long)max_items + (long long)max_tok / CHUNK;
-  const long long units = chunks * (sh.d_ff / 8 + sh.d / 16);
+  const long long units = chunks * (sh.d_ff / 8 + sh.d / 16) / (fp4 ? tiles_for<true>() : 1);
   // Streamed experts come over the host link: reads from host memory peak at
   // about 128 warps in flight (more warps, more scattered streams, less
   // bandwidth), which also leaves the SMs to the HBM work of the hit and
