@@ -610,8 +610,7 @@ def main():
 
     for _ in range(args.warmup):
         run_step(h, xs, bias, ys)
-    st0 = ft.ft_cache_stats(h.ctx)
-    launches0 = st0["kernel_launches"]
+    launches0 = ft.ft_cache_stats(h.ctx)["kernel_launches"]
     barrier(world)
     torch.cuda.synchronize(device)
     sampler = ClockSampler(local)
@@ -628,8 +627,10 @@ def main():
     st = ft.ft_cache_stats(h.ctx)
     launches = (st["kernel_launches"] - launches0) / args.steps
     # every miss byte crosses the host link once: staged blobs by the copy
-    # engine, streamed blobs by the GEMV's zero-copy reads
-    link_bytes = ((st["bytes_h2d"] - st0["bytes_h2d"]) + (st["bytes_zero_copy"] - st0["bytes_zero_copy"])) / args.steps
+    # engine, streamed blobs by the GEMV's zero-copy reads. A step starts from
+    # a cold cache (the reset zeroes the counters), so the counters after the
+    # last timed step are one step's bytes; every step replays the same trace.
+    link_bytes = st["bytes_h2d"] + st["bytes_zero_copy"]
     ms_max = max_over_ranks(ms, world, device)
     total_tokens = sum_over_ranks(tokens_per_step * args.steps, world, device)
     value = total_tokens / (ms_max / 1e3)
