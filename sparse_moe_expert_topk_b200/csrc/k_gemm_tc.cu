@@ -28,6 +28,7 @@
 #include <new>
 
 #include "ft_internal.cuh"
+#include "mbarrier.cuh"
 
 namespace ft {
 
@@ -51,45 +52,15 @@ constexpr int B_BYTES = MAX_N * BK * 2;    // 32 KB
 constexpr int STAGE_BYTES = 2 * A_BYTES + B_BYTES;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 constexpr int THREADS = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
-constexpr long long WAIT_CYCLES = 4000000000ll;  // ~2 s at 2 GHz
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait on an mbarrier phase. Returns false (and raises the CTA's
-// abort flag and the device error) if it does not complete in time or the
-// CTA already aborted.
+using mb::smem_u32;
+using mb::WAIT_CYCLES;
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) { mb::init(bar, count); }
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) { mb::expect_tx(bar, bytes); }
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) { mb::arrive(bar); }
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) { return mb::try_wait(bar, parity); }
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, uint32_t* err) {
-  const long long t0 = clock64();
-  for (uint32_t i = 0;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255) == 255) {
-      if (*abort) return false;
-      if (clock64() - t0 > WAIT_CYCLES) {
-        *abort = 1;
-        atomicExch(err, (uint32_t)DERR_TIMEOUT);
-        return false;
-      }
-    }
-  }
+  return mb::wait(bar, parity, abort, err);
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y) {

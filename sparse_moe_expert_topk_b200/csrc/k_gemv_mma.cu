@@ -7,16 +7,22 @@
 // か」が決まっていない", paper §2.2): every weight byte is read once, so the
 // kernel keeps many loads in flight and spends few instructions per byte.
 //
-// Work unit: 16 weight rows x one chunk of <= 16 tokens of one expert, done
-// by one CTA of NW warps that split the unit's K range (split-K) and reduce
-// their partial sums in warp order through shared memory. Inside a warp,
-// lane (g, q) = (lane/4, lane%4) loads 16 consecutive bytes of rows g and
-// g+8 per step and hands them to the MMA unchanged as its A fragment; that
-// fixes a lane-dependent order of the K positions, which a dot product does
-// not care about as long as the activations (B fragment) are loaded in the
-// same order. No shuffles, and the summation order is fixed by the code, so an
-// expert's result does not depend on where its weights were read from
-// ([paperlens] "設計: 2階建てのエキスパート記憶", paper §3.3).
+// Work unit: 16 weight rows x one chunk of <= 16 tokens of one expert. One
+// producer warp takes the units by atomic ticket and has the TMA engine copy
+// their weight rows (K slices of <= 2 KB per row, cp.async.bulk) into a
+// 4-stage shared-memory ring; eight MMA warps split each slice's K range
+// (split-K), accumulate over the unit's slices and reduce their partial sums in
+// warp order through shared memory. The ring decouples the bytes in flight
+// from registers, and every host read of a streamed expert is a large
+// contiguous request instead of scattered 64-byte fragments.
+//
+// Inside a warp, lane (g, q) = (lane/4, lane%4) reads 16 consecutive bytes of
+// rows g and g+8 per step and hands them to the MMA unchanged as its A
+// fragment; that fixes a lane-dependent order of the K positions, which a dot
+// product does not care about as long as the activations (B fragment) are
+// loaded in the same order. No shuffles, and the summation order is fixed by
+// the code, so an expert's result does not depend on where its weights were
+// read from ([paperlens] "設計: 2階建てのエキスパート記憶", paper §3.3).
 //
 // Phase 0 units (gate/up): tile rows 0..7 are gate rows f0..f0+7 and rows
 // 8..15 the matching up rows, so one lane holds gate and up of the same
@@ -27,9 +33,10 @@
 // Phase 1 units (down) of an (expert, chunk) start once all its phase-0 units
 // have published h: units are handed out in ticket order (gate/up tickets
 // first) and a down unit waits, bounded, on a per-chunk completion counter.
-// Tickets are only taken by running CTAs, so every unit a CTA waits for is
-// held by a running CTA that never waits itself: no deadlock whatever the
-// residency.
+// A CTA holds tickets in increasing order and finishes them in that order, so
+// when it waits on a down unit it holds no unfinished gate/up unit; every unit
+// waited for is held by a running CTA that does not wait: no deadlock whatever
+// the residency.
 //
 // NVFP4: 32 e2m1 codes per lane are converted to f16 pairs (cvt e2m1x2) and
 // multiplied by their e4m3 block scale (exact in f16); the per-matrix fp32
@@ -37,21 +44,23 @@
 #include <cuda_fp16.h>
 
 #include "ft_internal.cuh"
+#include "mbarrier.cuh"
 
 namespace ft {
 
 namespace {
 
 constexpr int CHUNK = 16;  // tokens per unit (two n8 tiles)
-constexpr long long WAIT_CYCLES = 4000000000ll;  // ~2 s
-
-__device__ __forceinline__ uint4 ld_stream(const void* p) {
-  uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
-}
+constexpr long long WAIT_CYCLES = mb::WAIT_CYCLES;
+constexpr int NW = 8;                            // MMA (consumer) warps
+constexpr int THREADS = (NW + 1) * 32;           // + one producer warp
+constexpr int NST = 4;                           // ring stages
+constexpr int ROWS = 16;                         // weight rows per unit / stage
+constexpr int SLICE = 2048;                      // max code bytes per row per stage
+constexpr int CODE_RS = SLICE + 16;              // smem row stride: rows start 4 banks apart
+constexpr int SC_RS = SLICE / 8 + 16;            // same for the NVFP4 block scales
+constexpr int STAGE_BYTES = ROWS * CODE_RS + ROWS * SC_RS;
+constexpr int RING_BYTES = NST * STAGE_BYTES;
 
 // L2-coherent load (for h, written by other CTAs of the same launch).
 __device__ __forceinline__ uint4 ld_cg(const void* p) {
@@ -138,86 +147,65 @@ __device__ __forceinline__ const uint8_t* blob_of(const MmaArgs& a, const WorkIt
   return a.slots + (size_t)it.slot * a.slot_bytes;
 }
 
-// One BF16 step: 8 K values of rows g and g+8 per lane, two MMAs per token
-// tile (and two more for the low part of h in phase 1).
-template <int NB, bool P1>
-__device__ __forceinline__ void bf16_step(const uint4 wa, const uint4 wb, const uint16_t* const (&xr)[NB],
-                                          const uint16_t* const (&xl)[NB], int e0, float (&acc)[NB][4]) {
-#pragma unroll
-  for (int t = 0; t < NB; ++t) {
-    const uint4 xv = P1 ? ld_cg(xr[t] + e0) : __ldg(reinterpret_cast<const uint4*>(xr[t] + e0));
-    mma_bf16(acc[t], wa.x, wb.x, wa.y, wb.y, xv.x, xv.y);
-    mma_bf16(acc[t], wa.z, wb.z, wa.w, wb.w, xv.z, xv.w);
-    if constexpr (P1) {
-      const uint4 xo = ld_cg(xl[t] + e0);
-      mma_bf16(acc[t], wa.x, wb.x, wa.y, wb.y, xo.x, xo.y);
-      mma_bf16(acc[t], wa.z, wb.z, wa.w, wb.w, xo.z, xo.w);
-    }
-  }
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 r;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(addr));
+  return r;
 }
-
-// acc[t][.] += W[rows g, g+8] . X[tokens] over steps [s0, s1) of 32 K values
-// (lane q covers K = 32 s + 8 q .. +8). U steps of loads in flight; steps past
-// s1 reload the last step and are not used.
-template <int NB, int U, bool P1>
-__device__ __forceinline__ void dot_bf16(const uint8_t* ra, const uint8_t* rb, int s0, int s1,
-                                         const uint16_t* const (&xr)[NB], const uint16_t* const (&xl)[NB], int q,
-                                         float (&acc)[NB][4]) {
-  for (int s = s0; s < s1; s += U) {
-    uint4 wa[U], wb[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int ss = s + u < s1 ? s + u : s1 - 1;
-      wa[u] = ld_stream(ra + (size_t)ss * 64);
-      wb[u] = ld_stream(rb + (size_t)ss * 64);
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u)
-      if (s + u < s1) bf16_step<NB, P1>(wa[u], wb[u], xr, xl, (s + u) * 32 + q * 8, acc);
-  }
+__device__ __forceinline__ uint32_t lds16(uint32_t addr) {
+  unsigned short r;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(r) : "r"(addr));
+  return r;
 }
+// Barrier among the MMA warps only (the producer warp runs on its own).
+__device__ __forceinline__ void mma_warps_sync() { asm volatile("bar.sync 1, %0;" ::"r"(NW * 32) : "memory"); }
 
-// NVFP4: steps of 128 K values (lane q covers K = 128 s + 32 q .. +32: 16
-// code bytes and one scale pair per row); RT row tiles per step, the tiles
-// tstride code bytes (tsc scale pairs) apart, sharing one activation
-// fragment; eight MMAs per step, tile and token tile.
-template <int NB, int RT, bool P1>
-__device__ __forceinline__ void dot_nvfp4(const uint8_t* ra, const uint8_t* rb, const unsigned short* sa,
-                                          const unsigned short* sb, size_t tstride, size_t tsc, int s0, int s1,
-                                          const uint16_t* const (&xr)[NB], int q, float (&acc)[RT][NB][4]) {
+// acc[t] += rows g, g+8 of one stage . X over this warp's steps [s0, s1) of
+// the stage; step s covers 64 code bytes of each row (32 bf16 / 128 e2m1
+// values), lane q its 16-byte quarter; kb = first global step of the stage.
+// The activation rows xr / xl (h hi / lo parts for BF16 down units) are read
+// in the same lane-permuted K order.
+template <int NB, bool FP4, bool P1>
+__device__ __forceinline__ void stage_dot(uint32_t code, uint32_t sc, int s0, int s1, int kb,
+                                          const uint16_t* const (&xr)[NB], const uint16_t* const (&xl)[NB], int g,
+                                          int q, float (&acc)[NB][4]) {
+  const uint32_t ra = code + g * CODE_RS + q * 16, rb = ra + 8 * CODE_RS;
   for (int s = s0; s < s1; ++s) {
-    uint4 wa[RT], wb[RT];
-    uint32_t ca[RT], cb[RT];
-#pragma unroll
-    for (int r = 0; r < RT; ++r) {
-      wa[r] = ld_stream(ra + r * tstride + (size_t)s * 64);
-      wb[r] = ld_stream(rb + r * tstride + (size_t)s * 64);
-      ca[r] = __ldg(sa + r * tsc + s * 4);
-      cb[r] = __ldg(sb + r * tsc + s * 4);
-    }
-    uint32_t xh[NB][16];
-#pragma unroll
-    for (int t = 0; t < NB; ++t) {
-      const uint16_t* xp = xr[t] + s * 128 + q * 32;
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        const uint4 xv = P1 ? ld_cg(xp + 8 * v) : __ldg(reinterpret_cast<const uint4*>(xp) + v);
-        xh[t][4 * v] = xv.x;
-        xh[t][4 * v + 1] = xv.y;
-        xh[t][4 * v + 2] = xv.z;
-        xh[t][4 * v + 3] = xv.w;
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < RT; ++r) {
+    const uint4 wa = lds128(ra + s * 64), wb = lds128(rb + s * 64);
+    if constexpr (FP4) {
+      const uint32_t ca = lds16(sc + g * SC_RS + s * 8 + q * 2), cb = lds16(sc + (g + 8) * SC_RS + s * 8 + q * 2);
       uint32_t ha[16], hb[16];
-      decode_nvfp4(wa[r], ca[r], ha);
-      decode_nvfp4(wb[r], cb[r], hb);
+      decode_nvfp4(wa, ca, ha);
+      decode_nvfp4(wb, cb, hb);
 #pragma unroll
-      for (int t = 0; t < NB; ++t)
+      for (int t = 0; t < NB; ++t) {
+        const uint16_t* xp = xr[t] + (kb + s) * 128 + q * 32;
+        uint32_t xh[16];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint4 xv = P1 ? ld_cg(xp + 8 * v) : __ldg(reinterpret_cast<const uint4*>(xp) + v);
+          xh[4 * v] = xv.x;
+          xh[4 * v + 1] = xv.y;
+          xh[4 * v + 2] = xv.z;
+          xh[4 * v + 3] = xv.w;
+        }
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-          mma_f16(acc[r][t], ha[2 * j], hb[2 * j], ha[2 * j + 1], hb[2 * j + 1], xh[t][2 * j], xh[t][2 * j + 1]);
+          mma_f16(acc[t], ha[2 * j], hb[2 * j], ha[2 * j + 1], hb[2 * j + 1], xh[2 * j], xh[2 * j + 1]);
+      }
+    } else {
+      const int e0 = (kb + s) * 32 + q * 8;
+#pragma unroll
+      for (int t = 0; t < NB; ++t) {
+        const uint4 xv = P1 ? ld_cg(xr[t] + e0) : __ldg(reinterpret_cast<const uint4*>(xr[t] + e0));
+        mma_bf16(acc[t], wa.x, wb.x, wa.y, wb.y, xv.x, xv.y);
+        mma_bf16(acc[t], wa.z, wb.z, wa.w, wb.w, xv.z, xv.w);
+        if constexpr (P1) {
+          const uint4 xo = ld_cg(xl[t] + e0);
+          mma_bf16(acc[t], wa.x, wb.x, wa.y, wb.y, xo.x, xo.y);
+          mma_bf16(acc[t], wa.z, wb.z, wa.w, wb.w, xo.z, xo.w);
+        }
+      }
     }
   }
 }
@@ -239,139 +227,122 @@ __device__ __forceinline__ bool unit_of(const int* pref, int n_items, int rblock
   return true;
 }
 
-// One unit: RT tiles of 16 weight rows x one chunk of <= 16 tokens, the K
-// range split over the NW warps, partial sums reduced in warp order, epilogue
-// of tile r by warp r. Tile r of unit rb is row block rb*RT + r: gate rows
-// 8 (rb*RT + r) + g with the matching up rows (phase 0), down rows
-// 16 (rb*RT + r) + g and + 8 (phase 1).
-template <int NB, int PHASE, bool FP4, int NW, int RT>
-__device__ void unit_work(const MmaArgs& a, const WorkItem& it, int chunk, int rb, int warp, int lane, float* red) {
-  const int g = lane >> 2, q = lane & 3;
-  const uint8_t* blob = blob_of(a, it);
-  const size_t n = (size_t)a.d * a.d_ff;
-  const int K = PHASE == 0 ? a.d : a.d_ff;
-  const size_t rbytes = FP4 ? (size_t)K / 2 : (size_t)K * 2;
-  const size_t sbytes = (size_t)K / 16;
-  const int steps = FP4 ? K / 128 : K / 32;
-  const int s0 = (warp * steps) / NW, s1 = ((warp + 1) * steps) / NW;
-  const int rows_per_tile = PHASE == 0 ? 8 : 16;  // per weight matrix
-  const int blk0 = rb * RT;                       // first row block of the unit
-  size_t oa, ob, sa0, sb0;
-  if (PHASE == 0) {
-    oa = (size_t)(blk0 * 8 + g) * rbytes;
-    ob = (FP4 ? n / 2 : n * 2) + (size_t)(blk0 * 8 + g) * rbytes;
-    sa0 = 3 * (n / 2) + (size_t)(blk0 * 8 + g) * sbytes;
-    sb0 = 3 * (n / 2) + n / 16 + (size_t)(blk0 * 8 + g) * sbytes;
-  } else {
-    oa = (FP4 ? n : n * 4) + (size_t)(blk0 * 16 + g) * rbytes;
-    ob = oa + 8 * rbytes;
-    sa0 = 3 * (n / 2) + 2 * (n / 16) + (size_t)(blk0 * 16 + g) * sbytes;
-    sb0 = sa0 + 8 * sbytes;
-  }
-  const int base = it.tok_off + chunk * CHUNK;
-  const int nt = min(CHUNK, it.n_tok - chunk * CHUNK);
-  const uint16_t* xr[NB];
-  const uint16_t* xl[NB];
-#pragma unroll
-  for (int t = 0; t < NB; ++t) {
-    const int j = t * 8 + g;
-    const int pos = base + (j < nt ? j : 0);
-    if (PHASE == 0) {
-      xr[t] = reinterpret_cast<const uint16_t*>(a.x) + (size_t)(a.perm[pos] / a.k) * a.d;
-      xl[t] = xr[t];
-    } else {
-      xr[t] = a.h16 + (size_t)pos * a.d_ff;
-      xl[t] = FP4 ? xr[t] : a.h16lo + (size_t)pos * a.d_ff;
-    }
-  }
-  float acc[RT][NB][4];
-#pragma unroll
-  for (int r = 0; r < RT; ++r)
-#pragma unroll
-    for (int t = 0; t < NB; ++t) acc[r][t][0] = acc[r][t][1] = acc[r][t][2] = acc[r][t][3] = 0.f;
-  if constexpr (FP4) {
-    dot_nvfp4<NB, RT, PHASE == 1>(blob + oa + q * 16, blob + ob + q * 16,
-                                  reinterpret_cast<const unsigned short*>(blob + sa0) + q,
-                                  reinterpret_cast<const unsigned short*>(blob + sb0) + q,
-                                  (size_t)rows_per_tile * rbytes, (size_t)rows_per_tile * sbytes / 2, s0, s1, xr, q,
-                                  acc);
-  } else {
-    static_assert(FP4 || RT == 1, "BF16 units are one row tile");
-    dot_bf16<NB, (NB == 1 ? 8 : 4), PHASE == 1>(blob + oa + q * 16, blob + ob + q * 16, s0, s1, xr, xl, q, acc[0]);
-  }
-  // split-K reduction over the warps, in warp order; red is [NW][RT][NB][4][32]
-#pragma unroll
-  for (int r = 0; r < RT; ++r)
-#pragma unroll
-    for (int t = 0; t < NB; ++t)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) red[(((warp * RT + r) * NB + t) * 4 + c) * 32 + lane] = acc[r][t][c];
-  __syncthreads();
-  if (warp < RT) {
-    const int r = warp;
-    float v[NB][4];
-#pragma unroll
-    for (int t = 0; t < NB; ++t)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float x = red[((r * NB + t) * 4 + c) * 32 + lane];
-        for (int w = 1; w < NW; ++w) x += red[(((w * RT + r) * NB + t) * 4 + c) * 32 + lane];
-        v[t][c] = x;
-      }
-    // d0,d1: row g, tokens 2q, 2q+1; d2,d3: row g+8, same tokens (per n8 tile)
-    float t0 = 1.f, t1 = 1.f;
-    if constexpr (FP4) {
-      const float* ts = a.tscale + ((size_t)a.layer * a.E + it.e) * 3;
-      t0 = PHASE == 0 ? ts[0] : ts[2];
-      t1 = PHASE == 0 ? ts[1] : ts[2];
-    }
-    const int blk = blk0 + r;
-#pragma unroll
-    for (int t = 0; t < NB; ++t) {
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int j = t * 8 + 2 * q + c;
-        if (j >= nt) continue;
-        const float v0 = v[t][c] * t0, v1 = v[t][2 + c] * t1;
-        if (PHASE == 0) {
-          const float hv = v0 / (1.f + expf(-v0)) * v1;
-          const size_t o = (size_t)(base + j) * a.d_ff + blk * 8 + g;
-          if constexpr (FP4) {
-            a.h16[o] = __half_as_ushort(__float2half_rn(hv));
-          } else {
-            const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
-            a.h16[o] = __bfloat16_as_ushort(hi);
-            a.h16lo[o] = __bfloat16_as_ushort(__float2bfloat16_rn(hv - __bfloat162float(hi)));
-          }
-        } else {
-          float* yr = a.ybuf + (size_t)(base + j) * a.d;
-          yr[blk * 16 + g] = v0;
-          yr[blk * 16 + g + 8] = v1;
-        }
-      }
-    }
-    if (PHASE == 0) __threadfence();  // publish h before the unit is counted done
-  }
-  __syncthreads();  // red is reused by the next unit
+// Row geometry of a phase: 64-byte steps per row and how they are cut into
+// ring slices of <= SLICE bytes (an even number of steps, so an NVFP4
+// slice's scales are a multiple of 16 bytes).
+struct Geo {
+  int steps, nsl, ss;       // steps per row, slices, steps per slice (last may be shorter)
+  size_t row_bytes, sc_row; // code / scale bytes per row
+};
+__device__ __forceinline__ Geo geo_of(const MmaArgs& a, int phase, bool fp4) {
+  Geo g;
+  const int K = phase == 0 ? a.d : a.d_ff;
+  g.row_bytes = fp4 ? (size_t)K / 2 : (size_t)K * 2;
+  g.sc_row = fp4 ? (size_t)K / 16 : 0;
+  g.steps = (int)(g.row_bytes / 64);
+  g.nsl = (int)((g.row_bytes + SLICE - 1) / SLICE);
+  g.ss = (g.steps + g.nsl - 1) / g.nsl;
+  g.ss += g.ss & 1;
+  return g;
 }
 
-// Row tiles per unit: NVFP4 rows are a quarter of the BF16 bytes, so a unit
-// takes four tiles to keep the loads in flight per warp and the per-unit
-// reduction and barriers amortised.
-template <bool FP4>
-constexpr int tiles_for() { return FP4 ? 4 : 1; }
+struct StageMeta {
+  int u, slice, flags;
+};
+constexpr int SM_FIRST = 1, SM_LAST = 2, SM_BAD = 4, SM_END = 8;
 
-template <int NB, bool FP4, int NW>
-__global__ void __launch_bounds__(NW * 32) gemv_fused_kernel(MmaArgs a) {
-  constexpr int RT = tiles_for<FP4>();
+// Producer: one lane takes tickets and fills the ring.
+template <bool FP4>
+__device__ void produce(const MmaArgs& a, const WorkItem* items, const int* pref, int n_items, int rb0, int rb1,
+                        int U0, int U1, uint8_t* ring, volatile StageMeta* meta, uint32_t full, uint32_t empty,
+                        volatile int* abort) {
+  const size_t n = (size_t)a.d * a.d_ff;
+  const size_t mat = FP4 ? n / 2 : n * 2;          // code bytes per matrix
+  const size_t sc0 = 3 * (n / 2), scm = n / 16;     // NVFP4 scales: start, bytes per matrix
+  int it = 0;
+  int last_round[NST];
+#pragma unroll
+  for (int i = 0; i < NST; ++i) last_round[i] = -1;
+  for (bool done = false; !done;) {
+    const int u = atomicAdd(a.ticket, 1);
+    if (u >= U0 + U1) {  // end of work: one sentinel stage
+      const int slot = it % NST, r = it / NST;
+      if (mb::wait(empty + 8 * slot, (r & 1) ^ 1, abort, a.error)) {
+        meta[slot].flags = SM_END;
+        mb::arrive(full + 8 * slot);
+      }
+      break;
+    }
+    const int phase = u < U0 ? 0 : 1;
+    int item, chunk, rb, qi;
+    unit_of(pref, n_items, phase == 0 ? rb0 : rb1, phase == 0 ? u : u - U0, item, chunk, rb, qi);
+    const WorkItem wi = items[item];
+    const bool bad = a.cls != KIND_STREAMED && (wi.slot < 0 || wi.slot >= a.C);  // error already latched
+    const uint8_t* blob = bad ? nullptr : blob_of(a, wi);
+    const Geo g = geo_of(a, phase, FP4);
+    for (int sl = 0; sl < g.nsl; ++sl, ++it) {
+      const int slot = it % NST, r = it / NST;
+      if (!mb::wait(empty + 8 * slot, (r & 1) ^ 1, abort, a.error)) {
+        done = true;
+        break;
+      }
+      meta[slot].u = u;
+      meta[slot].slice = sl;
+      meta[slot].flags = (sl == 0 ? SM_FIRST : 0) | (sl == g.nsl - 1 ? SM_LAST : 0) | (bad ? SM_BAD : 0);
+      const uint32_t bar = full + 8 * slot;
+      if (bad) {
+        mb::arrive(bar);
+        continue;
+      }
+      const int s0 = sl * g.ss, ns = min(g.ss, g.steps - s0);
+      const uint32_t cb = (uint32_t)ns * 64, sb = FP4 ? (uint32_t)ns * 8 : 0;
+      mb::expect_tx(bar, ROWS * (cb + sb));
+      const uint32_t code = mb::smem_u32(ring + slot * STAGE_BYTES), scs = code + ROWS * CODE_RS;
+#pragma unroll 1
+      for (int i = 0; i < ROWS; ++i) {
+        // smem row i: phase 0 -> gate row 8 rb + i (i < 8) or up row 8 rb + i - 8; phase 1 -> down row 16 rb + i
+        size_t m, row;
+        if (phase == 0) {
+          m = i < 8 ? 0 : 1;
+          row = (size_t)rb * 8 + (i & 7);
+        } else {
+          m = 2;
+          row = (size_t)rb * 16 + i;
+        }
+        mb::bulk_g2s(code + i * CODE_RS, blob + m * mat + row * g.row_bytes + (size_t)s0 * 64, cb, bar);
+        if (FP4) mb::bulk_g2s(scs + i * SC_RS, blob + sc0 + m * scm + row * g.sc_row + (size_t)s0 * 8, sb, bar);
+      }
+      last_round[slot] = r;
+    }
+  }
+  // every copy issued must have landed before the CTA's shared memory goes away
+#pragma unroll
+  for (int i = 0; i < NST; ++i)
+    if (last_round[i] >= 0) mb::wait_quiet(full + 8 * i, last_round[i] & 1, WAIT_CYCLES / 4);
+}
+
+template <int NB, bool FP4>
+__global__ void __launch_bounds__(THREADS, 1) gemv_fused_kernel(MmaArgs a) {
+  extern __shared__ __align__(128) uint8_t ring[];
   __shared__ int s_pref[MAX_E + 1];
   __shared__ WorkItem s_items[MAX_E];
-  __shared__ float red[NW * RT * NB * 4 * 32];
-  __shared__ int s_unit;
+  __shared__ float red[NW * NB * 4 * 32];
+  __shared__ StageMeta meta[NST];
+  __shared__ __align__(8) uint64_t bars[2 * NST];
+  __shared__ int s_abort, s_go[2];
   const int n_items = a.work->n_items[a.cls];
   if (n_items == 0) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int i = tid; i < n_items; i += blockDim.x) s_items[i] = a.work->items[a.cls][i];
+  const uint32_t full = mb::smem_u32(bars), empty = full + 8 * NST;
+  if (tid == 0) {
+    s_abort = 0;
+    for (int i = 0; i < NST; ++i) {
+      mb::init(full + 8 * i, 1);
+      mb::init(empty + 8 * i, NW);
+    }
+    mb::fence_init();
+  }
   __syncthreads();
   if (warp == 0) {  // exclusive scan of the chunks per item
     int carry = 0;
@@ -390,46 +361,136 @@ __global__ void __launch_bounds__(NW * 32) gemv_fused_kernel(MmaArgs a) {
     if (lane == 0) s_pref[n_items] = carry;
   }
   __syncthreads();
+  volatile int* abort = &s_abort;
   const int n_qi = s_pref[n_items];
-  const int rb0 = a.d_ff / 8 / RT, rb1 = a.d / 16 / RT;
+  const int rb0 = a.d_ff / 8, rb1 = a.d / 16;
   const int U0 = n_qi * rb0, U1 = n_qi * rb1;
-  if (tid == 0) s_unit = atomicAdd(a.ticket, 1);
-  __syncthreads();
-  for (;;) {
-    const int u = s_unit;
-    if (u >= U0 + U1) break;
-    // the next ticket is fetched while this unit runs (phase-0 tickets all
-    // precede phase-1 ones, so holding one never blocks a waited-on unit)
-    int nxt = 0;
-    if (tid == 0) nxt = atomicAdd(a.ticket, 1);
-    const int phase = u < U0 ? 0 : 1;
-    int item, chunk, rb, qi;
-    unit_of(s_pref, n_items, phase == 0 ? rb0 : rb1, phase == 0 ? u : u - U0, item, chunk, rb, qi);
-    const WorkItem it = s_items[item];
-    const bool bad = a.cls != KIND_STREAMED && (it.slot < 0 || it.slot >= a.C);  // error already latched
-    if (phase == 1) {
-      // wait until every gate/up unit of this (item, chunk) has published h
-      if (tid == 0) {
-        const long long t0 = clock64();
-        volatile int32_t* dn = a.done + qi;
-        while (*dn < rb0) {
-          if (clock64() - t0 > WAIT_CYCLES) {
-            atomicExch(a.error, (uint32_t)DERR_TIMEOUT);
-            break;
+
+  if (warp == NW) {
+    if (lane == 0) produce<FP4>(a, s_items, s_pref, n_items, rb0, rb1, U0, U1, ring, meta, full, empty, abort);
+  } else {
+    const int g = lane >> 2, q = lane & 3;
+    float acc[NB][4];
+    const uint16_t* xr[NB];
+    const uint16_t* xl[NB];
+    int phase = 0, item = 0, chunk = 0, rb = 0, qi = 0, base = 0, nt = 0;
+    Geo geo{};
+    for (int it = 0;; ++it) {
+      const int slot = it % NST, r = it / NST;
+      // one waiter, then everyone reads its verdict: the exit decision is
+      // uniform (the producer may raise the abort flag at any time, so the
+      // flag itself is not read here); two verdict slots, because thread 0
+      // writes the next one before a slow warp may have read this one
+      if (tid == 0) s_go[it & 1] = mb::wait(full + 8 * slot, r & 1, abort, a.error) ? 1 : 0;
+      mma_warps_sync();
+      if (!s_go[it & 1]) break;
+      const int flags = meta[slot].flags;
+      if (flags & SM_END) break;
+      const int sl = meta[slot].slice;
+      if (flags & SM_FIRST) {
+        const int u = meta[slot].u;
+        phase = u < U0 ? 0 : 1;
+        unit_of(s_pref, n_items, phase == 0 ? rb0 : rb1, phase == 0 ? u : u - U0, item, chunk, rb, qi);
+        const WorkItem wi = s_items[item];
+        geo = geo_of(a, phase, FP4);
+        base = wi.tok_off + chunk * CHUNK;
+        nt = min(CHUNK, wi.n_tok - chunk * CHUNK);
+#pragma unroll
+        for (int t = 0; t < NB; ++t) {
+          const int j = t * 8 + g;
+          const int pos = base + (j < nt ? j : 0);
+          if (phase == 0) {
+            xr[t] = reinterpret_cast<const uint16_t*>(a.x) + (size_t)(a.perm[pos] / a.k) * a.d;
+            xl[t] = xr[t];
+          } else {
+            xr[t] = a.h16 + (size_t)pos * a.d_ff;
+            xl[t] = FP4 ? xr[t] : a.h16lo + (size_t)pos * a.d_ff;
+          }
+          acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+        }
+        if (phase == 1) {
+          // every gate/up unit of this (item, chunk) must have published h
+          if (tid == 0) {
+            const long long t0 = clock64();
+            volatile int32_t* dn = a.done + qi;
+            while (*dn < rb0) {
+              if (clock64() - t0 > WAIT_CYCLES) {
+                atomicExch(a.error, (uint32_t)DERR_TIMEOUT);
+                break;
+              }
+            }
+            __threadfence();
+          }
+          mma_warps_sync();
+        }
+      }
+      if (!(flags & SM_BAD)) {
+        const int s0 = sl * geo.ss, ns = min(geo.ss, geo.steps - s0);
+        const int w0 = (warp * ns) / NW, w1 = ((warp + 1) * ns) / NW;
+        const uint32_t code = mb::smem_u32(ring + slot * STAGE_BYTES), scs = code + ROWS * CODE_RS;
+        if (phase == 0)
+          stage_dot<NB, FP4, false>(code, scs, w0, w1, s0, xr, xl, g, q, acc);
+        else
+          stage_dot<NB, FP4, true>(code, scs, w0, w1, s0, xr, xl, g, q, acc);
+      }
+      __syncwarp();
+      if (lane == 0) mb::arrive(empty + 8 * slot);  // this warp is done with the stage
+      if (!(flags & SM_LAST)) continue;
+
+      // end of the unit: split-K reduction over the warps in warp order, epilogue by warp 0
+#pragma unroll
+      for (int t = 0; t < NB; ++t)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) red[((warp * NB + t) * 4 + c) * 32 + lane] = acc[t][c];
+      mma_warps_sync();
+      if (warp == 0 && !(flags & SM_BAD)) {
+        float v[NB][4];
+#pragma unroll
+        for (int t = 0; t < NB; ++t)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float x = red[(t * 4 + c) * 32 + lane];
+            for (int w = 1; w < NW; ++w) x += red[((w * NB + t) * 4 + c) * 32 + lane];
+            v[t][c] = x;
+          }
+        // d0,d1: row g, tokens 2q, 2q+1; d2,d3: row g+8, same tokens (per n8 tile)
+        float t0 = 1.f, t1 = 1.f;
+        if constexpr (FP4) {
+          const float* ts = a.tscale + ((size_t)a.layer * a.E + s_items[item].e) * 3;
+          t0 = phase == 0 ? ts[0] : ts[2];
+          t1 = phase == 0 ? ts[1] : ts[2];
+        }
+#pragma unroll
+        for (int t = 0; t < NB; ++t) {
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const int j = t * 8 + 2 * q + c;
+            if (j >= nt) continue;
+            const float v0 = v[t][c] * t0, v1 = v[t][2 + c] * t1;
+            if (phase == 0) {
+              const float hv = v0 / (1.f + expf(-v0)) * v1;
+              const size_t o = (size_t)(base + j) * a.d_ff + rb * 8 + g;
+              if constexpr (FP4) {
+                a.h16[o] = __half_as_ushort(__float2half_rn(hv));
+              } else {
+                const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
+                a.h16[o] = __bfloat16_as_ushort(hi);
+                a.h16lo[o] = __bfloat16_as_ushort(__float2bfloat16_rn(hv - __bfloat162float(hi)));
+              }
+            } else {
+              float* yr = a.ybuf + (size_t)(base + j) * a.d;
+              yr[rb * 16 + g] = v0;
+              yr[rb * 16 + g + 8] = v1;
+            }
           }
         }
-        __threadfence();
+        if (phase == 0) __threadfence();  // publish h before the unit is counted done
       }
-      __syncthreads();
-      if (!bad) unit_work<NB, 1, FP4, NW, RT>(a, it, chunk, rb, warp, lane, red);
-    } else {
-      if (!bad) unit_work<NB, 0, FP4, NW, RT>(a, it, chunk, rb, warp, lane, red);
-      if (tid == 0) atomicAdd(a.done + qi, 1);
+      mma_warps_sync();  // red is free again; h of this unit is published
+      if (tid == 0 && phase == 0) atomicAdd(a.done + qi, 1);
     }
-    __syncthreads();  // every thread has read s_unit
-    if (tid == 0) s_unit = nxt;
-    __syncthreads();
   }
+  __syncthreads();
 }
 
 // bf16 -> f16 copy of the activations (NVFP4 experts take f16 MMA operands).
@@ -437,35 +498,30 @@ __global__ void __launch_bounds__(256) to_f16_kernel(const __nv_bfloat16* __rest
   for (int i = blockIdx.x * 256 + threadIdx.x; i < n; i += gridDim.x * 256) y[i] = __float2half_rn(__bfloat162float(x[i]));
 }
 
-// Warps per CTA: up to 8 tokens per unit (small decode batches, single
-// staged experts) the work is short and 8 warps split K finer; at 9..16
-// tokens 4 warps per CTA give more CTAs per SM to overlap their stalls.
-template <int NB>
-constexpr int warps_for() { return NB == 1 ? 8 : 4; }
-
-int g_grid[2][3] = {{0, 0, 0}, {0, 0, 0}};  // [fp4][NB]
+int g_grid[2][3] = {{0, 0, 0}, {0, 0, 0}};  // [fp4][NB]: resident CTAs (one per SM)
 
 template <int NB, bool FP4>
 cudaError_t kernel_setup(int sms) {
-  constexpr int NW = warps_for<NB>();
+  cudaError_t e = cudaFuncSetAttribute(gemv_fused_kernel<NB, FP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       RING_BYTES);
+  if (e != cudaSuccess) return e;
   int per = 0;
-  const cudaError_t e =
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, gemv_fused_kernel<NB, FP4, NW>, NW * 32, 0);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, gemv_fused_kernel<NB, FP4>, THREADS, RING_BYTES);
   g_grid[FP4][NB] = sms * (per > 0 ? per : 1);
   return e;
 }
 
 template <int NB, bool FP4>
 void launch_nb(int grid, const MmaArgs& a, cudaStream_t st) {
-  constexpr int NW = warps_for<NB>();
-  gemv_fused_kernel<NB, FP4, NW><<<grid, NW * 32, 0, st>>>(a);
+  gemv_fused_kernel<NB, FP4><<<grid, THREADS, RING_BYTES, st>>>(a);
 }
 
 }  // namespace
 
 bool gemv_mma_supported(const Shape& sh) {
   if (sh.wtype == FT_W_BF16) return sh.d % 32 == 0 && sh.d_ff % 32 == 0;
-  if (sh.wtype == FT_W_NVFP4) return sh.d % 128 == 0 && sh.d_ff % 128 == 0;
+  // NVFP4: a row's block scales are a multiple of 16 bytes (bulk copies)
+  if (sh.wtype == FT_W_NVFP4) return sh.d % 256 == 0 && sh.d_ff % 256 == 0;
   return false;
 }
 
@@ -511,13 +567,12 @@ void launch_gemv_mma(const Shape& sh, int cls, int layer, const void* x16, int T
   const bool fp4 = sh.wtype == FT_W_NVFP4;
   const int NB = T > 8 ? 2 : 1;
   const long long chunks = (long long)max_items + (long long)max_tok / CHUNK;
-  const long long units = chunks * (sh.d_ff / 8 + sh.d / 16) / (fp4 ? tiles_for<true>() : 1);
-  // Streamed experts come over the host link: reads from host memory peak at
-  // about 128 warps in flight (more warps, more scattered streams, less
-  // bandwidth), which also leaves the SMs to the HBM work of the hit and
-  // staged experts running meanwhile.
+  const long long units = chunks * (sh.d_ff / 8 + sh.d / 16);
+  // Streamed experts come over the host link, which a few CTAs' rings keep
+  // busy (16 CTAs x 4 stages x 37 KB of bulk reads in flight); the other SMs
+  // stay with the HBM work of the hit and staged experts running meanwhile.
   int cap = g_grid[fp4][NB];
-  const int stream_ctas = 128 / (NB == 1 ? warps_for<1>() : warps_for<2>());
+  constexpr int stream_ctas = 16;
   if (cls == KIND_STREAMED && cap > stream_ctas) cap = stream_ctas;
   const int grid = (int)(units < cap ? units : cap);
   if (grid <= 0) return;
