@@ -142,7 +142,7 @@ void free_all(ft_ctx* c) {
   if (c->s_comp || c->s_side) cudaDeviceSynchronize();
   DevState& d = c->ds;
   void* dev_ptrs[] = {d.slot_of, d.key_of, d.stamp, d.clk, d.ctr, d.error, d.work, d.scores, d.ids, d.wts,
-                      d.counts, d.offsets, d.perm, d.inv, d.hbuf, d.ybuf, d.xs, d.hs, d.tscale, d.slots,
+                      d.counts, d.offsets, d.perm, d.inv, d.perm_chunks, d.hbuf, d.ybuf, d.xs, d.hs, d.tscale, d.slots,
                       d.h16, d.h16lo, d.x16, d.sched, d.route_ctr, c->probe_sink};
   for (void* p : dev_ptrs)
     if (p) cudaFree(p);
@@ -346,6 +346,7 @@ ft_status ft_moe_init(const ft_config* cfg, void* compute_stream, void* copy_str
   TRY(cuda_try(cudaMalloc((void**)&d.offsets, sizeof(int32_t) * (sh.E + 1))));
   TRY(cuda_try(cudaMalloc((void**)&d.perm, sizeof(int32_t) * Tk)));
   TRY(cuda_try(cudaMalloc((void**)&d.inv, sizeof(int32_t) * Tk)));
+  TRY(cuda_try(cudaMalloc((void**)&d.perm_chunks, sizeof(int32_t) * perm_chunks_ints((int)Tk, sh.E))));
   TRY(cuda_try(cudaMalloc((void**)&d.hbuf, sizeof(float) * Tk * sh.d_ff)));
   TRY(cuda_try(cudaMalloc((void**)&d.ybuf, sizeof(float) * Tk * sh.d)));
   TRY(cuda_try(cudaMalloc((void**)&d.tscale, sizeof(float) * sh.L * sh.E * 3)));
@@ -528,9 +529,9 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
     launch_topk(sh, d.scores, T, d, cs);
     prof_end(c, p, cs);
     p = prof_begin(c, P_PERMUTE, cs, Tk * 12.0 + sh.E * 8.0);
-    launch_permute(sh, T, d, cs);
+    const int n_perm = launch_permute(sh, T, d, cs);
     prof_end(c, p, cs);
-    c->kernel_launches += 3;
+    c->kernel_launches += 2 + n_perm;
   }
   if (ids_opt) CK(cudaMemcpyAsync(ids_opt, d.ids, sizeof(int32_t) * Tk, cudaMemcpyDeviceToDevice, cs));
   if (w_opt) CK(cudaMemcpyAsync(w_opt, d.wts, sizeof(float) * Tk, cudaMemcpyDeviceToDevice, cs));

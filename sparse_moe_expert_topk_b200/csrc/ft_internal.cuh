@@ -109,6 +109,7 @@ struct DevState {
   int32_t* offsets;          // [E+1]
   int32_t* perm;             // [Tmax*k]
   int32_t* inv;              // [Tmax*k]
+  int32_t* perm_chunks;      // [ceil(Tmax*k / 1024)][E] per-chunk counts, then offsets (large-T permutation)
   // expert scratch
   float* hbuf;               // [Tmax*k, d_ff] SwiGLU activations (fp32)
   float* ybuf;               // [Tmax*k, d] expert outputs (fp32)
@@ -133,7 +134,8 @@ void launch_router_scores(const Shape& sh, const void* x, const void* w_router, 
 // top-k + softmax weights (ids, wts)
 void launch_topk(const Shape& sh, const float* scores, int T, DevState& ds, cudaStream_t st);
 // stable permutation (counts, offsets, perm, inv)
-void launch_permute(const Shape& sh, int T, DevState& ds, cudaStream_t st);
+int launch_permute(const Shape& sh, int T, DevState& ds, cudaStream_t st);  // returns kernels launched
+size_t perm_chunks_ints(int max_entries, int E);
 // decode routing in one launch (T <= 32): logits, top-k, permutation, lookup
 void launch_route_decode(const Shape& sh, const void* x, const void* w_router, const float* bias, int bias_per_token,
                          int T, const LookupArgs& la, DevState& ds, cudaStream_t st);

@@ -447,6 +447,89 @@ void launch_router_scores(const Shape& sh, const void* x, const void* w_router, 
                                                                   bias_per_token, T, sh.E, sh.d, scores);
 }
 
+// ---------------------------------------------------------------------------
+// The same stable counting sort over many CTAs, for large T*k: chunks of 1024
+// entries; (1) each chunk counts its experts, (2) one CTA turns the counts into
+// the global offsets and, per (expert, chunk), the position of the chunk's
+// first entry of that expert (expert-major, chunks in order: stable), (3) each
+// chunk ranks its entries among equal experts as permute_body does and
+// scatters them.
+// ---------------------------------------------------------------------------
+constexpr int PCHUNK = 1024;
+
+__global__ void __launch_bounds__(PCHUNK) perm_hist_kernel(const int32_t* __restrict__ ids, int n, int E,
+                                                           int32_t* __restrict__ chunk) {
+  extern __shared__ int32_t cnt[];  // [E]
+  const int tid = threadIdx.x;
+  for (int e = tid; e < E; e += PCHUNK) cnt[e] = 0;
+  __syncthreads();
+  const int i = blockIdx.x * PCHUNK + tid;
+  if (i < n) atomicAdd(&cnt[ids[i]], 1);
+  __syncthreads();
+  for (int e = tid; e < E; e += PCHUNK) chunk[(size_t)blockIdx.x * E + e] = cnt[e];
+}
+
+// One CTA of MAX_E threads, thread e = expert e.
+__global__ void __launch_bounds__(MAX_E) perm_scan_kernel(int32_t* __restrict__ chunk, int nch, int E,
+                                                          int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
+  __shared__ int wsum[MAX_E / 32];
+  const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
+  int tot = 0;
+  if (e < E)
+    for (int c = 0; c < nch; ++c) tot += chunk[(size_t)c * E + e];
+  int incl = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  int base = incl - tot;
+  for (int w = 0; w < warp; ++w) base += wsum[w];
+  if (e < E) {
+    counts[e] = tot;
+    offsets[e] = base;
+    if (e == E - 1) offsets[E] = base + tot;
+    int run = base;
+    for (int c = 0; c < nch; ++c) {
+      const int v = chunk[(size_t)c * E + e];
+      chunk[(size_t)c * E + e] = run;
+      run += v;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(PCHUNK) perm_scatter_kernel(const int32_t* __restrict__ ids, int n, int E,
+                                                              const int32_t* __restrict__ chunk,
+                                                              int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
+  extern __shared__ int32_t wcnt[];  // [32][E]: per warp count, then exclusive prefix over the warps
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int x = tid; x < 32 * E; x += PCHUNK) wcnt[x] = 0;
+  __syncthreads();
+  const int i = blockIdx.x * PCHUNK + tid;
+  const bool valid = i < n;
+  const int e = valid ? ids[i] : E;  // E = sentinel for padding lanes
+  const unsigned same = __match_any_sync(0xffffffffu, e);
+  const int rank = __popc(same & ((1u << lane) - 1u));
+  if (valid && rank == 0) wcnt[warp * E + e] = __popc(same);
+  __syncthreads();
+  for (int x = tid; x < E; x += PCHUNK) {
+    int r = 0;
+    for (int w = 0; w < 32; ++w) {
+      const int c = wcnt[w * E + x];
+      wcnt[w * E + x] = r;
+      r += c;
+    }
+  }
+  __syncthreads();
+  if (valid) {
+    const int pos = chunk[(size_t)blockIdx.x * E + e] + wcnt[warp * E + e] + rank;
+    perm[pos] = i;
+    inv[i] = pos;
+  }
+}
+
 size_t permute_smem_bytes(int E) { return sizeof(int32_t) * (size_t)(32 * E + 3 * E); }
 
 void launch_topk(const Shape& sh, const float* scores, int T, DevState& ds, cudaStream_t st) {
@@ -455,10 +538,21 @@ void launch_topk(const Shape& sh, const float* scores, int T, DevState& ds, cuda
       scores, T, sh.E, sh.k, ds.ids, ds.wts);
 }
 
-void launch_permute(const Shape& sh, int T, DevState& ds, cudaStream_t st) {
-  permute_kernel<<<1, 1024, permute_smem_bytes(sh.E), st>>>(ds.ids, T * sh.k, sh.E, ds.counts, ds.offsets, ds.perm,
-                                                           ds.inv);
+int launch_permute(const Shape& sh, int T, DevState& ds, cudaStream_t st) {
+  const int n = T * sh.k;
+  if (n <= 2 * PCHUNK) {
+    permute_kernel<<<1, 1024, permute_smem_bytes(sh.E), st>>>(ds.ids, n, sh.E, ds.counts, ds.offsets, ds.perm, ds.inv);
+    return 1;
+  }
+  const int nch = (n + PCHUNK - 1) / PCHUNK;
+  perm_hist_kernel<<<nch, PCHUNK, sizeof(int32_t) * sh.E, st>>>(ds.ids, n, sh.E, ds.perm_chunks);
+  perm_scan_kernel<<<1, MAX_E, 0, st>>>(ds.perm_chunks, nch, sh.E, ds.counts, ds.offsets);
+  perm_scatter_kernel<<<nch, PCHUNK, sizeof(int32_t) * 32 * sh.E, st>>>(ds.ids, n, sh.E, ds.perm_chunks, ds.perm,
+                                                                         ds.inv);
+  return 3;
 }
+
+size_t perm_chunks_ints(int max_entries, int E) { return (size_t)((max_entries + PCHUNK - 1) / PCHUNK) * E; }
 
 // ---------------------------------------------------------------------------
 // Router + top-k without any allocation (ft_route_topk_static in ft_moe.h).
@@ -533,6 +627,9 @@ void launch_route_decode(const Shape& sh, const void* x, const void* w_router, c
 cudaError_t route_kernels_init(int E) {
   const int smem = (int)permute_smem_bytes(E), smem_f = (int)route_decode_smem(E);
   cudaError_t e = cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(perm_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(sizeof(int32_t) * 32 * E));
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(route_decode_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_f);
   if (e == cudaSuccess)
