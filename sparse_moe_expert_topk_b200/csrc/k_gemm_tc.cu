@@ -166,10 +166,13 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
   __shared__ uint32_t s_tmem;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-  // bars: full[STAGES], empty[STAGES], acc_full, acc_empty, drain
+  // bars: full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain
   const uint32_t bar_full = smem_u32(bars), bar_empty = bar_full + 8 * STAGES;
-  const uint32_t bar_acc_full = bar_full + 16 * STAGES, bar_acc_empty = bar_acc_full + 8;
-  const uint32_t bar_drain = bar_acc_empty + 8;
+  // accumulator buffers: phase 0 uses all 512 TMEM columns (gate | up), one
+  // buffer; phase 1 needs 256, so two buffers let the epilogue drain one while
+  // the MMAs of the next unit fill the other
+  const uint32_t bar_acc_full = bar_full + 16 * STAGES, bar_acc_empty = bar_acc_full + 16;
+  const uint32_t bar_drain = bar_acc_empty + 16;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort = &s_abort;
 
@@ -181,8 +184,10 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
       mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, 1);
     }
-    mbar_init(bar_acc_full, 1);
-    mbar_init(bar_acc_empty, 4);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_acc_full + 8 * b, 1);
+      mbar_init(bar_acc_empty + 8 * b, 4);
+    }
     mbar_init(bar_drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -249,7 +254,9 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
       if (!unit_at(a, s_items, s_pref, n_items, u, un)) break;
       const int n_mma = (un.nrows + 15) & ~15;
       const uint32_t idesc = idesc_bf16(BM, n_mma);
-      if (!mbar_wait(bar_acc_empty, (ui & 1) ^ 1, abort, a.error)) break;
+      const int ab = two_a ? 0 : (ui & 1), use = two_a ? ui : (ui >> 1);  // buffer, its use count
+      if (!mbar_wait(bar_acc_empty + 8 * ab, (use & 1) ^ 1, abort, a.error)) break;
+      const uint32_t dacc = tmem + (uint32_t)(ab * 256);
       tc_fence_after();
       bool ok = true;
       for (int kb = 0; kb < a.k_blocks; ++kb, ++it) {
@@ -264,11 +271,11 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t bd = sw128_desc(base + 2 * A_BYTES + kk * 32);
-            umma_bf16(tmem, sw128_desc(base + kk * 32), bd, idesc, (kb | kk) != 0);
+            umma_bf16(dacc, sw128_desc(base + kk * 32), bd, idesc, (kb | kk) != 0);
             if (two_a) umma_bf16(tmem + 256, sw128_desc(base + A_BYTES + kk * 32), bd, idesc, (kb | kk) != 0);
           }
           umma_commit(bar_empty + 8 * s);  // stage free once these MMAs have read it
-          if (kb == a.k_blocks - 1) umma_commit(bar_acc_full);
+          if (kb == a.k_blocks - 1) umma_commit(bar_acc_full + 8 * ab);
         }
         __syncwarp();
       }
@@ -282,12 +289,13 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
     for (int u = blockIdx.x; u < n_units && !*abort; u += gridDim.x, ++ui) {
       Unit un;
       if (!unit_at(a, s_items, s_pref, n_items, u, un)) break;
-      if (!mbar_wait(bar_acc_full, ui & 1, abort, a.error)) break;
+      const int ab = two_a ? 0 : (ui & 1), use = two_a ? ui : (ui >> 1);
+      if (!mbar_wait(bar_acc_full + 8 * ab, use & 1, abort, a.error)) break;
       tc_fence_after();
       const int row = un.mt * BM + 32 * q + lane;  // weight row = output feature
       for (int c0 = 0; c0 < un.nrows; c0 += 32) {
         uint32_t g[32];
-        tmem_ld32(tmem + lane_base + c0, g);
+        tmem_ld32(tmem + (uint32_t)(ab * 256) + lane_base + c0, g);
         if (two_a) {
           uint32_t uu[32];
           tmem_ld32(tmem + lane_base + 256 + c0, uu);
@@ -309,7 +317,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_acc_empty);
+      if (lane == 0) mbar_arrive(bar_acc_empty + 8 * ab);
     }
   }
   __syncthreads();
