@@ -259,10 +259,16 @@ __device__ void produce(const MmaArgs& a, const WorkItem* items, const int* pref
   const size_t n = (size_t)a.d * a.d_ff;
   const size_t mat = FP4 ? n / 2 : n * 2;          // code bytes per matrix
   const size_t sc0 = 3 * (n / 2), scm = n / 16;     // NVFP4 scales: start, bytes per matrix
+  // per slot: the last round posted and whether it carried copies. Only that
+  // round can still be in flight at exit (posting a round waits for the
+  // consumers to release the one before it); a sentinel or skipped stage
+  // posted after a copy round advances the slot's phase, so an older copy
+  // round's parity must not be waited on.
   int it = 0;
   int last_round[NST];
+  bool last_copy[NST];
 #pragma unroll
-  for (int i = 0; i < NST; ++i) last_round[i] = -1;
+  for (int i = 0; i < NST; ++i) last_round[i] = -1, last_copy[i] = false;
   for (bool done = false; !done;) {
     const int u = atomicAdd(a.ticket, 1);
     if (u >= U0 + U1) {  // end of work: one sentinel stage
@@ -270,6 +276,8 @@ __device__ void produce(const MmaArgs& a, const WorkItem* items, const int* pref
       if (mb::wait(empty + 8 * slot, (r & 1) ^ 1, abort, a.error)) {
         meta[slot].flags = SM_END;
         mb::arrive(full + 8 * slot);
+        last_round[slot] = r;
+        last_copy[slot] = false;
       }
       break;
     }
@@ -290,6 +298,8 @@ __device__ void produce(const MmaArgs& a, const WorkItem* items, const int* pref
       meta[slot].slice = sl;
       meta[slot].flags = (sl == 0 ? SM_FIRST : 0) | (sl == g.nsl - 1 ? SM_LAST : 0) | (bad ? SM_BAD : 0);
       const uint32_t bar = full + 8 * slot;
+      last_round[slot] = r;
+      last_copy[slot] = !bad;
       if (bad) {
         mb::arrive(bar);
         continue;
@@ -312,13 +322,12 @@ __device__ void produce(const MmaArgs& a, const WorkItem* items, const int* pref
         mb::bulk_g2s(code + i * CODE_RS, blob + m * mat + row * g.row_bytes + (size_t)s0 * 64, cb, bar);
         if (FP4) mb::bulk_g2s(scs + i * SC_RS, blob + sc0 + m * scm + row * g.sc_row + (size_t)s0 * 8, sb, bar);
       }
-      last_round[slot] = r;
     }
   }
   // every copy issued must have landed before the CTA's shared memory goes away
 #pragma unroll
   for (int i = 0; i < NST; ++i)
-    if (last_round[i] >= 0) mb::wait_quiet(full + 8 * i, last_round[i] & 1, WAIT_CYCLES / 4);
+    if (last_copy[i]) mb::wait_quiet(full + 8 * i, last_round[i] & 1, WAIT_CYCLES / 4);
 }
 
 template <int NB, bool FP4>
