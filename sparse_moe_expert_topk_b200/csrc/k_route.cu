@@ -292,69 +292,59 @@ __device__ void logits_bf16_block(const __nv_bfloat16* __restrict__ x, const __n
   }
 }
 
-// BF16 router logits for larger T on mma.sync: a warp computes 64 experts
-// (four m16 tiles, rows of W_r as the A operand) x 16 tokens (two n8 tiles),
-// so each activation fragment feeds four expert tiles; the four warps of a CTA
-// take four token groups of the same 64 experts, whose W_r rows L1 serves.
-// K runs in steps of 32 values, lane-permuted as in logits_bf16_block.
-// grid (ceil(E/64), ceil(T/64)), 128 threads.
-constexpr int RT_E = 4;  // expert tiles of 16 per warp
+// BF16 router logits for many tokens (prefill) on mma.sync: CTA = 16 experts
+// x 64 tokens, warp w takes tokens t0+16w .. +16 over the full K (steps of 32
+// K values, lane-permuted K as in logits_bf16_block; the four warps read the
+// same W_r rows, which L1 serves). grid (ceil(E/16), ceil(T/64)), 128 threads.
 __global__ void __launch_bounds__(128) router_mma_kernel(const __nv_bfloat16* __restrict__ x,
                                                          const __nv_bfloat16* __restrict__ wr,
                                                          const float* __restrict__ bias, int bias_per_token, int T,
                                                          int E, int d, float* __restrict__ scores) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-  const int e0 = blockIdx.x * 16 * RT_E, t0 = blockIdx.y * 64 + warp * 16;
+  const int e0 = blockIdx.x * 16, t0 = blockIdx.y * 64 + warp * 16;
   if (t0 >= T) return;
   const int nt = min(16, T - t0);
-  const uint8_t* pa[RT_E];
-  const uint8_t* pb[RT_E];
-#pragma unroll
-  for (int i = 0; i < RT_E; ++i) {  // clamp: rows past E are computed but not stored
-    const int ra = min(e0 + 16 * i + g, E - 1), rb = min(e0 + 16 * i + g + 8, E - 1);
-    pa[i] = reinterpret_cast<const uint8_t*>(wr + (size_t)ra * d) + q * 16;
-    pb[i] = reinterpret_cast<const uint8_t*>(wr + (size_t)rb * d) + q * 16;
-  }
+  const int ra = min(e0 + g, E - 1), rb = min(e0 + g + 8, E - 1);
+  const uint8_t* pa = reinterpret_cast<const uint8_t*>(wr + (size_t)ra * d) + q * 16;
+  const uint8_t* pb = reinterpret_cast<const uint8_t*>(wr + (size_t)rb * d) + q * 16;
   const __nv_bfloat16* xr0 = x + (size_t)(t0 + (g < nt ? g : 0)) * d + q * 8;
   const __nv_bfloat16* xr1 = x + (size_t)(t0 + (g + 8 < nt ? g + 8 : 0)) * d + q * 8;
-  float acc[RT_E][2][4];
-#pragma unroll
-  for (int i = 0; i < RT_E; ++i)
-#pragma unroll
-    for (int t = 0; t < 2; ++t) acc[i][t][0] = acc[i][t][1] = acc[i][t][2] = acc[i][t][3] = 0.f;
+  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   const int steps = d / 32;
-  for (int s = 0; s < steps; ++s) {
-    const uint4 x0 = __ldg(reinterpret_cast<const uint4*>(xr0 + s * 32));
-    const uint4 x1 = __ldg(reinterpret_cast<const uint4*>(xr1 + s * 32));
-    uint4 wa[RT_E], wb[RT_E];
+  constexpr int U = 4;
+  for (int s = 0; s < steps; s += U) {
+    uint4 wa[U], wb[U], x0[U], x1[U];
 #pragma unroll
-    for (int i = 0; i < RT_E; ++i) {
-      wa[i] = __ldg(reinterpret_cast<const uint4*>(pa[i] + (size_t)s * 64));
-      wb[i] = __ldg(reinterpret_cast<const uint4*>(pb[i] + (size_t)s * 64));
+    for (int u = 0; u < U; ++u) {
+      const int ss = s + u < steps ? s + u : steps - 1;
+      wa[u] = __ldg(reinterpret_cast<const uint4*>(pa + (size_t)ss * 64));
+      wb[u] = __ldg(reinterpret_cast<const uint4*>(pb + (size_t)ss * 64));
+      x0[u] = __ldg(reinterpret_cast<const uint4*>(xr0 + ss * 32));
+      x1[u] = __ldg(reinterpret_cast<const uint4*>(xr1 + ss * 32));
     }
 #pragma unroll
-    for (int i = 0; i < RT_E; ++i) {
-      mma_bf16_16816(acc[i][0], wa[i].x, wb[i].x, wa[i].y, wb[i].y, x0.x, x0.y);
-      mma_bf16_16816(acc[i][0], wa[i].z, wb[i].z, wa[i].w, wb[i].w, x0.z, x0.w);
-      mma_bf16_16816(acc[i][1], wa[i].x, wb[i].x, wa[i].y, wb[i].y, x1.x, x1.y);
-      mma_bf16_16816(acc[i][1], wa[i].z, wb[i].z, wa[i].w, wb[i].w, x1.z, x1.w);
+    for (int u = 0; u < U; ++u) {
+      if (s + u < steps) {
+        mma_bf16_16816(acc[0], wa[u].x, wb[u].x, wa[u].y, wb[u].y, x0[u].x, x0[u].y);
+        mma_bf16_16816(acc[0], wa[u].z, wb[u].z, wa[u].w, wb[u].w, x0[u].z, x0[u].w);
+        mma_bf16_16816(acc[1], wa[u].x, wb[u].x, wa[u].y, wb[u].y, x1[u].x, x1[u].y);
+        mma_bf16_16816(acc[1], wa[u].z, wb[u].z, wa[u].w, wb[u].w, x1[u].z, x1[u].w);
+      }
     }
   }
 #pragma unroll
-  for (int i = 0; i < RT_E; ++i)
+  for (int t = 0; t < 2; ++t)
 #pragma unroll
-    for (int t = 0; t < 2; ++t)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int j = t * 8 + 2 * q + (c & 1);  // token within the tile
-        const int e = e0 + 16 * i + g + (c >> 1) * 8;
-        if (j < nt && e < E) {
-          const int tok = t0 + j;
-          float b = 0.f;
-          if (bias) b = bias_per_token ? bias[(size_t)tok * E + e] : bias[e];
-          scores[(size_t)tok * E + e] = acc[i][t][c] + b;
-        }
+    for (int c = 0; c < 4; ++c) {
+      const int j = t * 8 + 2 * q + (c & 1);  // token within the tile
+      const int e = e0 + g + (c >> 1) * 8;
+      if (j < nt && e < E) {
+        const int tok = t0 + j;
+        float b = 0.f;
+        if (bias) b = bias_per_token ? bias[(size_t)tok * E + e] : bias[e];
+        scores[(size_t)tok * E + e] = acc[t][c] + b;
       }
+    }
 }
 
 // Decode routing in one launch (T <= 32 tokens): CTAs of 32 warps compute the
@@ -441,7 +431,7 @@ __global__ void __launch_bounds__(1024) route_decode_kernel(const AT* __restrict
 void launch_router_scores(const Shape& sh, const void* x, const void* w_router, const float* bias, int bias_per_token,
                           int T, float* scores, cudaStream_t st) {
   if (sh.wtype != FT_W_F32 && T > 32 && sh.d % 32 == 0) {
-    dim3 grid((sh.E + 16 * RT_E - 1) / (16 * RT_E), (T + 63) / 64);
+    dim3 grid((sh.E + 15) / 16, (T + 63) / 64);
     router_mma_kernel<<<grid, 128, 0, st>>>((const __nv_bfloat16*)x, (const __nv_bfloat16*)w_router, bias,
                                             bias_per_token, T, sh.E, sh.d, scores);
     return;
