@@ -21,6 +21,8 @@
 #include <thread>
 #include <vector>
 
+#include <cuda.h>
+
 #include "ft_internal.cuh"
 
 namespace ft {
@@ -62,6 +64,9 @@ struct ft_ctx {
   bool use_tc = false;
   bool use_mma = false;  // tensor-core decode GEMV (BF16 / NVFP4), else SIMT
   unsigned long long* probe_sink = nullptr;
+  // stream memory operation that marks a staged blob as landed (null: not available)
+  CUresult (*write_value)(CUstream, CUdeviceptr, cuuint32_t, unsigned int) = nullptr;
+  uint32_t epoch = 0;
   // launch accounting and optional per-launch CUDA-event profiling
   unsigned long long kernel_launches = 0;
   bool profiling = false;
@@ -143,7 +148,7 @@ void free_all(ft_ctx* c) {
   DevState& d = c->ds;
   void* dev_ptrs[] = {d.slot_of, d.key_of, d.stamp, d.clk, d.ctr, d.error, d.work, d.scores, d.ids, d.wts,
                       d.counts, d.offsets, d.perm, d.inv, d.perm_chunks, d.hbuf, d.ybuf, d.xs, d.hs, d.tscale, d.slots,
-                      d.h16, d.h16lo, d.x16, d.sched, d.route_ctr, c->probe_sink};
+                      d.h16, d.h16lo, d.x16, d.sched, d.route_ctr, d.landed, c->probe_sink};
   for (void* p : dev_ptrs)
     if (p) cudaFree(p);
   for (uint8_t* p : c->pool_host)
@@ -364,6 +369,24 @@ ft_status ft_moe_init(const ft_config* cfg, void* compute_stream, void* copy_str
   TRY(cuda_try(cudaMemset(d.sched, 0, sizeof(int32_t) * (N_CLASSES + (size_t)N_CLASSES * d.sched_chunks))));
   TRY(cuda_try(cudaMalloc((void**)&d.route_ctr, sizeof(int32_t))));
   TRY(cuda_try(cudaMemset(d.route_ctr, 0, sizeof(int32_t))));
+  TRY(cuda_try(cudaMalloc((void**)&d.landed, sizeof(uint32_t) * MAX_E)));
+  TRY(cuda_try(cudaMemset(d.landed, 0, sizeof(uint32_t) * MAX_E)));
+  d.landed_epoch = 0;
+  {
+    // cuStreamWriteValue32 lets the copy stream mark each staged blob as it
+    // lands, so the staged experts' GEMV can start before the last copy ends;
+    // without it the staged GEMV waits for every copy (an event)
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuStreamWriteValue32", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess && fn) {
+      c->write_value = reinterpret_cast<CUresult (*)(CUstream, CUdeviceptr, cuuint32_t, unsigned int)>(fn);
+      if (c->write_value((CUstream)c->s_side, (CUdeviceptr)d.landed, 0u, 0) != CUDA_SUCCESS ||
+          cudaStreamSynchronize(c->s_side) != cudaSuccess)
+        c->write_value = nullptr;
+    }
+    cudaGetLastError();
+  }
   c->use_tc = prefill_tc_supported(sh) && sh.C >= 2ll * sh.E;
   if (c->use_tc) {
     TRY(cuda_try(cudaMalloc((void**)&d.xs, sizeof(__nv_bfloat16) * (Tk + 256) * sh.d)));
@@ -465,7 +488,9 @@ static void gemv_class_cost(ft_ctx* c, const int (&pr)[2], int n_items, int n_to
   }
 }
 
-static ft_status issue_copies(ft_ctx* c, int from, int to) {
+// One cudaMemcpyAsync per staged blob on the copy stream; with epoch != 0,
+// each copy is followed by a stream write of the epoch into landed[i - from].
+static ft_status issue_copies(ft_ctx* c, int from, int to, uint32_t epoch = 0) {
   const Mailbox* mb = c->mbox_host;
   const Shape& sh = c->sh;
   for (int i = from; i < to; ++i) {
@@ -475,6 +500,9 @@ static ft_status issue_copies(ft_ctx* c, int from, int to) {
     if (fault("memcpy")) return FT_ECUDA;
     CK(cudaMemcpyAsync(c->ds.slots + (size_t)slot * sh.slot_bytes, c->pool_host[l] + (size_t)e * sh.slot_bytes,
                        sh.slot_bytes, cudaMemcpyHostToDevice, c->s_copy));
+    if (epoch && c->write_value((CUstream)c->s_copy, (CUdeviceptr)(c->ds.landed + (i - from)), epoch, 0) !=
+                     CUDA_SUCCESS)
+      return FT_ECUDA;
   }
   return FT_OK;
 }
@@ -561,13 +589,21 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
     gemv_class_cost(c, pr_stream, mb->n_streamed_cls, mb->n_tok_cls[KIND_STREAMED]);
     gemv_class_cost(c, pr_hit, mb->n_hit_cls, mb->n_tok_cls[KIND_HIT]);
     if (n_copy > 0) {
+      // with landed flags the staged GEMV starts at once and each of its
+      // experts waits (on the device) for its own copy; else it waits for all
+      const bool flags = c->write_value != nullptr && c->use_mma && n_copy <= MAX_E;
+      if (flags && ++c->epoch == 0) ++c->epoch;
       p = prof_begin(c, P_STAGE_COPY, c->s_copy, n_copy * (double)sh.slot_bytes);
-      st = issue_copies(c, 0, n_copy);
+      st = issue_copies(c, 0, n_copy, flags ? c->epoch : 0);
       prof_end(c, p, c->s_copy);
       if (st != FT_OK) return c->latched = st;
       CK(cudaEventRecord(c->ev_copy, c->s_copy));
-      CK(cudaStreamWaitEvent(cs, c->ev_copy, 0));
+      if (flags)
+        d.landed_epoch = c->epoch;
+      else
+        CK(cudaStreamWaitEvent(cs, c->ev_copy, 0));
       gemv_class(c, KIND_STAGED, layer, x, T, max_items, Tk, cs, pr_staged);
+      d.landed_epoch = 0;
       gemv_class_cost(c, pr_staged, mb->n_staged_cls, mb->n_tok_cls[KIND_STAGED]);
     }
     CK(cudaStreamWaitEvent(cs, c->ev_side, 0));

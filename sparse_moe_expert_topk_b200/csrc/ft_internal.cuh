@@ -125,6 +125,8 @@ struct DevState {
   int32_t* sched;            // [N_CLASSES] unit tickets + [N_CLASSES][sched_chunks] chunk completion counters
   int sched_chunks;
   int32_t* route_ctr;        // last-CTA ticket of the fused decode routing kernel (0 between calls)
+  uint32_t* landed;          // [MAX_E] per staged blob of a decode call: the call's epoch once its copy landed
+  uint32_t landed_epoch;     // epoch of the current call (0: staged experts wait for all copies on the host side)
 };
 
 // ---- launchers (all enqueue on `st`) ----

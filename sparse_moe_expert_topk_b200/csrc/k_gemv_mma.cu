@@ -140,7 +140,15 @@ struct MmaArgs {
   int32_t* ticket;      // this class's unit ticket counter (zeroed by the lookup)
   int32_t* done;        // this class's per-(item, chunk) phase-0 completion counters (zeroed)
   uint32_t* error;
+  const uint32_t* landed;  // staged class: landed[item] == epoch once the copy engine wrote the item's slot
+  uint32_t epoch;          // (null: the launch was ordered after every copy)
 };
+
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 
 __device__ __forceinline__ const uint8_t* blob_of(const MmaArgs& a, const WorkItem& it) {
   if (a.cls == KIND_STREAMED) return a.pool + (size_t)it.e * a.slot_bytes;
@@ -265,6 +273,7 @@ __device__ void produce(const MmaArgs& a, const WorkItem* items, const int* pref
   // posted after a copy round advances the slot's phase, so an older copy
   // round's parity must not be waited on.
   int it = 0;
+  int landed_upto = -1;  // items known to be in their slots
   int last_round[NST];
   bool last_copy[NST];
 #pragma unroll
@@ -287,6 +296,20 @@ __device__ void produce(const MmaArgs& a, const WorkItem* items, const int* pref
     const WorkItem wi = items[item];
     const bool bad = a.cls != KIND_STREAMED && (wi.slot < 0 || wi.slot >= a.C);  // error already latched
     const uint8_t* blob = bad ? nullptr : blob_of(a, wi);
+    if (a.landed && !bad && item > landed_upto) {
+      // a staged expert: its slot is readable once the copy stream has
+      // written this call's epoch behind the blob's copy (items are in copy order)
+      const long long t0 = clock64();
+      while (ld_acquire(a.landed + item) != a.epoch) {
+        if (*abort) break;
+        if (clock64() - t0 > WAIT_CYCLES) {
+          *abort = 1;
+          atomicExch(a.error, (uint32_t)DERR_TIMEOUT);
+          break;
+        }
+      }
+      landed_upto = item;
+    }
     const Geo g = geo_of(a, phase, FP4);
     for (int sl = 0; sl < g.nsl; ++sl, ++it) {
       const int slot = it % NST, r = it / NST;
@@ -573,6 +596,8 @@ void launch_gemv_mma(const Shape& sh, int cls, int layer, const void* x16, int T
   a.ticket = ds.sched + cls;
   a.done = ds.sched + N_CLASSES + (size_t)cls * ds.sched_chunks;
   a.error = ds.error;
+  a.landed = cls == KIND_STAGED && ds.landed_epoch ? ds.landed : nullptr;
+  a.epoch = ds.landed_epoch;
   const bool fp4 = sh.wtype == FT_W_NVFP4;
   const int NB = T > 8 ? 2 : 1;
   const long long chunks = (long long)max_items + (long long)max_tok / CHUNK;
