@@ -259,17 +259,21 @@ struct StageMeta {
 };
 constexpr int SM_FIRST = 1, SM_LAST = 2, SM_BAD = 4, SM_END = 8;
 
-// Producer: one lane takes tickets and fills the ring.
+// Producer: the last warp fills the ring. Lane 0 takes the tickets (the next
+// one always in flight), waits for free slots and posts each stage; then each
+// lane issues one bulk copy of the stage (lane i < 16: the codes of smem row i;
+// lane 16 + i, NVFP4 only: that row's block scales), so the 16-32 copies of a
+// stage go out in parallel instead of one after another.
 template <bool FP4>
 __device__ void produce(const MmaArgs& a, const WorkItem* items, const int* pref, int n_items, int rb0, int rb1,
                         int U0, int U1, uint8_t* ring, volatile StageMeta* meta, uint32_t full, uint32_t empty,
-                        volatile int* abort) {
+                        volatile int* abort, int lane) {
   const size_t n = (size_t)a.d * a.d_ff;
   const size_t mat = FP4 ? n / 2 : n * 2;          // code bytes per matrix
   const size_t sc0 = 3 * (n / 2), scm = n / 16;     // NVFP4 scales: start, bytes per matrix
-  // per slot: the last round posted and whether it carried copies. Only that
-  // round can still be in flight at exit (posting a round waits for the
-  // consumers to release the one before it); a sentinel or skipped stage
+  // per slot (lane 0): the last round posted and whether it carried copies.
+  // Only that round can still be in flight at exit (posting a round waits for
+  // the consumers to release the one before it); a sentinel or skipped stage
   // posted after a copy round advances the slot's phase, so an older copy
   // round's parity must not be waited on.
   int it = 0;
@@ -278,18 +282,28 @@ __device__ void produce(const MmaArgs& a, const WorkItem* items, const int* pref
   bool last_copy[NST];
 #pragma unroll
   for (int i = 0; i < NST; ++i) last_round[i] = -1, last_copy[i] = false;
+  // the next ticket is always in flight while a unit's copies are issued (a
+  // global atomic's round trip would otherwise stall every unit); holding it
+  // keeps the order argument: every ticket a CTA holds is later than the unit
+  // its MMA warps work on
+  int nxt = lane == 0 ? atomicAdd(a.ticket, 1) : 0;
+  const int row = lane & 15;  // smem row this lane copies
+  const bool sc_lane = lane >= 16;
   for (bool done = false; !done;) {
-    const int u = atomicAdd(a.ticket, 1);
+    const int u = __shfl_sync(0xffffffffu, nxt, 0);
     if (u >= U0 + U1) {  // end of work: one sentinel stage
-      const int slot = it % NST, r = it / NST;
-      if (mb::wait(empty + 8 * slot, (r & 1) ^ 1, abort, a.error)) {
-        meta[slot].flags = SM_END;
-        mb::arrive(full + 8 * slot);
-        last_round[slot] = r;
-        last_copy[slot] = false;
+      if (lane == 0) {
+        const int slot = it % NST, r = it / NST;
+        if (mb::wait(empty + 8 * slot, (r & 1) ^ 1, abort, a.error)) {
+          meta[slot].flags = SM_END;
+          mb::arrive(full + 8 * slot);
+          last_round[slot] = r;
+          last_copy[slot] = false;
+        }
       }
       break;
     }
+    if (lane == 0) nxt = atomicAdd(a.ticket, 1);
     const int phase = u < U0 ? 0 : 1;
     int item, chunk, rb, qi;
     unit_of(pref, n_items, phase == 0 ? rb0 : rb1, phase == 0 ? u : u - U0, item, chunk, rb, qi);
@@ -299,58 +313,68 @@ __device__ void produce(const MmaArgs& a, const WorkItem* items, const int* pref
     if (a.landed && !bad && item > landed_upto) {
       // a staged expert: its slot is readable once the copy stream has
       // written this call's epoch behind the blob's copy (items are in copy order)
-      const long long t0 = clock64();
-      while (ld_acquire(a.landed + item) != a.epoch) {
-        if (*abort) break;
-        if (clock64() - t0 > WAIT_CYCLES) {
-          *abort = 1;
-          atomicExch(a.error, (uint32_t)DERR_TIMEOUT);
-          break;
+      if (lane == 0) {
+        const long long t0 = clock64();
+        while (ld_acquire(a.landed + item) != a.epoch) {
+          if (*abort) break;
+          if (clock64() - t0 > WAIT_CYCLES) {
+            *abort = 1;
+            atomicExch(a.error, (uint32_t)DERR_TIMEOUT);
+            break;
+          }
         }
       }
+      __syncwarp();
       landed_upto = item;
     }
     const Geo g = geo_of(a, phase, FP4);
+    // this lane's source row: smem row i -> gate row 8 rb + i (i < 8) or up row
+    // 8 rb + i - 8 (phase 0); down row 16 rb + i (phase 1)
+    const size_t m = phase == 0 ? (row < 8 ? 0 : 1) : 2;
+    const size_t grow = phase == 0 ? (size_t)rb * 8 + (row & 7) : (size_t)rb * 16 + row;
     for (int sl = 0; sl < g.nsl; ++sl, ++it) {
       const int slot = it % NST, r = it / NST;
-      if (!mb::wait(empty + 8 * slot, (r & 1) ^ 1, abort, a.error)) {
+      int ok = 1;
+      if (lane == 0) {
+        ok = mb::wait(empty + 8 * slot, (r & 1) ^ 1, abort, a.error) ? 1 : 0;
+        if (ok) {
+          meta[slot].u = u;
+          meta[slot].slice = sl;
+          meta[slot].flags = (sl == 0 ? SM_FIRST : 0) | (sl == g.nsl - 1 ? SM_LAST : 0) | (bad ? SM_BAD : 0);
+          last_round[slot] = r;
+          last_copy[slot] = !bad;
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
         done = true;
         break;
       }
-      meta[slot].u = u;
-      meta[slot].slice = sl;
-      meta[slot].flags = (sl == 0 ? SM_FIRST : 0) | (sl == g.nsl - 1 ? SM_LAST : 0) | (bad ? SM_BAD : 0);
       const uint32_t bar = full + 8 * slot;
-      last_round[slot] = r;
-      last_copy[slot] = !bad;
-      if (bad) {
-        mb::arrive(bar);
-        continue;
-      }
       const int s0 = sl * g.ss, ns = min(g.ss, g.steps - s0);
       const uint32_t cb = (uint32_t)ns * 64, sb = FP4 ? (uint32_t)ns * 8 : 0;
-      mb::expect_tx(bar, ROWS * (cb + sb));
-      const uint32_t code = mb::smem_u32(ring + slot * STAGE_BYTES), scs = code + ROWS * CODE_RS;
-#pragma unroll 1
-      for (int i = 0; i < ROWS; ++i) {
-        // smem row i: phase 0 -> gate row 8 rb + i (i < 8) or up row 8 rb + i - 8; phase 1 -> down row 16 rb + i
-        size_t m, row;
-        if (phase == 0) {
-          m = i < 8 ? 0 : 1;
-          row = (size_t)rb * 8 + (i & 7);
-        } else {
-          m = 2;
-          row = (size_t)rb * 16 + i;
-        }
-        mb::bulk_g2s(code + i * CODE_RS, blob + m * mat + row * g.row_bytes + (size_t)s0 * 64, cb, bar);
-        if (FP4) mb::bulk_g2s(scs + i * SC_RS, blob + sc0 + m * scm + row * g.sc_row + (size_t)s0 * 8, sb, bar);
+      if (lane == 0) {
+        if (bad)
+          mb::arrive(bar);
+        else
+          mb::expect_tx(bar, ROWS * (cb + sb));
       }
+      __syncwarp();  // the expected bytes are posted before any copy can complete them
+      if (bad) continue;
+      const uint32_t code = mb::smem_u32(ring + slot * STAGE_BYTES), scs = code + ROWS * CODE_RS;
+      if (!sc_lane)
+        mb::bulk_g2s(code + row * CODE_RS, blob + m * mat + grow * g.row_bytes + (size_t)s0 * 64, cb, bar);
+      else if (FP4)
+        mb::bulk_g2s(scs + row * SC_RS, blob + sc0 + m * scm + grow * g.sc_row + (size_t)s0 * 8, sb, bar);
     }
   }
   // every copy issued must have landed before the CTA's shared memory goes away
+  if (lane == 0) {
 #pragma unroll
-  for (int i = 0; i < NST; ++i)
-    if (last_copy[i]) mb::wait_quiet(full + 8 * i, last_round[i] & 1, WAIT_CYCLES / 4);
+    for (int i = 0; i < NST; ++i)
+      if (last_copy[i]) mb::wait_quiet(full + 8 * i, last_round[i] & 1, WAIT_CYCLES / 4);
+  }
+  __syncwarp();
 }
 
 template <int NB, bool FP4>
@@ -399,7 +423,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_fused_kernel(MmaArgs a) {
   const int U0 = n_qi * rb0, U1 = n_qi * rb1;
 
   if (warp == NW) {
-    if (lane == 0) produce<FP4>(a, s_items, s_pref, n_items, rb0, rb1, U0, U1, ring, meta, full, empty, abort);
+    produce<FP4>(a, s_items, s_pref, n_items, rb0, rb1, U0, U1, ring, meta, full, empty, abort, lane);
   } else {
     const int g = lane >> 2, q = lane & 3;
     float acc[NB][4];
