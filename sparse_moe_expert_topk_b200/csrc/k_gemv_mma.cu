@@ -62,6 +62,14 @@ constexpr int SC_RS = SLICE / 8 + 16;            // same for the NVFP4 block sca
 constexpr int STAGE_BYTES = ROWS * CODE_RS + ROWS * SC_RS;
 constexpr int RING_BYTES = NST * STAGE_BYTES;
 
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
 // L2-coherent load (for h, written by other CTAs of the same launch).
 __device__ __forceinline__ uint4 ld_cg(const void* p) {
   uint4 r;
@@ -493,51 +501,45 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_fused_kernel(MmaArgs a) {
       if (lane == 0) mb::arrive(empty + 8 * slot);  // this warp is done with the stage
       if (!(flags & SM_LAST)) continue;
 
-      // end of the unit: split-K reduction over the warps in warp order, epilogue by warp 0
+      // end of the unit: split-K reduction over the warps in warp order, one
+      // output pair per thread: thread o < NB*64 takes token tile t, element
+      // pair c (rows g and g+8 of lane l's fragment)
 #pragma unroll
       for (int t = 0; t < NB; ++t)
 #pragma unroll
         for (int c = 0; c < 4; ++c) red[((warp * NB + t) * 4 + c) * 32 + lane] = acc[t][c];
       mma_warps_sync();
-      if (warp == 0 && !(flags & SM_BAD)) {
-        float v[NB][4];
+      if (!(flags & SM_BAD) && tid < NB * 64) {
+        const int t = tid >> 6, c = (tid >> 5) & 1, l = tid & 31;
+        const int lg = l >> 2, lq = l & 3;
+        float v0 = 0.f, v1 = 0.f;
 #pragma unroll
-        for (int t = 0; t < NB; ++t)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float x = red[(t * 4 + c) * 32 + lane];
-            for (int w = 1; w < NW; ++w) x += red[((w * NB + t) * 4 + c) * 32 + lane];
-            v[t][c] = x;
-          }
-        // d0,d1: row g, tokens 2q, 2q+1; d2,d3: row g+8, same tokens (per n8 tile)
-        float t0 = 1.f, t1 = 1.f;
-        if constexpr (FP4) {
-          const float* ts = a.tscale + ((size_t)a.layer * a.E + s_items[item].e) * 3;
-          t0 = phase == 0 ? ts[0] : ts[2];
-          t1 = phase == 0 ? ts[1] : ts[2];
+        for (int w = 0; w < NW; ++w) {
+          v0 += red[((w * NB + t) * 4 + c) * 32 + l];
+          v1 += red[((w * NB + t) * 4 + c + 2) * 32 + l];
         }
-#pragma unroll
-        for (int t = 0; t < NB; ++t) {
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const int j = t * 8 + 2 * q + c;
-            if (j >= nt) continue;
-            const float v0 = v[t][c] * t0, v1 = v[t][2 + c] * t1;
-            if (phase == 0) {
-              const float hv = v0 / (1.f + expf(-v0)) * v1;
-              const size_t o = (size_t)(base + j) * a.d_ff + rb * 8 + g;
-              if constexpr (FP4) {
-                a.h16[o] = __half_as_ushort(__float2half_rn(hv));
-              } else {
-                const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
-                a.h16[o] = __bfloat16_as_ushort(hi);
-                a.h16lo[o] = __bfloat16_as_ushort(__float2bfloat16_rn(hv - __bfloat162float(hi)));
-              }
+        // row lg (gate / first down row) and lg+8 (up / second down row), token 2 lq + c of tile t
+        const int j = t * 8 + 2 * lq + c;
+        if (j < nt) {
+          if constexpr (FP4) {
+            const float* ts = a.tscale + ((size_t)a.layer * a.E + s_items[item].e) * 3;
+            v0 *= phase == 0 ? ts[0] : ts[2];
+            v1 *= phase == 0 ? ts[1] : ts[2];
+          }
+          if (phase == 0) {
+            const float hv = v0 / (1.f + expf(-v0)) * v1;
+            const size_t o = (size_t)(base + j) * a.d_ff + rb * 8 + lg;
+            if constexpr (FP4) {
+              a.h16[o] = __half_as_ushort(__float2half_rn(hv));
             } else {
-              float* yr = a.ybuf + (size_t)(base + j) * a.d;
-              yr[rb * 16 + g] = v0;
-              yr[rb * 16 + g + 8] = v1;
+              const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
+              a.h16[o] = __bfloat16_as_ushort(hi);
+              a.h16lo[o] = __bfloat16_as_ushort(__float2bfloat16_rn(hv - __bfloat162float(hi)));
             }
+          } else {
+            float* yr = a.ybuf + (size_t)(base + j) * a.d;
+            yr[rb * 16 + lg] = v0;
+            yr[rb * 16 + lg + 8] = v1;
           }
         }
         if (phase == 0) __threadfence();  // publish h before the unit is counted done
@@ -547,6 +549,291 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_fused_kernel(MmaArgs a) {
     }
   }
   __syncthreads();
+}
+
+// One BF16 step: 8 K values of rows g and g+8 per lane, two MMAs per token
+// tile (and two more for the low part of h in phase 1).
+template <int NB, bool P1>
+__device__ __forceinline__ void bf16_step(const uint4 wa, const uint4 wb, const uint16_t* const (&xr)[NB],
+                                          const uint16_t* const (&xl)[NB], int e0, float (&acc)[NB][4]) {
+#pragma unroll
+  for (int t = 0; t < NB; ++t) {
+    const uint4 xv = P1 ? ld_cg(xr[t] + e0) : __ldg(reinterpret_cast<const uint4*>(xr[t] + e0));
+    mma_bf16(acc[t], wa.x, wb.x, wa.y, wb.y, xv.x, xv.y);
+    mma_bf16(acc[t], wa.z, wb.z, wa.w, wb.w, xv.z, xv.w);
+    if constexpr (P1) {
+      const uint4 xo = ld_cg(xl[t] + e0);
+      mma_bf16(acc[t], wa.x, wb.x, wa.y, wb.y, xo.x, xo.y);
+      mma_bf16(acc[t], wa.z, wb.z, wa.w, wb.w, xo.z, xo.w);
+    }
+  }
+}
+
+// acc[t][.] += W[rows g, g+8] . X[tokens] over steps [s0, s1) of 32 K values
+// (lane q covers K = 32 s + 8 q .. +8). U steps of loads in flight; steps past
+// s1 reload the last step and are not used.
+template <int NB, int U, bool P1>
+__device__ __forceinline__ void dot_bf16(const uint8_t* ra, const uint8_t* rb, int s0, int s1,
+                                         const uint16_t* const (&xr)[NB], const uint16_t* const (&xl)[NB], int q,
+                                         float (&acc)[NB][4]) {
+  for (int s = s0; s < s1; s += U) {
+    uint4 wa[U], wb[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int ss = s + u < s1 ? s + u : s1 - 1;
+      wa[u] = ld_stream(ra + (size_t)ss * 64);
+      wb[u] = ld_stream(rb + (size_t)ss * 64);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (s + u < s1) bf16_step<NB, P1>(wa[u], wb[u], xr, xl, (s + u) * 32 + q * 8, acc);
+  }
+}
+
+// NVFP4: steps of 128 K values (lane q covers K = 128 s + 32 q .. +32: 16
+// code bytes and one scale pair per row); RT row tiles per step, the tiles
+// tstride code bytes (tsc scale pairs) apart, sharing one activation
+// fragment; eight MMAs per step, tile and token tile.
+template <int NB, int RT, bool P1>
+__device__ __forceinline__ void dot_nvfp4(const uint8_t* ra, const uint8_t* rb, const unsigned short* sa,
+                                          const unsigned short* sb, size_t tstride, size_t tsc, int s0, int s1,
+                                          const uint16_t* const (&xr)[NB], int q, float (&acc)[RT][NB][4]) {
+  for (int s = s0; s < s1; ++s) {
+    uint4 wa[RT], wb[RT];
+    uint32_t ca[RT], cb[RT];
+#pragma unroll
+    for (int r = 0; r < RT; ++r) {
+      wa[r] = ld_stream(ra + r * tstride + (size_t)s * 64);
+      wb[r] = ld_stream(rb + r * tstride + (size_t)s * 64);
+      ca[r] = __ldg(sa + r * tsc + s * 4);
+      cb[r] = __ldg(sb + r * tsc + s * 4);
+    }
+    uint32_t xh[NB][16];
+#pragma unroll
+    for (int t = 0; t < NB; ++t) {
+      const uint16_t* xp = xr[t] + s * 128 + q * 32;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const uint4 xv = P1 ? ld_cg(xp + 8 * v) : __ldg(reinterpret_cast<const uint4*>(xp) + v);
+        xh[t][4 * v] = xv.x;
+        xh[t][4 * v + 1] = xv.y;
+        xh[t][4 * v + 2] = xv.z;
+        xh[t][4 * v + 3] = xv.w;
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < RT; ++r) {
+      uint32_t ha[16], hb[16];
+      decode_nvfp4(wa[r], ca[r], ha);
+      decode_nvfp4(wb[r], cb[r], hb);
+#pragma unroll
+      for (int t = 0; t < NB; ++t)
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          mma_f16(acc[r][t], ha[2 * j], hb[2 * j], ha[2 * j + 1], hb[2 * j + 1], xh[t][2 * j], xh[t][2 * j + 1]);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Direct-load variant for experts resident in HBM slots (the hit class): the
+// MMA warps load their weight fragments straight into registers, U steps in
+// flight, several CTAs per SM, so load latency is hidden by many warps. (The
+// TMA ring above serves the staged and streamed classes, whose bytes arrive
+// over the host link anyway.)
+// ---------------------------------------------------------------------------
+
+// One unit: RT tiles of 16 weight rows x one chunk of <= 16 tokens, the K
+// range split over the NW warps, partial sums reduced in warp order, epilogue
+// of tile r by warp r. Tile r of unit rb is row block rb*RT + r: gate rows
+// 8 (rb*RT + r) + g with the matching up rows (phase 0), down rows
+// 16 (rb*RT + r) + g and + 8 (phase 1).
+template <int NB, int PHASE, bool FP4, int NW, int RT>
+__device__ void direct_unit(const MmaArgs& a, const WorkItem& it, int chunk, int rb, int warp, int lane, float* red) {
+  const int g = lane >> 2, q = lane & 3;
+  const uint8_t* blob = blob_of(a, it);
+  const size_t n = (size_t)a.d * a.d_ff;
+  const int K = PHASE == 0 ? a.d : a.d_ff;
+  const size_t rbytes = FP4 ? (size_t)K / 2 : (size_t)K * 2;
+  const size_t sbytes = (size_t)K / 16;
+  const int steps = FP4 ? K / 128 : K / 32;
+  const int s0 = (warp * steps) / NW, s1 = ((warp + 1) * steps) / NW;
+  const int rows_per_tile = PHASE == 0 ? 8 : 16;  // per weight matrix
+  const int blk0 = rb * RT;                       // first row block of the unit
+  size_t oa, ob, sa0, sb0;
+  if (PHASE == 0) {
+    oa = (size_t)(blk0 * 8 + g) * rbytes;
+    ob = (FP4 ? n / 2 : n * 2) + (size_t)(blk0 * 8 + g) * rbytes;
+    sa0 = 3 * (n / 2) + (size_t)(blk0 * 8 + g) * sbytes;
+    sb0 = 3 * (n / 2) + n / 16 + (size_t)(blk0 * 8 + g) * sbytes;
+  } else {
+    oa = (FP4 ? n : n * 4) + (size_t)(blk0 * 16 + g) * rbytes;
+    ob = oa + 8 * rbytes;
+    sa0 = 3 * (n / 2) + 2 * (n / 16) + (size_t)(blk0 * 16 + g) * sbytes;
+    sb0 = sa0 + 8 * sbytes;
+  }
+  const int base = it.tok_off + chunk * CHUNK;
+  const int nt = min(CHUNK, it.n_tok - chunk * CHUNK);
+  const uint16_t* xr[NB];
+  const uint16_t* xl[NB];
+#pragma unroll
+  for (int t = 0; t < NB; ++t) {
+    const int j = t * 8 + g;
+    const int pos = base + (j < nt ? j : 0);
+    if (PHASE == 0) {
+      xr[t] = reinterpret_cast<const uint16_t*>(a.x) + (size_t)(a.perm[pos] / a.k) * a.d;
+      xl[t] = xr[t];
+    } else {
+      xr[t] = a.h16 + (size_t)pos * a.d_ff;
+      xl[t] = FP4 ? xr[t] : a.h16lo + (size_t)pos * a.d_ff;
+    }
+  }
+  float acc[RT][NB][4];
+#pragma unroll
+  for (int r = 0; r < RT; ++r)
+#pragma unroll
+    for (int t = 0; t < NB; ++t) acc[r][t][0] = acc[r][t][1] = acc[r][t][2] = acc[r][t][3] = 0.f;
+  if constexpr (FP4) {
+    dot_nvfp4<NB, RT, PHASE == 1>(blob + oa + q * 16, blob + ob + q * 16,
+                                  reinterpret_cast<const unsigned short*>(blob + sa0) + q,
+                                  reinterpret_cast<const unsigned short*>(blob + sb0) + q,
+                                  (size_t)rows_per_tile * rbytes, (size_t)rows_per_tile * sbytes / 2, s0, s1, xr, q,
+                                  acc);
+  } else {
+    static_assert(FP4 || RT == 1, "BF16 units are one row tile");
+    dot_bf16<NB, (NB == 1 ? 8 : 4), PHASE == 1>(blob + oa + q * 16, blob + ob + q * 16, s0, s1, xr, xl, q, acc[0]);
+  }
+  // split-K reduction over the warps, in warp order; red is [NW][RT][NB][4][32]
+#pragma unroll
+  for (int r = 0; r < RT; ++r)
+#pragma unroll
+    for (int t = 0; t < NB; ++t)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) red[(((warp * RT + r) * NB + t) * 4 + c) * 32 + lane] = acc[r][t][c];
+  __syncthreads();
+  if (warp < RT) {
+    const int r = warp;
+    float v[NB][4];
+#pragma unroll
+    for (int t = 0; t < NB; ++t)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float x = red[((r * NB + t) * 4 + c) * 32 + lane];
+        for (int w = 1; w < NW; ++w) x += red[(((w * RT + r) * NB + t) * 4 + c) * 32 + lane];
+        v[t][c] = x;
+      }
+    // d0,d1: row g, tokens 2q, 2q+1; d2,d3: row g+8, same tokens (per n8 tile)
+    float t0 = 1.f, t1 = 1.f;
+    if constexpr (FP4) {
+      const float* ts = a.tscale + ((size_t)a.layer * a.E + it.e) * 3;
+      t0 = PHASE == 0 ? ts[0] : ts[2];
+      t1 = PHASE == 0 ? ts[1] : ts[2];
+    }
+    const int blk = blk0 + r;
+#pragma unroll
+    for (int t = 0; t < NB; ++t) {
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int j = t * 8 + 2 * q + c;
+        if (j >= nt) continue;
+        const float v0 = v[t][c] * t0, v1 = v[t][2 + c] * t1;
+        if (PHASE == 0) {
+          const float hv = v0 / (1.f + expf(-v0)) * v1;
+          const size_t o = (size_t)(base + j) * a.d_ff + blk * 8 + g;
+          if constexpr (FP4) {
+            a.h16[o] = __half_as_ushort(__float2half_rn(hv));
+          } else {
+            const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
+            a.h16[o] = __bfloat16_as_ushort(hi);
+            a.h16lo[o] = __bfloat16_as_ushort(__float2bfloat16_rn(hv - __bfloat162float(hi)));
+          }
+        } else {
+          float* yr = a.ybuf + (size_t)(base + j) * a.d;
+          yr[blk * 16 + g] = v0;
+          yr[blk * 16 + g + 8] = v1;
+        }
+      }
+    }
+    if (PHASE == 0) __threadfence();  // publish h before the unit is counted done
+  }
+  __syncthreads();  // red is reused by the next unit
+}
+
+// Row tiles per unit: NVFP4 rows are a quarter of the BF16 bytes, so a unit
+// takes four tiles to keep the loads in flight per warp and the per-unit
+// reduction and barriers amortised.
+template <bool FP4>
+constexpr int tiles_for() { return FP4 ? 4 : 1; }
+
+template <int NB, bool FP4, int NW>
+__global__ void __launch_bounds__(NW * 32) gemv_direct_kernel(MmaArgs a) {
+  constexpr int RT = tiles_for<FP4>();
+  __shared__ int s_pref[MAX_E + 1];
+  __shared__ WorkItem s_items[MAX_E];
+  __shared__ float red[NW * RT * NB * 4 * 32];
+  __shared__ int s_unit;
+  const int n_items = a.work->n_items[a.cls];
+  if (n_items == 0) return;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < n_items; i += blockDim.x) s_items[i] = a.work->items[a.cls][i];
+  __syncthreads();
+  if (warp == 0) {  // exclusive scan of the chunks per item
+    int carry = 0;
+    for (int b = 0; b < n_items; b += 32) {
+      const int i = b + lane;
+      const int c = i < n_items ? (s_items[i].n_tok + CHUNK - 1) / CHUNK : 0;
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (i < n_items) s_pref[i] = carry + incl - c;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) s_pref[n_items] = carry;
+  }
+  __syncthreads();
+  const int n_qi = s_pref[n_items];
+  const int rb0 = a.d_ff / 8 / RT, rb1 = a.d / 16 / RT;
+  const int U0 = n_qi * rb0, U1 = n_qi * rb1;
+  if (tid == 0) s_unit = atomicAdd(a.ticket, 1);
+  __syncthreads();
+  for (;;) {
+    const int u = s_unit;
+    if (u >= U0 + U1) break;
+    // the next ticket is fetched while this unit runs (phase-0 tickets all
+    // precede phase-1 ones, so holding one never blocks a waited-on unit)
+    int nxt = 0;
+    if (tid == 0) nxt = atomicAdd(a.ticket, 1);
+    const int phase = u < U0 ? 0 : 1;
+    int item, chunk, rb, qi;
+    unit_of(s_pref, n_items, phase == 0 ? rb0 : rb1, phase == 0 ? u : u - U0, item, chunk, rb, qi);
+    const WorkItem it = s_items[item];
+    const bool bad = a.cls != KIND_STREAMED && (it.slot < 0 || it.slot >= a.C);  // error already latched
+    if (phase == 1) {
+      // wait until every gate/up unit of this (item, chunk) has published h
+      if (tid == 0) {
+        const long long t0 = clock64();
+        volatile int32_t* dn = a.done + qi;
+        while (*dn < rb0) {
+          if (clock64() - t0 > WAIT_CYCLES) {
+            atomicExch(a.error, (uint32_t)DERR_TIMEOUT);
+            break;
+          }
+        }
+        __threadfence();
+      }
+      __syncthreads();
+      if (!bad) direct_unit<NB, 1, FP4, NW, RT>(a, it, chunk, rb, warp, lane, red);
+    } else {
+      if (!bad) direct_unit<NB, 0, FP4, NW, RT>(a, it, chunk, rb, warp, lane, red);
+      if (tid == 0) atomicAdd(a.done + qi, 1);
+    }
+    __syncthreads();  // every thread has read s_unit
+    if (tid == 0) s_unit = nxt;
+    __syncthreads();
+  }
 }
 
 // bf16 -> f16 copy of the activations (NVFP4 experts take f16 MMA operands).
@@ -572,6 +859,30 @@ void launch_nb(int grid, const MmaArgs& a, cudaStream_t st) {
   gemv_fused_kernel<NB, FP4><<<grid, THREADS, RING_BYTES, st>>>(a);
 }
 
+// Warps per CTA: up to 8 tokens per unit (small decode batches, single
+// staged experts) the work is short and 8 warps split K finer; at 9..16
+// tokens 4 warps per CTA give more CTAs per SM to overlap their stalls.
+template <int NB>
+constexpr int warps_for() { return NB == 1 ? 8 : 4; }
+
+int g_grid_direct[2][3] = {{0, 0, 0}, {0, 0, 0}};  // [fp4][NB]
+
+template <int NB, bool FP4>
+cudaError_t direct_setup(int sms) {
+  constexpr int NW = warps_for<NB>();
+  int per = 0;
+  const cudaError_t e =
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, gemv_direct_kernel<NB, FP4, NW>, NW * 32, 0);
+  g_grid_direct[FP4][NB] = sms * (per > 0 ? per : 1);
+  return e;
+}
+
+template <int NB, bool FP4>
+void launch_direct(int grid, const MmaArgs& a, cudaStream_t st) {
+  constexpr int NW = warps_for<NB>();
+  gemv_direct_kernel<NB, FP4, NW><<<grid, NW * 32, 0, st>>>(a);
+}
+
 }  // namespace
 
 bool gemv_mma_supported(const Shape& sh) {
@@ -588,6 +899,10 @@ cudaError_t gemv_mma_init(int device) {
   if (e == cudaSuccess) e = kernel_setup<2, false>(sms);
   if (e == cudaSuccess) e = kernel_setup<1, true>(sms);
   if (e == cudaSuccess) e = kernel_setup<2, true>(sms);
+  if (e == cudaSuccess) e = direct_setup<1, false>(sms);
+  if (e == cudaSuccess) e = direct_setup<2, false>(sms);
+  if (e == cudaSuccess) e = direct_setup<1, true>(sms);
+  if (e == cudaSuccess) e = direct_setup<2, true>(sms);
   return e;
 }
 
@@ -625,10 +940,24 @@ void launch_gemv_mma(const Shape& sh, int cls, int layer, const void* x16, int T
   const bool fp4 = sh.wtype == FT_W_NVFP4;
   const int NB = T > 8 ? 2 : 1;
   const long long chunks = (long long)max_items + (long long)max_tok / CHUNK;
+  if (cls == KIND_HIT) {
+    const long long units = chunks * (sh.d_ff / 8 + sh.d / 16) / (fp4 ? tiles_for<true>() : 1);
+    const int cap = g_grid_direct[fp4][NB];
+    const int grid = (int)(units < cap ? units : cap);
+    if (grid <= 0) return;
+    if (fp4) {
+      if (NB == 1) launch_direct<1, true>(grid, a, st);
+      else launch_direct<2, true>(grid, a, st);
+    } else {
+      if (NB == 1) launch_direct<1, false>(grid, a, st);
+      else launch_direct<2, false>(grid, a, st);
+    }
+    return;
+  }
   const long long units = chunks * (sh.d_ff / 8 + sh.d / 16);
   // Streamed experts come over the host link, which a few CTAs' rings keep
   // busy (16 CTAs x 4 stages x 37 KB of bulk reads in flight); the other SMs
-  // stay with the HBM work of the hit and staged experts running meanwhile.
+  // stay with the HBM work of the hit experts running meanwhile.
   int cap = g_grid[fp4][NB];
   constexpr int stream_ctas = 16;
   if (cls == KIND_STREAMED && cap > stream_ctas) cap = stream_ctas;
