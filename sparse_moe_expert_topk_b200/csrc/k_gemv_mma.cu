@@ -53,6 +53,7 @@ namespace {
 constexpr int CHUNK = 16;  // tokens per unit (two n8 tiles)
 constexpr long long WAIT_CYCLES = mb::WAIT_CYCLES;
 constexpr int NW = 8;                            // MMA (consumer) warps
+constexpr int RING_WARPS = NW;
 constexpr int THREADS = (NW + 1) * 32;           // + one producer warp
 constexpr int NST = 4;                           // ring stages
 constexpr int ROWS = 16;                         // weight rows per unit / stage
@@ -657,7 +658,7 @@ __device__ void direct_unit(const MmaArgs& a, const WorkItem& it, int chunk, int
   const size_t rbytes = FP4 ? (size_t)K / 2 : (size_t)K * 2;
   const size_t sbytes = (size_t)K / 16;
   const int steps = FP4 ? K / 128 : K / 32;
-  const int s0 = (warp * steps) / NW, s1 = ((warp + 1) * steps) / NW;
+  (void)steps;
   const int rows_per_tile = PHASE == 0 ? 8 : 16;  // per weight matrix
   const int blk0 = rb * RT;                       // first row block of the unit
   size_t oa, ob, sa0, sb0;
@@ -693,15 +694,25 @@ __device__ void direct_unit(const MmaArgs& a, const WorkItem& it, int chunk, int
   for (int r = 0; r < RT; ++r)
 #pragma unroll
     for (int t = 0; t < NB; ++t) acc[r][t][0] = acc[r][t][1] = acc[r][t][2] = acc[r][t][3] = 0.f;
-  if constexpr (FP4) {
-    dot_nvfp4<NB, RT, PHASE == 1>(blob + oa + q * 16, blob + ob + q * 16,
-                                  reinterpret_cast<const unsigned short*>(blob + sa0) + q,
-                                  reinterpret_cast<const unsigned short*>(blob + sb0) + q,
-                                  (size_t)rows_per_tile * rbytes, (size_t)rows_per_tile * sbytes / 2, s0, s1, xr, q,
-                                  acc);
-  } else {
-    static_assert(FP4 || RT == 1, "BF16 units are one row tile");
-    dot_bf16<NB, (NB == 1 ? 8 : 4), PHASE == 1>(blob + oa + q * 16, blob + ob + q * 16, s0, s1, xr, xl, q, acc[0]);
+  // The K steps this warp covers are the TMA-ring kernel's: for each ring
+  // slice j in order, sub-range w of NW = 8. With the same MMA order inside a
+  // warp and the same warp-order reduction, an expert's output is bit-identical
+  // whichever class (and kernel) computes it.
+  static_assert(NW == RING_WARPS, "the K partition must match the TMA-ring kernel's");
+  const Geo gg = geo_of(a, PHASE, FP4);
+  for (int j = 0; j < gg.nsl; ++j) {
+    const int b0 = j * gg.ss, ns = min(gg.ss, gg.steps - b0);
+    const int s0 = b0 + (warp * ns) / NW, s1 = b0 + ((warp + 1) * ns) / NW;
+    if constexpr (FP4) {
+      dot_nvfp4<NB, RT, PHASE == 1>(blob + oa + q * 16, blob + ob + q * 16,
+                                    reinterpret_cast<const unsigned short*>(blob + sa0) + q,
+                                    reinterpret_cast<const unsigned short*>(blob + sb0) + q,
+                                    (size_t)rows_per_tile * rbytes, (size_t)rows_per_tile * sbytes / 2, s0, s1, xr, q,
+                                    acc);
+    } else {
+      static_assert(FP4 || RT == 1, "BF16 units are one row tile");
+      dot_bf16<NB, (NB == 1 ? 8 : 4), PHASE == 1>(blob + oa + q * 16, blob + ob + q * 16, s0, s1, xr, xl, q, acc[0]);
+    }
   }
   // split-K reduction over the warps, in warp order; red is [NW][RT][NB][4][32]
 #pragma unroll
@@ -859,11 +870,10 @@ void launch_nb(int grid, const MmaArgs& a, cudaStream_t st) {
   gemv_fused_kernel<NB, FP4><<<grid, THREADS, RING_BYTES, st>>>(a);
 }
 
-// Warps per CTA: up to 8 tokens per unit (small decode batches, single
-// staged experts) the work is short and 8 warps split K finer; at 9..16
-// tokens 4 warps per CTA give more CTAs per SM to overlap their stalls.
+// Warps per CTA of the direct-load kernel: the ring kernel's eight, so both
+// split K the same way (see direct_unit).
 template <int NB>
-constexpr int warps_for() { return NB == 1 ? 8 : 4; }
+constexpr int warps_for() { return RING_WARPS; }
 
 int g_grid_direct[2][3] = {{0, 0, 0}, {0, 0, 0}};  // [fp4][NB]
 
