@@ -287,6 +287,15 @@ def cpu_blob_source(wl):
     return blob
 
 
+def decode_config(wl, world):
+    """The `config` object of the decode line, shared by both arms."""
+    return {"workload": "single-layer BF16 decode, E=256 top-6 d=4096 d_ff=1536, 37% cache (94 slots), "
+                        "LRU, B_P:B_H=52.7:77.3, 64-step trace at batch 1/4/16 from a cold cache",
+            "tokens_per_step": wl.steps * sum(wl.batches), "layer_calls_per_step": wl.steps * len(wl.batches),
+            "l2": "inputs larger than L2 (9.7 GB pinned pool, 3.5 GB slot pool)",
+            "parallelism": f"replicas x{world}"}
+
+
 def run_reference(args, wl, world, rank):
     if rank != 0:
         return 0
@@ -306,8 +315,7 @@ def run_reference(args, wl, world, rank):
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * el / args.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "E": wl.E, "top_k": wl.k, "d": wl.d, "d_ff": wl.d_ff,
-                       "cache_slots": wl.cache_slots, "batches": list(wl.batches), "decode_steps": wl.steps},
+            "config": decode_config(wl, world),
             "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": f"first {calls} decode calls of the trace in {args.steps} steps of "
                                        f"~{per_step_s:.0f} s each (routing, shared LRU with q*, fp64 experts)"},
@@ -708,11 +716,7 @@ def main():
             "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "single-layer BF16 decode, E=256 top-6 d=4096 d_ff=1536, 37% cache (94 slots), "
-                                   "LRU, B_P:B_H=52.7:77.3, 64-step trace at batch 1/4/16 from a cold cache",
-                       "tokens_per_step": tokens_per_step, "layer_calls_per_step": wl.steps * len(wl.batches),
-                       "l2": "inputs larger than L2 (9.7 GB pinned pool, 3.5 GB slot pool)",
-                       "parallelism": f"replicas x{world}"},
+            "config": decode_config(wl, world),
             "miss_rate": round(miss_rate, 4),
             "miss_rate_second_half": round(half["misses"] / max(half["lookups"], 1), 4),
             "overlap": overlap,
