@@ -174,8 +174,9 @@ def run_step_e2e(h, xs_host, bias, x_dev, y_dev, y_host):
 # --------------------------------------------------------------------------
 KERNEL_SOURCES = {"gemv": "sparse_moe_expert_topk_b200/csrc/k_gemv_mma.cu",
                   "gemm_tc": "sparse_moe_expert_topk_b200/csrc/k_gemm_tc.cu",
-                  "router": "sparse_moe_expert_topk_b200/csrc/k_route.cu",
-                  "lookup": "sparse_moe_expert_topk_b200/csrc/k_lookup.cu"}
+                  "route": "sparse_moe_expert_topk_b200/csrc/k_route.cu",
+                  "lookup": "sparse_moe_expert_topk_b200/csrc/k_lookup.cu",
+                  "combine": "sparse_moe_expert_topk_b200/csrc/k_expert.cu"}
 
 
 def _source_sha(kernel_name):
