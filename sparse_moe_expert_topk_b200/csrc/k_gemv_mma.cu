@@ -591,6 +591,45 @@ __device__ __forceinline__ void dot_bf16(const uint8_t* ra, const uint8_t* rb, i
   }
 }
 
+// The same over this warp's K steps of every ring slice (slice j: sub-range
+// warp of NW of [j*ss, j*ss + ns_j)), gathered across slice boundaries into
+// batches of U loads in flight; the MMAs run in slice order, step by step, so
+// the sum is exactly the TMA-ring kernel's.
+template <int NB, int U, bool P1, int NWARPS>
+__device__ __forceinline__ void dot_bf16_slices(const uint8_t* ra, const uint8_t* rb, const Geo& g, int warp,
+                                                const uint16_t* const (&xr)[NB], const uint16_t* const (&xl)[NB],
+                                                int q, float (&acc)[NB][4]) {
+  int j = 0;
+  int lo = (warp * min(g.ss, g.steps)) / NWARPS, hi = ((warp + 1) * min(g.ss, g.steps)) / NWARPS;
+  int s = lo;
+  for (;;) {
+    int st[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      while (s >= hi && j + 1 < g.nsl) {
+        ++j;
+        const int b0 = j * g.ss, ns = min(g.ss, g.steps - b0);
+        lo = b0 + (warp * ns) / NWARPS;
+        hi = b0 + ((warp + 1) * ns) / NWARPS;
+        s = lo;
+      }
+      st[u] = s < hi ? s : -1;
+      s += s < hi ? 1 : 0;
+    }
+    if (st[0] < 0) break;
+    uint4 wa[U], wb[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int ss = st[u] >= 0 ? st[u] : st[0];
+      wa[u] = ld_stream(ra + (size_t)ss * 64);
+      wb[u] = ld_stream(rb + (size_t)ss * 64);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (st[u] >= 0) bf16_step<NB, P1>(wa[u], wb[u], xr, xl, st[u] * 32 + q * 8, acc);
+  }
+}
+
 // NVFP4: steps of 128 K values (lane q covers K = 128 s + 32 q .. +32: 16
 // code bytes and one scale pair per row); RT row tiles per step, the tiles
 // tstride code bytes (tsc scale pairs) apart, sharing one activation
@@ -700,19 +739,19 @@ __device__ void direct_unit(const MmaArgs& a, const WorkItem& it, int chunk, int
   // whichever class (and kernel) computes it.
   static_assert(NW == RING_WARPS, "the K partition must match the TMA-ring kernel's");
   const Geo gg = geo_of(a, PHASE, FP4);
-  for (int j = 0; j < gg.nsl; ++j) {
-    const int b0 = j * gg.ss, ns = min(gg.ss, gg.steps - b0);
-    const int s0 = b0 + (warp * ns) / NW, s1 = b0 + ((warp + 1) * ns) / NW;
-    if constexpr (FP4) {
+  if constexpr (FP4) {
+    for (int j = 0; j < gg.nsl; ++j) {
+      const int b0 = j * gg.ss, ns = min(gg.ss, gg.steps - b0);
+      const int s0 = b0 + (warp * ns) / NW, s1 = b0 + ((warp + 1) * ns) / NW;
       dot_nvfp4<NB, RT, PHASE == 1>(blob + oa + q * 16, blob + ob + q * 16,
                                     reinterpret_cast<const unsigned short*>(blob + sa0) + q,
                                     reinterpret_cast<const unsigned short*>(blob + sb0) + q,
                                     (size_t)rows_per_tile * rbytes, (size_t)rows_per_tile * sbytes / 2, s0, s1, xr, q,
                                     acc);
-    } else {
-      static_assert(FP4 || RT == 1, "BF16 units are one row tile");
-      dot_bf16<NB, (NB == 1 ? 8 : 4), PHASE == 1>(blob + oa + q * 16, blob + ob + q * 16, s0, s1, xr, xl, q, acc[0]);
     }
+  } else {
+    static_assert(FP4 || RT == 1, "BF16 units are one row tile");
+    dot_bf16_slices<NB, 8, PHASE == 1, NW>(blob + oa + q * 16, blob + ob + q * 16, gg, warp, xr, xl, q, acc[0]);
   }
   // split-K reduction over the warps, in warp order; red is [NW][RT][NB][4][32]
 #pragma unroll
