@@ -1,29 +1,28 @@
 // Decode grouped GEMV for BF16 and NVFP4 experts on warp-level tensor-core
 // MMAs (mma.sync m16n8k16, fp32 accumulate): gate/up + SwiGLU and down in one
-// persistent launch per work class (experts hit in HBM slots, staged into
-// slots by the copy engine, or streamed from the mapped host pool).
+// persistent launch per work class, weights streamed with 128-bit loads from
+// HBM slots or straight from the mapped host pool.
 //
 // Small-batch decode is memory bound ([paperlens] "壁2: デコードのミスを「どう捌く
 // か」が決まっていない", paper §2.2): every weight byte is read once, so the
-// kernel keeps many bytes in flight and spends few instructions per byte.
+// kernel keeps many loads in flight and spends few instructions per byte.
 //
 // Work unit: 16 weight rows x one chunk of <= 16 tokens of one expert. One
-// producer warp takes the units by atomic ticket and has the TMA engine copy,
-// per K slice, the unit's 16 weight-row pieces AND the matching pieces of the
-// chunk's activation rows (x for gate/up, h for down) into one stage of a
-// 4-stage shared-memory ring (cp.async.bulk, mbarrier completion, one row per
-// lane). Eight MMA warps split each slice's K steps and read every operand
-// from shared memory, so no warp waits on a global load; they accumulate over
-// the unit's slices and reduce their partial sums in warp order. Host reads
-// of a streamed expert are large contiguous requests.
+// producer warp takes the units by atomic ticket and has the TMA engine copy
+// their weight rows (K slices of <= 2 KB per row, cp.async.bulk) into a
+// 4-stage shared-memory ring; eight MMA warps split each slice's K range
+// (split-K), accumulate over the unit's slices and reduce their partial sums in
+// warp order through shared memory. The ring decouples the bytes in flight
+// from registers, and every host read of a streamed expert is a large
+// contiguous request instead of scattered 64-byte fragments.
 //
 // Inside a warp, lane (g, q) = (lane/4, lane%4) reads 16 consecutive bytes of
 // rows g and g+8 per step and hands them to the MMA unchanged as its A
 // fragment; that fixes a lane-dependent order of the K positions, which a dot
-// product does not care about as long as the activations (B fragment) are read
-// in the same order. The summation order is fixed by the code and every class
-// runs the same kernel, so an expert's result does not depend on where its
-// weights were read from ([paperlens] "設計: 2階建てのエキスパート記憶", paper §3.3).
+// product does not care about as long as the activations (B fragment) are
+// loaded in the same order. No shuffles, and the summation order is fixed by
+// the code, so an expert's result does not depend on where its weights were
+// read from ([paperlens] "設計: 2階建てのエキスパート記憶", paper §3.3).
 //
 // Phase 0 units (gate/up): tile rows 0..7 are gate rows f0..f0+7 and rows
 // 8..15 the matching up rows, so one lane holds gate and up of the same
@@ -31,13 +30,12 @@
 // f16 (NVFP4 experts) or as bf16 hi + lo parts (BF16 experts: both parts are
 // multiplied by W_down, keeping h to ~2^-16; one bf16 rounding of h would eat
 // most of the 2e-2 rms budget that the bf16 output rounding leaves).
-// Phase 1 units (down) of an (expert, chunk) need all its phase-0 units'
-// h: units are handed out in ticket order (gate/up tickets first) and the
-// producer, before it copies a down unit's h rows, waits (bounded) on a
-// per-chunk completion counter. A CTA holds tickets in increasing order and
-// posts each unit's stages before taking the next, so when its producer waits
-// every gate/up unit it holds is fully posted and its MMA warps finish it
-// alone; every unit waited for is held by a running CTA: no deadlock whatever
+// Phase 1 units (down) of an (expert, chunk) start once all its phase-0 units
+// have published h: units are handed out in ticket order (gate/up tickets
+// first) and a down unit waits, bounded, on a per-chunk completion counter.
+// A CTA holds tickets in increasing order and finishes them in that order, so
+// when it waits on a down unit it holds no unfinished gate/up unit; every unit
+// waited for is held by a running CTA that does not wait: no deadlock whatever
 // the residency.
 //
 // NVFP4: 32 e2m1 codes per lane are converted to f16 pairs (cvt e2m1x2) and
@@ -54,29 +52,31 @@ namespace {
 
 constexpr int CHUNK = 16;  // tokens per unit (two n8 tiles)
 constexpr long long WAIT_CYCLES = mb::WAIT_CYCLES;
-constexpr int NW = 8;                   // MMA (consumer) warps
-constexpr int THREADS = (NW + 1) * 32;  // + one producer warp
-constexpr int NST = 4;                  // ring stages
-constexpr int ROWS = 16;                // weight rows per unit
-
-// Stage layout, per K slice of KS values: 16 weight-row pieces, (NVFP4) their
-// block scales, up to 16 activation-row pieces and (BF16 down units) the h low
-// parts. Rows are padded by 16 bytes so that consecutive rows start 4 banks
-// apart and a warp's fragment reads are conflict-free.
-template <bool FP4> struct Lay {
-  static constexpr int KS = FP4 ? 1024 : 512;                    // K values per slice
-  static constexpr int STEP = FP4 ? 128 : 32;                    // K values per MMA step (64 code bytes)
-  static constexpr int WROW = (FP4 ? KS / 2 : KS * 2) + 16;      // code bytes per row + pad
-  static constexpr int SROW = FP4 ? KS / 16 + 16 : 0;            // scale bytes per row + pad
-  static constexpr int XROW = KS * 2 + 16;                       // activation bytes per row + pad (bf16 / f16)
-  static constexpr int S_OFF = ROWS * WROW;
-  static constexpr int X_OFF = S_OFF + ROWS * SROW;
-  static constexpr int L_OFF = X_OFF + CHUNK * XROW;
-  static constexpr int BYTES = L_OFF + (FP4 ? 0 : CHUNK * XROW);
-};
-constexpr int STAGE_BYTES = Lay<false>::BYTES > Lay<true>::BYTES ? Lay<false>::BYTES : Lay<true>::BYTES;
+constexpr int NW = 8;                            // MMA (consumer) warps
+constexpr int RING_WARPS = NW;
+constexpr int THREADS = (NW + 1) * 32;           // + one producer warp
+constexpr int NST = 4;                           // ring stages
+constexpr int ROWS = 16;                         // weight rows per unit / stage
+constexpr int SLICE = 2048;                      // max code bytes per row per stage
+constexpr int CODE_RS = SLICE + 16;              // smem row stride: rows start 4 banks apart
+constexpr int SC_RS = SLICE / 8 + 16;            // same for the NVFP4 block scales
+constexpr int STAGE_BYTES = ROWS * CODE_RS + ROWS * SC_RS;
 constexpr int RING_BYTES = NST * STAGE_BYTES;
-static_assert(STAGE_BYTES % 16 == 0, "stages start 16-byte aligned");
+
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// L2-coherent load (for h, written by other CTAs of the same launch).
+__device__ __forceinline__ uint4 ld_cg(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
 
 __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
@@ -177,6 +177,56 @@ __device__ __forceinline__ uint32_t lds16(uint32_t addr) {
 // Barrier among the MMA warps only (the producer warp runs on its own).
 __device__ __forceinline__ void mma_warps_sync() { asm volatile("bar.sync 1, %0;" ::"r"(NW * 32) : "memory"); }
 
+// acc[t] += rows g, g+8 of one stage . X over this warp's steps [s0, s1) of
+// the stage; step s covers 64 code bytes of each row (32 bf16 / 128 e2m1
+// values), lane q its 16-byte quarter; kb = first global step of the stage.
+// The activation rows xr / xl (h hi / lo parts for BF16 down units) are read
+// in the same lane-permuted K order.
+template <int NB, bool FP4, bool P1>
+__device__ __forceinline__ void stage_dot(uint32_t code, uint32_t sc, int s0, int s1, int kb,
+                                          const uint16_t* const (&xr)[NB], const uint16_t* const (&xl)[NB], int g,
+                                          int q, float (&acc)[NB][4]) {
+  const uint32_t ra = code + g * CODE_RS + q * 16, rb = ra + 8 * CODE_RS;
+  for (int s = s0; s < s1; ++s) {
+    const uint4 wa = lds128(ra + s * 64), wb = lds128(rb + s * 64);
+    if constexpr (FP4) {
+      const uint32_t ca = lds16(sc + g * SC_RS + s * 8 + q * 2), cb = lds16(sc + (g + 8) * SC_RS + s * 8 + q * 2);
+      uint32_t ha[16], hb[16];
+      decode_nvfp4(wa, ca, ha);
+      decode_nvfp4(wb, cb, hb);
+#pragma unroll
+      for (int t = 0; t < NB; ++t) {
+        const uint16_t* xp = xr[t] + (kb + s) * 128 + q * 32;
+        uint32_t xh[16];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint4 xv = P1 ? ld_cg(xp + 8 * v) : __ldg(reinterpret_cast<const uint4*>(xp) + v);
+          xh[4 * v] = xv.x;
+          xh[4 * v + 1] = xv.y;
+          xh[4 * v + 2] = xv.z;
+          xh[4 * v + 3] = xv.w;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          mma_f16(acc[t], ha[2 * j], hb[2 * j], ha[2 * j + 1], hb[2 * j + 1], xh[2 * j], xh[2 * j + 1]);
+      }
+    } else {
+      const int e0 = (kb + s) * 32 + q * 8;
+#pragma unroll
+      for (int t = 0; t < NB; ++t) {
+        const uint4 xv = P1 ? ld_cg(xr[t] + e0) : __ldg(reinterpret_cast<const uint4*>(xr[t] + e0));
+        mma_bf16(acc[t], wa.x, wb.x, wa.y, wb.y, xv.x, xv.y);
+        mma_bf16(acc[t], wa.z, wb.z, wa.w, wb.w, xv.z, xv.w);
+        if constexpr (P1) {
+          const uint4 xo = ld_cg(xl[t] + e0);
+          mma_bf16(acc[t], wa.x, wb.x, wa.y, wb.y, xo.x, xo.y);
+          mma_bf16(acc[t], wa.z, wb.z, wa.w, wb.w, xo.z, xo.w);
+        }
+      }
+    }
+  }
+}
+
 // Map a unit index within a phase to (item, 16-token chunk, row block) and
 // the item-chunk index qi.
 __device__ __forceinline__ bool unit_of(const int* pref, int n_items, int rblocks, int u, int& item, int& chunk,
@@ -194,77 +244,23 @@ __device__ __forceinline__ bool unit_of(const int* pref, int n_items, int rblock
   return true;
 }
 
-// Generic-proxy writes of other CTAs (h), made visible by their release and
-// this thread's acquire, before the async proxy (TMA) reads them.
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
-
-// K geometry of a phase: steps of 64 code bytes per row, cut into slices of
-// KS values (the last may be shorter; NVFP4 slices hold an even number of
-// steps, so a slice's scales are a multiple of 16 bytes).
+// Row geometry of a phase: 64-byte steps per row and how they are cut into
+// ring slices of <= SLICE bytes (an even number of steps, so an NVFP4
+// slice's scales are a multiple of 16 bytes).
 struct Geo {
-  int K, steps, nsl, ss;  // K values, steps per row, slices, steps per slice
+  int steps, nsl, ss;       // steps per row, slices, steps per slice (last may be shorter)
+  size_t row_bytes, sc_row; // code / scale bytes per row
 };
-template <bool FP4>
-__device__ __forceinline__ Geo geo_of(const MmaArgs& a, int phase) {
+__device__ __forceinline__ Geo geo_of(const MmaArgs& a, int phase, bool fp4) {
   Geo g;
-  g.K = phase == 0 ? a.d : a.d_ff;
-  g.steps = g.K / Lay<FP4>::STEP;
-  g.ss = Lay<FP4>::KS / Lay<FP4>::STEP;
-  g.nsl = (g.steps + g.ss - 1) / g.ss;
+  const int K = phase == 0 ? a.d : a.d_ff;
+  g.row_bytes = fp4 ? (size_t)K / 2 : (size_t)K * 2;
+  g.sc_row = fp4 ? (size_t)K / 16 : 0;
+  g.steps = (int)(g.row_bytes / 64);
+  g.nsl = (int)((g.row_bytes + SLICE - 1) / SLICE);
+  g.ss = (g.steps + g.nsl - 1) / g.nsl;
+  g.ss += g.ss & 1;
   return g;
-}
-
-// acc[t] += rows g, g+8 of a stage . X over this warp's steps [s0, s1) of the
-// stage; the activation rows come from the same stage (row j of token tile t
-// is token t*8+g of the chunk, or row 0 for padding lanes, whose results are
-// not stored).
-template <int NB, bool FP4, bool P1>
-__device__ __forceinline__ void stage_dot(uint32_t st, int s0, int s1, int nt, int g, int q, float (&acc)[NB][4]) {
-  using L = Lay<FP4>;
-  const uint32_t ra = st + g * L::WROW + q * 16, rb = ra + 8 * L::WROW;
-  uint32_t xa[NB];
-#pragma unroll
-  for (int t = 0; t < NB; ++t) {
-    const int j = t * 8 + g;
-    xa[t] = st + L::X_OFF + (j < nt ? j : 0) * L::XROW;
-  }
-  for (int s = s0; s < s1; ++s) {
-    const uint4 wa = lds128(ra + s * 64), wb = lds128(rb + s * 64);
-    if constexpr (FP4) {
-      const uint32_t sc = st + L::S_OFF + s * 8 + q * 2;
-      const uint32_t ca = lds16(sc + g * L::SROW), cb = lds16(sc + (g + 8) * L::SROW);
-      uint32_t ha[16], hb[16];
-      decode_nvfp4(wa, ca, ha);
-      decode_nvfp4(wb, cb, hb);
-#pragma unroll
-      for (int t = 0; t < NB; ++t) {
-        uint32_t xh[16];
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const uint4 xv = lds128(xa[t] + s * 256 + q * 64 + v * 16);
-          xh[4 * v] = xv.x;
-          xh[4 * v + 1] = xv.y;
-          xh[4 * v + 2] = xv.z;
-          xh[4 * v + 3] = xv.w;
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          mma_f16(acc[t], ha[2 * j], hb[2 * j], ha[2 * j + 1], hb[2 * j + 1], xh[2 * j], xh[2 * j + 1]);
-      }
-    } else {
-#pragma unroll
-      for (int t = 0; t < NB; ++t) {
-        const uint4 xv = lds128(xa[t] + s * 64 + q * 16);
-        mma_bf16(acc[t], wa.x, wb.x, wa.y, wb.y, xv.x, xv.y);
-        mma_bf16(acc[t], wa.z, wb.z, wa.w, wb.w, xv.z, xv.w);
-        if constexpr (P1) {
-          const uint4 xo = lds128(xa[t] + (L::L_OFF - L::X_OFF) + s * 64 + q * 16);
-          mma_bf16(acc[t], wa.x, wb.x, wa.y, wb.y, xo.x, xo.y);
-          mma_bf16(acc[t], wa.z, wb.z, wa.w, wb.w, xo.z, xo.w);
-        }
-      }
-    }
-  }
 }
 
 struct StageMeta {
@@ -273,18 +269,17 @@ struct StageMeta {
 constexpr int SM_FIRST = 1, SM_LAST = 2, SM_BAD = 4, SM_END = 8;
 
 // Producer: the last warp fills the ring. Lane 0 takes the tickets (the next
-// one always in flight), waits for free slots and posts each stage; then the
-// lanes issue the stage's bulk copies in parallel: lane i < 16 the code piece
-// of weight row i, lane 16 + i (NVFP4) its scales; then lane j < nt the piece
-// of activation row j and (BF16 down units) lane 16 + j its h low part.
+// one always in flight), waits for free slots and posts each stage; then each
+// lane issues one bulk copy of the stage (lane i < 16: the codes of smem row i;
+// lane 16 + i, NVFP4 only: that row's block scales), so the 16-32 copies of a
+// stage go out in parallel instead of one after another.
 template <bool FP4>
 __device__ void produce(const MmaArgs& a, const WorkItem* items, const int* pref, int n_items, int rb0, int rb1,
                         int U0, int U1, uint8_t* ring, volatile StageMeta* meta, uint32_t full, uint32_t empty,
                         volatile int* abort, int lane) {
-  using L = Lay<FP4>;
   const size_t n = (size_t)a.d * a.d_ff;
-  const size_t mat = FP4 ? n / 2 : n * 2;           // code bytes per matrix
-  const size_t sc0 = 3 * (n / 2), scm = n / 16;      // NVFP4 scales: start, bytes per matrix
+  const size_t mat = FP4 ? n / 2 : n * 2;          // code bytes per matrix
+  const size_t sc0 = 3 * (n / 2), scm = n / 16;     // NVFP4 scales: start, bytes per matrix
   // per slot (lane 0): the last round posted and whether it carried copies.
   // Only that round can still be in flight at exit (posting a round waits for
   // the consumers to release the one before it); a sentinel or skipped stage
@@ -296,9 +291,13 @@ __device__ void produce(const MmaArgs& a, const WorkItem* items, const int* pref
   bool last_copy[NST];
 #pragma unroll
   for (int i = 0; i < NST; ++i) last_round[i] = -1, last_copy[i] = false;
+  // the next ticket is always in flight while a unit's copies are issued (a
+  // global atomic's round trip would otherwise stall every unit); holding it
+  // keeps the order argument: every ticket a CTA holds is later than the unit
+  // its MMA warps work on
   int nxt = lane == 0 ? atomicAdd(a.ticket, 1) : 0;
-  const int row = lane & 15;
-  const bool hi_lane = lane >= 16;
+  const int row = lane & 15;  // smem row this lane copies
+  const bool sc_lane = lane >= 16;
   for (bool done = false; !done;) {
     const int u = __shfl_sync(0xffffffffu, nxt, 0);
     if (u >= U0 + U1) {  // end of work: one sentinel stage
@@ -320,57 +319,28 @@ __device__ void produce(const MmaArgs& a, const WorkItem* items, const int* pref
     const WorkItem wi = items[item];
     const bool bad = a.cls != KIND_STREAMED && (wi.slot < 0 || wi.slot >= a.C);  // error already latched
     const uint8_t* blob = bad ? nullptr : blob_of(a, wi);
-    const int base = wi.tok_off + chunk * CHUNK;
-    const int nt = min(CHUNK, wi.n_tok - chunk * CHUNK);
-    if (!bad && ((a.landed && item > landed_upto) || phase == 1)) {
+    if (a.landed && !bad && item > landed_upto) {
+      // a staged expert: its slot is readable once the copy stream has
+      // written this call's epoch behind the blob's copy (items are in copy order)
       if (lane == 0) {
         const long long t0 = clock64();
-        if (a.landed && item > landed_upto) {
-          // a staged expert: its slot is readable once the copy stream has
-          // written this call's epoch behind the blob's copy (items in copy order)
-          while (ld_acquire(a.landed + item) != a.epoch) {
-            if (*abort) break;
-            if (clock64() - t0 > WAIT_CYCLES) {
-              *abort = 1;
-              atomicExch(a.error, (uint32_t)DERR_TIMEOUT);
-              break;
-            }
+        while (ld_acquire(a.landed + item) != a.epoch) {
+          if (*abort) break;
+          if (clock64() - t0 > WAIT_CYCLES) {
+            *abort = 1;
+            atomicExch(a.error, (uint32_t)DERR_TIMEOUT);
+            break;
           }
         }
-        if (phase == 1) {
-          // every gate/up unit of this (item, chunk) must have published h
-          while (ld_acquire(reinterpret_cast<const uint32_t*>(a.done + qi)) < (uint32_t)rb0) {
-            if (*abort) break;
-            if (clock64() - t0 > WAIT_CYCLES) {
-              *abort = 1;
-              atomicExch(a.error, (uint32_t)DERR_TIMEOUT);
-              break;
-            }
-          }
-        }
-        fence_proxy_async();
       }
       __syncwarp();
-      if (a.landed) landed_upto = max(landed_upto, item);
+      landed_upto = item;
     }
-    // this lane's rows: weight row `row` (phase 0: gate row 8 rb + row for row
-    // < 8, else up row 8 rb + row - 8; phase 1: down row 16 rb + row) and
-    // activation row `row` of the chunk (x of its token, or its h row)
+    const Geo g = geo_of(a, phase, FP4);
+    // this lane's source row: smem row i -> gate row 8 rb + i (i < 8) or up row
+    // 8 rb + i - 8 (phase 0); down row 16 rb + i (phase 1)
     const size_t m = phase == 0 ? (row < 8 ? 0 : 1) : 2;
     const size_t grow = phase == 0 ? (size_t)rb * 8 + (row & 7) : (size_t)rb * 16 + row;
-    const Geo g = geo_of<FP4>(a, phase);
-    const size_t wrow_bytes = FP4 ? (size_t)g.K / 2 : (size_t)g.K * 2, srow_bytes = (size_t)g.K / 16;
-    const uint8_t* xsrc = nullptr;
-    const uint8_t* lsrc = nullptr;
-    if (row < nt) {
-      if (phase == 0) {
-        const int tok = a.perm[base + row] / a.k;
-        xsrc = reinterpret_cast<const uint8_t*>(a.x) + (size_t)tok * a.d * 2;
-      } else {
-        xsrc = reinterpret_cast<const uint8_t*>(a.h16) + (size_t)(base + row) * a.d_ff * 2;
-        if (!FP4) lsrc = reinterpret_cast<const uint8_t*>(a.h16lo) + (size_t)(base + row) * a.d_ff * 2;
-      }
-    }
     for (int sl = 0; sl < g.nsl; ++sl, ++it) {
       const int slot = it % NST, r = it / NST;
       int ok = 1;
@@ -391,29 +361,20 @@ __device__ void produce(const MmaArgs& a, const WorkItem* items, const int* pref
       }
       const uint32_t bar = full + 8 * slot;
       const int s0 = sl * g.ss, ns = min(g.ss, g.steps - s0);
-      const int k0 = s0 * L::STEP, kv = ns * L::STEP;  // first K value and K values of the slice
-      const uint32_t cb = FP4 ? (uint32_t)kv / 2 : (uint32_t)kv * 2, sb = FP4 ? (uint32_t)kv / 16 : 0;
-      const uint32_t xb = (uint32_t)kv * 2;
+      const uint32_t cb = (uint32_t)ns * 64, sb = FP4 ? (uint32_t)ns * 8 : 0;
       if (lane == 0) {
         if (bad)
           mb::arrive(bar);
         else
-          mb::expect_tx(bar, ROWS * (cb + sb) + nt * xb * ((!FP4 && phase == 1) ? 2 : 1));
+          mb::expect_tx(bar, ROWS * (cb + sb));
       }
       __syncwarp();  // the expected bytes are posted before any copy can complete them
       if (bad) continue;
-      const uint32_t st = mb::smem_u32(ring + slot * STAGE_BYTES);
-      if (!hi_lane)
-        mb::bulk_g2s(st + row * L::WROW, blob + m * mat + grow * wrow_bytes + (FP4 ? (size_t)k0 / 2 : (size_t)k0 * 2),
-                     cb, bar);
+      const uint32_t code = mb::smem_u32(ring + slot * STAGE_BYTES), scs = code + ROWS * CODE_RS;
+      if (!sc_lane)
+        mb::bulk_g2s(code + row * CODE_RS, blob + m * mat + grow * g.row_bytes + (size_t)s0 * 64, cb, bar);
       else if (FP4)
-        mb::bulk_g2s(st + L::S_OFF + row * L::SROW, blob + sc0 + m * scm + grow * srow_bytes + (size_t)k0 / 16, sb, bar);
-      if (row < nt) {
-        if (!hi_lane)
-          mb::bulk_g2s(st + L::X_OFF + row * L::XROW, xsrc + (size_t)k0 * 2, xb, bar);
-        else if (!FP4 && phase == 1)
-          mb::bulk_g2s(st + L::L_OFF + row * L::XROW, lsrc + (size_t)k0 * 2, xb, bar);
-      }
+        mb::bulk_g2s(scs + row * SC_RS, blob + sc0 + m * scm + grow * g.sc_row + (size_t)s0 * 8, sb, bar);
     }
   }
   // every copy issued must have landed before the CTA's shared memory goes away
@@ -475,6 +436,8 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_fused_kernel(MmaArgs a) {
   } else {
     const int g = lane >> 2, q = lane & 3;
     float acc[NB][4];
+    const uint16_t* xr[NB];
+    const uint16_t* xl[NB];
     int phase = 0, item = 0, chunk = 0, rb = 0, qi = 0, base = 0, nt = 0;
     Geo geo{};
     for (int it = 0;; ++it) {
@@ -494,20 +457,46 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_fused_kernel(MmaArgs a) {
         phase = u < U0 ? 0 : 1;
         unit_of(s_pref, n_items, phase == 0 ? rb0 : rb1, phase == 0 ? u : u - U0, item, chunk, rb, qi);
         const WorkItem wi = s_items[item];
-        geo = geo_of<FP4>(a, phase);
+        geo = geo_of(a, phase, FP4);
         base = wi.tok_off + chunk * CHUNK;
         nt = min(CHUNK, wi.n_tok - chunk * CHUNK);
 #pragma unroll
-        for (int t = 0; t < NB; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+        for (int t = 0; t < NB; ++t) {
+          const int j = t * 8 + g;
+          const int pos = base + (j < nt ? j : 0);
+          if (phase == 0) {
+            xr[t] = reinterpret_cast<const uint16_t*>(a.x) + (size_t)(a.perm[pos] / a.k) * a.d;
+            xl[t] = xr[t];
+          } else {
+            xr[t] = a.h16 + (size_t)pos * a.d_ff;
+            xl[t] = FP4 ? xr[t] : a.h16lo + (size_t)pos * a.d_ff;
+          }
+          acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+        }
+        if (phase == 1) {
+          // every gate/up unit of this (item, chunk) must have published h
+          if (tid == 0) {
+            const long long t0 = clock64();
+            volatile int32_t* dn = a.done + qi;
+            while (*dn < rb0) {
+              if (clock64() - t0 > WAIT_CYCLES) {
+                atomicExch(a.error, (uint32_t)DERR_TIMEOUT);
+                break;
+              }
+            }
+            __threadfence();
+          }
+          mma_warps_sync();
+        }
       }
       if (!(flags & SM_BAD)) {
-        const int ns = min(geo.ss, geo.steps - sl * geo.ss);
+        const int s0 = sl * geo.ss, ns = min(geo.ss, geo.steps - s0);
         const int w0 = (warp * ns) / NW, w1 = ((warp + 1) * ns) / NW;
-        const uint32_t st = mb::smem_u32(ring + slot * STAGE_BYTES);
+        const uint32_t code = mb::smem_u32(ring + slot * STAGE_BYTES), scs = code + ROWS * CODE_RS;
         if (phase == 0)
-          stage_dot<NB, FP4, false>(st, w0, w1, nt, g, q, acc);
+          stage_dot<NB, FP4, false>(code, scs, w0, w1, s0, xr, xl, g, q, acc);
         else
-          stage_dot<NB, FP4, true>(st, w0, w1, nt, g, q, acc);
+          stage_dot<NB, FP4, true>(code, scs, w0, w1, s0, xr, xl, g, q, acc);
       }
       __syncwarp();
       if (lane == 0) mb::arrive(empty + 8 * slot);  // this warp is done with the stage
@@ -563,6 +552,340 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_fused_kernel(MmaArgs a) {
   __syncthreads();
 }
 
+// One BF16 step: 8 K values of rows g and g+8 per lane, two MMAs per token
+// tile (and two more for the low part of h in phase 1).
+template <int NB, bool P1>
+__device__ __forceinline__ void bf16_step(const uint4 wa, const uint4 wb, const uint16_t* const (&xr)[NB],
+                                          const uint16_t* const (&xl)[NB], int e0, float (&acc)[NB][4]) {
+#pragma unroll
+  for (int t = 0; t < NB; ++t) {
+    const uint4 xv = P1 ? ld_cg(xr[t] + e0) : __ldg(reinterpret_cast<const uint4*>(xr[t] + e0));
+    mma_bf16(acc[t], wa.x, wb.x, wa.y, wb.y, xv.x, xv.y);
+    mma_bf16(acc[t], wa.z, wb.z, wa.w, wb.w, xv.z, xv.w);
+    if constexpr (P1) {
+      const uint4 xo = ld_cg(xl[t] + e0);
+      mma_bf16(acc[t], wa.x, wb.x, wa.y, wb.y, xo.x, xo.y);
+      mma_bf16(acc[t], wa.z, wb.z, wa.w, wb.w, xo.z, xo.w);
+    }
+  }
+}
+
+// acc[t][.] += W[rows g, g+8] . X[tokens] over steps [s0, s1) of 32 K values
+// (lane q covers K = 32 s + 8 q .. +8). U steps of loads in flight; steps past
+// s1 reload the last step and are not used.
+template <int NB, int U, bool P1>
+__device__ __forceinline__ void dot_bf16(const uint8_t* ra, const uint8_t* rb, int s0, int s1,
+                                         const uint16_t* const (&xr)[NB], const uint16_t* const (&xl)[NB], int q,
+                                         float (&acc)[NB][4]) {
+  for (int s = s0; s < s1; s += U) {
+    uint4 wa[U], wb[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int ss = s + u < s1 ? s + u : s1 - 1;
+      wa[u] = ld_stream(ra + (size_t)ss * 64);
+      wb[u] = ld_stream(rb + (size_t)ss * 64);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (s + u < s1) bf16_step<NB, P1>(wa[u], wb[u], xr, xl, (s + u) * 32 + q * 8, acc);
+  }
+}
+
+// The same over this warp's K steps of every ring slice (slice j: sub-range
+// warp of NW of [j*ss, j*ss + ns_j)), gathered across slice boundaries into
+// batches of U loads in flight; the MMAs run in slice order, step by step, so
+// the sum is exactly the TMA-ring kernel's.
+template <int NB, int U, bool P1, int NWARPS>
+__device__ __forceinline__ void dot_bf16_slices(const uint8_t* ra, const uint8_t* rb, const Geo& g, int warp,
+                                                const uint16_t* const (&xr)[NB], const uint16_t* const (&xl)[NB],
+                                                int q, float (&acc)[NB][4]) {
+  int j = 0;
+  int lo = (warp * min(g.ss, g.steps)) / NWARPS, hi = ((warp + 1) * min(g.ss, g.steps)) / NWARPS;
+  int s = lo;
+  for (;;) {
+    int st[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      while (s >= hi && j + 1 < g.nsl) {
+        ++j;
+        const int b0 = j * g.ss, ns = min(g.ss, g.steps - b0);
+        lo = b0 + (warp * ns) / NWARPS;
+        hi = b0 + ((warp + 1) * ns) / NWARPS;
+        s = lo;
+      }
+      st[u] = s < hi ? s : -1;
+      s += s < hi ? 1 : 0;
+    }
+    if (st[0] < 0) break;
+    uint4 wa[U], wb[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int ss = st[u] >= 0 ? st[u] : st[0];
+      wa[u] = ld_stream(ra + (size_t)ss * 64);
+      wb[u] = ld_stream(rb + (size_t)ss * 64);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (st[u] >= 0) bf16_step<NB, P1>(wa[u], wb[u], xr, xl, st[u] * 32 + q * 8, acc);
+  }
+}
+
+// NVFP4: steps of 128 K values (lane q covers K = 128 s + 32 q .. +32: 16
+// code bytes and one scale pair per row); RT row tiles per step, the tiles
+// tstride code bytes (tsc scale pairs) apart, sharing one activation
+// fragment; eight MMAs per step, tile and token tile.
+template <int NB, int RT, bool P1>
+__device__ __forceinline__ void dot_nvfp4(const uint8_t* ra, const uint8_t* rb, const unsigned short* sa,
+                                          const unsigned short* sb, size_t tstride, size_t tsc, int s0, int s1,
+                                          const uint16_t* const (&xr)[NB], int q, float (&acc)[RT][NB][4]) {
+  for (int s = s0; s < s1; ++s) {
+    uint4 wa[RT], wb[RT];
+    uint32_t ca[RT], cb[RT];
+#pragma unroll
+    for (int r = 0; r < RT; ++r) {
+      wa[r] = ld_stream(ra + r * tstride + (size_t)s * 64);
+      wb[r] = ld_stream(rb + r * tstride + (size_t)s * 64);
+      ca[r] = __ldg(sa + r * tsc + s * 4);
+      cb[r] = __ldg(sb + r * tsc + s * 4);
+    }
+    uint32_t xh[NB][16];
+#pragma unroll
+    for (int t = 0; t < NB; ++t) {
+      const uint16_t* xp = xr[t] + s * 128 + q * 32;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const uint4 xv = P1 ? ld_cg(xp + 8 * v) : __ldg(reinterpret_cast<const uint4*>(xp) + v);
+        xh[t][4 * v] = xv.x;
+        xh[t][4 * v + 1] = xv.y;
+        xh[t][4 * v + 2] = xv.z;
+        xh[t][4 * v + 3] = xv.w;
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < RT; ++r) {
+      uint32_t ha[16], hb[16];
+      decode_nvfp4(wa[r], ca[r], ha);
+      decode_nvfp4(wb[r], cb[r], hb);
+#pragma unroll
+      for (int t = 0; t < NB; ++t)
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          mma_f16(acc[r][t], ha[2 * j], hb[2 * j], ha[2 * j + 1], hb[2 * j + 1], xh[t][2 * j], xh[t][2 * j + 1]);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Direct-load variant for experts resident in HBM slots (the hit class): the
+// MMA warps load their weight fragments straight into registers, U steps in
+// flight, several CTAs per SM, so load latency is hidden by many warps. (The
+// TMA ring above serves the staged and streamed classes, whose bytes arrive
+// over the host link anyway.)
+// ---------------------------------------------------------------------------
+
+// One unit: RT tiles of 16 weight rows x one chunk of <= 16 tokens, the K
+// range split over the NW warps, partial sums reduced in warp order, epilogue
+// of tile r by warp r. Tile r of unit rb is row block rb*RT + r: gate rows
+// 8 (rb*RT + r) + g with the matching up rows (phase 0), down rows
+// 16 (rb*RT + r) + g and + 8 (phase 1).
+template <int NB, int PHASE, bool FP4, int NW, int RT>
+__device__ void direct_unit(const MmaArgs& a, const WorkItem& it, int chunk, int rb, int warp, int lane, float* red) {
+  const int g = lane >> 2, q = lane & 3;
+  const uint8_t* blob = blob_of(a, it);
+  const size_t n = (size_t)a.d * a.d_ff;
+  const int K = PHASE == 0 ? a.d : a.d_ff;
+  const size_t rbytes = FP4 ? (size_t)K / 2 : (size_t)K * 2;
+  const size_t sbytes = (size_t)K / 16;
+  const int steps = FP4 ? K / 128 : K / 32;
+  (void)steps;
+  const int rows_per_tile = PHASE == 0 ? 8 : 16;  // per weight matrix
+  const int blk0 = rb * RT;                       // first row block of the unit
+  size_t oa, ob, sa0, sb0;
+  if (PHASE == 0) {
+    oa = (size_t)(blk0 * 8 + g) * rbytes;
+    ob = (FP4 ? n / 2 : n * 2) + (size_t)(blk0 * 8 + g) * rbytes;
+    sa0 = 3 * (n / 2) + (size_t)(blk0 * 8 + g) * sbytes;
+    sb0 = 3 * (n / 2) + n / 16 + (size_t)(blk0 * 8 + g) * sbytes;
+  } else {
+    oa = (FP4 ? n : n * 4) + (size_t)(blk0 * 16 + g) * rbytes;
+    ob = oa + 8 * rbytes;
+    sa0 = 3 * (n / 2) + 2 * (n / 16) + (size_t)(blk0 * 16 + g) * sbytes;
+    sb0 = sa0 + 8 * sbytes;
+  }
+  const int base = it.tok_off + chunk * CHUNK;
+  const int nt = min(CHUNK, it.n_tok - chunk * CHUNK);
+  const uint16_t* xr[NB];
+  const uint16_t* xl[NB];
+#pragma unroll
+  for (int t = 0; t < NB; ++t) {
+    const int j = t * 8 + g;
+    const int pos = base + (j < nt ? j : 0);
+    if (PHASE == 0) {
+      xr[t] = reinterpret_cast<const uint16_t*>(a.x) + (size_t)(a.perm[pos] / a.k) * a.d;
+      xl[t] = xr[t];
+    } else {
+      xr[t] = a.h16 + (size_t)pos * a.d_ff;
+      xl[t] = FP4 ? xr[t] : a.h16lo + (size_t)pos * a.d_ff;
+    }
+  }
+  float acc[RT][NB][4];
+#pragma unroll
+  for (int r = 0; r < RT; ++r)
+#pragma unroll
+    for (int t = 0; t < NB; ++t) acc[r][t][0] = acc[r][t][1] = acc[r][t][2] = acc[r][t][3] = 0.f;
+  // The K steps this warp covers are the TMA-ring kernel's: for each ring
+  // slice j in order, sub-range w of NW = 8. With the same MMA order inside a
+  // warp and the same warp-order reduction, an expert's output is bit-identical
+  // whichever class (and kernel) computes it.
+  static_assert(NW == RING_WARPS, "the K partition must match the TMA-ring kernel's");
+  const Geo gg = geo_of(a, PHASE, FP4);
+  if constexpr (FP4) {
+    for (int j = 0; j < gg.nsl; ++j) {
+      const int b0 = j * gg.ss, ns = min(gg.ss, gg.steps - b0);
+      const int s0 = b0 + (warp * ns) / NW, s1 = b0 + ((warp + 1) * ns) / NW;
+      dot_nvfp4<NB, RT, PHASE == 1>(blob + oa + q * 16, blob + ob + q * 16,
+                                    reinterpret_cast<const unsigned short*>(blob + sa0) + q,
+                                    reinterpret_cast<const unsigned short*>(blob + sb0) + q,
+                                    (size_t)rows_per_tile * rbytes, (size_t)rows_per_tile * sbytes / 2, s0, s1, xr, q,
+                                    acc);
+    }
+  } else {
+    static_assert(FP4 || RT == 1, "BF16 units are one row tile");
+    dot_bf16_slices<NB, 8, PHASE == 1, NW>(blob + oa + q * 16, blob + ob + q * 16, gg, warp, xr, xl, q, acc[0]);
+  }
+  // split-K reduction over the warps, in warp order; red is [NW][RT][NB][4][32]
+#pragma unroll
+  for (int r = 0; r < RT; ++r)
+#pragma unroll
+    for (int t = 0; t < NB; ++t)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) red[(((warp * RT + r) * NB + t) * 4 + c) * 32 + lane] = acc[r][t][c];
+  __syncthreads();
+  if (warp < RT) {
+    const int r = warp;
+    float v[NB][4];
+#pragma unroll
+    for (int t = 0; t < NB; ++t)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float x = red[((r * NB + t) * 4 + c) * 32 + lane];
+        for (int w = 1; w < NW; ++w) x += red[(((w * RT + r) * NB + t) * 4 + c) * 32 + lane];
+        v[t][c] = x;
+      }
+    // d0,d1: row g, tokens 2q, 2q+1; d2,d3: row g+8, same tokens (per n8 tile)
+    float t0 = 1.f, t1 = 1.f;
+    if constexpr (FP4) {
+      const float* ts = a.tscale + ((size_t)a.layer * a.E + it.e) * 3;
+      t0 = PHASE == 0 ? ts[0] : ts[2];
+      t1 = PHASE == 0 ? ts[1] : ts[2];
+    }
+    const int blk = blk0 + r;
+#pragma unroll
+    for (int t = 0; t < NB; ++t) {
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int j = t * 8 + 2 * q + c;
+        if (j >= nt) continue;
+        const float v0 = v[t][c] * t0, v1 = v[t][2 + c] * t1;
+        if (PHASE == 0) {
+          const float hv = v0 / (1.f + expf(-v0)) * v1;
+          const size_t o = (size_t)(base + j) * a.d_ff + blk * 8 + g;
+          if constexpr (FP4) {
+            a.h16[o] = __half_as_ushort(__float2half_rn(hv));
+          } else {
+            const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
+            a.h16[o] = __bfloat16_as_ushort(hi);
+            a.h16lo[o] = __bfloat16_as_ushort(__float2bfloat16_rn(hv - __bfloat162float(hi)));
+          }
+        } else {
+          float* yr = a.ybuf + (size_t)(base + j) * a.d;
+          yr[blk * 16 + g] = v0;
+          yr[blk * 16 + g + 8] = v1;
+        }
+      }
+    }
+    if (PHASE == 0) __threadfence();  // publish h before the unit is counted done
+  }
+  __syncthreads();  // red is reused by the next unit
+}
+
+// Row tiles per unit: NVFP4 rows are a quarter of the BF16 bytes, so a unit
+// takes four tiles to keep the loads in flight per warp and the per-unit
+// reduction and barriers amortised.
+template <bool FP4>
+constexpr int tiles_for() { return FP4 ? 4 : 1; }
+
+template <int NB, bool FP4, int NW>
+__global__ void __launch_bounds__(NW * 32) gemv_direct_kernel(MmaArgs a) {
+  constexpr int RT = tiles_for<FP4>();
+  __shared__ int s_pref[MAX_E + 1];
+  __shared__ WorkItem s_items[MAX_E];
+  __shared__ float red[NW * RT * NB * 4 * 32];
+  __shared__ int s_unit;
+  const int n_items = a.work->n_items[a.cls];
+  if (n_items == 0) return;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < n_items; i += blockDim.x) s_items[i] = a.work->items[a.cls][i];
+  __syncthreads();
+  if (warp == 0) {  // exclusive scan of the chunks per item
+    int carry = 0;
+    for (int b = 0; b < n_items; b += 32) {
+      const int i = b + lane;
+      const int c = i < n_items ? (s_items[i].n_tok + CHUNK - 1) / CHUNK : 0;
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (i < n_items) s_pref[i] = carry + incl - c;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) s_pref[n_items] = carry;
+  }
+  __syncthreads();
+  const int n_qi = s_pref[n_items];
+  const int rb0 = a.d_ff / 8 / RT, rb1 = a.d / 16 / RT;
+  const int U0 = n_qi * rb0, U1 = n_qi * rb1;
+  if (tid == 0) s_unit = atomicAdd(a.ticket, 1);
+  __syncthreads();
+  for (;;) {
+    const int u = s_unit;
+    if (u >= U0 + U1) break;
+    // the next ticket is fetched while this unit runs (phase-0 tickets all
+    // precede phase-1 ones, so holding one never blocks a waited-on unit)
+    int nxt = 0;
+    if (tid == 0) nxt = atomicAdd(a.ticket, 1);
+    const int phase = u < U0 ? 0 : 1;
+    int item, chunk, rb, qi;
+    unit_of(s_pref, n_items, phase == 0 ? rb0 : rb1, phase == 0 ? u : u - U0, item, chunk, rb, qi);
+    const WorkItem it = s_items[item];
+    const bool bad = a.cls != KIND_STREAMED && (it.slot < 0 || it.slot >= a.C);  // error already latched
+    if (phase == 1) {
+      // wait until every gate/up unit of this (item, chunk) has published h
+      if (tid == 0) {
+        const long long t0 = clock64();
+        volatile int32_t* dn = a.done + qi;
+        while (*dn < rb0) {
+          if (clock64() - t0 > WAIT_CYCLES) {
+            atomicExch(a.error, (uint32_t)DERR_TIMEOUT);
+            break;
+          }
+        }
+        __threadfence();
+      }
+      __syncthreads();
+      if (!bad) direct_unit<NB, 1, FP4, NW, RT>(a, it, chunk, rb, warp, lane, red);
+    } else {
+      if (!bad) direct_unit<NB, 0, FP4, NW, RT>(a, it, chunk, rb, warp, lane, red);
+      if (tid == 0) atomicAdd(a.done + qi, 1);
+    }
+    __syncthreads();  // every thread has read s_unit
+    if (tid == 0) s_unit = nxt;
+    __syncthreads();
+  }
+}
+
 // bf16 -> f16 copy of the activations (NVFP4 experts take f16 MMA operands).
 __global__ void __launch_bounds__(256) to_f16_kernel(const __nv_bfloat16* __restrict__ x, int n, __half* __restrict__ y) {
   for (int i = blockIdx.x * 256 + threadIdx.x; i < n; i += gridDim.x * 256) y[i] = __float2half_rn(__bfloat162float(x[i]));
@@ -586,11 +909,34 @@ void launch_nb(int grid, const MmaArgs& a, cudaStream_t st) {
   gemv_fused_kernel<NB, FP4><<<grid, THREADS, RING_BYTES, st>>>(a);
 }
 
+// Warps per CTA of the direct-load kernel: the ring kernel's eight, so both
+// split K the same way (see direct_unit).
+template <int NB>
+constexpr int warps_for() { return RING_WARPS; }
+
+int g_grid_direct[2][3] = {{0, 0, 0}, {0, 0, 0}};  // [fp4][NB]
+
+template <int NB, bool FP4>
+cudaError_t direct_setup(int sms) {
+  constexpr int NW = warps_for<NB>();
+  int per = 0;
+  const cudaError_t e =
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, gemv_direct_kernel<NB, FP4, NW>, NW * 32, 0);
+  g_grid_direct[FP4][NB] = sms * (per > 0 ? per : 1);
+  return e;
+}
+
+template <int NB, bool FP4>
+void launch_direct(int grid, const MmaArgs& a, cudaStream_t st) {
+  constexpr int NW = warps_for<NB>();
+  gemv_direct_kernel<NB, FP4, NW><<<grid, NW * 32, 0, st>>>(a);
+}
+
 }  // namespace
 
 bool gemv_mma_supported(const Shape& sh) {
-  if (sh.wtype == FT_W_BF16) return sh.d % 64 == 0 && sh.d_ff % 64 == 0;
-  // NVFP4: a slice's block scales are a multiple of 16 bytes (bulk copies)
+  if (sh.wtype == FT_W_BF16) return sh.d % 32 == 0 && sh.d_ff % 32 == 0;
+  // NVFP4: a row's block scales are a multiple of 16 bytes (bulk copies)
   if (sh.wtype == FT_W_NVFP4) return sh.d % 256 == 0 && sh.d_ff % 256 == 0;
   return false;
 }
@@ -602,6 +948,10 @@ cudaError_t gemv_mma_init(int device) {
   if (e == cudaSuccess) e = kernel_setup<2, false>(sms);
   if (e == cudaSuccess) e = kernel_setup<1, true>(sms);
   if (e == cudaSuccess) e = kernel_setup<2, true>(sms);
+  if (e == cudaSuccess) e = direct_setup<1, false>(sms);
+  if (e == cudaSuccess) e = direct_setup<2, false>(sms);
+  if (e == cudaSuccess) e = direct_setup<1, true>(sms);
+  if (e == cudaSuccess) e = direct_setup<2, true>(sms);
   return e;
 }
 
@@ -639,10 +989,24 @@ void launch_gemv_mma(const Shape& sh, int cls, int layer, const void* x16, int T
   const bool fp4 = sh.wtype == FT_W_NVFP4;
   const int NB = T > 8 ? 2 : 1;
   const long long chunks = (long long)max_items + (long long)max_tok / CHUNK;
+  if (cls == KIND_HIT) {
+    const long long units = chunks * (sh.d_ff / 8 + sh.d / 16) / (fp4 ? tiles_for<true>() : 1);
+    const int cap = g_grid_direct[fp4][NB];
+    const int grid = (int)(units < cap ? units : cap);
+    if (grid <= 0) return;
+    if (fp4) {
+      if (NB == 1) launch_direct<1, true>(grid, a, st);
+      else launch_direct<2, true>(grid, a, st);
+    } else {
+      if (NB == 1) launch_direct<1, false>(grid, a, st);
+      else launch_direct<2, false>(grid, a, st);
+    }
+    return;
+  }
   const long long units = chunks * (sh.d_ff / 8 + sh.d / 16);
   // Streamed experts come over the host link, which a few CTAs' rings keep
-  // busy (16 CTAs x 4 stages of bulk reads in flight); the other SMs stay with
-  // the HBM work of the hit experts running meanwhile.
+  // busy (16 CTAs x 4 stages x 37 KB of bulk reads in flight); the other SMs
+  // stay with the HBM work of the hit experts running meanwhile.
   int cap = g_grid[fp4][NB];
   constexpr int stream_ctas = 16;
   if (cls == KIND_STREAMED && cap > stream_ctas) cap = stream_ctas;
