@@ -151,7 +151,8 @@ __device__ __forceinline__ void permute_body(const int32_t* __restrict__ ids, in
   int32_t* wcnt = smem;                // [32][E]
   int32_t* run = smem + 32 * E;        // [E] next free position per expert
   int32_t* tot = run + E;              // [E] per-chunk totals
-  int32_t* cnt = tot + E;              // [E]
+  int32_t* cnt = tot + E;              // [E] counts (kept after the call)
+  int32_t* off = cnt + E;              // [E] offsets (kept after the call)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int e = tid; e < E; e += 1024) cnt[e] = 0;
   __syncthreads();
@@ -178,6 +179,7 @@ __device__ __forceinline__ void permute_body(const int32_t* __restrict__ ids, in
       const int e = lane * PER + i;
       if (e < E) {
         run[e] = base;
+        off[e] = base;
         offsets[e] = base;
         counts[e] = local[i];
       }
@@ -422,7 +424,8 @@ __global__ void __launch_bounds__(1024) route_decode_kernel(const AT* __restrict
   __syncthreads();
   permute_body(ds.ids, T * k, E, ds.counts, ds.offsets, ds.perm, ds.inv, smem);
   __syncthreads();
-  lookup_detail::lookup_body(la, E, C, slot_bytes, ds);
+  // counts and offsets are still in this CTA's shared memory (permute_body)
+  lookup_detail::lookup_body(la, E, C, slot_bytes, ds, smem + 34 * E, smem + 35 * E);
   if (threadIdx.x == 0) *ds.route_ctr = 0;  // ready for the next call
 }
 
@@ -530,7 +533,7 @@ __global__ void __launch_bounds__(PCHUNK) perm_scatter_kernel(const int32_t* __r
   }
 }
 
-size_t permute_smem_bytes(int E) { return sizeof(int32_t) * (size_t)(32 * E + 3 * E); }
+size_t permute_smem_bytes(int E) { return sizeof(int32_t) * (size_t)(32 * E + 4 * E); }
 
 void launch_topk(const Shape& sh, const float* scores, int T, DevState& ds, cudaStream_t st) {
   const int warps_per_cta = 8;

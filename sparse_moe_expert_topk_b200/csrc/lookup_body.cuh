@@ -100,8 +100,13 @@ __device__ __forceinline__ unsigned long long slot_key(const unsigned long long*
   return st < epoch ? ((st << SLOT_BITS) | (unsigned long long)s) : NOKEY;
 }
 
+// s_counts / s_offsets: the routing counts and offsets when the calling CTA
+// already holds them in shared memory (else null: read from global memory).
 __device__ __forceinline__ void lookup_body(const LookupArgs& a, int E, long long C, size_t slot_bytes,
-                                            DevState& ds) {
+                                            DevState& ds, const int32_t* s_counts = nullptr,
+                                            const int32_t* s_offsets = nullptr) {
+  const int32_t* counts = s_counts ? s_counts : ds.counts;
+  const int32_t* offsets = s_offsets ? s_offsets : ds.offsets;
   __shared__ int s_e[MAX_E];
   __shared__ int s_slot[MAX_E];
   __shared__ int s_vic[MAX_E];
@@ -119,7 +124,7 @@ __device__ __forceinline__ void lookup_body(const LookupArgs& a, int E, long lon
   const int layer = a.layer;
 
   // 1. the batch: routed experts (counts > 0) or all E, ascending
-  const bool in = tid < E && (a.use_counts ? ds.counts[tid] > 0 : true);
+  const bool in = tid < E && (a.use_counts ? counts[tid] > 0 : true);
   int n_u;
   const int upos = block_scan_flag(in, scan, n_u);
   if (in) s_e[upos] = tid;
@@ -292,13 +297,13 @@ __device__ __forceinline__ void lookup_body(const LookupArgs& a, int E, long lon
   // tensor-core GEMV scheduling state of each class (ticket and one
   // completion counter per (item, 16-token chunk)) cleared
   if (a.build_work) {
-    const int tok = act ? ds.counts[e] : 0;
+    const int tok = act ? counts[e] : 0;
     const int r = block_scan3(act ? kind : -1, tok, (tok + MMA_CHUNK - 1) / MMA_CHUNK, scan3);
     if (act) {
       WorkItem it;
       it.e = e;
       it.slot = s_slot[tid];
-      it.tok_off = ds.offsets[e];
+      it.tok_off = offsets[e];
       it.n_tok = tok;
       ds.work->items[kind][r] = it;
     }
