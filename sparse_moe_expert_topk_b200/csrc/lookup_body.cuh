@@ -117,7 +117,7 @@ __device__ __forceinline__ void lookup_body(const LookupArgs& a, int E, long lon
   __shared__ unsigned long long s_prefix, s_mask;
   __shared__ int s_remaining, s_ncand, s_avail;
   __shared__ unsigned long long s_c0, s_epoch, s_bstart;
-  __shared__ int s_cbase, s_lbase, s_tok, s_chunks;
+  __shared__ int s_cbase, s_lbase;
 
   const int tid = threadIdx.x;
   Mailbox* mb = ds.mbox;
