@@ -125,13 +125,13 @@ size_t slot_bytes_of(const ft_config* c) {
 
 // Host wait for an event with a deadline; the compute stream keeps running.
 ft_status wait_event(cudaEvent_t ev, double seconds) {
+  if (fault("poll_timeout")) return FT_ETIMEOUT;  // injected: a wait that never completes
   const auto t0 = std::chrono::steady_clock::now();
   long spins = 0;
   for (;;) {
     const cudaError_t e = cudaEventQuery(ev);
     if (e == cudaSuccess) return FT_OK;
     if (e != cudaErrorNotReady) return FT_ECUDA;
-    if (fault("poll_timeout")) return FT_ETIMEOUT;
     if ((++spins & 1023) == 0) {
       const double dt = std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count();
       if (dt > seconds) return FT_ETIMEOUT;
