@@ -71,7 +71,7 @@ typedef enum {
   FT_ECUDA = 3,        /* a CUDA runtime call failed */
   FT_ETIMEOUT = 4,     /* a bounded wait (host or device) gave up */
   FT_ESTATE = 5,       /* call out of order (e.g. no router set) or latched device error */
-  FT_EUNSUPPORTED = 6  /* valid request this build does not implement */
+  FT_EUNSUPPORTED = 6  /* valid request this library does not implement */
 } ft_status;
 
 /* Expert weight format. F32 implies fp32 activations (x, y, W_r); BF16 and
