@@ -147,6 +147,23 @@ def test_nvfp4_multilayer_trace(cuda_ok):
         _check_cache_state(h, oc)
 
 
+def test_nvfp4_shape_off_the_tensor_core_path(cuda_ok):
+    """NVFP4 with d and d_ff multiples of 64 but not of 256 (d = 320,
+    d_ff = 192): the experts run on the SIMT GEMV instead of the tensor-core
+    one; same parity bar, decode at batch 1..5 on a small shared cache."""
+    wl = ftgen.Workload("nvfp4_odd", L=2, E=16, k=2, d=320, d_ff=192, wtype=ftgen.W_NVFP4, cache_slots=6,
+                        bp_mbps=52700, bh_mbps=77300)
+    with _harness(wl, max_tokens=5) as h:
+        oc = oracle_cache(h)
+        W = ExpertWeights(h, keep=32)
+        for step in range(6):
+            for l in range(wl.L):
+                T = 1 + (step + l) % 5
+                x = gap_hidden(wl, T, wl.seed("odd", step, l), h.routers[l], None)
+                _run_and_check(h, oc, W, l, x, None)
+        _check_cache_state(h, oc)
+
+
 def test_error_paths(cuda_ok):
     wl = ftgen.workload("tiny_f32")
     with _harness(wl, gen_device="cpu") as h:
