@@ -43,6 +43,11 @@ Readings taken where the pages are silent:
   slot, to the lowest free slots below C'; the clock is kept and the
   layer-ahead prefetch state is cleared.
 
+For the miss-rate comparison with engines that pin a fixed hot subset
+([techfeed] "セマンティック認識キャッシング" sets the shared LRU against such
+static placements), `static_hot_placement` gives the best static placement of
+C slots in hindsight and `static_placement_misses` its misses.
+
 Pins (tests/test_oracle_cache.py): q* against the table derived from the
 pages' two B_P:B_H profiles (tests/golden/qstar_profiles.txt) and the bound
 |q* - m B_P / B_H| <= 1/2; q* = 0 at B_P = 0 and q* = m at B_P >= B_H; with
@@ -63,6 +68,25 @@ def qstar(m: int, bp_mbps: int, bh_mbps: int) -> int:
         return 0
     q = (2 * m * bp_mbps + bh_mbps) // (2 * bh_mbps)
     return max(0, min(m, q))
+
+
+def static_hot_placement(key_counts: dict, C: int) -> set:
+    """The C keys with the most lookups, ties to the lower key: on a trace known
+    in advance, no static placement of C slots misses less (every lookup of a
+    pinned key hits, every other lookup misses, whatever the order)."""
+    order = sorted(key_counts, key=lambda k: (-key_counts[k], k))
+    return set(order[:max(C, 0)])
+
+
+def static_placement_misses(batches, hot: set):
+    """(lookups, misses) of a static placement over lookup batches (each an
+    iterable of unique keys): nothing is ever inserted or evicted."""
+    lookups = misses = 0
+    for batch in batches:
+        for key in batch:
+            lookups += 1
+            misses += key not in hot
+    return lookups, misses
 
 
 class ExpertCache:

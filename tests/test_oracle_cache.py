@@ -262,3 +262,42 @@ def test_prefill_after_resize_reloads_its_layer():
     rec = c.forward(1, PREFILL, full)
     assert [k for (l, _, k) in rec["lookups"] if l == 1] == [HIT] * E
     assert rec["n_cur"] == E
+
+
+def test_static_hot_placement_is_the_best_static_placement():
+    """Brute force over every placement of C slots on small random traces:
+    none misses less than the most-looked-up keys."""
+    import itertools
+    rng = np.random.default_rng(7)
+    for _ in range(6):
+        keys = 7
+        batches = [sorted(set(int(k) for k in rng.choice(keys, size=rng.integers(1, 4),
+                                                          p=np.arange(keys, 0, -1) / (keys * (keys + 1) / 2))))
+                   for _ in range(30)]
+        counts = {}
+        for b in batches:
+            for k in b:
+                counts[k] = counts.get(k, 0) + 1
+        for C in range(0, keys + 1):
+            hot = cache.static_hot_placement(counts, C)
+            assert len(hot) == min(C, len(counts))
+            _, m = cache.static_placement_misses(batches, hot)
+            best = min(cache.static_placement_misses(batches, set(S))[1]
+                       for S in itertools.combinations(range(keys), C))
+            assert m == best, (C, m, best)
+    # the extremes
+    lookups, m = cache.static_placement_misses(batches, set())
+    assert m == lookups
+    assert cache.static_placement_misses(batches, set(range(keys)))[1] == 0
+
+
+def test_policy_comparison_runs_on_a_short_trace():
+    """The LRU-against-static comparison script on 8 steps of the 43-layer
+    trace: rates in [0, 1], hindsight never worse than the profiled placement."""
+    from oracle import policy_compare
+    rows = policy_compare.run(steps=8, fracs=(0.37,))
+    (C, f, lru, lru_half, st_prior, st_best), = rows
+    assert C == int(0.37 * 43 * 256)
+    for r in (lru, lru_half, st_prior, st_best):
+        assert 0.0 <= r <= 1.0
+    assert st_best <= st_prior
