@@ -14,7 +14,10 @@ Modules
   formats  e2m1 / e4m3 decoding and slot-blob unpacking
   moe      router logits, top-k, softmax weights, permutation, SwiGLU expert,
            per-token layer forward
-  cache    q* split and the shared LRU expert cache (hit / staged / streamed)
+  cache    q* split and the shared LRU expert cache (hit / staged / streamed);
+           the best static placement, for the miss-rate comparison
+  policy_compare  the shared LRU against static placements on the 43-layer
+           trace (an analysis run of the oracle: python -m oracle.policy_compare)
 
 Parity pins (tests/test_oracle_*.py): every function above is pinned to
 something other than itself; see each module's docstring. Expert-value parity
