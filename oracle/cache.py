@@ -197,6 +197,25 @@ class ExpertCache:
         return dict(lookups=look, kinds={e: HIT for e in routed}, m=m, qstar=-1, qstage=qs,
                     n_cur=n_cur)
 
+    # --- predictive prefetch (a policy simulation) -------------------------
+    def prefetch(self, layer: int, experts, pinned_keys=()) -> int:
+        """Stage the non-resident `experts` of `layer` ahead of its lookup, in
+        ascending e, each with a fresh stamp (as staged inserts); the keys in
+        `pinned_keys` (the layer computing meanwhile) are not evicted. Returns
+        the number of blobs copied; only the `prefetched` counter changes."""
+        pinned = {self.slot_of[k] for k in pinned_keys if k in self.slot_of}
+        n = 0
+        for e in sorted(set(int(x) for x in experts)):
+            key = layer * self.E + e
+            if key in self.slot_of:
+                continue
+            if len(pinned) >= self.C:
+                break
+            self._insert(key, pinned)
+            n += 1
+        self.n["prefetched"] = self.n.get("prefetched", 0) + n
+        return n
+
     # --- elastic capacity -------------------------------------------------
     def resize(self, C_new: int):
         """Change the capacity to C_new slots at a safe point (between calls)."""

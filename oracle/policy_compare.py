@@ -59,15 +59,38 @@ def run(steps: int = 512, fracs=(0.10, 0.20, 0.37, 0.60), profile=(52700, 77300)
             prior |= {l * E + int(e) for e in ranks[l][:take]}
         _, m_prior = cache.static_placement_misses(batches, prior)
         look, m_best = cache.static_placement_misses(batches, cache.static_hot_placement(counts, C))
-        rows.append((C, f, lru, lru_half, m_prior / look, m_best / look))
+        # the same LRU with a predictive prefetch: while layer l computes,
+        # layer l+1's experts of the previous step are staged (the reuse of
+        # the Markov trace); cost: every prefetched blob crosses the link
+        cp = cache.ExpertCache(L, E, C, *profile)
+        prev = [None] * L
+        for st in range(steps):
+            for l in range(L):
+                if prev[l] is not None:
+                    cur_prev = [(l - 1) * E + int(e) for e in prev[l - 1]] if l > 0 and prev[l - 1] is not None else []
+                    cp.prefetch(l, prev[l], cur_prev)
+                cnt = np.zeros(E, int)
+                cnt[traces[l][st][0]] = 1
+                cp.forward(l, cache.DECODE, cnt)
+                prev[l] = traces[l][st][0]
+        pf_miss = cp.n["misses"] / cp.n["lookups"]
+        link_lru = c.n["misses"] / steps          # blobs over the link per step (staged + streamed)
+        link_pf = (cp.n["misses"] + cp.n.get("prefetched", 0)) / steps
+        rows.append((C, f, lru, lru_half, m_prior / look, m_best / look, pf_miss, link_lru, link_pf))
     return rows
 
 
 if __name__ == "__main__":
     steps = int(sys.argv[1]) if len(sys.argv) > 1 else 512
+    rows = run(steps)
     print(f"43-layer NVFP4 trace, {steps} steps at batch 1, B_P:B_H = 52.7:77.3; static placements pre-loaded")
     print("| slots | capacity | shared LRU (cold start) | shared LRU, second half | static, profiled | static, best in hindsight |")
     print("|---|---|---|---|---|---|")
-    for C, f, lru, lru_half, st_prior, st_best in run(steps):
+    for C, f, lru, lru_half, st_prior, st_best, *_ in rows:
         print(f"| {C} | {100 * f:.0f}% | {100 * lru:.1f}% | {100 * lru_half:.1f}% | {100 * st_prior:.1f}% | "
               f"{100 * st_best:.1f}% |")
+    print()
+    print("| slots | capacity | LRU miss rate | LRU + prefetch miss rate | link blobs per step, LRU | with prefetch |")
+    print("|---|---|---|---|---|---|")
+    for C, f, lru, _, _, _, pf, link_lru, link_pf in rows:
+        print(f"| {C} | {100 * f:.0f}% | {100 * lru:.1f}% | {100 * pf:.1f}% | {link_lru:.1f} | {link_pf:.1f} |")

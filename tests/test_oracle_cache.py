@@ -296,8 +296,9 @@ def test_policy_comparison_runs_on_a_short_trace():
     trace: rates in [0, 1], hindsight never worse than the profiled placement."""
     from oracle import policy_compare
     rows = policy_compare.run(steps=8, fracs=(0.37,))
-    (C, f, lru, lru_half, st_prior, st_best), = rows
+    (C, f, lru, lru_half, st_prior, st_best, pf, link_lru, link_pf), = rows
     assert C == int(0.37 * 43 * 256)
     for r in (lru, lru_half, st_prior, st_best):
         assert 0.0 <= r <= 1.0
     assert st_best <= st_prior
+    assert 0.0 <= pf <= 1.0 and link_lru > 0 and link_pf > 0
