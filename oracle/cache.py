@@ -48,13 +48,18 @@ For the miss-rate comparison with engines that pin a fixed hot subset
 static placements), `static_hot_placement` gives the best static placement of
 C slots in hindsight and `static_placement_misses` its misses.
 
+A predictive prefetch (`ExpertCache.prefetch`, a policy simulation of the
+next layer staged during the current one) inserts like a staged miss.
+
 Pins (tests/test_oracle_cache.py): q* against the table derived from the
 pages' two B_P:B_H profiles (tests/golden/qstar_profiles.txt) and the bound
 |q* - m B_P / B_H| <= 1/2; q* = 0 at B_P = 0 and q* = m at B_P >= B_H; with
 one access per step and B_P = B_H the hit/miss sequence equals a textbook
 move-to-front LRU list; misses are never fewer than Belady's optimal policy;
 C >= L*E gives only compulsory misses; C = 0 makes every lookup a streamed
-miss.
+miss; a resize equals a move-to-front list truncated at each shrink; a
+prefetch equals an insert at the most-recent end of that list; the best static
+placement equals the brute-force minimum over all placements.
 """
 from __future__ import annotations
 

@@ -302,3 +302,50 @@ def test_policy_comparison_runs_on_a_short_trace():
         assert 0.0 <= r <= 1.0
     assert st_best <= st_prior
     assert 0.0 <= pf <= 1.0 and link_lru > 0 and link_pf > 0
+
+
+@pytest.mark.parametrize("C", [1, 3, 6])
+def test_prefetch_matches_a_textbook_lru_list(C):
+    """Accesses mixed with prefetches, one key per call, q* = m: a prefetch
+    inserts a non-resident key at the most-recent end (evicting the least
+    recent) and leaves a resident key where it is; the hit/miss sequence and
+    the contents match a move-to-front list doing the same."""
+    L, E = 2, 6
+    rng = np.random.default_rng(100 + C)
+    c = cache.ExpertCache(L, E, C, 1, 1)
+    lru = OrderedDict()
+    for _ in range(400):
+        key = int(rng.integers(0, L * E))
+        layer, e = divmod(key, E)
+        if rng.random() < 0.4:
+            n = c.prefetch(layer, [e])
+            if key in lru:
+                assert n == 0
+            else:
+                assert n == 1
+                if len(lru) >= C:
+                    lru.popitem(last=False)
+                lru[key] = True
+            continue
+        counts = np.zeros(E, int); counts[e] = 1
+        kind = c.forward(layer, DECODE, counts)["kinds"][e]
+        if key in lru:
+            lru.move_to_end(key)
+            assert kind == HIT
+        else:
+            assert kind == STAGED
+            if len(lru) >= C:
+                lru.popitem(last=False)
+            lru[key] = True
+        assert sorted(k for k in c.contents()[0] if k >= 0) == sorted(lru)
+
+
+def test_prefetch_keeps_pinned_keys():
+    c = cache.ExpertCache(2, 4, 3, 1, 1)
+    c.forward(0, DECODE, np.array([1, 1, 1, 0]))          # layer 0 experts 0..2 fill the cache
+    before = set(k for k in c.contents()[0] if k >= 0)
+    assert c.prefetch(1, [0, 1], pinned_keys=[0, 1, 2]) == 0  # everything pinned: nothing moves
+    assert set(k for k in c.contents()[0] if k >= 0) == before
+    assert c.prefetch(1, [0], pinned_keys=[0, 1]) == 1        # evicts the one unpinned key, 2
+    assert set(k for k in c.contents()[0] if k >= 0) == {0, 1, 4}
+    assert c.n["prefetched"] == 1 and c.n["misses"] == 3 and c.n["lookups"] == 3
