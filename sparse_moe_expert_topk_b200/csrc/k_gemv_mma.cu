@@ -1,20 +1,28 @@
 // Decode grouped GEMV for BF16 and NVFP4 experts on warp-level tensor-core
 // MMAs (mma.sync m16n8k16, fp32 accumulate): gate/up + SwiGLU and down in one
-// persistent launch per work class, weights streamed with 128-bit loads from
-// HBM slots or straight from the mapped host pool.
+// persistent launch per work class, weights read from HBM slots or straight
+// from the mapped host pool.
 //
 // Small-batch decode is memory bound ([paperlens] "壁2: デコードのミスを「どう捌く
 // か」が決まっていない", paper §2.2): every weight byte is read once, so the
 // kernel keeps many loads in flight and spends few instructions per byte.
 //
-// Work unit: 16 weight rows x one chunk of <= 16 tokens of one expert. One
-// producer warp takes the units by atomic ticket and has the TMA engine copy
-// their weight rows (K slices of <= 2 KB per row, cp.async.bulk) into a
-// 4-stage shared-memory ring; eight MMA warps split each slice's K range
-// (split-K), accumulate over the unit's slices and reduce their partial sums in
-// warp order through shared memory. The ring decouples the bytes in flight
-// from registers, and every host read of a streamed expert is a large
-// contiguous request instead of scattered 64-byte fragments.
+// Work unit: 16 weight rows x one chunk of <= 16 tokens of one expert, taken
+// by atomic ticket; the K range of the unit is split over eight MMA warps
+// (split-K), whose partial sums are reduced in warp order through shared
+// memory. Two kernels share this arithmetic exactly:
+//   * gemv_fused_kernel (staged and streamed experts): a producer warp has the
+//     TMA engine copy the unit's weight rows (K slices of <= 2 KB per row,
+//     cp.async.bulk) into a 4-stage shared-memory ring that the MMA warps
+//     consume. The ring decouples the bytes in flight from registers, a
+//     streamed expert's host reads become large contiguous requests, and a
+//     staged expert is consumed blob by blob as the copy engine lands it.
+//   * gemv_direct_kernel (experts hit in HBM slots): the MMA warps load their
+//     fragments straight into registers, several steps in flight and several
+//     CTAs per SM, which hides HBM latency better than the ring here.
+// Both split K identically (for each ring slice in order, warp w takes the
+// same sub-range of its steps), so an expert's result is bit-identical
+// whichever kernel computes it.
 //
 // Inside a warp, lane (g, q) = (lane/4, lane%4) reads 16 consecutive bytes of
 // rows g and g+8 per step and hands them to the MMA unchanged as its A
