@@ -76,3 +76,32 @@ def test_init_without_gpu_fails_cleanly(lib):
     with pytest.raises(ft.FtError) as ei:
         ft.ft_moe_init(cfg, None, 1)
     assert ei.value.status == ft.FT_ECUDA
+
+
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    """The boundary is a C ABI: a C99 translation unit that includes the header
+    and takes the address of every declared entry point compiles with warnings
+    as errors and links against the library (no C++ in any signature)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    names = _declared()
+    src = tmp_path / "use_abi.c"
+    src.write_text('#include "ft_moe.h"\n#include <stdio.h>\n'
+                   "typedef void (*fn_t)(void);\n"
+                   "int main(void) {\n  const fn_t fns[] = {\n"
+                   + "".join(f"    (fn_t)&{n},\n" for n in names)
+                   + "  };\n  printf(\"%d %s\\n\", (int)(sizeof fns / sizeof fns[0]), ft_status_str(FT_EINVAL));\n"
+                   "  return 0;\n}\n")
+    lib_dir = os.path.join(ROOT, "sparse_moe_expert_topk_b200")
+    exe = tmp_path / "use_abi"
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                        str(src), "-o", str(exe), "-L", lib_dir, "-lft_moe", f"-Wl,-rpath,{lib_dir}"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, out.stderr
+    n, msg = out.stdout.strip().split(" ", 1)
+    assert int(n) == len(names) and msg == "invalid argument"
