@@ -37,6 +37,12 @@ Readings taken where the pages are silent:
   did not already prefetch it, then prefetches layer l+1 (if l+1 < L), all E
   experts each, no q*; with C < 2E a prefill call follows the decode rules
   for its routed experts; a call with T = 0 changes nothing;
+* optional predictive prefetch: right after the decode lookup of layer l,
+  the experts that layer (l+1) mod L was routed to in its last decode call and
+  that are not resident are staged, ascending e, as staged inserts (fresh
+  stamps), never evicting what layer l's lookup touched or inserted; resident
+  ones are left untouched; only decode calls record their routing and
+  prefetch; a resize clears the record;
 * a resize to C' slots between layer calls keeps the min(C', resident)
   most recently stamped entries with their stamps; a survivor whose slot is
   below C' stays there, the others move, in ascending order of their old
@@ -105,7 +111,11 @@ class ExpertCache:
         self.slot_of = {}        # key -> slot
         self.clock = 0
         self.prefetched = -1     # layer whose experts the last prefill call loaded ahead
-        self.n = dict(lookups=0, hits=0, misses=0, staged=0, streamed=0, layer_calls=0)
+        self.n = dict(lookups=0, hits=0, misses=0, staged=0, streamed=0, layer_calls=0, prefetched=0)
+        # predictive prefetch (opt-in): after the decode lookup of layer l,
+        # stage the experts layer (l+1) mod L was routed to in its last decode call
+        self.prefetch_on = False
+        self.last_routed = {}    # layer -> experts of its last decode call
 
     # --- primitives -------------------------------------------------------
     def _touch(self, slot: int):
@@ -181,8 +191,14 @@ class ExpertCache:
         self.n["layer_calls"] += 1
         routed = [e for e in range(E) if counts[e] > 0]
         if mode == DECODE or self.C < 2 * E:
-            kinds, m, q, qs = self._batch(layer, routed, set(), True)
+            pinned = set()
+            kinds, m, q, qs = self._batch(layer, routed, pinned, True)
             self.prefetched = -1
+            if mode == DECODE:
+                nxt = (layer + 1) % self.L
+                if self.prefetch_on and nxt in self.last_routed:
+                    self._prefetch(nxt, self.last_routed[nxt], pinned)
+                self.last_routed[layer] = routed
             look = [(layer, e, kinds[e]) for e in routed]
             return dict(lookups=look, kinds=kinds, m=m, qstar=q, qstage=qs, n_cur=len(look))
         look = []
@@ -208,7 +224,10 @@ class ExpertCache:
         ascending e, each with a fresh stamp (as staged inserts); the keys in
         `pinned_keys` (the layer computing meanwhile) are not evicted. Returns
         the number of blobs copied; only the `prefetched` counter changes."""
-        pinned = {self.slot_of[k] for k in pinned_keys if k in self.slot_of}
+        return self._prefetch(layer, experts, {self.slot_of[k] for k in pinned_keys if k in self.slot_of})
+
+    def _prefetch(self, layer: int, experts, pinned: set) -> int:
+        """prefetch() with the pinned slots given; `pinned` grows by the inserts."""
         n = 0
         for e in sorted(set(int(x) for x in experts)):
             key = layer * self.E + e
@@ -218,7 +237,7 @@ class ExpertCache:
                 break
             self._insert(key, pinned)
             n += 1
-        self.n["prefetched"] = self.n.get("prefetched", 0) + n
+        self.n["prefetched"] += n
         return n
 
     # --- elastic capacity -------------------------------------------------
@@ -241,6 +260,7 @@ class ExpertCache:
         self.key_of, self.stamp = key_of, stamp
         self.slot_of = {k: s for s, k in enumerate(key_of) if k >= 0}
         self.prefetched = -1
+        self.last_routed = {}
 
     def contents(self):
         """(key_of [C], stamp [C]) as lists."""

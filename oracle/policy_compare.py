@@ -59,23 +59,19 @@ def run(steps: int = 512, fracs=(0.10, 0.20, 0.37, 0.60), profile=(52700, 77300)
             prior |= {l * E + int(e) for e in ranks[l][:take]}
         _, m_prior = cache.static_placement_misses(batches, prior)
         look, m_best = cache.static_placement_misses(batches, cache.static_hot_placement(counts, C))
-        # the same LRU with a predictive prefetch: while layer l computes,
-        # layer l+1's experts of the previous step are staged (the reuse of
-        # the Markov trace); cost: every prefetched blob crosses the link
+        # the same LRU with the predictive prefetch: after layer l's lookup,
+        # layer l+1's experts of its last call are staged (the reuse of the
+        # Markov trace); cost: every prefetched blob crosses the link
         cp = cache.ExpertCache(L, E, C, *profile)
-        prev = [None] * L
+        cp.prefetch_on = True
         for st in range(steps):
             for l in range(L):
-                if prev[l] is not None:
-                    cur_prev = [(l - 1) * E + int(e) for e in prev[l - 1]] if l > 0 and prev[l - 1] is not None else []
-                    cp.prefetch(l, prev[l], cur_prev)
                 cnt = np.zeros(E, int)
                 cnt[traces[l][st][0]] = 1
                 cp.forward(l, cache.DECODE, cnt)
-                prev[l] = traces[l][st][0]
         pf_miss = cp.n["misses"] / cp.n["lookups"]
         link_lru = c.n["misses"] / steps          # blobs over the link per step (staged + streamed)
-        link_pf = (cp.n["misses"] + cp.n.get("prefetched", 0)) / steps
+        link_pf = (cp.n["misses"] + cp.n["prefetched"]) / steps
         rows.append((C, f, lru, lru_half, m_prior / look, m_best / look, pf_miss, link_lru, link_pf))
     return rows
 

@@ -349,3 +349,48 @@ def test_prefetch_keeps_pinned_keys():
     assert c.prefetch(1, [0], pinned_keys=[0, 1]) == 1        # evicts the one unpinned key, 2
     assert set(k for k in c.contents()[0] if k >= 0) == {0, 1, 4}
     assert c.n["prefetched"] == 1 and c.n["misses"] == 3 and c.n["lookups"] == 3
+
+
+@pytest.mark.parametrize("C,L", [(1, 3), (2, 3), (2, 4), (4, 3), (3, 1)])
+def test_prefetch_mode_matches_a_textbook_lru_list(C, L):
+    """One key per call, q* = m, prefetch on: after the access of (l, e) the
+    key layer (l+1) mod L accessed last is inserted at the most-recent end if
+    absent, evicting the least recent key other than the one just accessed
+    (nothing if there is none); contents and hit/miss sequence match."""
+    E = 4
+    rng = np.random.default_rng(300 + 10 * C + L)
+    c = cache.ExpertCache(L, E, C, 1, 1)
+    c.prefetch_on = True
+    lru = OrderedDict()
+    last = {}
+    for step in range(150):
+        for layer in range(L):
+            e = int(rng.integers(0, E))
+            key = layer * E + e
+            counts = np.zeros(E, int); counts[e] = 1
+            kind = c.forward(layer, DECODE, counts)["kinds"][e]
+            if key in lru:
+                lru.move_to_end(key)
+                assert kind == HIT
+            else:
+                assert kind == STAGED
+                if len(lru) >= C:
+                    lru.popitem(last=False)
+                lru[key] = True
+            nxt = (layer + 1) % L
+            if nxt in last and last[nxt] not in lru:
+                if len(lru) < C:
+                    lru[last[nxt]] = True
+                else:
+                    victims = [k for k in lru if k != key]
+                    if victims:
+                        del lru[victims[0]]
+                        lru[last[nxt]] = True
+            last[layer] = key
+            assert sorted(k for k in c.contents()[0] if k >= 0) == sorted(lru), (step, layer)
+    # with one key per call the next layer's last key was used within the last
+    # L calls: it can only have been evicted (and need a prefetch) when C < L
+    if 1 < C < L:
+        assert c.n["prefetched"] > 0
+    else:
+        assert c.n["prefetched"] == 0
