@@ -411,6 +411,8 @@ def run_secondary(args, wl, world, rank, local):
             wl = dataclasses.replace(wl, L=L, cache_slots=int(0.37 * L * wl.E))
         steps = min(wl.steps, int(os.environ.get("FT_TRACE_STEPS", wl.steps)))
         h = Harness(wl, max_tokens=1, device=local)
+        prefetch = os.environ.get("FT_PREFETCH", "0") == "1"  # the decode prefetch (opt-in)
+        ft.ft_moe_set_prefetch(h.ctx, prefetch)
         traces = [ftgen.markov_trace(steps, 1, wl.E, wl.k, wl.extra["p_reuse"], wl.extra["zipf_s"],
                                      wl.seed("trace", rank, l)) for l in range(L)]
         zb = [ftgen.zipf_log_bias(wl.E, wl.extra["zipf_s"], wl.seed("pi", l)) for l in range(L)]
@@ -437,11 +439,12 @@ def run_secondary(args, wl, world, rank, local):
         h.close()
         out.update(value=round(steps / (ms / 1e3), 2), ms_per_step=round(ms / steps, 4), dtype="nvfp4",
                    config={"workload": f"{L}-layer NVFP4 decode trace, batch 1, {steps} steps, Markov p=0.8 + "
-                                       f"Zipf(1.1), shared LRU at 37% ({wl.cache_slots} slots), 52.7:77.3"},
+                                       f"Zipf(1.1), shared LRU at 37% ({wl.cache_slots} slots), 52.7:77.3"
+                                       + (", decode prefetch on" if prefetch else "")},
                    tokens_per_s_all_layers=round(steps / (ms / 1e3), 2),
                    layer_calls_per_s=round(steps * L / (ms / 1e3), 1),
                    miss_rate=round(stt["misses"] / max(stt["lookups"], 1), 4),
-                   cache={k: stt[k] for k in ("lookups", "hits", "misses", "staged", "streamed")},
+                   cache={k: stt[k] for k in ("lookups", "hits", "misses", "staged", "streamed", "prefetched")},
                    host_link={"h2d_copy_gbs": round(h2d, 2), "zero_copy_read_gbs": round(zc, 2)},
                    roofline=roof, kernels=rows)
     if rank == 0:

@@ -177,6 +177,7 @@ typedef struct {
   int32_t last_qstage;      /* misses actually staged in that batch */
   int32_t device_error;     /* 0, or the latched ft_status of a device failure */
   uint64_t kernel_launches; /* CUDA kernels this context launched */
+  uint64_t prefetched;      /* blobs staged by the decode prefetch (ft_moe_set_prefetch) */
 } ft_stats;
 ft_status ft_cache_stats(ft_ctx* ctx, ft_stats* out);
 
@@ -188,6 +189,23 @@ ft_status ft_set_bandwidths(ft_ctx* ctx, uint32_t bp_mbps, uint32_t bh_mbps);
 
 /* Empty the cache and zero the counters (cold start). Synchronises. */
 ft_status ft_moe_reset_cache(ft_ctx* ctx);
+
+/* Predictive prefetch for decode, off by default. When on, every decode call
+ * of layer l, right after its lookup, stages into slots the experts that layer
+ * (l+1) mod L was routed to in its own last decode call and that are not
+ * resident: ascending expert id, each inserted like a staged miss (a fresh LRU
+ * stamp), evicting nothing that layer l's lookup touched or inserted, and as
+ * many as unpinned slots allow; resident ones are left untouched. The copies
+ * go out on the copy stream behind layer l's staged copies, so they overlap
+ * layer l's compute; the next call's experts read from those slots wait for
+ * them. Lookup counters are unchanged (the next layer's lookup then sees hits);
+ * ft_stats.prefetched counts the blobs. Only decode calls record their routing
+ * and prefetch; ft_moe_reset_cache and ft_moe_resize_cache clear the record.
+ * This extends the layer-ahead loading of prefill ([paperlens] プレフィル:
+ * 全層ダブルバッファと「意味の錨」, paper §3.1) to decode, predicting the next
+ * layer from its previous step; the pages give no decode prefetch policy.
+ * enable: 0 off, non-zero on. Errors: FT_EINVAL (NULL ctx). */
+ft_status ft_moe_set_prefetch(ft_ctx* ctx, int32_t enable);
 
 /* Grow or shrink the HBM slot pool to new_slots at a safe point, without
  * touching the host pool: the elastic memory manager of [techfeed]

@@ -27,7 +27,7 @@ KIND_HIT, KIND_STAGED, KIND_STREAMED = 0, 1, 2
 EXPORTS = (
     "ft_moe_slot_bytes", "ft_moe_init", "ft_moe_destroy", "ft_moe_expert_ptr", "ft_moe_set_tensor_scales",
     "ft_moe_set_router", "ft_moe_layer_forward", "ft_cache_stats", "ft_set_bandwidths", "ft_moe_reset_cache",
-    "ft_moe_resize_cache", "ft_moe_last_route", "ft_moe_cache_contents", "ft_moe_probe_link", "ft_moe_profile", "ft_moe_profile_read",
+    "ft_moe_resize_cache", "ft_moe_set_prefetch", "ft_moe_last_route", "ft_moe_cache_contents", "ft_moe_probe_link", "ft_moe_profile", "ft_moe_profile_read",
     "ft_route_topk_static", "ft_status_str",
 )
 FT_ROUTE_STATIC_MAX_TOKENS = 1024
@@ -44,7 +44,7 @@ class FtStats(ctypes.Structure):
                 ("misses", ctypes.c_uint64), ("staged", ctypes.c_uint64), ("streamed", ctypes.c_uint64),
                 ("bytes_h2d", ctypes.c_uint64), ("bytes_zero_copy", ctypes.c_uint64),
                 ("last_m", ctypes.c_int32), ("last_qstar", ctypes.c_int32), ("last_qstage", ctypes.c_int32),
-                ("device_error", ctypes.c_int32), ("kernel_launches", ctypes.c_uint64)]
+                ("device_error", ctypes.c_int32), ("kernel_launches", ctypes.c_uint64), ("prefetched", ctypes.c_uint64)]
 
     def as_dict(self):
         return {k: getattr(self, k) for k, _ in self._fields_}
@@ -84,6 +84,7 @@ def lib() -> ctypes.CDLL:
             "ft_set_bandwidths": [P, U32, U32],
             "ft_moe_reset_cache": [P],
             "ft_moe_resize_cache": [P, ctypes.c_int64],
+            "ft_moe_set_prefetch": [P, I32],
             "ft_moe_last_route": [P] + [P] * 11,
             "ft_moe_cache_contents": [P, P, P],
             "ft_moe_probe_link": [P, U64, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)],
@@ -183,6 +184,10 @@ def ft_moe_reset_cache(ctx):
 
 def ft_moe_resize_cache(ctx, new_slots):
     _check("ft_moe_resize_cache", lib().ft_moe_resize_cache(ctx, int(new_slots)))
+
+
+def ft_moe_set_prefetch(ctx, enable):
+    _check("ft_moe_set_prefetch", lib().ft_moe_set_prefetch(ctx, 1 if enable else 0))
 
 
 def ft_moe_last_route(ctx, E, Tk):

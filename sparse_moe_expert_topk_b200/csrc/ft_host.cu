@@ -67,6 +67,12 @@ struct ft_ctx {
   // stream memory operation that marks a staged blob as landed (null: not available)
   CUresult (*write_value)(CUstream, CUdeviceptr, cuuint32_t, unsigned int) = nullptr;
   uint32_t epoch = 0;
+  // decode prefetch (opt-in): after layer l's lookup, stage the experts layer
+  // (l+1) mod L was routed to in its last decode call
+  bool prefetch_on = false;
+  std::vector<char> has_prev;           // per layer: prev_counts holds its last decode routing
+  bool pf_pending = false;              // prefetch copies in flight; readers wait on ev_pfd
+  cudaEvent_t ev_pfd = nullptr;
   // launch accounting and optional per-launch CUDA-event profiling
   unsigned long long kernel_launches = 0;
   bool profiling = false;
@@ -148,14 +154,14 @@ void free_all(ft_ctx* c) {
   DevState& d = c->ds;
   void* dev_ptrs[] = {d.slot_of, d.key_of, d.stamp, d.clk, d.ctr, d.error, d.work, d.scores, d.ids, d.wts,
                       d.counts, d.offsets, d.perm, d.inv, d.perm_chunks, d.hbuf, d.ybuf, d.xs, d.hs, d.tscale, d.slots,
-                      d.h16, d.h16lo, d.x16, d.sched, d.route_ctr, d.landed, c->probe_sink};
+                      d.h16, d.h16lo, d.x16, d.sched, d.route_ctr, d.landed, d.prev_counts, c->probe_sink};
   for (void* p : dev_ptrs)
     if (p) cudaFree(p);
   for (uint8_t* p : c->pool_host)
     if (p) cudaFreeHost(p);
   prefill_tc_free(d);
   if (c->mbox_host) cudaFreeHost(c->mbox_host);
-  cudaEvent_t evs[] = {c->ev_look, c->ev_side, c->ev_copy, c->ev_pf[0], c->ev_pf[1], c->ev_t0, c->ev_t1};
+  cudaEvent_t evs[] = {c->ev_look, c->ev_side, c->ev_copy, c->ev_pf[0], c->ev_pf[1], c->ev_t0, c->ev_t1, c->ev_pfd};
   for (cudaEvent_t e : evs)
     if (e) cudaEventDestroy(e);
   for (auto& r : c->pend) {
@@ -181,6 +187,8 @@ ft_status reset_state(ft_ctx* c) {
   CK(cudaStreamSynchronize(c->s_comp));
   memset(c->mbox_host, 0, sizeof(Mailbox));
   c->prefetched = -1;
+  c->has_prev.assign(sh.L, 0);
+  c->pf_pending = false;
   c->latched = FT_OK;
   c->last_m = c->last_qstar = c->last_qstage = 0;
   c->layer_calls = 0;
@@ -198,13 +206,13 @@ ft_status check_device_error(ft_ctx* c) {
 enum ProfName {
   P_ROUTER, P_TOPK, P_PERMUTE, P_LOOKUP, P_GU_HIT, P_DN_HIT, P_GU_STAGED, P_DN_STAGED, P_GU_STREAM, P_DN_STREAM,
   P_COMBINE, P_STAGE_COPY, P_PREFILL_WORK, P_GATHER, P_GEMM_GU, P_GEMM_DN, P_GEMV_HIT, P_GEMV_STAGED,
-  P_GEMV_STREAM, P_TO_F16, P_ROUTE_FUSED, P_COUNT
+  P_GEMV_STREAM, P_TO_F16, P_ROUTE_FUSED, P_PF_COPY, P_COUNT
 };
 const char* const kProfNames[P_COUNT] = {
     "router_scores", "topk_softmax", "permute", "lookup", "gemv_gateup_hit", "gemv_down_hit",
     "gemv_gateup_staged", "gemv_down_staged", "gemv_gateup_streamed", "gemv_down_streamed", "combine",
     "h2d_stage_copies", "prefill_work", "prefill_gather", "gemm_tc_gateup", "gemm_tc_down", "gemv_hit",
-    "gemv_staged", "gemv_streamed", "to_f16", "route_decode_fused"};
+    "gemv_staged", "gemv_streamed", "to_f16", "route_decode_fused", "h2d_prefetch_copies"};
 
 cudaEvent_t pooled_event(ft_ctx* c) {
   if (!c->evpool.empty()) {
@@ -369,6 +377,7 @@ ft_status ft_moe_init(const ft_config* cfg, void* compute_stream, void* copy_str
   TRY(cuda_try(cudaMemset(d.sched, 0, sizeof(int32_t) * (N_CLASSES + (size_t)N_CLASSES * d.sched_chunks))));
   TRY(cuda_try(cudaMalloc((void**)&d.route_ctr, sizeof(int32_t))));
   TRY(cuda_try(cudaMemset(d.route_ctr, 0, sizeof(int32_t))));
+  TRY(cuda_try(cudaMalloc((void**)&d.prev_counts, sizeof(int32_t) * (size_t)sh.L * sh.E)));
   TRY(cuda_try(cudaMalloc((void**)&d.landed, sizeof(uint32_t) * MAX_E)));
   TRY(cuda_try(cudaMemset(d.landed, 0, sizeof(uint32_t) * MAX_E)));
   d.landed_epoch = 0;
@@ -401,6 +410,7 @@ ft_status ft_moe_init(const ft_config* cfg, void* compute_stream, void* copy_str
   TRY(cuda_try(cudaEventCreateWithFlags(&c->ev_copy, cudaEventDisableTiming)));
   TRY(cuda_try(cudaEventCreateWithFlags(&c->ev_pf[0], cudaEventDisableTiming)));
   TRY(cuda_try(cudaEventCreateWithFlags(&c->ev_pf[1], cudaEventDisableTiming)));
+  TRY(cuda_try(cudaEventCreateWithFlags(&c->ev_pfd, cudaEventDisableTiming)));
   TRY(cuda_try(cudaEventCreate(&c->ev_t0)));
   TRY(cuda_try(cudaEventCreate(&c->ev_t1)));
   TRY(cuda_try(route_kernels_init(sh.E)));
@@ -572,17 +582,44 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
       prof_end(c, p, cs);
       c->kernel_launches += 1;
     }
+    if (mode == FT_DECODE) {
+      // predictive prefetch: right behind this lookup, a batch for the next
+      // layer from its last decode routing (pins this batch's slots), then
+      // this call's routing becomes this layer's record
+      const int nxt = (layer + 1) % sh.L;
+      if (c->prefetch_on && c->has_prev[nxt]) {
+        LookupArgs pa{};
+        pa.layer = nxt;
+        pa.use_counts = 1;
+        pa.pin_prev = 1;
+        pa.append = 1;
+        pa.prefetch = 1;
+        pa.counts_src = d.prev_counts + (size_t)nxt * sh.E;
+        p = prof_begin(c, P_LOOKUP, cs, sh.C * 8.0 + sh.E * 16.0);
+        launch_lookup(sh, pa, d, cs);
+        prof_end(c, p, cs);
+        c->kernel_launches += 1;
+      }
+      CK(cudaMemcpyAsync(d.prev_counts + (size_t)layer * sh.E, d.counts, sizeof(int32_t) * sh.E,
+                         cudaMemcpyDeviceToDevice, cs));
+      c->has_prev[layer] = 1;
+    }
     CK(cudaEventRecord(c->ev_look, cs));
     CK(cudaStreamWaitEvent(c->s_side, c->ev_look, 0));
     int pr_stream[2], pr_hit[2], pr_staged[2];
     gemv_class(c, KIND_STREAMED, layer, x, T, max_items, Tk, c->s_side, pr_stream);
     CK(cudaEventRecord(c->ev_side, c->s_side));
+    if (c->pf_pending) {  // slots the last call prefetched may be this call's hits
+      CK(cudaStreamWaitEvent(cs, c->ev_pfd, 0));
+      c->pf_pending = false;
+    }
     gemv_class(c, KIND_HIT, layer, x, T, max_items, Tk, cs, pr_hit);
     st = wait_event(c->ev_look, WAIT_S);
     if (st != FT_OK) return c->latched = st;
     if (check_device_error(c) != FT_OK) return c->latched;
     const Mailbox* mb = c->mbox_host;
-    const int n_copy = mb->n_copy;
+    const int n_copy = mb->qstage;       // this layer's staged blobs come first in the copy list
+    const int n_copy_all = mb->n_copy;   // then the prefetched ones
     c->last_m = mb->m;
     c->last_qstar = mb->qstar;
     c->last_qstage = mb->qstage;
@@ -605,6 +642,14 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
       gemv_class(c, KIND_STAGED, layer, x, T, max_items, Tk, cs, pr_staged);
       d.landed_epoch = 0;
       gemv_class_cost(c, pr_staged, mb->n_staged_cls, mb->n_tok_cls[KIND_STAGED]);
+    }
+    if (n_copy_all > n_copy) {
+      p = prof_begin(c, P_PF_COPY, c->s_copy, (n_copy_all - n_copy) * (double)sh.slot_bytes);
+      st = issue_copies(c, n_copy, n_copy_all);
+      prof_end(c, p, c->s_copy);
+      if (st != FT_OK) return c->latched = st;
+      CK(cudaEventRecord(c->ev_pfd, c->s_copy));
+      c->pf_pending = true;
     }
     CK(cudaStreamWaitEvent(cs, c->ev_side, 0));
     c->prefetched = -1;
@@ -671,6 +716,10 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
     prof_end(c, p, cs);
     c->kernel_launches += 1;
     CK(cudaStreamWaitEvent(cs, c->ev_pf[layer & 1], 0));
+    if (c->pf_pending) {  // slots a decode prefetch is still writing
+      CK(cudaStreamWaitEvent(cs, c->ev_pfd, 0));
+      c->pf_pending = false;
+    }
     if (c->use_tc) {
       // algorithmic bytes with every routed expert read once; at prefill
       // sizes nearly all E experts are routed, so min(E, T*k) is used
@@ -724,6 +773,13 @@ ft_status ft_cache_stats(ft_ctx* c, ft_stats* out) {
   out->last_qstage = c->last_qstage;
   out->device_error = err ? (err == DERR_TIMEOUT ? FT_ETIMEOUT : FT_ESTATE) : (int32_t)c->latched;
   out->kernel_launches = c->kernel_launches;
+  out->prefetched = h.prefetched;
+  return FT_OK;
+}
+
+ft_status ft_moe_set_prefetch(ft_ctx* c, int32_t enable) {
+  if (!c) return FT_EINVAL;
+  c->prefetch_on = enable != 0;
   return FT_OK;
 }
 
@@ -774,6 +830,8 @@ ft_status ft_moe_resize_cache(ft_ctx* c, int64_t new_slots) {
   if (check_device_error(c) != FT_OK) return c->latched;
   const long long C = sh.C, Cn = new_slots;
   c->prefetched = -1;
+  c->has_prev.assign(sh.L, 0);  // the prefetch record does not survive a resize
+  c->pf_pending = false;
   if (Cn == C) return FT_OK;
 
   // 1. what is resident now

@@ -65,6 +65,7 @@ struct Mailbox {
 struct DevCounters {
   unsigned long long layer_calls, lookups, hits, misses, staged, streamed, bytes_h2d, bytes_zero_copy;
   int32_t last_m, last_qstar, last_qstage, pad;
+  unsigned long long prefetched;  // blobs staged by the decode prefetch
 };
 
 // LRU clock state (device).
@@ -89,6 +90,9 @@ struct LookupArgs {
   int is_current;     // 1: this batch is the called layer's (m, q*, q_stage are reported)
   int build_work;     // 1: (re)build the work lists from this batch
   unsigned bp_mbps, bh_mbps;
+  int prefetch;       // 1: decode prefetch batch: resident experts are not touched, missing ones staged
+                      //    while victims last, no lookup record, only the prefetched counter moves
+  const int32_t* counts_src;  // routing counts of the batch (null: this call's)
 };
 
 // Device pointers of a context.
@@ -125,6 +129,7 @@ struct DevState {
   int32_t* sched;            // [N_CLASSES] unit tickets + [N_CLASSES][sched_chunks] chunk completion counters
   int sched_chunks;
   int32_t* route_ctr;        // last-CTA ticket of the fused decode routing kernel (0 between calls)
+  int32_t* prev_counts;      // [L][E] routing counts of each layer's last decode call (prefetch)
   uint32_t* landed;          // [MAX_E] per staged blob of a decode call: the call's epoch once its copy landed
   uint32_t landed_epoch;     // epoch of the current call (0: staged experts wait for all copies on the host side)
 };

@@ -105,7 +105,8 @@ __device__ __forceinline__ unsigned long long slot_key(const unsigned long long*
 __device__ __forceinline__ void lookup_body(const LookupArgs& a, int E, long long C, size_t slot_bytes,
                                             DevState& ds, const int32_t* s_counts = nullptr,
                                             const int32_t* s_offsets = nullptr) {
-  const int32_t* counts = s_counts ? s_counts : ds.counts;
+  const int32_t* counts = s_counts ? s_counts : (a.counts_src ? a.counts_src : ds.counts);
+  const bool pf = a.prefetch != 0;
   const int32_t* offsets = s_offsets ? s_offsets : ds.offsets;
   __shared__ int s_e[MAX_E];
   __shared__ int s_slot[MAX_E];
@@ -158,7 +159,7 @@ __device__ __forceinline__ void lookup_body(const LookupArgs& a, int E, long lon
   }
   __syncthreads();
   const unsigned long long c0 = s_c0, epoch = s_epoch;
-  if (hit) ds.stamp[sl] = c0 + 1 + (unsigned long long)hrank;
+  if (hit && !pf) ds.stamp[sl] = c0 + 1 + (unsigned long long)hrank;  // a prefetch leaves hits alone
 
   // 4. q*
   int q, q_stage;
@@ -186,8 +187,8 @@ __device__ __forceinline__ void lookup_body(const LookupArgs& a, int E, long lon
     for (int o = 16; o > 0; o >>= 1) avail_local += __shfl_xor_sync(0xffffffffu, avail_local, o);
     if ((tid & 31) == 0) atomicAdd(&s_avail, avail_local);
     __syncthreads();
-    if (s_avail < q_stage) {
-      if (tid == 0) atomicExch(ds.error, (uint32_t)DERR_NO_VICTIM);
+    if (s_avail < q_stage) {  // a prefetch stages what fits; a lookup must not run short
+      if (tid == 0 && !pf) atomicExch(ds.error, (uint32_t)DERR_NO_VICTIM);
       q_stage = s_avail;
     }
   }
@@ -281,13 +282,13 @@ __device__ __forceinline__ void lookup_body(const LookupArgs& a, int E, long lon
     if (old >= 0) ds.slot_of[old] = -1;
     ds.key_of[v] = key;
     ds.slot_of[key] = v;
-    ds.stamp[v] = c0 + (unsigned long long)h + 1ull + (unsigned long long)mrank;
+    ds.stamp[v] = c0 + (unsigned long long)(pf ? 0 : h) + 1ull + (unsigned long long)mrank;
     s_slot[tid] = v;
   } else if (act) {
     s_slot[tid] = hit ? sl : -1;
   }
   if (tid == 0) {
-    ds.clk->clock = c0 + (unsigned long long)h + (unsigned long long)q_stage;
+    ds.clk->clock = c0 + (unsigned long long)(pf ? 0 : h) + (unsigned long long)q_stage;
     ds.clk->batch_start = s_bstart;
   }
   __syncthreads();
@@ -325,14 +326,14 @@ __device__ __forceinline__ void lookup_body(const LookupArgs& a, int E, long lon
     mb->copy_key[cbase + mrank] = key;
     mb->copy_slot[cbase + mrank] = s_slot[tid];
   }
-  if (act) {
+  if (act && !pf) {
     mb->lookup_e[lbase + tid] = e;
     mb->lookup_kind[lbase + tid] = kind;
   }
   __syncthreads();
   if (tid == 0) {
     mb->n_copy = cbase + q_stage;
-    mb->n_lookup = lbase + n_u;
+    mb->n_lookup = lbase + (pf ? 0 : n_u);
     if (a.is_current) {
       mb->m = m;
       mb->qstar = q;
@@ -354,13 +355,18 @@ __device__ __forceinline__ void lookup_body(const LookupArgs& a, int E, long lon
     }
     mb->pad_error = *ds.error;
     DevCounters* c = ds.ctr;
-    c->lookups += n_u;
-    c->hits += h;
-    c->misses += m;
-    c->staged += q_stage;
-    c->streamed += m - q_stage;
-    c->bytes_h2d += (unsigned long long)q_stage * slot_bytes;
-    c->bytes_zero_copy += (unsigned long long)(m - q_stage) * slot_bytes;
+    if (pf) {
+      c->prefetched += q_stage;
+      c->bytes_h2d += (unsigned long long)q_stage * slot_bytes;
+    } else {
+      c->lookups += n_u;
+      c->hits += h;
+      c->misses += m;
+      c->staged += q_stage;
+      c->streamed += m - q_stage;
+      c->bytes_h2d += (unsigned long long)q_stage * slot_bytes;
+      c->bytes_zero_copy += (unsigned long long)(m - q_stage) * slot_bytes;
+    }
     // no fence needed: the host reads the mailbox only after an event recorded
     // behind this kernel has completed
   }
