@@ -16,6 +16,8 @@ Modules
            per-token layer forward
   cache    q* split and the shared LRU expert cache (hit / staged / streamed);
            the best static placement, for the miss-rate comparison
+  ep       the layer with its experts split among G devices: dispatch plan,
+           the all-to-all exchange, owner caches, combine at the source
   policy_compare  the shared LRU against static placements on the 43-layer
            trace (an analysis run of the oracle: python -m oracle.policy_compare)
 
@@ -24,4 +26,4 @@ something other than itself; see each module's docstring. Expert-value parity
 has no printed example on the pages, so the expert math is pinned by a dense
 brute-force evaluation, closed-form special cases and library routines.
 """
-from . import cache, formats, moe  # noqa: F401
+from . import cache, ep, formats, moe  # noqa: F401
