@@ -1,0 +1,88 @@
+"""Expert parallelism: the routed-MoE layer with its experts split among the
+ranks of a process group, one rank per GPU.
+
+Rank r of G owns experts [r E/G, (r+1) E/G) of every layer: its slot cache,
+its share of the host expert pool and its host link serve only those, so G
+ranks bring G host links to the misses. The router is replicated; each rank
+routes its own tokens. Per layer call every rank takes the same steps in the
+same order, with empty blocks where it has nothing to send:
+
+1. route its tokens and pack the rows (t, j) it sends, owner by owner, in
+   its expert-permutation order (expert ascending, then t*k + j) -- ops.dispatch;
+2. exchange the per-owner row counts (an all-to-all of one integer per pair);
+3. exchange the rows and their expert ids (all-to-all with those splits);
+4. run the experts it owns on the rows it received, blocks of ranks 0..G-1
+   one after the other -- ops.experts;
+5. send every output row back the way its input came (all-to-all, splits
+   swapped);
+6. combine its tokens' k outputs in rank order -- ops.combine.
+
+Each output row is the same function of the same input row as on one GPU and
+the combine adds in the same order, so the layer's result does not depend on
+G. The pages serve one GPU and give no split; this one follows the layer's
+definition ([wiki] "FreeToken：エッジネイティブMoEセットアップガイドと比較":
+each token passes through a few of many experts, and a miss costs a move over
+the bus; [ainew] "UC バークレーと MIT、MoE モデルを一般ハードウェアで動かす推論
+エンジン「FreeToken」公開": in a datacenter NVLink hides moves between devices).
+
+This module moves data and sizes between the compute steps with
+torch.distributed (NCCL between GPUs); the compute steps are the `ops`
+object's. An ops object provides
+
+    dispatch(layer, x, bias) -> (rows [n, d], eids [n] int64,
+                                 send_counts: list of G ints, state)
+    experts(layer, mode, rows [m, d], eids [m] int64) -> out [m, d]
+    combine(out_back [n, d], state) -> y [T, d]
+
+where rows are sent in the order described in step 1, `state` is whatever
+the combine needs from the dispatch (the inverse order and the weights), and
+experts() keeps the row order.
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+
+def owned_experts(E: int, G: int, rank: int) -> range:
+    """The experts of every layer that `rank` owns when E experts are split
+    among G ranks."""
+    if E % G:
+        raise ValueError(f"{G} ranks do not divide {E} experts")
+    n = E // G
+    return range(rank * n, (rank + 1) * n)
+
+
+class ExpertParallelLayer:
+    """One rank's side of the expert-parallel layer call."""
+
+    def __init__(self, ops, n_experts: int, group=None):
+        self.ops = ops
+        self.group = group
+        self.G = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        self.E = n_experts
+        self.owned = owned_experts(n_experts, self.G, self.rank)
+
+    def _exchange(self, send, send_counts, recv_counts):
+        """All-to-all of the first axis of `send`, split by send_counts among
+        the ranks; returns the blocks received, in rank order."""
+        out = send.new_empty((sum(recv_counts),) + tuple(send.shape[1:]))
+        dist.all_to_all_single(out, send.contiguous(), recv_counts, send_counts, group=self.group)
+        return out
+
+    def forward(self, layer: int, mode: int, x, bias=None):
+        """The layer on this rank's tokens x [T, d] (T may be 0)."""
+        rows, eids, send_counts, state = self.ops.dispatch(layer, x, bias)
+        send_counts = [int(n) for n in send_counts]
+        if len(send_counts) != self.G or sum(send_counts) != rows.shape[0]:
+            raise ValueError("dispatch: one count per rank, summing to the rows sent")
+        sc = torch.tensor(send_counts, dtype=torch.int64, device=rows.device)
+        rc = torch.empty_like(sc)
+        dist.all_to_all_single(rc, sc, group=self.group)
+        recv_counts = [int(n) for n in rc.tolist()]
+        recv_rows = self._exchange(rows, send_counts, recv_counts)
+        recv_eids = self._exchange(eids, send_counts, recv_counts)
+        out = self.ops.experts(layer, mode, recv_rows, recv_eids)
+        back = self._exchange(out, recv_counts, send_counts)
+        return self.ops.combine(back, state)
