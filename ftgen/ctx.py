@@ -23,17 +23,24 @@ def host_view(addr: int, nbytes: int) -> torch.Tensor:
 
 
 class Harness:
-    """A context plus the tensors it points at (router weights, streams)."""
+    """A context plus the tensors it points at (router weights, streams).
+
+    With n_experts set, the context holds only the global experts
+    expert_base .. expert_base + n_experts - 1 of every layer (one device's
+    share of an expert-parallel layer), as its local experts 0..n_experts-1,
+    and routes nothing; self.routers still holds the full [E, d] routers."""
 
     def __init__(self, wl: ftgen.Workload, L=None, cache_slots=None, max_tokens=None, gen_device="cuda",
-                 device=0, fill=True):
+                 device=0, fill=True, expert_base=0, n_experts=None):
         self.wl = wl
+        self.E = wl.E if n_experts is None else n_experts
+        self.expert_base = expert_base
         self.L = wl.L if L is None else L
         self.C = wl.cache_slots if cache_slots is None else cache_slots
         self.max_tokens = max(wl.batches) if max_tokens is None else max_tokens
         self.dev = torch.device("cuda", device)
         self.gen_device = gen_device
-        self.cfg = ft.make_config(self.L, wl.E, wl.k, wl.d, wl.d_ff, wl.wtype, self.C, self.max_tokens, device)
+        self.cfg = ft.make_config(self.L, self.E, wl.k, wl.d, wl.d_ff, wl.wtype, self.C, self.max_tokens, device)
         self.slot_bytes = ft.ft_moe_slot_bytes(self.cfg)
         assert self.slot_bytes == wl.slot_bytes
         self.stream = torch.cuda.current_stream(self.dev)
@@ -43,7 +50,8 @@ class Harness:
         for l in range(self.L):
             w = ftgen.router_weight(wl.E, wl.d, wl.wtype, wl.seed("router", l)).to(self.dev)
             self.routers.append(w)
-            ft.ft_moe_set_router(self.ctx, l, w)
+            if n_experts is None:
+                ft.ft_moe_set_router(self.ctx, l, w)
         self.tscales = {}
         if fill:
             self.fill_pool()
@@ -52,7 +60,7 @@ class Harness:
     # --- expert pool --------------------------------------------------------
     def layer_view(self, layer: int) -> torch.Tensor:
         base = ft.ft_moe_expert_ptr(self.ctx, layer, 0)
-        return host_view(base, self.wl.E * self.slot_bytes)
+        return host_view(base, self.E * self.slot_bytes)
 
     def blob(self, layer: int, e: int) -> np.ndarray:
         """numpy view of one pinned blob (read by the oracle)."""
@@ -63,11 +71,12 @@ class Harness:
         wl = self.wl
         for l in range(self.L):
             view = self.layer_view(l)
-            for e in range(wl.E):
-                b = ftgen.expert_blob(wl.d, wl.d_ff, wl.wtype, wl.seed("expert", l, e), device=self.gen_device)
+            for e in range(self.E):
+                g = self.expert_base + e  # global expert id: the blob is the same on any device
+                b = ftgen.expert_blob(wl.d, wl.d_ff, wl.wtype, wl.seed("expert", l, g), device=self.gen_device)
                 view[e * self.slot_bytes:(e + 1) * self.slot_bytes].copy_(b)
                 if wl.wtype == ftgen.W_NVFP4:
-                    ts = ftgen.tensor_scales(wl.seed("tscale", l, e))
+                    ts = ftgen.tensor_scales(wl.seed("tscale", l, g))
                     self.tscales[(l, e)] = ts
                     ft.ft_moe_set_tensor_scales(self.ctx, l, e, ts)
         torch.cuda.synchronize(self.dev)

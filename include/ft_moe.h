@@ -12,6 +12,8 @@
  *   [leadeas]    "FreeToken ― コンシューマGPUで大規模MoEモデルをローカル高速推論する
  *                エンジン" (leadeas.co.jp)
  *   [wiki]       "FreeToken：エッジネイティブMoEセットアップガイドと比較"
+ *   [ainew]      "UC バークレーと MIT、MoE モデルを一般ハードウェアで動かす推論エンジン
+ *                「FreeToken」公開"
  *
  * What one layer call computes (the result never depends on where a weight
  * was read from: [paperlens] 設計: 2階建てのエキスパート記憶, paper §3.3; the
@@ -162,6 +164,32 @@ ft_status ft_moe_layer_forward(ft_ctx* ctx, int32_t layer, int32_t mode, const v
                                const float* bias_dev, int32_t bias_per_token, void* y_dev,
                                int32_t* ids_dev_opt, float* w_dev_opt);
 
+/* Expert outputs of rows that are already routed: the owner's half of an
+ * expert-parallel layer, where G devices split the E experts of every layer
+ * in G contiguous blocks and each device runs only the experts it owns on the
+ * rows other devices send it (see ft_ep_pack). The pages serve one GPU; in a
+ * datacenter a fast interconnect hides the moves between devices ([ainew]
+ * "UC バークレーと MIT、MoE モデルを一般ハードウェアで動かす推論エンジン
+ * 「FreeToken」公開", opening paragraph), and here each device's misses go over
+ * its own host link.
+ *
+ * The context is this device's: its n_experts are the experts it owns, local
+ * ids 0..n_experts-1, with their pool, slots and LRU. Row i goes through expert
+ * eids_dev[i] - expert_base with weight 1, exactly as a token routed to that
+ * expert alone: the same lookup, q* split, staging and expert kernels as
+ * ft_moe_layer_forward with top_k = 1 (mode FT_DECODE or FT_PREFILL), and no
+ * router.
+ *   rows_dev  [n][d] activations (fp32 for FT_W_F32, else bf16), 16-byte aligned
+ *   eids_dev  [n] int32 global expert ids, device pointer
+ *   expert_base  global id of local expert 0
+ *   out_dev   [n][d] fp32 expert outputs in row order (unrounded, so that the
+ *             source device's combine rounds once), 16-byte aligned
+ * n may be 0; n <= max_tokens (FT_EINVAL otherwise). An id outside
+ * [expert_base, expert_base + n_experts) latches a device error (FT_ESTATE
+ * on the next call) and that row is computed with local expert 0. */
+ft_status ft_moe_expert_rows(ft_ctx* ctx, int32_t layer, int32_t mode, const void* rows_dev,
+                             const int32_t* eids_dev, int32_t expert_base, int32_t n, float* out_dev);
+
 /* Counters since init (or the last ft_moe_reset_cache). Synchronises. */
 typedef struct {
   uint64_t layer_calls;     /* forward calls with T > 0 */
@@ -302,6 +330,44 @@ ft_status ft_moe_profile_read(ft_ctx* ctx, ft_kernel_time* out, int32_t cap, int
 ft_status ft_route_topk_static(const void* x_dev, const void* w_router_dev, const float* bias_dev,
                                int32_t bias_per_token, int32_t T, int32_t n_experts, int32_t d_model, int32_t top_k,
                                int32_t wtype, int32_t* ids_dev, float* w_dev, void* stream);
+
+/* Expert parallelism, the two context-free steps around the exchange. G
+ * devices split the E experts of every layer in G contiguous blocks (device o
+ * owns [o E/G, (o+1) E/G)); each routes its own tokens (ft_route_topk_static),
+ * sends every routed row (t, j) to the owner of its expert, gets the expert
+ * output back and combines ([ainew] page as for ft_moe_expert_rows).
+ *
+ * ft_ep_pack orders the T*k routed rows of this device by expert, then by flat
+ * index t*k + j (the stable permutation of ft_moe_last_route), so the rows for
+ * owner o are one contiguous block and the blocks follow owner order:
+ *   ids_dev   [T][top_k] int32 routing ids (rank order), device pointer
+ *   x_dev     [T][d_model] activations (fp32 for FT_W_F32, else bf16)
+ *   rows_dev  [T*top_k][d_model] out: x[t] for the row at each sorted position
+ *   eids_dev  [T*top_k] int32 out: the row's expert
+ *   owner_counts_dev [n_owners] int64 out: rows for each owner, in order
+ *   inv_dev   [T*top_k] int32 out: flat index t*k+j -> its row's position
+ *   bad_ids_dev  NULL, or int32 out: number of ids outside [0, n_experts)
+ *             (such ids are treated as expert n_experts - 1)
+ *   scratch_dev / scratch_bytes: device scratch of at least
+ *             ft_ep_pack_scratch_bytes(T, top_k, n_experts) bytes, 256-byte
+ *             aligned, not read before it is written
+ *   stream: cudaStream_t to enqueue on (0 = legacy default stream)
+ * x, rows 16-byte aligned; n_experts <= 512 and a multiple of n_owners;
+ * top_k <= 16; d_model a multiple of 8. Nothing is allocated. */
+ft_status ft_ep_pack_scratch_bytes(int32_t T, int32_t top_k, int32_t n_experts, uint64_t* out_bytes);
+ft_status ft_ep_pack(const int32_t* ids_dev, int32_t T, int32_t top_k, int32_t n_experts, int32_t n_owners,
+                     const void* x_dev, int32_t d_model, int32_t wtype, void* rows_dev, int32_t* eids_dev,
+                     int64_t* owner_counts_dev, int32_t* inv_dev, int32_t* bad_ids_dev, void* scratch_dev,
+                     uint64_t scratch_bytes, void* stream);
+
+/* y[t] = sum_{j<k} w[t,j] * Y[inv[t*k+j]] in rank order, fp32, one rounding to
+ * the activation type: the combine of ft_moe_layer_forward over the expert
+ * outputs that came back from the owners, in the order ft_ep_pack sent them.
+ *   y_rows_dev [T*top_k][d_model] fp32; w_dev [T][top_k] fp32; inv_dev from
+ *   ft_ep_pack (a permutation of 0..T*k-1); y_dev [T][d_model] (fp32 for
+ *   FT_W_F32, else bf16). 16-byte aligned; d_model a multiple of 4. */
+ft_status ft_ep_combine(const float* y_rows_dev, const float* w_dev, const int32_t* inv_dev, int32_t T,
+                        int32_t top_k, int32_t d_model, int32_t wtype, void* y_dev, void* stream);
 
 /* Static string for a status code. */
 const char* ft_status_str(ft_status s);

@@ -28,7 +28,8 @@ EXPORTS = (
     "ft_moe_slot_bytes", "ft_moe_init", "ft_moe_destroy", "ft_moe_expert_ptr", "ft_moe_set_tensor_scales",
     "ft_moe_set_router", "ft_moe_layer_forward", "ft_cache_stats", "ft_set_bandwidths", "ft_moe_reset_cache",
     "ft_moe_resize_cache", "ft_moe_set_prefetch", "ft_moe_last_route", "ft_moe_cache_contents", "ft_moe_probe_link", "ft_moe_profile", "ft_moe_profile_read",
-    "ft_route_topk_static", "ft_status_str",
+    "ft_route_topk_static", "ft_moe_expert_rows", "ft_ep_pack_scratch_bytes", "ft_ep_pack", "ft_ep_combine",
+    "ft_status_str",
 )
 FT_ROUTE_STATIC_MAX_TOKENS = 1024
 
@@ -91,6 +92,10 @@ def lib() -> ctypes.CDLL:
             "ft_moe_profile": [P, I32],
             "ft_moe_profile_read": [P, ctypes.POINTER(FtKernelTime), I32, ctypes.POINTER(I32), I32],
             "ft_route_topk_static": [P, P, P, I32, I32, I32, I32, I32, I32, P, P, P],
+            "ft_moe_expert_rows": [P, I32, I32, P, P, I32, I32, P],
+            "ft_ep_pack_scratch_bytes": [I32, I32, I32, ctypes.POINTER(U64)],
+            "ft_ep_pack": [P, I32, I32, I32, I32, P, I32, I32, P, P, P, P, P, P, U64, P],
+            "ft_ep_combine": [P, P, P, I32, I32, I32, I32, P, P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -243,3 +248,31 @@ def ft_route_topk_static(x, w_router, bias, bias_per_token, T, n_experts, d_mode
     _check("ft_route_topk_static",
            lib().ft_route_topk_static(_ptr(x), _ptr(w_router), _ptr(bias), bias_per_token, T, n_experts, d_model,
                                       top_k, wtype, _ptr(ids), _ptr(w), _stream(stream)))
+
+
+def ft_moe_expert_rows(ctx, layer, mode, rows, eids, expert_base, n, out):
+    """Owner side of the expert-parallel layer: rows routed to this context's
+    experts (global ids eids, local id = eid - expert_base) -> fp32 outputs."""
+    _check("ft_moe_expert_rows",
+           lib().ft_moe_expert_rows(ctx, layer, mode, _ptr(rows), _ptr(eids), expert_base, n, _ptr(out)))
+
+
+def ft_ep_pack_scratch_bytes(T, top_k, n_experts) -> int:
+    out = ctypes.c_uint64()
+    _check("ft_ep_pack_scratch_bytes", lib().ft_ep_pack_scratch_bytes(T, top_k, n_experts, ctypes.byref(out)))
+    return out.value
+
+
+def ft_ep_pack(ids, T, top_k, n_experts, n_owners, x, d_model, wtype, rows, eids, owner_counts, inv, bad_ids,
+               scratch, stream):
+    """Routed rows of this device in expert order, with the rows per owner."""
+    _check("ft_ep_pack",
+           lib().ft_ep_pack(_ptr(ids), T, top_k, n_experts, n_owners, _ptr(x), d_model, wtype, _ptr(rows),
+                            _ptr(eids), _ptr(owner_counts), _ptr(inv), _ptr(bad_ids), _ptr(scratch),
+                            0 if scratch is None else scratch.numel() * scratch.element_size(), _stream(stream)))
+
+
+def ft_ep_combine(y_rows, w, inv, T, top_k, d_model, wtype, y, stream):
+    """Combine of the expert outputs returned by the owners (rank order)."""
+    _check("ft_ep_combine",
+           lib().ft_ep_combine(_ptr(y_rows), _ptr(w), _ptr(inv), T, top_k, d_model, wtype, _ptr(y), _stream(stream)))

@@ -26,7 +26,7 @@
 #include "ft_internal.cuh"
 
 namespace ft {
-cudaError_t route_kernels_init(int E);
+cudaError_t route_kernels_init();
 cudaError_t expert_kernels_init(int device);
 void launch_prefill_work(const Shape& sh, int layer, DevState& ds, cudaStream_t st);
 bool prefill_tc_supported(const Shape& sh);
@@ -39,6 +39,9 @@ void launch_to_f16(const void* x, int n, void* y, cudaStream_t st);
 void launch_gemv_mma(const Shape& sh, int cls, int layer, const void* x16, int T, DevState& ds, int max_items,
                      int max_tok, cudaStream_t st);
 void launch_gemm_tc(const Shape& sh, int phase, int T, DevState& ds, cudaStream_t st);
+void launch_rows_in(const int32_t* eids, int n, int base, int E, DevState& ds, cudaStream_t st);
+void launch_combine_rows(const float* ybuf, const float* wts, const int32_t* inv, int T, int k, int d, bool out_f32,
+                         void* y, cudaStream_t st);
 }  // namespace ft
 
 using namespace ft;
@@ -57,7 +60,7 @@ struct ft_ctx {
   cudaEvent_t ev_t0 = nullptr, ev_t1 = nullptr;
   unsigned bp = 1, bh = 1;
   int prefetched = -1;   // layer whose experts the previous prefill call loaded ahead
-  int last_T = 0;
+  int last_T = 0, last_k = 0;  // rows and top-k of the last call (k = 1 after ft_moe_expert_rows)
   unsigned long long layer_calls = 0;
   int last_m = 0, last_qstar = 0, last_qstage = 0;
   ft_status latched = FT_OK;
@@ -413,7 +416,7 @@ ft_status ft_moe_init(const ft_config* cfg, void* compute_stream, void* copy_str
   TRY(cuda_try(cudaEventCreateWithFlags(&c->ev_pfd, cudaEventDisableTiming)));
   TRY(cuda_try(cudaEventCreate(&c->ev_t0)));
   TRY(cuda_try(cudaEventCreate(&c->ev_t1)));
-  TRY(cuda_try(route_kernels_init(sh.E)));
+  TRY(cuda_try(route_kernels_init()));
   TRY(cuda_try(expert_kernels_init(cfg->device)));
   TRY(reset_state(c));
 #undef TRY
@@ -517,9 +520,14 @@ static ft_status issue_copies(ft_ctx* c, int from, int to, uint32_t epoch = 0) {
   return FT_OK;
 }
 
-ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const void* x, int32_t T, const float* bias,
-                               int32_t bias_per_token, void* y, int32_t* ids_opt, float* w_opt) {
-  if (!c) return FT_EINVAL;
+// One layer call. With rows_eids == null: routing of T tokens, then lookup,
+// experts and combine (ft_moe_layer_forward). With rows_eids: T rows already
+// routed, row i to expert rows_eids[i] - rows_base, weight 1, no router; the
+// caller has set sh.k to 1, and y receives the fp32 expert outputs in row
+// order (ft_moe_expert_rows).
+static ft_status layer_call(ft_ctx* c, int32_t layer, int32_t mode, const void* x, int32_t T, const float* bias,
+                            int32_t bias_per_token, void* y, int32_t* ids_opt, float* w_opt,
+                            const int32_t* rows_eids, int32_t rows_base) {
   const Shape& sh = c->sh;
   if (layer < 0 || layer >= sh.L || (mode != FT_DECODE && mode != FT_PREFILL)) return FT_EINVAL;
   if (T < 0 || T > c->cfg.max_tokens) return FT_EINVAL;
@@ -528,17 +536,18 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
   if (!x || !y || x == y) return FT_EINVAL;
   if (((uintptr_t)x | (uintptr_t)y) & 15) return FT_EINVAL;  // 16-byte vector loads and stores
   if (bias && ((uintptr_t)bias & 3)) return FT_EINVAL;
-  if (!c->router[layer]) return FT_ESTATE;
+  if (!rows_eids && !c->router[layer]) return FT_ESTATE;
   DevState& d = c->ds;
   cudaStream_t cs = c->s_comp;
   c->last_T = T;
+  c->last_k = sh.k;
   c->layer_calls += 1;
   const double ab = sh.wtype == FT_W_F32 ? 4.0 : 2.0;
   const int Tk = T * sh.k;
   const bool full_prefill = mode == FT_PREFILL && sh.C >= 2ll * sh.E;
   // decode (and the on-demand prefill fallback) at small T: router, top-k,
   // permutation and lookup in one launch
-  const bool fused_route = !full_prefill && T <= 32;
+  const bool fused_route = !full_prefill && T <= 32 && !rows_eids;
   LookupArgs la{};
   la.layer = layer;
   la.use_counts = 1;
@@ -553,7 +562,13 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
     c->kernel_launches += 1;
   }
   int p = -1;
-  if (fused_route) {
+  if (rows_eids) {
+    p = prof_begin(c, P_PERMUTE, cs, Tk * 16.0 + sh.E * 8.0);
+    launch_rows_in(rows_eids, T, rows_base, sh.E, d, cs);
+    const int n_perm = launch_permute(sh, T, d, cs);
+    prof_end(c, p, cs);
+    c->kernel_launches += 1 + n_perm;
+  } else if (fused_route) {
     p = prof_begin(c, P_ROUTE_FUSED, cs, T * (double)sh.d * ab + sh.E * (double)sh.d * ab + sh.C * 8.0);
     launch_route_decode(sh, x, c->router[layer], bias, bias_per_token, T, la, d, cs);
     prof_end(c, p, cs);
@@ -743,12 +758,38 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
       gemv_class_cost(c, pr, max_items, Tk);  // upper bound: every routed expert
     }
   }
-  p = prof_begin(c, P_COMBINE, cs, Tk * (double)sh.d * 4.0 + T * (double)sh.d * ab + Tk * 8.0);
-  launch_combine(sh, T, d, y, cs);
+  if (rows_eids) {  // k = 1, weight 1: each row's fp32 output, back in row order
+    p = prof_begin(c, P_COMBINE, cs, Tk * (double)sh.d * 8.0 + Tk * 8.0);
+    launch_combine_rows(d.ybuf, d.wts, d.inv, T, 1, sh.d, true, y, cs);
+  } else {
+    p = prof_begin(c, P_COMBINE, cs, Tk * (double)sh.d * 4.0 + T * (double)sh.d * ab + Tk * 8.0);
+    launch_combine(sh, T, d, y, cs);
+  }
   prof_end(c, p, cs);
   c->kernel_launches += 1;
   CK(cudaGetLastError());
   return FT_OK;
+}
+
+ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const void* x, int32_t T, const float* bias,
+                               int32_t bias_per_token, void* y, int32_t* ids_opt, float* w_opt) {
+  if (!c) return FT_EINVAL;
+  return layer_call(c, layer, mode, x, T, bias, bias_per_token, y, ids_opt, w_opt, nullptr, 0);
+}
+
+ft_status ft_moe_expert_rows(ft_ctx* c, int32_t layer, int32_t mode, const void* rows, const int32_t* eids,
+                             int32_t expert_base, int32_t n, float* out) {
+  if (!c) return FT_EINVAL;
+  if (n > 0 && !eids) return FT_EINVAL;
+  // every row is its own "token" routed to one expert: the pipeline runs with
+  // k = 1 for this call (launch arguments are taken by value when enqueued)
+  struct KeepK {
+    Shape& sh;
+    int k;
+    ~KeepK() { sh.k = k; }
+  } keep{c->sh, c->sh.k};
+  c->sh.k = 1;
+  return layer_call(c, layer, mode, rows, n, nullptr, 0, out, nullptr, nullptr, eids, expert_base);
 }
 
 ft_status ft_cache_stats(ft_ctx* c, ft_stats* out) {
@@ -791,7 +832,7 @@ ft_status ft_moe_last_route(ft_ctx* c, int32_t* counts, int32_t* offsets, int32_
   CK(cudaStreamSynchronize(c->s_side));
   CK(cudaStreamSynchronize(c->s_comp));
   const Shape& sh = c->sh;
-  const size_t Tk = (size_t)c->last_T * sh.k;
+  const size_t Tk = (size_t)c->last_T * c->last_k;
   if (counts) CK(cudaMemcpy(counts, c->ds.counts, sizeof(int32_t) * sh.E, cudaMemcpyDeviceToHost));
   if (offsets) CK(cudaMemcpy(offsets, c->ds.offsets, sizeof(int32_t) * (sh.E + 1), cudaMemcpyDeviceToHost));
   if (perm && Tk) CK(cudaMemcpy(perm, c->ds.perm, sizeof(int32_t) * Tk, cudaMemcpyDeviceToHost));

@@ -510,6 +510,17 @@ void launch_combine(const Shape& sh, int T, DevState& ds, void* y, cudaStream_t 
     combine_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(ds.ybuf, ds.wts, ds.inv, sh.k, sh.d, (__nv_bfloat16*)y);
 }
 
+// The same combine over caller buffers: Y rows [*, d] fp32 in sorted order,
+// weights [T*k], inv [T*k]; y fp32 or bf16.
+void launch_combine_rows(const float* ybuf, const float* wts, const int32_t* inv, int T, int k, int d, bool out_f32,
+                         void* y, cudaStream_t st) {
+  dim3 grid(T, (d / 4 + 255) / 256);
+  if (out_f32)
+    combine_kernel<float><<<grid, 256, 0, st>>>(ybuf, wts, inv, k, d, (float*)y);
+  else
+    combine_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(ybuf, wts, inv, k, d, (__nv_bfloat16*)y);
+}
+
 void launch_read_probe(const uint8_t* src, size_t bytes, unsigned long long* sink, cudaStream_t st) {
   read_probe_kernel<<<g_gemv_grid > 0 ? g_gemv_grid : 148, 256, 0, st>>>(reinterpret_cast<const uint4*>(src),
                                                                         bytes / 16, sink);

@@ -627,7 +627,12 @@ void launch_route_decode(const Shape& sh, const void* x, const void* w_router, c
                                                                  T, sh.E, sh.d, sh.k, la, sh.C, sh.slot_bytes, ds);
 }
 
-cudaError_t route_kernels_init(int E) {
+// Dynamic shared-memory limits of the permutation and fused routing kernels,
+// set for the largest supported E (MAX_E): the attribute is per kernel and
+// process-wide, so a limit set for a small E would break the launches of a
+// context (or ft_ep_pack call) with a larger one.
+cudaError_t route_kernels_init() {
+  const int E = MAX_E;
   const int smem = (int)permute_smem_bytes(E), smem_f = (int)route_decode_smem(E);
   cudaError_t e = cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess)

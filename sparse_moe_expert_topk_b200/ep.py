@@ -86,3 +86,64 @@ class ExpertParallelLayer:
         out = self.ops.experts(layer, mode, recv_rows, recv_eids)
         back = self._exchange(out, recv_counts, send_counts)
         return self.ops.combine(back, state)
+
+
+class CudaEpOps:
+    """The compute steps on this rank's GPU, every one a library call.
+
+    ctx is this rank's context whose n_experts are the experts it owns
+    (owned_experts(E, G, rank), local ids 0..E/G-1, with their host pool,
+    slots and LRU) and whose max_tokens bounds the rows it can receive;
+    routers[l] is layer l's full router [E, d] on this GPU (replicated). All
+    calls are enqueued on `stream`, which must be the context's compute
+    stream and the stream torch.distributed runs on (torch's current stream
+    when the layer is called)."""
+
+    def __init__(self, ctx, routers, n_experts: int, top_k: int, d_model: int, wtype: int, group=None, stream=None):
+        from . import (FT_ROUTE_STATIC_MAX_TOKENS, FT_W_F32, ft_ep_combine, ft_ep_pack, ft_ep_pack_scratch_bytes,
+                       ft_moe_expert_rows, ft_route_topk_static)
+        self._route, self._pack, self._rows, self._combine = (ft_route_topk_static, ft_ep_pack,
+                                                              ft_moe_expert_rows, ft_ep_combine)
+        self._scratch_bytes = ft_ep_pack_scratch_bytes
+        self.route_chunk = FT_ROUTE_STATIC_MAX_TOKENS
+        self.ctx, self.routers = ctx, routers
+        self.E, self.k, self.d, self.wtype = n_experts, top_k, d_model, wtype
+        self.act_dtype = torch.float32 if wtype == FT_W_F32 else torch.bfloat16
+        self.G = dist.get_world_size(group)
+        self.base = owned_experts(n_experts, self.G, dist.get_rank(group)).start
+        self.stream = stream
+        self.scratch = None
+
+    def dispatch(self, layer, x, bias):
+        T, dev, k = x.shape[0], x.device, self.k
+        ids = torch.empty((T, k), dtype=torch.int32, device=dev)
+        w = torch.empty((T, k), dtype=torch.float32, device=dev)
+        per_token = 1 if (bias is not None and bias.dim() == 2) else 0
+        for t0 in range(0, T, self.route_chunk):  # routing is per token: chunks are exact
+            t1 = min(T, t0 + self.route_chunk)
+            b = bias[t0:t1] if per_token else bias
+            self._route(x[t0:t1], self.routers[layer], b, per_token, t1 - t0, self.E, self.d, k, self.wtype,
+                        ids[t0:t1], w[t0:t1], self.stream)
+        n = T * k
+        need = self._scratch_bytes(T, k, self.E)
+        if self.scratch is None or self.scratch.numel() < need:
+            self.scratch = torch.empty(need, dtype=torch.uint8, device=dev)
+        rows = torch.empty((n, self.d), dtype=self.act_dtype, device=dev)
+        eids = torch.empty(n, dtype=torch.int32, device=dev)
+        counts = torch.empty(self.G, dtype=torch.int64, device=dev)
+        inv = torch.empty(n, dtype=torch.int32, device=dev)
+        self._pack(ids, T, k, self.E, self.G, x, self.d, self.wtype, rows, eids, counts, inv, None, self.scratch,
+                   self.stream)
+        return rows, eids, counts.tolist(), (w, inv, T)
+
+    def experts(self, layer, mode, rows, eids):
+        n = rows.shape[0]
+        out = torch.empty((n, self.d), dtype=torch.float32, device=rows.device)
+        self._rows(self.ctx, layer, mode, rows, eids, self.base, n, out)
+        return out
+
+    def combine(self, back, state):
+        w, inv, T = state
+        y = torch.empty((T, self.d), dtype=self.act_dtype, device=back.device)
+        self._combine(back, w, inv, T, self.k, self.d, self.wtype, y, self.stream)
+        return y

@@ -67,7 +67,39 @@ def test_null_arguments_are_rejected(lib):
     assert lib.ft_set_bandwidths(None, 1, 1) == ft.FT_EINVAL
     assert lib.ft_cache_stats(None, None) == ft.FT_EINVAL
     assert lib.ft_moe_layer_forward(None, 0, 0, None, 0, None, 0, None, None, None) == ft.FT_EINVAL
+    assert lib.ft_moe_expert_rows(None, 0, 0, None, None, 0, 0, None) == ft.FT_EINVAL
     lib.ft_moe_destroy(None)
+
+
+def test_ep_argument_checks_without_a_gpu(lib):
+    """The expert-parallel entry points reject bad sizes before touching the
+    device; the pack's scratch covers its arrays."""
+    u = ctypes.c_uint64()
+    for T, k, E in [(0, 6, 256), (1, 6, 256), (4096, 6, 256), (5, 1, 8)]:
+        assert lib.ft_ep_pack_scratch_bytes(T, k, E, ctypes.byref(u)) == ft.FT_OK
+        n = T * k
+        chunks = -(-n // 1024) * E
+        assert u.value >= 4 * (n + E + (E + 1) + n + chunks) and u.value % 256 == 0
+    small = ft.ft_ep_pack_scratch_bytes(1, 6, 256)
+    assert ft.ft_ep_pack_scratch_bytes(4096, 6, 256) > small
+    for T, k, E in [(-1, 6, 256), (1, 0, 256), (1, 17, 256), (1, 6, 0), (1, 6, 513)]:
+        assert lib.ft_ep_pack_scratch_bytes(T, k, E, ctypes.byref(u)) == ft.FT_EINVAL
+    assert lib.ft_ep_pack_scratch_bytes(1, 6, 256, None) == ft.FT_EINVAL
+    P = ctypes.c_void_p
+    pack = lambda T, k, E, G, d, wt, counts: lib.ft_ep_pack(  # noqa: E731
+        P(16), T, k, E, G, P(16), d, wt, P(16), P(16), counts, P(16), None, P(256), 1 << 20, None)
+    assert pack(1, 6, 256, 3, 64, ft.FT_W_BF16, P(16)) == ft.FT_EINVAL   # 3 does not divide 256
+    assert pack(1, 6, 8, 16, 64, ft.FT_W_BF16, P(16)) == ft.FT_EINVAL    # more owners than experts
+    assert pack(1, 6, 256, 8, 60, ft.FT_W_BF16, P(16)) == ft.FT_EINVAL   # d not a multiple of 8
+    assert pack(1, 6, 256, 8, 64, 7, P(16)) == ft.FT_EINVAL              # no such weight type
+    assert pack(1, 6, 256, 8, 64, ft.FT_W_BF16, None) == ft.FT_EINVAL    # counts output missing
+    assert pack(1, 0, 256, 8, 64, ft.FT_W_BF16, P(16)) == ft.FT_EINVAL
+    comb = lambda T, k, d, wt, y: lib.ft_ep_combine(P(16), P(16), P(16), T, k, d, wt, y, None)  # noqa: E731
+    assert comb(0, 6, 64, ft.FT_W_BF16, None) == ft.FT_OK                # no tokens, nothing launched
+    assert comb(1, 6, 62, ft.FT_W_BF16, P(32)) == ft.FT_EINVAL
+    assert comb(1, 17, 64, ft.FT_W_BF16, P(32)) == ft.FT_EINVAL
+    assert comb(1, 6, 64, ft.FT_W_BF16, None) == ft.FT_EINVAL
+    assert comb(1, 6, 64, ft.FT_W_BF16, P(16)) == ft.FT_EINVAL           # y aliases the rows
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
