@@ -30,8 +30,6 @@ def gap_hidden(wl, T, seed, w_router, bias, max_rounds=60):
         for t in bad:
             attempts[t] += 1
             x[t] = ftgen.hidden_row(wl.d, wl.wtype, seed, int(t), int(attempts[t]))
-        if bias is not None and np.ndim(bias) == 2:
-            pass
     raise RuntimeError("could not enforce the top-k gap")
 
 

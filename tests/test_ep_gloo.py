@@ -9,6 +9,7 @@ import socket
 import sys
 
 import numpy as np
+import pytest
 import torch.multiprocessing as mp
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -135,3 +136,34 @@ def test_expert_parallel_layer_on_two_gloo_ranks(tmp_path):
         assert got[r]["owned"] == list(range(r * E // G, (r + 1) * E // G))
         assert all(got[r]["exact"]), got[r]["exact"]
         assert got[r]["records"] == want[r]
+
+
+def test_owned_experts_blocks():
+    from sparse_moe_expert_topk_b200.ep import owned_experts
+    assert [list(owned_experts(8, 4, r)) for r in range(4)] == [[0, 1], [2, 3], [4, 5], [6, 7]]
+    assert list(owned_experts(256, 1, 0)) == list(range(256))
+    with pytest.raises(ValueError):
+        owned_experts(256, 3, 0)
+
+
+def test_dispatch_counts_are_checked_before_any_exchange():
+    """A dispatch whose counts do not cover its rows is refused on the host,
+    before the first collective (one gloo rank in this process)."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    from sparse_moe_expert_topk_b200.ep import ExpertParallelLayer
+
+    class BadOps:
+        def dispatch(self, layer, x, bias):
+            return x, torch.zeros(x.shape[0], dtype=torch.int64), [x.shape[0] + 1], None
+
+    store = dist.HashStore()
+    dist.init_process_group("gloo", store=store, rank=0, world_size=1, timeout=datetime.timedelta(seconds=30))
+    try:
+        layer = ExpertParallelLayer(BadOps(), 4)
+        with pytest.raises(ValueError):
+            layer.forward(0, 0, torch.zeros((3, 2), dtype=torch.float64))
+    finally:
+        dist.destroy_process_group()
