@@ -18,6 +18,8 @@ Modules
            the best static placement, for the miss-rate comparison
   ep       the layer with its experts split among G devices: dispatch plan,
            the all-to-all exchange, owner caches, combine at the source
+  ep_compare  expert parallelism against replicas on the same trace: miss
+           rates and blobs over each device's host link (python -m oracle.ep_compare)
   policy_compare  the shared LRU against static placements on the 43-layer
            trace (an analysis run of the oracle: python -m oracle.policy_compare)
 

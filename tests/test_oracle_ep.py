@@ -135,3 +135,14 @@ def test_full_share_caches_have_only_compulsory_misses():
                 seen |= {(layer, int(e)) for e in out["ids"][s].reshape(-1)}
     assert sum(c.n["misses"] for c in caches) == len(seen)
     assert sum(c.n["streamed"] for c in caches) == 0
+
+
+def test_ep_compare_g1_equals_replicas_and_runs():
+    """The expert-parallel simulation: with one device both arms are the same
+    cache on the same stream; with several it runs and counts sensibly."""
+    from oracle import ep_compare
+    rows = ep_compare.run(steps=4, gs=(1, 2), fracs=(0.10,))
+    g1 = rows[0]
+    assert g1[0] == 1 and g1[3] == g1[4] and g1[5] == g1[6]
+    g2 = rows[1]
+    assert 0 < g2[3] <= 1 and 0 < g2[4] <= 1 and g2[5] > 0 and g2[6] > 0
