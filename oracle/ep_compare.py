@@ -10,7 +10,10 @@ draws Zipf(1.1)), each with the same number of slots:
   shared LRU with the q* admission;
 * expert parallelism (oracle/ep.py): device o owns experts [o E/G, (o+1) E/G)
   of every layer and caches only those, for the rows all G streams route to
-  them.
+  them;
+* the same with the decode prefetch on every owner (after its lookup for
+  layer l it stages layer l+1's experts of its last call); a prefetched blob
+  crosses the owner's link during layer l and counts there.
 
 A miss costs a blob over the device's own host link either way (staged or
 streamed). Replicas run independently: each device's step takes its own
@@ -53,8 +56,11 @@ def run(steps: int = 256, gs=(1, 2, 4, 8), fracs=(0.10, 0.37), profile=(52700, 7
             C = int(f * L * E)
             rep = [cache.ExpertCache(L, E, C, *profile) for _ in range(G)]
             own = [cache.ExpertCache(L, E // G, C, *profile) for _ in range(G)]
+            own_pf = [cache.ExpertCache(L, E // G, C, *profile) for _ in range(G)]
+            for c in own_pf:
+                c.prefetch_on = True
             blobs_rep = np.zeros(G)  # per device, over all steps
-            link_ep = 0
+            link_ep = link_pf = 0
             for st in range(steps):
                 for l in range(L):
                     m_rep, per_owner = [], [np.zeros(E // G, int) for _ in range(G)]
@@ -66,15 +72,24 @@ def run(steps: int = 256, gs=(1, 2, 4, 8), fracs=(0.10, 0.37), profile=(52700, 7
                                 per_owner[int(e) // (E // G)][int(e) % (E // G)] += 1
                         m_rep.append(rep[g].forward(l, cache.DECODE, cnt)["m"])
                     m_own = [own[o].forward(l, cache.DECODE, per_owner[o])["m"] for o in range(G)]
+                    m_pf = []
+                    for o in range(G):
+                        before = own_pf[o].n["prefetched"]
+                        m = own_pf[o].forward(l, cache.DECODE, per_owner[o])["m"]
+                        m_pf.append(m + own_pf[o].n["prefetched"] - before)
                     blobs_rep += m_rep
                     link_ep += max(m_own)
+                    link_pf += max(m_pf)
             miss_rep = sum(c.n["misses"] for c in rep) / sum(c.n["lookups"] for c in rep)
             miss_ep = sum(c.n["misses"] for c in own) / sum(c.n["lookups"] for c in own)
+            miss_pf = sum(c.n["misses"] for c in own_pf) / sum(c.n["lookups"] for c in own_pf)
             # tokens per second on the link model (`batch` tokens per device per step)
             sec = blob / (link_gbs * 1e9)
             tps_rep = sum(batch * steps / (b * sec) for b in blobs_rep if b) if blobs_rep.all() else float("inf")
             tps_ep = G * batch * steps / (link_ep * sec) if link_ep else float("inf")
-            rows.append((G, C, f, miss_rep, miss_ep, blobs_rep.mean() / steps, link_ep / steps, tps_rep, tps_ep))
+            tps_pf = G * batch * steps / (link_pf * sec) if link_pf else float("inf")
+            rows.append((G, C, f, miss_rep, miss_ep, blobs_rep.mean() / steps, link_ep / steps, tps_rep, tps_ep,
+                         miss_pf, link_pf / steps, tps_pf))
     return rows
 
 
@@ -88,6 +103,13 @@ if __name__ == "__main__":
           "link blobs per step, replicas (mean device) | expert parallel (slowest owner per layer) | "
           "tokens/s on the link model, replicas | expert parallel |")
     print("|---|---|---|---|---|---|---|---|---|")
-    for G, C, f, mr, me, lr, le, tr, te in rows:
+    for G, C, f, mr, me, lr, le, tr, te, *_ in rows:
         print(f"| {G} | {C} | {100 * f:.0f}% | {100 * mr:.1f}% | {100 * me:.1f}% | {lr:.1f} | {le:.1f} | "
               f"{tr:.1f} | {te:.1f} |")
+    print()
+    print("| devices | capacity | expert parallel: miss rate | with prefetch | link blobs per step (slowest owner) | "
+          "with prefetch | tokens/s on the link model | with prefetch |")
+    print("|---|---|---|---|---|---|---|---|")
+    for G, C, f, mr, me, lr, le, tr, te, mp, lp, tp in rows:
+        print(f"| {G} | {100 * f:.0f}% | {100 * me:.1f}% | {100 * mp:.1f}% | {le:.1f} | {lp:.1f} | {te:.1f} | "
+              f"{tp:.1f} |")
