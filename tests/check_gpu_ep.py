@@ -162,3 +162,43 @@ def test_ep_prefill_bf16_full_layer(cuda_ok):
         _layer(ow, xs, None, mode=ft.FT_PREFILL, sample=sample)
     finally:
         ow.close()
+
+
+def test_ep_layer_module_on_one_nccl_rank(cuda_ok):
+    """ExpertParallelLayer with CudaEpOps on a one-rank NCCL group: the owner
+    holds every expert, the all-to-alls are local, and the layer must agree
+    with the one-device forward of a context over the same pool and router
+    (the same cache counters; outputs within the BF16 tolerance, since the
+    decode forward routes with its fused kernel, whose logits may differ from
+    the separate router's in the last bit)."""
+    import datetime
+    import os
+
+    import torch.distributed as dist
+    from ftgen.ctx import Harness
+    from sparse_moe_expert_topk_b200.ep import CudaEpOps, ExpertParallelLayer
+
+    wl = ftgen.workload("decode_bf16")
+    bias = ftgen.zipf_log_bias(wl.E, 1.1, wl.seed("zipf"))
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ.setdefault("MASTER_PORT", "29561")
+    dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=60))
+    one = Harness(wl, cache_slots=48, max_tokens=16)
+    own = Harness(wl, cache_slots=48, max_tokens=16 * wl.k, expert_base=0, n_experts=wl.E, fill=True)
+    try:
+        ops = CudaEpOps(own.ctx, own.routers, wl.E, wl.k, wl.d, wl.wtype, stream=own.stream)
+        layer = ExpertParallelLayer(ops, wl.E)
+        b = torch.as_tensor(bias, dtype=torch.float32).to(own.dev)
+        for step, T in enumerate([1, 4, 16, 16, 4, 1]):
+            x = gap_hidden(wl, T, wl.seed("ep_one", step), own.routers[0], bias).to(own.dev)
+            y_ep = layer.forward(0, ft.FT_DECODE, x, b)
+            y_one = one.forward(0, x, b)
+            torch.cuda.synchronize()
+            check_close(to_np(y_ep), to_np(y_one).astype(np.float64), wl.wtype, f"step {step}")
+        s_one, s_own = one.stats(), own.stats()
+        for key in ("lookups", "hits", "misses", "staged", "streamed"):
+            assert s_one[key] == s_own[key], key
+    finally:
+        one.close()
+        own.close()
+        dist.destroy_process_group()
