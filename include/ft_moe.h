@@ -206,6 +206,14 @@ typedef struct {
   int32_t device_error;     /* 0, or the latched ft_status of a device failure */
   uint64_t kernel_launches; /* CUDA kernels this context launched */
   uint64_t prefetched;      /* blobs staged by the decode prefetch (ft_moe_set_prefetch) */
+  /* Device time, from CUDA events the context records on its own streams
+   * around every layer call: ms_compute sums each call's span on the compute
+   * stream (first launch to the combine, the streamed class's side stream
+   * joined in), ms_copy each call's span of copy-engine staging on the copy
+   * stream (the staged misses and the prefill layer-ahead loads). Where
+   * ms_copy is close to ms_compute the copies ran hidden behind compute. */
+  double ms_compute;
+  double ms_copy;
 } ft_stats;
 ft_status ft_cache_stats(ft_ctx* ctx, ft_stats* out);
 

@@ -27,7 +27,8 @@ to the top-k weights; k = 1 (output = one expert, weight exactly 1); k = E
 logits (ids 0..k-1, output 0); duplicate router rows (lower index wins);
 structured weights with a closed-form SwiGLU output; silu against
 torch.nn.functional.silu; top-k against numpy's stable lexsort on random
-logits with planted ties; the permutation against its defining sort.
+logits with planted ties; the permutation against its defining sort;
+layer_forward_grouped against layer_forward.
 """
 from __future__ import annotations
 
@@ -142,3 +143,47 @@ def layer_forward(x, w_router, bias, k, expert_weights, tokens=None):
             acc = acc + w[n, j] * expert_ffn(*cache[e], x[t])
         y[n] = acc
     return y, ids, w
+
+
+def layer_forward_grouped(x, w_router, bias, k, expert_weights, tokens=None):
+    """The same layer as layer_forward, evaluated expert by expert: each
+    chosen expert is applied once to the matrix whose columns are the tokens
+    routed to it (expert_ffn on a [d, n] argument is n independent columns),
+    then every token adds its k outputs with its weights in rank order. Every
+    output element is the same fp64 expression as in layer_forward; only the
+    order in which the experts are visited differs, so large layers (thousands
+    of tokens over hundreds of experts) decode each expert's weights once.
+
+    Arguments and result as layer_forward."""
+    return layer_forward_batches([(x, w_router, bias, tokens)], k, expert_weights)[0]
+
+
+def layer_forward_batches(batches, k, expert_weights):
+    """layer_forward_grouped over several batches of one layer's experts at
+    once, so that each expert's weights are decoded once for all of them:
+    batches is a list of (x, w_router, bias, tokens); returns one
+    (y, ids, w) per batch, each as layer_forward would."""
+    routed = []
+    for x, w_router, bias, tokens in batches:
+        x = np.asarray(x, np.float64)
+        tok = np.arange(x.shape[0]) if tokens is None else np.asarray(tokens)
+        b = bias
+        if bias is not None and np.ndim(bias) == 2:
+            b = np.asarray(bias)[tok]
+        ids, w, _ = route(x[tok], w_router, b, k)
+        out = np.zeros((len(tok), k, x.shape[1]), dtype=np.float64)  # expert output of (token, rank)
+        routed.append((x, tok, ids, w, out))
+    experts = np.unique(np.concatenate([r[2].ravel() for r in routed])) if routed else []
+    for e in experts:
+        wg, wu, wd = expert_weights(int(e))
+        for x, tok, ids, _, out in routed:
+            rows, ranks = np.nonzero(ids == e)
+            if rows.size:
+                out[rows, ranks] = expert_ffn(wg, wu, wd, x[tok[rows]].T).T
+    res = []
+    for x, tok, ids, w, out in routed:
+        y = np.zeros((len(tok), x.shape[1]), dtype=np.float64)
+        for j in range(k):
+            y = y + w[:, j:j + 1] * out[:, j]
+        res.append((y, ids, w))
+    return res

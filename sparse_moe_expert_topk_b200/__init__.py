@@ -45,7 +45,8 @@ class FtStats(ctypes.Structure):
                 ("misses", ctypes.c_uint64), ("staged", ctypes.c_uint64), ("streamed", ctypes.c_uint64),
                 ("bytes_h2d", ctypes.c_uint64), ("bytes_zero_copy", ctypes.c_uint64),
                 ("last_m", ctypes.c_int32), ("last_qstar", ctypes.c_int32), ("last_qstage", ctypes.c_int32),
-                ("device_error", ctypes.c_int32), ("kernel_launches", ctypes.c_uint64), ("prefetched", ctypes.c_uint64)]
+                ("device_error", ctypes.c_int32), ("kernel_launches", ctypes.c_uint64), ("prefetched", ctypes.c_uint64),
+                ("ms_compute", ctypes.c_double), ("ms_copy", ctypes.c_double)]
 
     def as_dict(self):
         return {k: getattr(self, k) for k, _ in self._fields_}

@@ -86,6 +86,14 @@ struct ft_ctx {
   };
   std::vector<ProfRec> pend;
   std::vector<cudaEvent_t> evpool;
+  // always-on spans of each call on the compute stream and of its staging
+  // copies on the copy stream (ft_stats.ms_compute / ms_copy)
+  struct Span {
+    cudaEvent_t a, b;
+    bool copy;
+  };
+  std::vector<Span> spans;
+  double ms_compute = 0, ms_copy = 0;
   struct Agg {
     unsigned long long n = 0;
     double ms = 0, bytes = 0, flops = 0;
@@ -171,10 +179,17 @@ void free_all(ft_ctx* c) {
     cudaEventDestroy(r.a);
     cudaEventDestroy(r.b);
   }
+  for (auto& r : c->spans) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
   for (cudaEvent_t e : c->evpool) cudaEventDestroy(e);
   if (c->s_side) cudaStreamDestroy(c->s_side);
   delete c;
 }
+
+void fold_spans(ft_ctx* c, bool wait);
+cudaEvent_t pooled_event(ft_ctx* c);
 
 ft_status reset_state(ft_ctx* c) {
   const Shape& sh = c->sh;
@@ -189,6 +204,9 @@ ft_status reset_state(ft_ctx* c) {
   CK(cudaMemsetAsync(d.error, 0, sizeof(uint32_t), c->s_comp));
   CK(cudaStreamSynchronize(c->s_comp));
   memset(c->mbox_host, 0, sizeof(Mailbox));
+  CK(cudaStreamSynchronize(c->s_copy));
+  fold_spans(c, true);
+  c->ms_compute = c->ms_copy = 0;
   c->prefetched = -1;
   c->has_prev.assign(sh.L, 0);
   c->pf_pending = false;
@@ -247,6 +265,23 @@ void prof_bytes(ft_ctx* c, int idx, double bytes, double flops) {
     c->pend[idx].bytes = bytes;
     c->pend[idx].flops = flops;
   }
+}
+
+// Fold finished spans into ms_compute / ms_copy, oldest first; with wait,
+// every span (the caller has synchronised the streams). A span whose end has
+// not been reached stops the non-blocking fold, so the list stays short.
+void fold_spans(ft_ctx* c, bool wait) {
+  size_t n = 0;
+  for (; n < c->spans.size(); ++n) {
+    const ft_ctx::Span& r = c->spans[n];
+    if (!wait && cudaEventQuery(r.b) != cudaSuccess) break;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, r.a, r.b) == cudaSuccess) (r.copy ? c->ms_copy : c->ms_compute) += ms;
+    c->evpool.push_back(r.a);
+    c->evpool.push_back(r.b);
+  }
+  c->spans.erase(c->spans.begin(), c->spans.begin() + n);
+  cudaGetLastError();  // a not-ready query is not an error of the next call
 }
 
 // Weight bytes per element of the expert format (codes plus block scales for NVFP4).
@@ -506,6 +541,19 @@ static void gemv_class_cost(ft_ctx* c, const int (&pr)[2], int n_items, int n_to
 static ft_status issue_copies(ft_ctx* c, int from, int to, uint32_t epoch = 0) {
   const Mailbox* mb = c->mbox_host;
   const Shape& sh = c->sh;
+  if (to <= from) return FT_OK;
+  ft_ctx::Span sp{pooled_event(c), pooled_event(c), true};
+  CK(cudaEventRecord(sp.a, c->s_copy));
+  struct Close {  // the span ends behind whatever copies were issued
+    ft_ctx* c;
+    ft_ctx::Span sp;
+    ~Close() {
+      if (cudaEventRecord(sp.b, c->s_copy) == cudaSuccess)
+        c->spans.push_back(sp);
+      else
+        c->evpool.push_back(sp.a), c->evpool.push_back(sp.b);
+    }
+  } close{c, sp};
   for (int i = from; i < to; ++i) {
     const int key = mb->copy_key[i], slot = mb->copy_slot[i];
     const int l = key / sh.E, e = key % sh.E;
@@ -539,6 +587,18 @@ static ft_status layer_call(ft_ctx* c, int32_t layer, int32_t mode, const void* 
   if (!rows_eids && !c->router[layer]) return FT_ESTATE;
   DevState& d = c->ds;
   cudaStream_t cs = c->s_comp;
+  fold_spans(c, false);
+  struct CallSpan {  // this call's span on the compute stream, recorded on every return path
+    ft_ctx* c;
+    ft_ctx::Span sp;
+    ~CallSpan() {
+      if (cudaEventRecord(sp.b, c->s_comp) == cudaSuccess)
+        c->spans.push_back(sp);
+      else
+        c->evpool.push_back(sp.a), c->evpool.push_back(sp.b);
+    }
+  } call_span{c, {pooled_event(c), pooled_event(c), false}};
+  CK(cudaEventRecord(call_span.sp.a, cs));
   c->last_T = T;
   c->last_k = sh.k;
   c->layer_calls += 1;
@@ -815,6 +875,9 @@ ft_status ft_cache_stats(ft_ctx* c, ft_stats* out) {
   out->device_error = err ? (err == DERR_TIMEOUT ? FT_ETIMEOUT : FT_ESTATE) : (int32_t)c->latched;
   out->kernel_launches = c->kernel_launches;
   out->prefetched = h.prefetched;
+  fold_spans(c, true);
+  out->ms_compute = c->ms_compute;
+  out->ms_copy = c->ms_copy;
   return FT_OK;
 }
 

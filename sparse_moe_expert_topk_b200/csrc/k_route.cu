@@ -294,6 +294,20 @@ __device__ void logits_bf16_block(const __nv_bfloat16* __restrict__ x, const __n
   }
 }
 
+// BF16 logits of up to 32 tokens by the fused decode routing's device
+// function, as a kernel of its own: the router of every other small-batch
+// call (a prefill of few tokens, the allocation-free entry point) then sums
+// each logit in exactly the order the fused decode routing does. grid
+// ceil(E/16), 1024 threads, dynamic shared memory for the warp partial sums.
+__global__ void __launch_bounds__(1024) router_small_kernel(const __nv_bfloat16* __restrict__ x,
+                                                            const __nv_bfloat16* __restrict__ wr,
+                                                            const float* __restrict__ bias, int bias_per_token,
+                                                            int T, int E, int d, float* __restrict__ scores) {
+  extern __shared__ float red_small[];
+  logits_bf16_block(x, wr, bias, bias_per_token, T, E, d, blockIdx.x * 16, scores, red_small);
+}
+constexpr int SMALL_RED_BYTES = sizeof(float) * 32 * 8 * 32;
+
 // BF16 router logits for many tokens (prefill) on mma.sync: CTA = 16 experts
 // x 64 tokens, warp w takes tokens t0+16w .. +16 over the full K (steps of 32
 // K values, lane-permuted K as in logits_bf16_block; the four warps read the
@@ -433,6 +447,11 @@ __global__ void __launch_bounds__(1024) route_decode_kernel(const AT* __restrict
 
 void launch_router_scores(const Shape& sh, const void* x, const void* w_router, const float* bias, int bias_per_token,
                           int T, float* scores, cudaStream_t st) {
+  if (sh.wtype != FT_W_F32 && T <= 32 && sh.d % 32 == 0) {
+    router_small_kernel<<<(sh.E + 15) / 16, 1024, SMALL_RED_BYTES, st>>>(
+        (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_router, bias, bias_per_token, T, sh.E, sh.d, scores);
+    return;
+  }
   if (sh.wtype != FT_W_F32 && T > 32 && sh.d % 32 == 0) {
     dim3 grid((sh.E + 15) / 16, (T + 63) / 64);
     router_mma_kernel<<<grid, 128, 0, st>>>((const __nv_bfloat16*)x, (const __nv_bfloat16*)w_router, bias,
@@ -638,6 +657,8 @@ cudaError_t route_kernels_init() {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(perm_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)(sizeof(int32_t) * 32 * E));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(router_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMALL_RED_BYTES);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(route_decode_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_f);
   if (e == cudaSuccess)

@@ -18,8 +18,21 @@ same order, with empty blocks where it has nothing to send:
 6. combine its tokens' k outputs in rank order -- ops.combine.
 
 Each output row is the same function of the same input row as on one GPU and
-the combine adds in the same order, so the layer's result does not depend on
-G. The pages serve one GPU and give no split; this one follows the layer's
+the combine adds in the same order. The routing of a token depends only on its
+own row and on its batch size class: batches of up to 32 tokens and larger
+ones sum the router logits with two different kernels, whose fp32 results can
+differ in the last bit, so a token whose k-th and (k+1)-th logits lie within
+that rounding (about sqrt(d) * 2^-24 * sum_i |x_i W_ei|) may route differently
+when its rank holds a batch of the other size class than one GPU would. Away
+from such near-ties the layer's result does not depend on G, and with equal
+batch size classes it is the one-GPU result bit for bit.
+
+Before any row moves, the ranks agree (one all-reduce of a flag) that every
+owner can take the rows sent to it (ops.max_rows, when the ops object has
+one); otherwise every rank raises the same error and no rank is left waiting
+in a later exchange.
+
+The pages serve one GPU and give no split; this one follows the layer's
 definition ([wiki] "FreeToken：エッジネイティブMoEセットアップガイドと比較":
 each token passes through a few of many experts, and a miss costs a move over
 the bus; [ainew] "UC バークレーと MIT、MoE モデルを一般ハードウェアで動かす推論
@@ -33,6 +46,7 @@ object's. An ops object provides
                                  send_counts: list of G ints, state)
     experts(layer, mode, rows [m, d], eids [m] int64) -> out [m, d]
     combine(out_back [n, d], state) -> y [T, d]
+    max_rows (optional attribute): the most rows experts() takes in one call
 
 where rows are sent in the order described in step 1, `state` is whatever
 the combine needs from the dispatch (the inverse order and the weights), and
@@ -81,6 +95,15 @@ class ExpertParallelLayer:
         rc = torch.empty_like(sc)
         dist.all_to_all_single(rc, sc, group=self.group)
         recv_counts = [int(n) for n in rc.tolist()]
+        # every rank takes the same collective steps: agree on the owners'
+        # capacity before the rows move, so that all raise or none does
+        cap = getattr(self.ops, "max_rows", None)
+        ok = torch.tensor([1 if cap is None or sum(recv_counts) <= cap else 0], dtype=torch.int64,
+                          device=rows.device)
+        dist.all_reduce(ok, op=dist.ReduceOp.MIN, group=self.group)
+        if int(ok.item()) == 0:
+            raise ValueError(f"an owner cannot take the rows sent to it this call (this rank receives "
+                             f"{sum(recv_counts)}, takes at most {cap})")
         recv_rows = self._exchange(rows, send_counts, recv_counts)
         recv_eids = self._exchange(eids, send_counts, recv_counts)
         out = self.ops.experts(layer, mode, recv_rows, recv_eids)
@@ -97,9 +120,12 @@ class CudaEpOps:
     routers[l] is layer l's full router [E, d] on this GPU (replicated). All
     calls are enqueued on `stream`, which must be the context's compute
     stream and the stream torch.distributed runs on (torch's current stream
-    when the layer is called)."""
+    when the layer is called). max_rows is the context's max_tokens (the most
+    rows one ft_moe_expert_rows call takes); ExpertParallelLayer checks it on
+    every rank before the rows are exchanged."""
 
-    def __init__(self, ctx, routers, n_experts: int, top_k: int, d_model: int, wtype: int, group=None, stream=None):
+    def __init__(self, ctx, routers, n_experts: int, top_k: int, d_model: int, wtype: int, group=None, stream=None,
+                 max_rows=None):
         from . import (FT_ROUTE_STATIC_MAX_TOKENS, FT_W_F32, ft_ep_combine, ft_ep_pack, ft_ep_pack_scratch_bytes,
                        ft_moe_expert_rows, ft_route_topk_static)
         self._route, self._pack, self._rows, self._combine = (ft_route_topk_static, ft_ep_pack,
@@ -112,6 +138,7 @@ class CudaEpOps:
         self.G = dist.get_world_size(group)
         self.base = owned_experts(n_experts, self.G, dist.get_rank(group)).start
         self.stream = stream
+        self.max_rows = max_rows  # the context's max_tokens: rows ft_moe_expert_rows takes per call
         self.scratch = None
 
     def dispatch(self, layer, x, bias):

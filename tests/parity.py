@@ -110,3 +110,34 @@ def oracle_cache(harness):
 
 def to_np(t):
     return t.detach().float().cpu().numpy()
+
+
+class PrefetchWeights:
+    """Expert weights of one layer decoded by the oracle ahead of use, in
+    ascending expert order, on a few threads (the grouped oracle visits the
+    experts in ascending order and each is decoded once). Keeps only the
+    experts of the window in memory."""
+
+    def __init__(self, harness, layer, workers=8, window=12):
+        from concurrent.futures import ThreadPoolExecutor
+        self.h, self.layer, self.window = harness, layer, window
+        self.pool = ThreadPoolExecutor(max_workers=workers)
+        self.fut = {}
+
+    def _decode(self, e):
+        wl = self.h.wl
+        ts = self.h.tscales.get((self.layer, e))
+        return ofmt.unpack_expert(self.h.blob(self.layer, e).copy(), wl.d, wl.d_ff, wl.wtype, ts)
+
+    def __call__(self, e):
+        for n in range(e, min(self.h.E, e + self.window)):
+            if n not in self.fut:
+                self.fut[n] = self.pool.submit(self._decode, n)
+        w = self.fut.pop(e).result()
+        for n in [n for n in self.fut if n < e]:
+            self.fut.pop(n).cancel()
+        return w
+
+    def close(self):
+        self.pool.shutdown(wait=True, cancel_futures=True)
+        self.fut.clear()

@@ -137,3 +137,32 @@ def test_header_is_plain_c_and_links(lib, tmp_path):
     assert out.returncode == 0, out.stderr
     n, msg = out.stdout.strip().split(" ", 1)
     assert int(n) == len(names) and msg == "invalid argument"
+
+
+def test_struct_layouts_match_the_binding(lib, tmp_path):
+    """sizeof and field offsets of ft_config, ft_stats and ft_kernel_time as
+    a C compiler lays them out equal the ctypes mirrors of the binding."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    mirrors = {"ft_config": ft.FtConfig, "ft_stats": ft.FtStats, "ft_kernel_time": ft.FtKernelTime}
+    lines = []
+    for cname, py in mirrors.items():
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for f, _ in py._fields_:
+            lines.append(f'  printf("{cname} {f} %zu\\n", offsetof({cname}, {f}));')
+    src = tmp_path / "layout.c"
+    src.write_text('#include "ft_moe.h"\n#include <stdio.h>\n#include <stddef.h>\nint main(void) {\n'
+                   + "\n".join(lines) + "\n  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src), "-o",
+                        str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    got = {tuple(l.split()[:2]): int(l.split()[2]) for l in out if l.strip()}
+    for cname, py in mirrors.items():
+        assert got[(cname, "size")] == ctypes.sizeof(py), cname
+        for f, _ in py._fields_:
+            assert got[(cname, f)] == getattr(py, f).offset, (cname, f)

@@ -167,3 +167,48 @@ def test_dispatch_counts_are_checked_before_any_exchange():
             layer.forward(0, 0, torch.zeros((3, 2), dtype=torch.float64))
     finally:
         dist.destroy_process_group()
+
+
+class _SmallOwnerOps(OracleOps):
+    """OracleOps whose owner on rank 1 takes at most two rows per call."""
+
+    def __init__(self, rank, wr, W):
+        super().__init__(rank, wr, W)
+        self.max_rows = 2 if rank == 1 else 10 ** 6
+
+
+def _rank_small_owner(rank, world, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    from sparse_moe_expert_topk_b200.ep import ExpertParallelLayer
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    wr, W = _model()
+    layer_fn = ExpertParallelLayer(_SmallOwnerOps(rank, wr, W), E)
+    res = {}
+    try:
+        layer_fn.forward(0, 0, torch.from_numpy(_tokens(0, 0, rank)))  # 3 + 2 tokens, k = 3: 15 rows
+        res["raised"] = False
+    except ValueError as e:
+        res["raised"] = "owner cannot take" in str(e)
+    # both ranks are still in step: a later collective completes
+    t = torch.ones(1)
+    dist.all_reduce(t)
+    res["after"] = float(t.item())
+    dist.destroy_process_group()
+    with open(os.path.join(out_dir, f"small{rank}.json"), "w") as f:
+        json.dump(res, f)
+
+
+def test_owner_capacity_is_agreed_before_rows_move(tmp_path):
+    """One owner too small for what it is sent: every rank raises the same
+    error before the row exchange, and no rank is left waiting (a collective
+    after the failed call completes on both)."""
+    port = _free_port()
+    mp.start_processes(_rank_small_owner, args=(G, port, str(tmp_path)), nprocs=G, start_method="spawn")
+    got = [json.load(open(tmp_path / f"small{r}.json")) for r in range(G)]
+    assert all(g["raised"] for g in got), got
+    assert all(g["after"] == G for g in got), got

@@ -84,6 +84,11 @@ def test_decode_bf16_64_steps(cuda_ok, T):
         _check_cache_state(h, oc)
         st = h.stats()
         assert st["misses"] > 0 and st["hits"] > 0 and st["staged"] > 0 and st["streamed"] > 0
+        # device time of the calls and of their staging copies, through the ABI
+        assert st["ms_compute"] > 0 and st["ms_copy"] > 0
+        ft.ft_moe_reset_cache(h.ctx)
+        st = h.stats()
+        assert st["ms_compute"] == 0 and st["ms_copy"] == 0
 
 
 def test_outputs_independent_of_cache_state(cuda_ok):

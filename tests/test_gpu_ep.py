@@ -7,10 +7,8 @@ sparse_moe_expert_topk_b200.ep produce (blocks of sources 0..G-1 per owner,
 then the return trip). Against the oracle (oracle/ep.py, oracle/moe.py):
 routing ids, the pack order, the rows per owner, the inverse order and each
 owner's lookup record bit-exact; the layer's outputs within the BF16
-tolerance.
-
-This file is not matched by the suite's test_*.py pattern; run it by name:
-python -m pytest tests/check_gpu_ep.py -m gpu"""
+tolerance. The module layer (ExpertParallelLayer with CudaEpOps) on a
+one-rank NCCL group gives the one-device forward's outputs bit for bit."""
 import numpy as np
 import pytest
 import torch
@@ -167,10 +165,10 @@ def test_ep_prefill_bf16_full_layer(cuda_ok):
 def test_ep_layer_module_on_one_nccl_rank(cuda_ok):
     """ExpertParallelLayer with CudaEpOps on a one-rank NCCL group: the owner
     holds every expert, the all-to-alls are local, and the layer must agree
-    with the one-device forward of a context over the same pool and router
-    (the same cache counters; outputs within the BF16 tolerance, since the
-    decode forward routes with its fused kernel, whose logits may differ from
-    the separate router's in the last bit)."""
+    with the one-device forward of a context over the same pool and router:
+    the same cache counters, and the same output bytes (at up to 32 tokens
+    both route with the same logits code, every expert row is computed by the
+    same GEMV with the same K order, and both combine in rank order)."""
     import datetime
     import os
 
@@ -186,7 +184,7 @@ def test_ep_layer_module_on_one_nccl_rank(cuda_ok):
     one = Harness(wl, cache_slots=48, max_tokens=16)
     own = Harness(wl, cache_slots=48, max_tokens=16 * wl.k, expert_base=0, n_experts=wl.E, fill=True)
     try:
-        ops = CudaEpOps(own.ctx, own.routers, wl.E, wl.k, wl.d, wl.wtype, stream=own.stream)
+        ops = CudaEpOps(own.ctx, own.routers, wl.E, wl.k, wl.d, wl.wtype, stream=own.stream, max_rows=16 * wl.k)
         layer = ExpertParallelLayer(ops, wl.E)
         b = torch.as_tensor(bias, dtype=torch.float32).to(own.dev)
         for step, T in enumerate([1, 4, 16, 16, 4, 1]):
@@ -195,6 +193,7 @@ def test_ep_layer_module_on_one_nccl_rank(cuda_ok):
             y_one = one.forward(0, x, b)
             torch.cuda.synchronize()
             check_close(to_np(y_ep), to_np(y_one).astype(np.float64), wl.wtype, f"step {step}")
+            assert torch.equal(y_ep.view(torch.int16), y_one.view(torch.int16)), f"step {step}"
         s_one, s_own = one.stats(), own.stats()
         for key in ("lookups", "hits", "misses", "staged", "streamed"):
             assert s_one[key] == s_own[key], key

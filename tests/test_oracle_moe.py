@@ -181,3 +181,47 @@ def test_router_logits_round_once_to_fp32():
     assert s.dtype == np.float32
     exact = np.array([[sum(x[t, i] * wr[e, i] for i in range(300)) + b[e] for e in range(5)] for t in range(4)])
     np.testing.assert_array_equal(s, exact.astype(np.float32))
+
+
+@pytest.mark.parametrize("E,k,T,d,d_ff,per_token", [(8, 2, 16, 64, 128, False), (6, 3, 40, 16, 24, True),
+                                                    (9, 1, 7, 12, 20, False), (5, 5, 3, 8, 8, True)])
+def test_grouped_layer_matches_dense_bruteforce_and_per_token(E, k, T, d, d_ff, per_token):
+    """The expert-by-expert evaluation against the dense masked brute force
+    and the per-token layer, on full batches and on token subsets (with a
+    per-token bias, the subset's bias rows are taken)."""
+    rng = np.random.default_rng(7 * E + k)
+    x = rng.normal(0, 1, (T, d))
+    wr = rng.normal(0, 0.5, (E, d))
+    b = rng.normal(0, 0.1, (T, E) if per_token else E)
+    W = _experts(E, d, d_ff, rng)
+    y, ids, w = moe.layer_forward_grouped(x, wr, b, k, lambda e: W[e])
+    yd, _ = dense_masked(x, wr, b if not per_token else None, k, W) if not per_token else (None, None)
+    y1, ids1, w1 = moe.layer_forward(x, wr, b, k, lambda e: W[e])
+    rms = np.sqrt(np.mean(y1 ** 2))
+    np.testing.assert_array_equal(ids, ids1)
+    np.testing.assert_array_equal(w, w1)
+    assert np.max(np.abs(y - y1)) <= 1e-12 * rms
+    if yd is not None:
+        assert np.max(np.abs(y - yd)) <= 1e-9 * rms
+    sub = np.array([T - 1, 0, T // 2])
+    ys, _, _ = moe.layer_forward_grouped(x, wr, b, k, lambda e: W[e], tokens=sub)
+    assert np.max(np.abs(ys - y1[sub])) <= 1e-12 * rms
+
+
+def test_batches_match_each_batch_alone():
+    """Several batches through one expert pass: each result equals the
+    per-token layer on that batch (different routers, biases and subsets)."""
+    rng = np.random.default_rng(11)
+    E, k, d, d_ff = 7, 3, 16, 24
+    W = _experts(E, d, d_ff, rng)
+    batches = []
+    for T, per_token, sub in ((9, False, None), (4, True, [3, 1]), (1, False, None)):
+        x = rng.normal(0, 1, (T, d))
+        wr = rng.normal(0, 0.5, (E, d))
+        b = rng.normal(0, 0.1, (T, E) if per_token else E)
+        batches.append((x, wr, b, sub))
+    res = moe.layer_forward_batches(batches, k, lambda e: W[e])
+    for (x, wr, b, sub), (y, ids, w) in zip(batches, res):
+        y1, ids1, w1 = moe.layer_forward(x, wr, b, k, lambda e: W[e], tokens=sub)
+        np.testing.assert_array_equal(ids, ids1)
+        assert np.max(np.abs(y - y1)) <= 1e-12 * np.sqrt(np.mean(y1 ** 2))
