@@ -202,26 +202,43 @@ def ncu_traffic(kernel_name, launches_per_step):
     return e.get("dram_bytes_per_launch")
 
 
-def roofline(prof, peaks, peak_kind, link_gbs):
+def roofline(prof, peaks, peak_kind, link_gbs, zc_gbs=None):
+    """Per-kernel roofline rows from the library's CUDA-event profile, and the
+    dominant row (the largest summed event time). Each row divides its
+    algorithmic bytes (or flops) by its own event window:
+    * HBM-resident work (hit GEMV, routing, combine, the prefill GEMMs below
+      the ridge) against the measured HBM peak; a GEMM above the ridge against
+      the bf16 tensor peak;
+    * the copy engine's staging copies (events on the copy stream around each
+      call's copies) against the H2D copy rate measured in the same run;
+    * the staged class, whose window opens with its first copy and closes
+      when its last expert is computed, against the same H2D rate;
+    * the streamed class, which reads its weights zero-copy over the host
+      link, against the zero-copy read rate measured in the same run."""
+    zc = zc_gbs if zc_gbs else link_gbs
     rows = {}
     for name, r in prof.items():
-        if r["ms"] <= 0 or name == "h2d_stage_copies":
+        if r["ms"] <= 0:
             continue
         gbs = r["bytes"] / (r["ms"] * 1e6)
         # the binding roof is the larger of the HBM time and the tensor time
         t_hbm = r["bytes"] / (peaks["hbm_gbs"] * 1e9)
         t_tc = r["flops"] / (peaks["bf16_tflops"] * 1e12)
+        src = peak_kind
         if name.startswith("gemm_tc") and t_tc > t_hbm:
             bound, peak, unit, ach = "tensor", peaks["bf16_tflops"], "TFLOP/s", r["flops"] / (r["ms"] * 1e9)
-        elif name.endswith("streamed") or name.endswith("staged"):
-            # streamed experts are read over the host link; the staged GEMV
-            # starts with the copies and consumes each blob as it lands
+        elif name.endswith("streamed"):
+            bound, peak, unit, ach = "host_link", zc, "GB/s", gbs
+            src = "measured zero-copy read GB/s, this run"
+        elif name.endswith("staged") or name.startswith("h2d_"):
             bound, peak, unit, ach = "host_link", link_gbs, "GB/s", gbs
+            src = "measured H2D copy-engine GB/s, this run"
         else:
             bound, peak, unit, ach = "hbm", peaks["hbm_gbs"], "GB/s", gbs
         rows[name] = {"bound": bound, "achieved": round(ach, 2), "peak": round(peak, 2), "unit": unit,
                       "frac": round(ach / peak, 4) if peak else None, "ms_total": round(r["ms"], 3),
-                      "launches": int(r["launches"]), "bytes_per_launch": r["bytes"] / max(r["launches"], 1)}
+                      "launches": int(r["launches"]), "bytes_per_launch": r["bytes"] / max(r["launches"], 1),
+                      "peak_source": src}
     tot = sum(v["ms_total"] for v in rows.values()) or 1.0
     for v in rows.values():
         v["share"] = round(v["ms_total"] / tot, 4)
@@ -230,8 +247,7 @@ def roofline(prof, peaks, peak_kind, link_gbs):
     if dom:
         v = rows[dom]
         out = {"kernel": dom, "bound": v["bound"], "achieved": v["achieved"], "peak": v["peak"], "unit": v["unit"],
-               "frac": v["frac"], "traffic": ncu_traffic(dom, v["launches"]),
-               "peak_source": (peak_kind if v["bound"] != "host_link" else "measured H2D copy-engine GB/s, this run"),
+               "frac": v["frac"], "traffic": ncu_traffic(dom, v["launches"]), "peak_source": v["peak_source"],
                "algorithmic_bytes_per_launch": round(v["bytes_per_launch"])}
     return out, rows
 
@@ -240,39 +256,45 @@ def roofline(prof, peaks, peak_kind, link_gbs):
 # CPU oracle timing (baseline and reference arm)
 # --------------------------------------------------------------------------
 def oracle_sample(wl, blob_of, seconds, rank=0):
-    """Run the oracle (routing + shared LRU with q* + per-token SwiGLU experts)
-    over the workload's decode calls, in trace order, until `seconds` elapse.
-    Returns (tokens, elapsed_s, calls)."""
+    """Run the C++ oracle (oracle/moe_oracle.cpp: routing, the shared LRU with
+    q*, and the per-token SwiGLU experts, one thread per token) over the
+    workload's decode calls, in trace order, until `seconds` of oracle work
+    have elapsed (the generation of expert blobs on first use is not
+    counted). Returns (tokens, elapsed_s, calls, threads): threads = the most
+    threads one call ran at once."""
     import ftgen
-    from oracle import cache as ocache
-    from oracle import formats as ofmt
-    from oracle import moe as omoe
-    bias = ftgen.zipf_log_bias(wl.E, wl.extra["zipf_s"], wl.seed("zipf"))
+    from oracle import cpp
+    bias = ftgen.zipf_log_bias(wl.E, wl.extra["zipf_s"], wl.seed("zipf")).astype(np.float64)
     wr = ftgen.router_weight(wl.E, wl.d, wl.wtype, wl.seed("router", 0)).float().numpy()
-    oc = ocache.ExpertCache(1, wl.E, wl.cache_slots, wl.bp_mbps, wl.bh_mbps)
-    tokens = calls = 0
-    t0 = time.perf_counter()
+    cache = cpp.Cache(1, wl.E, wl.cache_slots, wl.bp_mbps, wl.bh_mbps)
+    cores = os.cpu_count() or 1
+    blobs = [None] * wl.E
+    unused = np.zeros(16, np.uint8)  # stands for experts the call does not route to (never read)
+    tokens = calls = threads = 0
+    el = 0.0
     for T in wl.batches:
         for s in range(wl.steps):
             x = ftgen.hidden(T, wl.d, wl.wtype, wl.seed("bench", rank, T, s)).float().numpy()
-            ids, _, _ = omoe.route(x, wr, bias, wl.k)
-            counts, _, _, _ = omoe.permutation(ids, wl.E)
-            oc.forward(0, ocache.DECODE, counts)
-            omoe.layer_forward(x, wr, bias, wl.k, lambda e: ofmt.unpack_expert(blob_of(e), wl.d, wl.d_ff, wl.wtype))
+            t0 = time.perf_counter()
+            ids, _ = cpp.route(x, wr, bias, wl.k)
+            cache.forward(0, 0, np.bincount(ids.ravel(), minlength=wl.E))
+            el += time.perf_counter() - t0
+            for e in np.unique(ids):
+                if blobs[e] is None:
+                    blobs[e] = blob_of(int(e))
+            n = min(T, cores)
+            t0 = time.perf_counter()
+            cpp.layer_forward(x, wr, bias, wl.k, [b if b is not None else unused for b in blobs], wl.wtype, wl.d,
+                              wl.d_ff, threads=n)
+            el += time.perf_counter() - t0
             tokens += T
             calls += 1
-            if time.perf_counter() - t0 >= seconds:
-                return tokens, time.perf_counter() - t0, calls
-    return tokens, time.perf_counter() - t0, calls
-
-
-def blas_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return max(n) if n else 1
-    except Exception:
-        return 1
+            threads = max(threads, n)
+            if el >= seconds:
+                cache.close()
+                return tokens, el, calls, threads
+    cache.close()
+    return tokens, el, calls, threads
 
 
 def cpu_blob_source(wl):
@@ -305,21 +327,22 @@ def run_reference(args, wl, world, rank):
     for _ in range(args.warmup):
         oracle_sample(wl, blob, 0.5)
     tok = el = 0.0
-    calls = 0
+    calls = cores = 0
     for _ in range(args.steps):
-        t, e, c = oracle_sample(wl, blob, per_step_s)
+        t, e, c, n = oracle_sample(wl, blob, per_step_s)
         tok += t
         el += e
         calls += c
+        cores = max(cores, n)
     value = tok / el
-    cores = blas_threads()
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * el / args.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": decode_config(wl, world),
             "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": f"first {calls} decode calls of the trace in {args.steps} steps of "
-                                       f"~{per_step_s:.0f} s each (routing, shared LRU with q*, fp64 experts)"},
+                                       f"~{per_step_s:.0f} s each (C++ oracle: routing, shared LRU with q*, "
+                                       f"per-token SwiGLU experts, one thread per token)"},
             "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -385,8 +408,8 @@ def run_secondary(args, wl, world, rank, local):
         prof_big = ft.ft_moe_profile_read(h.ctx)
         ft.ft_moe_profile(h.ctx, False)
         h2d, zc = ft.ft_moe_probe_link(h.ctx, 1 << 30)
-        roof, rows = roofline(prof, peaks, peak_kind, h2d)
-        roof_big, rows_big = roofline(prof_big, peaks, peak_kind, h2d)
+        roof, rows = roofline(prof, peaks, peak_kind, h2d, zc)
+        roof_big, rows_big = roofline(prof_big, peaks, peak_kind, h2d, zc)
         flops_big = 2.0 * T_big * wl.k * 3 * wl.d * wl.d_ff
         h.close()
         link_bytes = wl.E * wl.slot_bytes
@@ -435,7 +458,7 @@ def run_secondary(args, wl, world, rank, local):
         prof = ft.ft_moe_profile_read(h.ctx)
         ft.ft_moe_profile(h.ctx, False)
         h2d, zc = ft.ft_moe_probe_link(h.ctx, 1 << 30)
-        roof, rows = roofline(prof, peaks, peak_kind, h2d)
+        roof, rows = roofline(prof, peaks, peak_kind, h2d, zc)
         h.close()
         out.update(value=round(steps / (ms / 1e3), 2), ms_per_step=round(ms / steps, 4), dtype="nvfp4",
                    config={"workload": f"{L}-layer NVFP4 decode trace, batch 1, {steps} steps, Markov p=0.8 + "
@@ -677,7 +700,7 @@ def main():
     # host link: copy engine and zero-copy kernel reads, 1 GiB
     h2d_gbs, zc_gbs = ft.ft_moe_probe_link(h.ctx, 1 << 30)
     peaks, peak_kind = load_peaks()
-    roof, rows = roofline(prof, peaks, peak_kind, h2d_gbs)
+    roof, rows = roofline(prof, peaks, peak_kind, h2d_gbs, zc_gbs)
 
     # overlap: the step against its two legs run alone, each at its bound --
     # the expert kernel on HBM-resident weights (hit class, as profiled) and
@@ -709,10 +732,10 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tok, el, calls = oracle_sample(wl, lambda e: h.blob(0, e), args.cpu_seconds, rank)
-        cpu = {"value": round(tok / el, 4), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+        tok, el, calls, n_thr = oracle_sample(wl, lambda e: h.blob(0, e), args.cpu_seconds, rank)
+        cpu = {"value": round(tok / el, 4), "unit": UNIT, "cores": n_thr, "kind": "oracle",
                "sample": f"first {calls} decode calls ({tok} tokens, batch 1 first) of the same trace and pool, "
-                         f"{el:.1f} s of CPU work"}
+                         f"{el:.1f} s of CPU work; C++ oracle, one thread per token (at most {n_thr} at once)"}
 
     h.close()
     if rank == 0:

@@ -16,6 +16,11 @@ Modules
            per-token layer forward
   cache    q* split and the shared LRU expert cache (hit / staged / streamed);
            the best static placement, for the miss-rate comparison
+  cpp      the plain C++ oracle (moe_oracle.cpp, built with the host
+           compiler): the layer per token, one std::thread per token, with
+           the roundings of the layer's fp32 definition, and the shared LRU
+           simulator; pinned against the numpy modules; the CPU baseline
+           that bench.py times
   ep       the layer with its experts split among G devices: dispatch plan,
            the all-to-all exchange, owner caches, combine at the source
   ep_compare  expert parallelism against replicas on the same trace: miss

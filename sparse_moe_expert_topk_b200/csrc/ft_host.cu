@@ -705,6 +705,14 @@ static ft_status layer_call(ft_ctx* c, int32_t layer, int32_t mode, const void* 
       // experts waits (on the device) for its own copy; else it waits for all
       const bool flags = c->write_value != nullptr && c->use_mma && n_copy <= MAX_E;
       if (flags && ++c->epoch == 0) ++c->epoch;
+      // the staged class's profile window opens with its first copy: its
+      // bytes cross the host link inside that window, whatever the GEMV's
+      // own launch time
+      cudaEvent_t stage_open = nullptr;
+      if (c->profiling) {
+        stage_open = pooled_event(c);
+        CK(cudaEventRecord(stage_open, c->s_copy));
+      }
       p = prof_begin(c, P_STAGE_COPY, c->s_copy, n_copy * (double)sh.slot_bytes);
       st = issue_copies(c, 0, n_copy, flags ? c->epoch : 0);
       prof_end(c, p, c->s_copy);
@@ -715,6 +723,14 @@ static ft_status layer_call(ft_ctx* c, int32_t layer, int32_t mode, const void* 
       else
         CK(cudaStreamWaitEvent(cs, c->ev_copy, 0));
       gemv_class(c, KIND_STAGED, layer, x, T, max_items, Tk, cs, pr_staged);
+      if (stage_open) {
+        if (pr_staged[0] >= 0 && pr_staged[1] < 0) {
+          c->evpool.push_back(c->pend[pr_staged[0]].a);
+          c->pend[pr_staged[0]].a = stage_open;
+        } else {
+          c->evpool.push_back(stage_open);
+        }
+      }
       d.landed_epoch = 0;
       gemv_class_cost(c, pr_staged, mb->n_staged_cls, mb->n_tok_cls[KIND_STAGED]);
     }

@@ -21,20 +21,27 @@ def test_roofline_classes_and_dominant_kernel():
         "gemv_hit": {"launches": 4, "ms": 0.5, "bytes": 2.0e9, "flops": 0.0},
         "gemv_streamed": {"launches": 2, "ms": 3.0, "bytes": 0.1e9, "flops": 0.0},
         "gemv_staged": {"launches": 2, "ms": 0.2, "bytes": 0.01e9, "flops": 0.0},
-        "h2d_stage_copies": {"launches": 2, "ms": 9.0, "bytes": 0.5e9, "flops": 0.0},  # not a kernel
+        "h2d_stage_copies": {"launches": 2, "ms": 9.0, "bytes": 0.45e9, "flops": 0.0},
     }
-    roof, rows = bench.roofline(prof, PEAKS, "measured", 55.0)
-    assert "h2d_stage_copies" not in rows
+    roof, rows = bench.roofline(prof, PEAKS, "measured", 55.0, 50.0)
     assert rows["gemm_tc_gateup"]["bound"] == "hbm" and rows["gemm_tc_gateup"]["unit"] == "GB/s"
     assert abs(rows["gemm_tc_gateup"]["achieved"] - 6000.0) < 0.01
     assert rows["gemm_tc_down"]["bound"] == "tensor" and abs(rows["gemm_tc_down"]["achieved"] - 1000.0) < 0.01
     assert rows["gemv_hit"]["bound"] == "hbm"
-    for k in ("gemv_streamed", "gemv_staged"):
+    # the copy engine and the staged class against the H2D copy rate, the
+    # streamed class against the zero-copy read rate
+    for k in ("gemv_staged", "h2d_stage_copies"):
         assert rows[k]["bound"] == "host_link" and rows[k]["peak"] == 55.0
-    assert abs(rows["gemv_streamed"]["frac"] - round(0.1e9 / 3.0e6 / 55.0, 4)) < 1e-4
+    assert rows["gemv_streamed"]["bound"] == "host_link" and rows["gemv_streamed"]["peak"] == 50.0
+    assert abs(rows["gemv_streamed"]["frac"] - round(0.1e9 / 3.0e6 / 50.0, 4)) < 1e-4
     assert abs(sum(v["share"] for v in rows.values()) - 1.0) < 1e-3
-    assert roof["kernel"] == "gemv_streamed" and roof["bound"] == "host_link"
-    assert roof["algorithmic_bytes_per_launch"] == round(0.1e9 / 2)
+    # the copy engine's staging takes the most time: it is the dominant row
+    assert roof["kernel"] == "h2d_stage_copies" and roof["bound"] == "host_link"
+    assert abs(roof["frac"] - round(0.45e9 / 9.0e6 / 55.0, 4)) < 1e-4
+    assert roof["algorithmic_bytes_per_launch"] == round(0.45e9 / 2)
+    # without a zero-copy figure the streamed class falls back to the H2D rate
+    _, rows2 = bench.roofline(prof, PEAKS, "measured", 55.0)
+    assert rows2["gemv_streamed"]["peak"] == 55.0
 
 
 def test_traffic_lookup_follows_the_source(tmp_path, monkeypatch):
