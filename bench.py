@@ -474,116 +474,174 @@ def run_secondary(args, wl, world, rank, local):
         print(json.dumps(out), flush=True)
     return 0
 
-def run_mixed(args, wl, world, rank, local):
-    """43-layer mixed NVFP4 workload: a cold prefill of T = 8192 tokens through
-    every layer (layer-ahead double buffer), then decode steps at batch 1, 2,
-    4 and 8 (equal blocks) with Markov routing, for every cache capacity and
-    B_P:B_H profile of the sweep. One context serves the whole sweep: the slot
-    pool is resized between capacities (the host pool is filled once)."""
+def host_mem_available():
+    """Bytes of host memory the kernel reports available (None if unknown)."""
+    try:
+        with open("/proc/meminfo") as f:
+            for line in f:
+                if line.startswith("MemAvailable:"):
+                    return int(line.split()[1]) * 1024
+    except OSError:
+        pass
+    return None
+
+
+def mixed_sweep(wl, caps, profiles, steps, warmup, rank, local):
+    """The 43-layer mixed NVFP4 workload on one context: for every cache
+    capacity and B_P:B_H profile, a cold prefill of T = 8192 tokens through
+    every layer (layer-ahead double buffer), then `steps` decode steps split
+    in equal blocks at batch 1, 2, 4 and 8 with Markov routing. The slot pool
+    is resized between capacities (the host pool is filled once). Returns
+    (rows, host_link, clocks)."""
     import dataclasses
     import ftgen
     import sparse_moe_expert_topk_b200 as ft
     from ftgen.ctx import Harness
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    peaks, peak_kind = load_peaks()
     L, E, k, d = wl.L, wl.E, wl.k, wl.d
     ex = wl.extra
-    steps = min(wl.steps, int(os.environ.get("FT_MIXED_STEPS", 256)))
     steps -= steps % len(wl.batches)
     per_batch = steps // len(wl.batches)
     Bmax = max(wl.batches)
-    caps = [int(f * L * E) for f in ex["cache_fracs"]]
     T_pf = ex["prefill_T"]
     h = Harness(dataclasses.replace(wl, cache_slots=caps[0]), max_tokens=T_pf, device=local)
-    # inputs: one prefill block reused by every layer (each layer routes it
-    # with its own router), decode activations and per-token trace biases
-    g = torch.Generator(device=device)
-    g.manual_seed(ftgen.subseed("mixed-x", rank))
-    x_pf = torch.randn(T_pf, d, generator=g, device=device).to(torch.bfloat16)
-    y_pf = torch.empty_like(x_pf)
-    x_dec = torch.randn(steps, L, Bmax, d, generator=g, device=device).to(torch.bfloat16)
-    y_dec = torch.empty(Bmax, d, dtype=torch.bfloat16, device=device)
-    zb = [ftgen.zipf_log_bias(E, ex["zipf_s"], wl.seed("pi", l)) for l in range(L)]
-    bias = np.empty((steps, L, Bmax, E), np.float32)
-    for l in range(L):
-        tr = ftgen.markov_trace(steps, Bmax, E, k, ex["p_reuse"], ex["zipf_s"], wl.seed("trace", rank, l))
-        for st in range(steps):
-            bias[st, l] = ftgen.trace_bias(tr[st], zb[l], ex["beta"])
-    bias = torch.from_numpy(bias).to(device)
-    h2d, zc = ft.ft_moe_probe_link(h.ctx, 1 << 30)
-    stream = h.stream
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-
-    def prefill():
+    try:
+        # inputs: one prefill block reused by every layer (each layer routes it
+        # with its own router), decode activations and per-token trace biases
+        g = torch.Generator(device=device)
+        g.manual_seed(ftgen.subseed("mixed-x", rank))
+        x_pf = torch.randn(T_pf, d, generator=g, device=device).to(torch.bfloat16)
+        y_pf = torch.empty_like(x_pf)
+        x_dec = torch.randn(steps, L, Bmax, d, generator=g, device=device).to(torch.bfloat16)
+        y_dec = torch.empty(Bmax, d, dtype=torch.bfloat16, device=device)
+        zb = [ftgen.zipf_log_bias(E, ex["zipf_s"], wl.seed("pi", l)) for l in range(L)]
+        bias = np.empty((steps, L, Bmax, E), np.float32)
         for l in range(L):
-            ft.ft_moe_layer_forward(h.ctx, l, ft.FT_PREFILL, x_pf, T_pf, None, 0, y_pf)
+            tr = ftgen.markov_trace(steps, Bmax, E, k, ex["p_reuse"], ex["zipf_s"], wl.seed("trace", rank, l))
+            for st in range(steps):
+                bias[st, l] = ftgen.trace_bias(tr[st], zb[l], ex["beta"])
+        bias = torch.from_numpy(bias).to(device)
+        h2d, zc = ft.ft_moe_probe_link(h.ctx, 1 << 30)
+        stream = h.stream
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
-    def decode(st0, n, B):
-        for st in range(st0, st0 + n):
+        def prefill():
             for l in range(L):
-                ft.ft_moe_layer_forward(h.ctx, l, ft.FT_DECODE, x_dec[st, l, :B], B, bias[st, l, :B], 1,
-                                        y_dec[:B])
+                ft.ft_moe_layer_forward(h.ctx, l, ft.FT_PREFILL, x_pf, T_pf, None, 0, y_pf)
 
-    def timed(fn, *a):
-        torch.cuda.synchronize(device)
-        e0.record(stream)
-        fn(*a)
-        e1.record(stream)
-        torch.cuda.synchronize(device)
-        return e0.elapsed_time(e1)
+        def decode(st0, n, B):
+            for st in range(st0, st0 + n):
+                for l in range(L):
+                    ft.ft_moe_layer_forward(h.ctx, l, ft.FT_DECODE, x_dec[st, l, :B], B, bias[st, l, :B], 1,
+                                            y_dec[:B])
 
-    # warm-up on the first point (kernels, events, pages)
-    ft.ft_set_bandwidths(h.ctx, *ex["profiles"][-1])
-    for _ in range(max(1, args.warmup - 2)):
-        ft.ft_moe_reset_cache(h.ctx)
-        prefill()
-        decode(0, min(4, per_batch), 1)
-    sweep = []
-    sampler = ClockSampler(local)
-    sampler.start()
-    for C in caps:
-        ft.ft_moe_resize_cache(h.ctx, C)
-        for bp, bh in ex["profiles"]:
+        def timed(fn, *a):
+            torch.cuda.synchronize(device)
+            e0.record(stream)
+            fn(*a)
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+            return e0.elapsed_time(e1)
+
+        # warm-up on the first point (kernels, events, pages)
+        ft.ft_set_bandwidths(h.ctx, *profiles[-1])
+        for _ in range(max(1, warmup)):
             ft.ft_moe_reset_cache(h.ctx)
-            ft.ft_set_bandwidths(h.ctx, bp, bh)
-            ms_pf = timed(prefill)
-            st_pf = h.stats()
-            row = {"cache_slots": C, "cache_frac": round(C / (L * E), 3), "bp_bh": f"{bp / 1000:.1f}:{bh / 1000:.1f}",
-                   "prefill": {"tokens_per_s": round(T_pf / (ms_pf / 1e3), 1), "ms_43_layers": round(ms_pf, 1),
-                               "link_gbs": round(st_pf["bytes_h2d"] / (ms_pf * 1e6), 2)},
-                   "decode": {}}
-            tok = 0
-            ms_dec = 0.0
-            for i, B in enumerate(wl.batches):
-                s0 = h.stats()
-                ms = timed(decode, i * per_batch, per_batch, B)
-                s1 = h.stats()
-                look = s1["lookups"] - s0["lookups"]
-                miss = s1["misses"] - s0["misses"]
-                link = (s1["bytes_h2d"] - s0["bytes_h2d"]) + (s1["bytes_zero_copy"] - s0["bytes_zero_copy"])
-                row["decode"][str(B)] = {"tokens_per_s": round(per_batch * B / (ms / 1e3), 2),
-                                         "ms_per_step": round(ms / per_batch, 3),
-                                         "miss_rate": round(miss / max(look, 1), 4),
-                                         "qstar_staged": s1["staged"] - s0["staged"],
-                                         "streamed": s1["streamed"] - s0["streamed"],
-                                         "link_gbs": round(link / (ms * 1e6), 2)}
-                tok += per_batch * B
-                ms_dec += ms
-            row["decode_tokens_per_s"] = round(tok / (ms_dec / 1e3), 2)
-            sweep.append(row)
-    clocks = sampler.stop()
-    h.close()
+            prefill()
+            decode(0, min(4, per_batch), 1)
+        sweep = []
+        sampler = ClockSampler(local)
+        sampler.start()
+        for C in caps:
+            ft.ft_moe_resize_cache(h.ctx, C)
+            for bp, bh in profiles:
+                ft.ft_moe_reset_cache(h.ctx)
+                ft.ft_set_bandwidths(h.ctx, bp, bh)
+                ms_pf = timed(prefill)
+                st_pf = h.stats()
+                pf_link = st_pf["bytes_h2d"] / (ms_pf * 1e6)
+                row = {"cache_slots": C, "cache_frac": round(C / (L * E), 3),
+                       "bp_bh": f"{bp / 1000:.1f}:{bh / 1000:.1f}",
+                       "prefill": {"tokens_per_s": round(T_pf / (ms_pf / 1e3), 1), "ms_43_layers": round(ms_pf, 1),
+                                   "link_gbs": round(pf_link, 2), "link_frac": round(pf_link / h2d, 4)},
+                       "decode": {}}
+                tok = 0
+                ms_dec = 0.0
+                s_all0 = h.stats()
+                for i, B in enumerate(wl.batches):
+                    s0 = h.stats()
+                    ms = timed(decode, i * per_batch, per_batch, B)
+                    s1 = h.stats()
+                    look = s1["lookups"] - s0["lookups"]
+                    miss = s1["misses"] - s0["misses"]
+                    link = (s1["bytes_h2d"] - s0["bytes_h2d"]) + (s1["bytes_zero_copy"] - s0["bytes_zero_copy"])
+                    row["decode"][str(B)] = {"tokens_per_s": round(per_batch * B / (ms / 1e3), 2),
+                                             "ms_per_step": round(ms / per_batch, 3),
+                                             "miss_rate": round(miss / max(look, 1), 4),
+                                             "qstar_staged": s1["staged"] - s0["staged"],
+                                             "streamed": s1["streamed"] - s0["streamed"],
+                                             "link_gbs": round(link / (ms * 1e6), 2),
+                                             "link_frac": round(link / (ms * 1e6) / h2d, 4)}
+                    tok += per_batch * B
+                    ms_dec += ms
+                s_all1 = h.stats()
+                look = s_all1["lookups"] - s_all0["lookups"]
+                row["decode_tokens_per_s"] = round(tok / (ms_dec / 1e3), 2)
+                row["decode_steps"] = steps
+                row["decode_miss_rate"] = round((s_all1["misses"] - s_all0["misses"]) / max(look, 1), 4)
+                sweep.append(row)
+        clocks = sampler.stop()
+    finally:
+        h.close()
+    return sweep, {"h2d_copy_gbs": round(h2d, 2), "zero_copy_read_gbs": round(zc, 2)}, clocks
+
+
+def mixed_point(rank, local):
+    """The largest single-GPU workload at its headline point, for the default
+    line: 43-layer mixed NVFP4 at 37% capacity and B_P:B_H = 52.7:77.3, cold
+    prefill of 8192 tokens, then the full 1024 decode steps at batch 1/2/4/8.
+    Skipped (with the reason) when the host cannot hold the 117 GB pool."""
+    import ftgen
+    wl = ftgen.workload("mixed_nvfp4")
+    need = wl.L * wl.E * wl.slot_bytes
+    avail = host_mem_available()
+    if avail is not None and avail < need + (24 << 30):
+        return {"skipped": f"host memory: {avail / 1e9:.0f} GB available, the pinned pool needs {need / 1e9:.0f} GB"}
+    t0 = time.perf_counter()
+    try:
+        rows, link, clocks = mixed_sweep(wl, [int(0.37 * wl.L * wl.E)], [(52700, 77300)], wl.steps, 1, rank, local)
+    except Exception as e:  # the default line must still be printed
+        return {"skipped": f"{type(e).__name__}: {e}"}
+    r = rows[0]
+    return {"workload": f"43-layer mixed NVFP4, E=256 top-6 d=4096 d_ff=1536 ({need / 1e9:.1f} GB pinned pool): cold "
+                        f"prefill T={wl.extra['prefill_T']} through all layers, then {r['decode_steps']} decode steps "
+                        f"at batch 1/2/4/8, Markov p=0.8 + Zipf(1.1), 37% cache ({r['cache_slots']} slots), 52.7:77.3",
+            "decode_tokens_per_s": r["decode_tokens_per_s"], "decode_miss_rate": r["decode_miss_rate"],
+            "prefill": r["prefill"], "decode": r["decode"], "host_link": link, "clocks": clocks,
+            "wall_s": round(time.perf_counter() - t0, 1)}
+
+
+def run_mixed(args, wl, world, rank, local):
+    """--workload mixed_nvfp4: the sweep over every capacity {10, 20, 37,
+    60}% x profile {11.8:47.5, 52.7:77.3} (FT_MIXED_STEPS decode steps per
+    point, default 256 of the 1024)."""
+    L, E = wl.L, wl.E
+    ex = wl.extra
+    steps = min(wl.steps, int(os.environ.get("FT_MIXED_STEPS", 256)))
+    caps = [int(f * L * E) for f in ex["cache_fracs"]]
+    sweep, link, clocks = mixed_sweep(wl, caps, list(ex["profiles"]), steps, max(1, args.warmup - 2), rank, local)
     main_pt = next(r for r in sweep if r["cache_slots"] == int(0.37 * L * E) and r["bp_bh"] == "52.7:77.3")
+    steps -= steps % len(wl.batches)
     out = {"metric": METRIC, "value": main_pt["decode_tokens_per_s"], "unit": UNIT, "n_gpus": world,
            "steps": steps, "warmup": args.warmup, "ms_per_step": round(1e3 * sum(wl.batches) / len(wl.batches)
                                                                       / main_pt["decode_tokens_per_s"], 3),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
-           "config": {"workload": f"43-layer mixed NVFP4: cold prefill T={T_pf} then {steps} decode steps at batch "
-                                  f"1/2/4/8 ({per_batch} each), Markov p=0.8 + Zipf(1.1); value at 37% and 52.7:77.3",
+           "config": {"workload": f"43-layer mixed NVFP4: cold prefill T={ex['prefill_T']} then {steps} decode steps "
+                                  f"at batch 1/2/4/8 ({steps // len(wl.batches)} each), Markov p=0.8 + Zipf(1.1); "
+                                  f"value at 37% and 52.7:77.3",
                       "pool_gb": round(L * E * wl.slot_bytes / 1e9, 1)},
-           "host_link": {"h2d_copy_gbs": round(h2d, 2), "zero_copy_read_gbs": round(zc, 2)},
-           "sweep": sweep, "clocks": clocks}
+           "host_link": link, "sweep": sweep, "clocks": clocks}
     if rank == 0:
         print(json.dumps(out), flush=True)
     return 0
@@ -600,6 +658,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-mixed", action="store_true", help="skip the 43-layer mixed NVFP4 leg of the default line")
     ap.add_argument("--profile-only", action="store_true", help="one warm-up and one profiled step (for ncu)")
     args = ap.parse_args()
     if args.warmup < 3 and not args.profile_only:
@@ -738,6 +797,13 @@ def main():
                          f"{el:.1f} s of CPU work; C++ oracle, one thread per token (at most {n_thr} at once)"}
 
     h.close()
+    del xs, ys
+    torch.cuda.empty_cache()
+    # the largest single-GPU workload (43-layer mixed NVFP4), one GPU only:
+    # each rank of a multi-GPU run would pin its own 117 GB pool
+    mixed = None
+    if world == 1 and not args.no_mixed:
+        mixed = mixed_point(rank, local)
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -758,6 +824,7 @@ def main():
             "roofline": roof, "kernels": rows, "kernels_by_batch": by_batch, "gpu_launches": int(round(launches * args.steps)),
             "gpu_launches_per_step": round(launches, 1), "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,
             "peaks": {"kind": peak_kind, "hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"]},
+            "mixed_nvfp4": mixed,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
