@@ -35,7 +35,7 @@ void prefill_tc_free(DevState& ds);
 void launch_prefill_gather(const Shape& sh, const void* x, int T, DevState& ds, cudaStream_t st);
 bool gemv_mma_supported(const Shape& sh);
 cudaError_t gemv_mma_init(int device);
-void launch_to_f16(const void* x, int n, void* y, cudaStream_t st);
+void launch_to_f16(const void* x, int T, int d, void* y, float* xscale, cudaStream_t st);
 void launch_gemv_mma(const Shape& sh, int cls, int layer, const void* x16, int T, DevState& ds, int max_items,
                      int max_tok, cudaStream_t st);
 void launch_gemm_tc(const Shape& sh, int phase, int T, DevState& ds, cudaStream_t st);
@@ -165,7 +165,7 @@ void free_all(ft_ctx* c) {
   DevState& d = c->ds;
   void* dev_ptrs[] = {d.slot_of, d.key_of, d.stamp, d.clk, d.ctr, d.error, d.work, d.scores, d.ids, d.wts,
                       d.counts, d.offsets, d.perm, d.inv, d.perm_chunks, d.hbuf, d.ybuf, d.xs, d.hs, d.tscale, d.slots,
-                      d.h16, d.h16lo, d.x16, d.sched, d.route_ctr, d.landed, d.prev_counts, c->probe_sink};
+                      d.h16, d.h16lo, d.x16, d.xscale, d.sched, d.route_ctr, d.landed, d.prev_counts, c->probe_sink};
   for (void* p : dev_ptrs)
     if (p) cudaFree(p);
   for (uint8_t* p : c->pool_host)
@@ -405,9 +405,11 @@ ft_status ft_moe_init(const ft_config* cfg, void* compute_stream, void* copy_str
   c->use_mma = gemv_mma_supported(sh);
   if (c->use_mma) {
     TRY(cuda_try(cudaMalloc((void**)&d.h16, sizeof(uint16_t) * Tk * sh.d_ff)));
-    if (sh.wtype == FT_W_BF16) TRY(cuda_try(cudaMalloc((void**)&d.h16lo, sizeof(uint16_t) * Tk * sh.d_ff)));
-    if (sh.wtype == FT_W_NVFP4)
+    TRY(cuda_try(cudaMalloc((void**)&d.h16lo, sizeof(uint16_t) * Tk * sh.d_ff)));
+    if (sh.wtype == FT_W_NVFP4) {
       TRY(cuda_try(cudaMalloc((void**)&d.x16, sizeof(uint16_t) * (size_t)cfg->max_tokens * sh.d)));
+      TRY(cuda_try(cudaMalloc((void**)&d.xscale, sizeof(float) * (size_t)cfg->max_tokens)));
+    }
     TRY(cuda_try(gemv_mma_init(cfg->device)));
   }
   d.sched_chunks = sh.E + (int)((Tk + MMA_CHUNK - 1) / MMA_CHUNK) + 1;
@@ -618,7 +620,7 @@ static ft_status layer_call(ft_ctx* c, int32_t layer, int32_t mode, const void* 
   la.bh_mbps = c->bh;
   d.pool_dev = c->pool_dev[layer];
   if (c->use_mma && sh.wtype == FT_W_NVFP4 && !(full_prefill && c->use_tc)) {
-    launch_to_f16(x, T * sh.d, d.x16, cs);
+    launch_to_f16(x, T, sh.d, d.x16, d.xscale, cs);
     c->kernel_launches += 1;
   }
   int p = -1;

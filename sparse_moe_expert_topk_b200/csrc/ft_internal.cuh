@@ -120,8 +120,9 @@ struct DevState {
   __nv_bfloat16* xs;         // [Tmax*k, d] gathered bf16 activations (prefill)
   __nv_bfloat16* hs;         // [Tmax*k, d_ff] bf16 SwiGLU activations (prefill)
   uint16_t* h16;             // [Tmax*k, d_ff] 16-bit SwiGLU activations (MMA decode path)
-  uint16_t* h16lo;           // [Tmax*k, d_ff] bf16 residual of h16 (BF16 experts)
-  uint16_t* x16;             // [Tmax, d] f16 copy of the activations (NVFP4 MMA path)
+  uint16_t* h16lo;           // [Tmax*k, d_ff] bf16 residual of h16 (BF16), f16 rest h - 2^24 h16 (NVFP4)
+  uint16_t* x16;             // [Tmax, d] f16 copy of the activations times 2^-s_t (NVFP4 MMA path)
+  float* xscale;             // [Tmax] 2^s_t of each token's f16 copy (NVFP4 MMA path)
   float* tscale;             // [L*E*3] NVFP4 tensor scales
   uint8_t* slots;            // HBM slot pool [C * slot_bytes]
   const uint8_t* pool_dev;   // device address of the called layer's blobs in the mapped host pool

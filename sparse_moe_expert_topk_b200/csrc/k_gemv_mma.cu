@@ -47,8 +47,18 @@
 // the residency.
 //
 // NVFP4: 32 e2m1 codes per lane are converted to f16 pairs (cvt e2m1x2) and
-// multiplied by their e4m3 block scale (exact in f16); the per-matrix fp32
-// tensor scale is applied to the fp32 result.
+// multiplied by their e4m3 block scale (exact in f16: at most 6 significant
+// bits, magnitudes 2^-10 .. 2688); the per-matrix fp32 tensor scale is applied
+// to the fp32 result. The activation-side f16 MMA operands stay in f16
+// range whatever the activations' magnitude: token t enters as
+// f16(x_t * 2^-s_t), the power of two bringing max|x_t| into [1, 2) (exact
+// scaling; the gate sees g = 2^s_t * sum before SwiGLU); h enters the down
+// projection as h' = h * 2^-2 s_t (h scales with x^2), stored as two f16 terms
+// h' = 2^24 hi + lo, each multiplied by W_down into its own accumulator and
+// joined in fp32, then scaled back by 2^2 s_t. So h' keeps ~22 significant
+// bits for any |h'| < 2^40; with max|x'| < 2, |h'| <= 4 |W_gate row|_1
+// |W_up row|_1, below 2^40 for any weights whose rows' absolute sums stay
+// below 2^19 (at d = 4096 that is a mean |weight| up to 128).
 #include <cuda_fp16.h>
 
 #include "ft_internal.cuh"
@@ -70,6 +80,8 @@ constexpr int CODE_RS = SLICE + 16;              // smem row stride: rows start 
 constexpr int SC_RS = SLICE / 8 + 16;            // same for the NVFP4 block scales
 constexpr int STAGE_BYTES = ROWS * CODE_RS + ROWS * SC_RS;
 constexpr int RING_BYTES = NST * STAGE_BYTES;
+constexpr float H_SPLIT = 16777216.0f;         // 2^24: h = H_SPLIT * hi + lo (NVFP4)
+constexpr float H_SPLIT_INV = 1.0f / 16777216.0f;
 
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
   uint4 r;
@@ -148,11 +160,12 @@ struct MmaArgs {
   size_t slot_bytes;
   const uint8_t* slots;
   const uint8_t* pool;
-  const void* x;        // [T, d] bf16 activations (BF16) or f16 copy (NVFP4)
+  const void* x;        // [T, d] bf16 activations (BF16) or scaled f16 copy (NVFP4)
+  const float* xscale;  // NVFP4: [T] power of two the f16 copy of token t is to be multiplied by
   const int32_t* perm;
   const float* tscale;  // [L*E*3]
   uint16_t* h16;        // [T*k, d_ff] bf16 (BF16) or f16 (NVFP4) SwiGLU output
-  uint16_t* h16lo;      // [T*k, d_ff] BF16 experts: bf16 residual h - h16
+  uint16_t* h16lo;      // [T*k, d_ff] BF16: bf16 residual h - h16; NVFP4: f16 rest h - 2^24 h16
   float* ybuf;          // [T*k, d]
   int32_t* ticket;      // this class's unit ticket counter (zeroed by the lookup)
   int32_t* done;        // this class's per-(item, chunk) phase-0 completion counters (zeroed)
@@ -182,6 +195,23 @@ __device__ __forceinline__ uint32_t lds16(uint32_t addr) {
   asm volatile("ld.shared.u16 %0, [%1];" : "=h"(r) : "r"(addr));
   return r;
 }
+// NVFP4 gate/up epilogue of one (feature, token) pair: v0, v1 are the gate
+// and up sums of the scaled f16 activations (x * 2^-s), ts0 / ts1 the tensor
+// scales, xs = 2^s. The true gate is g = v0 ts0 xs; the stored value is
+// h' = h / xs^2 = (v0 ts0) sigmoid(g) (v1 ts1), the SwiGLU output of the
+// scaled token (h scales with x^2), split into two f16 terms
+// h' = 2^24 hi + lo. Shared by both GEMV kernels, so that they agree bit for bit.
+__device__ __forceinline__ void fp4_gateup_store(float v0, float v1, float ts0, float ts1, float xs, uint16_t* hi_out,
+                                                 uint16_t* lo_out) {
+  const float gs = v0 * ts0, us = v1 * ts1;
+  const float hv = gs / (1.f + expf(-(gs * xs))) * us;
+  const __half hi = __float2half_rn(hv * H_SPLIT_INV);
+  *hi_out = __half_as_ushort(hi);
+  *lo_out = __half_as_ushort(__float2half_rn(fmaf(-__half2float(hi), H_SPLIT, hv)));
+}
+// NVFP4 down epilogue: the down sum over h' times the tensor scale and xs^2.
+__device__ __forceinline__ float fp4_down_value(float v, float ts2, float xs) { return v * (ts2 * (xs * xs)); }
+
 // Barrier among the MMA warps only (the producer warp runs on its own).
 __device__ __forceinline__ void mma_warps_sync() { asm volatile("bar.sync 1, %0;" ::"r"(NW * 32) : "memory"); }
 
@@ -193,7 +223,7 @@ __device__ __forceinline__ void mma_warps_sync() { asm volatile("bar.sync 1, %0;
 template <int NB, bool FP4, bool P1>
 __device__ __forceinline__ void stage_dot(uint32_t code, uint32_t sc, int s0, int s1, int kb,
                                           const uint16_t* const (&xr)[NB], const uint16_t* const (&xl)[NB], int g,
-                                          int q, float (&acc)[NB][4]) {
+                                          int q, float (&acc)[NB][4], float (&acc2)[NB][4]) {
   const uint32_t ra = code + g * CODE_RS + q * 16, rb = ra + 8 * CODE_RS;
   for (int s = s0; s < s1; ++s) {
     const uint4 wa = lds128(ra + s * 64), wb = lds128(rb + s * 64);
@@ -217,6 +247,20 @@ __device__ __forceinline__ void stage_dot(uint32_t code, uint32_t sc, int s0, in
 #pragma unroll
         for (int j = 0; j < 8; ++j)
           mma_f16(acc[t], ha[2 * j], hb[2 * j], ha[2 * j + 1], hb[2 * j + 1], xh[2 * j], xh[2 * j + 1]);
+        if constexpr (P1) {  // the lo term of h into its own accumulator
+          const uint16_t* lp = xl[t] + (kb + s) * 128 + q * 32;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const uint4 xv = ld_cg(lp + 8 * v);
+            xh[4 * v] = xv.x;
+            xh[4 * v + 1] = xv.y;
+            xh[4 * v + 2] = xv.z;
+            xh[4 * v + 3] = xv.w;
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            mma_f16(acc2[t], ha[2 * j], hb[2 * j], ha[2 * j + 1], hb[2 * j + 1], xh[2 * j], xh[2 * j + 1]);
+        }
       }
     } else {
       const int e0 = (kb + s) * 32 + q * 8;
@@ -443,7 +487,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_fused_kernel(MmaArgs a) {
     produce<FP4>(a, s_items, s_pref, n_items, rb0, rb1, U0, U1, ring, meta, full, empty, abort, lane);
   } else {
     const int g = lane >> 2, q = lane & 3;
-    float acc[NB][4];
+    float acc[NB][4], acc2[NB][4];
     const uint16_t* xr[NB];
     const uint16_t* xl[NB];
     int phase = 0, item = 0, chunk = 0, rb = 0, qi = 0, base = 0, nt = 0;
@@ -477,9 +521,10 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_fused_kernel(MmaArgs a) {
             xl[t] = xr[t];
           } else {
             xr[t] = a.h16 + (size_t)pos * a.d_ff;
-            xl[t] = FP4 ? xr[t] : a.h16lo + (size_t)pos * a.d_ff;
+            xl[t] = a.h16lo + (size_t)pos * a.d_ff;
           }
           acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+          acc2[t][0] = acc2[t][1] = acc2[t][2] = acc2[t][3] = 0.f;
         }
         if (phase == 1) {
           // every gate/up unit of this (item, chunk) must have published h
@@ -502,9 +547,9 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_fused_kernel(MmaArgs a) {
         const int w0 = (warp * ns) / NW, w1 = ((warp + 1) * ns) / NW;
         const uint32_t code = mb::smem_u32(ring + slot * STAGE_BYTES), scs = code + ROWS * CODE_RS;
         if (phase == 0)
-          stage_dot<NB, FP4, false>(code, scs, w0, w1, s0, xr, xl, g, q, acc);
+          stage_dot<NB, FP4, false>(code, scs, w0, w1, s0, xr, xl, g, q, acc, acc2);
         else
-          stage_dot<NB, FP4, true>(code, scs, w0, w1, s0, xr, xl, g, q, acc);
+          stage_dot<NB, FP4, true>(code, scs, w0, w1, s0, xr, xl, g, q, acc, acc2);
       }
       __syncwarp();
       if (lane == 0) mb::arrive(empty + 8 * slot);  // this warp is done with the stage
@@ -512,7 +557,14 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_fused_kernel(MmaArgs a) {
 
       // end of the unit: split-K reduction over the warps in warp order, one
       // output pair per thread: thread o < NB*64 takes token tile t, element
-      // pair c (rows g and g+8 of lane l's fragment)
+      // pair c (rows g and g+8 of lane l's fragment). NVFP4 down units first
+      // join the two terms of h in each warp.
+      if (FP4 && phase == 1) {
+#pragma unroll
+        for (int t = 0; t < NB; ++t)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[t][c] = fmaf(acc[t][c], H_SPLIT, acc2[t][c]);
+      }
 #pragma unroll
       for (int t = 0; t < NB; ++t)
 #pragma unroll
@@ -530,17 +582,22 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_fused_kernel(MmaArgs a) {
         // row lg (gate / first down row) and lg+8 (up / second down row), token 2 lq + c of tile t
         const int j = t * 8 + 2 * lq + c;
         if (j < nt) {
+          float ts0 = 1.f, ts1 = 1.f, ts2 = 1.f, xs = 1.f;
           if constexpr (FP4) {
             const float* ts = a.tscale + ((size_t)a.layer * a.E + s_items[item].e) * 3;
-            v0 *= phase == 0 ? ts[0] : ts[2];
-            v1 *= phase == 0 ? ts[1] : ts[2];
+            ts0 = ts[0], ts1 = ts[1], ts2 = ts[2];
+            xs = a.xscale[a.perm[base + j] / a.k];
+            if (phase == 1) {
+              v0 = fp4_down_value(v0, ts2, xs);
+              v1 = fp4_down_value(v1, ts2, xs);
+            }
           }
           if (phase == 0) {
-            const float hv = v0 / (1.f + expf(-v0)) * v1;
             const size_t o = (size_t)(base + j) * a.d_ff + rb * 8 + lg;
             if constexpr (FP4) {
-              a.h16[o] = __half_as_ushort(__float2half_rn(hv));
+              fp4_gateup_store(v0, v1, ts0, ts1, xs, a.h16 + o, a.h16lo + o);
             } else {
+              const float hv = v0 / (1.f + expf(-v0)) * v1;
               const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
               a.h16[o] = __bfloat16_as_ushort(hi);
               a.h16lo[o] = __bfloat16_as_ushort(__float2bfloat16_rn(hv - __bfloat162float(hi)));
@@ -645,7 +702,8 @@ __device__ __forceinline__ void dot_bf16_slices(const uint8_t* ra, const uint8_t
 template <int NB, int RT, bool P1>
 __device__ __forceinline__ void dot_nvfp4(const uint8_t* ra, const uint8_t* rb, const unsigned short* sa,
                                           const unsigned short* sb, size_t tstride, size_t tsc, int s0, int s1,
-                                          const uint16_t* const (&xr)[NB], int q, float (&acc)[RT][NB][4]) {
+                                          const uint16_t* const (&xr)[NB], const uint16_t* const (&xl)[NB], int q,
+                                          float (&acc)[RT][NB][4], float (&acc2)[P1 ? RT : 1][NB][4]) {
   for (int s = s0; s < s1; ++s) {
     uint4 wa[RT], wb[RT];
     uint32_t ca[RT], cb[RT];
@@ -669,16 +727,37 @@ __device__ __forceinline__ void dot_nvfp4(const uint8_t* ra, const uint8_t* rb, 
         xh[t][4 * v + 3] = xv.w;
       }
     }
+    uint32_t xo[P1 ? NB : 1][16];  // the lo term of h (down units)
+    if constexpr (P1) {
+#pragma unroll
+      for (int t = 0; t < NB; ++t) {
+        const uint16_t* xp = xl[t] + s * 128 + q * 32;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint4 xv = ld_cg(xp + 8 * v);
+          xo[t][4 * v] = xv.x;
+          xo[t][4 * v + 1] = xv.y;
+          xo[t][4 * v + 2] = xv.z;
+          xo[t][4 * v + 3] = xv.w;
+        }
+      }
+    }
 #pragma unroll
     for (int r = 0; r < RT; ++r) {
       uint32_t ha[16], hb[16];
       decode_nvfp4(wa[r], ca[r], ha);
       decode_nvfp4(wb[r], cb[r], hb);
 #pragma unroll
-      for (int t = 0; t < NB; ++t)
+      for (int t = 0; t < NB; ++t) {
 #pragma unroll
         for (int j = 0; j < 8; ++j)
           mma_f16(acc[r][t], ha[2 * j], hb[2 * j], ha[2 * j + 1], hb[2 * j + 1], xh[t][2 * j], xh[t][2 * j + 1]);
+        if constexpr (P1) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            mma_f16(acc2[r][t], ha[2 * j], hb[2 * j], ha[2 * j + 1], hb[2 * j + 1], xo[t][2 * j], xo[t][2 * j + 1]);
+        }
+      }
     }
   }
 }
@@ -733,14 +812,19 @@ __device__ void direct_unit(const MmaArgs& a, const WorkItem& it, int chunk, int
       xl[t] = xr[t];
     } else {
       xr[t] = a.h16 + (size_t)pos * a.d_ff;
-      xl[t] = FP4 ? xr[t] : a.h16lo + (size_t)pos * a.d_ff;
+      xl[t] = a.h16lo + (size_t)pos * a.d_ff;
     }
   }
   float acc[RT][NB][4];
+  float acc2[FP4 && PHASE == 1 ? RT : 1][NB][4];  // NVFP4 down units: the lo term of h
 #pragma unroll
   for (int r = 0; r < RT; ++r)
 #pragma unroll
     for (int t = 0; t < NB; ++t) acc[r][t][0] = acc[r][t][1] = acc[r][t][2] = acc[r][t][3] = 0.f;
+#pragma unroll
+  for (int r = 0; r < (FP4 && PHASE == 1 ? RT : 1); ++r)
+#pragma unroll
+    for (int t = 0; t < NB; ++t) acc2[r][t][0] = acc2[r][t][1] = acc2[r][t][2] = acc2[r][t][3] = 0.f;
   // The K steps this warp covers are the TMA-ring kernel's: for each ring
   // slice j in order, sub-range w of NW = 8. With the same MMA order inside a
   // warp and the same warp-order reduction, an expert's output is bit-identical
@@ -751,11 +835,26 @@ __device__ void direct_unit(const MmaArgs& a, const WorkItem& it, int chunk, int
     for (int j = 0; j < gg.nsl; ++j) {
       const int b0 = j * gg.ss, ns = min(gg.ss, gg.steps - b0);
       const int s0 = b0 + (warp * ns) / NW, s1 = b0 + ((warp + 1) * ns) / NW;
-      dot_nvfp4<NB, RT, PHASE == 1>(blob + oa + q * 16, blob + ob + q * 16,
-                                    reinterpret_cast<const unsigned short*>(blob + sa0) + q,
-                                    reinterpret_cast<const unsigned short*>(blob + sb0) + q,
-                                    (size_t)rows_per_tile * rbytes, (size_t)rows_per_tile * sbytes / 2, s0, s1, xr, q,
-                                    acc);
+      if constexpr (PHASE == 1)
+        dot_nvfp4<NB, RT, true>(blob + oa + q * 16, blob + ob + q * 16,
+                                reinterpret_cast<const unsigned short*>(blob + sa0) + q,
+                                reinterpret_cast<const unsigned short*>(blob + sb0) + q,
+                                (size_t)rows_per_tile * rbytes, (size_t)rows_per_tile * sbytes / 2, s0, s1, xr, xl, q,
+                                acc, acc2);
+      else
+        dot_nvfp4<NB, RT, false>(blob + oa + q * 16, blob + ob + q * 16,
+                                 reinterpret_cast<const unsigned short*>(blob + sa0) + q,
+                                 reinterpret_cast<const unsigned short*>(blob + sb0) + q,
+                                 (size_t)rows_per_tile * rbytes, (size_t)rows_per_tile * sbytes / 2, s0, s1, xr, xl,
+                                 q, acc, acc2);
+    }
+    if constexpr (PHASE == 1) {  // join the two terms of h in each warp, as the ring kernel does
+#pragma unroll
+      for (int r = 0; r < RT; ++r)
+#pragma unroll
+        for (int t = 0; t < NB; ++t)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[r][t][c] = fmaf(acc[r][t][c], H_SPLIT, acc2[r][t][c]);
     }
   } else if constexpr (NB == 1) {
     // up to 8 tokens: a warp's steps gathered across slices, 8 loads in flight
@@ -804,13 +903,20 @@ __device__ void direct_unit(const MmaArgs& a, const WorkItem& it, int chunk, int
       for (int c = 0; c < 2; ++c) {
         const int j = t * 8 + 2 * q + c;
         if (j >= nt) continue;
-        const float v0 = v[t][c] * t0, v1 = v[t][2 + c] * t1;
+        float v0 = v[t][c], v1 = v[t][2 + c], xs = 1.f;
+        if constexpr (FP4) {
+          xs = a.xscale[a.perm[base + j] / a.k];
+          if (PHASE == 1) {
+            v0 = fp4_down_value(v0, t0, xs);
+            v1 = fp4_down_value(v1, t1, xs);
+          }
+        }
         if (PHASE == 0) {
-          const float hv = v0 / (1.f + expf(-v0)) * v1;
           const size_t o = (size_t)(base + j) * a.d_ff + blk * 8 + g;
           if constexpr (FP4) {
-            a.h16[o] = __half_as_ushort(__float2half_rn(hv));
+            fp4_gateup_store(v0, v1, t0, t1, xs, a.h16 + o, a.h16lo + o);
           } else {
+            const float hv = v0 / (1.f + expf(-v0)) * v1;
             const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
             a.h16[o] = __bfloat16_as_ushort(hi);
             a.h16lo[o] = __bfloat16_as_ushort(__float2bfloat16_rn(hv - __bfloat162float(hi)));
@@ -832,10 +938,16 @@ __device__ void direct_unit(const MmaArgs& a, const WorkItem& it, int chunk, int
 // reduction and barriers amortised.
 template <bool FP4>
 constexpr int tiles_for() { return FP4 ? 4 : 1; }
+// NVFP4 down units carry two accumulators (the two terms of h), so they take
+// two row tiles, which keeps the kernel's registers where four gate/up tiles
+// put them (a unit's row tiles change which rows it covers, not the K order
+// of any row, so results do not depend on this choice).
+template <bool FP4>
+constexpr int tiles_down_for() { return FP4 ? 2 : 1; }
 
 template <int NB, bool FP4, int NW>
 __global__ void __launch_bounds__(NW * 32) gemv_direct_kernel(MmaArgs a) {
-  constexpr int RT = tiles_for<FP4>();
+  constexpr int RT = tiles_for<FP4>(), RT1 = tiles_down_for<FP4>();
   __shared__ int s_pref[MAX_E + 1];
   __shared__ WorkItem s_items[MAX_E];
   __shared__ float red[NW * RT * NB * 4 * 32];
@@ -863,7 +975,7 @@ __global__ void __launch_bounds__(NW * 32) gemv_direct_kernel(MmaArgs a) {
   }
   __syncthreads();
   const int n_qi = s_pref[n_items];
-  const int rb0 = a.d_ff / 8 / RT, rb1 = a.d / 16 / RT;
+  const int rb0 = a.d_ff / 8 / RT, rb1 = a.d / 16 / RT1;
   const int U0 = n_qi * rb0, U1 = n_qi * rb1;
   if (tid == 0) s_unit = atomicAdd(a.ticket, 1);
   __syncthreads();
@@ -893,7 +1005,7 @@ __global__ void __launch_bounds__(NW * 32) gemv_direct_kernel(MmaArgs a) {
         __threadfence();
       }
       __syncthreads();
-      if (!bad) direct_unit<NB, 1, FP4, NW, RT>(a, it, chunk, rb, warp, lane, red);
+      if (!bad) direct_unit<NB, 1, FP4, NW, RT1>(a, it, chunk, rb, warp, lane, red);
     } else {
       if (!bad) direct_unit<NB, 0, FP4, NW, RT>(a, it, chunk, rb, warp, lane, red);
       if (tid == 0) atomicAdd(a.done + qi, 1);
@@ -904,9 +1016,36 @@ __global__ void __launch_bounds__(NW * 32) gemv_direct_kernel(MmaArgs a) {
   }
 }
 
-// bf16 -> f16 copy of the activations (NVFP4 experts take f16 MMA operands).
-__global__ void __launch_bounds__(256) to_f16_kernel(const __nv_bfloat16* __restrict__ x, int n, __half* __restrict__ y) {
-  for (int i = blockIdx.x * 256 + threadIdx.x; i < n; i += gridDim.x * 256) y[i] = __float2half_rn(__bfloat162float(x[i]));
+// f16 copy of the bf16 activations for the NVFP4 experts' f16 MMAs, one CTA
+// per token: y[t] = f16(x[t] * 2^-s_t) and xscale[t] = 2^s_t, where the power
+// of two s_t brings max_i |x[t, i]| into [1, 2) (bf16 carries 8 significant
+// bits, so every element down to 2^-14 of the largest is exact in f16; the
+// smaller ones, below 2^-14 of the largest, keep an absolute error under
+// 2^-25 of it). A token of zeros keeps s_t = 0; s_t is held to [-60, 60], so
+// that xscale^2 is an fp32 power of two; non-finite values pass through.
+__global__ void __launch_bounds__(256) to_f16_scaled_kernel(const __nv_bfloat16* __restrict__ x, int d,
+                                                            __half* __restrict__ y, float* __restrict__ xscale) {
+  __shared__ float s_max[8];
+  const int t = blockIdx.x;
+  const __nv_bfloat16* xr = x + (size_t)t * d;
+  float m = 0.f;
+  for (int i = threadIdx.x; i < d; i += 256) m = fmaxf(m, fabsf(__bfloat162float(xr[i])));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) s_max[threadIdx.x >> 5] = m;
+  __syncthreads();
+  m = s_max[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) m = fmaxf(m, s_max[w]);
+  int sh = 0;
+  if (m > 0.f && m <= 3.0e38f) {
+    int e;
+    frexpf(m, &e);  // m = f * 2^e, f in [0.5, 1)
+    sh = min(60, max(-60, e - 1));
+  }
+  const float down = ldexpf(1.f, -sh);
+  for (int i = threadIdx.x; i < d; i += 256) y[(size_t)t * d + i] = __float2half_rn(__bfloat162float(xr[i]) * down);
+  if (threadIdx.x == 0) xscale[t] = ldexpf(1.f, sh);
 }
 
 int g_grid[2][3] = {{0, 0, 0}, {0, 0, 0}};  // [fp4][NB]: resident CTAs (one per SM)
@@ -973,9 +1112,8 @@ cudaError_t gemv_mma_init(int device) {
   return e;
 }
 
-void launch_to_f16(const void* x, int n, void* y, cudaStream_t st) {
-  const int grid = (n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184;
-  to_f16_kernel<<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, n, (__half*)y);
+void launch_to_f16(const void* x, int T, int d, void* y, float* xscale, cudaStream_t st) {
+  to_f16_scaled_kernel<<<T, 256, 0, st>>>((const __nv_bfloat16*)x, d, (__half*)y, xscale);
 }
 
 // Both phases of one work class in one launch.
@@ -994,6 +1132,7 @@ void launch_gemv_mma(const Shape& sh, int cls, int layer, const void* x16, int T
   a.slots = ds.slots;
   a.pool = ds.pool_dev;
   a.x = x16;
+  a.xscale = ds.xscale;
   a.perm = ds.perm;
   a.tscale = ds.tscale;
   a.h16 = ds.h16;
@@ -1008,7 +1147,8 @@ void launch_gemv_mma(const Shape& sh, int cls, int layer, const void* x16, int T
   const int NB = T > 8 ? 2 : 1;
   const long long chunks = (long long)max_items + (long long)max_tok / CHUNK;
   if (cls == KIND_HIT) {
-    const long long units = chunks * (sh.d_ff / 8 + sh.d / 16) / (fp4 ? tiles_for<true>() : 1);
+    const long long units =
+        chunks * (sh.d_ff / 8 / (fp4 ? tiles_for<true>() : 1) + sh.d / 16 / (fp4 ? tiles_down_for<true>() : 1));
     const int cap = g_grid_direct[fp4][NB];
     const int grid = (int)(units < cap ? units : cap);
     if (grid <= 0) return;

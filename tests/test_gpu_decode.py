@@ -184,3 +184,28 @@ def test_error_paths(cuda_ok):
         with pytest.raises(ft.FtError):
             ft.ft_set_bandwidths(h.ctx, 1, 0)
         assert h.stats()["device_error"] == 0
+
+
+@pytest.mark.parametrize("scale", [2.0 ** 15, 1.0, 2.0 ** -20])
+def test_nvfp4_activation_range(cuda_ok, scale):
+    """NVFP4 experts run f16 tensor-core MMAs; activations of any magnitude
+    must come through: x * 2^15 makes |h| ~ 1e9, far above the f16 maximum
+    65504, and x * 2^-20 makes |h| ~ 1e-12, below the smallest f16 subnormal
+    (powers of two, so the bf16 inputs keep the top-k gap exactly).
+    Decode at batch 1..5 through all three classes (hit, staged, streamed) on
+    a small cache; routing bit-exact and outputs within 4e-2 rms of the
+    oracle."""
+    wl = ftgen.Workload("nvfp4_range", L=1, E=16, k=4, d=1024, d_ff=512, wtype=ftgen.W_NVFP4, cache_slots=6,
+                        bp_mbps=52700, bh_mbps=77300)
+    with _harness(wl, max_tokens=5) as h:
+        oc = oracle_cache(h)
+        W = ExpertWeights(h, keep=16)
+        for step in range(8):
+            T = 1 + step % 5
+            x = gap_hidden(wl, T, wl.seed("range", step), h.routers[0], None)
+            x = (x.float() * scale).to(torch.bfloat16)
+            y, _ = _run_and_check(h, oc, W, 0, x, None)
+            assert torch.isfinite(y.float()).all()
+        _check_cache_state(h, oc)
+        st = h.stats()
+        assert st["hits"] > 0 and st["staged"] > 0 and st["streamed"] > 0
