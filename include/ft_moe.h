@@ -164,6 +164,20 @@ ft_status ft_moe_layer_forward(ft_ctx* ctx, int32_t layer, int32_t mode, const v
                                const float* bias_dev, int32_t bias_per_token, void* y_dev,
                                int32_t* ids_dev_opt, float* w_dev_opt);
 
+/* ft_moe_layer_forward with the activations in host memory: x_host [T][d]
+ * is copied into a device buffer the context owns, the layer runs, and its
+ * output is copied back into y_host [T][d], all enqueued on the compute
+ * stream in that order (the call returns once the work is enqueued; in
+ * decode mode it also waits for the layer's lookup as ft_moe_layer_forward
+ * does). Page-locked host buffers make both copies asynchronous; pageable
+ * ones make the runtime copy through its own staging. The caller reads y_host
+ * after synchronising the compute stream, and keeps x_host unchanged until
+ * then. Types, sizes and the other arguments as ft_moe_layer_forward (bias
+ * stays a device pointer: it is model data); x_host and y_host may not
+ * overlap. T <= max_tokens. */
+ft_status ft_moe_layer_forward_host(ft_ctx* ctx, int32_t layer, int32_t mode, const void* x_host, int32_t T,
+                                    const float* bias_dev, int32_t bias_per_token, void* y_host);
+
 /* Expert outputs of rows that are already routed: the owner's half of an
  * expert-parallel layer, where G devices split the E experts of every layer
  * in G contiguous blocks and each device runs only the experts it owns on the

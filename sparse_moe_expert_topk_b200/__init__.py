@@ -26,7 +26,7 @@ KIND_HIT, KIND_STAGED, KIND_STREAMED = 0, 1, 2
 # Every symbol include/ft_moe.h declares.
 EXPORTS = (
     "ft_moe_slot_bytes", "ft_moe_init", "ft_moe_destroy", "ft_moe_expert_ptr", "ft_moe_set_tensor_scales",
-    "ft_moe_set_router", "ft_moe_layer_forward", "ft_cache_stats", "ft_set_bandwidths", "ft_moe_reset_cache",
+    "ft_moe_set_router", "ft_moe_layer_forward", "ft_moe_layer_forward_host", "ft_cache_stats", "ft_set_bandwidths", "ft_moe_reset_cache",
     "ft_moe_resize_cache", "ft_moe_set_prefetch", "ft_moe_last_route", "ft_moe_cache_contents", "ft_moe_probe_link", "ft_moe_profile", "ft_moe_profile_read",
     "ft_route_topk_static", "ft_moe_expert_rows", "ft_ep_pack_scratch_bytes", "ft_ep_pack", "ft_ep_combine",
     "ft_status_str",
@@ -82,6 +82,7 @@ def lib() -> ctypes.CDLL:
             "ft_moe_set_tensor_scales": [P, I32, I32, pF],
             "ft_moe_set_router": [P, I32, P],
             "ft_moe_layer_forward": [P, I32, I32, P, I32, P, I32, P, P, P],
+            "ft_moe_layer_forward_host": [P, I32, I32, P, I32, P, I32, P],
             "ft_cache_stats": [P, ctypes.POINTER(FtStats)],
             "ft_set_bandwidths": [P, U32, U32],
             "ft_moe_reset_cache": [P],
@@ -172,6 +173,14 @@ def ft_moe_layer_forward(ctx, layer, mode, x, T, bias, bias_per_token, y, ids=No
     _check("ft_moe_layer_forward",
            lib().ft_moe_layer_forward(ctx, layer, mode, _ptr(x), T, _ptr(bias), bias_per_token, _ptr(y),
                                       _ptr(ids), _ptr(w)))
+
+
+def ft_moe_layer_forward_host(ctx, layer, mode, x_host, T, bias, bias_per_token, y_host):
+    """The layer on host tensors (pinned for asynchronous copies): x_host in,
+    y_host out, both copied by the library on the compute stream."""
+    _check("ft_moe_layer_forward_host",
+           lib().ft_moe_layer_forward_host(ctx, layer, mode, _ptr(x_host), T, _ptr(bias), bias_per_token,
+                                           _ptr(y_host)))
 
 
 def ft_cache_stats(ctx) -> dict:

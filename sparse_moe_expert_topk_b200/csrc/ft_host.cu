@@ -165,7 +165,7 @@ void free_all(ft_ctx* c) {
   DevState& d = c->ds;
   void* dev_ptrs[] = {d.slot_of, d.key_of, d.stamp, d.clk, d.ctr, d.error, d.work, d.scores, d.ids, d.wts,
                       d.counts, d.offsets, d.perm, d.inv, d.perm_chunks, d.hbuf, d.ybuf, d.xs, d.hs, d.tscale, d.slots,
-                      d.h16, d.h16lo, d.x16, d.xscale, d.sched, d.route_ctr, d.landed, d.prev_counts, c->probe_sink};
+                      d.h16, d.h16lo, d.x16, d.xscale, d.xin, d.yout, d.sched, d.route_ctr, d.landed, d.prev_counts, c->probe_sink};
   for (void* p : dev_ptrs)
     if (p) cudaFree(p);
   for (uint8_t* p : c->pool_host)
@@ -401,6 +401,11 @@ ft_status ft_moe_init(const ft_config* cfg, void* compute_stream, void* copy_str
   TRY(cuda_try(cudaMalloc((void**)&d.hbuf, sizeof(float) * Tk * sh.d_ff)));
   TRY(cuda_try(cudaMalloc((void**)&d.ybuf, sizeof(float) * Tk * sh.d)));
   TRY(cuda_try(cudaMalloc((void**)&d.tscale, sizeof(float) * sh.L * sh.E * 3)));
+  {
+    const size_t act = (size_t)cfg->max_tokens * sh.d * (sh.wtype == FT_W_F32 ? 4 : 2);
+    TRY(cuda_try(cudaMalloc(&d.xin, act)));
+    TRY(cuda_try(cudaMalloc(&d.yout, act)));
+  }
   TRY(cuda_try(cudaMalloc((void**)&c->probe_sink, sizeof(unsigned long long))));
   c->use_mma = gemv_mma_supported(sh);
   if (c->use_mma) {
@@ -853,6 +858,24 @@ ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, int32_t mode, const voi
                                int32_t bias_per_token, void* y, int32_t* ids_opt, float* w_opt) {
   if (!c) return FT_EINVAL;
   return layer_call(c, layer, mode, x, T, bias, bias_per_token, y, ids_opt, w_opt, nullptr, 0);
+}
+
+ft_status ft_moe_layer_forward_host(ft_ctx* c, int32_t layer, int32_t mode, const void* x_host, int32_t T,
+                                    const float* bias, int32_t bias_per_token, void* y_host) {
+  if (!c) return FT_EINVAL;
+  if (T < 0 || T > c->cfg.max_tokens) return FT_EINVAL;
+  if (c->latched != FT_OK) return c->latched;
+  if (T == 0) return FT_OK;
+  if (!x_host || !y_host) return FT_EINVAL;
+  const size_t bytes = (size_t)T * c->sh.d * (c->sh.wtype == FT_W_F32 ? 4 : 2);
+  const uintptr_t xa = (uintptr_t)x_host, ya = (uintptr_t)y_host;
+  if (xa < ya + bytes && ya < xa + bytes) return FT_EINVAL;  // overlapping host buffers
+  CK(cudaMemcpyAsync(c->ds.xin, x_host, bytes, cudaMemcpyHostToDevice, c->s_comp));
+  const ft_status st = layer_call(c, layer, mode, c->ds.xin, T, bias, bias_per_token, c->ds.yout, nullptr, nullptr,
+                                  nullptr, 0);
+  if (st != FT_OK) return st;
+  CK(cudaMemcpyAsync(y_host, c->ds.yout, bytes, cudaMemcpyDeviceToHost, c->s_comp));
+  return FT_OK;
 }
 
 ft_status ft_moe_expert_rows(ft_ctx* c, int32_t layer, int32_t mode, const void* rows, const int32_t* eids,

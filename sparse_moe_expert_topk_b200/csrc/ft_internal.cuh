@@ -124,6 +124,8 @@ struct DevState {
   uint16_t* x16;             // [Tmax, d] f16 copy of the activations times 2^-s_t (NVFP4 MMA path)
   float* xscale;             // [Tmax] 2^s_t of each token's f16 copy (NVFP4 MMA path)
   float* tscale;             // [L*E*3] NVFP4 tensor scales
+  void* xin;                 // [Tmax, d] activations copied in from host memory (ft_moe_layer_forward_host)
+  void* yout;                // [Tmax, d] output copied back to host memory
   uint8_t* slots;            // HBM slot pool [C * slot_bytes]
   const uint8_t* pool_dev;   // device address of the called layer's blobs in the mapped host pool
   void* tc_plan;             // host: tensor maps of the prefill GEMM (owned, see prefill_tc_free)

@@ -67,6 +67,7 @@ def test_null_arguments_are_rejected(lib):
     assert lib.ft_set_bandwidths(None, 1, 1) == ft.FT_EINVAL
     assert lib.ft_cache_stats(None, None) == ft.FT_EINVAL
     assert lib.ft_moe_layer_forward(None, 0, 0, None, 0, None, 0, None, None, None) == ft.FT_EINVAL
+    assert lib.ft_moe_layer_forward_host(None, 0, 0, None, 0, None, 0, None) == ft.FT_EINVAL
     assert lib.ft_moe_expert_rows(None, 0, 0, None, None, 0, 0, None) == ft.FT_EINVAL
     lib.ft_moe_destroy(None)
 

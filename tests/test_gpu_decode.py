@@ -209,3 +209,29 @@ def test_nvfp4_activation_range(cuda_ok, scale):
         _check_cache_state(h, oc)
         st = h.stats()
         assert st["hits"] > 0 and st["staged"] > 0 and st["streamed"] > 0
+
+
+def test_host_buffer_call_matches_device_call(cuda_ok):
+    """ft_moe_layer_forward_host (host x and y, copied by the library on the
+    compute stream) gives the device-pointer call's output bytes, from pinned
+    and from pageable host memory, and the same cache record."""
+    import dataclasses
+    wl = dataclasses.replace(ftgen.workload("decode_bf16"), name="host_call", E=64, cache_slots=24)
+    bias = ftgen.zipf_log_bias(wl.E, 1.1, wl.seed("zipf"))
+    with _harness(wl, max_tokens=16) as a, _harness(wl, max_tokens=16) as b:
+        bd = torch.as_tensor(bias).to(a.dev)
+        for step, T in enumerate((1, 4, 16, 3)):
+            x = gap_hidden(wl, T, wl.seed("host", step), a.routers[0], bias)
+            y_dev = a.forward(0, x.to(a.dev), bd)
+            xh = x.pin_memory() if step % 2 == 0 else x.clone()
+            yh = torch.empty_like(x)
+            yh = yh.pin_memory() if step % 2 == 0 else yh
+            ft.ft_moe_layer_forward_host(b.ctx, 0, ft.FT_DECODE, xh, T, bd, 0, yh)
+            torch.cuda.synchronize()
+            assert torch.equal(y_dev.cpu().view(torch.int16), yh.view(torch.int16)), step
+        sa, sb = a.stats(), b.stats()
+        for k in ("lookups", "hits", "misses", "staged", "streamed"):
+            assert sa[k] == sb[k], k
+        with pytest.raises(ft.FtError):
+            x = torch.zeros(17, wl.d, dtype=torch.bfloat16)
+            ft.ft_moe_layer_forward_host(b.ctx, 0, ft.FT_DECODE, x, 17, None, 0, torch.empty_like(x))
