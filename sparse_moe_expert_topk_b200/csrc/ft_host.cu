@@ -38,7 +38,7 @@ cudaError_t gemv_mma_init(int device);
 void launch_to_f16(const void* x, int T, int d, void* y, float* xscale, cudaStream_t st);
 void launch_gemv_mma(const Shape& sh, int cls, int layer, const void* x16, int T, DevState& ds, int max_items,
                      int max_tok, cudaStream_t st);
-void launch_gemm_tc(const Shape& sh, int phase, int T, DevState& ds, cudaStream_t st);
+void launch_gemm_tc(const Shape& sh, int phase, int layer, int T, DevState& ds, cudaStream_t st);
 void launch_rows_in(const int32_t* eids, int n, int base, int E, DevState& ds, cudaStream_t st);
 void launch_combine_rows(const float* ybuf, const float* wts, const int32_t* inv, int T, int k, int d, bool out_f32,
                          void* y, cudaStream_t st);
@@ -164,7 +164,7 @@ void free_all(ft_ctx* c) {
   if (c->s_comp || c->s_side) cudaDeviceSynchronize();
   DevState& d = c->ds;
   void* dev_ptrs[] = {d.slot_of, d.key_of, d.stamp, d.clk, d.ctr, d.error, d.work, d.scores, d.ids, d.wts,
-                      d.counts, d.offsets, d.perm, d.inv, d.perm_chunks, d.hbuf, d.ybuf, d.xs, d.hs, d.tscale, d.slots,
+                      d.counts, d.offsets, d.perm, d.inv, d.perm_chunks, d.hbuf, d.ybuf, d.xs, d.hs, d.hs_lo, d.tscale, d.slots,
                       d.h16, d.h16lo, d.x16, d.xscale, d.xin, d.yout, d.sched, d.route_ctr, d.landed, d.prev_counts, c->probe_sink};
   for (void* p : dev_ptrs)
     if (p) cudaFree(p);
@@ -445,6 +445,7 @@ ft_status ft_moe_init(const ft_config* cfg, void* compute_stream, void* copy_str
   if (c->use_tc) {
     TRY(cuda_try(cudaMalloc((void**)&d.xs, sizeof(__nv_bfloat16) * (Tk + 256) * sh.d)));
     TRY(cuda_try(cudaMalloc((void**)&d.hs, sizeof(__nv_bfloat16) * (Tk + 256) * sh.d_ff)));
+    TRY(cuda_try(cudaMalloc((void**)&d.hs_lo, sizeof(__nv_bfloat16) * (Tk + 256) * sh.d_ff)));
     TRY(cuda_try(prefill_tc_init(sh, d, (int)Tk)));
   }
   d.pool_dev = nullptr;
@@ -825,13 +826,14 @@ static ft_status layer_call(ft_ctx* c, int32_t layer, int32_t mode, const void* 
       p = prof_begin(c, P_GATHER, cs, Tk * (double)sh.d * 2.0 + T * (double)sh.d * ab);
       launch_prefill_gather(sh, x, T, d, cs);
       prof_end(c, p, cs);
-      p = prof_begin(c, P_GEMM_GU, cs, n_it * 2.0 * dd * 2.0 + Tk * (double)sh.d * 2.0 + Tk * (double)sh.d_ff * 2.0,
+      const double wb = weight_bytes_per_elem(sh.wtype);
+      p = prof_begin(c, P_GEMM_GU, cs, n_it * 2.0 * dd * wb + Tk * (double)sh.d * 2.0 + Tk * (double)sh.d_ff * 2.0,
                      2.0 * Tk * 2.0 * dd);
-      launch_gemm_tc(sh, 0, T, d, cs);
+      launch_gemm_tc(sh, 0, layer, T, d, cs);
       prof_end(c, p, cs);
-      p = prof_begin(c, P_GEMM_DN, cs, n_it * dd * 2.0 + Tk * (double)sh.d_ff * 2.0 + Tk * (double)sh.d * 4.0,
+      p = prof_begin(c, P_GEMM_DN, cs, n_it * dd * wb + Tk * (double)sh.d_ff * 2.0 + Tk * (double)sh.d * 4.0,
                      2.0 * Tk * dd);
-      launch_gemm_tc(sh, 1, T, d, cs);
+      launch_gemm_tc(sh, 1, layer, T, d, cs);
       prof_end(c, p, cs);
       c->kernel_launches += 3;
     } else {
@@ -1018,10 +1020,10 @@ ft_status ft_moe_resize_cache(ft_ctx* c, int64_t new_slots) {
   uint8_t* nslots = nullptr;
   int32_t* nk = nullptr;
   unsigned long long* ns = nullptr;
-  __nv_bfloat16 *nxs = nullptr, *nhs = nullptr;
+  __nv_bfloat16 *nxs = nullptr, *nhs = nullptr, *nhl = nullptr;
   const size_t Tk = (size_t)c->cfg.max_tokens * sh.k;
   auto undo = [&]() {
-    void* ps[] = {nslots, nk, ns, nxs, nhs};
+    void* ps[] = {nslots, nk, ns, nxs, nhs, nhl};
     for (void* p : ps)
       if (p) cudaFree(p);
     cudaGetLastError();
@@ -1032,7 +1034,8 @@ ft_status ft_moe_resize_cache(ft_ctx* c, int64_t new_slots) {
   if (ok) ok = cudaMalloc((void**)&ns, sizeof(unsigned long long) * nC) == cudaSuccess;
   if (ok && tc_new && !d.xs) {
     ok = cudaMalloc((void**)&nxs, sizeof(__nv_bfloat16) * (Tk + 256) * sh.d) == cudaSuccess &&
-         cudaMalloc((void**)&nhs, sizeof(__nv_bfloat16) * (Tk + 256) * sh.d_ff) == cudaSuccess;
+         cudaMalloc((void**)&nhs, sizeof(__nv_bfloat16) * (Tk + 256) * sh.d_ff) == cudaSuccess &&
+         cudaMalloc((void**)&nhl, sizeof(__nv_bfloat16) * (Tk + 256) * sh.d_ff) == cudaSuccess;
   }
   if (!ok) {
     undo();
@@ -1071,11 +1074,12 @@ ft_status ft_moe_resize_cache(ft_ctx* c, int64_t new_slots) {
   sh.C = Cn;
   c->cfg.cache_slots = Cn;
   prefill_tc_free(d);
-  if (nxs) d.xs = nxs, d.hs = nhs;
+  if (nxs) d.xs = nxs, d.hs = nhs, d.hs_lo = nhl;
   if (!tc_new && d.xs) {
     cudaFree(d.xs);
     cudaFree(d.hs);
-    d.xs = d.hs = nullptr;
+    cudaFree(d.hs_lo);
+    d.xs = d.hs = d.hs_lo = nullptr;
   }
   c->use_tc = tc_new;
   if (tc_new && prefill_tc_init(sh, d, (int)Tk) != cudaSuccess) {

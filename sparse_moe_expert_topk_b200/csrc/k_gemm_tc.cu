@@ -11,8 +11,15 @@
 // expert's tokens the N side (N = tokens rounded up to 16, <= 256), so no
 // weight tile is padded:
 //   phase 0: D_g[f, p] = W_gate[f, :] . X_s[p, :],  D_u[f, p] = W_up[f, :] . X_s[p, :]
-//            H_s[p, f] = bf16(silu(D_g) * D_u)          (two accumulators in TMEM)
-//   phase 1: Y[p, r]   = W_down[r, :] . H_s[p, :]        (fp32 into the expert output buffer)
+//            h = silu(D_g) * D_u                         (two accumulators in TMEM)
+//            H_s[p, f] = bf16(h), H_lo[p, f] = bf16(h - H_s[p, f])   (BF16 experts)
+//   phase 1: Y[p, r]   = W_down[r, :] . H_s[p, :] (+ W_down[r, :] . H_lo[p, :])
+//                                                        (fp32 into the expert output buffer)
+// BF16 experts carry h as a bf16 pair (hi + lo, ~16 bits): one bf16 rounding of
+// h alone, together with the bf16 rounding of y, takes the largest errors of
+// a full layer past 2e-2 of rms. The down GEMM runs its K loop twice, the
+// second time over H_lo with the same weight tiles (reloaded from L2), into
+// the same accumulator.
 // X_s / H_s hold the activations in expert-sorted order (row p = sorted
 // position), so an expert's tokens are consecutive rows.
 //
@@ -33,10 +40,15 @@
 namespace ft {
 
 struct TcPlan {
-  CUtensorMap a_gu;  // slot pool as rows of d bf16 (gate/up rows)
-  CUtensorMap a_dn;  // slot pool as rows of d_ff bf16 (down rows)
+  CUtensorMap a_gu;  // BF16: slot pool as rows of d bf16 (gate/up rows)
+  CUtensorMap a_dn;  // BF16: slot pool as rows of d_ff bf16 (down rows)
   CUtensorMap b_x;   // X_s [rows, d]
   CUtensorMap b_h;   // H_s [rows, d_ff]
+  CUtensorMap b_hlo; // BF16: H_lo [rows, d_ff]
+  // NVFP4: the codes of each matrix over the slot pool
+  // (3D: bytes of a row, rows of the matrix, slot), phase 0 and phase 1
+  CUtensorMap f_code[3];  // gate, up, down
+  bool fp4;
   int sms;
 };
 
@@ -124,17 +136,23 @@ __device__ __forceinline__ uint32_t idesc_bf16(int M, int N) {
 
 struct TcArgs {
   const WorkLists* work;
+  int two_b;            // phase 1 of BF16: a second token operand (H_lo) over the same weights
+  const float* tscale;  // NVFP4: [L*E*3] per-matrix tensor scales
+  const uint8_t* slots; // NVFP4: the slot pool (block scales are read from it)
+  size_t slot_bytes;
+  int layer, E;
   int phase;
   int d, d_ff;
   int m_tiles;   // weight-row tiles of 128
   int k_blocks;  // K / 64
   __nv_bfloat16* hs;  // phase 0 output [rows, d_ff]
+  __nv_bfloat16* hs_lo;  // BF16 phase 0: bf16 rest of h [rows, d_ff] (null: h is one bf16)
   float* ybuf;        // phase 1 output [rows, d]
   uint32_t* error;
 };
 
 struct Unit {
-  int slot, p0, nrows, mt;
+  int slot, p0, nrows, mt, e;
 };
 
 // Units: (item, token tile of <= 256, weight-row tile); item-major so that the
@@ -151,6 +169,7 @@ __device__ __forceinline__ bool unit_at(const TcArgs& a, const WorkItem* items, 
   const WorkItem it = items[lo];
   const int j = q - pref[lo];
   out.slot = it.slot;
+  out.e = it.e;
   out.p0 = it.tok_off + j * MAX_N;
   out.nrows = min(MAX_N, it.n_tok - j * MAX_N);
   out.mt = u - q * a.m_tiles;
@@ -158,7 +177,8 @@ __device__ __forceinline__ bool unit_at(const TcArgs& a, const WorkItem* items, 
 }
 
 __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a,
-                                                             const __grid_constant__ CUtensorMap tm_b, TcArgs a) {
+                                                             const __grid_constant__ CUtensorMap tm_b,
+                                                             const __grid_constant__ CUtensorMap tm_b2, TcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ WorkItem s_items[MAX_E];
   __shared__ int s_pref[MAX_E + 1];
@@ -230,8 +250,12 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
         row_a0 = un.slot * 3 * a.d + 2 * a.d + un.mt * BM;    // down rows
         row_a1 = 0;
       }
-      for (int kb = 0; kb < a.k_blocks; ++kb, ++it) {
+      // with a second token operand (H_lo) the K loop runs twice
+      const int kbs = a.k_blocks * (a.two_b ? 2 : 1);
+      for (int kb2 = 0; kb2 < kbs; ++kb2, ++it) {
         const int s = it % STAGES, r = it / STAGES;
+        const int kb = kb2 % a.k_blocks;
+        const CUtensorMap* mb_tok = kb2 < a.k_blocks ? &tm_b : &tm_b2;
         if (!mbar_wait(bar_empty + 8 * s, (r & 1) ^ 1, abort, a.error)) break;
         last_round[s] = r;
         if (lane == 0) {
@@ -240,7 +264,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
           tma_load_2d(base, &tm_a, bar_full + 8 * s, kb * BK, row_a0);
           if (two_a) tma_load_2d(base + A_BYTES, &tm_a, bar_full + 8 * s, kb * BK, row_a1);
           for (int b = 0; b < nb; ++b)
-            tma_load_2d(base + 2 * A_BYTES + b * BOX_ROWS * 128, &tm_b, bar_full + 8 * s, kb * BK,
+            tma_load_2d(base + 2 * A_BYTES + b * BOX_ROWS * 128, mb_tok, bar_full + 8 * s, kb * BK,
                         un.p0 + b * BOX_ROWS);
         }
         __syncwarp();
@@ -259,7 +283,8 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
       const uint32_t dacc = tmem + (uint32_t)(ab * 256);
       tc_fence_after();
       bool ok = true;
-      for (int kb = 0; kb < a.k_blocks; ++kb, ++it) {
+      const int kbs = a.k_blocks * (a.two_b ? 2 : 1);
+      for (int kb = 0; kb < kbs; ++kb, ++it) {
         const int s = it % STAGES, r = it / STAGES;
         if (!mbar_wait(bar_full + 8 * s, r & 1, abort, a.error)) {
           ok = false;
@@ -275,7 +300,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
             if (two_a) umma_bf16(tmem + 256, sw128_desc(base + A_BYTES + kk * 32), bd, idesc, (kb | kk) != 0);
           }
           umma_commit(bar_empty + 8 * s);  // stage free once these MMAs have read it
-          if (kb == a.k_blocks - 1) umma_commit(bar_acc_full + 8 * ab);
+          if (kb == kbs - 1) umma_commit(bar_acc_full + 8 * ab);
         }
         __syncwarp();
       }
@@ -305,7 +330,10 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
             if (c0 + i < un.nrows) {
               const float gv = __uint_as_float(g[i]), uv = __uint_as_float(uu[i]);
               const float hv = gv / (1.f + expf(-gv)) * uv;
-              a.hs[(size_t)(un.p0 + c0 + i) * a.d_ff + row] = __float2bfloat16_rn(hv);
+              const size_t o = (size_t)(un.p0 + c0 + i) * a.d_ff + row;
+              const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
+              a.hs[o] = hi;
+              if (a.hs_lo) a.hs_lo[o] = __float2bfloat16_rn(hv - __bfloat162float(hi));
             }
           }
         } else {
@@ -346,6 +374,336 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
   }
 }
 
+// ---------------------------------------------------------------------------
+// NVFP4 experts on the same tensor cores. tcgen05 has no MMA kind that takes
+// 4-bit weights against 16-bit activations, so the weight tiles are widened
+// on chip: the TMA engine brings each tile's e2m1 codes (straight from the
+// slot, no bytes added in HBM), eight dequantising warps, which read the
+// tile's e4m3 block scales themselves one k-block ahead,
+// turn them into the bf16 128B-swizzled tile the bf16 MMA reads (e2m1 x e4m3
+// has at most 6 significant bits, exact in bf16), and the per-matrix fp32
+// tensor scale multiplies the accumulators in the epilogue. Activations and
+// the rest of the pipeline are the bf16 kernel's: tokens on the N side,
+// gate and up in two TMEM halves, SwiGLU in the epilogue.
+//
+// Rings: the A (weights) and B (tokens) tiles in STAGES stages as above, the
+// raw codes in F_RAW stages of their own. Barriers per A/B stage: full (TMA
+// of the token tile), deq (256 dequantising threads wrote the A tile), empty
+// (the MMAs that read the stage completed); per raw stage: raw_full (TMA of
+// the codes), raw_empty (the dequantising threads read them).
+// ---------------------------------------------------------------------------
+constexpr int F_RAW = 2;
+constexpr int F_CODE_BYTES = BM * BK / 2;  // 4 KB: 128 rows x 32 code bytes (64 values)
+constexpr int F_RAW_BYTES = 2 * F_CODE_BYTES;
+constexpr int F_DEQ_WARPS = 8;
+constexpr int F_THREADS = (6 + F_DEQ_WARPS) * 32;
+constexpr int F_SMEM_BYTES = STAGES * STAGE_BYTES + F_RAW * F_RAW_BYTES + 1024 + 256;
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+// Four e2m1 code bytes (8 values, even value in the low nibble) times one
+// e4m3 block scale -> four bf16 pairs, exactly.
+__device__ __forceinline__ uint4 fp4x8_to_bf16x8(uint32_t codes, uint32_t scale_byte) {
+  uint32_t h[4];
+  asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %4;\n"
+      " cvt.rn.f16x2.e2m1x2 %0, b0;\n cvt.rn.f16x2.e2m1x2 %1, b1;\n"
+      " cvt.rn.f16x2.e2m1x2 %2, b2;\n cvt.rn.f16x2.e2m1x2 %3, b3;\n}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(codes));
+  uint32_t s2;
+  asm("{\n .reg .b16 t;\n cvt.u16.u32 t, %1;\n cvt.rn.f16x2.e4m3x2 %0, t;\n}" : "=r"(s2) : "r"(scale_byte));
+  const __half2 sc = __low2half2(*reinterpret_cast<const __half2*>(&s2));
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&h[i]), sc);
+    const float2 f = __half22float2(v);
+    const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
+    o[i] = *reinterpret_cast<const uint32_t*>(&b);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+struct TcFp4Maps {
+  CUtensorMap code_a, code_b;  // phase 0: gate / up codes; phase 1: down codes (b unused)
+};
+
+__global__ void __launch_bounds__(F_THREADS, 1) gemm_tc_fp4_kernel(const __grid_constant__ CUtensorMap tm_b,
+                                                                   const __grid_constant__ TcFp4Maps fm, TcArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ WorkItem s_items[MAX_E];
+  __shared__ int s_pref[MAX_E + 1];
+  __shared__ int s_abort;
+  __shared__ uint32_t s_tmem;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* raw = smem + STAGES * STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(raw + F_RAW * F_RAW_BYTES);
+  const uint32_t bar_full = smem_u32(bars), bar_empty = bar_full + 8 * STAGES, bar_deq = bar_empty + 8 * STAGES;
+  const uint32_t bar_rfull = bar_deq + 8 * STAGES, bar_rempty = bar_rfull + 8 * F_RAW;
+  const uint32_t bar_acc_full = bar_rempty + 8 * F_RAW, bar_acc_empty = bar_acc_full + 16;
+  const uint32_t bar_drain = bar_acc_empty + 16;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort = &s_abort;
+  constexpr int DEQ_THREADS = F_DEQ_WARPS * 32;
+
+  const int n_items = a.work->n_items[KIND_HIT];
+  for (int i = threadIdx.x; i < n_items; i += F_THREADS) s_items[i] = a.work->items[KIND_HIT][i];
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+      mbar_init(bar_deq + 8 * s, DEQ_THREADS);
+    }
+    for (int r = 0; r < F_RAW; ++r) {
+      mbar_init(bar_rfull + 8 * r, 1);
+      mbar_init(bar_rempty + 8 * r, DEQ_THREADS);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_acc_full + 8 * b, 1);
+      mbar_init(bar_acc_empty + 8 * b, 4);
+    }
+    mbar_init(bar_drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&s_tmem), 512);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int p = 0;
+    for (int i = 0; i < n_items; ++i) {
+      s_pref[i] = p;
+      p += (s_items[i].n_tok + MAX_N - 1) / MAX_N;
+    }
+    s_pref[n_items] = p;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  const int n_units = n_items > 0 ? s_pref[n_items] * a.m_tiles : 0;
+  const int two_a = a.phase == 0;
+  const int n_mat = two_a ? 2 : 1;
+
+  int last_round[STAGES], last_raw[F_RAW];  // producer: last round issued per stage (-1 none)
+#pragma unroll
+  for (int s = 0; s < STAGES; ++s) last_round[s] = -1;
+#pragma unroll
+  for (int r = 0; r < F_RAW; ++r) last_raw[r] = -1;
+  if (warp == 0) {
+    // ---------------- TMA producer: token tiles, codes and scales ----------------
+    int it = 0;
+    for (int u = blockIdx.x; u < n_units && !*abort; u += gridDim.x) {
+      Unit un;
+      if (!unit_at(a, s_items, s_pref, n_items, u, un)) break;
+      const int nb = (un.nrows + BOX_ROWS - 1) / BOX_ROWS;
+      const uint32_t b_bytes = nb * BOX_ROWS * BK * 2;
+      const uint32_t r_bytes = n_mat * F_CODE_BYTES;
+      const int row0 = un.mt * BM;
+      bool ok = true;
+      for (int kb = 0; kb < a.k_blocks; ++kb, ++it) {
+        const int s = it % STAGES, r = it / STAGES, q = it % F_RAW, rq = it / F_RAW;
+        if (!mbar_wait(bar_empty + 8 * s, (r & 1) ^ 1, abort, a.error) ||
+            !mbar_wait(bar_rempty + 8 * q, (rq & 1) ^ 1, abort, a.error)) {
+          ok = false;
+          break;
+        }
+        last_round[s] = r;
+        last_raw[q] = rq;
+        if (lane == 0) {
+          const uint32_t rb = smem_u32(raw + q * F_RAW_BYTES);
+          mbar_expect_tx(bar_rfull + 8 * q, r_bytes);
+          tma_load_3d(rb, &fm.code_a, bar_rfull + 8 * q, kb * (BK / 2), row0, un.slot);
+          if (two_a) tma_load_3d(rb + F_CODE_BYTES, &fm.code_b, bar_rfull + 8 * q, kb * (BK / 2), row0, un.slot);
+          const uint32_t base = smem_u32(smem + s * STAGE_BYTES);
+          mbar_expect_tx(bar_full + 8 * s, b_bytes);
+          for (int b = 0; b < nb; ++b)
+            tma_load_2d(base + 2 * A_BYTES + b * BOX_ROWS * 128, &tm_b, bar_full + 8 * s, kb * BK,
+                        un.p0 + b * BOX_ROWS);
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    int it = 0, ui = 0;
+    for (int u = blockIdx.x; u < n_units && !*abort; u += gridDim.x, ++ui) {
+      Unit un;
+      if (!unit_at(a, s_items, s_pref, n_items, u, un)) break;
+      const int n_mma = (un.nrows + 15) & ~15;
+      const uint32_t idesc = idesc_bf16(BM, n_mma);
+      const int ab = two_a ? 0 : (ui & 1), use = two_a ? ui : (ui >> 1);
+      if (!mbar_wait(bar_acc_empty + 8 * ab, (use & 1) ^ 1, abort, a.error)) break;
+      const uint32_t dacc = tmem + (uint32_t)(ab * 256);
+      tc_fence_after();
+      bool ok = true;
+      for (int kb = 0; kb < a.k_blocks; ++kb, ++it) {
+        const int s = it % STAGES, r = it / STAGES;
+        if (!mbar_wait(bar_full + 8 * s, r & 1, abort, a.error) || !mbar_wait(bar_deq + 8 * s, r & 1, abort, a.error)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t base = smem_u32(smem + s * STAGE_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t bd = sw128_desc(base + 2 * A_BYTES + kk * 32);
+            umma_bf16(dacc, sw128_desc(base + kk * 32), bd, idesc, (kb | kk) != 0);
+            if (two_a) umma_bf16(tmem + 256, sw128_desc(base + A_BYTES + kk * 32), bd, idesc, (kb | kk) != 0);
+          }
+          umma_commit(bar_empty + 8 * s);
+          if (kb == a.k_blocks - 1) umma_commit(bar_acc_full + 8 * ab);
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+    }
+  } else if (warp < 6) {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int q = warp & 3;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    int ui = 0;
+    for (int u = blockIdx.x; u < n_units && !*abort; u += gridDim.x, ++ui) {
+      Unit un;
+      if (!unit_at(a, s_items, s_pref, n_items, u, un)) break;
+      const int ab = two_a ? 0 : (ui & 1), use = two_a ? ui : (ui >> 1);
+      if (!mbar_wait(bar_acc_full + 8 * ab, use & 1, abort, a.error)) break;
+      tc_fence_after();
+      const float* ts = a.tscale + ((size_t)a.layer * a.E + un.e) * 3;
+      const int row = un.mt * BM + 32 * q + lane;
+      for (int c0 = 0; c0 < un.nrows; c0 += 32) {
+        uint32_t g[32];
+        tmem_ld32(tmem + (uint32_t)(ab * 256) + lane_base + c0, g);
+        if (two_a) {
+          uint32_t uu[32];
+          tmem_ld32(tmem + lane_base + 256 + c0, uu);
+          tmem_ld_wait();
+          const float t0 = ts[0], t1 = ts[1];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (c0 + i < un.nrows) {
+              const float gv = __uint_as_float(g[i]) * t0, uv = __uint_as_float(uu[i]) * t1;
+              const float hv = gv / (1.f + expf(-gv)) * uv;
+              a.hs[(size_t)(un.p0 + c0 + i) * a.d_ff + row] = __float2bfloat16_rn(hv);
+            }
+          }
+        } else {
+          tmem_ld_wait();
+          const float t2 = ts[2];
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (c0 + i < un.nrows) a.ybuf[(size_t)(un.p0 + c0 + i) * a.d + row] = __uint_as_float(g[i]) * t2;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_acc_empty + 8 * ab);
+    }
+  } else {
+    // ---------------- dequantising warps (6..13) ----------------
+    // thread dt owns half-rows dt (and dt + 256 for gate/up): (matrix, row,
+    // half) = (i / 256, (i % 256) / 2, i % 2); its two block scales of a
+    // k-block are one 16-bit word of the matrix's scale rows, read one
+    // k-block ahead
+    const int dt = threadIdx.x - 6 * 32;  // 0..255
+    const size_t n = (size_t)a.d * a.d_ff;
+    const int K = two_a ? a.d : a.d_ff;
+    const size_t sc0 = 3 * (n / 2) + (two_a ? 0 : n / 8);  // scales of gate (phase 0) or down (phase 1)
+    int it = 0;
+    for (int u = blockIdx.x; u < n_units && !*abort; u += gridDim.x) {
+      Unit un;
+      if (!unit_at(a, s_items, s_pref, n_items, u, un)) break;
+      const uint8_t* blob = a.slots + (size_t)un.slot * a.slot_bytes;
+      const unsigned short* scp[2];
+#pragma unroll
+      for (int v = 0; v < 2; ++v) {
+        const int i = dt + v * DEQ_THREADS;
+        const int m = i / (2 * BM), row = un.mt * BM + ((i % (2 * BM)) >> 1), h = i & 1;
+        scp[v] = reinterpret_cast<const unsigned short*>(blob + sc0 + m * (n / 16) + (size_t)row * (K / 16)) + h;
+      }
+      uint32_t scn[2] = {0, 0};
+#pragma unroll
+      for (int v = 0; v < 2; ++v)
+        if (v < n_mat) scn[v] = __ldg(scp[v]);
+      bool ok = true;
+      for (int kb = 0; kb < a.k_blocks; ++kb, ++it) {
+        const int s = it % STAGES, r = it / STAGES, q = it % F_RAW, rq = it / F_RAW;
+        uint32_t scc[2] = {scn[0], scn[1]};
+        if (kb + 1 < a.k_blocks) {
+#pragma unroll
+          for (int v = 0; v < 2; ++v)
+            if (v < n_mat) scn[v] = __ldg(scp[v] + 2 * (kb + 1));
+        }
+        if (!mbar_wait(bar_rfull + 8 * q, rq & 1, abort, a.error) ||
+            !mbar_wait(bar_empty + 8 * s, (r & 1) ^ 1, abort, a.error)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* rb = raw + q * F_RAW_BYTES;
+        uint8_t* ab_tile = smem + s * STAGE_BYTES;
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+          if (v >= n_mat) break;
+          const int i = dt + v * DEQ_THREADS;
+          const int m = i / (2 * BM), row = (i % (2 * BM)) >> 1, h = i & 1;
+          const uint4 codes = *reinterpret_cast<const uint4*>(rb + m * F_CODE_BYTES + row * 32 + h * 16);
+          const uint32_t s0 = scc[v] & 0xFF, s1 = (scc[v] >> 8) & 0xFF;
+          uint8_t* dst = ab_tile + m * A_BYTES + row * 128;
+          const int sw = row & 7;
+          *reinterpret_cast<uint4*>(dst + (((4 * h + 0) ^ sw) << 4)) = fp4x8_to_bf16x8(codes.x, s0);
+          *reinterpret_cast<uint4*>(dst + (((4 * h + 1) ^ sw) << 4)) = fp4x8_to_bf16x8(codes.y, s0);
+          *reinterpret_cast<uint4*>(dst + (((4 * h + 2) ^ sw) << 4)) = fp4x8_to_bf16x8(codes.z, s1);
+          *reinterpret_cast<uint4*>(dst + (((4 * h + 3) ^ sw) << 4)) = fp4x8_to_bf16x8(codes.w, s1);
+        }
+        // the MMAs read the tile through the async proxy
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive(bar_deq + 8 * s);
+        mbar_arrive(bar_rempty + 8 * q);
+      }
+      if (!ok) break;
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // producer tail: every stage's last round released (normal exit) or at
+    // least landed (abort) before shared memory goes away
+    for (int s = 0; s < STAGES; ++s) {
+      if (last_round[s] < 0) continue;
+      const uint32_t bar = *abort ? bar_full + 8 * s : bar_empty + 8 * s;
+      const long long t0 = clock64();
+      while (!mbar_try_wait(bar, last_round[s] & 1) && clock64() - t0 < WAIT_CYCLES / 4) {
+      }
+    }
+    for (int q = 0; q < F_RAW; ++q) {
+      if (last_raw[q] < 0) continue;
+      const long long t0 = clock64();
+      while (!mbar_try_wait(bar_rfull + 8 * q, last_raw[q] & 1) && clock64() - t0 < WAIT_CYCLES / 4) {
+      }
+    }
+  } else if (warp == 1 && *abort) {
+    if (lane == 0) umma_commit(bar_drain);
+    __syncwarp();
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar_drain, 0) && clock64() - t0 < WAIT_CYCLES / 4) {
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 // X_s[p, :] = x[perm[p] / k, :] (bf16 rows, 16-byte vectors); grid (rows), 256 threads.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* __restrict__ x,
                                                           const int32_t* __restrict__ perm, int k, int d,
@@ -370,10 +728,26 @@ bool encode_2d(CUtensorMap* m, void* base, uint64_t rows, uint64_t cols, uint32_
   return r == CUDA_SUCCESS;
 }
 
+// 3D byte map over the slot pool: `row_bytes` per row, `rows` rows per slot,
+// `slots` slots `slot_bytes` apart, starting `off` bytes into each slot; box
+// of box_x bytes x BM rows x 1 slot.
+bool encode_3d_u8(CUtensorMap* m, const uint8_t* slots, size_t off, uint64_t row_bytes, uint64_t rows,
+                  uint64_t n_slots, uint64_t slot_bytes, uint32_t box_x) {
+  cuuint64_t dims[3] = {row_bytes, rows, n_slots};
+  cuuint64_t strides[2] = {row_bytes, slot_bytes};
+  cuuint32_t box[3] = {box_x, (cuuint32_t)BM, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, (void*)(slots + off), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 bool prefill_tc_supported(const Shape& sh) {
-  return sh.wtype == FT_W_BF16 && sh.d % BM == 0 && sh.d_ff % BM == 0 && sh.C > 0;
+  if (sh.C <= 0 || sh.d % BM || sh.d_ff % BM) return false;
+  return sh.wtype == FT_W_BF16 || sh.wtype == FT_W_NVFP4;
 }
 
 cudaError_t prefill_tc_init(const Shape& sh, DevState& ds, int max_rows) {
@@ -386,11 +760,25 @@ cudaError_t prefill_tc_init(const Shape& sh, DevState& ds, int max_rows) {
   if (!p) return cudaErrorMemoryAllocation;
   ds.tc_plan = p;  // owned by the context (prefill_tc_free)
   const uint64_t C = (uint64_t)sh.C;
-  if (!encode_2d(&p->a_gu, ds.slots, C * 3 * sh.d_ff, sh.d, BM)) return cudaErrorInvalidValue;
-  if (!encode_2d(&p->a_dn, ds.slots, C * 3 * sh.d, sh.d_ff, BM)) return cudaErrorInvalidValue;
+  p->fp4 = sh.wtype == FT_W_NVFP4;
+  if (!p->fp4) {
+    if (!encode_2d(&p->a_gu, ds.slots, C * 3 * sh.d_ff, sh.d, BM)) return cudaErrorInvalidValue;
+    if (!encode_2d(&p->a_dn, ds.slots, C * 3 * sh.d, sh.d_ff, BM)) return cudaErrorInvalidValue;
+  } else {
+    const size_t n = (size_t)sh.d * sh.d_ff;
+    const uint8_t* sl = ds.slots;
+    const bool ok = encode_3d_u8(&p->f_code[0], sl, 0, sh.d / 2, sh.d_ff, C, sh.slot_bytes, BK / 2) &&
+                    encode_3d_u8(&p->f_code[1], sl, n / 2, sh.d / 2, sh.d_ff, C, sh.slot_bytes, BK / 2) &&
+                    encode_3d_u8(&p->f_code[2], sl, n, sh.d_ff / 2, sh.d, C, sh.slot_bytes, BK / 2);
+    if (!ok) return cudaErrorInvalidValue;
+  }
   if (!encode_2d(&p->b_x, ds.xs, (uint64_t)max_rows + 256, sh.d, BOX_ROWS)) return cudaErrorInvalidValue;
   if (!encode_2d(&p->b_h, ds.hs, (uint64_t)max_rows + 256, sh.d_ff, BOX_ROWS)) return cudaErrorInvalidValue;
+  if (!p->fp4 && !encode_2d(&p->b_hlo, ds.hs_lo, (uint64_t)max_rows + 256, sh.d_ff, BOX_ROWS))
+    return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gemm_tc_fp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, F_SMEM_BYTES);
   if (e != cudaSuccess) return e;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -406,20 +794,35 @@ void launch_prefill_gather(const Shape& sh, const void* x, int T, DevState& ds, 
   gather_rows_kernel<<<T * sh.k, 256, 0, st>>>((const __nv_bfloat16*)x, ds.perm, sh.k, sh.d, ds.xs);
 }
 
-void launch_gemm_tc(const Shape& sh, int phase, int T, DevState& ds, cudaStream_t st) {
+void launch_gemm_tc(const Shape& sh, int phase, int layer, int T, DevState& ds, cudaStream_t st) {
   (void)T;
   const TcPlan& p = *static_cast<const TcPlan*>(ds.tc_plan);
   TcArgs a;
   a.work = ds.work;
+  a.tscale = ds.tscale;
+  a.slots = ds.slots;
+  a.slot_bytes = sh.slot_bytes;
+  a.layer = layer;
+  a.E = sh.E;
   a.phase = phase;
   a.d = sh.d;
   a.d_ff = sh.d_ff;
   a.m_tiles = (phase == 0 ? sh.d_ff : sh.d) / BM;
   a.k_blocks = (phase == 0 ? sh.d : sh.d_ff) / BK;
   a.hs = ds.hs;
+  a.hs_lo = p.fp4 ? nullptr : ds.hs_lo;
+  a.two_b = !p.fp4 && phase == 1;
   a.ybuf = ds.ybuf;
   a.error = ds.error;
-  gemm_tc_kernel<<<p.sms, THREADS, SMEM_BYTES, st>>>(phase == 0 ? p.a_gu : p.a_dn, phase == 0 ? p.b_x : p.b_h, a);
+  if (p.fp4) {
+    TcFp4Maps fm;
+    fm.code_a = p.f_code[phase == 0 ? 0 : 2];
+    fm.code_b = p.f_code[1];
+    gemm_tc_fp4_kernel<<<p.sms, F_THREADS, F_SMEM_BYTES, st>>>(phase == 0 ? p.b_x : p.b_h, fm, a);
+    return;
+  }
+  gemm_tc_kernel<<<p.sms, THREADS, SMEM_BYTES, st>>>(phase == 0 ? p.a_gu : p.a_dn, phase == 0 ? p.b_x : p.b_h,
+                                                     p.b_hlo, a);
 }
 
 }  // namespace ft

@@ -697,6 +697,65 @@ __device__ __forceinline__ void dot_bf16_slices(const uint8_t* ra, const uint8_t
   }
 }
 
+// The same over RT row tiles per step (tile r's rows tstride bytes after
+// tile 0's), which share each step's activation fragments: U steps of RT x 2
+// weight loads in flight, and per tile the MMAs of bf16_step in its order, so
+// every row's sum is the single-tile kernels' exactly.
+template <int NB, int RT, int U, bool P1, int NWARPS>
+__device__ __forceinline__ void dot_bf16_rt(const uint8_t* ra, const uint8_t* rb, size_t tstride, const Geo& g,
+                                            int warp, const uint16_t* const (&xr)[NB], const uint16_t* const (&xl)[NB],
+                                            int q, float (&acc)[RT][NB][4]) {
+  int j = 0;
+  int lo = (warp * min(g.ss, g.steps)) / NWARPS, hi = ((warp + 1) * min(g.ss, g.steps)) / NWARPS;
+  int s = lo;
+  for (;;) {
+    int st[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      while (s >= hi && j + 1 < g.nsl) {
+        ++j;
+        const int b0 = j * g.ss, ns = min(g.ss, g.steps - b0);
+        lo = b0 + (warp * ns) / NWARPS;
+        hi = b0 + ((warp + 1) * ns) / NWARPS;
+        s = lo;
+      }
+      st[u] = s < hi ? s : -1;
+      s += s < hi ? 1 : 0;
+    }
+    if (st[0] < 0) break;
+    uint4 wa[U][RT], wb[U][RT];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int ss = st[u] >= 0 ? st[u] : st[0];
+#pragma unroll
+      for (int r = 0; r < RT; ++r) {
+        wa[u][r] = ld_stream(ra + r * tstride + (size_t)ss * 64);
+        wb[u][r] = ld_stream(rb + r * tstride + (size_t)ss * 64);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (st[u] < 0) continue;
+      const int e0 = st[u] * 32 + q * 8;
+#pragma unroll
+      for (int t = 0; t < NB; ++t) {
+        const uint4 xv = P1 ? ld_cg(xr[t] + e0) : __ldg(reinterpret_cast<const uint4*>(xr[t] + e0));
+        uint4 xo = xv;
+        if constexpr (P1) xo = ld_cg(xl[t] + e0);
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+          mma_bf16(acc[r][t], wa[u][r].x, wb[u][r].x, wa[u][r].y, wb[u][r].y, xv.x, xv.y);
+          mma_bf16(acc[r][t], wa[u][r].z, wb[u][r].z, wa[u][r].w, wb[u][r].w, xv.z, xv.w);
+          if constexpr (P1) {
+            mma_bf16(acc[r][t], wa[u][r].x, wb[u][r].x, wa[u][r].y, wb[u][r].y, xo.x, xo.y);
+            mma_bf16(acc[r][t], wa[u][r].z, wb[u][r].z, wa[u][r].w, wb[u][r].w, xo.z, xo.w);
+          }
+        }
+      }
+    }
+  }
+}
+
 // NVFP4: steps of 128 K values (lane q covers K = 128 s + 32 q .. +32: 16
 // code bytes and one scale pair per row); RT row tiles per step, the tiles
 // tstride code bytes (tsc scale pairs) apart, sharing one activation
@@ -858,14 +917,16 @@ __device__ void direct_unit(const MmaArgs& a, const WorkItem& it, int chunk, int
 #pragma unroll
           for (int c = 0; c < 4; ++c) acc[r][t][c] = fmaf(acc[r][t][c], H_SPLIT, acc2[r][t][c]);
     }
+  } else if constexpr (RT > 1) {
+    // several row tiles share each step's activations: two steps in flight
+    dot_bf16_rt<NB, RT, 2, PHASE == 1, NW>(blob + oa + q * 16, blob + ob + q * 16,
+                                           (size_t)rows_per_tile * rbytes, gg, warp, xr, xl, q, acc);
   } else if constexpr (NB == 1) {
     // up to 8 tokens: a warp's steps gathered across slices, 8 loads in flight
-    static_assert(FP4 || RT == 1, "BF16 units are one row tile");
     dot_bf16_slices<NB, 8, PHASE == 1, NW>(blob + oa + q * 16, blob + ob + q * 16, gg, warp, xr, xl, q, acc[0]);
   } else {
     // 9..16 tokens: slice by slice, 4 loads in flight, fewer registers and
     // more CTAs per SM (measured faster at this size); the same step order
-    static_assert(FP4 || RT == 1, "BF16 units are one row tile");
     for (int j = 0; j < gg.nsl; ++j) {
       const int b0 = j * gg.ss, ns = min(gg.ss, gg.steps - b0);
       const int s0 = b0 + (warp * ns) / NW, s1 = b0 + ((warp + 1) * ns) / NW;
@@ -945,14 +1006,15 @@ constexpr int tiles_for() { return FP4 ? 4 : 1; }
 // put them (a unit's row tiles change which rows it covers, not the K order
 // of any row, so results do not depend on this choice).
 template <bool FP4>
-constexpr int tiles_down_for() { return FP4 ? 2 : 1; }
+constexpr int tiles_down_for() { return FP4 ? 2 : 4; }
 
 template <int NB, bool FP4, int NW>
 __global__ void __launch_bounds__(NW * 32) gemv_direct_kernel(MmaArgs a) {
   constexpr int RT = tiles_for<FP4>(), RT1 = tiles_down_for<FP4>();
+  constexpr int RTM = RT > RT1 ? RT : RT1;
   __shared__ int s_pref[MAX_E + 1];
   __shared__ WorkItem s_items[MAX_E];
-  __shared__ float red[NW * RT * NB * 4 * 32];
+  __shared__ float red[NW * RTM * NB * 4 * 32];
   __shared__ int s_unit;
   const int n_items = a.work->n_items[a.cls];
   if (n_items == 0) return;
@@ -1438,20 +1500,9 @@ void launch_gemv_mma(const Shape& sh, int cls, int layer, const void* x16, int T
   const bool fp4 = sh.wtype == FT_W_NVFP4;
   const int NB = T > 8 ? 2 : 1;
   const long long chunks = (long long)max_items + (long long)max_tok / CHUNK;
-  if (cls == KIND_HIT && !fp4) {
-    const long long units = chunks * (sh.d_ff / 8 + sh.d / 16);
-    const int cap = g_grid_hit[NB];
-    const int grid = (int)(units < cap ? units : cap);
-    if (grid <= 0) return;
-    if (NB == 1)
-      gemv_hit_bf16_kernel<1><<<grid, RING_WARPS * 32, 0, st>>>(a);
-    else
-      gemv_hit_bf16_kernel<2><<<grid, RING_WARPS * 32, 0, st>>>(a);
-    return;
-  }
   if (cls == KIND_HIT) {
-    const long long units =
-        chunks * (sh.d_ff / 8 / (fp4 ? tiles_for<true>() : 1) + sh.d / 16 / (fp4 ? tiles_down_for<true>() : 1));
+    const long long units = chunks * (fp4 ? sh.d_ff / 8 / tiles_for<true>() + sh.d / 16 / tiles_down_for<true>()
+                                          : sh.d_ff / 8 / tiles_for<false>() + sh.d / 16 / tiles_down_for<false>());
     const int cap = g_grid_direct[fp4][NB];
     const int grid = (int)(units < cap ? units : cap);
     if (grid <= 0) return;

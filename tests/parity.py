@@ -13,18 +13,32 @@ from oracle import cache as ocache
 from oracle import formats as ofmt
 from oracle import moe as omoe
 
-GAP = 1e-3  # minimum k-th vs (k+1)-th logit gap of every token
+GAP = 1e-3  # minimum gap between consecutive logits among each token's k+1 largest
+
+
+def rank_gaps(s32, k):
+    """Per token, the smallest gap between consecutive logits among its k+1
+    largest: the k-th vs (k+1)-th gap decides which experts are chosen, the
+    others their rank order (inf where E = k)."""
+    srt = -np.sort(-np.asarray(s32, np.float64), axis=1)
+    m = min(k + 1, srt.shape[1])
+    if m < 2:
+        return np.full(srt.shape[0], np.inf)
+    return (srt[:, :m - 1] - srt[:, 1:m]).min(axis=1)
 
 
 def gap_hidden(wl, T, seed, w_router, bias, max_rounds=60):
-    """x [T, d] from ftgen with every token's top-k gap >= GAP (tokens whose
-    oracle logits fall short are redrawn with the next attempt number)."""
+    """x [T, d] from ftgen whose top-k is decided with a margin: for every
+    token the k+1 largest logits are at least GAP apart from each other, so
+    that the chosen experts and their rank order are the same whatever order
+    a dot product is summed in (tokens that fall short are redrawn with the
+    next attempt number)."""
     attempts = np.zeros(T, dtype=np.int64)
     x = ftgen.hidden(T, wl.d, wl.wtype, seed)
     wr = w_router.float().cpu().numpy()
     for _ in range(max_rounds):
         s32 = omoe.router_logits(x.float().numpy(), wr, bias)
-        bad = np.nonzero(omoe.topk_gap(s32, wl.k) < GAP)[0]
+        bad = np.nonzero(rank_gaps(s32, wl.k) < GAP)[0]
         if bad.size == 0:
             return x
         for t in bad:
