@@ -155,3 +155,40 @@ class PrefetchWeights:
     def close(self):
         self.pool.shutdown(wait=True, cancel_futures=True)
         self.fut.clear()
+
+
+class ParallelExpertWeights:
+    """fp64 expert matrices decoded by the oracle on a few threads, with an
+    LRU of `keep` decoded experts: `need(layer, experts)` decodes the missing
+    ones of a call at once, then the object is called like ExpertWeights."""
+
+    def __init__(self, harness, keep=64, workers=8):
+        from concurrent.futures import ThreadPoolExecutor
+        self.h = harness
+        self.keep = keep
+        self.cache = OrderedDict()
+        self.pool = ThreadPoolExecutor(max_workers=workers)
+
+    def _decode(self, layer, e):
+        wl = self.h.wl
+        ts = self.h.tscales.get((layer, e))
+        return ofmt.unpack_expert(self.h.blob(layer, e).copy(), wl.d, wl.d_ff, wl.wtype, ts)
+
+    def need(self, layer, experts):
+        missing = [int(e) for e in experts if (layer, int(e)) not in self.cache]
+        for e, w in zip(missing, self.pool.map(lambda e: self._decode(layer, e), missing)):
+            self.cache[(layer, e)] = w
+        for e in experts:
+            self.cache.move_to_end((layer, int(e)))
+        while len(self.cache) > max(self.keep, len(experts)):
+            self.cache.popitem(last=False)
+
+    def __call__(self, layer, e):
+        key = (layer, int(e))
+        if key not in self.cache:
+            self.need(layer, [e])
+        return self.cache[key]
+
+    def close(self):
+        self.pool.shutdown(wait=True)
+        self.cache.clear()
