@@ -243,3 +243,41 @@ def test_host_buffer_call_matches_device_call(cuda_ok):
         with pytest.raises(ft.FtError):
             x = torch.zeros(17, wl.d, dtype=torch.bfloat16)
             ft.ft_moe_layer_forward_host(b.ctx, 0, ft.FT_DECODE, x, 17, None, 0, torch.empty_like(x))
+
+
+@pytest.mark.parametrize("wname", ["decode_bf16", "trace_nvfp4"])
+def test_decode_against_the_cpp_oracle(cuda_ok, wname):
+    """The plain C++ oracle (one thread per token, the layer's fp32 roundings)
+    and its LRU simulator, against the library on decode calls at batch 1..16:
+    ids bit-exact, the lookup record, m, q* and q_stage identical to the C++
+    cache's, outputs within the BF16 / NVFP4 tolerance."""
+    import dataclasses
+    from oracle import cpp as ocpp
+    base = ftgen.workload(wname)
+    wl = dataclasses.replace(base, name=f"cpp_{wname}", L=2, E=64, cache_slots=20)
+    with _harness(wl, max_tokens=16) as h:
+        cc = ocpp.Cache(wl.L, wl.E, wl.cache_slots, wl.bp_mbps, wl.bh_mbps)
+        zb = ftgen.zipf_log_bias(wl.E, 1.1, wl.seed("zipf"))
+        for step in range(10):
+            for l in range(wl.L):
+                T = (1, 4, 16, 3, 8)[(step + l) % 5]
+                x = gap_hidden(wl, T, wl.seed("cpp", step, l), h.routers[l], zb)
+                y, ids, _ = h.forward(l, x.to(h.dev), torch.as_tensor(zb).to(h.dev), want_route=True)
+                torch.cuda.synchronize()
+                blobs = [h.blob(l, e) for e in range(wl.E)]
+                ts = np.array([h.tscales[(l, e)] for e in range(wl.E)]) if wl.wtype == ftgen.W_NVFP4 else None
+                y_c, ids_c, _ = ocpp.layer_forward(x.float().numpy(), h.routers[l].float().cpu().numpy(), zb, wl.k,
+                                                   blobs, wl.wtype, wl.d, wl.d_ff, ts)
+                np.testing.assert_array_equal(ids.cpu().numpy(), ids_c)
+                check_close(to_np(y), y_c.astype(np.float64), wl.wtype, f"step {step} layer {l}")
+                rec = cc.forward(l, 0, np.bincount(ids_c.ravel(), minlength=wl.E))
+                r = gpu_route(h, T)
+                assert r["lookup_e"].tolist() == [e for (_, e, _) in rec["lookups"]]
+                assert r["lookup_kind"].tolist() == [k for (_, _, k) in rec["lookups"]]
+                assert (r["m"], r["qstar"], r["qstage"]) == (rec["m"], rec["qstar"], rec["qstage"])
+        key_of, stamp = ft.ft_moe_cache_contents(h.ctx, h.C)
+        assert (key_of.tolist(), stamp.tolist()) == cc.contents()
+        cnt, st = cc.counters(), h.stats()
+        for k in ("lookups", "hits", "misses", "staged", "streamed"):
+            assert st[k] == cnt[k], k
+        cc.close()
