@@ -164,7 +164,7 @@ void free_all(ft_ctx* c) {
   if (c->s_comp || c->s_side) cudaDeviceSynchronize();
   DevState& d = c->ds;
   void* dev_ptrs[] = {d.slot_of, d.key_of, d.stamp, d.clk, d.ctr, d.error, d.work, d.scores, d.ids, d.wts,
-                      d.counts, d.offsets, d.perm, d.inv, d.perm_chunks, d.hbuf, d.ybuf, d.xs, d.hs, d.hs_lo, d.tscale, d.slots,
+                      d.counts, d.offsets, d.perm, d.inv, d.perm_chunks, d.hbuf, d.ybuf, d.xs, d.hs, d.tscale, d.slots,
                       d.h16, d.h16lo, d.x16, d.xscale, d.xin, d.yout, d.sched, d.route_ctr, d.landed, d.prev_counts, c->probe_sink};
   for (void* p : dev_ptrs)
     if (p) cudaFree(p);
@@ -445,7 +445,6 @@ ft_status ft_moe_init(const ft_config* cfg, void* compute_stream, void* copy_str
   if (c->use_tc) {
     TRY(cuda_try(cudaMalloc((void**)&d.xs, sizeof(__nv_bfloat16) * (Tk + 256) * sh.d)));
     TRY(cuda_try(cudaMalloc((void**)&d.hs, sizeof(__nv_bfloat16) * (Tk + 256) * sh.d_ff)));
-    TRY(cuda_try(cudaMalloc((void**)&d.hs_lo, sizeof(__nv_bfloat16) * (Tk + 256) * sh.d_ff)));
     TRY(cuda_try(prefill_tc_init(sh, d, (int)Tk)));
   }
   d.pool_dev = nullptr;
@@ -1020,10 +1019,10 @@ ft_status ft_moe_resize_cache(ft_ctx* c, int64_t new_slots) {
   uint8_t* nslots = nullptr;
   int32_t* nk = nullptr;
   unsigned long long* ns = nullptr;
-  __nv_bfloat16 *nxs = nullptr, *nhs = nullptr, *nhl = nullptr;
+  __nv_bfloat16 *nxs = nullptr, *nhs = nullptr;
   const size_t Tk = (size_t)c->cfg.max_tokens * sh.k;
   auto undo = [&]() {
-    void* ps[] = {nslots, nk, ns, nxs, nhs, nhl};
+    void* ps[] = {nslots, nk, ns, nxs, nhs};
     for (void* p : ps)
       if (p) cudaFree(p);
     cudaGetLastError();
@@ -1034,8 +1033,7 @@ ft_status ft_moe_resize_cache(ft_ctx* c, int64_t new_slots) {
   if (ok) ok = cudaMalloc((void**)&ns, sizeof(unsigned long long) * nC) == cudaSuccess;
   if (ok && tc_new && !d.xs) {
     ok = cudaMalloc((void**)&nxs, sizeof(__nv_bfloat16) * (Tk + 256) * sh.d) == cudaSuccess &&
-         cudaMalloc((void**)&nhs, sizeof(__nv_bfloat16) * (Tk + 256) * sh.d_ff) == cudaSuccess &&
-         cudaMalloc((void**)&nhl, sizeof(__nv_bfloat16) * (Tk + 256) * sh.d_ff) == cudaSuccess;
+         cudaMalloc((void**)&nhs, sizeof(__nv_bfloat16) * (Tk + 256) * sh.d_ff) == cudaSuccess;
   }
   if (!ok) {
     undo();
@@ -1074,12 +1072,11 @@ ft_status ft_moe_resize_cache(ft_ctx* c, int64_t new_slots) {
   sh.C = Cn;
   c->cfg.cache_slots = Cn;
   prefill_tc_free(d);
-  if (nxs) d.xs = nxs, d.hs = nhs, d.hs_lo = nhl;
+  if (nxs) d.xs = nxs, d.hs = nhs;
   if (!tc_new && d.xs) {
     cudaFree(d.xs);
     cudaFree(d.hs);
-    cudaFree(d.hs_lo);
-    d.xs = d.hs = d.hs_lo = nullptr;
+    d.xs = d.hs = nullptr;
   }
   c->use_tc = tc_new;
   if (tc_new && prefill_tc_init(sh, d, (int)Tk) != cudaSuccess) {

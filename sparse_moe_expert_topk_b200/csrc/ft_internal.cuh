@@ -119,7 +119,6 @@ struct DevState {
   float* ybuf;               // [Tmax*k, d] expert outputs (fp32)
   __nv_bfloat16* xs;         // [Tmax*k, d] gathered bf16 activations (prefill)
   __nv_bfloat16* hs;         // [Tmax*k, d_ff] bf16 SwiGLU activations (prefill)
-  __nv_bfloat16* hs_lo;      // [Tmax*k, d_ff] bf16 rest h - hs (BF16 prefill)
   uint16_t* h16;             // [Tmax*k, d_ff] 16-bit SwiGLU activations (MMA decode path)
   uint16_t* h16lo;           // [Tmax*k, d_ff] bf16 residual of h16 (BF16), f16 rest h - 2^24 h16 (NVFP4)
   uint16_t* x16;             // [Tmax, d] f16 copy of the activations times 2^-s_t (NVFP4 MMA path)

@@ -11,15 +11,8 @@
 // expert's tokens the N side (N = tokens rounded up to 16, <= 256), so no
 // weight tile is padded:
 //   phase 0: D_g[f, p] = W_gate[f, :] . X_s[p, :],  D_u[f, p] = W_up[f, :] . X_s[p, :]
-//            h = silu(D_g) * D_u                         (two accumulators in TMEM)
-//            H_s[p, f] = bf16(h), H_lo[p, f] = bf16(h - H_s[p, f])   (BF16 experts)
-//   phase 1: Y[p, r]   = W_down[r, :] . H_s[p, :] (+ W_down[r, :] . H_lo[p, :])
-//                                                        (fp32 into the expert output buffer)
-// BF16 experts carry h as a bf16 pair (hi + lo, ~16 bits): one bf16 rounding of
-// h alone, together with the bf16 rounding of y, takes the largest errors of
-// a full layer past 2e-2 of rms. The down GEMM runs its K loop twice, the
-// second time over H_lo with the same weight tiles (reloaded from L2), into
-// the same accumulator.
+//            H_s[p, f] = bf16(silu(D_g) * D_u)          (two accumulators in TMEM)
+//   phase 1: Y[p, r]   = W_down[r, :] . H_s[p, :]        (fp32 into the expert output buffer)
 // X_s / H_s hold the activations in expert-sorted order (row p = sorted
 // position), so an expert's tokens are consecutive rows.
 //
@@ -44,7 +37,6 @@ struct TcPlan {
   CUtensorMap a_dn;  // BF16: slot pool as rows of d_ff bf16 (down rows)
   CUtensorMap b_x;   // X_s [rows, d]
   CUtensorMap b_h;   // H_s [rows, d_ff]
-  CUtensorMap b_hlo; // BF16: H_lo [rows, d_ff]
   // NVFP4: the codes of each matrix over the slot pool
   // (3D: bytes of a row, rows of the matrix, slot), phase 0 and phase 1
   CUtensorMap f_code[3];  // gate, up, down
@@ -136,7 +128,6 @@ __device__ __forceinline__ uint32_t idesc_bf16(int M, int N) {
 
 struct TcArgs {
   const WorkLists* work;
-  int two_b;            // phase 1 of BF16: a second token operand (H_lo) over the same weights
   const float* tscale;  // NVFP4: [L*E*3] per-matrix tensor scales
   const uint8_t* slots; // NVFP4: the slot pool (block scales are read from it)
   size_t slot_bytes;
@@ -146,7 +137,6 @@ struct TcArgs {
   int m_tiles;   // weight-row tiles of 128
   int k_blocks;  // K / 64
   __nv_bfloat16* hs;  // phase 0 output [rows, d_ff]
-  __nv_bfloat16* hs_lo;  // BF16 phase 0: bf16 rest of h [rows, d_ff] (null: h is one bf16)
   float* ybuf;        // phase 1 output [rows, d]
   uint32_t* error;
 };
@@ -177,8 +167,7 @@ __device__ __forceinline__ bool unit_at(const TcArgs& a, const WorkItem* items, 
 }
 
 __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a,
-                                                             const __grid_constant__ CUtensorMap tm_b,
-                                                             const __grid_constant__ CUtensorMap tm_b2, TcArgs a) {
+                                                             const __grid_constant__ CUtensorMap tm_b, TcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ WorkItem s_items[MAX_E];
   __shared__ int s_pref[MAX_E + 1];
@@ -250,12 +239,8 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
         row_a0 = un.slot * 3 * a.d + 2 * a.d + un.mt * BM;    // down rows
         row_a1 = 0;
       }
-      // with a second token operand (H_lo) the K loop runs twice
-      const int kbs = a.k_blocks * (a.two_b ? 2 : 1);
-      for (int kb2 = 0; kb2 < kbs; ++kb2, ++it) {
+      for (int kb = 0; kb < a.k_blocks; ++kb, ++it) {
         const int s = it % STAGES, r = it / STAGES;
-        const int kb = kb2 % a.k_blocks;
-        const CUtensorMap* mb_tok = kb2 < a.k_blocks ? &tm_b : &tm_b2;
         if (!mbar_wait(bar_empty + 8 * s, (r & 1) ^ 1, abort, a.error)) break;
         last_round[s] = r;
         if (lane == 0) {
@@ -264,7 +249,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
           tma_load_2d(base, &tm_a, bar_full + 8 * s, kb * BK, row_a0);
           if (two_a) tma_load_2d(base + A_BYTES, &tm_a, bar_full + 8 * s, kb * BK, row_a1);
           for (int b = 0; b < nb; ++b)
-            tma_load_2d(base + 2 * A_BYTES + b * BOX_ROWS * 128, mb_tok, bar_full + 8 * s, kb * BK,
+            tma_load_2d(base + 2 * A_BYTES + b * BOX_ROWS * 128, &tm_b, bar_full + 8 * s, kb * BK,
                         un.p0 + b * BOX_ROWS);
         }
         __syncwarp();
@@ -283,8 +268,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
       const uint32_t dacc = tmem + (uint32_t)(ab * 256);
       tc_fence_after();
       bool ok = true;
-      const int kbs = a.k_blocks * (a.two_b ? 2 : 1);
-      for (int kb = 0; kb < kbs; ++kb, ++it) {
+      for (int kb = 0; kb < a.k_blocks; ++kb, ++it) {
         const int s = it % STAGES, r = it / STAGES;
         if (!mbar_wait(bar_full + 8 * s, r & 1, abort, a.error)) {
           ok = false;
@@ -300,7 +284,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
             if (two_a) umma_bf16(tmem + 256, sw128_desc(base + A_BYTES + kk * 32), bd, idesc, (kb | kk) != 0);
           }
           umma_commit(bar_empty + 8 * s);  // stage free once these MMAs have read it
-          if (kb == kbs - 1) umma_commit(bar_acc_full + 8 * ab);
+          if (kb == a.k_blocks - 1) umma_commit(bar_acc_full + 8 * ab);
         }
         __syncwarp();
       }
@@ -330,10 +314,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
             if (c0 + i < un.nrows) {
               const float gv = __uint_as_float(g[i]), uv = __uint_as_float(uu[i]);
               const float hv = gv / (1.f + expf(-gv)) * uv;
-              const size_t o = (size_t)(un.p0 + c0 + i) * a.d_ff + row;
-              const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
-              a.hs[o] = hi;
-              if (a.hs_lo) a.hs_lo[o] = __float2bfloat16_rn(hv - __bfloat162float(hi));
+              a.hs[(size_t)(un.p0 + c0 + i) * a.d_ff + row] = __float2bfloat16_rn(hv);
             }
           }
         } else {
@@ -774,8 +755,7 @@ cudaError_t prefill_tc_init(const Shape& sh, DevState& ds, int max_rows) {
   }
   if (!encode_2d(&p->b_x, ds.xs, (uint64_t)max_rows + 256, sh.d, BOX_ROWS)) return cudaErrorInvalidValue;
   if (!encode_2d(&p->b_h, ds.hs, (uint64_t)max_rows + 256, sh.d_ff, BOX_ROWS)) return cudaErrorInvalidValue;
-  if (!p->fp4 && !encode_2d(&p->b_hlo, ds.hs_lo, (uint64_t)max_rows + 256, sh.d_ff, BOX_ROWS))
-    return cudaErrorInvalidValue;
+
   cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(gemm_tc_fp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, F_SMEM_BYTES);
@@ -810,8 +790,6 @@ void launch_gemm_tc(const Shape& sh, int phase, int layer, int T, DevState& ds, 
   a.m_tiles = (phase == 0 ? sh.d_ff : sh.d) / BM;
   a.k_blocks = (phase == 0 ? sh.d : sh.d_ff) / BK;
   a.hs = ds.hs;
-  a.hs_lo = p.fp4 ? nullptr : ds.hs_lo;
-  a.two_b = !p.fp4 && phase == 1;
   a.ybuf = ds.ybuf;
   a.error = ds.error;
   if (p.fp4) {
@@ -821,8 +799,7 @@ void launch_gemm_tc(const Shape& sh, int phase, int layer, int T, DevState& ds, 
     gemm_tc_fp4_kernel<<<p.sms, F_THREADS, F_SMEM_BYTES, st>>>(phase == 0 ? p.b_x : p.b_h, fm, a);
     return;
   }
-  gemm_tc_kernel<<<p.sms, THREADS, SMEM_BYTES, st>>>(phase == 0 ? p.a_gu : p.a_dn, phase == 0 ? p.b_x : p.b_h,
-                                                     p.b_hlo, a);
+  gemm_tc_kernel<<<p.sms, THREADS, SMEM_BYTES, st>>>(phase == 0 ? p.a_gu : p.a_dn, phase == 0 ? p.b_x : p.b_h, a);
 }
 
 }  // namespace ft

@@ -75,12 +75,33 @@ def tol_for(wtype):
     return {ftgen.W_F32: 1e-4, ftgen.W_BF16: 2e-2, ftgen.W_NVFP4: 4e-2}[wtype]
 
 
+def half_ulp_bf16(v):
+    """Half the bf16 spacing at |v| (taken one bf16 step above |v|, so that a
+    value rounded up into the next binade is covered); 0 where v is 0."""
+    a = np.abs(np.asarray(v, np.float64)) * (1.0 + 2.0 ** -7)
+    out = np.zeros_like(a)
+    nz = a > 0
+    out[nz] = 2.0 ** (np.floor(np.log2(a[nz])) - 8)
+    return out
+
+
 def check_close(y_gpu, y_ref, wtype, what=""):
+    """Layer outputs against the oracle: max |gpu - oracle| <= tol * rms(oracle)
+    element by element, where the output type is bf16 (BF16 and NVFP4 experts)
+    plus half a bf16 step of the oracle's value: the layer's output is bf16 by
+    definition, and its own rounding of an element at five standard
+    deviations already reaches 2% of rms, whatever the arithmetic before it."""
     y_gpu = np.asarray(y_gpu, np.float64)
     rms = float(np.sqrt(np.mean(y_ref ** 2)))
-    err = float(np.max(np.abs(y_gpu - y_ref))) if y_ref.size else 0.0
-    assert err <= tol_for(wtype) * rms, f"{what}: max|d| {err:.3e} > {tol_for(wtype)} * rms {rms:.3e}"
-    return err / rms if rms > 0 else 0.0
+    if not y_ref.size:
+        return 0.0
+    d = np.abs(y_gpu - y_ref)
+    slack = half_ulp_bf16(y_ref) if wtype != ftgen.W_F32 else 0.0
+    bad = d > tol_for(wtype) * rms + slack
+    i = int(np.argmax(d - slack))
+    assert not bad.any(), (f"{what}: {int(bad.sum())} elements off; worst |d| {d.flat[i]:.3e} > {tol_for(wtype)} * "
+                           f"rms {rms:.3e} + half bf16 step {np.broadcast_to(slack, d.shape).flat[i]:.3e}")
+    return float(np.max(d)) / rms if rms > 0 else 0.0
 
 
 def check_route_weights(w_gpu, w_ref, x, w_router, what=""):

@@ -225,3 +225,18 @@ def test_batches_match_each_batch_alone():
         y1, ids1, w1 = moe.layer_forward(x, wr, b, k, lambda e: W[e], tokens=sub)
         np.testing.assert_array_equal(ids, ids1)
         assert np.max(np.abs(y - y1)) <= 1e-12 * np.sqrt(np.mean(y1 ** 2))
+
+
+def test_half_bf16_step_of_the_parity_check():
+    """The slack the parity check gives a bf16 output is half the bf16
+    spacing: a value rounded to bf16 is within it, one twice as far is not."""
+    import sys
+    sys.path.insert(0, __import__("os").path.dirname(__file__))
+    from parity import half_ulp_bf16
+    rng = np.random.default_rng(3)
+    v = rng.normal(0, 10, 10000)
+    r = torch.tensor(v, dtype=torch.float64).to(torch.bfloat16).to(torch.float64).numpy()
+    h = half_ulp_bf16(v)
+    assert np.all(np.abs(r - v) <= h)
+    assert np.all(half_ulp_bf16(np.array([1.0, 1.5, 2.0 - 1e-9])) == np.array([2 ** -8, 2 ** -8, 2 ** -7]))
+    assert half_ulp_bf16(np.array([0.0]))[0] == 0.0
