@@ -1080,283 +1080,6 @@ __global__ void __launch_bounds__(NW * 32) gemv_direct_kernel(MmaArgs a) {
   }
 }
 
-// ---------------------------------------------------------------------------
-// BF16 hit class, pipelined across units. The arithmetic is the direct-load
-// and ring kernels' (warp w takes the same K sub-range of every ring slice,
-// the MMAs of a warp run in step order, the warps reduce in warp order), so an
-// expert's output is bit-identical whichever kernel computes it. What changes
-// is when the weights are loaded: each warp keeps two batches of PU steps in
-// flight, and once its current unit has no step left to load it starts on the
-// next unit's first batch, so the loads stay in flight through the current
-// unit's reduction, epilogue and barriers instead of draining at every unit.
-// A CTA holds two tickets ahead (the next unit, fetched a unit earlier, and
-// the one after it), still in increasing order, so the deadlock argument of
-// the direct-load kernel holds: a CTA that holds an unstarted gate/up unit is
-// itself working on a gate/up unit, which never waits.
-// ---------------------------------------------------------------------------
-constexpr int PU = 4;  // weight steps per batch (two batches in flight per warp)
-
-// The K steps one warp takes in one unit, in the order its MMAs consume them
-// (geometry of the unit's phase passed in, to keep the state small).
-struct StepIter {
-  int j, s, hi;
-  __device__ __forceinline__ void init(const Geo& g, int w) {
-    j = 0;
-    const int ns = min(g.ss, g.steps);
-    s = (w * ns) / RING_WARPS;
-    hi = ((w + 1) * ns) / RING_WARPS;
-    skip(g, w);
-  }
-  __device__ __forceinline__ void skip(const Geo& g, int w) {
-    while (s >= hi && j + 1 < g.nsl) {
-      ++j;
-      const int b0 = j * g.ss, ns = min(g.ss, g.steps - b0);
-      s = b0 + (w * ns) / RING_WARPS;
-      hi = b0 + ((w + 1) * ns) / RING_WARPS;
-    }
-  }
-  __device__ __forceinline__ bool more() const { return s < hi; }
-  __device__ __forceinline__ int next(const Geo& g, int w) {
-    const int r = s++;
-    skip(g, w);
-    return r;
-  }
-};
-
-// Where one unit's weight rows and activations are, for one lane.
-struct HitUnit {
-  const uint8_t* ra;   // row g (gate row, or first down row) + this lane's 16-byte quarter
-  const uint8_t* rb2;  // row g + 8 of the tile (up row, or second down row)
-  int base, nt, rb, qi;
-  int flags;           // HU_VALID | HU_BAD | HU_DOWN
-};
-constexpr int HU_VALID = 1, HU_BAD = 2, HU_DOWN = 4;
-
-__device__ __forceinline__ HitUnit hit_unit(const MmaArgs& a, const WorkItem* items, const int* pref, int n_items,
-                                            int rb0, int rb1, int U0, int U1, int u, int g, int q) {
-  HitUnit h{};
-  if (u >= U0 + U1) return h;
-  const int phase = u < U0 ? 0 : 1;
-  int item, chunk;
-  unit_of(pref, n_items, phase == 0 ? rb0 : rb1, phase == 0 ? u : u - U0, item, chunk, h.rb, h.qi);
-  const WorkItem it = items[item];
-  const bool bad = it.slot < 0 || it.slot >= a.C;  // error already latched by the lookup
-  h.flags = HU_VALID | (bad ? HU_BAD : 0) | (phase ? HU_DOWN : 0);
-  h.base = it.tok_off + chunk * CHUNK;
-  h.nt = min(CHUNK, it.n_tok - chunk * CHUNK);
-  const uint8_t* blob = a.slots + (size_t)(bad ? 0 : it.slot) * a.slot_bytes;
-  const size_t n = (size_t)a.d * a.d_ff;
-  if (phase == 0) {
-    const size_t rbytes = (size_t)a.d * 2;
-    h.ra = blob + (size_t)(h.rb * 8 + g) * rbytes + q * 16;
-    h.rb2 = blob + n * 2 + (size_t)(h.rb * 8 + g) * rbytes + q * 16;
-  } else {
-    const size_t rbytes = (size_t)a.d_ff * 2;
-    h.ra = blob + n * 4 + (size_t)(h.rb * 16 + g) * rbytes + q * 16;
-    h.rb2 = h.ra + 8 * rbytes;
-  }
-  return h;
-}
-
-// Load the next PU steps of `it` (rows ra, rb2) into w / v; st[] = -1 past the end.
-__device__ __forceinline__ void hit_fill(StepIter& it, const Geo& geo, int warp, const HitUnit& hu, uint4 (&w)[PU],
-                                         uint4 (&v)[PU], int (&st)[PU]) {
-#pragma unroll
-  for (int i = 0; i < PU; ++i) {
-    st[i] = it.more() ? it.next(geo, warp) : -1;
-    if (st[i] >= 0) {  // the same for every lane of the warp
-      w[i] = ld_stream(hu.ra + (size_t)st[i] * 64);
-      v[i] = ld_stream(hu.rb2 + (size_t)st[i] * 64);
-    } else {
-      w[i] = v[i] = make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
-}
-
-template <int NB>
-__device__ __forceinline__ void hit_compute(bool down, const uint4 (&w)[PU], const uint4 (&v)[PU],
-                                            const int (&st)[PU], const uint16_t* const (&xr)[NB],
-                                            const uint16_t* const (&xl)[NB], int q, float (&acc)[NB][4]) {
-#pragma unroll
-  for (int i = 0; i < PU; ++i) {
-    if (st[i] < 0) continue;
-    if (!down)
-      bf16_step<NB, false>(w[i], v[i], xr, xl, st[i] * 32 + q * 8, acc);
-    else
-      bf16_step<NB, true>(w[i], v[i], xr, xl, st[i] * 32 + q * 8, acc);
-  }
-}
-
-template <int NB>
-__global__ void __launch_bounds__(RING_WARPS * 32, 1) gemv_hit_bf16_kernel(MmaArgs a) {
-  constexpr int NW = RING_WARPS;
-  __shared__ int s_pref[MAX_E + 1];
-  __shared__ WorkItem s_items[MAX_E];
-  __shared__ float red[NW * NB * 4 * 32];
-  __shared__ int s_tk[2];
-  const int n_items = a.work->n_items[a.cls];
-  if (n_items == 0) return;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, q = lane & 3;
-  for (int i = tid; i < n_items; i += blockDim.x) s_items[i] = a.work->items[a.cls][i];
-  __syncthreads();
-  if (warp == 0) {  // exclusive scan of the chunks per item
-    int carry = 0;
-    for (int b = 0; b < n_items; b += 32) {
-      const int i = b + lane;
-      const int c = i < n_items ? (s_items[i].n_tok + CHUNK - 1) / CHUNK : 0;
-      int incl = c;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      if (i < n_items) s_pref[i] = carry + incl - c;
-      carry += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (lane == 0) s_pref[n_items] = carry;
-  }
-  if (tid == 0) {
-    s_tk[0] = atomicAdd(a.ticket, 1);
-    s_tk[1] = atomicAdd(a.ticket, 1);
-  }
-  __syncthreads();
-  const int n_qi = s_pref[n_items];
-  const int rb0 = a.d_ff / 8, rb1 = a.d / 16;
-  const int U0 = n_qi * rb0, U1 = n_qi * rb1;
-  int tk_cur = s_tk[0], tk_nxt = s_tk[1];
-  const Geo geo0 = geo_of(a, 0, false), geo1 = geo_of(a, 1, false);
-
-  HitUnit cur = hit_unit(a, s_items, s_pref, n_items, rb0, rb1, U0, U1, tk_cur, g, q);
-  StepIter it_cur;
-  it_cur.init((cur.flags & HU_DOWN) ? geo1 : geo0, warp);
-  uint4 wA[PU], vA[PU], wB[PU], vB[PU];
-  int sA[PU], sB[PU];
-  if (cur.flags == HU_VALID || cur.flags == (HU_VALID | HU_DOWN))
-    hit_fill(it_cur, (cur.flags & HU_DOWN) ? geo1 : geo0, warp, cur, wA, vA, sA);
-  while (cur.flags & HU_VALID) {
-    const bool down = cur.flags & HU_DOWN, bad = cur.flags & HU_BAD;
-    const Geo& gc = down ? geo1 : geo0;
-    // the ticket after the next one, fetched while this unit runs
-    int tk_after = 0;
-    if (tid == 0) tk_after = atomicAdd(a.ticket, 1);
-    HitUnit nxt = hit_unit(a, s_items, s_pref, n_items, rb0, rb1, U0, U1, tk_nxt, g, q);
-    const Geo& gn = (nxt.flags & HU_DOWN) ? geo1 : geo0;
-    StepIter it_nxt;
-    it_nxt.init(gn, warp);
-    if (down) {
-      // every gate/up unit of this (item, chunk) must have published h
-      if (tid == 0) {
-        const long long t0 = clock64();
-        volatile int32_t* dn = a.done + cur.qi;
-        while (*dn < rb0) {
-          if (clock64() - t0 > WAIT_CYCLES) {
-            atomicExch(a.error, (uint32_t)DERR_TIMEOUT);
-            break;
-          }
-        }
-        __threadfence();
-      }
-      __syncthreads();
-    }
-    const uint16_t* xr[NB];
-    const uint16_t* xl[NB];
-#pragma unroll
-    for (int t = 0; t < NB; ++t) {
-      const int j = t * 8 + g;
-      const int pos = cur.base + (j < cur.nt ? j : 0);
-      if (!down) {
-        xr[t] = reinterpret_cast<const uint16_t*>(a.x) + (size_t)(a.perm[pos] / a.k) * a.d;
-        xl[t] = xr[t];
-      } else {
-        xr[t] = a.h16 + (size_t)pos * a.d_ff;
-        xl[t] = a.h16lo + (size_t)pos * a.d_ff;
-      }
-    }
-    float acc[NB][4];
-#pragma unroll
-    for (int t = 0; t < NB; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-    // batches of this unit; the batch after its last one is the next unit's first
-    bool first_in_B = false;
-    const bool pre = (nxt.flags & (HU_VALID | HU_BAD)) == HU_VALID;
-    if (!bad) {
-      for (;;) {
-        bool own = it_cur.more();
-        if (own)
-          hit_fill(it_cur, gc, warp, cur, wB, vB, sB);
-        else if (pre)
-          hit_fill(it_nxt, gn, warp, nxt, wB, vB, sB);
-        hit_compute<NB>(down, wA, vA, sA, xr, xl, q, acc);
-        if (!own) {
-          first_in_B = true;
-          break;
-        }
-        own = it_cur.more();
-        if (own)
-          hit_fill(it_cur, gc, warp, cur, wA, vA, sA);
-        else if (pre)
-          hit_fill(it_nxt, gn, warp, nxt, wA, vA, sA);
-        hit_compute<NB>(down, wB, vB, sB, xr, xl, q, acc);
-        if (!own) break;
-      }
-    } else if (pre) {
-      hit_fill(it_nxt, gn, warp, nxt, wA, vA, sA);
-    }
-    if (first_in_B) {
-#pragma unroll
-      for (int i = 0; i < PU; ++i) {
-        wA[i] = wB[i];
-        vA[i] = vB[i];
-        sA[i] = sB[i];
-      }
-    }
-    // split-K reduction over the warps, in warp order, and the epilogue
-#pragma unroll
-    for (int t = 0; t < NB; ++t)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) red[((warp * NB + t) * 4 + c) * 32 + lane] = acc[t][c];
-    __syncthreads();
-    if (warp == 0 && !bad) {
-      float v[NB][4];
-#pragma unroll
-      for (int t = 0; t < NB; ++t)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float x = red[(t * 4 + c) * 32 + lane];
-          for (int w = 1; w < NW; ++w) x += red[((w * NB + t) * 4 + c) * 32 + lane];
-          v[t][c] = x;
-        }
-#pragma unroll
-      for (int t = 0; t < NB; ++t) {
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const int j = t * 8 + 2 * q + c;
-          if (j >= cur.nt) continue;
-          const float v0 = v[t][c], v1 = v[t][2 + c];
-          if (!down) {
-            const size_t o = (size_t)(cur.base + j) * a.d_ff + cur.rb * 8 + g;
-            const float hv = v0 / (1.f + expf(-v0)) * v1;
-            const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
-            a.h16[o] = __bfloat16_as_ushort(hi);
-            a.h16lo[o] = __bfloat16_as_ushort(__float2bfloat16_rn(hv - __bfloat162float(hi)));
-          } else {
-            float* yr = a.ybuf + (size_t)(cur.base + j) * a.d;
-            yr[cur.rb * 16 + g] = v0;
-            yr[cur.rb * 16 + g + 8] = v1;
-          }
-        }
-      }
-      if (!down) __threadfence();  // publish h before the unit is counted done
-    }
-    if (tid == 0) s_tk[0] = tk_after;
-    __syncthreads();  // red is free; h of this unit is published; the new ticket is visible
-    if (tid == 0 && !down) atomicAdd(a.done + cur.qi, 1);
-    tk_nxt = s_tk[0];
-    cur = nxt;
-    it_cur = it_nxt;
-    __syncthreads();  // every thread has read the ticket before thread 0 writes the next one
-  }
-}
-
 // f16 copy of the bf16 activations for the NVFP4 experts' f16 MMAs, one CTA
 // per token: y[t] = f16(x[t] * 2^-s_t) and xscale[t] = 2^s_t, where the power
 // of two s_t brings max_i |x[t, i]| into [1, 2) (bf16 carries 8 significant
@@ -1424,17 +1147,6 @@ cudaError_t direct_setup(int sms) {
   return e;
 }
 
-int g_grid_hit[3] = {0, 0, 0};  // [NB]: resident CTAs of the pipelined BF16 hit kernel
-
-template <int NB>
-cudaError_t hit_setup(int sms) {
-  int per = 0;
-  const cudaError_t e =
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, gemv_hit_bf16_kernel<NB>, RING_WARPS * 32, 0);
-  g_grid_hit[NB] = sms * (per > 0 ? per : 1);
-  return e;
-}
-
 template <int NB, bool FP4>
 void launch_direct(int grid, const MmaArgs& a, cudaStream_t st) {
   constexpr int NW = warps_for<NB>();
@@ -1461,8 +1173,6 @@ cudaError_t gemv_mma_init(int device) {
   if (e == cudaSuccess) e = direct_setup<2, false>(sms);
   if (e == cudaSuccess) e = direct_setup<1, true>(sms);
   if (e == cudaSuccess) e = direct_setup<2, true>(sms);
-  if (e == cudaSuccess) e = hit_setup<1>(sms);
-  if (e == cudaSuccess) e = hit_setup<2>(sms);
   return e;
 }
 
