@@ -993,7 +993,7 @@ __device__ void direct_unit(const MmaArgs& a, const WorkItem& it, int chunk, int
     }
     if (PHASE == 0) __threadfence();  // publish h before the unit is counted done
   }
-  __syncthreads();  // red is reused by the next unit
+  // the caller's barrier ends the unit: red is reused by the next one
 }
 
 // Row tiles per unit: NVFP4 rows are a quarter of the BF16 bytes, so a unit
@@ -1015,7 +1015,7 @@ __global__ void __launch_bounds__(NW * 32) gemv_direct_kernel(MmaArgs a) {
   __shared__ int s_pref[MAX_E + 1];
   __shared__ WorkItem s_items[MAX_E];
   __shared__ float red[NW * RTM * NB * 4 * 32];
-  __shared__ int s_unit;
+  __shared__ int s_unit[2];  // this unit's ticket and the next one's, alternating
   const int n_items = a.work->n_items[a.cls];
   if (n_items == 0) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1041,10 +1041,10 @@ __global__ void __launch_bounds__(NW * 32) gemv_direct_kernel(MmaArgs a) {
   const int n_qi = s_pref[n_items];
   const int rb0 = a.d_ff / 8 / RT, rb1 = a.d / 16 / RT1;
   const int U0 = n_qi * rb0, U1 = n_qi * rb1;
-  if (tid == 0) s_unit = atomicAdd(a.ticket, 1);
+  if (tid == 0) s_unit[0] = atomicAdd(a.ticket, 1);
   __syncthreads();
-  for (;;) {
-    const int u = s_unit;
+  for (int i = 0;; ++i) {
+    const int u = s_unit[i & 1];
     if (u >= U0 + U1) break;
     // the next ticket is fetched while this unit runs (phase-0 tickets all
     // precede phase-1 ones, so holding one never blocks a waited-on unit)
@@ -1072,11 +1072,12 @@ __global__ void __launch_bounds__(NW * 32) gemv_direct_kernel(MmaArgs a) {
       if (!bad) direct_unit<NB, 1, FP4, NW, RT1>(a, it, chunk, rb, warp, lane, red);
     } else {
       if (!bad) direct_unit<NB, 0, FP4, NW, RT>(a, it, chunk, rb, warp, lane, red);
-      if (tid == 0) atomicAdd(a.done + qi, 1);
     }
-    __syncthreads();  // every thread has read s_unit
-    if (tid == 0) s_unit = nxt;
-    __syncthreads();
+    // the other entry held the previous unit's ticket, which every thread
+    // read before the last barrier: it is free for the next one
+    if (tid == 0) s_unit[(i + 1) & 1] = nxt;
+    __syncthreads();  // red is free; this unit's h is published; the next ticket is visible
+    if (tid == 0 && phase == 0) atomicAdd(a.done + qi, 1);
   }
 }
 

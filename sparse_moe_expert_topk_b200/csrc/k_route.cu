@@ -156,6 +156,52 @@ __device__ __forceinline__ void permute_body(const int32_t* __restrict__ ids, in
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int e = tid; e < E; e += 1024) cnt[e] = 0;
   __syncthreads();
+  if (n <= 32) {
+    // one warp holds every entry (decode at a few tokens): an entry's place
+    // among equal experts is the number of earlier lanes with its expert,
+    // the same stable order as the general path below
+    if (warp == 0) {
+      const bool valid = lane < n;
+      const int e = valid ? ids[lane] : E;
+      const unsigned same = __match_any_sync(0xffffffffu, e);
+      const int rank = __popc(same & ((1u << lane) - 1u));
+      if (valid && rank == 0) cnt[e] = __popc(same);
+      __syncwarp();
+      constexpr int PER = MAX_E / 32;
+      int local[PER], sum = 0;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        const int x = lane * PER + i;
+        local[i] = x < E ? cnt[x] : 0;
+        sum += local[i];
+      }
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int base = incl - sum;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        const int x = lane * PER + i;
+        if (x < E) {
+          off[x] = base;
+          offsets[x] = base;
+          counts[x] = local[i];
+        }
+        base += local[i];
+      }
+      if (lane == 31) offsets[E] = incl;
+      __syncwarp();
+      if (valid) {
+        const int pos = off[e] + rank;
+        perm[pos] = lane;
+        inv[lane] = pos;
+      }
+    }
+    return;
+  }
   for (int i = tid; i < n; i += 1024) atomicAdd(&cnt[ids[i]], 1);
   __syncthreads();
   if (warp == 0) {  // exclusive scan of cnt over E <= 512 entries, 16 per lane
@@ -256,16 +302,29 @@ __device__ void logits_bf16_block(const __nv_bfloat16* __restrict__ x, const __n
     const __nv_bfloat16* xr0 = x + (size_t)(t0 + (g < nt ? g : 0)) * d;
     const __nv_bfloat16* xr1 = x + (size_t)(t0 + (g + 8 < nt ? g + 8 : 0)) * d;
     float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    for (int s = s0; s < s1; ++s) {
-      const uint4 wa = __ldg(reinterpret_cast<const uint4*>(pa + (size_t)s * 64));
-      const uint4 wb = __ldg(reinterpret_cast<const uint4*>(pb + (size_t)s * 64));
-      const uint4 x0 = __ldg(reinterpret_cast<const uint4*>(xr0 + s * 32 + q * 8));
-      mma_bf16_16816(acc[0], wa.x, wb.x, wa.y, wb.y, x0.x, x0.y);
-      mma_bf16_16816(acc[0], wa.z, wb.z, wa.w, wb.w, x0.z, x0.w);
-      if (nt > 8) {
-        const uint4 x1 = __ldg(reinterpret_cast<const uint4*>(xr1 + s * 32 + q * 8));
-        mma_bf16_16816(acc[1], wa.x, wb.x, wa.y, wb.y, x1.x, x1.y);
-        mma_bf16_16816(acc[1], wa.z, wb.z, wa.w, wb.w, x1.z, x1.w);
+    // RU steps of router rows in flight, then their MMAs in step order (the
+    // order, and so every logit, is the one-step loop's)
+    constexpr int RU = 4;
+    for (int sb = s0; sb < s1; sb += RU) {
+      uint4 wa[RU], wb[RU];
+#pragma unroll
+      for (int u = 0; u < RU; ++u) {
+        const int s = sb + u < s1 ? sb + u : s1 - 1;
+        wa[u] = __ldg(reinterpret_cast<const uint4*>(pa + (size_t)s * 64));
+        wb[u] = __ldg(reinterpret_cast<const uint4*>(pb + (size_t)s * 64));
+      }
+#pragma unroll
+      for (int u = 0; u < RU; ++u) {
+        if (sb + u >= s1) break;
+        const int s = sb + u;
+        const uint4 x0 = __ldg(reinterpret_cast<const uint4*>(xr0 + s * 32 + q * 8));
+        mma_bf16_16816(acc[0], wa[u].x, wb[u].x, wa[u].y, wb[u].y, x0.x, x0.y);
+        mma_bf16_16816(acc[0], wa[u].z, wb[u].z, wa[u].w, wb[u].w, x0.z, x0.w);
+        if (nt > 8) {
+          const uint4 x1 = __ldg(reinterpret_cast<const uint4*>(xr1 + s * 32 + q * 8));
+          mma_bf16_16816(acc[1], wa[u].x, wb[u].x, wa[u].y, wb[u].y, x1.x, x1.y);
+          mma_bf16_16816(acc[1], wa[u].z, wb[u].z, wa[u].w, wb[u].w, x1.z, x1.w);
+        }
       }
     }
 #pragma unroll
