@@ -647,6 +647,67 @@ def run_mixed(args, wl, world, rank, local):
 
 
 # --------------------------------------------------------------------------
+# kernel microbenchmarks: every expert of one layer resident in its slot, so
+# the expert kernels read HBM only; per-kernel CUDA-event times from the
+# library's profiler, one JSON line per weight type. For the roofline
+# fractions of single kernels and for small ncu captures; not a bench line.
+def run_kernels(args, rank, local):
+    import dataclasses
+
+    import sparse_moe_expert_topk_b200 as ft
+    import ftgen
+    from ftgen.ctx import Harness
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    base = ftgen.workload("decode_bf16" if args.workload == "hit_gemv" else "prefill_bf16")
+    wts = {"bf16": ftgen.W_BF16, "nvfp4": ftgen.W_NVFP4}
+    for wname in args.wtypes.split(","):
+        E = args.experts
+        wl = dataclasses.replace(base, name=f"{args.workload}_{wname}", wtype=wts[wname], E=E, cache_slots=2 * E)
+        sizes = [int(t) for t in args.tokens.split(",")]
+        h = Harness(wl, max_tokens=max(max(sizes), 512), device=local)
+        x0 = ftgen.hidden(512, wl.d, wl.wtype, 1).to(device)
+        y0 = torch.empty_like(x0)
+        ft.ft_moe_layer_forward(h.ctx, 0, ft.FT_PREFILL, x0, 512, None, 0, y0)  # the whole layer into its slots
+        torch.cuda.synchronize(device)
+        decode = args.workload == "hit_gemv"
+        mode = ft.FT_DECODE if decode else ft.FT_PREFILL
+        bias = torch.as_tensor(ftgen.zipf_log_bias(E, 1.1, wl.seed("zipf"))).to(device) if decode else None
+        out = {}
+        for T in sizes:
+            n_in = args.calls if decode else 1
+            xs = [ftgen.hidden(T, wl.d, wl.wtype, 100 + i).to(device) for i in range(n_in)]
+            yT = torch.empty(T, wl.d, dtype=xs[0].dtype, device=device)
+            for i in range(args.warmup):
+                ft.ft_moe_layer_forward(h.ctx, 0, mode, xs[i % n_in], T, bias, 0, yT)
+            torch.cuda.synchronize(device)
+            ft.ft_moe_profile(h.ctx, True)
+            for i in range(args.calls):
+                ft.ft_moe_layer_forward(h.ctx, 0, mode, xs[i % n_in], T, bias, 0, yT)
+            prof = ft.ft_moe_profile_read(h.ctx)
+            ft.ft_moe_profile(h.ctx, False)
+            torch.cuda.synchronize(device)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(h.stream)
+            for i in range(args.calls):
+                ft.ft_moe_layer_forward(h.ctx, 0, mode, xs[i % n_in], T, bias, 0, yT)
+            e1.record(h.stream)
+            torch.cuda.synchronize(device)
+            r = {k: {"us_per_launch": round(v["ms"] * 1e3 / max(v["launches"], 1), 2),
+                     "GBps": round(v["bytes"] / max(v["ms"], 1e-9) / 1e6, 1),
+                     "TFLOPs": round(v["flops"] / max(v["ms"], 1e-9) / 1e9, 1),
+                     "MB_per_launch": round(v["bytes"] / max(v["launches"], 1) / 1e6, 2)} for k, v in prof.items()}
+            r["call_us"] = round(e0.elapsed_time(e1) * 1e3 / args.calls, 2)
+            r["misses"] = h.stats()["misses"]
+            out[str(T)] = r
+        h.close()
+        if rank == 0:
+            print(json.dumps({"workload": args.workload, "wtype": wname, "experts": E, "d": wl.d, "d_ff": wl.d_ff,
+                              "top_k": wl.k, "calls": args.calls, "kernels": out}), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -659,10 +720,19 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-mixed", action="store_true", help="skip the 43-layer mixed NVFP4 leg of the default line")
     ap.add_argument("--profile-only", action="store_true", help="one warm-up and one profiled step (for ncu)")
+    km = ap.add_argument_group("kernel microbenchmarks (--workload hit_gemv | prefill_gemm)")
+    km.add_argument("--wtypes", default="bf16,nvfp4", help="weight types, comma-separated")
+    km.add_argument("--experts", type=int, default=256, help="experts of the resident layer")
+    km.add_argument("--tokens", default="1,4,16", help="tokens per call, comma-separated")
+    km.add_argument("--calls", type=int, default=48, help="profiled calls per size")
     args = ap.parse_args()
     if args.warmup < 3 and not args.profile_only:
         raise SystemExit("--warmup must be >= 3")
 
+    if args.workload in ("hit_gemv", "prefill_gemm"):
+        if args.gpus != 1 or args.impl != "ours":
+            raise SystemExit("kernel microbenchmarks run on one GPU, our implementation only")
+        return run_kernels(args, 0, 0)
     import ftgen
     wl = ftgen.workload(args.workload)
     world, rank, local = dist_setup(args.gpus)
@@ -671,7 +741,8 @@ def main():
     if args.workload == "mixed_nvfp4" and args.impl == "ours":
         return run_mixed(args, wl, world, rank, local)
     if args.workload != "decode_bf16":
-        raise SystemExit("workloads: decode_bf16 (default), prefill_bf16, trace_nvfp4, mixed_nvfp4")
+        raise SystemExit("workloads: decode_bf16 (default), prefill_bf16, trace_nvfp4, mixed_nvfp4; "
+                         "kernel microbenchmarks: hit_gemv, prefill_gemm")
     if args.impl == "reference":
         r = run_reference(args, wl, world, rank)
         if world > 1:

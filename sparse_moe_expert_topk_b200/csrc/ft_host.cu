@@ -624,10 +624,19 @@ static ft_status layer_call(ft_ctx* c, int32_t layer, int32_t mode, const void* 
   la.bp_mbps = c->bp;
   la.bh_mbps = c->bh;
   d.pool_dev = c->pool_dev[layer];
-  if (c->use_mma && sh.wtype == FT_W_NVFP4 && !(full_prefill && c->use_tc)) {
+  // NVFP4 experts read an f16 copy of x; the fused routing writes it itself
+  const bool want_f16 = c->use_mma && sh.wtype == FT_W_NVFP4 && !(full_prefill && c->use_tc);
+  if (want_f16 && !fused_route) {
     launch_to_f16(x, T, sh.d, d.x16, d.xscale, cs);
     c->kernel_launches += 1;
   }
+  // this decode call's routing counts become the layer's record for the
+  // decode prefetch; the fused routing stores them itself unless a prefetch
+  // batch of this same layer (one-layer models) must still read the old ones
+  const int nxt_layer = (layer + 1) % sh.L;
+  const bool pf_reads_this = c->prefetch_on && c->has_prev[nxt_layer] && nxt_layer == layer;
+  const bool record_in_route = mode == FT_DECODE && fused_route && !full_prefill && !pf_reads_this;
+  if (record_in_route) la.record_counts = d.prev_counts + (size_t)layer * sh.E;
   int p = -1;
   if (rows_eids) {
     p = prof_begin(c, P_PERMUTE, cs, Tk * 16.0 + sh.E * 8.0);
@@ -637,7 +646,7 @@ static ft_status layer_call(ft_ctx* c, int32_t layer, int32_t mode, const void* 
     c->kernel_launches += 1 + n_perm;
   } else if (fused_route) {
     p = prof_begin(c, P_ROUTE_FUSED, cs, T * (double)sh.d * ab + sh.E * (double)sh.d * ab + sh.C * 8.0);
-    launch_route_decode(sh, x, c->router[layer], bias, bias_per_token, T, la, d, cs);
+    launch_route_decode(sh, x, c->router[layer], bias, bias_per_token, T, la, d, want_f16, cs);
     prof_end(c, p, cs);
     c->kernel_launches += 1;
   } else {
@@ -682,8 +691,9 @@ static ft_status layer_call(ft_ctx* c, int32_t layer, int32_t mode, const void* 
         prof_end(c, p, cs);
         c->kernel_launches += 1;
       }
-      CK(cudaMemcpyAsync(d.prev_counts + (size_t)layer * sh.E, d.counts, sizeof(int32_t) * sh.E,
-                         cudaMemcpyDeviceToDevice, cs));
+      if (!record_in_route)
+        CK(cudaMemcpyAsync(d.prev_counts + (size_t)layer * sh.E, d.counts, sizeof(int32_t) * sh.E,
+                           cudaMemcpyDeviceToDevice, cs));
       c->has_prev[layer] = 1;
     }
     CK(cudaEventRecord(c->ev_look, cs));

@@ -93,6 +93,7 @@ struct LookupArgs {
   int prefetch;       // 1: decode prefetch batch: resident experts are not touched, missing ones staged
                       //    while victims last, no lookup record, only the prefetched counter moves
   const int32_t* counts_src;  // routing counts of the batch (null: this call's)
+  int32_t* record_counts;     // fused decode routing: also store this call's routing counts here (null: no)
 };
 
 // Device pointers of a context.
@@ -148,7 +149,7 @@ int launch_permute(const Shape& sh, int T, DevState& ds, cudaStream_t st);  // r
 size_t perm_chunks_ints(int max_entries, int E);
 // decode routing in one launch (T <= 32): logits, top-k, permutation, lookup
 void launch_route_decode(const Shape& sh, const void* x, const void* w_router, const float* bias, int bias_per_token,
-                         int T, const LookupArgs& la, DevState& ds, cudaStream_t st);
+                         int T, const LookupArgs& la, DevState& ds, bool to_f16, cudaStream_t st);
 // one lookup batch; writes work lists, mailbox, counters
 void launch_lookup(const Shape& sh, const LookupArgs& a, DevState& ds, cudaStream_t st);
 // decode / fallback experts (SIMT grouped GEMV) for one work class;

@@ -401,7 +401,10 @@ __global__ void __launch_bounds__(WARPS * 32) expert_gemv_kernel(GemvArgs a, int
 }
 
 // y[t, :] = sum_{j<k} w[t, j] * Y[inv[t*k + j], :], ranks in order, fp32, one
-// rounding to the output type. grid: (T, ceil(d / (4*256))).
+// rounding to the output type. grid: (T, ceil(d / (4*256))). The weights and
+// row indices of up to eight ranks are loaded first, then their rows, then
+// the sums run in rank order: two dependent memory round trips per eight
+// ranks instead of two per rank, with the same arithmetic.
 template <typename OT>
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ ybuf, const float* __restrict__ wts,
                                                       const int32_t* __restrict__ inv, int k, int d,
@@ -410,13 +413,30 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
   const int c = (blockIdx.y * 256 + threadIdx.x) * 4;
   if (c >= d) return;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int j = 0; j < k; ++j) {
-    const float w = wts[(size_t)t * k + j];
-    const float4 v = *reinterpret_cast<const float4*>(ybuf + (size_t)inv[(size_t)t * k + j] * d + c);
-    acc.x = fmaf(w, v.x, acc.x);
-    acc.y = fmaf(w, v.y, acc.y);
-    acc.z = fmaf(w, v.z, acc.z);
-    acc.w = fmaf(w, v.w, acc.w);
+  constexpr int B = 8;
+  for (int j0 = 0; j0 < k; j0 += B) {
+    float w[B];
+    int r[B];
+    float4 v[B];
+#pragma unroll
+    for (int j = 0; j < B; ++j) {
+      if (j0 + j < k) {
+        w[j] = wts[(size_t)t * k + j0 + j];
+        r[j] = inv[(size_t)t * k + j0 + j];
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < B; ++j)
+      if (j0 + j < k) v[j] = *reinterpret_cast<const float4*>(ybuf + (size_t)r[j] * d + c);
+#pragma unroll
+    for (int j = 0; j < B; ++j) {
+      if (j0 + j < k) {
+        acc.x = fmaf(w[j], v[j].x, acc.x);
+        acc.y = fmaf(w[j], v[j].y, acc.y);
+        acc.z = fmaf(w[j], v[j].z, acc.z);
+        acc.w = fmaf(w[j], v[j].w, acc.w);
+      }
+    }
   }
   if constexpr (sizeof(OT) == 4) {
     *reinterpret_cast<float4*>(y + (size_t)t * d + c) = acc;

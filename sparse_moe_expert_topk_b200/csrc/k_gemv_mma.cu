@@ -61,6 +61,7 @@
 // below 2^19 (at d = 4096 that is a mean |weight| up to 128).
 #include <cuda_fp16.h>
 
+#include "f16_scale.cuh"
 #include "ft_internal.cuh"
 #include "mbarrier.cuh"
 
@@ -1003,19 +1004,25 @@ template <bool FP4>
 constexpr int tiles_for() { return FP4 ? 4 : 1; }
 // NVFP4 down units carry two accumulators (the two terms of h), so they take
 // two row tiles, which keeps the kernel's registers where four gate/up tiles
-// put them (a unit's row tiles change which rows it covers, not the K order
-// of any row, so results do not depend on this choice).
-template <bool FP4>
+// put them (four measured slower: fewer, longer units and spills). A unit's
+// row tiles change which rows it covers, not the K order of any row, so
+// results do not depend on this choice.
+template <bool FP4, int NB>
 constexpr int tiles_down_for() { return FP4 ? 2 : 4; }
 
 template <int NB, bool FP4, int NW>
 __global__ void __launch_bounds__(NW * 32) gemv_direct_kernel(MmaArgs a) {
-  constexpr int RT = tiles_for<FP4>(), RT1 = tiles_down_for<FP4>();
+  constexpr int RT = tiles_for<FP4>(), RT1 = tiles_down_for<FP4, NB>();
   constexpr int RTM = RT > RT1 ? RT : RT1;
   __shared__ int s_pref[MAX_E + 1];
   __shared__ WorkItem s_items[MAX_E];
   __shared__ float red[NW * RTM * NB * 4 * 32];
-  __shared__ int s_unit[2];  // this unit's ticket and the next one's, alternating
+  // Tickets taken ahead of the unit being worked on: two for BF16 (measured
+  // faster than one), one for NVFP4, whose gate/up units fill about one wave
+  // at a few tokens, so a second early ticket would stack two of them on some
+  // CTAs while others wait for their h.
+  constexpr int AHEAD = FP4 ? 1 : 2;
+  __shared__ int s_unit[AHEAD + 1];  // tickets of this unit and the ones after it, in rotation
   const int n_items = a.work->n_items[a.cls];
   if (n_items == 0) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1041,13 +1048,17 @@ __global__ void __launch_bounds__(NW * 32) gemv_direct_kernel(MmaArgs a) {
   const int n_qi = s_pref[n_items];
   const int rb0 = a.d_ff / 8 / RT, rb1 = a.d / 16 / RT1;
   const int U0 = n_qi * rb0, U1 = n_qi * rb1;
-  if (tid == 0) s_unit[0] = atomicAdd(a.ticket, 1);
+  if (tid == 0)
+    for (int j = 0; j < AHEAD; ++j) s_unit[j] = atomicAdd(a.ticket, 1);
   __syncthreads();
   for (int i = 0;; ++i) {
-    const int u = s_unit[i & 1];
+    const int u = s_unit[i % (AHEAD + 1)];
     if (u >= U0 + U1) break;
-    // the next ticket is fetched while this unit runs (phase-0 tickets all
-    // precede phase-1 ones, so holding one never blocks a waited-on unit)
+    // The next ticket of the rotation is fetched while this unit runs.
+    // Tickets are taken in increasing order and phase-0 tickets all precede
+    // phase-1 ones, so a CTA waiting in a phase-1 unit holds no phase-0
+    // ticket: every waited-on unit is running or held by a CTA that runs it
+    // without waiting.
     int nxt = 0;
     if (tid == 0) nxt = atomicAdd(a.ticket, 1);
     const int phase = u < U0 ? 0 : 1;
@@ -1073,44 +1084,21 @@ __global__ void __launch_bounds__(NW * 32) gemv_direct_kernel(MmaArgs a) {
     } else {
       if (!bad) direct_unit<NB, 0, FP4, NW, RT>(a, it, chunk, rb, warp, lane, red);
     }
-    // the other entry held the previous unit's ticket, which every thread
-    // read before the last barrier: it is free for the next one
-    if (tid == 0) s_unit[(i + 1) & 1] = nxt;
+    // entry (i + AHEAD) % (AHEAD + 1) held the previous unit's ticket, which
+    // every thread read before the last barrier: it is free for the new one
+    if (tid == 0) s_unit[(i + AHEAD) % (AHEAD + 1)] = nxt;
     __syncthreads();  // red is free; this unit's h is published; the next ticket is visible
     if (tid == 0 && phase == 0) atomicAdd(a.done + qi, 1);
   }
 }
 
 // f16 copy of the bf16 activations for the NVFP4 experts' f16 MMAs, one CTA
-// per token: y[t] = f16(x[t] * 2^-s_t) and xscale[t] = 2^s_t, where the power
-// of two s_t brings max_i |x[t, i]| into [1, 2) (bf16 carries 8 significant
-// bits, so every element down to 2^-14 of the largest is exact in f16; the
-// smaller ones, below 2^-14 of the largest, keep an absolute error under
-// 2^-25 of it). A token of zeros keeps s_t = 0; s_t is held to [-60, 60], so
-// that xscale^2 is an fp32 power of two; non-finite values pass through.
+// per token (to_f16_scaled_row gives the scaling rule).
 __global__ void __launch_bounds__(256) to_f16_scaled_kernel(const __nv_bfloat16* __restrict__ x, int d,
                                                             __half* __restrict__ y, float* __restrict__ xscale) {
   __shared__ float s_max[8];
   const int t = blockIdx.x;
-  const __nv_bfloat16* xr = x + (size_t)t * d;
-  float m = 0.f;
-  for (int i = threadIdx.x; i < d; i += 256) m = fmaxf(m, fabsf(__bfloat162float(xr[i])));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if ((threadIdx.x & 31) == 0) s_max[threadIdx.x >> 5] = m;
-  __syncthreads();
-  m = s_max[0];
-#pragma unroll
-  for (int w = 1; w < 8; ++w) m = fmaxf(m, s_max[w]);
-  int sh = 0;
-  if (m > 0.f && m <= 3.0e38f) {
-    int e;
-    frexpf(m, &e);  // m = f * 2^e, f in [0.5, 1)
-    sh = min(60, max(-60, e - 1));
-  }
-  const float down = ldexpf(1.f, -sh);
-  for (int i = threadIdx.x; i < d; i += 256) y[(size_t)t * d + i] = __float2half_rn(__bfloat162float(xr[i]) * down);
-  if (threadIdx.x == 0) xscale[t] = ldexpf(1.f, sh);
+  to_f16_scaled_row<256>(x + (size_t)t * d, d, y + (size_t)t * d, xscale + t, s_max);
 }
 
 int g_grid[2][3] = {{0, 0, 0}, {0, 0, 0}};  // [fp4][NB]: resident CTAs (one per SM)
@@ -1212,8 +1200,8 @@ void launch_gemv_mma(const Shape& sh, int cls, int layer, const void* x16, int T
   const int NB = T > 8 ? 2 : 1;
   const long long chunks = (long long)max_items + (long long)max_tok / CHUNK;
   if (cls == KIND_HIT) {
-    const long long units = chunks * (fp4 ? sh.d_ff / 8 / tiles_for<true>() + sh.d / 16 / tiles_down_for<true>()
-                                          : sh.d_ff / 8 / tiles_for<false>() + sh.d / 16 / tiles_down_for<false>());
+    const int rt1 = fp4 ? (NB == 1 ? tiles_down_for<true, 1>() : tiles_down_for<true, 2>()) : tiles_down_for<false, 1>();
+    const long long units = chunks * (sh.d_ff / 8 / (fp4 ? tiles_for<true>() : tiles_for<false>()) + sh.d / 16 / rt1);
     const int cap = g_grid_direct[fp4][NB];
     const int grid = (int)(units < cap ? units : cap);
     if (grid <= 0) return;

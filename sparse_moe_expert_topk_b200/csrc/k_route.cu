@@ -8,6 +8,9 @@
 // expert index), softmax over those k.
 #include <atomic>
 
+#include <cooperative_groups.h>
+
+#include "f16_scale.cuh"
 #include "lookup_body.cuh"
 
 namespace ft {
@@ -79,9 +82,14 @@ __global__ void __launch_bounds__(256) router_scores_kernel(const AT* __restrict
 }
 
 // One warp per token: k rounds of a warp arg-max (larger logit first, equal
-// logits -> lower index), then softmax over the chosen k.
+// logits -> lower index), then softmax over the chosen k. SHARED: the scores
+// are in this CTA's shared memory (the cluster routing), else in global
+// memory, read through L2 (other CTAs of the same launch may have written
+// them). ids_sh, if set, receives a copy of the ids (shared memory).
+template <bool SHARED = false>
 __device__ __forceinline__ void topk_token(const float* __restrict__ scores, int warp, int E, int k,
-                                           int32_t* __restrict__ ids, float* __restrict__ wts, int lane) {
+                                           int32_t* __restrict__ ids, float* __restrict__ wts, int lane,
+                                           int32_t* ids_sh = nullptr) {
   constexpr int PER = MAX_E / 32;
   float v[PER];
   uint32_t taken = 0;
@@ -89,7 +97,10 @@ __device__ __forceinline__ void topk_token(const float* __restrict__ scores, int
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int e = i * 32 + lane;
-    v[i] = e < E ? __ldcg(s + e) : 0.f;  // L2: in the fused kernel other CTAs wrote these
+    if constexpr (SHARED)
+      v[i] = e < E ? s[e] : 0.f;
+    else
+      v[i] = e < E ? __ldcg(s + e) : 0.f;
   }
   // lane j keeps the j-th pick, so nothing is indexed by the runtime k
   float top0 = 0.f, my_s = 0.f;
@@ -130,6 +141,7 @@ __device__ __forceinline__ void topk_token(const float* __restrict__ scores, int
   if (lane < k) {
     ids[(size_t)warp * k + lane] = my_e;
     wts[(size_t)warp * k + lane] = ex / den;
+    if (ids_sh) ids_sh[warp * k + lane] = my_e;
   }
 }
 
@@ -423,17 +435,21 @@ __global__ void __launch_bounds__(128) router_mma_kernel(const __nv_bfloat16* __
 }
 
 // Decode routing in one launch (T <= 32 tokens): CTAs of 32 warps compute the
-// logits of 32 experts each (one warp per expert, all tokens); the last CTA to
-// finish (ticket on ds.route_ctr) runs top-k + softmax, the stable
-// permutation and the LRU lookup of the layer. Same device code as the
-// separate kernels, so the results are the same.
+// logits of 16 (BF16) or 32 (fp32) experts each; the last CTA to finish
+// (ticket on ds.route_ctr) runs top-k + softmax, the stable permutation and
+// the LRU lookup of the layer. Same device code as the separate kernels, so
+// the results are the same. With x16 set (NVFP4 experts), CTA b also writes
+// the f16 copy of tokens b, b + grid, ... (to_f16_scaled_row, as the
+// standalone conversion kernel does).
 template <typename AT>
 __global__ void __launch_bounds__(1024) route_decode_kernel(const AT* __restrict__ x, const AT* __restrict__ wr,
                                                             const float* __restrict__ bias, int bias_per_token, int T,
                                                             int E, int d, int k, LookupArgs la, long long C,
-                                                            size_t slot_bytes, DevState ds) {
+                                                            size_t slot_bytes, DevState ds, __half* x16,
+                                                            float* xscale) {
   extern __shared__ int32_t smem[];
   __shared__ int s_last;
+  __shared__ float s_max[32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if constexpr (sizeof(AT) == 2) {
     // BF16: 16 experts per CTA on the tensor cores (red reuses the dynamic smem)
@@ -487,6 +503,13 @@ __global__ void __launch_bounds__(1024) route_decode_kernel(const AT* __restrict
       }
     }
   }
+  if constexpr (sizeof(AT) == 2) {
+    if (x16) {
+      for (int t = blockIdx.x; t < T; t += gridDim.x)
+        to_f16_scaled_row<1024>(reinterpret_cast<const __nv_bfloat16*>(x) + (size_t)t * d, d, x16 + (size_t)t * d,
+                                xscale + t, s_max);
+    }
+  }
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) s_last = atomicAdd(ds.route_ctr, 1) == (int)gridDim.x - 1;
@@ -498,9 +521,56 @@ __global__ void __launch_bounds__(1024) route_decode_kernel(const AT* __restrict
   permute_body(ds.ids, T * k, E, ds.counts, ds.offsets, ds.perm, ds.inv, smem);
   __syncthreads();
   // counts and offsets are still in this CTA's shared memory (permute_body)
+  if (la.record_counts)
+    for (int e = threadIdx.x; e < E; e += blockDim.x) la.record_counts[e] = smem[34 * E + e];
   lookup_detail::lookup_body(la, E, C, slot_bytes, ds, smem + 34 * E, smem + 35 * E);
   if (threadIdx.x == 0) *ds.route_ctr = 0;  // ready for the next call
 }
+
+// Decode routing (T <= 32, BF16 router, E <= 256) as one thread-block
+// cluster of ceil(E/16) CTAs: CTA r computes the logits of experts 16r ..
+// 16r+15 (logits_bf16_block, the same sums as the other small-batch router
+// paths) and stores them straight into the shared memory of CTA 0; one
+// cluster barrier publishes them, and CTA 0 runs top-k + softmax, the stable
+// permutation and the LRU lookup with the scores and ids in its own shared
+// memory. No global round trip, fence or ticket between the logits and the
+// lookup. With x16 set (NVFP4 experts), CTA r also writes the f16 copy of
+// tokens r, r + grid, ...
+// Dynamic shared memory: [0, sc_off) the logits' partial sums and later the
+// permutation's tables, [sc_off, sc_off + 4*T*E) the scores (CTA 0's).
+__global__ void __launch_bounds__(1024) route_cluster_kernel(const __nv_bfloat16* __restrict__ x,
+                                                             const __nv_bfloat16* __restrict__ wr,
+                                                             const float* __restrict__ bias, int bias_per_token, int T,
+                                                             int E, int d, int k, LookupArgs la, long long C,
+                                                             size_t slot_bytes, DevState ds, __half* x16,
+                                                             float* xscale, int sc_off) {
+  namespace cg = cooperative_groups;
+  extern __shared__ __align__(16) int32_t smem[];
+  __shared__ float s_max[32];
+  __shared__ int32_t s_ids[32 * MAX_K];
+  cg::cluster_group cl = cg::this_cluster();
+  const unsigned rank = cl.block_rank();
+  float* scores = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(smem) + sc_off);
+  float* scores0 = cl.map_shared_rank(scores, 0);
+  cl.sync();  // every CTA of the cluster runs before its shared memory is written
+  logits_bf16_block(x, wr, bias, bias_per_token, T, E, d, (int)rank * 16, scores0, reinterpret_cast<float*>(smem));
+  if (x16) {
+    for (int t = (int)rank; t < T; t += (int)cl.num_blocks())
+      to_f16_scaled_row<1024>(x + (size_t)t * d, d, x16 + (size_t)t * d, xscale + t, s_max);
+  }
+  cl.sync();  // the scores are in CTA 0
+  if (rank != 0) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp < T) topk_token<true>(scores, warp, E, k, ds.ids, ds.wts, lane, s_ids);
+  __syncthreads();
+  permute_body(s_ids, T * k, E, ds.counts, ds.offsets, ds.perm, ds.inv, smem);
+  __syncthreads();
+  if (la.record_counts)
+    for (int e = threadIdx.x; e < E; e += blockDim.x) la.record_counts[e] = smem[34 * E + e];
+  lookup_detail::lookup_body(la, E, C, slot_bytes, ds, smem + 34 * E, smem + 35 * E);
+}
+
+bool g_route_cluster = false;  // cluster launches of 16 x 1024 threads fit on this device
 
 }  // namespace
 
@@ -691,18 +761,45 @@ size_t route_decode_smem(int E) {
   return red > perm ? red : perm;
 }
 
+static size_t route_cluster_sc_off(int E) {
+  const size_t red = sizeof(float) * 32 * 8 * 32, perm = permute_smem_bytes(E);
+  return ((red > perm ? red : perm) + 15) & ~size_t(15);
+}
+constexpr int CLUSTER_MAX_E = 256;  // 16 CTAs of 16 experts
+constexpr int CLUSTER_MAX_T = 32;
+
 void launch_route_decode(const Shape& sh, const void* x, const void* w_router, const float* bias, int bias_per_token,
-                         int T, const LookupArgs& la, DevState& ds, cudaStream_t st) {
+                         int T, const LookupArgs& la, DevState& ds, bool to_f16, cudaStream_t st) {
+  if (sh.wtype != FT_W_F32 && g_route_cluster && sh.E <= CLUSTER_MAX_E && T <= CLUSTER_MAX_T) {
+    const int cs = (sh.E + 15) / 16;
+    const int sc_off = (int)route_cluster_sc_off(sh.E);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cs, 1, 1);
+    cfg.blockDim = dim3(1024, 1, 1);
+    cfg.dynamicSmemBytes = sc_off + sizeof(float) * (size_t)T * sh.E;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, route_cluster_kernel, (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_router, bias,
+                       bias_per_token, T, sh.E, sh.d, sh.k, la, sh.C, sh.slot_bytes, ds,
+                       to_f16 ? reinterpret_cast<__half*>(ds.x16) : nullptr, to_f16 ? ds.xscale : nullptr, sc_off);
+    return;
+  }
   const int grid = sh.wtype == FT_W_F32 ? (sh.E + 31) / 32 : (sh.E + 15) / 16;
   const size_t smem = route_decode_smem(sh.E);
   if (sh.wtype == FT_W_F32)
     route_decode_kernel<float><<<grid, 1024, smem, st>>>((const float*)x, (const float*)w_router, bias,
                                                          bias_per_token, T, sh.E, sh.d, sh.k, la, sh.C, sh.slot_bytes,
-                                                         ds);
+                                                         ds, nullptr, nullptr);
   else
-    route_decode_kernel<__nv_bfloat16><<<grid, 1024, smem, st>>>((const __nv_bfloat16*)x,
-                                                                 (const __nv_bfloat16*)w_router, bias, bias_per_token,
-                                                                 T, sh.E, sh.d, sh.k, la, sh.C, sh.slot_bytes, ds);
+    route_decode_kernel<__nv_bfloat16><<<grid, 1024, smem, st>>>(
+        (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_router, bias, bias_per_token, T, sh.E, sh.d, sh.k, la, sh.C,
+        sh.slot_bytes, ds, to_f16 ? reinterpret_cast<__half*>(ds.x16) : nullptr, to_f16 ? ds.xscale : nullptr);
 }
 
 // Dynamic shared-memory limits of the permutation and fused routing kernels,
@@ -723,6 +820,29 @@ cudaError_t route_kernels_init() {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(route_decode_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem_f);
+  // the cluster routing: 16 CTAs of 1024 threads (a non-portable cluster
+  // size), used only if such a cluster fits on the device
+  const int smem_c = (int)(route_cluster_sc_off(CLUSTER_MAX_E) + sizeof(float) * CLUSTER_MAX_T * CLUSTER_MAX_E);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(route_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_c);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(route_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(16, 1, 1);
+    cfg.blockDim = dim3(1024, 1, 1);
+    cfg.dynamicSmemBytes = smem_c;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 16;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    const cudaError_t q = cudaOccupancyMaxActiveClusters(&n, route_cluster_kernel, &cfg);
+    g_route_cluster = q == cudaSuccess && n >= 1;
+    if (q != cudaSuccess) (void)cudaGetLastError();  // not fatal: the other routing kernel stays in use
+  }
   return e;
 }
 

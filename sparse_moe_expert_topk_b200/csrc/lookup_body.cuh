@@ -109,6 +109,7 @@ __device__ __forceinline__ void lookup_body(const LookupArgs& a, int E, long lon
   const bool pf = a.prefetch != 0;
   const int32_t* offsets = s_offsets ? s_offsets : ds.offsets;
   __shared__ int s_e[MAX_E];
+  __shared__ int s_slot_of[MAX_E];
   __shared__ int s_slot[MAX_E];
   __shared__ int s_vic[MAX_E];
   __shared__ unsigned long long s_cand[MAX_E];
@@ -123,12 +124,26 @@ __device__ __forceinline__ void lookup_body(const LookupArgs& a, int E, long lon
   const int tid = threadIdx.x;
   Mailbox* mb = ds.mbox;
   const int layer = a.layer;
+  // the loads every later step depends on go out first, so that their
+  // latency overlaps the batch scan: each expert's slot, and the clock
+  const int my_slot = tid < E ? ds.slot_of[layer * E + tid] : -1;
+  unsigned long long clk0 = 0, bstart0 = 0;
+  int cbase0 = 0, lbase0 = 0;
+  if (tid == 0) {
+    clk0 = ds.clk->clock;
+    bstart0 = ds.clk->batch_start;
+    if (a.append) {
+      cbase0 = mb->n_copy;
+      lbase0 = mb->n_lookup;
+    }
+  }
 
   // 1. the batch: routed experts (counts > 0) or all E, ascending
   const bool in = tid < E && (a.use_counts ? counts[tid] > 0 : true);
   int n_u;
   const int upos = block_scan_flag(in, scan, n_u);
   if (in) s_e[upos] = tid;
+  if (tid < E) s_slot_of[tid] = my_slot;
   __syncthreads();
 
   // 2. hits
@@ -137,7 +152,7 @@ __device__ __forceinline__ void lookup_body(const LookupArgs& a, int E, long lon
   if (act) {
     e = s_e[tid];
     key = layer * E + e;
-    sl = ds.slot_of[key];
+    sl = s_slot_of[e];
     if (sl >= C) {  // corrupt table: report and treat as a miss
       atomicExch(ds.error, (uint32_t)DERR_BAD_INDEX);
       sl = -1;
@@ -150,12 +165,11 @@ __device__ __forceinline__ void lookup_body(const LookupArgs& a, int E, long lon
 
   // 3. clock and pins
   if (tid == 0) {
-    const unsigned long long c0 = ds.clk->clock;
-    s_c0 = c0;
-    s_bstart = c0 + 1;
-    s_epoch = a.pin_prev ? ds.clk->batch_start : c0 + 1;
-    s_cbase = a.append ? mb->n_copy : 0;
-    s_lbase = a.append ? mb->n_lookup : 0;
+    s_c0 = clk0;
+    s_bstart = clk0 + 1;
+    s_epoch = a.pin_prev ? bstart0 : clk0 + 1;
+    s_cbase = cbase0;
+    s_lbase = lbase0;
   }
   __syncthreads();
   const unsigned long long c0 = s_c0, epoch = s_epoch;
