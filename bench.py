@@ -647,10 +647,14 @@ def run_mixed(args, wl, world, rank, local):
 
 
 # --------------------------------------------------------------------------
-# kernel microbenchmarks: every expert of one layer resident in its slot, so
-# the expert kernels read HBM only; per-kernel CUDA-event times from the
-# library's profiler, one JSON line per weight type. For the roofline
-# fractions of single kernels and for small ncu captures; not a bench line.
+# kernel microbenchmarks, one JSON line per weight type, per-kernel CUDA-event
+# times from the library's profiler; for the roofline fractions of single
+# kernels and for small ncu captures, not a bench line.
+#   hit_gemv, prefill_gemm: every expert of one layer resident in its slot,
+#     so the expert kernels read HBM only;
+#   stream_gemv: B_P = 0, so q* = 0 and every routed expert is streamed from
+#     the pinned pool (the cache stays empty): the streamed class alone on the
+#     host link, against the zero-copy read rate measured in the same run.
 def run_kernels(args, rank, local):
     import dataclasses
 
@@ -659,7 +663,7 @@ def run_kernels(args, rank, local):
     from ftgen.ctx import Harness
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    base = ftgen.workload("decode_bf16" if args.workload == "hit_gemv" else "prefill_bf16")
+    base = ftgen.workload("prefill_bf16" if args.workload == "prefill_gemm" else "decode_bf16")
     wts = {"bf16": ftgen.W_BF16, "nvfp4": ftgen.W_NVFP4}
     for wname in args.wtypes.split(","):
         E = args.experts
@@ -668,9 +672,15 @@ def run_kernels(args, rank, local):
         h = Harness(wl, max_tokens=max(max(sizes), 512), device=local)
         x0 = ftgen.hidden(512, wl.d, wl.wtype, 1).to(device)
         y0 = torch.empty_like(x0)
-        ft.ft_moe_layer_forward(h.ctx, 0, ft.FT_PREFILL, x0, 512, None, 0, y0)  # the whole layer into its slots
+        link = None
+        if args.workload == "stream_gemv":
+            ft.ft_set_bandwidths(h.ctx, 0, 77300)
+            h2d_gbs, zc_gbs = ft.ft_moe_probe_link(h.ctx, 1 << 30)
+            link = {"h2d_copy_gbs": round(h2d_gbs, 2), "zero_copy_read_gbs": round(zc_gbs, 2)}
+        else:
+            ft.ft_moe_layer_forward(h.ctx, 0, ft.FT_PREFILL, x0, 512, None, 0, y0)  # the whole layer into its slots
         torch.cuda.synchronize(device)
-        decode = args.workload == "hit_gemv"
+        decode = args.workload != "prefill_gemm"
         mode = ft.FT_DECODE if decode else ft.FT_PREFILL
         bias = torch.as_tensor(ftgen.zipf_log_bias(E, 1.1, wl.seed("zipf"))).to(device) if decode else None
         out = {}
@@ -699,11 +709,13 @@ def run_kernels(args, rank, local):
                      "MB_per_launch": round(v["bytes"] / max(v["launches"], 1) / 1e6, 2)} for k, v in prof.items()}
             r["call_us"] = round(e0.elapsed_time(e1) * 1e3 / args.calls, 2)
             r["misses"] = h.stats()["misses"]
+            if link and "gemv_streamed" in r:
+                r["gemv_streamed"]["frac_of_zero_copy"] = round(r["gemv_streamed"]["GBps"] / link["zero_copy_read_gbs"], 4)
             out[str(T)] = r
         h.close()
         if rank == 0:
             print(json.dumps({"workload": args.workload, "wtype": wname, "experts": E, "d": wl.d, "d_ff": wl.d_ff,
-                              "top_k": wl.k, "calls": args.calls, "kernels": out}), flush=True)
+                              "top_k": wl.k, "calls": args.calls, "host_link": link, "kernels": out}), flush=True)
     return 0
 
 
@@ -720,7 +732,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-mixed", action="store_true", help="skip the 43-layer mixed NVFP4 leg of the default line")
     ap.add_argument("--profile-only", action="store_true", help="one warm-up and one profiled step (for ncu)")
-    km = ap.add_argument_group("kernel microbenchmarks (--workload hit_gemv | prefill_gemm)")
+    km = ap.add_argument_group("kernel microbenchmarks (--workload hit_gemv | stream_gemv | prefill_gemm)")
     km.add_argument("--wtypes", default="bf16,nvfp4", help="weight types, comma-separated")
     km.add_argument("--experts", type=int, default=256, help="experts of the resident layer")
     km.add_argument("--tokens", default="1,4,16", help="tokens per call, comma-separated")
@@ -729,7 +741,7 @@ def main():
     if args.warmup < 3 and not args.profile_only:
         raise SystemExit("--warmup must be >= 3")
 
-    if args.workload in ("hit_gemv", "prefill_gemm"):
+    if args.workload in ("hit_gemv", "stream_gemv", "prefill_gemm"):
         if args.gpus != 1 or args.impl != "ours":
             raise SystemExit("kernel microbenchmarks run on one GPU, our implementation only")
         return run_kernels(args, 0, 0)
@@ -742,7 +754,7 @@ def main():
         return run_mixed(args, wl, world, rank, local)
     if args.workload != "decode_bf16":
         raise SystemExit("workloads: decode_bf16 (default), prefill_bf16, trace_nvfp4, mixed_nvfp4; "
-                         "kernel microbenchmarks: hit_gemv, prefill_gemm")
+                         "kernel microbenchmarks: hit_gemv, stream_gemv, prefill_gemm")
     if args.impl == "reference":
         r = run_reference(args, wl, world, rank)
         if world > 1:

@@ -81,60 +81,76 @@ __global__ void __launch_bounds__(256) router_scores_kernel(const AT* __restrict
   }
 }
 
-// One warp per token: k rounds of a warp arg-max (larger logit first, equal
-// logits -> lower index), then softmax over the chosen k. SHARED: the scores
-// are in this CTA's shared memory (the cluster routing), else in global
-// memory, read through L2 (other CTAs of the same launch may have written
-// them). ids_sh, if set, receives a copy of the ids (shared memory).
+// Orderable 64-bit key of a logit and its expert: a larger logit gives a
+// larger key, equal logits (+0 and -0 are equal) the lower expert index; a NaN
+// logit sorts below every number. Key 0 is never a valid key.
+__device__ __forceinline__ unsigned long long topk_key(float v, int e) {
+  uint32_t u = __float_as_uint(v + 0.0f);  // -0 -> +0
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  if (v != v) u = 0;
+  return ((unsigned long long)u << 32) | (0xFFFFFFFFu - (uint32_t)e);
+}
+__device__ __forceinline__ float topk_key_value(unsigned long long key) {
+  const uint32_t t = (uint32_t)(key >> 32);
+  return __uint_as_float((t & 0x80000000u) ? (t & 0x7FFFFFFFu) : ~t);
+}
+__device__ __forceinline__ int topk_key_expert(unsigned long long key) {
+  return (int)(0xFFFFFFFFu - (uint32_t)key);
+}
+
+// k rounds of a warp-wide maximum over the keys of E experts (expert
+// i*32 + lane in lane, slot i); lane j gets the j-th largest key.
+template <int PER, bool SHARED>
+__device__ __forceinline__ unsigned long long topk_keys(const float* __restrict__ s, int E, int k, int lane,
+                                                        unsigned long long& top) {
+  unsigned long long key[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int e = i * 32 + lane;
+    float v = 0.f;
+    if (e < E) {
+      if constexpr (SHARED)
+        v = s[e];
+      else
+        v = __ldcg(s + e);  // L2: in the fused kernel other CTAs wrote these
+    }
+    key[i] = e < E ? topk_key(v, e) : 0ull;
+  }
+  unsigned long long mine = 0;
+  for (int j = 0; j < k; ++j) {
+    unsigned long long b = key[0];
+#pragma unroll
+    for (int i = 1; i < PER; ++i) b = key[i] > b ? key[i] : b;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long ob = __shfl_xor_sync(0xffffffffu, b, o);
+      b = ob > b ? ob : b;
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+      if (key[i] == b) key[i] = 0;  // keys are unique: only the owner's entry matches
+    if (lane == j) mine = b;
+    if (j == 0) top = b;
+  }
+  return mine;
+}
+
+// One warp per token: the k largest logits (larger first, equal logits ->
+// lower index), as k rounds of a warp maximum over (logit, index) keys, then
+// softmax over the chosen k. SHARED: the scores are in this CTA's shared
+// memory (the cluster routing), else in global memory, read through L2
+// (other CTAs of the same launch may have written them). ids_sh, if set,
+// receives a copy of the ids (shared memory).
 template <bool SHARED = false>
 __device__ __forceinline__ void topk_token(const float* __restrict__ scores, int warp, int E, int k,
                                            int32_t* __restrict__ ids, float* __restrict__ wts, int lane,
                                            int32_t* ids_sh = nullptr) {
-  constexpr int PER = MAX_E / 32;
-  float v[PER];
-  uint32_t taken = 0;
   const float* s = scores + (size_t)warp * E;  // warp = token index
-#pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    const int e = i * 32 + lane;
-    if constexpr (SHARED)
-      v[i] = e < E ? s[e] : 0.f;
-    else
-      v[i] = e < E ? __ldcg(s + e) : 0.f;
-  }
-  // lane j keeps the j-th pick, so nothing is indexed by the runtime k
-  float top0 = 0.f, my_s = 0.f;
-  int my_e = 0;
-  for (int j = 0; j < k; ++j) {
-    float bv = 0.f;
-    int be = 0x7fffffff;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      const int e = i * 32 + lane;
-      if (e < E && !((taken >> i) & 1u)) {
-        if (be == 0x7fffffff || v[i] > bv) {  // ascending e per lane: strict > keeps the lower index
-          bv = v[i];
-          be = e;
-        }
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      const bool better = (oe != 0x7fffffff) && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be));
-      if (better) {
-        bv = ov;
-        be = oe;
-      }
-    }
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
-    if (lane == j) {
-      my_s = bv;
-      my_e = be;
-    }
-    if (j == 0) top0 = bv;
-  }
+  unsigned long long top = 0;
+  const unsigned long long mine =
+      E <= 256 ? topk_keys<8, SHARED>(s, E, k, lane, top) : topk_keys<MAX_E / 32, SHARED>(s, E, k, lane, top);
+  const float my_s = topk_key_value(mine), top0 = topk_key_value(top);
+  const int my_e = topk_key_expert(mine);
   const float ex = lane < k ? expf(my_s - top0) : 0.f;
   float den = 0.f;
   for (int j = 0; j < k; ++j) den += __shfl_sync(0xffffffffu, ex, j);  // rank order
