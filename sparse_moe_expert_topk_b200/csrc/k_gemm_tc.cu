@@ -39,7 +39,8 @@ struct TcPlan {
   CUtensorMap b_h;   // H_s [rows, d_ff]
   // NVFP4: the codes of each matrix over the slot pool
   // (3D: bytes of a row, rows of the matrix, slot), phase 0 and phase 1
-  CUtensorMap f_code[3];  // gate, up, down
+  CUtensorMap f_code[3];   // gate, up, down: boxes of one k-block (32 code bytes x 128 rows)
+  CUtensorMap f_code4[3];  // the same with boxes of four k-blocks (128 bytes x 128 rows, 128B-swizzled)
   bool fp4;
   int sms;
 };
@@ -55,7 +56,13 @@ constexpr int A_BYTES = BM * BK * 2;       // 16 KB
 constexpr int B_BYTES = MAX_N * BK * 2;    // 32 KB
 constexpr int STAGE_BYTES = 2 * A_BYTES + B_BYTES;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
-constexpr int THREADS = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+// Warps: 0 TMA, 1 MMA, 2 .. 2 + EPI_WARPS - 1 epilogue. The gate/up epilogue
+// (SwiGLU over 128 x 256 accumulators) runs while the MMAs wait for the one
+// accumulator buffer, so it takes two warps per TMEM lane quarter, each on
+// every other 32-column chunk (one warp per quarter took about as long as a
+// unit's main loop).
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = (2 + EPI_WARPS) * 32;
 
 using mb::smem_u32;
 using mb::WAIT_CYCLES;
@@ -195,7 +202,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_acc_full + 8 * b, 1);
-      mbar_init(bar_acc_empty + 8 * b, 4);
+      mbar_init(bar_acc_empty + 8 * b, EPI_WARPS);
     }
     mbar_init(bar_drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -291,8 +298,9 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
       if (!ok) break;
     }
   } else {
-    // ---------------- epilogue (warps 2..5) ----------------
+    // ---------------- epilogue (warps 2 .. 2 + EPI_WARPS - 1) ----------------
     const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int part = (warp - 2) >> 2, parts = EPI_WARPS / 4;  // which of the quarter's column chunks
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     int ui = 0;
     for (int u = blockIdx.x; u < n_units && !*abort; u += gridDim.x, ++ui) {
@@ -302,7 +310,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
       if (!mbar_wait(bar_acc_full + 8 * ab, use & 1, abort, a.error)) break;
       tc_fence_after();
       const int row = un.mt * BM + 32 * q + lane;  // weight row = output feature
-      for (int c0 = 0; c0 < un.nrows; c0 += 32) {
+      for (int c0 = 32 * part; c0 < un.nrows; c0 += 32 * parts) {
         uint32_t g[32];
         tmem_ld32(tmem + (uint32_t)(ab * 256) + lane_base + c0, g);
         if (two_a) {
@@ -367,18 +375,30 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
 // the rest of the pipeline are the bf16 kernel's: tokens on the N side,
 // gate and up in two TMEM halves, SwiGLU in the epilogue.
 //
-// Rings: the A (weights) and B (tokens) tiles in STAGES stages as above, the
-// raw codes in F_RAW stages of their own. Barriers per A/B stage: full (TMA
-// of the token tile), deq (256 dequantising threads wrote the A tile), empty
-// (the MMAs that read the stage completed); per raw stage: raw_full (TMA of
-// the codes), raw_empty (the dequantising threads read them).
+// Rings: the A (weights) and B (tokens) tiles in STG stages as above, the
+// raw codes in RAW stages of RK k-blocks each, filled by a producer warp of
+// their own, so the codes run ahead of the A/B ring. Barriers per A/B stage:
+// full (TMA of the token tile), deq (256 dequantising threads wrote the A
+// tile), empty (the MMAs that read the stage completed); per raw stage:
+// raw_full (TMA of the codes), raw_empty (the dequantising threads read
+// them). Two instances: few tokens per expert (weight-bound) STG 2, RAW 2,
+// RK 4: each stage fetches 128 contiguous bytes of each of 128 rows (a
+// one-k-block stage fetches 32, which kept DRAM at about 2 TB/s whatever the
+// ring depth), 128B-swizzled so the dequantising reads are conflict-free;
+// many tokens per expert (tensor-bound) STG 3, RAW 2, RK 1.
+// Warps: 0 token TMA, 1 MMA, 2..5 epilogue, 6..13 dequantising, 14 code TMA.
 // ---------------------------------------------------------------------------
-constexpr int F_RAW = 2;
 constexpr int F_CODE_BYTES = BM * BK / 2;  // 4 KB: 128 rows x 32 code bytes (64 values)
 constexpr int F_RAW_BYTES = 2 * F_CODE_BYTES;
 constexpr int F_DEQ_WARPS = 8;
-constexpr int F_THREADS = (6 + F_DEQ_WARPS) * 32;
-constexpr int F_SMEM_BYTES = STAGES * STAGE_BYTES + F_RAW * F_RAW_BYTES + 1024 + 256;
+constexpr int F_CODE_WARP = 6 + F_DEQ_WARPS;
+constexpr int F_THREADS = (F_CODE_WARP + 1) * 32;
+template <int STG, int RAW, int RK>
+constexpr int f_smem_bytes() {
+  static_assert((3 * STG + 2 * RAW + 5) * 8 <= 256, "barriers");
+  return STG * STAGE_BYTES + RAW * RK * F_RAW_BYTES + 1024 + 256;
+}
+constexpr int F_TOK_PER_EXPERT_DEEP = 128;  // up to this many rows per routed expert: the deep code ring
 
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y, int z) {
   asm volatile(
@@ -415,6 +435,7 @@ struct TcFp4Maps {
   CUtensorMap code_a, code_b;  // phase 0: gate / up codes; phase 1: down codes (b unused)
 };
 
+template <int STG, int RAW, int RK>
 __global__ void __launch_bounds__(F_THREADS, 1) gemm_tc_fp4_kernel(const __grid_constant__ CUtensorMap tm_b,
                                                                    const __grid_constant__ TcFp4Maps fm, TcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -423,11 +444,12 @@ __global__ void __launch_bounds__(F_THREADS, 1) gemm_tc_fp4_kernel(const __grid_
   __shared__ int s_abort;
   __shared__ uint32_t s_tmem;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* raw = smem + STAGES * STAGE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(raw + F_RAW * F_RAW_BYTES);
-  const uint32_t bar_full = smem_u32(bars), bar_empty = bar_full + 8 * STAGES, bar_deq = bar_empty + 8 * STAGES;
-  const uint32_t bar_rfull = bar_deq + 8 * STAGES, bar_rempty = bar_rfull + 8 * F_RAW;
-  const uint32_t bar_acc_full = bar_rempty + 8 * F_RAW, bar_acc_empty = bar_acc_full + 16;
+  uint8_t* raw = smem + STG * STAGE_BYTES;
+  constexpr int RAW_STAGE = RK * F_RAW_BYTES;  // RK k-blocks of codes of both matrices
+  uint64_t* bars = reinterpret_cast<uint64_t*>(raw + RAW * RAW_STAGE);
+  const uint32_t bar_full = smem_u32(bars), bar_empty = bar_full + 8 * STG, bar_deq = bar_empty + 8 * STG;
+  const uint32_t bar_rfull = bar_deq + 8 * STG, bar_rempty = bar_rfull + 8 * RAW;
+  const uint32_t bar_acc_full = bar_rempty + 8 * RAW, bar_acc_empty = bar_acc_full + 16;
   const uint32_t bar_drain = bar_acc_empty + 16;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort = &s_abort;
@@ -437,12 +459,12 @@ __global__ void __launch_bounds__(F_THREADS, 1) gemm_tc_fp4_kernel(const __grid_
   for (int i = threadIdx.x; i < n_items; i += F_THREADS) s_items[i] = a.work->items[KIND_HIT][i];
   if (threadIdx.x == 0) {
     s_abort = 0;
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < STG; ++s) {
       mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, 1);
       mbar_init(bar_deq + 8 * s, DEQ_THREADS);
     }
-    for (int r = 0; r < F_RAW; ++r) {
+    for (int r = 0; r < RAW; ++r) {
       mbar_init(bar_rfull + 8 * r, 1);
       mbar_init(bar_rempty + 8 * r, DEQ_THREADS);
     }
@@ -474,36 +496,28 @@ __global__ void __launch_bounds__(F_THREADS, 1) gemm_tc_fp4_kernel(const __grid_
   const int two_a = a.phase == 0;
   const int n_mat = two_a ? 2 : 1;
 
-  int last_round[STAGES], last_raw[F_RAW];  // producer: last round issued per stage (-1 none)
+  int last_round[STG], last_raw[RAW];  // producer: last round issued per stage (-1 none)
 #pragma unroll
-  for (int s = 0; s < STAGES; ++s) last_round[s] = -1;
+  for (int s = 0; s < STG; ++s) last_round[s] = -1;
 #pragma unroll
-  for (int r = 0; r < F_RAW; ++r) last_raw[r] = -1;
+  for (int r = 0; r < RAW; ++r) last_raw[r] = -1;
   if (warp == 0) {
-    // ---------------- TMA producer: token tiles, codes and scales ----------------
+    // ---------------- TMA producer: token tiles ----------------
     int it = 0;
     for (int u = blockIdx.x; u < n_units && !*abort; u += gridDim.x) {
       Unit un;
       if (!unit_at(a, s_items, s_pref, n_items, u, un)) break;
       const int nb = (un.nrows + BOX_ROWS - 1) / BOX_ROWS;
       const uint32_t b_bytes = nb * BOX_ROWS * BK * 2;
-      const uint32_t r_bytes = n_mat * F_CODE_BYTES;
-      const int row0 = un.mt * BM;
       bool ok = true;
       for (int kb = 0; kb < a.k_blocks; ++kb, ++it) {
-        const int s = it % STAGES, r = it / STAGES, q = it % F_RAW, rq = it / F_RAW;
-        if (!mbar_wait(bar_empty + 8 * s, (r & 1) ^ 1, abort, a.error) ||
-            !mbar_wait(bar_rempty + 8 * q, (rq & 1) ^ 1, abort, a.error)) {
+        const int s = it % STG, r = it / STG;
+        if (!mbar_wait(bar_empty + 8 * s, (r & 1) ^ 1, abort, a.error)) {
           ok = false;
           break;
         }
         last_round[s] = r;
-        last_raw[q] = rq;
         if (lane == 0) {
-          const uint32_t rb = smem_u32(raw + q * F_RAW_BYTES);
-          mbar_expect_tx(bar_rfull + 8 * q, r_bytes);
-          tma_load_3d(rb, &fm.code_a, bar_rfull + 8 * q, kb * (BK / 2), row0, un.slot);
-          if (two_a) tma_load_3d(rb + F_CODE_BYTES, &fm.code_b, bar_rfull + 8 * q, kb * (BK / 2), row0, un.slot);
           const uint32_t base = smem_u32(smem + s * STAGE_BYTES);
           mbar_expect_tx(bar_full + 8 * s, b_bytes);
           for (int b = 0; b < nb; ++b)
@@ -528,7 +542,7 @@ __global__ void __launch_bounds__(F_THREADS, 1) gemm_tc_fp4_kernel(const __grid_
       tc_fence_after();
       bool ok = true;
       for (int kb = 0; kb < a.k_blocks; ++kb, ++it) {
-        const int s = it % STAGES, r = it / STAGES;
+        const int s = it % STG, r = it / STG;
         if (!mbar_wait(bar_full + 8 * s, r & 1, abort, a.error) || !mbar_wait(bar_deq + 8 * s, r & 1, abort, a.error)) {
           ok = false;
           break;
@@ -544,6 +558,33 @@ __global__ void __launch_bounds__(F_THREADS, 1) gemm_tc_fp4_kernel(const __grid_
           }
           umma_commit(bar_empty + 8 * s);
           if (kb == a.k_blocks - 1) umma_commit(bar_acc_full + 8 * ab);
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+    }
+  } else if (warp == F_CODE_WARP) {
+    // ------- TMA producer: weight codes, RK k-blocks per stage, up to RAW stages ahead -------
+    int it = 0;
+    for (int u = blockIdx.x; u < n_units && !*abort; u += gridDim.x) {
+      Unit un;
+      if (!unit_at(a, s_items, s_pref, n_items, u, un)) break;
+      const uint32_t r_bytes = n_mat * RK * F_CODE_BYTES;
+      const int row0 = un.mt * BM;
+      bool ok = true;
+      for (int kb = 0; kb < a.k_blocks; kb += RK, ++it) {  // k_blocks is a multiple of RK
+        const int q = it % RAW, rq = it / RAW;
+        if (!mbar_wait(bar_rempty + 8 * q, (rq & 1) ^ 1, abort, a.error)) {
+          ok = false;
+          break;
+        }
+        last_raw[q] = rq;
+        if (lane == 0) {
+          const uint32_t rb = smem_u32(raw + q * RAW_STAGE);
+          mbar_expect_tx(bar_rfull + 8 * q, r_bytes);
+          tma_load_3d(rb, &fm.code_a, bar_rfull + 8 * q, kb * (BK / 2), row0, un.slot);
+          if (two_a)
+            tma_load_3d(rb + RK * F_CODE_BYTES, &fm.code_b, bar_rfull + 8 * q, kb * (BK / 2), row0, un.slot);
         }
         __syncwarp();
       }
@@ -593,51 +634,67 @@ __global__ void __launch_bounds__(F_THREADS, 1) gemm_tc_fp4_kernel(const __grid_
   } else {
     // ---------------- dequantising warps (6..13) ----------------
     // thread dt owns half-rows dt (and dt + 256 for gate/up): (matrix, row,
-    // half) = (i / 256, (i % 256) / 2, i % 2); its two block scales of a
-    // k-block are one 16-bit word of the matrix's scale rows, read one
-    // k-block ahead
+    // half) = (i / 256, (i % 256) / 2, i % 2). A k-block's block scales of a
+    // row are 4 bytes of the matrix's scale row, the thread's two are the
+    // 16-bit half h; one 16-byte load brings a row's scales of 4 k-blocks,
+    // issued a group of 4 k-blocks ahead of its use (loading each k-block's
+    // scales one k-block ahead held the kernel at the load latency), and the
+    // thread's halves of the 4 words are packed into two registers
     const int dt = threadIdx.x - 6 * 32;  // 0..255
     const size_t n = (size_t)a.d * a.d_ff;
-    const int K = two_a ? a.d : a.d_ff;
+    const int K = two_a ? a.d : a.d_ff;   // a multiple of 256: scale rows are 16-byte aligned
     const size_t sc0 = 3 * (n / 2) + (two_a ? 0 : n / 8);  // scales of gate (phase 0) or down (phase 1)
+    const uint32_t sel = (dt & 1) ? 0x7632u : 0x5410u;  // bytes 2h, 2h+1 of two words
     int it = 0;
     for (int u = blockIdx.x; u < n_units && !*abort; u += gridDim.x) {
       Unit un;
       if (!unit_at(a, s_items, s_pref, n_items, u, un)) break;
       const uint8_t* blob = a.slots + (size_t)un.slot * a.slot_bytes;
-      const unsigned short* scp[2];
+      const uint4* srow[2];
 #pragma unroll
       for (int v = 0; v < 2; ++v) {
         const int i = dt + v * DEQ_THREADS;
-        const int m = i / (2 * BM), row = un.mt * BM + ((i % (2 * BM)) >> 1), h = i & 1;
-        scp[v] = reinterpret_cast<const unsigned short*>(blob + sc0 + m * (n / 16) + (size_t)row * (K / 16)) + h;
+        const int m = i / (2 * BM), row = un.mt * BM + ((i % (2 * BM)) >> 1);
+        srow[v] = reinterpret_cast<const uint4*>(blob + sc0 + m * (n / 16) + (size_t)row * (K / 16));
       }
-      uint32_t scn[2] = {0, 0};
+      uint4 sraw[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+      uint2 scur[2] = {make_uint2(0, 0), make_uint2(0, 0)};
 #pragma unroll
       for (int v = 0; v < 2; ++v)
-        if (v < n_mat) scn[v] = __ldg(scp[v]);
+        if (v < n_mat) sraw[v] = __ldg(srow[v]);
       bool ok = true;
       for (int kb = 0; kb < a.k_blocks; ++kb, ++it) {
-        const int s = it % STAGES, r = it / STAGES, q = it % F_RAW, rq = it / F_RAW;
-        uint32_t scc[2] = {scn[0], scn[1]};
-        if (kb + 1 < a.k_blocks) {
+        const int s = it % STG, r = it / STG, q = (it / RK) % RAW, rq = (it / RK) / RAW, jr = it % RK;
+        const int j = kb & 3;
+        if (j == 0) {
 #pragma unroll
-          for (int v = 0; v < 2; ++v)
-            if (v < n_mat) scn[v] = __ldg(scp[v] + 2 * (kb + 1));
+          for (int v = 0; v < 2; ++v) {
+            if (v < n_mat) {
+              scur[v] = make_uint2(__byte_perm(sraw[v].x, sraw[v].y, sel), __byte_perm(sraw[v].z, sraw[v].w, sel));
+              if (kb + 4 < a.k_blocks) sraw[v] = __ldg(srow[v] + (kb / 4 + 1));
+            }
+          }
         }
+        uint32_t scc[2];
+#pragma unroll
+        for (int v = 0; v < 2; ++v) scc[v] = ((j < 2 ? scur[v].x : scur[v].y) >> (16 * (j & 1))) & 0xFFFFu;
         if (!mbar_wait(bar_rfull + 8 * q, rq & 1, abort, a.error) ||
             !mbar_wait(bar_empty + 8 * s, (r & 1) ^ 1, abort, a.error)) {
           ok = false;
           break;
         }
-        const uint8_t* rb = raw + q * F_RAW_BYTES;
+        const uint8_t* rb = raw + q * RAW_STAGE;
         uint8_t* ab_tile = smem + s * STAGE_BYTES;
 #pragma unroll
         for (int v = 0; v < 2; ++v) {
           if (v >= n_mat) break;
           const int i = dt + v * DEQ_THREADS;
           const int m = i / (2 * BM), row = (i % (2 * BM)) >> 1, h = i & 1;
-          const uint4 codes = *reinterpret_cast<const uint4*>(rb + m * F_CODE_BYTES + row * 32 + h * 16);
+          // row `row` of the stage holds RK k-blocks of codes (32 bytes each);
+          // with RK = 4 the 128-byte rows are 128B-swizzled by the TMA
+          const int chunk = RK == 4 ? ((2 * jr + h) ^ (row & 7)) : 2 * jr + h;
+          const uint4 codes =
+              *reinterpret_cast<const uint4*>(rb + m * RK * F_CODE_BYTES + row * (32 * RK) + chunk * 16);
           const uint32_t s0 = scc[v] & 0xFF, s1 = (scc[v] >> 8) & 0xFF;
           uint8_t* dst = ab_tile + m * A_BYTES + row * 128;
           const int sw = row & 7;
@@ -649,7 +706,7 @@ __global__ void __launch_bounds__(F_THREADS, 1) gemm_tc_fp4_kernel(const __grid_
         // the MMAs read the tile through the async proxy
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_arrive(bar_deq + 8 * s);
-        mbar_arrive(bar_rempty + 8 * q);
+        if (jr == RK - 1) mbar_arrive(bar_rempty + 8 * q);
       }
       if (!ok) break;
     }
@@ -658,14 +715,16 @@ __global__ void __launch_bounds__(F_THREADS, 1) gemm_tc_fp4_kernel(const __grid_
   if (warp == 0) {
     // producer tail: every stage's last round released (normal exit) or at
     // least landed (abort) before shared memory goes away
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < STG; ++s) {
       if (last_round[s] < 0) continue;
       const uint32_t bar = *abort ? bar_full + 8 * s : bar_empty + 8 * s;
       const long long t0 = clock64();
       while (!mbar_try_wait(bar, last_round[s] & 1) && clock64() - t0 < WAIT_CYCLES / 4) {
       }
     }
-    for (int q = 0; q < F_RAW; ++q) {
+  } else if (warp == F_CODE_WARP) {
+    // code producer tail: every raw stage's last copy landed
+    for (int q = 0; q < RAW; ++q) {
       if (last_raw[q] < 0) continue;
       const long long t0 = clock64();
       while (!mbar_try_wait(bar_rfull + 8 * q, last_raw[q] & 1) && clock64() - t0 < WAIT_CYCLES / 4) {
@@ -711,15 +770,16 @@ bool encode_2d(CUtensorMap* m, void* base, uint64_t rows, uint64_t cols, uint32_
 
 // 3D byte map over the slot pool: `row_bytes` per row, `rows` rows per slot,
 // `slots` slots `slot_bytes` apart, starting `off` bytes into each slot; box
-// of box_x bytes x BM rows x 1 slot.
+// of box_x bytes x BM rows x 1 slot (box_x = 128 with the 128-byte swizzle).
 bool encode_3d_u8(CUtensorMap* m, const uint8_t* slots, size_t off, uint64_t row_bytes, uint64_t rows,
-                  uint64_t n_slots, uint64_t slot_bytes, uint32_t box_x) {
+                  uint64_t n_slots, uint64_t slot_bytes, uint32_t box_x, bool swizzle128 = false) {
   cuuint64_t dims[3] = {row_bytes, rows, n_slots};
   cuuint64_t strides[2] = {row_bytes, slot_bytes};
   cuuint32_t box[3] = {box_x, (cuuint32_t)BM, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, (void*)(slots + off), dims, strides, box, estr,
-                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -728,7 +788,10 @@ bool encode_3d_u8(CUtensorMap* m, const uint8_t* slots, size_t off, uint64_t row
 
 bool prefill_tc_supported(const Shape& sh) {
   if (sh.C <= 0 || sh.d % BM || sh.d_ff % BM) return false;
-  return sh.wtype == FT_W_BF16 || sh.wtype == FT_W_NVFP4;
+  // NVFP4: the dequantising warps read each row's block scales 16 bytes (four
+  // k-blocks) at a time, so the scale rows (K / 16 bytes) are 16-byte multiples
+  if (sh.wtype == FT_W_NVFP4) return sh.d % 256 == 0 && sh.d_ff % 256 == 0;
+  return sh.wtype == FT_W_BF16;
 }
 
 cudaError_t prefill_tc_init(const Shape& sh, DevState& ds, int max_rows) {
@@ -750,7 +813,10 @@ cudaError_t prefill_tc_init(const Shape& sh, DevState& ds, int max_rows) {
     const uint8_t* sl = ds.slots;
     const bool ok = encode_3d_u8(&p->f_code[0], sl, 0, sh.d / 2, sh.d_ff, C, sh.slot_bytes, BK / 2) &&
                     encode_3d_u8(&p->f_code[1], sl, n / 2, sh.d / 2, sh.d_ff, C, sh.slot_bytes, BK / 2) &&
-                    encode_3d_u8(&p->f_code[2], sl, n, sh.d_ff / 2, sh.d, C, sh.slot_bytes, BK / 2);
+                    encode_3d_u8(&p->f_code[2], sl, n, sh.d_ff / 2, sh.d, C, sh.slot_bytes, BK / 2) &&
+                    encode_3d_u8(&p->f_code4[0], sl, 0, sh.d / 2, sh.d_ff, C, sh.slot_bytes, 4 * BK / 2, true) &&
+                    encode_3d_u8(&p->f_code4[1], sl, n / 2, sh.d / 2, sh.d_ff, C, sh.slot_bytes, 4 * BK / 2, true) &&
+                    encode_3d_u8(&p->f_code4[2], sl, n, sh.d_ff / 2, sh.d, C, sh.slot_bytes, 4 * BK / 2, true);
     if (!ok) return cudaErrorInvalidValue;
   }
   if (!encode_2d(&p->b_x, ds.xs, (uint64_t)max_rows + 256, sh.d, BOX_ROWS)) return cudaErrorInvalidValue;
@@ -758,7 +824,11 @@ cudaError_t prefill_tc_init(const Shape& sh, DevState& ds, int max_rows) {
 
   cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(gemm_tc_fp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, F_SMEM_BYTES);
+    e = cudaFuncSetAttribute(gemm_tc_fp4_kernel<2, 2, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             f_smem_bytes<2, 2, 4>());
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gemm_tc_fp4_kernel<3, 2, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             f_smem_bytes<3, 2, 1>());
   if (e != cudaSuccess) return e;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -775,7 +845,6 @@ void launch_prefill_gather(const Shape& sh, const void* x, int T, DevState& ds, 
 }
 
 void launch_gemm_tc(const Shape& sh, int phase, int layer, int T, DevState& ds, cudaStream_t st) {
-  (void)T;
   const TcPlan& p = *static_cast<const TcPlan*>(ds.tc_plan);
   TcArgs a;
   a.work = ds.work;
@@ -793,10 +862,17 @@ void launch_gemm_tc(const Shape& sh, int phase, int layer, int T, DevState& ds, 
   a.ybuf = ds.ybuf;
   a.error = ds.error;
   if (p.fp4) {
+    const CUtensorMap& tb = phase == 0 ? p.b_x : p.b_h;
     TcFp4Maps fm;
-    fm.code_a = p.f_code[phase == 0 ? 0 : 2];
-    fm.code_b = p.f_code[1];
-    gemm_tc_fp4_kernel<<<p.sms, F_THREADS, F_SMEM_BYTES, st>>>(phase == 0 ? p.b_x : p.b_h, fm, a);
+    if ((long long)T * sh.k <= (long long)F_TOK_PER_EXPERT_DEEP * sh.E) {
+      fm.code_a = p.f_code4[phase == 0 ? 0 : 2];
+      fm.code_b = p.f_code4[1];
+      gemm_tc_fp4_kernel<2, 2, 4><<<p.sms, F_THREADS, f_smem_bytes<2, 2, 4>(), st>>>(tb, fm, a);
+    } else {
+      fm.code_a = p.f_code[phase == 0 ? 0 : 2];
+      fm.code_b = p.f_code[1];
+      gemm_tc_fp4_kernel<3, 2, 1><<<p.sms, F_THREADS, f_smem_bytes<3, 2, 1>(), st>>>(tb, fm, a);
+    }
     return;
   }
   gemm_tc_kernel<<<p.sms, THREADS, SMEM_BYTES, st>>>(phase == 0 ? p.a_gu : p.a_dn, phase == 0 ? p.b_x : p.b_h, a);
