@@ -824,6 +824,119 @@ __device__ __forceinline__ void dot_nvfp4(const uint8_t* ra, const uint8_t* rb, 
   }
 }
 
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Bytes of one warp's code buffers in the NVFP4 direct kernel: two steps of
+// RT tiles x (gate or row a, up or row b) x 32 lanes x 16 bytes.
+constexpr int fp4_wbuf_bytes(int rt) { return 2 * rt * 2 * 32 * 16; }
+
+// The same sums as dot_nvfp4, with each step's code fragments brought into
+// the warp's own shared-memory buffers by cp.async one step ahead of their
+// MMAs (and the block scales into registers one step ahead), so a warp's
+// next loads are in flight while it decodes and multiplies the current step:
+// with every load of a step waited for before its arithmetic, a gate/up unit
+// took about 2.5 us per step. Each lane reads back only the 16 bytes it
+// copied. wbuf: shared address of this warp's buffers (fp4_wbuf_bytes(RT)).
+template <int NB, int RT, bool P1>
+__device__ __forceinline__ void dot_nvfp4_async(const uint8_t* ra, const uint8_t* rb, const unsigned short* sa,
+                                                const unsigned short* sb, size_t tstride, size_t tsc, int s0, int s1,
+                                                const uint16_t* const (&xr)[NB], const uint16_t* const (&xl)[NB],
+                                                int q, float (&acc)[RT][NB][4], float (&acc2)[P1 ? RT : 1][NB][4],
+                                                uint32_t wbuf, int lane) {
+  if (s0 >= s1) return;
+  constexpr uint32_t STEP_B = RT * 2 * 32 * 16;
+  const uint32_t mine = wbuf + lane * 16;
+  auto issue = [&](int s, int b) {
+#pragma unroll
+    for (int r = 0; r < RT; ++r) {
+      cp_async16(mine + b * STEP_B + (2 * r) * 512, ra + r * tstride + (size_t)s * 64);
+      cp_async16(mine + b * STEP_B + (2 * r + 1) * 512, rb + r * tstride + (size_t)s * 64);
+    }
+    cp_async_commit();
+  };
+  uint32_t ca[RT], cb[RT];
+  issue(s0, 0);
+#pragma unroll
+  for (int r = 0; r < RT; ++r) {
+    ca[r] = __ldg(sa + r * tsc + s0 * 4);
+    cb[r] = __ldg(sb + r * tsc + s0 * 4);
+  }
+  for (int s = s0; s < s1; ++s) {
+    const int b = (s - s0) & 1;
+    uint32_t na[RT], nb[RT];
+    if (s + 1 < s1) {
+      issue(s + 1, b ^ 1);
+#pragma unroll
+      for (int r = 0; r < RT; ++r) {
+        na[r] = __ldg(sa + r * tsc + (s + 1) * 4);
+        nb[r] = __ldg(sb + r * tsc + (s + 1) * 4);
+      }
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    uint32_t xh[NB][16];
+#pragma unroll
+    for (int t = 0; t < NB; ++t) {
+      const uint16_t* xp = xr[t] + s * 128 + q * 32;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const uint4 xv = P1 ? ld_cg(xp + 8 * v) : __ldg(reinterpret_cast<const uint4*>(xp) + v);
+        xh[t][4 * v] = xv.x;
+        xh[t][4 * v + 1] = xv.y;
+        xh[t][4 * v + 2] = xv.z;
+        xh[t][4 * v + 3] = xv.w;
+      }
+    }
+    uint32_t xo[P1 ? NB : 1][16];  // the lo term of h (down units)
+    if constexpr (P1) {
+#pragma unroll
+      for (int t = 0; t < NB; ++t) {
+        const uint16_t* xp = xl[t] + s * 128 + q * 32;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint4 xv = ld_cg(xp + 8 * v);
+          xo[t][4 * v] = xv.x;
+          xo[t][4 * v + 1] = xv.y;
+          xo[t][4 * v + 2] = xv.z;
+          xo[t][4 * v + 3] = xv.w;
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < RT; ++r) {
+      uint32_t ha[16], hb[16];
+      decode_nvfp4(lds128(mine + b * STEP_B + (2 * r) * 512), ca[r], ha);
+      decode_nvfp4(lds128(mine + b * STEP_B + (2 * r + 1) * 512), cb[r], hb);
+#pragma unroll
+      for (int t = 0; t < NB; ++t) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          mma_f16(acc[r][t], ha[2 * j], hb[2 * j], ha[2 * j + 1], hb[2 * j + 1], xh[t][2 * j], xh[t][2 * j + 1]);
+        if constexpr (P1) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            mma_f16(acc2[r][t], ha[2 * j], hb[2 * j], ha[2 * j + 1], hb[2 * j + 1], xo[t][2 * j], xo[t][2 * j + 1]);
+        }
+      }
+    }
+    if (s + 1 < s1) {
+#pragma unroll
+      for (int r = 0; r < RT; ++r) {
+        ca[r] = na[r];
+        cb[r] = nb[r];
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Direct-load variant for experts resident in HBM slots (the hit class): the
 // MMA warps load their weight fragments straight into registers, U steps in
@@ -838,7 +951,8 @@ __device__ __forceinline__ void dot_nvfp4(const uint8_t* ra, const uint8_t* rb, 
 // 8 (rb*RT + r) + g with the matching up rows (phase 0), down rows
 // 16 (rb*RT + r) + g and + 8 (phase 1).
 template <int NB, int PHASE, bool FP4, int NW, int RT>
-__device__ void direct_unit(const MmaArgs& a, const WorkItem& it, int chunk, int rb, int warp, int lane, float* red) {
+__device__ void direct_unit(const MmaArgs& a, const WorkItem& it, int chunk, int rb, int warp, int lane, float* red,
+                            uint32_t wbuf) {
   const int g = lane >> 2, q = lane & 3;
   const uint8_t* blob = blob_of(a, it);
   const size_t n = (size_t)a.d * a.d_ff;
@@ -898,17 +1012,17 @@ __device__ void direct_unit(const MmaArgs& a, const WorkItem& it, int chunk, int
       const int b0 = j * gg.ss, ns = min(gg.ss, gg.steps - b0);
       const int s0 = b0 + (warp * ns) / NW, s1 = b0 + ((warp + 1) * ns) / NW;
       if constexpr (PHASE == 1)
-        dot_nvfp4<NB, RT, true>(blob + oa + q * 16, blob + ob + q * 16,
-                                reinterpret_cast<const unsigned short*>(blob + sa0) + q,
-                                reinterpret_cast<const unsigned short*>(blob + sb0) + q,
-                                (size_t)rows_per_tile * rbytes, (size_t)rows_per_tile * sbytes / 2, s0, s1, xr, xl, q,
-                                acc, acc2);
+        dot_nvfp4_async<NB, RT, true>(blob + oa + q * 16, blob + ob + q * 16,
+                                      reinterpret_cast<const unsigned short*>(blob + sa0) + q,
+                                      reinterpret_cast<const unsigned short*>(blob + sb0) + q,
+                                      (size_t)rows_per_tile * rbytes, (size_t)rows_per_tile * sbytes / 2, s0, s1, xr,
+                                      xl, q, acc, acc2, wbuf, lane);
       else
-        dot_nvfp4<NB, RT, false>(blob + oa + q * 16, blob + ob + q * 16,
-                                 reinterpret_cast<const unsigned short*>(blob + sa0) + q,
-                                 reinterpret_cast<const unsigned short*>(blob + sb0) + q,
-                                 (size_t)rows_per_tile * rbytes, (size_t)rows_per_tile * sbytes / 2, s0, s1, xr, xl,
-                                 q, acc, acc2);
+        dot_nvfp4_async<NB, RT, false>(blob + oa + q * 16, blob + ob + q * 16,
+                                       reinterpret_cast<const unsigned short*>(blob + sa0) + q,
+                                       reinterpret_cast<const unsigned short*>(blob + sb0) + q,
+                                       (size_t)rows_per_tile * rbytes, (size_t)rows_per_tile * sbytes / 2, s0, s1, xr,
+                                       xl, q, acc, acc2, wbuf, lane);
     }
     if constexpr (PHASE == 1) {  // join the two terms of h in each warp, as the ring kernel does
 #pragma unroll
@@ -1017,6 +1131,7 @@ __global__ void __launch_bounds__(NW * 32) gemv_direct_kernel(MmaArgs a) {
   __shared__ int s_pref[MAX_E + 1];
   __shared__ WorkItem s_items[MAX_E];
   __shared__ float red[NW * RTM * NB * 4 * 32];
+  extern __shared__ __align__(16) uint8_t dsm_direct[];  // NVFP4: per-warp code buffers
   // Tickets taken ahead of the unit being worked on: two for BF16 (measured
   // faster than one), one for NVFP4, whose gate/up units fill about one wave
   // at a few tokens, so a second early ticket would stack two of them on some
@@ -1026,6 +1141,7 @@ __global__ void __launch_bounds__(NW * 32) gemv_direct_kernel(MmaArgs a) {
   const int n_items = a.work->n_items[a.cls];
   if (n_items == 0) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t wbuf = (uint32_t)__cvta_generic_to_shared(dsm_direct) + warp * (FP4 ? fp4_wbuf_bytes(RTM) : 0);
   for (int i = tid; i < n_items; i += blockDim.x) s_items[i] = a.work->items[a.cls][i];
   __syncthreads();
   if (warp == 0) {  // exclusive scan of the chunks per item
@@ -1080,9 +1196,9 @@ __global__ void __launch_bounds__(NW * 32) gemv_direct_kernel(MmaArgs a) {
         __threadfence();
       }
       __syncthreads();
-      if (!bad) direct_unit<NB, 1, FP4, NW, RT1>(a, it, chunk, rb, warp, lane, red);
+      if (!bad) direct_unit<NB, 1, FP4, NW, RT1>(a, it, chunk, rb, warp, lane, red, wbuf);
     } else {
-      if (!bad) direct_unit<NB, 0, FP4, NW, RT>(a, it, chunk, rb, warp, lane, red);
+      if (!bad) direct_unit<NB, 0, FP4, NW, RT>(a, it, chunk, rb, warp, lane, red, wbuf);
     }
     // entry (i + AHEAD) % (AHEAD + 1) held the previous unit's ticket, which
     // every thread read before the last barrier: it is free for the new one
@@ -1126,12 +1242,22 @@ constexpr int warps_for() { return RING_WARPS; }
 
 int g_grid_direct[2][3] = {{0, 0, 0}, {0, 0, 0}};  // [fp4][NB]
 
+// Dynamic shared memory of the direct kernel: the NVFP4 per-warp code buffers.
+template <int NB, bool FP4>
+constexpr int direct_dyn_smem() {
+  constexpr int rtm = tiles_for<FP4>() > tiles_down_for<FP4, NB>() ? tiles_for<FP4>() : tiles_down_for<FP4, NB>();
+  return FP4 ? warps_for<NB>() * fp4_wbuf_bytes(rtm) : 0;
+}
+
 template <int NB, bool FP4>
 cudaError_t direct_setup(int sms) {
   constexpr int NW = warps_for<NB>();
+  constexpr int dyn = direct_dyn_smem<NB, FP4>();
+  cudaError_t e = cudaFuncSetAttribute(gemv_direct_kernel<NB, FP4, NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       dyn);
+  if (e != cudaSuccess) return e;
   int per = 0;
-  const cudaError_t e =
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, gemv_direct_kernel<NB, FP4, NW>, NW * 32, 0);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, gemv_direct_kernel<NB, FP4, NW>, NW * 32, dyn);
   g_grid_direct[FP4][NB] = sms * (per > 0 ? per : 1);
   return e;
 }
@@ -1139,7 +1265,7 @@ cudaError_t direct_setup(int sms) {
 template <int NB, bool FP4>
 void launch_direct(int grid, const MmaArgs& a, cudaStream_t st) {
   constexpr int NW = warps_for<NB>();
-  gemv_direct_kernel<NB, FP4, NW><<<grid, NW * 32, 0, st>>>(a);
+  gemv_direct_kernel<NB, FP4, NW><<<grid, NW * 32, direct_dyn_smem<NB, FP4>(), st>>>(a);
 }
 
 }  // namespace
