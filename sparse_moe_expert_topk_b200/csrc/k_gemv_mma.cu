@@ -1116,13 +1116,16 @@ __device__ void direct_unit(const MmaArgs& a, const WorkItem& it, int chunk, int
 // reduction and barriers amortised.
 template <bool FP4>
 constexpr int tiles_for() { return FP4 ? 4 : 1; }
-// NVFP4 down units carry two accumulators (the two terms of h), so they take
-// two row tiles, which keeps the kernel's registers where four gate/up tiles
-// put them (four measured slower: fewer, longer units and spills). A unit's
-// row tiles change which rows it covers, not the K order of any row, so
-// results do not depend on this choice.
+// Row tiles per down unit. BF16: four sharing each step's h fragments at
+// 9-16 tokens; two up to 8, where the 384 four-tile units of a 6-expert call
+// left a tail of 12.7 us units on a third of the CTAs (two tiles measured 5%
+// faster at 1 and 4 tokens). NVFP4 down units carry two accumulators (the two
+// terms of h), so they take two row tiles, which keeps the kernel's registers
+// where four gate/up tiles put them (four measured slower: fewer, longer units
+// and spills). A unit's row tiles change which rows it covers, not the K order
+// of any row, so results do not depend on this choice.
 template <bool FP4, int NB>
-constexpr int tiles_down_for() { return FP4 ? 2 : 4; }
+constexpr int tiles_down_for() { return FP4 ? 2 : (NB == 1 ? 2 : 4); }
 
 template <int NB, bool FP4, int NW>
 __global__ void __launch_bounds__(NW * 32) gemv_direct_kernel(MmaArgs a) {
@@ -1326,7 +1329,8 @@ void launch_gemv_mma(const Shape& sh, int cls, int layer, const void* x16, int T
   const int NB = T > 8 ? 2 : 1;
   const long long chunks = (long long)max_items + (long long)max_tok / CHUNK;
   if (cls == KIND_HIT) {
-    const int rt1 = fp4 ? (NB == 1 ? tiles_down_for<true, 1>() : tiles_down_for<true, 2>()) : tiles_down_for<false, 1>();
+    const int rt1 = NB == 1 ? (fp4 ? tiles_down_for<true, 1>() : tiles_down_for<false, 1>())
+                            : (fp4 ? tiles_down_for<true, 2>() : tiles_down_for<false, 2>());
     const long long units = chunks * (sh.d_ff / 8 / (fp4 ? tiles_for<true>() : tiles_for<false>()) + sh.d / 16 / rt1);
     const int cap = g_grid_direct[fp4][NB];
     const int grid = (int)(units < cap ? units : cap);
