@@ -757,73 +757,6 @@ __device__ __forceinline__ void dot_bf16_rt(const uint8_t* ra, const uint8_t* rb
   }
 }
 
-// NVFP4: steps of 128 K values (lane q covers K = 128 s + 32 q .. +32: 16
-// code bytes and one scale pair per row); RT row tiles per step, the tiles
-// tstride code bytes (tsc scale pairs) apart, sharing one activation
-// fragment; eight MMAs per step, tile and token tile.
-template <int NB, int RT, bool P1>
-__device__ __forceinline__ void dot_nvfp4(const uint8_t* ra, const uint8_t* rb, const unsigned short* sa,
-                                          const unsigned short* sb, size_t tstride, size_t tsc, int s0, int s1,
-                                          const uint16_t* const (&xr)[NB], const uint16_t* const (&xl)[NB], int q,
-                                          float (&acc)[RT][NB][4], float (&acc2)[P1 ? RT : 1][NB][4]) {
-  for (int s = s0; s < s1; ++s) {
-    uint4 wa[RT], wb[RT];
-    uint32_t ca[RT], cb[RT];
-#pragma unroll
-    for (int r = 0; r < RT; ++r) {
-      wa[r] = ld_stream(ra + r * tstride + (size_t)s * 64);
-      wb[r] = ld_stream(rb + r * tstride + (size_t)s * 64);
-      ca[r] = __ldg(sa + r * tsc + s * 4);
-      cb[r] = __ldg(sb + r * tsc + s * 4);
-    }
-    uint32_t xh[NB][16];
-#pragma unroll
-    for (int t = 0; t < NB; ++t) {
-      const uint16_t* xp = xr[t] + s * 128 + q * 32;
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        const uint4 xv = P1 ? ld_cg(xp + 8 * v) : __ldg(reinterpret_cast<const uint4*>(xp) + v);
-        xh[t][4 * v] = xv.x;
-        xh[t][4 * v + 1] = xv.y;
-        xh[t][4 * v + 2] = xv.z;
-        xh[t][4 * v + 3] = xv.w;
-      }
-    }
-    uint32_t xo[P1 ? NB : 1][16];  // the lo term of h (down units)
-    if constexpr (P1) {
-#pragma unroll
-      for (int t = 0; t < NB; ++t) {
-        const uint16_t* xp = xl[t] + s * 128 + q * 32;
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const uint4 xv = ld_cg(xp + 8 * v);
-          xo[t][4 * v] = xv.x;
-          xo[t][4 * v + 1] = xv.y;
-          xo[t][4 * v + 2] = xv.z;
-          xo[t][4 * v + 3] = xv.w;
-        }
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < RT; ++r) {
-      uint32_t ha[16], hb[16];
-      decode_nvfp4(wa[r], ca[r], ha);
-      decode_nvfp4(wb[r], cb[r], hb);
-#pragma unroll
-      for (int t = 0; t < NB; ++t) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          mma_f16(acc[r][t], ha[2 * j], hb[2 * j], ha[2 * j + 1], hb[2 * j + 1], xh[t][2 * j], xh[t][2 * j + 1]);
-        if constexpr (P1) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            mma_f16(acc2[r][t], ha[2 * j], hb[2 * j], ha[2 * j + 1], hb[2 * j + 1], xo[t][2 * j], xo[t][2 * j + 1]);
-        }
-      }
-    }
-  }
-}
-
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
@@ -837,13 +770,17 @@ __device__ __forceinline__ void cp_async_wait() {
 // RT tiles x (gate or row a, up or row b) x 32 lanes x 16 bytes.
 constexpr int fp4_wbuf_bytes(int rt) { return 2 * rt * 2 * 32 * 16; }
 
-// The same sums as dot_nvfp4, with each step's code fragments brought into
-// the warp's own shared-memory buffers by cp.async one step ahead of their
-// MMAs (and the block scales into registers one step ahead), so a warp's
-// next loads are in flight while it decodes and multiplies the current step:
-// with every load of a step waited for before its arithmetic, a gate/up unit
-// took about 2.5 us per step. Each lane reads back only the 16 bytes it
-// copied. wbuf: shared address of this warp's buffers (fp4_wbuf_bytes(RT)).
+// NVFP4: steps of 128 K values (lane q covers K = 128 s + 32 q .. +32: 16
+// code bytes and one scale pair per row); RT row tiles per step, the tiles
+// tstride code bytes (tsc scale pairs) apart, sharing one activation
+// fragment; eight MMAs per step, tile and token tile.
+// Each step's code fragments are brought into the warp's own shared-memory
+// buffers by cp.async one step ahead of their MMAs (and the block scales into
+// registers one step ahead), so a warp's next loads are in flight while it
+// decodes and multiplies the current step (with every load of a step waited
+// for before its arithmetic, a gate/up unit took about 2.5 us per step). Each
+// lane reads back only the 16 bytes it copied. wbuf: shared address of this
+// warp's buffers (fp4_wbuf_bytes(RT)).
 template <int NB, int RT, bool P1>
 __device__ __forceinline__ void dot_nvfp4_async(const uint8_t* ra, const uint8_t* rb, const unsigned short* sa,
                                                 const unsigned short* sb, size_t tstride, size_t tsc, int s0, int s1,
