@@ -60,3 +60,22 @@ def test_traffic_lookup_follows_the_source(tmp_path, monkeypatch):
     assert bench.ncu_traffic("gemv_hit", 1) == 123
     assert bench.ncu_traffic("gemv_staged", 1) is None  # taken from an older source
     assert bench.ncu_traffic("route_decode_fused", 1) is None  # not recorded
+
+
+def test_kernel_microbenchmarks_are_single_gpu(monkeypatch):
+    """The kernel microbenchmark workloads run on one GPU and only for this
+    implementation; other requests stop before any device is touched."""
+    import pytest
+    for argv in (["--workload", "hit_gemv", "--gpus", "2"], ["--workload", "stream_gemv", "--impl", "reference"],
+                 ["--workload", "prefill_gemm", "--gpus", "8"]):
+        monkeypatch.setattr(sys, "argv", ["bench.py", *argv])
+        with pytest.raises(SystemExit) as e:
+            bench.main()
+        assert "one GPU" in str(e.value)
+
+
+def test_unknown_workload_is_rejected(monkeypatch):
+    import pytest
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--workload", "no_such_workload"])
+    with pytest.raises((SystemExit, KeyError, ValueError)):
+        bench.main()
