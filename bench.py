@@ -485,13 +485,14 @@ def host_mem_available():
     return None
 
 
-def mixed_sweep(wl, caps, profiles, steps, warmup, rank, local):
+def mixed_sweep(wl, caps, profiles, steps, warmup, rank, local, prefetch=False):
     """The 43-layer mixed NVFP4 workload on one context: for every cache
     capacity and B_P:B_H profile, a cold prefill of T = 8192 tokens through
     every layer (layer-ahead double buffer), then `steps` decode steps split
     in equal blocks at batch 1, 2, 4 and 8 with Markov routing. The slot pool
-    is resized between capacities (the host pool is filled once). Returns
-    (rows, host_link, clocks)."""
+    is resized between capacities (the host pool is filled once). prefetch:
+    the opt-in decode prefetch (layer l+1's experts of its previous decode
+    call staged while layer l computes). Returns (rows, host_link, clocks)."""
     import dataclasses
     import ftgen
     import sparse_moe_expert_topk_b200 as ft
@@ -506,6 +507,7 @@ def mixed_sweep(wl, caps, profiles, steps, warmup, rank, local):
     T_pf = ex["prefill_T"]
     h = Harness(dataclasses.replace(wl, cache_slots=caps[0]), max_tokens=T_pf, device=local)
     try:
+        ft.ft_moe_set_prefetch(h.ctx, prefetch)
         # inputs: one prefill block reused by every layer (each layer routes it
         # with its own router), decode activations and per-token trace biases
         g = torch.Generator(device=device)
@@ -596,7 +598,7 @@ def mixed_sweep(wl, caps, profiles, steps, warmup, rank, local):
     return sweep, {"h2d_copy_gbs": round(h2d, 2), "zero_copy_read_gbs": round(zc, 2)}, clocks
 
 
-def mixed_point(rank, local):
+def mixed_point(rank, local, prefetch=False):
     """The largest single-GPU workload at its headline point, for the default
     line: 43-layer mixed NVFP4 at 37% capacity and B_P:B_H = 52.7:77.3, cold
     prefill of 8192 tokens, then the full 1024 decode steps at batch 1/2/4/8.
@@ -609,13 +611,15 @@ def mixed_point(rank, local):
         return {"skipped": f"host memory: {avail / 1e9:.0f} GB available, the pinned pool needs {need / 1e9:.0f} GB"}
     t0 = time.perf_counter()
     try:
-        rows, link, clocks = mixed_sweep(wl, [int(0.37 * wl.L * wl.E)], [(52700, 77300)], wl.steps, 1, rank, local)
+        rows, link, clocks = mixed_sweep(wl, [int(0.37 * wl.L * wl.E)], [(52700, 77300)], wl.steps, 1, rank, local,
+                                         prefetch)
     except Exception as e:  # the default line must still be printed
         return {"skipped": f"{type(e).__name__}: {e}"}
     r = rows[0]
     return {"workload": f"43-layer mixed NVFP4, E=256 top-6 d=4096 d_ff=1536 ({need / 1e9:.1f} GB pinned pool): cold "
                         f"prefill T={wl.extra['prefill_T']} through all layers, then {r['decode_steps']} decode steps "
-                        f"at batch 1/2/4/8, Markov p=0.8 + Zipf(1.1), 37% cache ({r['cache_slots']} slots), 52.7:77.3",
+                        f"at batch 1/2/4/8, Markov p=0.8 + Zipf(1.1), 37% cache ({r['cache_slots']} slots), 52.7:77.3"
+                        + (", decode prefetch on" if prefetch else ""),
             "decode_tokens_per_s": r["decode_tokens_per_s"], "decode_miss_rate": r["decode_miss_rate"],
             "prefill": r["prefill"], "decode": r["decode"], "host_link": link, "clocks": clocks,
             "wall_s": round(time.perf_counter() - t0, 1)}
@@ -629,7 +633,9 @@ def run_mixed(args, wl, world, rank, local):
     ex = wl.extra
     steps = min(wl.steps, int(os.environ.get("FT_MIXED_STEPS", 256)))
     caps = [int(f * L * E) for f in ex["cache_fracs"]]
-    sweep, link, clocks = mixed_sweep(wl, caps, list(ex["profiles"]), steps, max(1, args.warmup - 2), rank, local)
+    prefetch = os.environ.get("FT_PREFETCH", "0") == "1"  # the decode prefetch (opt-in)
+    sweep, link, clocks = mixed_sweep(wl, caps, list(ex["profiles"]), steps, max(1, args.warmup - 2), rank, local,
+                                      prefetch)
     main_pt = next(r for r in sweep if r["cache_slots"] == int(0.37 * L * E) and r["bp_bh"] == "52.7:77.3")
     steps -= steps % len(wl.batches)
     out = {"metric": METRIC, "value": main_pt["decode_tokens_per_s"], "unit": UNIT, "n_gpus": world,
@@ -882,9 +888,12 @@ def main():
     torch.cuda.empty_cache()
     # the largest single-GPU workload (43-layer mixed NVFP4), one GPU only:
     # each rank of a multi-GPU run would pin its own 117 GB pool
-    mixed = None
+    mixed = mixed_pf = None
     if world == 1 and not args.no_mixed:
         mixed = mixed_point(rank, local)
+        # the same point with the decode prefetch: layer l+1's experts of its
+        # previous decode call staged while layer l computes
+        mixed_pf = mixed_point(rank, local, prefetch=True)
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -906,6 +915,7 @@ def main():
             "gpu_launches_per_step": round(launches, 1), "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,
             "peaks": {"kind": peak_kind, "hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"]},
             "mixed_nvfp4": mixed,
+            "mixed_nvfp4_prefetch": mixed_pf,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
