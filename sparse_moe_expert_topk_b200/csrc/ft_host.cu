@@ -630,12 +630,25 @@ static ft_status layer_call(ft_ctx* c, int32_t layer, int32_t mode, const void* 
     launch_to_f16(x, T, sh.d, d.x16, d.xscale, cs);
     c->kernel_launches += 1;
   }
-  // this decode call's routing counts become the layer's record for the
-  // decode prefetch; the fused routing stores them itself unless a prefetch
-  // batch of this same layer (one-layer models) must still read the old ones
+  // decode prefetch: right behind this call's lookup, a batch for the next
+  // layer from its last decode routing (pins this batch's slots); the fused
+  // routing runs it in the same launch. Then this call's routing counts become
+  // this layer's record (the fused routing stores them itself, after the
+  // prefetch batch has read the old ones, which matters for one-layer models)
   const int nxt_layer = (layer + 1) % sh.L;
-  const bool pf_reads_this = c->prefetch_on && c->has_prev[nxt_layer] && nxt_layer == layer;
-  const bool record_in_route = mode == FT_DECODE && fused_route && !full_prefill && !pf_reads_this;
+  const bool want_pf = mode == FT_DECODE && !full_prefill && c->prefetch_on && c->has_prev[nxt_layer];
+  LookupArgs pa{};
+  pa.layer = -1;  // none
+  if (want_pf) {
+    pa.layer = nxt_layer;
+    pa.use_counts = 1;
+    pa.pin_prev = 1;
+    pa.append = 1;
+    pa.prefetch = 1;
+    pa.counts_src = d.prev_counts + (size_t)nxt_layer * sh.E;
+  }
+  const bool pf_in_route = fused_route && want_pf;
+  const bool record_in_route = mode == FT_DECODE && fused_route && !full_prefill;
   if (record_in_route) la.record_counts = d.prev_counts + (size_t)layer * sh.E;
   int p = -1;
   if (rows_eids) {
@@ -646,7 +659,10 @@ static ft_status layer_call(ft_ctx* c, int32_t layer, int32_t mode, const void* 
     c->kernel_launches += 1 + n_perm;
   } else if (fused_route) {
     p = prof_begin(c, P_ROUTE_FUSED, cs, T * (double)sh.d * ab + sh.E * (double)sh.d * ab + sh.C * 8.0);
-    launch_route_decode(sh, x, c->router[layer], bias, bias_per_token, T, la, d, want_f16, cs);
+    LookupArgs none{};
+    none.layer = -1;
+    launch_route_decode(sh, x, c->router[layer], bias, bias_per_token, T, la, pf_in_route ? pa : none, d, want_f16,
+                        cs);
     prof_end(c, p, cs);
     c->kernel_launches += 1;
   } else {
@@ -674,18 +690,7 @@ static ft_status layer_call(ft_ctx* c, int32_t layer, int32_t mode, const void* 
       c->kernel_launches += 1;
     }
     if (mode == FT_DECODE) {
-      // predictive prefetch: right behind this lookup, a batch for the next
-      // layer from its last decode routing (pins this batch's slots), then
-      // this call's routing becomes this layer's record
-      const int nxt = (layer + 1) % sh.L;
-      if (c->prefetch_on && c->has_prev[nxt]) {
-        LookupArgs pa{};
-        pa.layer = nxt;
-        pa.use_counts = 1;
-        pa.pin_prev = 1;
-        pa.append = 1;
-        pa.prefetch = 1;
-        pa.counts_src = d.prev_counts + (size_t)nxt * sh.E;
+      if (want_pf && !pf_in_route) {
         p = prof_begin(c, P_LOOKUP, cs, sh.C * 8.0 + sh.E * 16.0);
         launch_lookup(sh, pa, d, cs);
         prof_end(c, p, cs);

@@ -149,7 +149,8 @@ int launch_permute(const Shape& sh, int T, DevState& ds, cudaStream_t st);  // r
 size_t perm_chunks_ints(int max_entries, int E);
 // decode routing in one launch (T <= 32): logits, top-k, permutation, lookup
 void launch_route_decode(const Shape& sh, const void* x, const void* w_router, const float* bias, int bias_per_token,
-                         int T, const LookupArgs& la, DevState& ds, bool to_f16, cudaStream_t st);
+                         int T, const LookupArgs& la, const LookupArgs& pf, DevState& ds, bool to_f16,
+                         cudaStream_t st);
 // one lookup batch; writes work lists, mailbox, counters
 void launch_lookup(const Shape& sh, const LookupArgs& a, DevState& ds, cudaStream_t st);
 // decode / fallback experts (SIMT grouped GEMV) for one work class;

@@ -450,6 +450,23 @@ __global__ void __launch_bounds__(128) router_mma_kernel(const __nv_bfloat16* __
     }
 }
 
+// After a fused routing's lookup: the decode prefetch batch of the next layer
+// (pf.layer >= 0; it reads that layer's recorded routing counts), then this
+// call's counts (s_counts, shared memory) become this layer's record. The
+// record is written after the prefetch batch has read its counts, so a
+// one-layer model prefetches from its previous call, not from this one.
+__device__ __forceinline__ void route_tail(const LookupArgs& la, const LookupArgs& pf, int E, long long C,
+                                           size_t slot_bytes, DevState& ds, const int32_t* s_counts) {
+  if (pf.layer >= 0) {
+    __syncthreads();
+    lookup_detail::lookup_body(pf, E, C, slot_bytes, ds);
+  }
+  if (la.record_counts) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) la.record_counts[e] = s_counts[e];
+  }
+}
+
 // Decode routing in one launch (T <= 32 tokens): CTAs of 32 warps compute the
 // logits of 16 (BF16) or 32 (fp32) experts each; the last CTA to finish
 // (ticket on ds.route_ctr) runs top-k + softmax, the stable permutation and
@@ -460,8 +477,8 @@ __global__ void __launch_bounds__(128) router_mma_kernel(const __nv_bfloat16* __
 template <typename AT>
 __global__ void __launch_bounds__(1024) route_decode_kernel(const AT* __restrict__ x, const AT* __restrict__ wr,
                                                             const float* __restrict__ bias, int bias_per_token, int T,
-                                                            int E, int d, int k, LookupArgs la, long long C,
-                                                            size_t slot_bytes, DevState ds, __half* x16,
+                                                            int E, int d, int k, LookupArgs la, LookupArgs pf,
+                                                            long long C, size_t slot_bytes, DevState ds, __half* x16,
                                                             float* xscale) {
   extern __shared__ int32_t smem[];
   __shared__ int s_last;
@@ -537,9 +554,8 @@ __global__ void __launch_bounds__(1024) route_decode_kernel(const AT* __restrict
   permute_body(ds.ids, T * k, E, ds.counts, ds.offsets, ds.perm, ds.inv, smem);
   __syncthreads();
   // counts and offsets are still in this CTA's shared memory (permute_body)
-  if (la.record_counts)
-    for (int e = threadIdx.x; e < E; e += blockDim.x) la.record_counts[e] = smem[34 * E + e];
   lookup_detail::lookup_body(la, E, C, slot_bytes, ds, smem + 34 * E, smem + 35 * E);
+  route_tail(la, pf, E, C, slot_bytes, ds, smem + 34 * E);
   if (threadIdx.x == 0) *ds.route_ctr = 0;  // ready for the next call
 }
 
@@ -557,8 +573,8 @@ __global__ void __launch_bounds__(1024) route_decode_kernel(const AT* __restrict
 __global__ void __launch_bounds__(1024) route_cluster_kernel(const __nv_bfloat16* __restrict__ x,
                                                              const __nv_bfloat16* __restrict__ wr,
                                                              const float* __restrict__ bias, int bias_per_token, int T,
-                                                             int E, int d, int k, LookupArgs la, long long C,
-                                                             size_t slot_bytes, DevState ds, __half* x16,
+                                                             int E, int d, int k, LookupArgs la, LookupArgs pf,
+                                                             long long C, size_t slot_bytes, DevState ds, __half* x16,
                                                              float* xscale, int sc_off) {
   namespace cg = cooperative_groups;
   extern __shared__ __align__(16) int32_t smem[];
@@ -581,9 +597,9 @@ __global__ void __launch_bounds__(1024) route_cluster_kernel(const __nv_bfloat16
   __syncthreads();
   permute_body(s_ids, T * k, E, ds.counts, ds.offsets, ds.perm, ds.inv, smem);
   __syncthreads();
-  if (la.record_counts)
-    for (int e = threadIdx.x; e < E; e += blockDim.x) la.record_counts[e] = smem[34 * E + e];
+  // counts and offsets are still in this CTA's shared memory (permute_body)
   lookup_detail::lookup_body(la, E, C, slot_bytes, ds, smem + 34 * E, smem + 35 * E);
+  route_tail(la, pf, E, C, slot_bytes, ds, smem + 34 * E);
 }
 
 bool g_route_cluster = false;  // cluster launches of 16 x 1024 threads fit on this device
@@ -785,7 +801,8 @@ constexpr int CLUSTER_MAX_E = 256;  // 16 CTAs of 16 experts
 constexpr int CLUSTER_MAX_T = 32;
 
 void launch_route_decode(const Shape& sh, const void* x, const void* w_router, const float* bias, int bias_per_token,
-                         int T, const LookupArgs& la, DevState& ds, bool to_f16, cudaStream_t st) {
+                         int T, const LookupArgs& la, const LookupArgs& pf, DevState& ds, bool to_f16,
+                         cudaStream_t st) {
   if (sh.wtype != FT_W_F32 && g_route_cluster && sh.E <= CLUSTER_MAX_E && T <= CLUSTER_MAX_T) {
     const int cs = (sh.E + 15) / 16;
     const int sc_off = (int)route_cluster_sc_off(sh.E);
@@ -802,7 +819,7 @@ void launch_route_decode(const Shape& sh, const void* x, const void* w_router, c
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaLaunchKernelEx(&cfg, route_cluster_kernel, (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_router, bias,
-                       bias_per_token, T, sh.E, sh.d, sh.k, la, sh.C, sh.slot_bytes, ds,
+                       bias_per_token, T, sh.E, sh.d, sh.k, la, pf, sh.C, sh.slot_bytes, ds,
                        to_f16 ? reinterpret_cast<__half*>(ds.x16) : nullptr, to_f16 ? ds.xscale : nullptr, sc_off);
     return;
   }
@@ -810,12 +827,12 @@ void launch_route_decode(const Shape& sh, const void* x, const void* w_router, c
   const size_t smem = route_decode_smem(sh.E);
   if (sh.wtype == FT_W_F32)
     route_decode_kernel<float><<<grid, 1024, smem, st>>>((const float*)x, (const float*)w_router, bias,
-                                                         bias_per_token, T, sh.E, sh.d, sh.k, la, sh.C, sh.slot_bytes,
-                                                         ds, nullptr, nullptr);
+                                                         bias_per_token, T, sh.E, sh.d, sh.k, la, pf, sh.C,
+                                                         sh.slot_bytes, ds, nullptr, nullptr);
   else
     route_decode_kernel<__nv_bfloat16><<<grid, 1024, smem, st>>>(
-        (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_router, bias, bias_per_token, T, sh.E, sh.d, sh.k, la, sh.C,
-        sh.slot_bytes, ds, to_f16 ? reinterpret_cast<__half*>(ds.x16) : nullptr, to_f16 ? ds.xscale : nullptr);
+        (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_router, bias, bias_per_token, T, sh.E, sh.d, sh.k, la, pf,
+        sh.C, sh.slot_bytes, ds, to_f16 ? reinterpret_cast<__half*>(ds.x16) : nullptr, to_f16 ? ds.xscale : nullptr);
 }
 
 // Dynamic shared-memory limits of the permutation and fused routing kernels,
