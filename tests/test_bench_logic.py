@@ -79,3 +79,13 @@ def test_unknown_workload_is_rejected(monkeypatch):
     monkeypatch.setattr(sys, "argv", ["bench.py", "--workload", "no_such_workload"])
     with pytest.raises((SystemExit, KeyError, ValueError)):
         bench.main()
+
+
+def test_mixed_point_skips_when_the_host_cannot_hold_the_pool(monkeypatch):
+    """The config-5 leg of the default line needs the 117 GB pinned pool; on a
+    host without that much memory it reports why it was skipped, with and
+    without the decode prefetch, and touches no device."""
+    monkeypatch.setattr(bench, "host_mem_available", lambda: 64 << 30)
+    for pf in (False, True):
+        r = bench.mixed_point(0, 0, prefetch=pf)
+        assert set(r) == {"skipped"} and "host memory" in r["skipped"]
